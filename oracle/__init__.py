@@ -1,0 +1,184 @@
+"""Plain fp64 CPU oracle for the hybrid-attention decode path.
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg
+of ``bench.py`` are the only callers. The product library never imports this package, and
+this package never imports the product library; the two share no code.
+
+The arithmetic lives in ``lad_oracle.c`` (double precision, loops written as the definitions
+read). This module compiles it with gcc on first use (or on ``build()``) and wraps each entry
+point for numpy arrays. bf16 tensors are widened exactly (a bf16 value is the top half of a
+binary32) before they reach the fp64 code; the MLA cache is passed as raw bf16 bit patterns
+so that a million-token cache need not be widened in memory.
+
+Sources are the two pages on Ling-3.1-flash; every C function names the page and section it
+follows: "Ling-3.1-flash and the 7:1 hybrid: how much KV cache does a 560B model need at 1M
+tokens?" (dev.to) and "Ling-3.1-flash: a 560B hybrid-attention MoE, counted from its
+safetensors headers" (ai.thesatyajit.com), section "How KDA and MLA split the work".
+
+Parity status: every function here is pinned by tests under ``tests/test_oracle_*.py``
+against closed forms, brute force, special cases and library routines.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lad_oracle.c")
+_LIB = os.path.join(_HERE, "liblad_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_ip = ctypes.POINTER(ctypes.c_int)
+_up = ctypes.POINTER(ctypes.c_uint16)
+
+
+def build(force: bool = False) -> str:
+    """Compile ``lad_oracle.c`` into ``liblad_oracle.so`` next to it and return the path."""
+    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall",
+               "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True, capture_output=True, text=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            lib.lado_kda_recurrent.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [_dp] * 7 + [ctypes.c_int]
+            lib.lado_kda_chunked.argtypes = [ctypes.c_int] * 6 + [ctypes.c_double] + [_dp] * 7 + [ctypes.c_int]
+            lib.lado_l2norm.argtypes = [ctypes.c_longlong, ctypes.c_int, ctypes.c_double, _dp, _dp]
+            lib.lado_short_conv_step.argtypes = [ctypes.c_int] * 3 + [_dp, _dp, _dp, _dp, ctypes.c_int, _dp]
+            lib.lado_mla_decode.argtypes = ([ctypes.c_int] * 4 + [ctypes.c_longlong, _dp, _up, _ip, _dp,
+                                            ctypes.c_double, _dp, _dp, ctypes.c_int])
+            lib.lado_num_threads_available.argtypes = []
+            for f in (lib.lado_kda_recurrent, lib.lado_kda_chunked, lib.lado_l2norm,
+                      lib.lado_short_conv_step, lib.lado_mla_decode, lib.lado_num_threads_available):
+                f.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    """Number of OpenMP threads the oracle may use on this host."""
+    return int(_load().lado_num_threads_available())
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray, t=_dp):
+    return a.ctypes.data_as(t)
+
+
+def _check(rc: int, name: str) -> None:
+    if rc != 0:
+        raise RuntimeError(f"oracle {name} failed with status {rc}")
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (uint16) to float64."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def kda_recurrent(q, k, v, alpha, beta, S0, scale: float = 1.0, nthreads: int = 1):
+    """Token-by-token KDA gated delta rule.
+
+    q, k, alpha: [B,T,H,dk]; v: [B,T,H,dv]; beta: [B,T,H]; S0: [B,H,dk,dv].
+    Returns (o [B,T,H,dv], S_T [B,H,dk,dv]) in float64.
+    """
+    q, k, v, alpha, beta = map(_f64, (q, k, v, alpha, beta))
+    S = _f64(S0).copy()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and alpha.shape == q.shape and v.shape == (B, T, H, dv)
+    assert beta.shape == (B, T, H) and S.shape == (B, H, dk, dv)
+    o = np.zeros((B, T, H, dv), dtype=np.float64)
+    rc = _load().lado_kda_recurrent(B, T, H, dk, dv, float(scale), _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(alpha), _ptr(beta), _ptr(S), _ptr(o), int(nthreads))
+    _check(rc, "kda_recurrent")
+    return o, S
+
+
+def kda_chunked(q, k, v, alpha, beta, S0, chunk: int, scale: float = 1.0, nthreads: int = 1):
+    """KDA in chunked WY/UT form; same arguments and results as :func:`kda_recurrent`."""
+    q, k, v, alpha, beta = map(_f64, (q, k, v, alpha, beta))
+    S = _f64(S0).copy()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv), dtype=np.float64)
+    rc = _load().lado_kda_chunked(B, T, H, dk, dv, int(chunk), float(scale), _ptr(q), _ptr(k),
+                                  _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S), _ptr(o), int(nthreads))
+    _check(rc, "kda_chunked")
+    return o, S
+
+
+def l2norm(x, eps: float = 1e-6):
+    """x / sqrt(sum x^2 + eps) over the last axis."""
+    x = _f64(x)
+    d = x.shape[-1]
+    y = np.empty_like(x)
+    _check(_load().lado_l2norm(x.size // d, d, float(eps), _ptr(x), _ptr(y)), "l2norm")
+    return y
+
+
+def short_conv_step(x, tail, w, bias=None, silu: bool = True):
+    """One decode step of the width-K causal depthwise convolution.
+
+    x: [B,Cch]; tail: [B,K-1,Cch] (oldest row first); w: [Cch,K]; bias: [Cch] or None.
+    Returns (y [B,Cch], new tail [B,K-1,Cch]) in float64.
+    """
+    x, w = _f64(x), _f64(w)
+    tail = _f64(tail).copy()
+    B, Cch = x.shape
+    K = w.shape[1]
+    assert tail.shape == (B, K - 1, Cch) and w.shape == (Cch, K)
+    y = np.zeros_like(x)
+    bptr = None
+    if bias is not None:
+        bias = _f64(bias)
+        bptr = _ptr(bias)
+    rc = _load().lado_short_conv_step(B, Cch, K, _ptr(x), _ptr(tail), _ptr(w), bptr, int(bool(silu)), _ptr(y))
+    _check(rc, "short_conv_step")
+    return y, tail
+
+
+def mla_decode(q, cache_bits, seq_lens, gate=None, scale: float = 192 ** -0.5, d_latent: int = 512,
+               nthreads: int = 1):
+    """Gated latent-attention decode.
+
+    q: [B,H,D] (float, absorbed query, D = d_latent + d_rope); cache_bits: uint16 bf16 bit
+    patterns [B,Lmax,D]; seq_lens: [B] ints; gate: [B,H] logits or None.
+    Returns (o [B,H,d_latent], lse [B,H]) in float64.
+    """
+    q = _f64(q)
+    cache_bits = np.ascontiguousarray(cache_bits, dtype=np.uint16)
+    B, H, D = q.shape
+    assert cache_bits.ndim == 3 and cache_bits.shape[0] == B and cache_bits.shape[2] == D
+    seq_stride = cache_bits.shape[1] * D
+    lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    assert lens.shape == (B,) and (lens <= cache_bits.shape[1]).all()
+    o = np.zeros((B, H, d_latent), dtype=np.float64)
+    lse = np.zeros((B, H), dtype=np.float64)
+    gptr = None
+    if gate is not None:
+        gate = _f64(gate)
+        gptr = _ptr(gate)
+    rc = _load().lado_mla_decode(B, H, d_latent, D - d_latent, seq_stride, _ptr(q),
+                                 _ptr(cache_bits, _up), _ptr(lens, _ip), gptr, float(scale),
+                                 _ptr(o), _ptr(lse), int(nthreads))
+    _check(rc, "mla_decode")
+    return o, lse

@@ -1,0 +1,366 @@
+/*
+ * Plain fp64 CPU oracle for the hybrid-attention decode path (KDA gated delta rule,
+ * its width-4 short convolution, and gated latent attention over the 576-wide MLA cache).
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product library links or calls this file; only
+ * the test suite, the smoke check and the benchmark's CPU-baseline leg load it. It shares no
+ * code, header, table or constant with the CUDA kernels.
+ *
+ * Sources (web pages on Ling-3.1-flash):
+ *   [P1] "Ling-3.1-flash and the 7:1 hybrid: how much KV cache does a 560B model need at 1M
+ *        tokens?" (dev.to), sections "How big is the cache per token, exactly?" and
+ *        "Why would a model keep only 9 full-attention layers?"
+ *   [P2] "Ling-3.1-flash: a 560B hybrid-attention MoE, counted from its safetensors headers"
+ *        (ai.thesatyajit.com), sections "How KDA and MLA split the work" and
+ *        "Does 292 GiB fit on four Hopper GPUs?"
+ *
+ * The display equation of the KDA update was lost from [P2] "How KDA and MLA split the work".
+ * What survives there: a gated delta-rule linear attention; per token the 128x128 state is
+ * decayed channel by channel (alpha_t, one decay per key channel) and the new key-value
+ * association is written with a per-head scalar strength beta_t; q, k, v come through a
+ * short causal convolution of width 4. [P1] "Why would a model keep only 9..." names the
+ * lineage: Gated DeltaNet with finer-grained (per-channel) gating. The readings taken where
+ * the page is silent are stated at each function and are:
+ *   (i)   the decay is applied before the delta correction (the correction predicts from the
+ *         decayed state), Gated-DeltaNet order;
+ *   (ii)  alpha scales the key (row) index of S, with S of shape d_k x d_v;
+ *   (iii) the readout is o_t = scale * S_t^T q_t, read after the write, scale a parameter;
+ *   (iv)  the convolution output passes through SiLU when the caller asks for it.
+ *
+ * Arithmetic is double precision throughout. Loops follow the definitions directly; the only
+ * parallelism is over independent (sequence, head) pairs, which changes no result.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define LADO_OK 0
+#define LADO_EINVAL -1
+#define LADO_ENOMEM -2
+
+int lado_num_threads_available(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* A bf16 value is the upper 16 bits of an IEEE binary32; widening it is exact. */
+static double bf16_bits_to_double(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/*
+ * KDA gated delta rule, token by token ([P2] "How KDA and MLA split the work"; [P1] "Why
+ * would a model keep only 9 full-attention layers?" for the Gated DeltaNet lineage).
+ * For every sequence b, head h and token t, with S the d_k x d_v state of (b, h):
+ *   S'  = Diag(alpha_t) S_{t-1}            decay, channel by channel (rows = key channels)
+ *   w   = S'^T k_t                         what the decayed state predicts for key k_t
+ *   u   = beta_t (v_t - w)                 delta-rule correction, strength beta_t
+ *   S_t = S' + k_t u^T                     write the new key-value association
+ *   o_t = scale * S_t^T q_t                readout after the write
+ * Layouts (row-major): q, k, alpha [B][T][H][dk]; v, o [B][T][H][dv]; beta [B][T][H];
+ * S [B][H][dk][dv], initial state in, final state out.
+ */
+int lado_kda_recurrent(int B, int T, int H, int dk, int dv, double scale,
+                       const double *q, const double *k, const double *v,
+                       const double *alpha, const double *beta,
+                       double *S, double *o, int nthreads) {
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return LADO_EINVAL;
+    if (nthreads < 1) nthreads = 1;
+    int err = 0;
+#pragma omp parallel for num_threads(nthreads) collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            double *Sbh = S + ((size_t)b * H + h) * (size_t)dk * dv;
+            double *w = (double *)malloc(sizeof(double) * dv);
+            double *u = (double *)malloc(sizeof(double) * dv);
+            if (!w || !u) {
+                free(w); free(u);
+#pragma omp atomic write
+                err = 1;
+                continue;
+            }
+            for (int t = 0; t < T; ++t) {
+                size_t tok = ((size_t)b * T + t) * H + h;
+                const double *qt = q + tok * dk;
+                const double *kt = k + tok * dk;
+                const double *at = alpha + tok * dk;
+                const double *vt = v + tok * dv;
+                double bt = beta[tok];
+                double *ot = o + tok * dv;
+                /* S' = Diag(alpha_t) S_{t-1} */
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dv; ++j)
+                        Sbh[(size_t)i * dv + j] *= at[i];
+                /* w = S'^T k_t */
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < dk; ++i) acc += Sbh[(size_t)i * dv + j] * kt[i];
+                    w[j] = acc;
+                }
+                /* u = beta_t (v_t - w) */
+                for (int j = 0; j < dv; ++j) u[j] = bt * (vt[j] - w[j]);
+                /* S_t = S' + k_t u^T */
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dv; ++j)
+                        Sbh[(size_t)i * dv + j] += kt[i] * u[j];
+                /* o_t = scale * S_t^T q_t */
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int i = 0; i < dk; ++i) acc += Sbh[(size_t)i * dv + j] * qt[i];
+                    ot[j] = scale * acc;
+                }
+            }
+            free(w);
+            free(u);
+        }
+    }
+    return err ? LADO_ENOMEM : LADO_OK;
+}
+
+/*
+ * The same recurrence in chunked (WY / UT) form, chunk length C, a last partial chunk allowed.
+ * The pages do not print it; it follows from lado_kda_recurrent by unrolling the recurrence
+ * inside a chunk. Within a chunk with rows r = 0..n-1 and initial state S0:
+ *   g_r   = prod_{s<=r} alpha_s                 cumulative decay per key channel
+ *   Kt    = K * g,  Kh = K / g,  Qt = Q * g     (elementwise, row r uses g_r)
+ *   A     = strict_lower(diag(beta) Kt Kh^T)
+ *   Tm    = (I + A)^{-1}                        by forward substitution (unit lower triangular)
+ *   W     = Tm diag(beta) Kt
+ *   U     = Tm diag(beta) V - W S0
+ *   O     = scale (Qt S0 + lower(Qt Kh^T) U)    lower() keeps the diagonal
+ *   S_new = Diag(g_{n-1}) S0 + (K * (g_{n-1} / g))^T U
+ * Same layouts as lado_kda_recurrent.
+ */
+int lado_kda_chunked(int B, int T, int H, int dk, int dv, int C, double scale,
+                     const double *q, const double *k, const double *v,
+                     const double *alpha, const double *beta,
+                     double *S, double *o, int nthreads) {
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0 || C <= 0) return LADO_EINVAL;
+    if (nthreads < 1) nthreads = 1;
+    int err = 0;
+#pragma omp parallel for num_threads(nthreads) collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            double *S0 = S + ((size_t)b * H + h) * (size_t)dk * dv;
+            size_t nk = (size_t)C * dk, nv = (size_t)C * dv, cc = (size_t)C * C;
+            double *g = malloc(sizeof(double) * nk), *Kt = malloc(sizeof(double) * nk);
+            double *Kh = malloc(sizeof(double) * nk), *Qt = malloc(sizeof(double) * nk);
+            double *A = malloc(sizeof(double) * cc), *Tm = malloc(sizeof(double) * cc);
+            double *QK = malloc(sizeof(double) * cc), *W = malloc(sizeof(double) * nk);
+            double *U = malloc(sizeof(double) * nv);
+            double *Snew = malloc(sizeof(double) * (size_t)dk * dv);
+            if (!g || !Kt || !Kh || !Qt || !A || !Tm || !QK || !W || !U || !Snew) {
+#pragma omp atomic write
+                err = 1;
+                goto done;
+            }
+            for (int c0 = 0; c0 < T; c0 += C) {
+                int n = (T - c0) < C ? (T - c0) : C;
+#define TOK(r) (((size_t)b * T + (size_t)(c0 + (r))) * H + h)
+                /* cumulative decay g and the scaled keys / queries */
+                for (int r = 0; r < n; ++r) {
+                    const double *ar = alpha + TOK(r) * dk;
+                    const double *kr = k + TOK(r) * dk;
+                    const double *qr = q + TOK(r) * dk;
+                    for (int i = 0; i < dk; ++i) {
+                        double prev = (r == 0) ? 1.0 : g[(size_t)(r - 1) * dk + i];
+                        double gi = prev * ar[i];
+                        g[(size_t)r * dk + i] = gi;
+                        Kt[(size_t)r * dk + i] = kr[i] * gi;
+                        Kh[(size_t)r * dk + i] = kr[i] / gi;
+                        Qt[(size_t)r * dk + i] = qr[i] * gi;
+                    }
+                }
+                /* A = strict_lower(diag(beta) Kt Kh^T); QK = lower(Qt Kh^T) */
+                for (int r = 0; r < n; ++r) {
+                    double br = beta[TOK(r)];
+                    for (int s = 0; s < n; ++s) {
+                        double kk = 0.0, qk = 0.0;
+                        for (int i = 0; i < dk; ++i) {
+                            kk += Kt[(size_t)r * dk + i] * Kh[(size_t)s * dk + i];
+                            qk += Qt[(size_t)r * dk + i] * Kh[(size_t)s * dk + i];
+                        }
+                        A[(size_t)r * C + s] = (s < r) ? br * kk : 0.0;
+                        QK[(size_t)r * C + s] = (s <= r) ? qk : 0.0;
+                    }
+                }
+                /* Tm = (I + A)^{-1}: solve (I + A) Tm = I row by row */
+                for (int r = 0; r < n; ++r) {
+                    for (int col = 0; col < n; ++col) {
+                        double acc = (r == col) ? 1.0 : 0.0;
+                        for (int s = 0; s < r; ++s) acc -= A[(size_t)r * C + s] * Tm[(size_t)s * C + col];
+                        Tm[(size_t)r * C + col] = acc;
+                    }
+                }
+                /* W = Tm diag(beta) Kt */
+                for (int r = 0; r < n; ++r)
+                    for (int i = 0; i < dk; ++i) {
+                        double acc = 0.0;
+                        for (int s = 0; s < n; ++s)
+                            acc += Tm[(size_t)r * C + s] * beta[TOK(s)] * Kt[(size_t)s * dk + i];
+                        W[(size_t)r * dk + i] = acc;
+                    }
+                /* U = Tm diag(beta) V - W S0 */
+                for (int r = 0; r < n; ++r)
+                    for (int j = 0; j < dv; ++j) {
+                        double acc = 0.0;
+                        for (int s = 0; s < n; ++s)
+                            acc += Tm[(size_t)r * C + s] * beta[TOK(s)] * v[TOK(s) * dv + j];
+                        for (int i = 0; i < dk; ++i) acc -= W[(size_t)r * dk + i] * S0[(size_t)i * dv + j];
+                        U[(size_t)r * dv + j] = acc;
+                    }
+                /* O = scale (Qt S0 + lower(Qt Kh^T) U) */
+                for (int r = 0; r < n; ++r)
+                    for (int j = 0; j < dv; ++j) {
+                        double acc = 0.0;
+                        for (int i = 0; i < dk; ++i) acc += Qt[(size_t)r * dk + i] * S0[(size_t)i * dv + j];
+                        for (int s = 0; s <= r; ++s) acc += QK[(size_t)r * C + s] * U[(size_t)s * dv + j];
+                        o[TOK(r) * dv + j] = scale * acc;
+                    }
+                /* S_new = Diag(g_last) S0 + (K * (g_last / g))^T U */
+                const double *gl = g + (size_t)(n - 1) * dk;
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dv; ++j) {
+                        double acc = gl[i] * S0[(size_t)i * dv + j];
+                        for (int s = 0; s < n; ++s)
+                            acc += k[TOK(s) * dk + i] * (gl[i] / g[(size_t)s * dk + i]) * U[(size_t)s * dv + j];
+                        Snew[(size_t)i * dv + j] = acc;
+                    }
+                memcpy(S0, Snew, sizeof(double) * (size_t)dk * dv);
+#undef TOK
+            }
+        done:
+            free(g); free(Kt); free(Kh); free(Qt); free(A); free(Tm);
+            free(QK); free(W); free(U); free(Snew);
+        }
+    }
+    return err ? LADO_ENOMEM : LADO_OK;
+}
+
+/*
+ * Per-vector L2 normalisation y = x / sqrt(sum x^2 + eps), applied to q and k per head before
+ * the recurrence. The pages do not mention it; it is the usual input conditioning of delta-rule
+ * layers and is kept behind a flag. x and y are [n][d].
+ */
+int lado_l2norm(long long n, int d, double eps, const double *x, double *y) {
+    if (n < 0 || d <= 0) return LADO_EINVAL;
+    for (long long r = 0; r < n; ++r) {
+        double ss = 0.0;
+        for (int i = 0; i < d; ++i) ss += x[r * d + i] * x[r * d + i];
+        double inv = 1.0 / sqrt(ss + eps);
+        for (int i = 0; i < d; ++i) y[r * d + i] = x[r * d + i] * inv;
+    }
+    return LADO_OK;
+}
+
+/*
+ * One decode step of the short causal depthwise convolution that q, k, v pass through
+ * ([P2] "How KDA and MLA split the work": width 4; [P2] "Does 292 GiB fit...": the kept
+ * "convolution tails"). For every sequence b and channel c, with K taps:
+ *   y[b][c] = sum_{i<K-1} w[c][i] tail[b][i][c] + w[c][K-1] x[b][c]  (+ bias[c] if given)
+ *   y       = y * sigmoid(y)                      when silu != 0
+ * tail[b][0] is the oldest kept input, tail[b][K-2] the newest. Afterwards the tail drops its
+ * oldest row and appends x: tail[b][i] = tail[b][i+1] for i < K-2, tail[b][K-2] = x[b].
+ * Layouts: x, y [B][Cch]; tail [B][K-1][Cch] (in/out); w [Cch][K]; bias [Cch] or NULL.
+ */
+int lado_short_conv_step(int B, int Cch, int K, const double *x, double *tail,
+                         const double *w, const double *bias, int silu, double *y) {
+    if (B < 0 || Cch <= 0 || K < 1) return LADO_EINVAL;
+    for (int b = 0; b < B; ++b) {
+        double *tb = tail + (size_t)b * (size_t)(K - 1) * Cch;
+        for (int c = 0; c < Cch; ++c) {
+            double acc = 0.0;
+            for (int i = 0; i < K - 1; ++i) acc += w[(size_t)c * K + i] * tb[(size_t)i * Cch + c];
+            acc += w[(size_t)c * K + (K - 1)] * x[(size_t)b * Cch + c];
+            if (bias) acc += bias[c];
+            if (silu) acc = acc / (1.0 + exp(-acc));
+            y[(size_t)b * Cch + c] = acc;
+        }
+        for (int i = 0; i + 1 < K - 1; ++i)
+            memcpy(tb + (size_t)i * Cch, tb + (size_t)(i + 1) * Cch, sizeof(double) * Cch);
+        if (K > 1) memcpy(tb + (size_t)(K - 2) * Cch, x + (size_t)b * Cch, sizeof(double) * Cch);
+    }
+    return LADO_OK;
+}
+
+/*
+ * Gated MLA decode over the compressed latent cache ([P2] "How KDA and MLA split the work":
+ * ordinary softmax attention over a cache whose rows are a 512-wide latent plus a 64-wide RoPE
+ * key, scaled by a per-head sigmoid gate; [P1] "How big is the cache per token, exactly?": the
+ * cached row is kv_lora_rank + qk_rope_head_dim = 576 elements; [P1] "For scale, plain
+ * multi-head attention..." gives the 192-wide key behind the softmax scale).
+ * The query arrives already absorbed (W_UK folded in), so it is Dc + Dr wide. For every
+ * sequence b with L = seq_lens[b] cached rows c_0..c_{L-1} and every head h:
+ *   s_t  = scale * <q_h, c_t>                 over all Dc + Dr dimensions
+ *   p_t  = exp(s_t - max s) / sum_t exp(s_t - max s)
+ *   o_h  = sum_t p_t c_t[0:Dc]                the values are the latent part only
+ *   o_h *= sigmoid(gate[b][h])                when gate is given
+ *   lse  = max s + log sum_t exp(s_t - max s) (natural log, before the gate)
+ * L = 0 gives o_h = 0 and lse = -inf.
+ * Layouts: q [B][H][Dc+Dr] (double); cache: bf16 bit patterns, row t of sequence b at
+ * element offset b*seq_stride + t*(Dc+Dr); gate [B][H] or NULL; o [B][H][Dc]; lse [B][H] or NULL.
+ */
+int lado_mla_decode(int B, int H, int Dc, int Dr, long long seq_stride,
+                    const double *q, const uint16_t *cache, const int *seq_lens,
+                    const double *gate, double scale, double *o, double *lse, int nthreads) {
+    if (B < 0 || H < 0 || Dc <= 0 || Dr < 0) return LADO_EINVAL;
+    if (nthreads < 1) nthreads = 1;
+    const int D = Dc + Dr;
+    int err = 0;
+#pragma omp parallel for num_threads(nthreads) collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            const int L = seq_lens[b];
+            const double *qh = q + ((size_t)b * H + h) * D;
+            double *oh = o + ((size_t)b * H + h) * Dc;
+            if (L <= 0) {
+                for (int d = 0; d < Dc; ++d) oh[d] = 0.0;
+                if (lse) lse[(size_t)b * H + h] = -INFINITY;
+                continue;
+            }
+            double *s = (double *)malloc(sizeof(double) * (size_t)L);
+            if (!s) {
+#pragma omp atomic write
+                err = 1;
+                continue;
+            }
+            const uint16_t *cb = cache + (size_t)b * (size_t)seq_stride;
+            double m = -INFINITY;
+            for (int t = 0; t < L; ++t) {
+                const uint16_t *ct = cb + (size_t)t * D;
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += qh[d] * bf16_bits_to_double(ct[d]);
+                s[t] = scale * acc;
+                if (s[t] > m) m = s[t];
+            }
+            double z = 0.0;
+            for (int t = 0; t < L; ++t) {
+                s[t] = exp(s[t] - m);
+                z += s[t];
+            }
+            for (int d = 0; d < Dc; ++d) oh[d] = 0.0;
+            for (int t = 0; t < L; ++t) {
+                const uint16_t *ct = cb + (size_t)t * D;
+                double p = s[t] / z;
+                for (int d = 0; d < Dc; ++d) oh[d] += p * bf16_bits_to_double(ct[d]);
+            }
+            if (gate) {
+                double sg = 1.0 / (1.0 + exp(-gate[(size_t)b * H + h]));
+                for (int d = 0; d < Dc; ++d) oh[d] *= sg;
+            }
+            if (lse) lse[(size_t)b * H + h] = m + log(z);
+            free(s);
+        }
+    }
+    return err ? LADO_ENOMEM : LADO_OK;
+}
