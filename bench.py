@@ -1,0 +1,673 @@
+#!/usr/bin/env python
+"""Benchmark of the hybrid-attention decode path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl lad|reference]
+
+A step is one pass of the workload's hot path over one batch of synthetic input:
+  hybrid_8layer_1m (default)  8-layer slice of the 7:1 hybrid, one decode token for 8 sequences:
+                              7 x (kda_conv_update + kda_decode_step) + 1 x mla_latent_decode over
+                              1,000,000 cached tokens per sequence
+  kda_decode_b64              one KDA layer: kda_conv_update + kda_decode_step, 64 sequences x 64 heads
+  mla_decode_b16              one gated MLA layer, 16 sequences, contexts uniform in [8192, 131072]
+  kda_prefill_32k             kda_prefill_chunked, 1 x 32768 tokens x 64 heads, chunk 64
+
+Multi-GPU (torchrun, one process per GPU): the path shards by sequence with no exchange, so each
+rank runs the same per-GPU workload on its own sequences ("weak" scaling); the step time is the
+max over ranks and `value` counts the tokens of all ranks.
+
+`--impl reference` times the fp64 CPU oracle (the only other implementation of the path) on the
+host cores, on a bounded sample of the same workload, and prints the same line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "decode tokens/s and achieved HBM GB/s (% of B200 roofline) per layer type"
+DEFAULT_WORKLOAD = "hybrid_8layer_1m"
+H, D = wl.HEADS, wl.HEAD_DIM
+
+
+# ---------------------------------------------------------------------------------------------
+# host-side plumbing shared with the multi-process tests
+# ---------------------------------------------------------------------------------------------
+
+def dist_env() -> tuple[int, int, int]:
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def shard_sequences(global_batch: int, rank: int, world: int) -> tuple[int, int]:
+    """Contiguous range [lo, hi) of the global batch that `rank` owns (sizes differ by <= 1)."""
+    base, rem = divmod(global_batch, world)
+    lo = rank * base + min(rank, rem)
+    return lo, lo + base + (1 if rank < rem else 0)
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device=None) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(device_index=None) -> None:
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device_index is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device_index])
+        else:
+            dist.barrier()
+
+
+def physical_gpu_index(local: int) -> int:
+    """nvidia-smi index of this process's GPU (CUDA_VISIBLE_DEVICES maps local ordinals)."""
+    vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    if local < len(vis) and vis[local].isdigit():
+        return int(vis[local])
+    return local
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# workloads: each builds its resident device state and returns a Step
+# ---------------------------------------------------------------------------------------------
+
+class Step:
+    """One workload on one GPU.
+
+    run(): enqueue one step on the current stream (inputs already resident).
+    run_e2e(): the same step with this step's inputs copied in from pinned host memory and the
+    step's outputs read back to pinned host memory, all on the current stream.
+    """
+
+    name = ""
+    tokens_per_step = 0          # decode tokens (or prefill tokens) one step produces on this GPU
+    launches_per_step = 0        # library kernels one step launches
+    dominant = ""                # name of the roofline kernel
+    dominant_unit = "GB/s"
+    dominant_bound = "hbm"
+    config: dict = {}
+
+    def run(self, timer=None):
+        raise NotImplementedError
+
+    def run_e2e(self):
+        raise NotImplementedError
+
+    def algorithmic_bytes(self) -> dict:
+        """Algorithmic bytes per launch of each kernel kind, and per step."""
+        raise NotImplementedError
+
+
+class _KdaLayer:
+    """State and per-token inputs of one KDA decode layer (conv + gated delta rule)."""
+
+    def __init__(self, lad, B, seed, dev, tag=""):
+        cfg = wl.KdaDecode(f"kda{tag}", B=B, seed=seed)
+        inp = wl.kda_decode_inputs(cfg, dev, tag=tag)
+        self.lad, self.B = lad, B
+        self.x, self.tail, self.w = inp["x"], inp["tail"], inp["w"]
+        self.alpha, self.beta, self.S = inp["alpha"], inp["beta"], inp["S"]
+        self.y = torch.empty_like(self.x)
+        self.o = torch.empty((B, H, D), device=dev, dtype=torch.bfloat16)
+        # pinned host copies of the per-token inputs and outputs (for the end-to-end timing)
+        self.h_x = self.x.cpu().pin_memory()
+        self.h_alpha = self.alpha.cpu().pin_memory()
+        self.h_beta = self.beta.cpu().pin_memory()
+        self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+
+    def run(self, timer=None):
+        lad, hd = self.lad, H * D
+        lad.kda_conv_update(self.x, self.tail, self.w, y=self.y, silu=True)
+        if timer:
+            timer.begin("kda_decode_step")
+        lad.kda_decode_step(self.y[:, :hd], self.y[:, hd:2 * hd], self.y[:, 2 * hd:], self.alpha, self.beta,
+                            self.S, o=self.o, l2norm_qk=True)
+        if timer:
+            timer.end("kda_decode_step")
+
+    def h2d(self):
+        self.x.copy_(self.h_x, non_blocking=True)
+        self.alpha.copy_(self.h_alpha, non_blocking=True)
+        self.beta.copy_(self.h_beta, non_blocking=True)
+
+    def d2h(self):
+        self.h_o.copy_(self.o, non_blocking=True)
+
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.h_x, self.h_alpha, self.h_beta))
+
+    def d2h_bytes(self):
+        return self.h_o.numel() * self.h_o.element_size()
+
+    @staticmethod
+    def bytes_conv(B):
+        C = 3 * H * D
+        # x, tail read, tail written, y per sequence (bf16); taps once per launch
+        return B * C * 2 * (1 + 3 + 3 + 1) + C * 4 * 2
+
+    @staticmethod
+    def bytes_decode(B):
+        # per (b, h): state read + write (fp32 128x128), q,k,v (bf16), alpha (fp32), beta, o (bf16)
+        return B * H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2)
+
+
+class KdaDecodeStep(Step):
+    name = "kda_decode_b64"
+
+    def __init__(self, lad, dev, rank, B=64):
+        self.layer = _KdaLayer(lad, B, 1235 + 1000 * rank, dev)
+        self.tokens_per_step = B
+        self.launches_per_step = 2
+        self.dominant = "kda_decode_step"
+        self.config = {"workload": self.name, "batch_per_gpu": B, "heads": H, "head_dim": D,
+                       "state": "fp32 128x128 per head", "conv": "width 4 over 3x8192 bf16 channels",
+                       "l2": "inputs larger than L2 (268 MB of state per step)"}
+
+    def run(self, timer=None):
+        self.layer.run(timer)
+
+    def run_e2e(self):
+        self.layer.h2d()
+        self.layer.run()
+        self.layer.d2h()
+
+    def e2e_bytes(self):
+        return self.layer.h2d_bytes(), self.layer.d2h_bytes()
+
+    def algorithmic_bytes(self):
+        B = self.layer.B
+        return {"kda_decode_step": _KdaLayer.bytes_decode(B), "kda_conv_update": _KdaLayer.bytes_conv(B),
+                "step": _KdaLayer.bytes_decode(B) + _KdaLayer.bytes_conv(B)}
+
+
+class MlaDecodeStep(Step):
+    name = "mla_decode_b16"
+
+    def __init__(self, lad, dev, rank, cfg: wl.MlaDecode | None = None):
+        cfg = cfg or wl.MlaDecode("mla", B=16, seed=1236 + 1000 * rank)
+        self.lad, self.cfg = lad, cfg
+        inp = wl.mla_inputs(cfg, dev)
+        self.q, self.cache, self.lens, self.gate = inp["q"], inp["cache"], inp["seq_lens"], inp["gate"]
+        self.total_len = int(self.lens.sum().item())
+        self.o = torch.empty((cfg.B, cfg.Hq, wl.D_LATENT), device=dev, dtype=torch.bfloat16)
+        self.ws = torch.empty(lad.mla_latent_decode_workspace_size(cfg.B, cfg.Hq, wl.D_LATENT, 0), device=dev,
+                              dtype=torch.uint8)
+        self.h_q = self.q.cpu().pin_memory()
+        self.h_gate = self.gate.cpu().pin_memory()
+        self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.tokens_per_step = cfg.B
+        self.launches_per_step = 2
+        self.dominant = "mla_latent_decode"
+        self.config = {"workload": self.name, "batch_per_gpu": cfg.B, "q_heads": cfg.Hq,
+                       "cache_row": "512 latent + 64 rope, bf16",
+                       "context": (f"{cfg.fixed_len} per sequence" if cfg.fixed_len else
+                                   f"uniform [{cfg.len_lo}, {cfg.len_hi}], total {self.total_len}"),
+                       "l2": "inputs larger than L2 (latent cache)"}
+
+    def run(self, timer=None):
+        if timer:
+            timer.begin("mla_latent_decode")
+        self.lad.mla_latent_decode(self.q, self.cache, self.lens, self.gate, o=self.o, workspace=self.ws)
+        if timer:
+            timer.end("mla_latent_decode")
+
+    def h2d(self):
+        self.q.copy_(self.h_q, non_blocking=True)
+        self.gate.copy_(self.h_gate, non_blocking=True)
+
+    def d2h(self):
+        self.h_o.copy_(self.o, non_blocking=True)
+
+    def run_e2e(self):
+        self.h2d()
+        self.run()
+        self.d2h()
+
+    def e2e_bytes(self):
+        hb = self.h_q.numel() * 2 + self.h_gate.numel() * 4
+        return hb, self.h_o.numel() * 2
+
+    def mla_bytes(self):
+        B, Hq = self.cfg.B, self.cfg.Hq
+        return self.total_len * wl.D_ROW * 2 + B * Hq * (wl.D_ROW * 2 + 4 + wl.D_LATENT * 2) + B * 4
+
+    def mla_flops(self):
+        return 2 * self.cfg.Hq * (wl.D_ROW + wl.D_LATENT) * self.total_len
+
+    def algorithmic_bytes(self):
+        b = self.mla_bytes()
+        return {"mla_latent_decode": b, "step": b}
+
+
+class HybridStep(Step):
+    name = "hybrid_8layer_1m"
+
+    def __init__(self, lad, dev, rank, B=8, ctx=1_000_000, kda_layers=7):
+        seed = 1238 + 1000 * rank
+        self.kda = [_KdaLayer(lad, B, seed, dev, tag=f"L{i}.") for i in range(kda_layers)]
+        self.mla = MlaDecodeStep(lad, dev, rank, wl.MlaDecode("mla", B=B, seed=seed, fixed_len=ctx))
+        self.tokens_per_step = B
+        self.launches_per_step = 2 * kda_layers + self.mla.launches_per_step
+        self.dominant = "mla_latent_decode"
+        self.config = {"workload": self.name, "batch_per_gpu": B, "layers": f"{kda_layers} KDA + 1 gated MLA",
+                       "mla_context": ctx, "heads": H, "head_dim": D,
+                       "l2": "inputs larger than L2 (9.2 GB latent cache + 235 MB KDA state per step)"}
+
+    def run(self, timer=None):
+        for layer in self.kda:
+            layer.run(timer)
+        self.mla.run(timer)
+
+    def run_e2e(self):
+        for layer in self.kda:
+            layer.h2d()
+        self.mla.h2d()
+        self.run()
+        for layer in self.kda:
+            layer.d2h()
+        self.mla.d2h()
+
+    def e2e_bytes(self):
+        hb = sum(layer.h2d_bytes() for layer in self.kda) + self.mla.e2e_bytes()[0]
+        db = sum(layer.d2h_bytes() for layer in self.kda) + self.mla.e2e_bytes()[1]
+        return hb, db
+
+    def algorithmic_bytes(self):
+        B = self.kda[0].B
+        n = len(self.kda)
+        kd, kc, m = _KdaLayer.bytes_decode(B), _KdaLayer.bytes_conv(B), self.mla.mla_bytes()
+        return {"kda_decode_step": kd, "kda_conv_update": kc, "mla_latent_decode": m,
+                "step": n * (kd + kc) + m}
+
+
+class PrefillStep(Step):
+    name = "kda_prefill_32k"
+
+    def __init__(self, lad, dev, rank, cfg: wl.KdaScan | None = None):
+        cfg = cfg or wl.KdaScan("prefill", B=1, H=64, T=32768, chunk=64, seed=1237 + 1000 * rank)
+        self.lad, self.cfg = lad, cfg
+        inp = wl.kda_scan_inputs(cfg, dev)
+        self.q, self.k, self.v = inp["q"], inp["k"], inp["v"]
+        self.alpha, self.beta, self.S0 = inp["alpha"], inp["beta"], inp["S0"]
+        self.S = self.S0.clone()
+        self.o = torch.empty_like(self.v)
+        self.ws = torch.empty(max(1, lad.kda_prefill_workspace_size(cfg.B, cfg.T, cfg.H, D, D, cfg.chunk)),
+                              device=dev, dtype=torch.uint8)
+        self.h_in = [t.cpu().pin_memory() for t in (self.q, self.k, self.v, self.alpha, self.beta)]
+        self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.tokens_per_step = cfg.B * cfg.T
+        self.launches_per_step = 1
+        self.dominant = "kda_prefill_chunked"
+        self.config = {"workload": self.name, "batch_per_gpu": cfg.B, "seq_len": cfg.T, "heads": cfg.H,
+                       "chunk": cfg.chunk, "l2": "inputs larger than L2 (3.2 GB per step)"}
+
+    def run(self, timer=None):
+        if timer:
+            timer.begin("kda_prefill_chunked")
+        self.S.copy_(self.S0)
+        self.lad.kda_prefill_chunked(self.q, self.k, self.v, self.alpha, self.beta, self.S, o=self.o,
+                                     chunk=self.cfg.chunk, workspace=self.ws)
+        if timer:
+            timer.end("kda_prefill_chunked")
+
+    def run_e2e(self):
+        for d, h in zip((self.q, self.k, self.v, self.alpha, self.beta), self.h_in):
+            d.copy_(h, non_blocking=True)
+        self.run()
+        self.h_o.copy_(self.o, non_blocking=True)
+
+    def e2e_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.h_in), self.h_o.numel() * 2
+
+    def algorithmic_bytes(self):
+        c = self.cfg
+        n = c.B * c.T * c.H
+        b = n * (3 * D * 2 + D * 4 + 4 + D * 2) + 2 * c.B * c.H * D * D * 4
+        return {"kda_prefill_chunked": b, "step": b}
+
+    def flops(self):
+        c = self.cfg
+        chunks = c.B * c.H * math.ceil(c.T / c.chunk)
+        C = c.chunk
+        per_chunk = 2 * (2 * C * C * D + C * C * D + C * D * D + C * C * D + C * D * D + C * D * D + C * C * D
+                         + D * D * C)
+        return chunks * per_chunk
+
+
+WORKLOADS = {
+    "hybrid_8layer_1m": HybridStep,
+    "kda_decode_b64": KdaDecodeStep,
+    "mla_decode_b16": MlaDecodeStep,
+    "kda_prefill_32k": PrefillStep,
+}
+
+
+class KernelTimer:
+    """CUDA events around each launch of named kernels, on the current (launching) stream."""
+
+    def __init__(self):
+        self.pairs: dict[str, list] = {}
+
+    def begin(self, name):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        self.pairs.setdefault(name, []).append([e, None])
+
+    def end(self, name):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        self.pairs[name][-1][1] = e
+
+    def mean_ms(self, name) -> float | None:
+        ps = self.pairs.get(name)
+        if not ps:
+            return None
+        return sum(a.elapsed_time(b) for a, b in ps) / len(ps)
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline key)
+# ---------------------------------------------------------------------------------------------
+
+def cpu_oracle_rate(workload: str, budget_s: float = 20.0) -> dict:
+    """Times the fp64 oracle on a bounded sample of the workload; returns tokens/s for the
+    whole workload step estimated from the sample, with the sample described."""
+    import oracle
+    nth = oracle.max_threads()
+    rng = np.random.default_rng(0)
+
+    def kda_layer_seconds(B):
+        # one KDA decode layer (conv + step) for B sequences, all 64 heads
+        Bs = min(B, max(1, nth))
+        x = rng.standard_normal((Bs, 3 * H * D))
+        tail = rng.standard_normal((Bs, 3, 3 * H * D))
+        w = 0.5 * rng.standard_normal((3 * H * D, 4))
+        q = rng.standard_normal((Bs, 1, H, D))
+        S = 0.02 * rng.standard_normal((Bs, H, D, D))
+        a = np.full((Bs, 1, H, D), 0.9)
+        b = np.full((Bs, 1, H), 0.5)
+        t0 = time.perf_counter()
+        y, _ = oracle.short_conv_step(x, tail, w, None, True)
+        qn = oracle.l2norm(y[:, : H * D].reshape(Bs, 1, H, D))
+        kn = oracle.l2norm(y[:, H * D: 2 * H * D].reshape(Bs, 1, H, D))
+        oracle.kda_recurrent(qn, kn, y[:, 2 * H * D:].reshape(Bs, 1, H, D), a, b, S, nthreads=nth)
+        dt = time.perf_counter() - t0
+        return dt * B / Bs, f"{Bs} of {B} sequences x 64 heads, one token"
+
+    def mla_seconds(B, lens):
+        # units = (sequence, head); sample `nth` heads of the longest sequence over its whole context
+        L = int(max(lens))
+        units = min(nth, H)
+        cache = (rng.standard_normal((1, L, wl.D_ROW)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+        qs = rng.standard_normal((1, units, wl.D_ROW))
+        t0 = time.perf_counter()
+        oracle.mla_decode(qs, cache, np.array([L], np.int32), None, nthreads=nth)
+        dt = time.perf_counter() - t0
+        total_units_tokens = H * float(sum(lens))
+        return dt * total_units_tokens / (units * L), f"{units} heads x {L} cached tokens of 1 sequence"
+
+    if workload == "kda_decode_b64":
+        sec, sample = kda_layer_seconds(64)
+        return {"value": 64 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": sample}
+    if workload == "mla_decode_b16":
+        lens = wl.mla_seq_lens(wl.MlaDecode("mla", B=16, seed=1236)).tolist()
+        sec, sample = mla_seconds(16, lens)
+        return {"value": 16 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": sample}
+    if workload == "hybrid_8layer_1m":
+        ks, s1 = kda_layer_seconds(8)
+        ms, s2 = mla_seconds(8, [1_000_000] * 8)
+        sec = 7 * ks + ms
+        return {"value": 8 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle",
+                "sample": f"KDA layer: {s1} (x7 layers); MLA: {s2}; scaled to 8 sequences x 64 heads"}
+    if workload == "kda_prefill_32k":
+        T = 1024
+        q = rng.standard_normal((1, T, nth, D))
+        a = np.full((1, T, nth, D), 0.95)
+        b = np.full((1, T, nth), 0.5)
+        S = np.zeros((1, nth, D, D))
+        t0 = time.perf_counter()
+        oracle.kda_recurrent(q, q, q, a, b, S, nthreads=nth)
+        dt = time.perf_counter() - t0
+        sec = dt * (32768 / T) * (64 / nth)
+        return {"value": 32768 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle",
+                "sample": f"{nth} heads x {T} tokens, scaled to 64 heads x 32768 tokens"}
+    raise ValueError(workload)
+
+
+# ---------------------------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    cb = cpu_oracle_rate(args.workload)
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * _tokens(args.workload) / cb["value"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "implementation": "fp64 CPU oracle (plain C, OpenMP over heads)"},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _tokens(workload):
+    return {"hybrid_8layer_1m": 8, "kda_decode_b64": 64, "mla_decode_b16": 16, "kda_prefill_32k": 32768}[workload]
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="lad", choices=["lad", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import latent_attention_decode_b200 as lad
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    step = WORKLOADS[args.workload](lad, dev, rank)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    barrier(local)
+
+    # timed region: device events around exactly K steps, clocks sampled meanwhile
+    timer = KernelTimer()
+    clocks = ClockSampler(physical_gpu_index(local))
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    barrier(local)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step.run(timer)
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(local)
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms, dev)
+
+    # end to end through the public API: pinned host inputs in, outputs back, every step
+    for _ in range(3):
+        step.run_e2e()
+    torch.cuda.synchronize()
+    barrier(local)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step.run_e2e()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    barrier(local)
+
+    tokens = sum_over_ranks(float(step.tokens_per_step), dev)
+    value = tokens / (ms / 1000.0)
+    peaks = measured_peaks()
+    ab = step.algorithmic_bytes()
+    dom_ms = timer.mean_ms(step.dominant)
+    achieved = ab[step.dominant] / (dom_ms / 1000.0) / 1e9
+    per_type = {}
+    for kname in ("kda_decode_step", "mla_latent_decode", "kda_prefill_chunked"):
+        km = timer.mean_ms(kname)
+        if km is not None and kname in ab:
+            gbs = ab[kname] / (km / 1000.0) / 1e9
+            per_type[kname] = {"ms_per_launch": round(km, 4), "gb_s": round(gbs, 1),
+                               "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                               "frac_of_8tbs_spec": round(gbs / 8000.0, 4)}
+    if isinstance(step, PrefillStep) and dom_ms:
+        per_type["kda_prefill_chunked"]["tflop_s"] = round(step.flops() / (dom_ms / 1000.0) / 1e12, 1)
+    if isinstance(step, (MlaDecodeStep, HybridStep)):
+        m = step if isinstance(step, MlaDecodeStep) else step.mla
+        km = timer.mean_ms("mla_latent_decode")
+        per_type["mla_latent_decode"]["mma_tflop_s"] = round(m.mla_flops() / (km / 1000.0) / 1e12, 1)
+
+    if rank == 0:
+        cb = None
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_oracle_rate(args.workload)
+        hb, db = step.e2e_bytes()
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 inputs, fp32 state and accumulation", "data": "synthetic",
+            "config": {**step.config, "global_batch": int(round(tokens)) if not isinstance(step, PrefillStep)
+                       else world * step.cfg.B, "parallelism": f"sequence-sharded x{world}, no exchange"},
+            "per_layer_type": per_type,
+            "step_gb_s": ab["step"] / (ms / 1000.0) / 1e9,
+            "roofline": {"kernel": step.dominant, "bound": step.dominant_bound, "achieved": achieved,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": None, "peak_source": f"{peaks['source']} hbm_gbs (copy)",
+                         "algorithmic_bytes_per_launch": ab[step.dominant]},
+            "cpu_baseline": cb,
+            "e2e": {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": hb * world,
+                    "d2h_bytes_per_step": db * world},
+            "gpu_launches": step.launches_per_step * args.steps,
+            "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
+        }
+        print(json.dumps(line), flush=True)
+
+    if world > 1:
+        import torch.distributed as dist
+        barrier(local)
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,179 @@
+/*
+ * lad.h — C ABI of the hybrid-attention decode library (sm_100a / B200).
+ *
+ * The library computes the attention hot path of a 7:1 KDA : gated-MLA hybrid model of the
+ * Ling-3.1-flash kind, as described on two pages:
+ *   [P1] "Ling-3.1-flash and the 7:1 hybrid: how much KV cache does a 560B model need at 1M
+ *        tokens?" (dev.to)
+ *   [P2] "Ling-3.1-flash: a 560B hybrid-attention MoE, counted from its safetensors headers"
+ *        (ai.thesatyajit.com)
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller. The library keeps no state
+ *     between calls and allocates no device memory; where scratch space is needed the caller
+ *     passes a workspace whose size a *_workspace_size() query returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Every
+ *     call only enqueues work on that stream and returns; results are ready when the stream
+ *     reaches that point.
+ *   - Tensors are dense, row-major, in the index order written next to each argument.
+ *     bf16 tensors hold IEEE bfloat16 bit patterns (lad_bf16); fp32 tensors hold float.
+ *   - Return value: LAD_OK (0) or a negative status. On error nothing was launched, except
+ *     LAD_ECUDA from a launch, where the CUDA error is recorded in the message.
+ *     lad_last_error() returns a description of the calling thread's last error.
+ *   - Kernels that wait on on-chip barriers bound every wait; a wait that runs out sets a
+ *     device-side error word (read with lad_device_error()) and the kernel returns early
+ *     instead of hanging. Outputs of such a launch are undefined.
+ */
+#ifndef LAD_H
+#define LAD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t lad_bf16; /* IEEE bfloat16 bit pattern */
+
+/* status codes */
+#define LAD_OK 0
+#define LAD_EINVAL (-1)        /* null pointer, negative or inconsistent size */
+#define LAD_EUNSUPPORTED (-2)  /* a size or alignment this build does not implement */
+#define LAD_ECUDA (-3)         /* a CUDA runtime error (launch, attribute, device query) */
+#define LAD_EWORKSPACE (-4)    /* workspace missing or smaller than the query returned */
+
+/* flags */
+#define LAD_FLAG_SILU (1u << 0)      /* kda_conv_update: apply SiLU to the conv output */
+#define LAD_FLAG_L2NORM_QK (1u << 1) /* KDA calls: L2-normalise q and k per head in fp32 first */
+#define LAD_FLAG_OUT_FP32 (1u << 2)  /* KDA and MLA calls: write o as fp32 instead of bf16 */
+
+/* Description of the calling thread's most recent error ("" if none). */
+const char *lad_last_error(void);
+
+/* Library ABI version (major * 100 + minor). */
+int lad_version(void);
+
+/*
+ * Reads and clears the device-side error word that bounded waits set (see above), after
+ * synchronising `stream`. *code receives 0 when no kernel gave up a wait, else a nonzero tag
+ * naming the kernel and the wait. Returns LAD_OK or LAD_ECUDA.
+ */
+int lad_device_error(void *stream, int *code);
+
+/*
+ * kda_conv_update — one decode step of the short causal depthwise convolution in front of
+ * the KDA recurrence. [P2] "How KDA and MLA split the work": q, k and v come through a short
+ * causal convolution of width 4; [P2] "Does 292 GiB fit on four Hopper GPUs?": the layer keeps
+ * "convolution tails" (K-1 past inputs per channel).
+ *
+ * For every sequence b and channel c (the Cch channels are q|k|v, 3 x 8192 at the pages'
+ * shape):
+ *   y[b][c] = sum_{i<K-1} w[c][i] * tail[b][i][c] + w[c][K-1] * x[b][c]  (+ bias[c])
+ *   y       = y * sigmoid(y)                       if flags & LAD_FLAG_SILU
+ * then the tail drops its oldest row and appends x: tail[b][i] <- tail[b][i+1], tail[b][K-2] <- x[b].
+ * Arithmetic is fp32; y is rounded once to bf16 (round to nearest even).
+ *
+ *   x         bf16 [B][Cch]       new token (read)
+ *   conv_tail bf16 [B][K-1][Cch]  row 0 oldest (read and updated in place)
+ *   w         bf16 [Cch][K]       taps; w[c][K-1] multiplies the newest input
+ *   bias      bf16 [Cch] or NULL
+ *   y         bf16 [B][Cch]       output; must not alias x or conv_tail
+ * Supported: K == 4, Cch % 8 == 0, all pointers 16-byte aligned. B == 0 is a no-op.
+ */
+int kda_conv_update(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 *w, const lad_bf16 *bias,
+                    lad_bf16 *y, int B, int Cch, int K, unsigned flags, void *stream);
+
+/*
+ * kda_decode_step — one token of Kimi Delta Attention (gated delta rule) for B sequences and
+ * H heads. [P2] "How KDA and MLA split the work": each head keeps a 128x128 state, decays it
+ * channel by channel (alpha, per key channel) and writes the new key-value association with a
+ * per-head strength beta; [P1] "Why would a model keep only 9 full-attention layers?": KDA
+ * extends Gated DeltaNet with finer-grained gating. The page's display equation is lost; the
+ * update implemented (decay first, then the delta correction from the decayed state, readout
+ * after the write) is:
+ *   S'  = Diag(alpha) S
+ *   u   = beta * (v - S'^T k)
+ *   S   = S' + k u^T
+ *   o   = scale * S^T q
+ * with q, k L2-normalised first (x / sqrt(sum x^2 + 1e-6), fp32) if flags & LAD_FLAG_L2NORM_QK.
+ * All state arithmetic is fp32.
+ *
+ *   q, k      bf16, row (b, h) at q + b*qkv_batch_stride + h*dk     (read)
+ *   v         bf16, row (b, h) at v + b*qkv_batch_stride + h*dv     (read)
+ *   qkv_batch_stride  elements between sequences in q, k and v; 0 means dense [B][H][d].
+ *             (Pass 3*H*d with q, k, v pointing into kda_conv_update's y to consume it directly.)
+ *   alpha     fp32 [B][H][dk]     decay per key channel, in (0, 1]
+ *   beta      fp32 [B][H]         write strength
+ *   S         fp32 [B][H][dk][dv] state, rows = key channels (read and updated in place)
+ *   o         [B][H][dv], bf16, or fp32 if flags & LAD_FLAG_OUT_FP32
+ * Supported: dk == dv == 128; S 16-byte aligned. B == 0 or H == 0 is a no-op.
+ */
+int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, long long qkv_batch_stride,
+                    const float *alpha, const float *beta, float *S, void *o, int B, int H, int dk, int dv,
+                    float scale, unsigned flags, void *stream);
+
+/*
+ * kda_prefill_chunked — the same recurrence as kda_decode_step over T tokens per sequence,
+ * computed chunk by chunk (chunk length `chunk`, a shorter last chunk allowed) in the WY / UT
+ * form: inside a chunk with cumulative decays g_r = prod_{s<=r} alpha_s,
+ *   A = strict_lower(diag(beta) (K*g) (K/g)^T),  Tm = (I + A)^-1,
+ *   U = Tm diag(beta) (V - (K*g) S0),
+ *   O = scale ((Q*g) S0 + lower((Q*g)(K/g)^T) U),
+ *   S = Diag(g_last) S0 + (K * g_last/g)^T U.
+ * The pages do not print this form; it is the recurrence above unrolled within a chunk.
+ *
+ *   q, k, alpha  [B][T][H][dk] (q, k bf16; alpha fp32)
+ *   v            bf16 [B][T][H][dv]
+ *   beta         fp32 [B][T][H]
+ *   S            fp32 [B][H][dk][dv]  initial state in, final state out
+ *   o            [B][T][H][dv] bf16, or fp32 if flags & LAD_FLAG_OUT_FP32
+ *   workspace    device scratch of ws_bytes >= kda_prefill_workspace_size(...) (may be NULL
+ *                when that size is 0)
+ * Supported: dk == dv == 128, chunk == 64; flags LAD_FLAG_L2NORM_QK, LAD_FLAG_OUT_FP32.
+ * alpha must keep prod(alpha) over one chunk above ~1e-30 per channel (fp32 range of 1/g).
+ */
+int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, const float *alpha,
+                        const float *beta, float *S, void *o, int B, int T, int H, int dk, int dv, int chunk,
+                        float scale, unsigned flags, void *workspace, size_t ws_bytes, void *stream);
+size_t kda_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk);
+
+/*
+ * mla_latent_decode — gated Multi-head Latent Attention for one query token per sequence over
+ * the compressed latent cache. [P2] "How KDA and MLA split the work": ordinary softmax
+ * attention over a compressed cache whose rows hold a 512-dim latent plus a 64-dim RoPE key,
+ * and a sigmoid gate per head scales the result; [P1] "How big is the cache per token,
+ * exactly?": the cached row is kv_lora_rank + qk_rope_head_dim = 576 bf16 elements, the way
+ * latent-attention kernels cache it; [P1] "...plain multi-head attention would be absurd":
+ * the per-head key is 192 wide, hence the usual scale 1/sqrt(192).
+ * The query arrives absorbed (W_UK folded in, RoPE applied), d_latent + d_rope wide. For each
+ * sequence b with L = seq_lens[b] rows and each head h:
+ *   s_t = scale * <q[b][h], c_t>            over all d_latent + d_rope dims
+ *   o   = sum_t softmax(s)_t * c_t[0:d_latent]
+ *   o  *= sigmoid(gate_logits[b][h])        if gate_logits != NULL
+ *   lse = log sum_t exp(s_t)                (natural log, before the gate) if lse_out != NULL
+ * L == 0 gives o = 0 and lse = -inf. Scores and softmax are fp32; q.c and p.c run on the
+ * tensor cores with bf16 operands and fp32 accumulation.
+ *
+ *   q           bf16 [B][Hq][d_latent + d_rope]
+ *   cache       bf16, row t of sequence b at cache + b*cache_seq_stride + t*(d_latent+d_rope)
+ *   cache_seq_stride  elements between sequences (>= Lmax*(d_latent+d_rope), multiple of 8)
+ *   seq_lens    int32 [B] device, each in [0, Lmax]
+ *   gate_logits fp32 [B][Hq] or NULL
+ *   o           [B][Hq][d_latent] bf16, or fp32 if flags & LAD_FLAG_OUT_FP32
+ *   lse_out     fp32 [B][Hq] or NULL
+ *   workspace   device scratch, ws_bytes >= mla_latent_decode_workspace_size(B, Hq, d_latent, 0)
+ * Supported: Hq == 64, d_latent == 512, d_rope == 64; cache and q 16-byte aligned.
+ */
+int mla_latent_decode(const lad_bf16 *q, const lad_bf16 *cache, long long cache_seq_stride, const int *seq_lens,
+                      const float *gate_logits, void *o, float *lse_out, int B, int Hq, int d_latent, int d_rope,
+                      int Lmax, float scale, unsigned flags, void *workspace, size_t ws_bytes, void *stream);
+
+/* Workspace bytes mla_latent_decode needs; num_sms == 0 queries the current device. */
+size_t mla_latent_decode_workspace_size(int B, int Hq, int d_latent, int num_sms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LAD_H */

@@ -1,0 +1,253 @@
+"""Python binding of the hybrid-attention decode library (``liblad.so``, CUDA for sm_100a).
+
+Each function has the name of a C entry point in ``include/lad.h`` and only marshals arguments:
+it checks devices, dtypes and shapes of torch CUDA tensors, allocates outputs or workspace
+when the caller passes none, and hands raw pointers plus the current CUDA stream to the
+library. All arithmetic runs in the library's kernels; there is no other implementation, and
+importing this package fails loudly if ``liblad.so`` is missing (build it with
+``python -m latent_attention_decode_b200.build``).
+
+Flags and layouts are documented in ``include/lad.h``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "kda_conv_update", "kda_decode_step", "kda_prefill_chunked", "kda_prefill_workspace_size",
+    "mla_latent_decode", "mla_latent_decode_workspace_size", "lad_device_error", "lad_version",
+    "LadError", "LIB_PATH", "FLAG_SILU", "FLAG_L2NORM_QK", "FLAG_OUT_FP32", "MLA_SCALE",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblad.so")
+
+FLAG_SILU = 1 << 0
+FLAG_L2NORM_QK = 1 << 1
+FLAG_OUT_FP32 = 1 << 2
+MLA_SCALE = 1.0 / math.sqrt(192.0)
+
+_c_vp = ctypes.c_void_p
+_c_int = ctypes.c_int
+_c_ll = ctypes.c_longlong
+_c_f = ctypes.c_float
+_c_u = ctypes.c_uint
+_c_sz = ctypes.c_size_t
+
+
+class LadError(RuntimeError):
+    """A library call returned a nonzero status; the message is lad_last_error()."""
+
+    def __init__(self, fn: str, status: int, message: str):
+        super().__init__(f"{fn} failed with status {status}: {message}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m latent_attention_decode_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "lad_last_error": ([], ctypes.c_char_p),
+        "lad_version": ([], _c_int),
+        "lad_device_error": ([_c_vp, ctypes.POINTER(_c_int)], _c_int),
+        "kda_conv_update": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_u, _c_vp], _c_int),
+        "kda_decode_step": ([_c_vp, _c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
+                             _c_int, _c_f, _c_u, _c_vp], _c_int),
+        "kda_prefill_chunked": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
+                                 _c_int, _c_int, _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
+        "kda_prefill_workspace_size": ([_c_int] * 6, _c_sz),
+        "mla_latent_decode": ([_c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int,
+                               _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
+        "mla_latent_decode_workspace_size": ([_c_int] * 4, _c_sz),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise LadError(fn, status, _lib.lad_last_error().decode(errors="replace"))
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def _contig(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
+    _cuda(t, name, dtype)
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def lad_version() -> int:
+    return int(_lib.lad_version())
+
+
+def lad_device_error(stream=None) -> int:
+    """Synchronises the stream, returns and clears the device error word (0 = no wait gave up)."""
+    code = _c_int(0)
+    _check("lad_device_error", _lib.lad_device_error(_stream(stream), ctypes.byref(code)))
+    return int(code.value)
+
+
+def kda_conv_update(x: torch.Tensor, conv_tail: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None,
+                    bias: torch.Tensor | None = None, silu: bool = True, stream=None) -> torch.Tensor:
+    """One step of the width-K causal conv. x [B,Cch], conv_tail [B,K-1,Cch] (updated), w [Cch,K]."""
+    bf = torch.bfloat16
+    _contig(x, "x", bf), _contig(conv_tail, "conv_tail", bf), _contig(w, "w", bf)
+    B, Cch = x.shape
+    K = w.shape[1]
+    if conv_tail.shape != (B, K - 1, Cch) or w.shape != (Cch, K):
+        raise ValueError("kda_conv_update: inconsistent shapes")
+    if bias is not None:
+        _contig(bias, "bias", bf)
+    if y is None:
+        y = torch.empty_like(x)
+    _contig(y, "y", bf)
+    flags = FLAG_SILU if silu else 0
+    _check("kda_conv_update", _lib.kda_conv_update(x.data_ptr(), conv_tail.data_ptr(), w.data_ptr(), _ptr(bias),
+                                                   y.data_ptr(), B, Cch, K, flags, _stream(stream)))
+    return y
+
+
+def _rows(t: torch.Tensor, name: str, B: int, H: int, d: int) -> int:
+    """Batch stride (elements) of a [B,H,d] or [B,H*d] bf16 view whose per-sequence block is dense."""
+    _cuda(t, name, torch.bfloat16)
+    if t.shape == (B, H, d):
+        dense = t.stride(2) == 1 and t.stride(1) == d
+    elif t.shape == (B, H * d):
+        dense = t.stride(1) == 1
+    else:
+        raise ValueError(f"{name} must be [B,H,{d}] or [B,H*{d}], got {tuple(t.shape)}")
+    if not dense:
+        raise ValueError(f"{name}: each sequence's H*{d} block must be contiguous")
+    return t.stride(0) if B > 1 else H * d
+
+
+def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor,
+                    S: torch.Tensor, o: torch.Tensor | None = None, scale: float = 1.0, l2norm_qk: bool = False,
+                    out_fp32: bool = False, stream=None) -> torch.Tensor:
+    """One KDA token: S [B,H,128,128] fp32 updated in place; returns o [B,H,128].
+
+    q, k, v may be [B,H,128] or [B,H*128] views sharing one batch stride (for example the
+    q, k and v thirds of kda_conv_update's output).
+    """
+    _contig(S, "S", torch.float32)
+    B, H, dk, dv = S.shape
+    sq, sk, sv = _rows(q, "q", B, H, dk), _rows(k, "k", B, H, dk), _rows(v, "v", B, H, dv)
+    if not (sq == sk == sv):
+        raise ValueError("q, k and v must share one batch stride")
+    _contig(alpha, "alpha", torch.float32), _contig(beta, "beta", torch.float32)
+    if alpha.numel() != B * H * dk or beta.numel() != B * H:
+        raise ValueError("alpha must be [B,H,dk] and beta [B,H]")
+    odt = torch.float32 if out_fp32 else torch.bfloat16
+    if o is None:
+        o = torch.empty((B, H, dv), device=S.device, dtype=odt)
+    _contig(o, "o", odt)
+    flags = (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
+    _check("kda_decode_step", _lib.kda_decode_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), sq, alpha.data_ptr(),
+                                                   beta.data_ptr(), S.data_ptr(), o.data_ptr(), B, H, dk, dv,
+                                                   float(scale), flags, _stream(stream)))
+    return o
+
+
+def kda_prefill_workspace_size(B: int, T: int, H: int, dk: int = 128, dv: int = 128, chunk: int = 64) -> int:
+    return int(_lib.kda_prefill_workspace_size(B, T, H, dk, dv, chunk))
+
+
+def kda_prefill_chunked(q, k, v, alpha, beta, S, o=None, chunk: int = 64, scale: float = 1.0,
+                        l2norm_qk: bool = False, out_fp32: bool = False, workspace=None, stream=None):
+    """KDA over T tokens in chunks: q,k,alpha [B,T,H,128], v [B,T,H,128], beta [B,T,H]; S in/out."""
+    bf = torch.bfloat16
+    _contig(q, "q", bf), _contig(k, "k", bf), _contig(v, "v", bf)
+    _contig(alpha, "alpha", torch.float32), _contig(beta, "beta", torch.float32), _contig(S, "S", torch.float32)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or alpha.shape != q.shape or v.shape != (B, T, H, dv) or beta.shape != (B, T, H) \
+            or S.shape != (B, H, dk, dv):
+        raise ValueError("kda_prefill_chunked: inconsistent shapes")
+    odt = torch.float32 if out_fp32 else bf
+    if o is None:
+        o = torch.empty((B, T, H, dv), device=q.device, dtype=odt)
+    _contig(o, "o", odt)
+    ws = kda_prefill_workspace_size(B, T, H, dk, dv, chunk)
+    if workspace is None and ws > 0:
+        workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
+    flags = (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
+    _check("kda_prefill_chunked", _lib.kda_prefill_chunked(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), alpha.data_ptr(), beta.data_ptr(), S.data_ptr(), o.data_ptr(),
+        B, T, H, dk, dv, chunk, float(scale), flags, _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o
+
+
+def mla_latent_decode_workspace_size(B: int, Hq: int = 64, d_latent: int = 512, num_sms: int = 0) -> int:
+    return int(_lib.mla_latent_decode_workspace_size(B, Hq, d_latent, num_sms))
+
+
+def mla_latent_decode(q: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tensor,
+                      gate_logits: torch.Tensor | None = None, o: torch.Tensor | None = None,
+                      lse: torch.Tensor | None = None, scale: float = MLA_SCALE, d_latent: int = 512,
+                      out_fp32: bool = False, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Gated latent attention: q [B,Hq,576], cache [B,Lmax,576] (rows contiguous), seq_lens int32 [B].
+
+    Returns o [B,Hq,d_latent]; fills lse [B,Hq] when given.
+    """
+    bf = torch.bfloat16
+    _contig(q, "q", bf)
+    _cuda(cache, "cache", bf)
+    B, Hq, D = q.shape
+    if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != D or cache.stride(2) != 1 \
+            or cache.stride(1) != D:
+        raise ValueError("cache must be [B,Lmax,D] with contiguous rows")
+    Lmax = cache.shape[1]
+    _contig(seq_lens, "seq_lens", torch.int32)
+    if seq_lens.shape != (B,):
+        raise ValueError("seq_lens must be [B]")
+    if gate_logits is not None:
+        _contig(gate_logits, "gate_logits", torch.float32)
+        if gate_logits.shape != (B, Hq):
+            raise ValueError("gate_logits must be [B,Hq]")
+    odt = torch.float32 if out_fp32 else bf
+    if o is None:
+        o = torch.empty((B, Hq, d_latent), device=q.device, dtype=odt)
+    _contig(o, "o", odt)
+    if lse is not None:
+        _contig(lse, "lse", torch.float32)
+    ws = mla_latent_decode_workspace_size(B, Hq, d_latent, 0)
+    if workspace is None and ws > 0:
+        workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
+    flags = FLAG_OUT_FP32 if out_fp32 else 0
+    seq_stride = cache.stride(0) if B > 1 else Lmax * D
+    _check("mla_latent_decode", _lib.mla_latent_decode(
+        q.data_ptr(), cache.data_ptr(), seq_stride, seq_lens.data_ptr(), _ptr(gate_logits), o.data_ptr(),
+        _ptr(lse), B, Hq, d_latent, D - d_latent, Lmax, float(scale), flags, _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o

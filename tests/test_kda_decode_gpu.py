@@ -1,0 +1,171 @@
+"""Parity of kda_conv_update and kda_decode_step (CUDA, through the C ABI) with the fp64 oracle.
+
+Inputs come from the seeded workload recipes; the oracle sees the same bf16/fp32 values widened
+exactly to fp64. Tolerances are in tests/parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from tests.parity import TOL_OUT, TOL_STATE, bf16_round, f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lad(cuda_device):
+    import latent_attention_decode_b200 as m
+    return m
+
+
+def _scan(lad, inp, out_fp32, dev, scale=1.0, l2=False):
+    q, k, v, a, b = (inp[n].to(dev) for n in ("q", "k", "v", "alpha", "beta"))
+    S = inp["S0"].to(dev).clone()
+    B, T, H, _ = q.shape
+    outs = []
+    for t in range(T):
+        outs.append(lad.kda_decode_step(q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(),
+                                        a[:, t].contiguous(), b[:, t].contiguous(), S, scale=scale,
+                                        out_fp32=out_fp32, l2norm_qk=l2))
+    torch.cuda.synchronize()
+    return torch.stack(outs, dim=1), S
+
+
+def _oracle_scan(inp, scale=1.0, l2=False):
+    q, k = f64(inp["q"]), f64(inp["k"])
+    if l2:
+        q, k = oracle.l2norm(q), oracle.l2norm(k)
+    return oracle.kda_recurrent(q, k, f64(inp["v"]), f64(inp["alpha"]), f64(inp["beta"]), f64(inp["S0"]),
+                                scale=scale, nthreads=oracle.max_threads())
+
+
+def test_scan_tiny_256_steps(lad, cuda_device):
+    """B=1, H=4, 256 tokens from zero state: every o_t and the final state."""
+    inp = wl.kda_scan_inputs(wl.CONFIGS["kda_scan_tiny"])
+    o_ref, S_ref = _oracle_scan(inp)
+    o32, S = _scan(lad, inp, True, cuda_device)
+    assert rel_l2(o32, o_ref) < 1e-5
+    assert rel_l2(S, S_ref) < TOL_STATE
+    o16, _ = _scan(lad, inp, False, cuda_device)
+    assert rel_l2(o16, o_ref) < TOL_OUT
+    assert rel_l2(o16, bf16_round(o_ref)) < 2e-4
+
+
+def test_scan_uniform_decay_nonzero_state_scaled(lad, cuda_device):
+    """Every channel decays differently (alpha ~ U[0.9,1)), a live initial state, scale != 1."""
+    cfg = wl.KdaScan("u", B=2, H=3, T=64, seed=99, state_std=0.02, alpha_mode="uniform")
+    inp = wl.kda_scan_inputs(cfg)
+    o_ref, S_ref = _oracle_scan(inp, scale=0.125)
+    o, S = _scan(lad, inp, True, cuda_device, scale=0.125)
+    assert rel_l2(o, o_ref) < 1e-5 and rel_l2(S, S_ref) < TOL_STATE
+
+
+def test_l2norm_flag(lad, cuda_device):
+    """Unnormalised q, k with the in-kernel L2 normalisation."""
+    cfg = wl.KdaScan("n", B=1, H=2, T=16, seed=5, state_std=0.02)
+    inp = wl.kda_scan_inputs(cfg)
+    inp["q"] = wl.normal_bf16(inp["q"].shape, 5, "qraw", std=3.0)
+    inp["k"] = wl.normal_bf16(inp["k"].shape, 5, "kraw", std=0.5)
+    o_ref, S_ref = _oracle_scan(inp, l2=True)
+    o, S = _scan(lad, inp, True, cuda_device, l2=True)
+    assert rel_l2(o, o_ref) < 1e-5 and rel_l2(S, S_ref) < TOL_STATE
+
+
+def test_identity_step_is_exact(lad, cuda_device):
+    """alpha = 1, beta = 0 leaves the fp32 state bit-identical."""
+    cfg = wl.KdaScan("i", B=2, H=5, T=1, seed=3, state_std=0.02)
+    inp = wl.kda_scan_inputs(cfg)
+    inp["alpha"] = torch.ones_like(inp["alpha"])
+    inp["beta"] = torch.zeros_like(inp["beta"])
+    _, S = _scan(lad, inp, True, cuda_device)
+    assert torch.equal(S.cpu(), inp["S0"])
+
+
+def test_unit_key_full_write(lad, cuda_device):
+    """||k|| = 1 (normalised in-kernel) and beta = 1: S^T k = v after the step, to fp32 rounding."""
+    cfg = wl.KdaScan("w", B=1, H=4, T=1, seed=4, state_std=0.02)
+    inp = wl.kda_scan_inputs(cfg)
+    inp["beta"] = torch.ones_like(inp["beta"])
+    _, S = _scan(lad, inp, True, cuda_device, l2=True)
+    k = oracle.l2norm(f64(inp["k"]))[0, 0]
+    v = f64(inp["v"])[0, 0]
+    Sk = np.einsum("hij,hi->hj", f64(S)[0], k)
+    assert np.abs(Sk - v).max() < 1e-5
+
+
+def test_decode_b64_conv_then_step(lad, cuda_device):
+    """The Ling-shape decode step: conv update of q|k|v for 64 sequences, then the KDA step on
+    the conv output (L2-normalised in-kernel) for 64 heads, states ~N(0, 0.02)."""
+    cfg = wl.CONFIGS["kda_decode_b64"]
+    inp = wl.kda_decode_inputs(cfg, cuda_device)
+    B, H, d = cfg.B, cfg.H, 128
+    x, tail, w = (f64(inp[n]) for n in ("x", "tail", "w"))
+    y_ref, tail_ref = oracle.short_conv_step(x, tail, w, None, silu=True)
+    y_ref16 = bf16_round(y_ref)   # the interface stores y in bf16
+    qr = oracle.l2norm(y_ref16[:, : H * d].reshape(B, 1, H, d))
+    kr = oracle.l2norm(y_ref16[:, H * d: 2 * H * d].reshape(B, 1, H, d))
+    vr = y_ref16[:, 2 * H * d:].reshape(B, 1, H, d)
+    o_ref, S_ref = oracle.kda_recurrent(qr, kr, vr, f64(inp["alpha"])[:, None], f64(inp["beta"])[:, None],
+                                        f64(inp["S"]), nthreads=oracle.max_threads())
+
+    y = lad.kda_conv_update(inp["x"], inp["tail"], inp["w"], silu=True)
+    o = lad.kda_decode_step(y[:, : H * d], y[:, H * d: 2 * H * d], y[:, 2 * H * d:], inp["alpha"], inp["beta"],
+                            inp["S"], l2norm_qk=True, out_fp32=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(f64(inp["tail"]), tail_ref)
+    yg = f64(y)
+    assert rel_l2(yg, y_ref) < TOL_OUT
+    # fp32 arithmetic then one bf16 rounding: at most one bf16 step away from the rounded oracle
+    assert np.all(np.abs(yg - y_ref16) <= np.abs(y_ref16) * 2.0 ** -7 + 1e-30)
+    assert rel_l2(o, o_ref[:, 0]) < 1e-4
+    assert rel_l2(inp["S"], S_ref) < TOL_STATE
+
+
+@pytest.mark.parametrize("B,H", [(1, 1), (3, 7), (256, 64)])
+def test_shapes(lad, cuda_device, B, H):
+    cfg = wl.KdaDecode("s", B=B, H=H, seed=11 + B)
+    inp = wl.kda_decode_inputs(cfg, cuda_device)
+    q = wl.unit_sphere_bf16((B, H, 128), 7, "q", cuda_device)
+    k = wl.unit_sphere_bf16((B, H, 128), 7, "k", cuda_device)
+    v = wl.normal_bf16((B, H, 128), 7, "v", cuda_device)
+    sel = [0, B // 2, B - 1]
+    S0 = f64(inp["S"][sel])
+    o = lad.kda_decode_step(q, k, v, inp["alpha"], inp["beta"], inp["S"], out_fp32=True)
+    torch.cuda.synchronize()
+    o_ref, S_ref = oracle.kda_recurrent(f64(q[sel])[:, None], f64(k[sel])[:, None], f64(v[sel])[:, None],
+                                        f64(inp["alpha"][sel])[:, None], f64(inp["beta"][sel])[:, None], S0,
+                                        nthreads=oracle.max_threads())
+    assert rel_l2(o[sel], o_ref[:, 0]) < 1e-5
+    assert rel_l2(inp["S"][sel], S_ref) < TOL_STATE
+
+
+def test_empty_batch_is_noop(lad, cuda_device):
+    S = torch.zeros((0, 64, 128, 128), device=cuda_device)
+    z = torch.zeros((0, 64, 128), device=cuda_device, dtype=torch.bfloat16)
+    o = lad.kda_decode_step(z, z, z, torch.zeros((0, 64, 128), device=cuda_device),
+                            torch.zeros((0, 64), device=cuda_device), S)
+    assert o.shape == (0, 64, 128)
+
+
+@pytest.mark.parametrize("silu,bias", [(False, False), (True, True)])
+def test_conv_variants(lad, cuda_device, silu, bias):
+    B, C = 5, 96
+    inp = wl.conv_inputs(B, 21, cuda_device, channels=C)
+    bvec = wl.normal_bf16((C,), 21, "bias", cuda_device) if bias else None
+    y_ref, tail_ref = oracle.short_conv_step(f64(inp["x"]), f64(inp["tail"]), f64(inp["w"]),
+                                             None if bvec is None else f64(bvec), silu=silu)
+    y = lad.kda_conv_update(inp["x"], inp["tail"], inp["w"], bias=bvec, silu=silu)
+    torch.cuda.synchronize()
+    assert np.array_equal(f64(inp["tail"]), tail_ref)
+    assert rel_l2(y, y_ref) < TOL_OUT
+    y16 = bf16_round(y_ref)
+    assert np.all(np.abs(f64(y) - y16) <= np.abs(y16) * 2.0 ** -7 + 1e-30)
+
+
+def test_conv_rejects_bad_width(lad, cuda_device):
+    inp = wl.conv_inputs(2, 1, cuda_device, channels=16, width=3)
+    with pytest.raises(lad.LadError) as e:
+        lad.kda_conv_update(inp["x"], inp["tail"], inp["w"])
+    assert e.value.status == -2
