@@ -1,16 +1,819 @@
-// Gated MLA latent decode (placeholder entry points; the kernel follows).
+// Gated MLA latent decode on B200: split-KV over the compressed 576-wide cache, tensor cores
+// (tcgen05) for both contractions, TMA-fed, with a log-sum-exp combine and the sigmoid gate.
+//
+// Sources: "Ling-3.1-flash: a 560B hybrid-attention MoE, counted from its safetensors headers",
+// section "How KDA and MLA split the work" (gated MLA is ordinary softmax attention over a
+// compressed cache of a 512-dim latent plus a 64-dim RoPE key per token; a sigmoid gate per
+// head scales the result); "Ling-3.1-flash and the 7:1 hybrid: how much KV cache does a 560B
+// model need at 1M tokens?", section "How big is the cache per token, exactly?" (576 bf16 values
+// per token, read in full at every decoding step; 192-wide per-head key, hence 1/sqrt(192)).
+//
+// For sequence b (L rows c_t) and head h, with the absorbed query q_h (576 wide):
+//   s_t = scale <q_h, c_t>,  o_h = sigmoid(g_h) * sum_t softmax(s)_t c_t[0:512].
+//
+// Work split. Every sequence is cut into tiles of 32 cached rows; the tiles of all sequences,
+// concatenated, are divided evenly between one CTA per SM. A CTA's share is a run of
+// "segments" (its tiles of one sequence); each segment leaves an unnormalised partial
+// (O, running max m, running sum l) in the workspace, and a second kernel merges the partials
+// of each sequence by log-sum-exp and applies the gate.
+//
+// Per tile, two contractions run on the tensor cores (bf16 operands, fp32 accumulation in TMEM):
+//   GEMM1  S[h][t]  = q[h][:] . c_t          M = 64 heads, N = 32 tokens, K = 576
+//   GEMM2  O^T[d][h] += sum_t c_t[d] P[h][t]  M = 128 latent dims (x4), N = 64 heads, K = 32
+// GEMM2 is written transposed so that its M is the 512 latent dimensions and runs at the full
+// 128-row rate; its A operand is the same cache tile GEMM1 used as B, read MN-major, so every
+// cached byte crosses HBM once. P (bf16) goes through shared memory.
+//
+// Roles (256 threads): warp 0 issues TMA loads (q once per segment, then a 4-deep ring of
+// 36 KiB cache tiles), warp 1 owns TMEM and issues the MMAs, warps 4-7 run the online softmax
+// (one head per lane, lanes 0-15 of each warp: the M = 64 accumulator occupies rows 16p..16p+15
+// of TMEM sub-partition p), rescale O when a head's running max grows by more than 2^8
+// (lazily, like FlashAttention-4), and write the segment's partial at its end.
+//
+// Every wait on an mbarrier is bounded (see lad_common.cuh); a wait that runs out records a tag
+// in the device error word, raises an abort flag the other roles see, and the CTA drains its
+// own copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+
+#include <cstring>
+#include <mutex>
+
 #include "lad_common.cuh"
 
+namespace {
+
+using lad::dev::globaltimer_ns;
+using lad::dev::kWaitLimitNs;
+
+constexpr int kHq = 64;            // query heads
+constexpr int kDl = 512;           // latent (value) width
+constexpr int kDr = 64;            // rope width
+constexpr int kDrow = kDl + kDr;   // 576 bf16 per cached row
+constexpr int kChunk = 64;         // bf16 per 128-byte swizzle row
+constexpr int kNChunk = kDrow / kChunk;  // 9
+constexpr int kTile = 32;          // cached rows per tile
+constexpr int kStages = 4;
+constexpr int kThreads = 256;
+
+constexpr int kQChunkBytes = kHq * 128;                 // 8 KiB: 64 heads x 64 dims
+constexpr int kQBytes = kNChunk * kQChunkBytes;         // 73,728
+constexpr int kTChunkBytes = kTile * 128;               // 4 KiB: 32 rows x 64 dims
+constexpr int kStageBytes = kNChunk * kTChunkBytes;     // 36,864
+constexpr int kPBytes = kHq * kTile * 2;                // 4 KiB: P[64 heads][32 tokens] bf16
+
+constexpr int kOffQ = 0;
+constexpr int kOffStage = kOffQ + kQBytes;                       // 73,728
+constexpr int kOffP = kOffStage + kStages * kStageBytes;         // 221,184
+constexpr int kOffBar = kOffP + 2 * kPBytes;                     // 229,376
+constexpr int kSmemBytes = kOffBar + 1024 + 1024;                // + barriers/scalars + alignment slack
+
+// TMEM columns (fp32): O^T blocks 0..255, S buffers 256..287 and 288..319.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 0;
+constexpr uint32_t kColS = 256;
+
+// barrier slots (8 bytes each) inside the kOffBar region
+enum Bar : int {
+    kBarFull = 0,                 // [kStages]   TMA -> MMA: cache tile landed
+    kBarEmpty = kBarFull + kStages,  // [kStages] MMA -> TMA: tile consumed by GEMM2
+    kBarSFull = kBarEmpty + kStages,   // [2] GEMM1 done
+    kBarSEmpty = kBarSFull + 2,        // [2] softmax has read S
+    kBarPFull = kBarSEmpty + 2,        // [2] P written (and O rescaled)
+    kBarPEmpty = kBarPFull + 2,        // [2] GEMM2 of the tile that used this P buffer is complete
+    kBarWg = kBarPEmpty + 2,           // [2] softmax warps exchanged their rescale decisions
+    kBarOFree = kBarWg + 2,            // epilogue has read O
+    kBarQFull = kBarOFree + 1,         // q of a segment landed
+    kBarQEmpty = kBarQFull + 1,        // GEMM1s of a segment done with q
+    kBarDrain = kBarQEmpty + 1,        // final MMA drain
+    kNumBars = kBarDrain + 1,
+};
+constexpr int kOffScalars = kNumBars * 8;  // inside the barrier region: tmem base, abort flag, ...
+
+__device__ int g_mla_error = 0;
+
+// ------------------------------------------------------------------------------------------
+// PTX wrappers
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase of `bar` with parity `parity`. Returns false if the CTA is
+// aborting (this wait ran out, or another role's did).
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag, int tag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicCAS(&g_mla_error, 0, tag);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (bf16 in, fp32 accumulate)
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+#define LAD_TMEM_LD32(taddr, r)                                                                                      \
+    asm volatile(                                                                                                    \
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18," \
+        "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                                              \
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),           \
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),     \
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),   \
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])    \
+        : "r"(taddr))
+
+#define LAD_TMEM_ST32(taddr, r)                                                                                      \
+    asm volatile(                                                                                                    \
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17," \
+        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),                              \
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),         \
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), \
+        "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]),            \
+        "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])                                      \
+        : "memory")
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ------------------------------------------------------------------------------------------
+// UMMA descriptors
+// ------------------------------------------------------------------------------------------
+// Shared-memory matrix descriptor: start address, leading / stride byte offsets (16-byte
+// units), descriptor version 1, layout type in bits 61..63.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;  // version
+    d |= static_cast<uint64_t>(layout & 7u) << 61;
+    return d;
+}
+constexpr uint32_t kLayoutSw128 = 2;
+constexpr uint32_t kLayoutNone = 0;
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, majors, N >> 3, M >> 4.
+constexpr uint32_t make_idesc(int M, int N, int a_mn_major, int b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn_major) << 15) |
+           (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+constexpr uint32_t kIdesc1 = make_idesc(64, kTile, 0, 0);   // S = q . C^T
+constexpr uint32_t kIdesc2 = make_idesc(128, kHq, 1, 0);    // O^T += V^T . P^T
+
+// ------------------------------------------------------------------------------------------
+// work split
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ int tiles_of(int len) { return (len + kTile - 1) / kTile; }
+
+__device__ __forceinline__ long long split_point(long long total, int parts, int c) {
+    return total * c / parts;
+}
+
+// Iterates the segments (runs of tiles of one sequence) of a CTA's tile range [t, t_end).
+struct SegIter {
+    const int *lens;
+    int B;
+    int b;             // current sequence
+    long long base;    // first global tile of sequence b
+    long long t, t_end;
+
+    __device__ bool next(int &seq, int &tile0, int &ntiles) {
+        while (t < t_end && b < B) {
+            const long long nb = tiles_of(lens[b]);
+            if (t < base + nb) {
+                const long long end = (t_end < base + nb) ? t_end : base + nb;
+                seq = b;
+                tile0 = static_cast<int>(t - base);
+                ntiles = static_cast<int>(end - t);
+                t = end;
+                if (t == base + nb) {
+                    base += nb;
+                    ++b;
+                }
+                return true;
+            }
+            base += nb;
+            ++b;
+        }
+        return false;
+    }
+};
+
+struct Partials {
+    float *O;        // [slots][64][512]
+    float *m;        // [slots][64]   running max, log2 units of the scaled score
+    float *l;        // [slots][64]
+    long long *tile_prefix;  // [B + 1]
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_constant__ CUtensorMap map_q,
+                 const int *__restrict__ seq_lens, int B, float score_scale_log2, Partials ws) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bars = sbase + kOffBar;
+    auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + kOffScalars);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + kOffScalars + 4);
+    long long *range = reinterpret_cast<long long *>(smem + kOffBar + kOffScalars + 8);  // [0]=t0 [1]=t1 [2]=b0 [3]=base0
+    float *rescale = reinterpret_cast<float *>(smem + kOffBar + kOffScalars + 64);         // [2][64]
+    int *any_rescale = reinterpret_cast<int *>(smem + kOffBar + kOffScalars + 64 + 512);   // [2][4]
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- the CTA's tile range; warp 2 scans the lengths (and CTA 0 publishes the prefix) ----
+    if (warp == 2) {
+        long long run = 0;
+        for (int b0 = 0; b0 < B; b0 += 32) {
+            const int b = b0 + lane;
+            long long n = (b < B) ? tiles_of(seq_lens[b]) : 0;
+            long long incl = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                long long y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (blockIdx.x == 0 && b < B) ws.tile_prefix[b] = run + incl - n;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (blockIdx.x == 0 && lane == 0) ws.tile_prefix[B] = run;
+        if (lane == 0) {
+            const long long t0 = split_point(run, gridDim.x, blockIdx.x);
+            const long long t1 = split_point(run, gridDim.x, blockIdx.x + 1);
+            long long base = 0;
+            int b = 0;
+            while (b < B) {
+                const long long nb = tiles_of(seq_lens[b]);
+                if (t0 < base + nb) break;
+                base += nb;
+                ++b;
+            }
+            range[0] = t0;
+            range[1] = t1;
+            range[2] = b;
+            range[3] = base;
+        }
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNumBars; ++i) {
+            uint32_t count = 1;
+            if (i == kBarSEmpty || i == kBarSEmpty + 1 || i == kBarPFull || i == kBarPFull + 1 || i == kBarWg ||
+                i == kBarWg + 1 || i == kBarOFree)
+                count = 4;  // one arrival per softmax warp
+            mbar_init(bar(i), count);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const long long t0 = range[0], t1 = range[1];
+    if (t0 >= t1) return;  // no work for this CTA (uniform exit before TMEM is touched)
+
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_base_slot)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_slot;
+
+    SegIter it{seq_lens, B, static_cast<int>(range[2]), range[3], t0, t1};
+
+    if (warp == 0) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            int seq, tile0, nt, k = 0;
+            uint32_t g = 0;
+            bool ok = true;
+            while (ok && it.next(seq, tile0, nt)) {
+                if (k > 0 && !wait_bar(bar(kBarQEmpty), (k - 1) & 1, abort_flag, lad::kErrMlaProducer)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_tx(bar(kBarQFull), kQBytes);
+                for (int c = 0; c < kNChunk; ++c)
+                    tma_load_2d(sbase + kOffQ + c * kQChunkBytes, &map_q, c * kChunk, seq * kHq, bar(kBarQFull));
+                for (int i = 0; i < nt; ++i, ++g) {
+                    const uint32_t s = g % kStages;
+                    if (!wait_bar(bar(kBarEmpty + s), ((g / kStages) & 1) ^ 1, abort_flag, lad::kErrMlaProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_tx(bar(kBarFull + s), kStageBytes);
+                    const uint32_t dst = sbase + kOffStage + s * kStageBytes;
+                    for (int c = 0; c < kNChunk; ++c)
+                        tma_load_3d(dst + c * kTChunkBytes, &map_cache, c * kChunk, (tile0 + i) * kTile, seq,
+                                    bar(kBarFull + s));
+                }
+                ++k;
+            }
+            if (!ok) {
+                // drain: every load this thread issued completes on its full barrier
+                const uint32_t issued = g;
+                for (uint32_t j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
+                    const uint32_t s = j % kStages;
+                    const uint64_t tt = globaltimer_ns();
+                    while (!mbar_try_wait(bar(kBarFull + s), (j / kStages) & 1) &&
+                           globaltimer_ns() - tt < kWaitLimitNs) {
+                    }
+                }
+                if (k > 0) {
+                    const uint64_t tt = globaltimer_ns();
+                    while (!mbar_try_wait(bar(kBarQFull), (k - 1) & 1) && globaltimer_ns() - tt < kWaitLimitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            int seq, tile0, nt, k = 0;
+            uint32_t g = 0;
+            bool ok = true;
+            // the previous tile's GEMM2 is issued after the current tile's GEMM1
+            bool have_prev = false;
+            uint32_t prev_g = 0;
+            bool prev_first = false;
+            int prev_seg = 0;
+            auto gemm2 = [&](uint32_t gg, bool first_of_seg, int seg) -> bool {
+                const uint32_t pb = gg & 1;
+                if (!wait_bar(bar(kBarPFull + pb), (gg >> 1) & 1, abort_flag, lad::kErrMlaMma)) return false;
+                if (first_of_seg && seg > 0 &&
+                    !wait_bar(bar(kBarOFree), (seg - 1) & 1, abort_flag, lad::kErrMlaMma))
+                    return false;
+                tc_fence_after();
+                const uint32_t s = gg % kStages;
+                const uint32_t vbase = sbase + kOffStage + s * kStageBytes;
+                const uint32_t pbase = sbase + kOffP + pb * kPBytes;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk) {
+                        // A = V^T: 128 latent dims (two 64-wide chunks, LBO apart) x 16 tokens (two 8-row groups)
+                        const uint64_t a = smem_desc(vbase + (2 * j) * kTChunkBytes + kk * 2048, kTChunkBytes, 1024,
+                                                     kLayoutSw128);
+                        // B = P: 64 heads (8-row core groups, SBO 512) x 16 tokens (two 8-token core columns, LBO 128)
+                        const uint64_t bdesc = smem_desc(pbase + kk * 256, 128, 512, kLayoutNone);
+                        tc_mma(tmem + kColO + 64 * j, a, bdesc, kIdesc2, (first_of_seg && kk == 0) ? 0u : 1u);
+                    }
+                }
+                tc_commit(bar(kBarEmpty + s));
+                tc_commit(bar(kBarPEmpty + pb));
+                return true;
+            };
+            while (ok && it.next(seq, tile0, nt)) {
+                if (!wait_bar(bar(kBarQFull), k & 1, abort_flag, lad::kErrMlaMma)) {
+                    ok = false;
+                    break;
+                }
+                for (int i = 0; i < nt; ++i, ++g) {
+                    const uint32_t s = g % kStages;
+                    const uint32_t sb = g & 1;
+                    if (!wait_bar(bar(kBarFull + s), (g / kStages) & 1, abort_flag, lad::kErrMlaMma) ||
+                        !wait_bar(bar(kBarSEmpty + sb), ((g >> 1) & 1) ^ 1, abort_flag, lad::kErrMlaMma)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t cbase = sbase + kOffStage + s * kStageBytes;
+#pragma unroll 1
+                    for (int c = 0; c < kNChunk; ++c) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t a = smem_desc(sbase + kOffQ + c * kQChunkBytes + kk * 32, 16, 1024,
+                                                         kLayoutSw128);
+                            const uint64_t bdesc = smem_desc(cbase + c * kTChunkBytes + kk * 32, 16, 1024,
+                                                             kLayoutSw128);
+                            tc_mma(tmem + kColS + sb * kTile, a, bdesc, kIdesc1, (c | kk) ? 1u : 0u);
+                        }
+                    }
+                    tc_commit(bar(kBarSFull + sb));
+                    if (i == nt - 1) tc_commit(bar(kBarQEmpty));
+                    if (have_prev && !gemm2(prev_g, prev_first, prev_seg)) {
+                        ok = false;
+                        break;
+                    }
+                    have_prev = true;
+                    prev_g = g;
+                    prev_first = (i == 0);
+                    prev_seg = k;
+                }
+                ++k;
+            }
+            if (ok && have_prev) ok = gemm2(prev_g, prev_first, prev_seg);
+            // drain every MMA this thread issued before TMEM is released
+            tc_commit(bar(kBarDrain));
+            const uint64_t tt = globaltimer_ns();
+            while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer_ns() - tt < kWaitLimitNs) {
+            }
+        }
+    } else if (warp >= 4) {
+        // ================= softmax, rescale and epilogue (warps 4..7) =================
+        const int p = warp & 3;                 // TMEM sub-partition
+        const bool owner = lane < 16;           // this lane owns head 16p + lane
+        const int h = 16 * p + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * p) << 16;
+        int seq, tile0, nt, k = 0;
+        uint32_t g = 0;
+        bool ok = true;
+        float m = -INFINITY, l = 0.f;
+        while (ok && it.next(seq, tile0, nt)) {
+            const int len = seq_lens[seq];
+            for (int i = 0; i < nt; ++i, ++g) {
+                const uint32_t sb = g & 1;
+                if (!wait_bar(bar(kBarSFull + sb), (g >> 1) & 1, abort_flag, lad::kErrMlaSoftmax)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t r[kTile];
+                LAD_TMEM_LD32(tmem + lane_addr + kColS + sb * kTile, r);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarSEmpty + sb));
+
+                const int tok0 = (tile0 + i) * kTile;
+                float x[kTile];
+                float tmax = -INFINITY;
+#pragma unroll
+                for (int t = 0; t < kTile; ++t) {
+                    x[t] = (tok0 + t < len) ? __uint_as_float(r[t]) * score_scale_log2 : -INFINITY;
+                    tmax = fmaxf(tmax, x[t]);
+                }
+                if (i == 0) {
+                    m = -INFINITY;
+                    l = 0.f;
+                }
+                float f = 1.f;
+                bool need = false;
+                if (m == -INFINITY) {
+                    m = tmax;
+                    f = 0.f;
+                } else if (tmax > m + 8.f) {
+                    f = exp2f(m - tmax);
+                    m = tmax;
+                    need = true;
+                }
+                uint32_t pk[kTile / 2];
+                float psum = 0.f;
+#pragma unroll
+                for (int t = 0; t < kTile; t += 2) {
+                    const float p0 = exp2f(x[t] - m), p1 = exp2f(x[t + 1] - m);
+                    psum += p0 + p1;  // the denominator keeps fp32 probabilities
+                    pk[t / 2] = lad::dev::f32x2_to_bf16x2(p0, p1);
+                }
+                l = l * f + psum;
+
+                const uint32_t pb = g & 1;
+                if (!wait_bar(bar(kBarPEmpty + pb), ((g >> 1) & 1) ^ 1, abort_flag, lad::kErrMlaSoftmax)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t rb = g & 1;
+                if (owner) {
+                    // P[h][t], K-major without swizzle: 8x8 core matrices of 128 bytes;
+                    // head group h/8 at 512 B, token group t/8 at 128 B, row h%8 at 16 B.
+                    uint8_t *prow = smem + kOffP + pb * kPBytes + (h >> 3) * 512 + (h & 7) * 16;
+#pragma unroll
+                    for (int j = 0; j < kTile / 8; ++j)
+                        *reinterpret_cast<uint4 *>(prow + j * 128) =
+                            make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                    rescale[rb * 64 + h] = f;
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                const int any = __any_sync(0xffffffffu, owner && need);
+                if (lane == 0) any_rescale[rb * 4 + p] = any;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarWg + rb));
+                if (!wait_bar(bar(kBarWg + rb), (g >> 1) & 1, abort_flag, lad::kErrMlaSoftmax)) {
+                    ok = false;
+                    break;
+                }
+                const bool do_rescale = (any_rescale[rb * 4 + 0] | any_rescale[rb * 4 + 1] |
+                                         any_rescale[rb * 4 + 2] | any_rescale[rb * 4 + 3]) != 0;
+                if (do_rescale) {
+                    // GEMM2 of the previous tile (same segment, since i > 0) must be complete
+                    const uint32_t gp = g - 1;
+                    if (!wait_bar(bar(kBarPEmpty + (gp & 1)), (gp >> 1) & 1, abort_flag, lad::kErrMlaSoftmax)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int j = 0; j < 4; ++j) {
+#pragma unroll 1
+                        for (int half = 0; half < 2; ++half) {
+                            uint32_t o[32];
+                            const uint32_t ta = tmem + lane_addr + kColO + 64 * j + 32 * half;
+                            LAD_TMEM_LD32(ta, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                o[c] = __float_as_uint(__uint_as_float(o[c]) * rescale[rb * 64 + 32 * half + c]);
+                            LAD_TMEM_ST32(ta, o);
+                        }
+                    }
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarPFull + pb));
+
+                if (i == nt - 1) {
+                    // ---- segment epilogue: O^T (unnormalised), m and l to the workspace ----
+                    if (!wait_bar(bar(kBarPEmpty + (g & 1)), (g >> 1) & 1, abort_flag, lad::kErrMlaEpilogue)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const long long slot = static_cast<long long>(blockIdx.x) + seq;
+                    float *Od = ws.O + slot * (kHq * kDl);
+#pragma unroll 1
+                    for (int j = 0; j < 4; ++j) {
+                        const int d = 128 * j + 32 * p + lane;
+#pragma unroll 1
+                        for (int half = 0; half < 2; ++half) {
+                            uint32_t o[32];
+                            LAD_TMEM_LD32(tmem + lane_addr + kColO + 64 * j + 32 * half, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) Od[(32 * half + c) * kDl + d] = __uint_as_float(o[c]);
+                        }
+                    }
+                    if (owner) {
+                        ws.m[slot * kHq + h] = m;
+                        ws.l[slot * kHq + h] = l;
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(kBarOFree));
+                }
+            }
+            ++k;
+        }
+        (void)ok;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
+
+// Merges the partials of each sequence by log-sum-exp, normalises and applies the gate.
+// Grid (B, 64 heads), 128 threads, 4 latent dims per thread.
+template <bool kOutF32>
+__global__ void __launch_bounds__(128)
+mla_combine_kernel(const int *__restrict__ seq_lens, int B, int G, const float *__restrict__ gate,
+                   Partials ws, void *__restrict__ out, float *__restrict__ lse_out) {
+    const int b = blockIdx.x, h = blockIdx.y;
+    const int d = 4 * threadIdx.x;
+    const long long total = ws.tile_prefix[B];
+    const long long lo = ws.tile_prefix[b], hi = ws.tile_prefix[b + 1];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float M = -INFINITY, Lsum = 0.f;
+    if (hi > lo) {
+        // first pass: the largest running max over the CTAs that touched this sequence
+        for (int c = 0; c < G; ++c) {
+            const long long c0 = split_point(total, G, c), c1 = split_point(total, G, c + 1);
+            if (c1 <= lo || c0 >= hi || c0 >= c1) continue;
+            M = fmaxf(M, ws.m[(static_cast<long long>(c) + b) * kHq + h]);
+        }
+        for (int c = 0; c < G; ++c) {
+            const long long c0 = split_point(total, G, c), c1 = split_point(total, G, c + 1);
+            if (c1 <= lo || c0 >= hi || c0 >= c1) continue;
+            const long long slot = static_cast<long long>(c) + b;
+            const float w = exp2f(ws.m[slot * kHq + h] - M);
+            Lsum += w * ws.l[slot * kHq + h];
+            const float4 v = *reinterpret_cast<const float4 *>(ws.O + (slot * kHq + h) * kDl + d);
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
+    }
+    float sc = (Lsum > 0.f) ? 1.f / Lsum : 0.f;
+    if (gate) sc *= 1.f / (1.f + expf(-gate[b * kHq + h]));
+    acc.x *= sc;
+    acc.y *= sc;
+    acc.z *= sc;
+    acc.w *= sc;
+    const long long o_off = (static_cast<long long>(b) * kHq + h) * kDl + d;
+    if constexpr (kOutF32) {
+        *reinterpret_cast<float4 *>(static_cast<float *>(out) + o_off) = acc;
+    } else {
+        uint2 pk;
+        pk.x = lad::dev::f32x2_to_bf16x2(acc.x, acc.y);
+        pk.y = lad::dev::f32x2_to_bf16x2(acc.z, acc.w);
+        *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(out) + o_off) = pk;
+    }
+    if (lse_out && threadIdx.x == 0)
+        lse_out[b * kHq + h] = (Lsum > 0.f) ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
+}
+
+// ------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+    size_t off_O, off_m, off_l, off_prefix, total;
+};
+
+WsLayout ws_layout(int B, int G) {
+    const size_t slots = static_cast<size_t>(G) + static_cast<size_t>(B);
+    WsLayout w{};
+    w.off_O = 0;
+    w.off_m = align_up(w.off_O + slots * kHq * kDl * sizeof(float), 256);
+    w.off_l = align_up(w.off_m + slots * kHq * sizeof(float), 256);
+    w.off_prefix = align_up(w.off_l + slots * kHq * sizeof(float), 256);
+    w.total = align_up(w.off_prefix + (static_cast<size_t>(B) + 1) * sizeof(long long), 256);
+    return w;
+}
+
+}  // namespace
+
 namespace lad {
-int take_device_error_mla(cudaStream_t, int *code) {
-    *code = 0;
+int take_device_error_mla(cudaStream_t s, int *code) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_mla_error, sizeof v, 0, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return set_error(LAD_ECUDA, "lad_device_error: %s", cudaGetErrorString(e));
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_mla_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return set_error(LAD_ECUDA, "lad_device_error: %s", cudaGetErrorString(e));
+    }
+    *code = v;
     return LAD_OK;
 }
 }  // namespace lad
 
-extern "C" size_t mla_latent_decode_workspace_size(int, int, int, int) { return 0; }
+extern "C" size_t mla_latent_decode_workspace_size(int B, int Hq, int d_latent, int num_sms) {
+    if (B < 0 || Hq != kHq || d_latent != kDl) return 0;
+    const int G = num_sms > 0 ? num_sms : lad::device_sm_count();
+    if (G <= 0) return 0;
+    return ws_layout(B, G).total;
+}
 
-extern "C" int mla_latent_decode(const lad_bf16 *, const lad_bf16 *, long long, const int *, const float *, void *,
-                                 float *, int, int, int, int, int, float, unsigned, void *, size_t, void *) {
-    return lad::set_error(LAD_EUNSUPPORTED, "mla_latent_decode: not built yet");
+extern "C" int mla_latent_decode(const lad_bf16 *q, const lad_bf16 *cache, long long cache_seq_stride,
+                                 const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B, int Hq,
+                                 int d_latent, int d_rope, int Lmax, float scale, unsigned flags, void *workspace,
+                                 size_t ws_bytes, void *stream) {
+    using lad::set_error;
+    if (B < 0 || Lmax < 0) return set_error(LAD_EINVAL, "mla_latent_decode: negative B or Lmax");
+    if (Hq != kHq || d_latent != kDl || d_rope != kDr)
+        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode: Hq = 64, d_latent = 512, d_rope = 64 only");
+    if (flags & ~LAD_FLAG_OUT_FP32) return set_error(LAD_EINVAL, "mla_latent_decode: unknown flags 0x%x", flags);
+    if (B == 0) return LAD_OK;
+    if (!q || !cache || !seq_lens || !o) return set_error(LAD_EINVAL, "mla_latent_decode: null pointer");
+    if (Lmax == 0) Lmax = 1;  // every length is then 0; the tensor map still needs a non-empty extent
+    if (cache_seq_stride < static_cast<long long>(Lmax) * kDrow || cache_seq_stride % 8 != 0)
+        return set_error(LAD_EINVAL, "mla_latent_decode: cache_seq_stride must be >= Lmax*576 and a multiple of 8");
+    if (!lad::aligned(q, 16) || !lad::aligned(cache, 16))
+        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode: q and cache must be 16-byte aligned");
+    const bool f32 = (flags & LAD_FLAG_OUT_FP32) != 0;
+    if (!lad::aligned(o, f32 ? 16 : 8)) return set_error(LAD_EUNSUPPORTED, "mla_latent_decode: o misaligned");
+    const int G = lad::device_sm_count();
+    if (G <= 0) return set_error(LAD_ECUDA, "mla_latent_decode: cannot query the SM count");
+    const WsLayout wl = ws_layout(B, G);
+    if (!workspace || ws_bytes < wl.total || !lad::aligned(workspace, 256))
+        return set_error(LAD_EWORKSPACE, "mla_latent_decode: workspace of %zu bytes (256-aligned) required",
+                         wl.total);
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return set_error(LAD_ECUDA, "mla_latent_decode: cuTensorMapEncodeTiled unavailable");
+
+    CUtensorMap map_cache, map_q;
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(Lmax),
+                                    static_cast<cuuint64_t>(B)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDrow) * 2,
+                                       static_cast<cuuint64_t>(cache_seq_stride) * 2};
+        const cuuint32_t box[3] = {kChunk, kTile, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        CUresult r = enc(&map_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<lad_bf16 *>(cache), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return set_error(LAD_ECUDA, "mla_latent_decode: cache tensor map failed (%d)", (int)r);
+    }
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(B) * kHq};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDrow) * 2};
+        const cuuint32_t box[2] = {kChunk, kHq};
+        const cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<lad_bf16 *>(q), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return set_error(LAD_ECUDA, "mla_latent_decode: q tensor map failed (%d)", (int)r);
+    }
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    Partials parts{reinterpret_cast<float *>(ws + wl.off_O), reinterpret_cast<float *>(ws + wl.off_m),
+                   reinterpret_cast<float *>(ws + wl.off_l), reinterpret_cast<long long *>(ws + wl.off_prefix)};
+
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(mla_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return set_error(LAD_ECUDA, "mla_latent_decode: smem attribute: %s", cudaGetErrorString(attr_err));
+
+    cudaStream_t s = lad::as_stream(stream);
+    const float score_scale_log2 = scale * 1.4426950408889634f;
+    mla_split_kernel<<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B, score_scale_log2, parts);
+    int rc = lad::check_launch("mla_latent_decode (split)");
+    if (rc != LAD_OK) return rc;
+    const dim3 cgrid(static_cast<unsigned>(B), kHq);
+    if (f32)
+        mla_combine_kernel<true><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
+    else
+        mla_combine_kernel<false><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
+    return lad::check_launch("mla_latent_decode (combine)");
 }
