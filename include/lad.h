@@ -163,7 +163,7 @@ size_t kda_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk
  *   o           [B][Hq][d_latent] bf16, or fp32 if flags & LAD_FLAG_OUT_FP32
  *   lse_out     fp32 [B][Hq] or NULL
  *   workspace   device scratch, ws_bytes >= mla_latent_decode_workspace_size(B, Hq, d_latent, 0)
- * Supported: Hq == 64, d_latent == 512, d_rope == 64; cache and q 16-byte aligned.
+ * Supported: Hq == 64, d_latent == 512, d_rope == 64; cache and q 16-byte aligned; scale > 0.
  */
 int mla_latent_decode(const lad_bf16 *q, const lad_bf16 *cache, long long cache_seq_stride, const int *seq_lens,
                       const float *gate_logits, void *o, float *lse_out, int B, int Hq, int d_latent, int d_rope,

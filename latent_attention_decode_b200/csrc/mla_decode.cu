@@ -67,10 +67,13 @@ constexpr int kOffP = kOffStage + kStages * kStageBytes;         // 221,184
 constexpr int kOffBar = kOffP + 2 * kPBytes;                     // 229,376
 constexpr int kSmemBytes = kOffBar + 1024 + 1024;                // + barriers/scalars + alignment slack
 
-// TMEM columns (fp32): O^T blocks 0..255, S buffers 256..287 and 288..319.
+// TMEM columns (fp32): O^T blocks 0..255; S buffer b at 256 + 64 b, holding two partial sums of
+// GEMM1 (even and odd K chunks) 32 columns apart, so consecutive MMAs never chain on one
+// accumulator.
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;
 constexpr uint32_t kColS = 256;
+constexpr uint32_t kSBufCols = 2 * kTile;
 
 // barrier slots (8 bytes each) inside the kOffBar region
 enum Bar : int {
@@ -124,8 +127,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase of `bar` with parity `parity`. Returns false if the CTA is
 // aborting (this wait ran out, or another role's did).
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag, int tag) {
-    if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag, int tag) {
     const uint64_t t0 = globaltimer_ns();
     while (true) {
 #pragma unroll 1
@@ -140,36 +142,68 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile in
     }
 }
 
+// Called by whole warps; the result is made warp-uniform so that every lane takes the same path
+// (the issue helpers rely on the warp staying converged).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag, int tag) {
+    const bool r = mbar_try_wait(bar, parity) || wait_bar_slow(bar, parity, abort_flag, tag);
+    return __all_sync(0xffffffffu, r);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// The issue helpers below are executed by a whole, converged warp; `elect.sync` picks one lane
+// (the same lowest lane every time) that actually issues. Keeping the warp converged lets the
+// descriptors and addresses live in uniform registers, which tcgen05.mma and TMA read directly.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z, uint32_t bar) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-        "[%5];" ::"r"(dst),
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];\n\t}" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
         : "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-            "r"(dst),
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];\n\t}" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_tx_elect(uint32_t bar, uint32_t bytes) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(bar),
+        "r"(bytes)
         : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// Warp-wide: the elected lane commits (the same lane that issued the MMAs).
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+        : "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (bf16 in, fp32 accumulate)
+// Warp-wide: D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (bf16 in, fp32 accumulate),
+// issued by the elected lane.
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -348,8 +382,8 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
     SegIter it{seq_lens, B, static_cast<int>(range[2]), range[3], t0, t1};
 
     if (warp == 0) {
-        // ================= TMA producer =================
-        if (lane == 0) {
+        // ================= TMA producer (whole warp, elected lane issues) =================
+        {
             int seq, tile0, nt, k = 0;
             uint32_t g = 0;
             bool ok = true;
@@ -358,7 +392,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     ok = false;
                     break;
                 }
-                mbar_arrive_tx(bar(kBarQFull), kQBytes);
+                mbar_arrive_tx_elect(bar(kBarQFull), kQBytes);
                 for (int c = 0; c < kNChunk; ++c)
                     tma_load_2d(sbase + kOffQ + c * kQChunkBytes, &map_q, c * kChunk, seq * kHq, bar(kBarQFull));
                 for (int i = 0; i < nt; ++i, ++g) {
@@ -367,7 +401,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                         ok = false;
                         break;
                     }
-                    mbar_arrive_tx(bar(kBarFull + s), kStageBytes);
+                    mbar_arrive_tx_elect(bar(kBarFull + s), kStageBytes);
                     const uint32_t dst = sbase + kOffStage + s * kStageBytes;
                     for (int c = 0; c < kNChunk; ++c)
                         tma_load_3d(dst + c * kTChunkBytes, &map_cache, c * kChunk, (tile0 + i) * kTile, seq,
@@ -393,11 +427,15 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             }
         }
     } else if (warp == 1) {
-        // ================= MMA issuer =================
-        if (lane == 0) {
+        // ================= MMA issuer (whole warp, elected lane issues) =================
+        {
             int seq, tile0, nt, k = 0;
             uint32_t g = 0;
             bool ok = true;
+            const uint64_t q_desc0 = smem_desc(sbase + kOffQ, 16, 1024, kLayoutSw128);
+            const uint64_t c_desc0 = smem_desc(sbase + kOffStage, 16, 1024, kLayoutSw128);
+            const uint64_t v_desc0 = smem_desc(sbase + kOffStage, kTChunkBytes, 1024, kLayoutSw128);
+            const uint64_t p_desc0 = smem_desc(sbase + kOffP, 128, 512, kLayoutNone);
             // the previous tile's GEMM2 is issued after the current tile's GEMM1
             bool have_prev = false;
             uint32_t prev_g = 0;
@@ -411,19 +449,17 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     return false;
                 tc_fence_after();
                 const uint32_t s = gg % kStages;
-                const uint32_t vbase = sbase + kOffStage + s * kStageBytes;
-                const uint32_t pbase = sbase + kOffP + pb * kPBytes;
+                // A = V^T: 128 latent dims (two 64-wide chunks, LBO apart) x 16 tokens (two 8-row groups)
+                const uint64_t a0 = v_desc0 + ((s * kStageBytes) >> 4);
+                // B = P: 64 heads (8-row core groups, SBO 512) x 16 tokens (two 8-token core columns, LBO 128)
+                const uint64_t b0 = p_desc0 + ((pb * kPBytes) >> 4);
+                const uint32_t acc0 = first_of_seg ? 0u : 1u;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int kk = 0; kk < kTile / 16; ++kk) {
 #pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        // A = V^T: 128 latent dims (two 64-wide chunks, LBO apart) x 16 tokens (two 8-row groups)
-                        const uint64_t a = smem_desc(vbase + (2 * j) * kTChunkBytes + kk * 2048, kTChunkBytes, 1024,
-                                                     kLayoutSw128);
-                        // B = P: 64 heads (8-row core groups, SBO 512) x 16 tokens (two 8-token core columns, LBO 128)
-                        const uint64_t bdesc = smem_desc(pbase + kk * 256, 128, 512, kLayoutNone);
-                        tc_mma(tmem + kColO + 64 * j, a, bdesc, kIdesc2, (first_of_seg && kk == 0) ? 0u : 1u);
-                    }
+                    for (int j = 0; j < 4; ++j)
+                        tc_mma(tmem + kColO + 64 * j, a0 + (((2 * j) * kTChunkBytes + kk * 2048) >> 4),
+                               b0 + ((kk * 256) >> 4), kIdesc2, kk == 0 ? acc0 : 1u);
                 }
                 tc_commit(bar(kBarEmpty + s));
                 tc_commit(bar(kBarPEmpty + pb));
@@ -443,17 +479,14 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t cbase = sbase + kOffStage + s * kStageBytes;
-#pragma unroll 1
+                    const uint64_t cd = c_desc0 + ((s * kStageBytes) >> 4);
+                    const uint32_t dS = tmem + kColS + sb * kSBufCols;
+#pragma unroll
                     for (int c = 0; c < kNChunk; ++c) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t a = smem_desc(sbase + kOffQ + c * kQChunkBytes + kk * 32, 16, 1024,
-                                                         kLayoutSw128);
-                            const uint64_t bdesc = smem_desc(cbase + c * kTChunkBytes + kk * 32, 16, 1024,
-                                                             kLayoutSw128);
-                            tc_mma(tmem + kColS + sb * kTile, a, bdesc, kIdesc1, (c | kk) ? 1u : 0u);
-                        }
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma(dS + (c & 1) * kTile, q_desc0 + ((c * kQChunkBytes + kk * 32) >> 4),
+                                   cd + ((c * kTChunkBytes + kk * 32) >> 4), kIdesc1, (c > 1 || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(bar(kBarSFull + sb));
                     if (i == nt - 1) tc_commit(bar(kBarQEmpty));
@@ -494,8 +527,9 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     break;
                 }
                 tc_fence_after();
-                uint32_t r[kTile];
-                LAD_TMEM_LD32(tmem + lane_addr + kColS + sb * kTile, r);
+                uint32_t r[kTile], r2[kTile];
+                LAD_TMEM_LD32(tmem + lane_addr + kColS + sb * kSBufCols, r);
+                LAD_TMEM_LD32(tmem + lane_addr + kColS + sb * kSBufCols + kTile, r2);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
@@ -503,12 +537,18 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
 
                 const int tok0 = (tile0 + i) * kTile;
                 float x[kTile];
-                float tmax = -INFINITY;
 #pragma unroll
-                for (int t = 0; t < kTile; ++t) {
-                    x[t] = (tok0 + t < len) ? __uint_as_float(r[t]) * score_scale_log2 : -INFINITY;
-                    tmax = fmaxf(tmax, x[t]);
+                for (int t = 0; t < kTile; ++t) x[t] = __uint_as_float(r[t]) + __uint_as_float(r2[t]);
+                if (tok0 + kTile > len) {
+#pragma unroll
+                    for (int t = 0; t < kTile; ++t)
+                        if (tok0 + t >= len) x[t] = -INFINITY;
                 }
+                // scores stay unscaled; the scale (with log2 e) is folded into the exponent below
+                float tmax = x[0];
+#pragma unroll
+                for (int t = 1; t < kTile; ++t) tmax = fmaxf(tmax, x[t]);
+                tmax *= score_scale_log2;
                 if (i == 0) {
                     m = -INFINITY;
                     l = 0.f;
@@ -519,7 +559,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     m = tmax;
                     f = 0.f;
                 } else if (tmax > m + 8.f) {
-                    f = exp2f(m - tmax);
+                    f = ex2(m - tmax);
                     m = tmax;
                     need = true;
                 }
@@ -527,7 +567,8 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                 float psum = 0.f;
 #pragma unroll
                 for (int t = 0; t < kTile; t += 2) {
-                    const float p0 = exp2f(x[t] - m), p1 = exp2f(x[t + 1] - m);
+                    const float p0 = ex2(fmaf(x[t], score_scale_log2, -m));
+                    const float p1 = ex2(fmaf(x[t + 1], score_scale_log2, -m));
                     psum += p0 + p1;  // the denominator keeps fp32 probabilities
                     pk[t / 2] = lad::dev::f32x2_to_bf16x2(p0, p1);
                 }
@@ -752,6 +793,7 @@ extern "C" int mla_latent_decode(const lad_bf16 *q, const lad_bf16 *cache, long 
     if (Hq != kHq || d_latent != kDl || d_rope != kDr)
         return set_error(LAD_EUNSUPPORTED, "mla_latent_decode: Hq = 64, d_latent = 512, d_rope = 64 only");
     if (flags & ~LAD_FLAG_OUT_FP32) return set_error(LAD_EINVAL, "mla_latent_decode: unknown flags 0x%x", flags);
+    if (!(scale > 0.f) || scale == INFINITY) return set_error(LAD_EINVAL, "mla_latent_decode: scale must be positive");
     if (B == 0) return LAD_OK;
     if (!q || !cache || !seq_lens || !o) return set_error(LAD_EINVAL, "mla_latent_decode: null pointer");
     if (Lmax == 0) Lmax = 1;  // every length is then 0; the tensor map still needs a non-empty extent
