@@ -172,6 +172,29 @@ int mla_latent_decode(const lad_bf16 *q, const lad_bf16 *cache, long long cache_
 /* Workspace bytes mla_latent_decode needs; num_sms == 0 queries the current device. */
 size_t mla_latent_decode_workspace_size(int B, int Hq, int d_latent, int num_sms);
 
+/*
+ * mla_latent_decode_noalloc — mla_latent_decode for callers that cannot allocate device memory
+ * (a plugin inside a runtime that owns every device allocation, or a decode loop where
+ * cudaMalloc's implicit synchronisation is not allowed). The pages have no counterpart: this is
+ * a property of the library, not of the method. Results equal mla_latent_decode's.
+ *
+ * The caller still passes all inputs and outputs (same meaning, layouts and limits as
+ * mla_latent_decode); only the scratch space differs: it is a fixed array compiled into the
+ * library (about 25 MB, allocated on every device that loads the library and held until the
+ * process exits), so this call itself allocates nothing.
+ *   - B must not exceed mla_latent_decode_noalloc_max_batch() (32); larger B returns
+ *     LAD_EUNSUPPORTED with a message. The device must have at most 160 SMs.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current); make that first call before any stream capture.
+ *   - All calls share the one array: calls whose kernels may overlap on the GPU (different
+ *     streams, or different host threads) race and give undefined results. Serialise them.
+ *   - The array keeps the last call's contents; nothing in it needs to start at zero.
+ */
+int mla_latent_decode_noalloc(const lad_bf16 *q, const lad_bf16 *cache, long long cache_seq_stride,
+                              const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B, int Hq,
+                              int d_latent, int d_rope, int Lmax, float scale, unsigned flags, void *stream);
+size_t mla_latent_decode_noalloc_max_batch(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,8 @@ import torch
 
 __all__ = [
     "kda_conv_update", "kda_decode_step", "kda_prefill_chunked", "kda_prefill_workspace_size",
-    "mla_latent_decode", "mla_latent_decode_workspace_size", "lad_device_error", "lad_version",
+    "mla_latent_decode", "mla_latent_decode_workspace_size", "mla_latent_decode_noalloc",
+    "lad_device_error", "lad_version",
     "LadError", "LIB_PATH", "FLAG_SILU", "FLAG_L2NORM_QK", "FLAG_OUT_FP32", "MLA_SCALE",
 ]
 
@@ -63,6 +64,9 @@ def _load() -> ctypes.CDLL:
         "mla_latent_decode": ([_c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int,
                                _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
         "mla_latent_decode_workspace_size": ([_c_int] * 4, _c_sz),
+        "mla_latent_decode_noalloc": ([_c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
+                                       _c_int, _c_int, _c_f, _c_u, _c_vp], _c_int),
+        "mla_latent_decode_noalloc_max_batch": ([], _c_sz),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -250,4 +254,38 @@ def mla_latent_decode(q: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tens
         q.data_ptr(), cache.data_ptr(), seq_stride, seq_lens.data_ptr(), _ptr(gate_logits), o.data_ptr(),
         _ptr(lse), B, Hq, d_latent, D - d_latent, Lmax, float(scale), flags, _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o
+
+
+def mla_latent_decode_noalloc(q: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tensor,
+                              gate_logits: torch.Tensor | None = None, o: torch.Tensor | None = None,
+                              lse: torch.Tensor | None = None, scale: float = MLA_SCALE, d_latent: int = 512,
+                              out_fp32: bool = False, stream=None) -> torch.Tensor:
+    """mla_latent_decode without a workspace, for callers that cannot allocate device memory.
+
+    The library's built-in scratch array limits B to mla_latent_decode_noalloc_max_batch();
+    calls that may overlap on the GPU share that array and must be serialised. If ``o`` is
+    None it is allocated here by torch; pass ``o`` to keep the whole call allocation-free.
+    """
+    bf = torch.bfloat16
+    _contig(q, "q", bf)
+    _cuda(cache, "cache", bf)
+    B, Hq, D = q.shape
+    if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != D or cache.stride(2) != 1 \
+            or cache.stride(1) != D:
+        raise ValueError("cache must be [B,Lmax,D] with contiguous rows")
+    _contig(seq_lens, "seq_lens", torch.int32)
+    if gate_logits is not None:
+        _contig(gate_logits, "gate_logits", torch.float32)
+    odt = torch.float32 if out_fp32 else bf
+    if o is None:
+        o = torch.empty((B, Hq, d_latent), device=q.device, dtype=odt)
+    _contig(o, "o", odt)
+    if lse is not None:
+        _contig(lse, "lse", torch.float32)
+    seq_stride = cache.stride(0) if B > 1 else cache.shape[1] * D
+    _check("mla_latent_decode_noalloc", _lib.mla_latent_decode_noalloc(
+        q.data_ptr(), cache.data_ptr(), seq_stride, seq_lens.data_ptr(), _ptr(gate_logits), o.data_ptr(),
+        _ptr(lse), B, Hq, d_latent, D - d_latent, cache.shape[1], float(scale), FLAG_OUT_FP32 if out_fp32 else 0,
+        _stream(stream)))
     return o

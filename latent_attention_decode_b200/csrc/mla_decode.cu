@@ -859,3 +859,139 @@ extern "C" int mla_latent_decode(const lad_bf16 *q, const lad_bf16 *cache, long 
         mla_combine_kernel<false><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
     return lad::check_launch("mla_latent_decode (combine)");
 }
+
+// ------------------------------------------------------------------------------------------
+// mla_latent_decode_noalloc: the same computation with the scratch space in a file-scope device
+// array instead of a caller-provided workspace, for callers that cannot allocate device memory
+// at all (for example a plugin inside a runtime that owns every device allocation, or a decode
+// loop where cudaMalloc's implicit device synchronisation is not allowed).
+// ------------------------------------------------------------------------------------------
+namespace {
+
+constexpr int kNoAllocMaxB = 32;    // sequences per call
+constexpr int kNoAllocMaxSms = 160; // CTAs of the split kernel (one per SM)
+// Partials for (SMs + B) slots plus the tile prefix: 192 x 64 x 514 x 4 B + (33 x 8 B) ~ 25.3 MB,
+// held by every device that loads the library until the process exits.
+constexpr size_t kNoAllocScratchBytes =
+    (static_cast<size_t>(kNoAllocMaxSms + kNoAllocMaxB) * kHq * (kDl + 2) * sizeof(float) + 4 * 256 +
+     (kNoAllocMaxB + 1) * sizeof(long long) + 255) / 256 * 256;
+
+static __device__ __align__(256) uint8_t g_mla_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch array, looked up once per device with that device current. The
+// host-side symbol is only a stand-in and must never be handed to a kernel.
+int noalloc_scratch_ptr(uint8_t **out) {
+    static std::mutex mu;
+    static uint8_t *ptrs[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return lad::set_error(LAD_ECUDA, "mla_latent_decode_noalloc: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= 64) return lad::set_error(LAD_EUNSUPPORTED, "mla_latent_decode_noalloc: device %d", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_mla_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return lad::set_error(LAD_ECUDA, "mla_latent_decode_noalloc: cudaGetSymbolAddress: %s",
+                                  cudaGetErrorString(e));
+        ptrs[dev] = static_cast<uint8_t *>(p);
+    }
+    *out = ptrs[dev];
+    return LAD_OK;
+}
+
+}  // namespace
+
+extern "C" size_t mla_latent_decode_noalloc_max_batch(void) { return kNoAllocMaxB; }
+
+extern "C" int mla_latent_decode_noalloc(const lad_bf16 *q, const lad_bf16 *cache, long long cache_seq_stride,
+                                         const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B,
+                                         int Hq, int d_latent, int d_rope, int Lmax, float scale, unsigned flags,
+                                         void *stream) {
+    using lad::set_error;
+    if (B < 0 || Lmax < 0) return set_error(LAD_EINVAL, "mla_latent_decode_noalloc: negative B or Lmax");
+    if (Hq != kHq || d_latent != kDl || d_rope != kDr)
+        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode_noalloc: Hq = 64, d_latent = 512, d_rope = 64 only");
+    if (flags & ~LAD_FLAG_OUT_FP32)
+        return set_error(LAD_EINVAL, "mla_latent_decode_noalloc: unknown flags 0x%x", flags);
+    if (!(scale > 0.f) || scale == INFINITY)
+        return set_error(LAD_EINVAL, "mla_latent_decode_noalloc: scale must be positive");
+    if (B > kNoAllocMaxB)
+        return set_error(LAD_EUNSUPPORTED,
+                         "mla_latent_decode_noalloc: B = %d exceeds the built-in scratch limit of %d sequences "
+                         "(use mla_latent_decode with a workspace)",
+                         B, kNoAllocMaxB);
+    if (B == 0) return LAD_OK;
+    if (!q || !cache || !seq_lens || !o) return set_error(LAD_EINVAL, "mla_latent_decode_noalloc: null pointer");
+    if (Lmax == 0) Lmax = 1;
+    if (cache_seq_stride < static_cast<long long>(Lmax) * kDrow || cache_seq_stride % 8 != 0)
+        return set_error(LAD_EINVAL,
+                         "mla_latent_decode_noalloc: cache_seq_stride must be >= Lmax*576 and a multiple of 8");
+    if (!lad::aligned(q, 16) || !lad::aligned(cache, 16))
+        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode_noalloc: q and cache must be 16-byte aligned");
+    const bool f32 = (flags & LAD_FLAG_OUT_FP32) != 0;
+    if (!lad::aligned(o, f32 ? 16 : 8)) return set_error(LAD_EUNSUPPORTED, "mla_latent_decode_noalloc: o misaligned");
+    const int G = lad::device_sm_count();
+    if (G <= 0) return set_error(LAD_ECUDA, "mla_latent_decode_noalloc: cannot query the SM count");
+    if (G > kNoAllocMaxSms)
+        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode_noalloc: %d SMs exceed the built-in limit of %d", G,
+                         kNoAllocMaxSms);
+    const WsLayout wl = ws_layout(B, G);
+    if (wl.total > kNoAllocScratchBytes)
+        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode_noalloc: scratch of %zu bytes exceeds %zu", wl.total,
+                         kNoAllocScratchBytes);
+    uint8_t *ws = nullptr;
+    int rc = noalloc_scratch_ptr(&ws);
+    if (rc != LAD_OK) return rc;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return set_error(LAD_ECUDA, "mla_latent_decode_noalloc: cuTensorMapEncodeTiled unavailable");
+
+    CUtensorMap map_cache, map_q;
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(Lmax),
+                                    static_cast<cuuint64_t>(B)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDrow) * 2,
+                                       static_cast<cuuint64_t>(cache_seq_stride) * 2};
+        const cuuint32_t box[3] = {kChunk, kTile, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        CUresult r = enc(&map_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<lad_bf16 *>(cache), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS)
+            return set_error(LAD_ECUDA, "mla_latent_decode_noalloc: cache tensor map failed (%d)", (int)r);
+    }
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(B) * kHq};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDrow) * 2};
+        const cuuint32_t box[2] = {kChunk, kHq};
+        const cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<lad_bf16 *>(q), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS)
+            return set_error(LAD_ECUDA, "mla_latent_decode_noalloc: q tensor map failed (%d)", (int)r);
+    }
+    // Every slot the combine reads is written earlier in the same call (partials by their CTA's
+    // epilogue, the tile prefix by CTA 0), so nothing left over from a previous call is read and
+    // nothing needs clearing.
+    Partials parts{reinterpret_cast<float *>(ws + wl.off_O), reinterpret_cast<float *>(ws + wl.off_m),
+                   reinterpret_cast<float *>(ws + wl.off_l), reinterpret_cast<long long *>(ws + wl.off_prefix)};
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(mla_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return set_error(LAD_ECUDA, "mla_latent_decode_noalloc: smem attribute: %s", cudaGetErrorString(attr_err));
+    cudaStream_t s = lad::as_stream(stream);
+    mla_split_kernel<<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B, scale * 1.4426950408889634f,
+                                                     parts);
+    rc = lad::check_launch("mla_latent_decode_noalloc (split)");
+    if (rc != LAD_OK) return rc;
+    const dim3 cgrid(static_cast<unsigned>(B), kHq);
+    if (f32)
+        mla_combine_kernel<true><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
+    else
+        mla_combine_kernel<false><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
+    return lad::check_launch("mla_latent_decode_noalloc (combine)");
+}
