@@ -1,17 +1,642 @@
-// KDA chunked prefill (placeholder entry points; the kernel follows).
-#include "lad_common.cuh"
+// KDA chunked prefill on B200: the gated delta rule over T tokens in chunks of 64, in the WY / UT
+// form, with every contraction on the tensor cores (tcgen05, kind::tf32) and the fp32 state
+// carried in tensor memory from chunk to chunk.
+//
+// Source: "Ling-3.1-flash: a 560B hybrid-attention MoE, counted from its safetensors headers",
+// section "How KDA and MLA split the work" (gated delta rule, per-channel decay alpha, per-head
+// strength beta, 128x128 state per head). The chunked form is not on the page; it is the
+// token-by-token recurrence (S' = Diag(alpha) S; u = beta (v - S'^T k); S = S' + k u^T;
+// o = scale S^T q) unrolled over a chunk. Inside a chunk (rows r = tokens, g_r = prod_{s<=r}
+// alpha_s per key channel, S0 the state entering the chunk):
+//   Kt = K*g, Kh = K/g, Qt = Q*g                                  (elementwise)
+//   A  = strict_lower(diag(beta) Kt Kh^T),  T = (I + A)^-1,  Tb = T diag(beta)
+//   W  = Tb Kt,  U = Tb V - W S0
+//   O  = scale (Qt S0 + lower(Qt Kh^T) U)
+//   S  = Diag(g_last) (S0 + Kh^T U)        (= Diag(g_last) S0 + (K * g_last/g)^T U)
+// d_v columns of S are independent, so a CTA owns one (sequence, head, half of d_v) and walks
+// its chunks in order: 128 CTAs for one sequence of 64 heads.
+//
+// Per chunk (one warpgroup; warp 0 issues the MMAs, converged, elect.sync):
+//   1. load q, k, alpha, v, beta; running products g; write the operand tiles
+//   2. MMA  [Qt; Kt] Kh^T  (M = 128: rows 0-63 give Qt Kh^T, rows 64-127 give Kt Kh^T)
+//   3. lower(Qt Kh^T) -> operand; A -> fp32 scratch; T = (I + A)^-1 by 16x16 blocked forward
+//      substitution on the CUDA cores; Tb -> operand
+//   4. MMA  W^T = Kt^T Tb^T,  U' = Tb V;   W -> operand
+//   5. MMA  X = W S0;  U = U' - X -> operand
+//   6. MMA  O = Qt S0 + lower(Qt Kh^T) U;  S += Kh^T U
+//   7. O -> HBM; S <- Diag(g_last) S in TMEM, and -> next chunk's S0 operand (HBM after the last)
+// Every operand tile is K-major fp32 with the 128-byte swizzle (tf32 operands read MN-major
+// would need a different swizzle; storing the transposes instead keeps one layout): the tiles
+// that a contraction needs "the other way round" (Kt^T, Kh^T, V^T / U^T, S0^T) are written
+// transposed by the threads that own the data. Values are rounded to tf32 to nearest (cvt.rna)
+// when written, so the tensor core's tf32 read loses nothing further. tf32 operands keep every
+// output within a few 1e-4 relative of fp64; bf16 operands for the derived matrices would cost
+// ~1.6e-3, too close to the 2e-3 output budget. The state master stays fp32 in TMEM.
+// Padded rows of a short last chunk get q = k = v = 0, alpha = 1, beta = 0, which makes them
+// contribute nothing; their outputs are not stored.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "sm100_ptx.cuh"
+
+namespace {
+
+using namespace lad::ptx;
+using lad::dev::bf16_to_f32;
+
+constexpr int kC = 64;         // chunk length
+constexpr int kDk = 128;       // key width
+constexpr int kDv = 128;       // value width
+constexpr int kDvh = 64;       // value columns per CTA
+constexpr int kThreads = 128;
+
+// Shared memory (bytes). An operand tile is a set of blocks, one per 32 fp32 columns, each block
+// holding the tile's rows as 128-byte swizzled rows; "stride" is the distance between blocks.
+constexpr uint32_t kOffXQK = 0;        // [Qt; Kt]: 128 rows (tokens) x 128 (d_k), stride 16 KiB
+constexpr uint32_t kOffTT = 8192;      //   Tb [64 r][64 s] in the Kt half of XQK blocks 0-1 (stride 16 KiB)
+constexpr uint32_t kOffQM = 40960;     //   lower(Qt Kh^T) [64][64] in the Kt half of blocks 2-3
+constexpr uint32_t kOffKH = 65536;     // Kh [64 tokens][128 d_k], stride 8 KiB; then A/T scratch; then W
+constexpr uint32_t kOffKTT = 98304;    // Kt^T [128 d_k][64 tokens], stride 16 KiB
+constexpr uint32_t kOffKHT = 131072;   // Kh^T [128 d_k][64 tokens], stride 16 KiB
+constexpr uint32_t kOffVT = 163840;    // V^T, then U^T: [64 d_v][64 tokens], stride 8 KiB
+constexpr uint32_t kOffSOT = 180224;   // S0^T [64 d_v][128 d_k], stride 8 KiB
+constexpr uint32_t kOffMisc = 212992;
+constexpr uint32_t kStr16 = 16384, kStr8 = 8192;
+constexpr uint32_t kMiscBeta = 0, kMiscRq = 256, kMiscRk = 512, kMiscGc = 768, kMiscBar = 1280, kMiscTmem = 1288,
+                   kMiscAbort = 1292, kMiscTmaBar = 1296;
+// Raw inputs of the next chunk, TMA-staged over tiles that are dead once a chunk's last MMA has
+// completed (Kt^T, Kh^T and U^T): alpha [64][128] fp32, q and k [64][128] bf16, v [64][64] bf16.
+constexpr uint32_t kOffStA = kOffKTT;            // 32 KiB
+constexpr uint32_t kOffStQ = kOffStA + 32768;    // 16 KiB
+constexpr uint32_t kOffStK = kOffStQ + 16384;    // 16 KiB
+constexpr uint32_t kOffStV = kOffStK + 16384;    // 8 KiB, ends inside the V^T tile
+constexpr uint32_t kStageTx = 32768 + 16384 + 16384 + 8192;
+constexpr uint32_t kSmemBytes = kOffMisc + 2048 + 1024;  // + alignment slack
+
+// TMEM columns (fp32)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColAcc1 = 0;    // M=128 x 64: [Qt Kh^T ; Kt Kh^T]
+constexpr uint32_t kColWT = 64;     // M=128 x 64: W^T (rows d_k, columns r)
+constexpr uint32_t kColU = 128;     // M=64 x 64: U' = Tb V
+constexpr uint32_t kColX = 192;     // M=64 x 64: W S0
+constexpr uint32_t kColO = 256;     // M=64 x 64
+constexpr uint32_t kColS = 320;     // M=128 x 64: state master (rows d_k)
+
+constexpr uint32_t kIdesc128 = make_idesc(128, 64, kFmtTf32, 0, 0);
+constexpr uint32_t kIdesc64 = make_idesc(64, 64, kFmtTf32, 0, 0);
+
+__device__ int g_prefill_error = 0;
+
+struct Args {
+    const uint16_t *q, *k, *v;
+    const float *alpha, *beta;
+    float *S;
+    void *o;
+    int B, T, H;
+    float scale;
+    int l2norm, out_f32;
+};
+
+__device__ __forceinline__ void st_tile4(uint8_t *tile, int row, int col, uint32_t stride, float a, float b, float c,
+                                         float d) {
+    *reinterpret_cast<float4 *>(tile + sw128_off32(row, col, stride)) =
+        make_float4(round_tf32(a), round_tf32(b), round_tf32(c), round_tf32(d));
+}
+
+__device__ __forceinline__ void st_tile1(uint8_t *tile, int row, int col, uint32_t stride, float a) {
+    *reinterpret_cast<float *>(tile + sw128_off32(row, col, stride)) = round_tf32(a);
+}
+
+// K-major SW128 descriptor of a tile at smem byte `addr` for k-step j (8 tf32 of K per step).
+__device__ __forceinline__ uint64_t kdesc(uint64_t base_desc, uint32_t stride, int j) {
+    return base_desc + ((static_cast<uint32_t>(j >> 2) * stride + static_cast<uint32_t>(j & 3) * 32u) >> 4);
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct Maps {
+    CUtensorMap q, k, alpha, v;  // 3-D views [B][T][H*128], boxes of 64 tokens
+};
+
+__global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const __grid_constant__ Maps maps) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    float *s_beta = reinterpret_cast<float *>(sm + kOffMisc + kMiscBeta);
+    float *s_rq = reinterpret_cast<float *>(sm + kOffMisc + kMiscRq);
+    float *s_rk = reinterpret_cast<float *>(sm + kOffMisc + kMiscRk);
+    float *s_gc = reinterpret_cast<float *>(sm + kOffMisc + kMiscGc);
+    const uint32_t bar = sbase + kOffMisc + kMiscBar;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc + kMiscTmem);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + kMiscAbort);
+    const uint32_t tma_bar = sbase + kOffMisc + kMiscTmaBar;
+    float *Apl = reinterpret_cast<float *>(sm + kOffKH);  // [64][64] fp32, plain row-major
+    float *Tpl = reinterpret_cast<float *>(sm + kOffKH + 64 * 64 * 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int half = blockIdx.x & 1;
+    const int bh = blockIdx.x >> 1;
+    const int b = bh / p.H, h = bh - b * p.H;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;  // this warp's TMEM sub-partition
+    const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);         // K-major SW128 at smem offset 0
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init(tma_bar, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    uint32_t phase = 0;
+    bool ok = true;
+
+    auto mma_sync = [&](auto &&issue) {
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) {
+            tc_fence_after();
+            issue();
+            tc_commit(bar);
+        }
+        const bool w = wait_bar(bar, phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
+        phase ^= 1;
+        tc_fence_after();
+        return __syncthreads_and(w) != 0;
+    };
+
+    // ---- initial state: thread = key channel i; TMEM master row i, S0^T column i ----
+    {
+        const float *S0 = p.S + (static_cast<size_t>(bh) * kDk + tid) * kDv + half * kDvh;
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 x = *reinterpret_cast<const float4 *>(S0 + 32 * c2 + j);
+                v[j] = x.x;
+                v[j + 1] = x.y;
+                v[j + 2] = x.z;
+                v[j + 3] = x.w;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) st_tile1(sm + kOffSOT, 32 * c2 + j, tid, kStr8, v[j]);
+            tmem_st32(tmem + lane_base + kColS + 32 * c2, v);
+        }
+        tmem_wait_st();
+    }
+
+    // the next chunk's raw inputs, staged by TMA (thread 0); rows past T read as zeros
+    auto stage = [&](int chunk) {
+        fence_async_smem();
+        mbar_arrive_tx_raw(tma_bar, kStageTx);
+        const int t = chunk * kC;
+        tma_load_3d(sbase + kOffStA, &maps.alpha, h * kDk, t, b, tma_bar);
+        tma_load_3d(sbase + kOffStQ, &maps.q, h * kDk, t, b, tma_bar);
+        tma_load_3d(sbase + kOffStK, &maps.k, h * kDk, t, b, tma_bar);
+        tma_load_3d(sbase + kOffStV, &maps.v, h * kDv + half * kDvh, t, b, tma_bar);
+    };
+    uint32_t tma_phase = 0;
+    int pending = 0;  // a staging copy is in flight
+    const int nchunks = (p.T + kC - 1) / kC;
+    if (tid == 0) stage(0);
+    pending = 1;
+    for (int ch = 0; ch < nchunks && ok; ++ch) {
+        const int t0 = ch * kC;
+        const int n = min(kC, p.T - t0);
+        const size_t tok0 = (static_cast<size_t>(b) * p.T + t0) * p.H + h;  // token row of (b, t0, h)
+        const size_t tstride = static_cast<size_t>(p.H);                      // rows between tokens
+
+        // ---- 1a. beta, the staged raw inputs, per-token inverse norms (L2 flag) ----
+        if (tid < kC) s_beta[tid] = (tid < n) ? p.beta[tok0 + tid * tstride] : 0.f;
+        {
+            const bool w = wait_bar(tma_bar, tma_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            tma_phase ^= 1;
+            pending = 0;
+            ok = __syncthreads_and(w) != 0;
+            if (!ok) break;
+        }
+        if (p.l2norm) {
+            const uint16_t *sq = reinterpret_cast<const uint16_t *>(sm + kOffStQ);
+            const uint16_t *sk = reinterpret_cast<const uint16_t *>(sm + kOffStK);
+#pragma unroll 1
+            for (int r = warp; r < kC; r += 4) {
+                const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + 4 * lane);
+                const uint2 kw = *reinterpret_cast<const uint2 *>(sk + r * kDk + 4 * lane);
+                const float2 q0 = lad::dev::bf16x2_to_f32(qw.x), q1 = lad::dev::bf16x2_to_f32(qw.y);
+                const float2 k0 = lad::dev::bf16x2_to_f32(kw.x), k1 = lad::dev::bf16x2_to_f32(kw.y);
+                float sqs = q0.x * q0.x + q0.y * q0.y + q1.x * q1.x + q1.y * q1.y;
+                float sks = k0.x * k0.x + k0.y * k0.y + k1.x * k1.x + k1.y * k1.y;
+#pragma unroll
+                for (int o = 16; o; o >>= 1) {
+                    sqs += __shfl_xor_sync(0xffffffffu, sqs, o);
+                    sks += __shfl_xor_sync(0xffffffffu, sks, o);
+                }
+                if (lane == 0) {
+                    s_rq[r] = rsqrtf(sqs + 1e-6f);
+                    s_rk[r] = rsqrtf(sks + 1e-6f);
+                }
+            }
+        } else if (tid < kC) {
+            s_rq[tid] = 1.f;
+            s_rk[tid] = 1.f;
+        }
+        __syncthreads();
+
+        // ---- 1b. running decay per key channel (thread = channel i) and the operand tiles ----
+        {
+            const int i = tid;
+            const float *sa = reinterpret_cast<const float *>(sm + kOffStA);
+            const uint16_t *sq = reinterpret_cast<const uint16_t *>(sm + kOffStQ);
+            const uint16_t *sk = reinterpret_cast<const uint16_t *>(sm + kOffStK);
+            const uint16_t *sv = reinterpret_cast<const uint16_t *>(sm + kOffStV);
+            float g = 1.f;
+#pragma unroll 8
+            for (int r = 0; r < kC; ++r) {
+                // staged rows past the sequence end are zeros; alpha = 1 there keeps g unchanged
+                const float a = (r < n) ? sa[r * kDk + i] : 1.f;
+                const float qv = bf16_to_f32(sq[r * kDk + i]) * s_rq[r];
+                const float kv = bf16_to_f32(sk[r * kDk + i]) * s_rk[r];
+                g *= a;
+                st_tile1(sm + kOffXQK, r, i, kStr16, qv * g);
+                st_tile1(sm + kOffXQK, kC + r, i, kStr16, kv * g);
+                st_tile1(sm + kOffKH, r, i, kStr8, kv / g);
+            }
+            s_gc[i] = g;
+            // V^T: thread -> value column j = tid % 64, tokens 32 * (tid / 64) .. + 31
+            const int j = tid & 63, r0 = 32 * (tid >> 6);
+            float vv[32];
+#pragma unroll
+            for (int r = 0; r < 32; ++r) vv[r] = bf16_to_f32(sv[(r0 + r) * kDvh + j]);
+            __syncthreads();  // the staging area is read; Kt^T, Kh^T and V^T overwrite it
+#pragma unroll
+            for (int r = 0; r < 32; r += 4) st_tile4(sm + kOffVT, j, r0 + r, kStr8, vv[r], vv[r + 1], vv[r + 2], vv[r + 3]);
+            // Kt^T and Kh^T: row i, from the [token][d_k] tiles just written (already tf32)
+#pragma unroll 4
+            for (int r = 0; r < kC; r += 4) {
+                float kt[4], kh[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    kt[u] = *reinterpret_cast<const float *>(sm + kOffXQK + sw128_off32(kC + r + u, i, kStr16));
+                    kh[u] = *reinterpret_cast<const float *>(sm + kOffKH + sw128_off32(r + u, i, kStr8));
+                }
+                st_tile4(sm + kOffKTT, i, r, kStr16, kt[0], kt[1], kt[2], kt[3]);
+                st_tile4(sm + kOffKHT, i, r, kStr16, kh[0], kh[1], kh[2], kh[3]);
+            }
+        }
+
+        // ---- 2. [Qt; Kt] Kh^T ----
+        ok = mma_sync([&] {
+#pragma unroll
+            for (int j = 0; j < kDk / 8; ++j)
+                tc_mma_tf32(tmem + kColAcc1, kdesc(d0 + (kOffXQK >> 4), kStr16, j), kdesc(d0 + (kOffKH >> 4), kStr8, j),
+                            kIdesc128, j > 0);
+        });
+        if (!ok) break;
+
+        // ---- 3a. lower(Qt Kh^T) -> QM (warps 0,1); A -> fp32 scratch (warps 2,3) ----
+        {
+            float x0[32], x1[32];
+            tmem_ld32(tmem + lane_base + kColAcc1, x0);
+            tmem_ld32(tmem + lane_base + kColAcc1 + 32, x1);
+            tmem_wait_ld();
+            const int m = tid;  // accumulator row
+            if (m < kC) {
+                const int r = m;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    st_tile4(sm + kOffQM, r, j, kStr16, j + 0 <= r ? x0[j] : 0.f, j + 1 <= r ? x0[j + 1] : 0.f,
+                             j + 2 <= r ? x0[j + 2] : 0.f, j + 3 <= r ? x0[j + 3] : 0.f);
+                    st_tile4(sm + kOffQM, r, 32 + j, kStr16, 32 + j <= r ? x1[j] : 0.f, 33 + j <= r ? x1[j + 1] : 0.f,
+                             34 + j <= r ? x1[j + 2] : 0.f, 35 + j <= r ? x1[j + 3] : 0.f);
+                }
+            } else {
+                const int r = m - kC;
+                const float br = s_beta[r];
+                float4 *dst = reinterpret_cast<float4 *>(Apl + r * 64);
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    dst[j / 4] = make_float4(j < r ? br * x0[j] : 0.f, j + 1 < r ? br * x0[j + 1] : 0.f,
+                                             j + 2 < r ? br * x0[j + 2] : 0.f, j + 3 < r ? br * x0[j + 3] : 0.f);
+                    dst[8 + j / 4] = make_float4(32 + j < r ? br * x1[j] : 0.f, 33 + j < r ? br * x1[j + 1] : 0.f,
+                                                 34 + j < r ? br * x1[j + 2] : 0.f, 35 + j < r ? br * x1[j + 3] : 0.f);
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- 3b. T = (I + A)^-1, A strictly lower: diagonal 16x16 blocks first ----
+        if (tid < kC) {
+            const int base = 16 * (tid >> 4), c = tid & 15;
+            float t[16];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                float acc = (rr == c) ? 1.f : 0.f;
+#pragma unroll
+                for (int ss = 0; ss < rr; ++ss) acc -= Apl[(base + rr) * 64 + base + ss] * t[ss];
+                t[rr] = acc;
+            }
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) Tpl[(base + rr) * 64 + base + c] = t[rr];
+        } else {
+            // zero the blocks above the diagonal: (bi, bj) with bi < bj
+            for (int e = tid - kC; e < 6 * 256; e += kThreads - kC) {
+                const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+                const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                Tpl[(16 * bi + rr) * 64 + 16 * bj + cc] = 0.f;
+            }
+        }
+        __syncthreads();
+        // block rows 1..3: T_ij = -T_ii * sum_{k=j}^{i-1} A_ik T_kj
+#pragma unroll 1
+        for (int bi = 1; bi < 4; ++bi) {
+            const int nel = bi * 256;
+            float rv[6];
+#pragma unroll
+            for (int u = 0; u < 6; ++u) {
+                const int e = tid + kThreads * u;
+                rv[u] = 0.f;
+                if (e < nel) {
+                    const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+                    float acc = 0.f;
+                    for (int kb = bj; kb < bi; ++kb)
+#pragma unroll
+                        for (int ss = 0; ss < 16; ++ss)
+                            acc += Apl[(16 * bi + rr) * 64 + 16 * kb + ss] * Tpl[(16 * kb + ss) * 64 + 16 * bj + cc];
+                    rv[u] = acc;
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int u = 0; u < 6; ++u) {
+                const int e = tid + kThreads * u;
+                if (e < nel) {
+                    const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+                    Tpl[(16 * bi + rr) * 64 + 16 * bj + cc] = rv[u];  // holds R_j for the next step
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int u = 0; u < 6; ++u) {
+                const int e = tid + kThreads * u;
+                rv[u] = 0.f;
+                if (e < nel) {
+                    const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int ss = 0; ss < 16; ++ss)
+                        acc -= Tpl[(16 * bi + rr) * 64 + 16 * bi + ss] * Tpl[(16 * bi + ss) * 64 + 16 * bj + cc];
+                    rv[u] = acc;
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int u = 0; u < 6; ++u) {
+                const int e = tid + kThreads * u;
+                if (e < nel) {
+                    const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+                    Tpl[(16 * bi + rr) * 64 + 16 * bj + cc] = rv[u];
+                }
+            }
+            __syncthreads();
+        }
+        // Tb = T diag(beta) -> operand tile (thread -> row tid/2, 32 columns)
+        {
+            const int r = tid >> 1, jc = (tid & 1) * 32;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(Tpl + r * 64 + jc + j);
+                st_tile4(sm + kOffTT, r, jc + j, kStr16, t4.x * s_beta[jc + j], t4.y * s_beta[jc + j + 1],
+                         t4.z * s_beta[jc + j + 2], t4.w * s_beta[jc + j + 3]);
+            }
+        }
+
+        // ---- 4. W^T = Kt^T Tb^T (M = 128 d_k),  U' = Tb V (B = V^T) ----
+        ok = mma_sync([&] {
+#pragma unroll
+            for (int j = 0; j < kC / 8; ++j) {
+                const uint64_t tt = kdesc(d0 + (kOffTT >> 4), kStr16, j);
+                tc_mma_tf32(tmem + kColWT, kdesc(d0 + (kOffKTT >> 4), kStr16, j), tt, kIdesc128, j > 0);
+                tc_mma_tf32(tmem + kColU, tt, kdesc(d0 + (kOffVT >> 4), kStr8, j), kIdesc64, j > 0);
+            }
+        });
+        if (!ok) break;
+        // W [r][d_k] -> operand in the Kh slot: thread = d_k row of W^T, writes column i of W
+        {
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                float w[32];
+                tmem_ld32(tmem + lane_base + kColWT + 32 * c2, w);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) st_tile1(sm + kOffKH, 32 * c2 + j, tid, kStr8, w[j]);
+            }
+        }
+
+        // ---- 5. X = W S0 (B = S0^T);  U = U' - X -> U^T operand ----
+        ok = mma_sync([&] {
+#pragma unroll
+            for (int j = 0; j < kDk / 8; ++j)
+                tc_mma_tf32(tmem + kColX, kdesc(d0 + (kOffKH >> 4), kStr8, j), kdesc(d0 + (kOffSOT >> 4), kStr8, j),
+                            kIdesc64, j > 0);
+        });
+        if (!ok) break;
+        {
+            const int r = 16 * warp + lane;  // M = 64 accumulator row (lanes 0-15 of each sub-partition)
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                float u[32], x[32];
+                tmem_ld32(tmem + lane_base + kColU + 32 * c2, u);
+                tmem_ld32(tmem + lane_base + kColX + 32 * c2, x);
+                tmem_wait_ld();
+                if (lane < 16) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) st_tile1(sm + kOffVT, 32 * c2 + j, r, kStr8, u[j] - x[j]);
+                }
+            }
+        }
+
+        // ---- 6. O = Qt S0 + lower(Qt Kh^T) U;  S += Kh^T U ----
+        ok = mma_sync([&] {
+#pragma unroll
+            for (int j = 0; j < kDk / 8; ++j)
+                tc_mma_tf32(tmem + kColO, kdesc(d0 + (kOffXQK >> 4), kStr16, j), kdesc(d0 + (kOffSOT >> 4), kStr8, j),
+                            kIdesc64, j > 0);
+#pragma unroll
+            for (int j = 0; j < kC / 8; ++j) {
+                const uint64_t ut = kdesc(d0 + (kOffVT >> 4), kStr8, j);
+                tc_mma_tf32(tmem + kColO, kdesc(d0 + (kOffQM >> 4), kStr16, j), ut, kIdesc64, 1);
+                tc_mma_tf32(tmem + kColS, kdesc(d0 + (kOffKHT >> 4), kStr16, j), ut, kIdesc128, 1);
+            }
+        });
+        if (!ok) break;
+
+        // ---- 7. O -> HBM; S <- Diag(g_last) S (TMEM), S^T -> operand (HBM after the last chunk) ----
+        if (ch + 1 < nchunks) {  // Kt^T, Kh^T, U^T are dead now
+            if (tid == 0) stage(ch + 1);
+            pending = 1;
+        }
+        {
+            const int r = 16 * warp + lane;
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                float ov[32];
+                tmem_ld32(tmem + lane_base + kColO + 32 * c2, ov);
+                tmem_wait_ld();
+                if (lane < 16 && r < n) {
+                    const size_t orow = (tok0 + r * tstride) * kDv + half * kDvh + 32 * c2;
+                    if (p.out_f32) {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow);
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            dst[j / 4] = make_float4(p.scale * ov[j], p.scale * ov[j + 1], p.scale * ov[j + 2],
+                                                     p.scale * ov[j + 3]);
+                    } else {
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) + orow);
+#pragma unroll
+                        for (int j = 0; j < 32; j += 8)
+                            dst[j / 8] = make_uint4(lad::dev::f32x2_to_bf16x2(p.scale * ov[j], p.scale * ov[j + 1]),
+                                                    lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 2], p.scale * ov[j + 3]),
+                                                    lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 4], p.scale * ov[j + 5]),
+                                                    lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 6], p.scale * ov[j + 7]));
+                    }
+                }
+            }
+            const bool last = (ch == nchunks - 1);
+            const float gc = s_gc[tid];
+            float *Sout = p.S + (static_cast<size_t>(bh) * kDk + tid) * kDv + half * kDvh;
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                float sv[32];
+                tmem_ld32(tmem + lane_base + kColS + 32 * c2, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    sv[j] *= gc;
+                    st_tile1(sm + kOffSOT, 32 * c2 + j, tid, kStr8, sv[j]);
+                }
+                tmem_st32(tmem + lane_base + kColS + 32 * c2, sv);
+                if (last) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4 *>(Sout + 32 * c2 + j) = make_float4(sv[j], sv[j + 1], sv[j + 2],
+                                                                                      sv[j + 3]);
+                }
+            }
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    // drain: a staging copy still in flight (after an abort) lands, and every MMA this CTA
+    // issued completes, before shared memory and TMEM are released
+    if (tid == 0 && pending) {
+        const uint64_t t0 = lad::dev::globaltimer_ns();
+        while (!mbar_try_wait(tma_bar, tma_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+        }
+    }
+    if (warp == 0) {
+        tc_commit(bar);
+        const uint64_t t0 = lad::dev::globaltimer_ns();
+        while (!mbar_try_wait(bar, phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
 
 namespace lad {
-int take_device_error_prefill(cudaStream_t, int *code) {
-    *code = 0;
+int take_device_error_prefill(cudaStream_t s, int *code) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_prefill_error, sizeof v, 0, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return set_error(LAD_ECUDA, "lad_device_error: %s", cudaGetErrorString(e));
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_prefill_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return set_error(LAD_ECUDA, "lad_device_error: %s", cudaGetErrorString(e));
+    }
+    *code = v;
     return LAD_OK;
 }
 }  // namespace lad
 
 extern "C" size_t kda_prefill_workspace_size(int, int, int, int, int, int) { return 0; }
 
-extern "C" int kda_prefill_chunked(const lad_bf16 *, const lad_bf16 *, const lad_bf16 *, const float *, const float *,
-                                   float *, void *, int, int, int, int, int, int, float, unsigned, void *, size_t,
-                                   void *) {
-    return lad::set_error(LAD_EUNSUPPORTED, "kda_prefill_chunked: not built yet");
+extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, const float *alpha,
+                                   const float *beta, float *S, void *o, int B, int T, int H, int dk, int dv,
+                                   int chunk, float scale, unsigned flags, void *workspace, size_t ws_bytes,
+                                   void *stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    using lad::set_error;
+    if (B < 0 || T < 0 || H < 0) return set_error(LAD_EINVAL, "kda_prefill_chunked: negative size");
+    if (dk != kDk || dv != kDv) return set_error(LAD_EUNSUPPORTED, "kda_prefill_chunked: dk = dv = 128 only");
+    if (chunk != kC) return set_error(LAD_EUNSUPPORTED, "kda_prefill_chunked: chunk = 64 only");
+    if (flags & ~(LAD_FLAG_OUT_FP32 | LAD_FLAG_L2NORM_QK))
+        return set_error(LAD_EINVAL, "kda_prefill_chunked: unknown flags 0x%x", flags);
+    if (B == 0 || H == 0) return LAD_OK;
+    if (!S) return set_error(LAD_EINVAL, "kda_prefill_chunked: null S");
+    if (T == 0) return LAD_OK;  // the state passes through unchanged
+    if (!q || !k || !v || !alpha || !beta || !o) return set_error(LAD_EINVAL, "kda_prefill_chunked: null pointer");
+    const bool f32 = (flags & LAD_FLAG_OUT_FP32) != 0;
+    if (!lad::aligned(S, 16) || !lad::aligned(v, 16) || !lad::aligned(o, 16) || !lad::aligned(q, 16) ||
+        !lad::aligned(k, 16) || !lad::aligned(alpha, 16))
+        return set_error(LAD_EUNSUPPORTED, "kda_prefill_chunked: q, k, v, alpha, S and o must be 16-byte aligned");
+    const long long ctas = 2LL * B * H;
+    if (ctas > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "kda_prefill_chunked: B*H too large");
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(kda_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return set_error(LAD_ECUDA, "kda_prefill_chunked: smem attribute: %s", cudaGetErrorString(attr_err));
+    Args a{reinterpret_cast<const uint16_t *>(q), reinterpret_cast<const uint16_t *>(k),
+           reinterpret_cast<const uint16_t *>(v), alpha, beta, S, o, B, T, H, scale,
+           (flags & LAD_FLAG_L2NORM_QK) ? 1 : 0, f32 ? 1 : 0};
+    auto enc = reinterpret_cast<EncodeTiledFn>(lad::tensor_map_encoder_raw());
+    if (!enc) return set_error(LAD_ECUDA, "kda_prefill_chunked: cuTensorMapEncodeTiled unavailable");
+    Maps maps;
+    auto make = [&](CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int box0) -> int {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(H) * kDk, static_cast<cuuint64_t>(T),
+                                    static_cast<cuuint64_t>(B)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * kDk * esize,
+                                       static_cast<cuuint64_t>(T) * H * kDk * esize};
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(box0), static_cast<cuuint32_t>(kC), 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        CUresult r = enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        return r == CUDA_SUCCESS ? LAD_OK : set_error(LAD_ECUDA, "kda_prefill_chunked: tensor map failed (%d)", (int)r);
+    };
+    int rc = make(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk);
+    if (rc == LAD_OK) rc = make(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk);
+    if (rc == LAD_OK) rc = make(&maps.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDk);
+    if (rc == LAD_OK) rc = make(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDvh);
+    if (rc != LAD_OK) return rc;
+    kda_prefill_kernel<<<static_cast<unsigned>(ctas), kThreads, kSmemBytes, lad::as_stream(stream)>>>(a, maps);
+    return lad::check_launch("kda_prefill_chunked");
 }

@@ -39,6 +39,19 @@ int device_sm_count() {
     return cache[dev];
 }
 
+void *tensor_map_encoder_raw() {
+    static std::once_flag once;
+    static void *fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = p;
+    });
+    return fn;
+}
+
 }  // namespace lad
 
 extern "C" const char *lad_last_error(void) { return lad::g_last_error; }

@@ -24,6 +24,10 @@ inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s
 // Streaming-multiprocessor count of the current device (cached per device).
 int device_sm_count();
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no libcuda link).
+// Returned untyped; the caller casts it to the driver signature from <cuda.h>.
+void *tensor_map_encoder_raw();
+
 // Tags stored in the device error word when a bounded wait gives up.
 enum DeviceErrorTag : int {
     kErrNone = 0,

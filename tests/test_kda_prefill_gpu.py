@@ -1,0 +1,109 @@
+"""Parity of kda_prefill_chunked (CUDA, tcgen05 tf32, through the C ABI) with the fp64 oracle's
+token-by-token recurrence.
+
+Outputs are held to the 2e-3 relative-L2 output budget (they come out near 3e-4: tf32 operands).
+The final state is held to 2e-3 as well: its chunk updates are tf32 contractions, so the 1e-4
+figure of the fp32 decode path does not apply (see the kernel header).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from tests.parity import TOL_OUT, bf16_round, f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+TOL_PREFILL_STATE = 2e-3
+
+
+@pytest.fixture(scope="module")
+def lad(cuda_device):
+    import latent_attention_decode_b200 as m
+    return m
+
+
+def _oracle(inp, scale=1.0, l2=False, heads=None):
+    q, k = f64(inp["q"]), f64(inp["k"])
+    v, a, b, S0 = f64(inp["v"]), f64(inp["alpha"]), f64(inp["beta"]), f64(inp["S0"])
+    if heads is not None:
+        q, k, v, a, b, S0 = q[:, :, heads], k[:, :, heads], v[:, :, heads], a[:, :, heads], b[:, :, heads], S0[:, heads]
+    if l2:
+        q, k = oracle.l2norm(q), oracle.l2norm(k)
+    return oracle.kda_recurrent(q, k, v, a, b, S0, scale=scale, nthreads=oracle.max_threads())
+
+
+def _run(lad, inp, dev, scale=1.0, l2=False, out_fp32=True):
+    t = {n: inp[n].to(dev) for n in ("q", "k", "v", "alpha", "beta")}
+    S = inp["S0"].to(dev).clone()
+    o = lad.kda_prefill_chunked(t["q"], t["k"], t["v"], t["alpha"], t["beta"], S, scale=scale, l2norm_qk=l2,
+                                out_fp32=out_fp32)
+    assert lad.lad_device_error() == 0
+    return o, S
+
+
+@pytest.mark.parametrize("B,H,T", [(1, 2, 64), (2, 3, 200), (1, 1, 1), (1, 2, 63), (1, 2, 65), (1, 4, 256)])
+def test_prefill_shapes(lad, cuda_device, B, H, T):
+    """One chunk, several chunks with a ragged tail, a single token, one short of / one past a chunk."""
+    cfg = wl.KdaScan("p", B=B, H=H, T=T, seed=100 + T, state_std=0.02, alpha_mode="uniform")
+    inp = wl.kda_scan_inputs(cfg)
+    o_ref, S_ref = _oracle(inp, scale=0.7)
+    o, S = _run(lad, inp, cuda_device, scale=0.7)
+    assert rel_l2(o, o_ref) < TOL_OUT
+    assert rel_l2(S, S_ref) < TOL_PREFILL_STATE
+
+
+def test_prefill_clamped_decays_zero_state(lad, cuda_device):
+    """The workload recipe: alpha mostly on the 0.9 clamp, zero initial state, bf16 output too."""
+    cfg = wl.KdaScan("p", B=1, H=2, T=300, seed=7)
+    inp = wl.kda_scan_inputs(cfg)
+    o_ref, S_ref = _oracle(inp)
+    o, S = _run(lad, inp, cuda_device)
+    assert rel_l2(o, o_ref) < TOL_OUT and rel_l2(S, S_ref) < TOL_PREFILL_STATE
+    o16, _ = _run(lad, inp, cuda_device, out_fp32=False)
+    assert rel_l2(o16, bf16_round(o_ref)) < TOL_OUT
+
+
+def test_prefill_l2norm_flag(lad, cuda_device):
+    cfg = wl.KdaScan("p", B=1, H=2, T=130, seed=9, state_std=0.02, alpha_mode="uniform")
+    inp = wl.kda_scan_inputs(cfg)
+    inp["q"] = wl.normal_bf16(inp["q"].shape, 9, "qraw", std=2.0)
+    inp["k"] = wl.normal_bf16(inp["k"].shape, 9, "kraw", std=0.3)
+    o_ref, S_ref = _oracle(inp, l2=True)
+    o, S = _run(lad, inp, cuda_device, l2=True)
+    assert rel_l2(o, o_ref) < TOL_OUT and rel_l2(S, S_ref) < TOL_PREFILL_STATE
+
+
+def test_prefill_matches_decode_steps(lad, cuda_device):
+    """Chunked prefill and the one-token decode kernel walk the same recurrence."""
+    cfg = wl.KdaScan("p", B=1, H=3, T=96, seed=11, state_std=0.02, alpha_mode="uniform")
+    inp = wl.kda_scan_inputs(cfg)
+    o_p, S_p = _run(lad, inp, cuda_device)
+    t = {n: inp[n].to(cuda_device) for n in ("q", "k", "v", "alpha", "beta")}
+    S = inp["S0"].to(cuda_device).clone()
+    outs = [lad.kda_decode_step(t["q"][:, i].contiguous(), t["k"][:, i].contiguous(), t["v"][:, i].contiguous(),
+                                t["alpha"][:, i].contiguous(), t["beta"][:, i].contiguous(), S, out_fp32=True)
+            for i in range(cfg.T)]
+    torch.cuda.synchronize()
+    assert rel_l2(o_p, torch.stack(outs, 1)) < TOL_OUT
+    assert rel_l2(S_p, S) < TOL_PREFILL_STATE
+
+
+def test_prefill_empty_sequence_keeps_state(lad, cuda_device):
+    cfg = wl.KdaScan("p", B=1, H=2, T=0, seed=12, state_std=0.02)
+    inp = wl.kda_scan_inputs(cfg)
+    _, S = _run(lad, inp, cuda_device)
+    assert torch.equal(S.cpu(), inp["S0"])
+
+
+@pytest.mark.slow
+def test_prefill_32k_full_size_sampled(lad, cuda_device):
+    """The 32,768-token, 64-head workload at full size; two heads checked over every token."""
+    cfg = wl.CONFIGS["kda_prefill_32k"]
+    inp = wl.kda_scan_inputs(cfg, cuda_device)
+    o, S = _run(lad, inp, cuda_device, out_fp32=True)
+    heads = [5, 60]
+    cpu = {n: inp[n].cpu() for n in inp}
+    o_ref, S_ref = _oracle(cpu, heads=heads)
+    assert rel_l2(o[:, :, heads], o_ref) < TOL_OUT
+    assert rel_l2(S[:, heads], S_ref) < TOL_PREFILL_STATE
