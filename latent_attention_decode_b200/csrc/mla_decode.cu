@@ -54,6 +54,7 @@ constexpr int kNChunk = kDrow / kChunk;  // 9
 constexpr int kTile = 32;          // cached rows per tile
 constexpr int kStages = 4;
 constexpr int kThreads = 256;
+constexpr int kMaxSplitCtas = 1024;  // one split CTA per SM; the combine tracks at most this many
 
 constexpr int kQChunkBytes = kHq * 128;                 // 8 KiB: 64 heads x 64 dims
 constexpr int kQBytes = kNChunk * kQChunkBytes;         // 73,728
@@ -678,29 +679,45 @@ mla_combine_kernel(const int *__restrict__ seq_lens, int B, int G, const float *
                    Partials ws, void *__restrict__ out, float *__restrict__ lse_out) {
     const int b = blockIdx.x, h = blockIdx.y;
     const int d = 4 * threadIdx.x;
+    __shared__ int s_c[2];
+    __shared__ unsigned char s_valid[kMaxSplitCtas];  // CTA c0 + i has a non-empty tile range
     const long long total = ws.tile_prefix[B];
     const long long lo = ws.tile_prefix[b], hi = ws.tile_prefix[b + 1];
+    if (threadIdx.x == 0) {
+        // CTAs whose tile range [split(c), split(c+1)) meets [lo, hi): start from the estimate
+        // lo*G/total and correct it (split points are floor(total*c/G)).
+        int c0 = 0, c1 = -1;
+        if (hi > lo) {
+            c0 = static_cast<int>(lo * G / total);
+            while (c0 > 0 && split_point(total, G, c0) > lo) --c0;
+            while (split_point(total, G, c0 + 1) <= lo) ++c0;
+            c1 = static_cast<int>((hi - 1) * G / total);
+            while (c1 > 0 && split_point(total, G, c1) > hi - 1) --c1;
+            while (split_point(total, G, c1 + 1) <= hi - 1) ++c1;
+        }
+        s_c[0] = c0;
+        s_c[1] = c1;
+    }
+    __syncthreads();
+    const int c0 = s_c[0], c1 = s_c[1];
+    // with fewer tiles than CTAs some CTAs own no tiles and wrote no partial
+    for (int c = c0 + static_cast<int>(threadIdx.x); c <= c1; c += blockDim.x)
+        s_valid[c - c0] = split_point(total, G, c) < split_point(total, G, c + 1);
+    __syncthreads();
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float M = -INFINITY, Lsum = 0.f;
-    if (hi > lo) {
-        // first pass: the largest running max over the CTAs that touched this sequence
-        for (int c = 0; c < G; ++c) {
-            const long long c0 = split_point(total, G, c), c1 = split_point(total, G, c + 1);
-            if (c1 <= lo || c0 >= hi || c0 >= c1) continue;
-            M = fmaxf(M, ws.m[(static_cast<long long>(c) + b) * kHq + h]);
-        }
-        for (int c = 0; c < G; ++c) {
-            const long long c0 = split_point(total, G, c), c1 = split_point(total, G, c + 1);
-            if (c1 <= lo || c0 >= hi || c0 >= c1) continue;
-            const long long slot = static_cast<long long>(c) + b;
-            const float w = exp2f(ws.m[slot * kHq + h] - M);
-            Lsum += w * ws.l[slot * kHq + h];
-            const float4 v = *reinterpret_cast<const float4 *>(ws.O + (slot * kHq + h) * kDl + d);
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
-        }
+    for (int c = c0; c <= c1; ++c)
+        if (s_valid[c - c0]) M = fmaxf(M, ws.m[(static_cast<long long>(c) + b) * kHq + h]);
+    for (int c = c0; c <= c1; ++c) {
+        if (!s_valid[c - c0]) continue;
+        const long long slot = static_cast<long long>(c) + b;
+        const float w = exp2f(ws.m[slot * kHq + h] - M);
+        Lsum += w * ws.l[slot * kHq + h];
+        const float4 v = *reinterpret_cast<const float4 *>(ws.O + (slot * kHq + h) * kDl + d);
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
     }
     float sc = (Lsum > 0.f) ? 1.f / Lsum : 0.f;
     if (gate) sc *= 1.f / (1.f + expf(-gate[b * kHq + h]));
@@ -805,6 +822,7 @@ extern "C" int mla_latent_decode(const lad_bf16 *q, const lad_bf16 *cache, long 
     if (!lad::aligned(o, f32 ? 16 : 8)) return set_error(LAD_EUNSUPPORTED, "mla_latent_decode: o misaligned");
     const int G = lad::device_sm_count();
     if (G <= 0) return set_error(LAD_ECUDA, "mla_latent_decode: cannot query the SM count");
+    if (G > kMaxSplitCtas) return set_error(LAD_EUNSUPPORTED, "mla_latent_decode: more than %d SMs", kMaxSplitCtas);
     const WsLayout wl = ws_layout(B, G);
     if (!workspace || ws_bytes < wl.total || !lad::aligned(workspace, 256))
         return set_error(LAD_EWORKSPACE, "mla_latent_decode: workspace of %zu bytes (256-aligned) required",
