@@ -16,7 +16,7 @@
 // d_v columns of S are independent, so a CTA owns one (sequence, head, half of d_v) and walks
 // its chunks in order: 128 CTAs for one sequence of 64 heads.
 //
-// Per chunk (one warpgroup; warp 0 issues the MMAs, converged, elect.sync):
+// Per chunk (two warpgroups; warp 0 issues the MMAs, converged, elect.sync):
 //   1. load q, k, alpha, v, beta; running products g; write the operand tiles
 //   2. MMA  [Qt; Kt] Kh^T  (M = 128: rows 0-63 give Qt Kh^T, rows 64-127 give Kt Kh^T)
 //   3. lower(Qt Kh^T) -> operand; A -> fp32 scratch; T = (I + A)^-1 by 16x16 blocked forward
@@ -49,7 +49,7 @@ constexpr int kC = 64;         // chunk length
 constexpr int kDk = 128;       // key width
 constexpr int kDv = 128;       // value width
 constexpr int kDvh = 64;       // value columns per CTA
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 
 // Shared memory (bytes). An operand tile is a set of blocks, one per 32 fp32 columns, each block
 // holding the tile's rows as 128-byte swizzled rows; "stride" is the distance between blocks.
@@ -64,7 +64,7 @@ constexpr uint32_t kOffSOT = 180224;   // S0^T [64 d_v][128 d_k], stride 8 KiB
 constexpr uint32_t kOffMisc = 212992;
 constexpr uint32_t kStr16 = 16384, kStr8 = 8192;
 constexpr uint32_t kMiscBeta = 0, kMiscRq = 256, kMiscRk = 512, kMiscGc = 768, kMiscBar = 1280, kMiscTmem = 1288,
-                   kMiscAbort = 1292, kMiscTmaBar = 1296;
+                   kMiscAbort = 1292, kMiscTmaBar = 1296, kMiscOct = 2048;  // s_oct: [8 octets][128] fp32
 // Raw inputs of the next chunk, TMA-staged over tiles that are dead once a chunk's last MMA has
 // completed (Kt^T, Kh^T and U^T): alpha [64][128] fp32, q and k [64][128] bf16, v [64][64] bf16.
 constexpr uint32_t kOffStA = kOffKTT;            // 32 KiB
@@ -72,7 +72,7 @@ constexpr uint32_t kOffStQ = kOffStA + 32768;    // 16 KiB
 constexpr uint32_t kOffStK = kOffStQ + 16384;    // 16 KiB
 constexpr uint32_t kOffStV = kOffStK + 16384;    // 8 KiB, ends inside the V^T tile
 constexpr uint32_t kStageTx = 32768 + 16384 + 16384 + 8192;
-constexpr uint32_t kSmemBytes = kOffMisc + 2048 + 1024;  // + alignment slack
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscOct + 8 * 128 * 4 + 1024;  // + alignment slack
 
 // TMEM columns (fp32)
 constexpr uint32_t kTmemCols = 512;
@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
     float *s_rq = reinterpret_cast<float *>(sm + kOffMisc + kMiscRq);
     float *s_rk = reinterpret_cast<float *>(sm + kOffMisc + kMiscRk);
     float *s_gc = reinterpret_cast<float *>(sm + kOffMisc + kMiscGc);
+    float *s_oct = reinterpret_cast<float *>(sm + kOffMisc + kMiscOct);
     const uint32_t bar = sbase + kOffMisc + kMiscBar;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc + kMiscTmem);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + kMiscAbort);
@@ -145,11 +146,16 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
     float *Tpl = reinterpret_cast<float *>(sm + kOffKH + 64 * 64 * 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // TMEM: warp w reads sub-partition w % 4; warps w and w + 4 split a 64-column accumulator
+    // into column halves.
+    const int sp = warp & 3, cg = warp >> 2;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * sp) << 16;
+    const int row128 = 32 * sp + lane;  // row of an M = 128 accumulator held by this thread
+    const int row64 = 16 * sp + lane;   // row of an M = 64 accumulator (lanes 0-15 hold rows)
     const int half = blockIdx.x & 1;
     const int bh = blockIdx.x >> 1;
     const int b = bh / p.H, h = bh - b * p.H;
-    const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;  // this warp's TMEM sub-partition
-    const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);         // K-major SW128 at smem offset 0
+    const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);  // K-major SW128 at smem offset 0
 
     if (tid == 0) {
         mbar_init(bar, 1);
@@ -180,24 +186,21 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
         return __syncthreads_and(w) != 0;
     };
 
-    // ---- initial state: thread = key channel i; TMEM master row i, S0^T column i ----
+    // ---- initial state: TMEM master row = key channel, S0^T column; 32 value columns per thread ----
     {
-        const float *S0 = p.S + (static_cast<size_t>(bh) * kDk + tid) * kDv + half * kDvh;
+        const float *S0 = p.S + (static_cast<size_t>(bh) * kDk + row128) * kDv + half * kDvh + 32 * cg;
+        float v[32];
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-            float v[32];
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                const float4 x = *reinterpret_cast<const float4 *>(S0 + 32 * c2 + j);
-                v[j] = x.x;
-                v[j + 1] = x.y;
-                v[j + 2] = x.z;
-                v[j + 3] = x.w;
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) st_tile1(sm + kOffSOT, 32 * c2 + j, tid, kStr8, v[j]);
-            tmem_st32(tmem + lane_base + kColS + 32 * c2, v);
+        for (int j = 0; j < 32; j += 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(S0 + j);
+            v[j] = x.x;
+            v[j + 1] = x.y;
+            v[j + 2] = x.z;
+            v[j + 3] = x.w;
         }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) st_tile1(sm + kOffSOT, 32 * cg + j, row128, kStr8, v[j]);
+        tmem_st32(tmem + lane_base + kColS + 32 * cg, v);
         tmem_wait_st();
     }
 
@@ -235,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
             const uint16_t *sq = reinterpret_cast<const uint16_t *>(sm + kOffStQ);
             const uint16_t *sk = reinterpret_cast<const uint16_t *>(sm + kOffStK);
 #pragma unroll 1
-            for (int r = warp; r < kC; r += 4) {
+            for (int r = warp; r < kC; r += kThreads / 32) {
                 const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + 4 * lane);
                 const uint2 kw = *reinterpret_cast<const uint2 *>(sk + r * kDk + 4 * lane);
                 const float2 q0 = lad::dev::bf16x2_to_f32(qw.x), q1 = lad::dev::bf16x2_to_f32(qw.y);
@@ -258,37 +261,69 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
         }
         __syncthreads();
 
-        // ---- 1b. running decay per key channel (thread = channel i) and the operand tiles ----
+        // ---- 1b. running decay and the operand tiles. Warp w takes tokens 8w .. 8w+7 and lane l
+        //          the key channels 4l .. 4l+3 (one 512-byte row segment per warp access); the
+        //          product over earlier token octets comes through shared memory ----
         {
-            const int i = tid;
+            const int o = warp, c4 = 4 * lane;
             const float *sa = reinterpret_cast<const float *>(sm + kOffStA);
             const uint16_t *sq = reinterpret_cast<const uint16_t *>(sm + kOffStQ);
             const uint16_t *sk = reinterpret_cast<const uint16_t *>(sm + kOffStK);
-            const uint16_t *sv = reinterpret_cast<const uint16_t *>(sm + kOffStV);
-            float g = 1.f;
-#pragma unroll 8
-            for (int r = 0; r < kC; ++r) {
-                // staged rows past the sequence end are zeros; alpha = 1 there keeps g unchanged
-                const float a = (r < n) ? sa[r * kDk + i] : 1.f;
-                const float qv = bf16_to_f32(sq[r * kDk + i]) * s_rq[r];
-                const float kv = bf16_to_f32(sk[r * kDk + i]) * s_rk[r];
-                g *= a;
-                st_tile1(sm + kOffXQK, r, i, kStr16, qv * g);
-                st_tile1(sm + kOffXQK, kC + r, i, kStr16, kv * g);
-                st_tile1(sm + kOffKH, r, i, kStr8, kv / g);
-            }
-            s_gc[i] = g;
-            // V^T: thread -> value column j = tid % 64, tokens 32 * (tid / 64) .. + 31
-            const int j = tid & 63, r0 = 32 * (tid >> 6);
-            float vv[32];
+            float4 gl[8];  // running product within the octet
+            float4 run = make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
-            for (int r = 0; r < 32; ++r) vv[r] = bf16_to_f32(sv[(r0 + r) * kDvh + j]);
+            for (int u = 0; u < 8; ++u) {
+                const int r = 8 * o + u;
+                const float4 a = (r < n) ? *reinterpret_cast<const float4 *>(sa + r * kDk + c4)
+                                         : make_float4(1.f, 1.f, 1.f, 1.f);
+                run.x *= a.x;
+                run.y *= a.y;
+                run.z *= a.z;
+                run.w *= a.w;
+                gl[u] = run;
+            }
+            *reinterpret_cast<float4 *>(s_oct + o * kDk + c4) = run;
+            __syncthreads();
+            float4 excl = make_float4(1.f, 1.f, 1.f, 1.f);  // product over the octets before o
+            for (int oo = 0; oo < o; ++oo) {
+                const float4 y = *reinterpret_cast<const float4 *>(s_oct + oo * kDk + c4);
+                excl.x *= y.x;
+                excl.y *= y.y;
+                excl.z *= y.z;
+                excl.w *= y.w;
+            }
+            if (o == kThreads / 32 - 1)
+                *reinterpret_cast<float4 *>(s_gc + c4) =
+                    make_float4(excl.x * run.x, excl.y * run.y, excl.z * run.z, excl.w * run.w);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int r = 8 * o + u;
+                const float gg[4] = {excl.x * gl[u].x, excl.y * gl[u].y, excl.z * gl[u].z, excl.w * gl[u].w};
+                const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + c4);
+                const uint2 kw = *reinterpret_cast<const uint2 *>(sk + r * kDk + c4);
+                const float2 q0 = lad::dev::bf16x2_to_f32(qw.x), q1 = lad::dev::bf16x2_to_f32(qw.y);
+                const float2 k0 = lad::dev::bf16x2_to_f32(kw.x), k1 = lad::dev::bf16x2_to_f32(kw.y);
+                const float rq = s_rq[r], rk = s_rk[r];
+                const float qv[4] = {q0.x * rq, q0.y * rq, q1.x * rq, q1.y * rq};
+                const float kv[4] = {k0.x * rk, k0.y * rk, k1.x * rk, k1.y * rk};
+                st_tile4(sm + kOffXQK, r, c4, kStr16, qv[0] * gg[0], qv[1] * gg[1], qv[2] * gg[2], qv[3] * gg[3]);
+                st_tile4(sm + kOffXQK, kC + r, c4, kStr16, kv[0] * gg[0], kv[1] * gg[1], kv[2] * gg[2], kv[3] * gg[3]);
+                st_tile4(sm + kOffKH, r, c4, kStr8, __fdividef(kv[0], gg[0]), __fdividef(kv[1], gg[1]),
+                         __fdividef(kv[2], gg[2]), __fdividef(kv[3], gg[3]));
+            }
+            // V^T: thread -> value column j = tid % 64, tokens 16 * (tid / 64) .. + 15
+            const uint16_t *sv = reinterpret_cast<const uint16_t *>(sm + kOffStV);
+            const int j = tid & 63, r0 = 16 * (tid >> 6);
+            float vv[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) vv[r] = bf16_to_f32(sv[(r0 + r) * kDvh + j]);
             __syncthreads();  // the staging area is read; Kt^T, Kh^T and V^T overwrite it
 #pragma unroll
-            for (int r = 0; r < 32; r += 4) st_tile4(sm + kOffVT, j, r0 + r, kStr8, vv[r], vv[r + 1], vv[r + 2], vv[r + 3]);
-            // Kt^T and Kh^T: row i, from the [token][d_k] tiles just written (already tf32)
-#pragma unroll 4
-            for (int r = 0; r < kC; r += 4) {
+            for (int r = 0; r < 16; r += 4) st_tile4(sm + kOffVT, j, r0 + r, kStr8, vv[r], vv[r + 1], vv[r + 2], vv[r + 3]);
+            // Kt^T and Kh^T: thread -> channel i (row), tokens of half th, from the tiles above
+            const int i = tid & (kDk - 1), th = tid >> 7;
+#pragma unroll 2
+            for (int r = (kC / 2) * th; r < (kC / 2) * (th + 1); r += 4) {
                 float kt[4], kh[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -309,38 +344,32 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
         });
         if (!ok) break;
 
-        // ---- 3a. lower(Qt Kh^T) -> QM (warps 0,1); A -> fp32 scratch (warps 2,3) ----
+        // ---- 3a. lower(Qt Kh^T) -> QM (rows 0-63); A = strict_lower(diag(beta) Kt Kh^T) -> fp32
+        //          scratch (rows 64-127); each thread has 32 of the 64 columns of its row ----
         {
-            float x0[32], x1[32];
-            tmem_ld32(tmem + lane_base + kColAcc1, x0);
-            tmem_ld32(tmem + lane_base + kColAcc1 + 32, x1);
+            float x[32];
+            tmem_ld32(tmem + lane_base + kColAcc1 + 32 * cg, x);
             tmem_wait_ld();
-            const int m = tid;  // accumulator row
-            if (m < kC) {
-                const int r = m;
+            const int c0 = 32 * cg;
+            if (row128 < kC) {
+                const int r = row128;
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    st_tile4(sm + kOffQM, r, j, kStr16, j + 0 <= r ? x0[j] : 0.f, j + 1 <= r ? x0[j + 1] : 0.f,
-                             j + 2 <= r ? x0[j + 2] : 0.f, j + 3 <= r ? x0[j + 3] : 0.f);
-                    st_tile4(sm + kOffQM, r, 32 + j, kStr16, 32 + j <= r ? x1[j] : 0.f, 33 + j <= r ? x1[j + 1] : 0.f,
-                             34 + j <= r ? x1[j + 2] : 0.f, 35 + j <= r ? x1[j + 3] : 0.f);
-                }
+                for (int j = 0; j < 32; j += 4)
+                    st_tile4(sm + kOffQM, r, c0 + j, kStr16, c0 + j <= r ? x[j] : 0.f, c0 + j + 1 <= r ? x[j + 1] : 0.f,
+                             c0 + j + 2 <= r ? x[j + 2] : 0.f, c0 + j + 3 <= r ? x[j + 3] : 0.f);
             } else {
-                const int r = m - kC;
+                const int r = row128 - kC;
                 const float br = s_beta[r];
-                float4 *dst = reinterpret_cast<float4 *>(Apl + r * 64);
+                float4 *dst = reinterpret_cast<float4 *>(Apl + r * 64 + c0);
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    dst[j / 4] = make_float4(j < r ? br * x0[j] : 0.f, j + 1 < r ? br * x0[j + 1] : 0.f,
-                                             j + 2 < r ? br * x0[j + 2] : 0.f, j + 3 < r ? br * x0[j + 3] : 0.f);
-                    dst[8 + j / 4] = make_float4(32 + j < r ? br * x1[j] : 0.f, 33 + j < r ? br * x1[j + 1] : 0.f,
-                                                 34 + j < r ? br * x1[j + 2] : 0.f, 35 + j < r ? br * x1[j + 3] : 0.f);
-                }
+                for (int j = 0; j < 32; j += 4)
+                    dst[j / 4] = make_float4(c0 + j < r ? br * x[j] : 0.f, c0 + j + 1 < r ? br * x[j + 1] : 0.f,
+                                             c0 + j + 2 < r ? br * x[j + 2] : 0.f, c0 + j + 3 < r ? br * x[j + 3] : 0.f);
             }
         }
         __syncthreads();
 
-        // ---- 3b. T = (I + A)^-1, A strictly lower: diagonal 16x16 blocks first ----
+        // ---- 3b. T = (I + A)^-1, A strictly lower: diagonal 16x16 blocks by forward substitution ----
         if (tid < kC) {
             const int base = 16 * (tid >> 4), c = tid & 15;
             float t[16];
@@ -354,73 +383,58 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) Tpl[(base + rr) * 64 + base + c] = t[rr];
         } else {
-            // zero the blocks above the diagonal: (bi, bj) with bi < bj
-            for (int e = tid - kC; e < 6 * 256; e += kThreads - kC) {
-                const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+            // zero the blocks above the diagonal: (bi, bj) with bi < bj, 4 floats per store
+            for (int e = tid - kC; e < 6 * 64; e += kThreads - kC) {
+                const int blk = e >> 6, rr = (e >> 2) & 15, cc = (e & 3) * 4;
                 const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
                 const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                Tpl[(16 * bi + rr) * 64 + 16 * bj + cc] = 0.f;
+                *reinterpret_cast<float4 *>(Tpl + (16 * bi + rr) * 64 + 16 * bj + cc) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
         __syncthreads();
-        // block rows 1..3: T_ij = -T_ii * sum_{k=j}^{i-1} A_ik T_kj
+        // block rows 1..3: T_ij = -T_ii * sum_{k=j}^{i-1} A_ik T_kj; a thread computes a 1x4 strip
 #pragma unroll 1
         for (int bi = 1; bi < 4; ++bi) {
-            const int nel = bi * 256;
-            float rv[6];
+            const bool act = tid < bi * 64;
+            const int bj = tid >> 6, rr = (tid >> 2) & 15, cc = (tid & 3) * 4;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (act) {
+                for (int kb = bj; kb < bi; ++kb) {
 #pragma unroll
-            for (int u = 0; u < 6; ++u) {
-                const int e = tid + kThreads * u;
-                rv[u] = 0.f;
-                if (e < nel) {
-                    const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-                    float acc = 0.f;
-                    for (int kb = bj; kb < bi; ++kb)
-#pragma unroll
-                        for (int ss = 0; ss < 16; ++ss)
-                            acc += Apl[(16 * bi + rr) * 64 + 16 * kb + ss] * Tpl[(16 * kb + ss) * 64 + 16 * bj + cc];
-                    rv[u] = acc;
+                    for (int ss = 0; ss < 16; ++ss) {
+                        const float a = Apl[(16 * bi + rr) * 64 + 16 * kb + ss];
+                        const float4 t4 = *reinterpret_cast<const float4 *>(Tpl + (16 * kb + ss) * 64 + 16 * bj + cc);
+                        acc.x = fmaf(a, t4.x, acc.x);
+                        acc.y = fmaf(a, t4.y, acc.y);
+                        acc.z = fmaf(a, t4.z, acc.z);
+                        acc.w = fmaf(a, t4.w, acc.w);
+                    }
                 }
             }
             __syncthreads();
+            if (act) *reinterpret_cast<float4 *>(Tpl + (16 * bi + rr) * 64 + 16 * bj + cc) = acc;  // R_j, for now
+            __syncthreads();
+            float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (act) {
 #pragma unroll
-            for (int u = 0; u < 6; ++u) {
-                const int e = tid + kThreads * u;
-                if (e < nel) {
-                    const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-                    Tpl[(16 * bi + rr) * 64 + 16 * bj + cc] = rv[u];  // holds R_j for the next step
+                for (int ss = 0; ss < 16; ++ss) {
+                    const float t = Tpl[(16 * bi + rr) * 64 + 16 * bi + ss];
+                    const float4 r4 = *reinterpret_cast<const float4 *>(Tpl + (16 * bi + ss) * 64 + 16 * bj + cc);
+                    out.x = fmaf(-t, r4.x, out.x);
+                    out.y = fmaf(-t, r4.y, out.y);
+                    out.z = fmaf(-t, r4.z, out.z);
+                    out.w = fmaf(-t, r4.w, out.w);
                 }
             }
             __syncthreads();
-#pragma unroll
-            for (int u = 0; u < 6; ++u) {
-                const int e = tid + kThreads * u;
-                rv[u] = 0.f;
-                if (e < nel) {
-                    const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int ss = 0; ss < 16; ++ss)
-                        acc -= Tpl[(16 * bi + rr) * 64 + 16 * bi + ss] * Tpl[(16 * bi + ss) * 64 + 16 * bj + cc];
-                    rv[u] = acc;
-                }
-            }
-            __syncthreads();
-#pragma unroll
-            for (int u = 0; u < 6; ++u) {
-                const int e = tid + kThreads * u;
-                if (e < nel) {
-                    const int bj = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-                    Tpl[(16 * bi + rr) * 64 + 16 * bj + cc] = rv[u];
-                }
-            }
+            if (act) *reinterpret_cast<float4 *>(Tpl + (16 * bi + rr) * 64 + 16 * bj + cc) = out;
             __syncthreads();
         }
-        // Tb = T diag(beta) -> operand tile (thread -> row tid/2, 32 columns)
+        // Tb = T diag(beta) -> operand tile (thread -> row tid/4, 16 columns)
         {
-            const int r = tid >> 1, jc = (tid & 1) * 32;
+            const int r = tid >> 2, jc = (tid & 3) * 16;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
+            for (int j = 0; j < 16; j += 4) {
                 const float4 t4 = *reinterpret_cast<const float4 *>(Tpl + r * 64 + jc + j);
                 st_tile4(sm + kOffTT, r, jc + j, kStr16, t4.x * s_beta[jc + j], t4.y * s_beta[jc + j + 1],
                          t4.z * s_beta[jc + j + 2], t4.w * s_beta[jc + j + 3]);
@@ -437,16 +451,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
             }
         });
         if (!ok) break;
-        // W [r][d_k] -> operand in the Kh slot: thread = d_k row of W^T, writes column i of W
+        // W [r][d_k] -> operand in the Kh slot: this thread has W^T row row128 (= d_k), 32 tokens
         {
+            float w[32];
+            tmem_ld32(tmem + lane_base + kColWT + 32 * cg, w);
+            tmem_wait_ld();
 #pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                float w[32];
-                tmem_ld32(tmem + lane_base + kColWT + 32 * c2, w);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) st_tile1(sm + kOffKH, 32 * c2 + j, tid, kStr8, w[j]);
-            }
+            for (int j = 0; j < 32; ++j) st_tile1(sm + kOffKH, 32 * cg + j, row128, kStr8, w[j]);
         }
 
         // ---- 5. X = W S0 (B = S0^T);  U = U' - X -> U^T operand ----
@@ -458,17 +469,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
         });
         if (!ok) break;
         {
-            const int r = 16 * warp + lane;  // M = 64 accumulator row (lanes 0-15 of each sub-partition)
+            float u[32], x[32];
+            tmem_ld32(tmem + lane_base + kColU + 32 * cg, u);
+            tmem_ld32(tmem + lane_base + kColX + 32 * cg, x);
+            tmem_wait_ld();
+            if (lane < 16) {
 #pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                float u[32], x[32];
-                tmem_ld32(tmem + lane_base + kColU + 32 * c2, u);
-                tmem_ld32(tmem + lane_base + kColX + 32 * c2, x);
-                tmem_wait_ld();
-                if (lane < 16) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) st_tile1(sm + kOffVT, 32 * c2 + j, r, kStr8, u[j] - x[j]);
-                }
+                for (int j = 0; j < 32; ++j) st_tile1(sm + kOffVT, 32 * cg + j, row64, kStr8, u[j] - x[j]);
             }
         }
 
@@ -493,51 +500,42 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
             pending = 1;
         }
         {
-            const int r = 16 * warp + lane;
-#pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                float ov[32];
-                tmem_ld32(tmem + lane_base + kColO + 32 * c2, ov);
-                tmem_wait_ld();
-                if (lane < 16 && r < n) {
-                    const size_t orow = (tok0 + r * tstride) * kDv + half * kDvh + 32 * c2;
-                    if (p.out_f32) {
-                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow);
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            dst[j / 4] = make_float4(p.scale * ov[j], p.scale * ov[j + 1], p.scale * ov[j + 2],
-                                                     p.scale * ov[j + 3]);
-                    } else {
-                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) + orow);
-#pragma unroll
-                        for (int j = 0; j < 32; j += 8)
-                            dst[j / 8] = make_uint4(lad::dev::f32x2_to_bf16x2(p.scale * ov[j], p.scale * ov[j + 1]),
-                                                    lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 2], p.scale * ov[j + 3]),
-                                                    lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 4], p.scale * ov[j + 5]),
-                                                    lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 6], p.scale * ov[j + 7]));
-                    }
-                }
-            }
-            const bool last = (ch == nchunks - 1);
-            const float gc = s_gc[tid];
-            float *Sout = p.S + (static_cast<size_t>(bh) * kDk + tid) * kDv + half * kDvh;
-#pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                float sv[32];
-                tmem_ld32(tmem + lane_base + kColS + 32 * c2, sv);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    sv[j] *= gc;
-                    st_tile1(sm + kOffSOT, 32 * c2 + j, tid, kStr8, sv[j]);
-                }
-                tmem_st32(tmem + lane_base + kColS + 32 * c2, sv);
-                if (last) {
+            float ov[32];
+            tmem_ld32(tmem + lane_base + kColO + 32 * cg, ov);
+            tmem_wait_ld();
+            if (lane < 16 && row64 < n) {
+                const size_t orow = (tok0 + row64 * tstride) * kDv + half * kDvh + 32 * cg;
+                if (p.out_f32) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow);
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4 *>(Sout + 32 * c2 + j) = make_float4(sv[j], sv[j + 1], sv[j + 2],
-                                                                                      sv[j + 3]);
+                        dst[j / 4] = make_float4(p.scale * ov[j], p.scale * ov[j + 1], p.scale * ov[j + 2],
+                                                 p.scale * ov[j + 3]);
+                } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) + orow);
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8)
+                        dst[j / 8] = make_uint4(lad::dev::f32x2_to_bf16x2(p.scale * ov[j], p.scale * ov[j + 1]),
+                                                lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 2], p.scale * ov[j + 3]),
+                                                lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 4], p.scale * ov[j + 5]),
+                                                lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 6], p.scale * ov[j + 7]));
                 }
+            }
+            const float gc = s_gc[row128];
+            float sv[32];
+            tmem_ld32(tmem + lane_base + kColS + 32 * cg, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                sv[j] *= gc;
+                st_tile1(sm + kOffSOT, 32 * cg + j, row128, kStr8, sv[j]);
+            }
+            tmem_st32(tmem + lane_base + kColS + 32 * cg, sv);
+            if (ch == nchunks - 1) {
+                float *Sout = p.S + (static_cast<size_t>(bh) * kDk + row128) * kDv + half * kDvh + 32 * cg;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(Sout + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
             }
             tmem_wait_st();
         }
