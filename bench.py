@@ -196,7 +196,12 @@ class Step:
 
 
 class _KdaLayer:
-    """State and per-token inputs of one KDA decode layer (conv + gated delta rule)."""
+    """State and per-token inputs of one KDA decode layer (conv + gated delta rule).
+
+    fused=True runs kda_conv_decode_step (one launch); fused=False runs kda_conv_update and
+    kda_decode_step on the conv output (two launches)."""
+
+    fused = True
 
     def __init__(self, lad, B, seed, dev, tag=""):
         cfg = wl.KdaDecode(f"kda{tag}", B=B, seed=seed)
@@ -214,6 +219,13 @@ class _KdaLayer:
 
     def run(self, timer=None):
         lad, hd = self.lad, H * D
+        if self.fused:
+            if timer:
+                timer.begin("kda_conv_decode_step")
+            lad.kda_conv_decode_step(self.x, self.tail, self.w, self.alpha, self.beta, self.S, o=self.o)
+            if timer:
+                timer.end("kda_conv_decode_step")
+            return
         lad.kda_conv_update(self.x, self.tail, self.w, y=self.y, silu=True)
         if timer:
             timer.begin("kda_decode_step")
@@ -243,6 +255,12 @@ class _KdaLayer:
         return B * C * 2 * (1 + 3 + 3 + 1) + C * 4 * 2
 
     @staticmethod
+    def bytes_fused(B):
+        # state read + write, raw token, tails read + written, alpha, beta, o per (b, h); taps once
+        C = 3 * H * D
+        return B * H * (2 * D * D * 4 + D * 4 + 4 + D * 2) + B * C * 2 * (1 + 3 + 3) + C * 4 * 2
+
+    @staticmethod
     def bytes_decode(B):
         # per (b, h): state read + write (fp32 128x128), q,k,v (bf16), alpha (fp32), beta, o (bf16)
         return B * H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2)
@@ -254,9 +272,10 @@ class KdaDecodeStep(Step):
     def __init__(self, lad, dev, rank, B=64):
         self.layer = _KdaLayer(lad, B, 1235 + 1000 * rank, dev)
         self.tokens_per_step = B
-        self.launches_per_step = 2
-        self.dominant = "kda_decode_step"
+        self.launches_per_step = 1 if _KdaLayer.fused else 2
+        self.dominant = "kda_conv_decode_step" if _KdaLayer.fused else "kda_decode_step"
         self.config = {"workload": self.name, "batch_per_gpu": B, "heads": H, "head_dim": D,
+                       "kda_path": "fused conv+step" if _KdaLayer.fused else "conv, then step",
                        "state": "fp32 128x128 per head", "conv": "width 4 over 3x8192 bf16 channels",
                        "l2": "inputs larger than L2 (268 MB of state per step)"}
 
@@ -274,7 +293,9 @@ class KdaDecodeStep(Step):
     def algorithmic_bytes(self):
         B = self.layer.B
         return {"kda_decode_step": _KdaLayer.bytes_decode(B), "kda_conv_update": _KdaLayer.bytes_conv(B),
-                "step": _KdaLayer.bytes_decode(B) + _KdaLayer.bytes_conv(B)}
+                "kda_conv_decode_step": _KdaLayer.bytes_fused(B),
+                "step": (_KdaLayer.bytes_fused(B) if _KdaLayer.fused
+                         else _KdaLayer.bytes_decode(B) + _KdaLayer.bytes_conv(B))}
 
 
 class MlaDecodeStep(Step):
@@ -344,9 +365,10 @@ class HybridStep(Step):
         self.kda = [_KdaLayer(lad, B, seed, dev, tag=f"L{i}.") for i in range(kda_layers)]
         self.mla = MlaDecodeStep(lad, dev, rank, wl.MlaDecode("mla", B=B, seed=seed, fixed_len=ctx))
         self.tokens_per_step = B
-        self.launches_per_step = 2 * kda_layers + self.mla.launches_per_step
+        self.launches_per_step = (1 if _KdaLayer.fused else 2) * kda_layers + self.mla.launches_per_step
         self.dominant = "mla_latent_decode"
         self.config = {"workload": self.name, "batch_per_gpu": B, "layers": f"{kda_layers} KDA + 1 gated MLA",
+                       "kda_path": "fused conv+step" if _KdaLayer.fused else "conv, then step",
                        "mla_context": ctx, "heads": H, "head_dim": D,
                        "l2": "inputs larger than L2 (9.2 GB latent cache + 235 MB KDA state per step)"}
 
@@ -373,8 +395,9 @@ class HybridStep(Step):
         B = self.kda[0].B
         n = len(self.kda)
         kd, kc, m = _KdaLayer.bytes_decode(B), _KdaLayer.bytes_conv(B), self.mla.mla_bytes()
-        return {"kda_decode_step": kd, "kda_conv_update": kc, "mla_latent_decode": m,
-                "step": n * (kd + kc) + m}
+        kf = _KdaLayer.bytes_fused(B)
+        return {"kda_decode_step": kd, "kda_conv_update": kc, "kda_conv_decode_step": kf, "mla_latent_decode": m,
+                "step": n * (kf if _KdaLayer.fused else kd + kc) + m}
 
 
 class PrefillStep(Step):
@@ -396,7 +419,7 @@ class PrefillStep(Step):
         self.launches_per_step = 1
         self.dominant = "kda_prefill_chunked"
         self.config = {"workload": self.name, "batch_per_gpu": cfg.B, "seq_len": cfg.T, "heads": cfg.H,
-                       "chunk": cfg.chunk, "l2": "inputs larger than L2 (3.2 GB per step)"}
+                       "chunk": cfg.chunk, "l2": f"inputs larger than L2 ({self.algorithmic_bytes()['step'] / 1e9:.2f} GB per step)"}
 
     def run(self, timer=None):
         if timer:
@@ -559,7 +582,11 @@ def main(argv=None) -> int:
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="lad", choices=["lad", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=32768, help="tokens of the kda_prefill_32k workload")
+    ap.add_argument("--unfused-conv", action="store_true",
+                    help="KDA layers as kda_conv_update + kda_decode_step instead of kda_conv_decode_step")
     args = ap.parse_args(argv)
+    _KdaLayer.fused = not args.unfused_conv
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
@@ -574,7 +601,11 @@ def main(argv=None) -> int:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    step = WORKLOADS[args.workload](lad, dev, rank)
+    if args.workload == "kda_prefill_32k":
+        step = PrefillStep(lad, dev, rank, wl.KdaScan("prefill", B=1, H=64, T=args.seq_len, chunk=64,
+                                                      seed=1237 + 1000 * rank))
+    else:
+        step = WORKLOADS[args.workload](lad, dev, rank)
     torch.cuda.synchronize()
 
     for _ in range(args.warmup):
@@ -623,7 +654,7 @@ def main(argv=None) -> int:
     dom_ms = timer.mean_ms(step.dominant)
     achieved = ab[step.dominant] / (dom_ms / 1000.0) / 1e9
     per_type = {}
-    for kname in ("kda_decode_step", "mla_latent_decode", "kda_prefill_chunked"):
+    for kname in ("kda_conv_decode_step", "kda_decode_step", "mla_latent_decode", "kda_prefill_chunked"):
         km = timer.mean_ms(kname)
         if km is not None and kname in ab:
             gbs = ab[kname] / (km / 1000.0) / 1e9

@@ -114,6 +114,24 @@ int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, lon
                     float scale, unsigned flags, void *stream);
 
 /*
+ * kda_conv_decode_step — kda_conv_update and kda_decode_step of one KDA layer in one launch: the
+ * short convolution of each head's q, k and v channels runs in the CTA that updates that head's
+ * state ([P2] "How KDA and MLA split the work": q, k, v come through the width-4 short causal
+ * convolution, then the gated delta rule). The conv output stays in fp32 (it is not rounded to
+ * bf16 on the way, unlike the two-call path) and never touches HBM.
+ *
+ *   x          bf16 [B][3*H*dk]       raw token, channels q | k | v (read)
+ *   conv_tail  bf16 [B][K-1][3*H*dk]  tails, oldest row first (read and updated in place)
+ *   conv_w     bf16 [3*H*dk][K]       taps (8-byte aligned); conv_bias bf16 [3*H*dk] or NULL
+ *   alpha, beta, S, o                 as in kda_decode_step
+ * flags: LAD_FLAG_SILU (conv output through SiLU), LAD_FLAG_L2NORM_QK, LAD_FLAG_OUT_FP32.
+ * Supported: dk == dv == 128, K == 4. B == 0 or H == 0 is a no-op.
+ */
+int kda_conv_decode_step(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 *conv_w, const lad_bf16 *conv_bias,
+                         const float *alpha, const float *beta, float *S, void *o, int B, int H, int dk, int dv, int K,
+                         float scale, unsigned flags, void *stream);
+
+/*
  * kda_prefill_chunked — the same recurrence as kda_decode_step over T tokens per sequence,
  * computed chunk by chunk (chunk length `chunk`, a shorter last chunk allowed) in the WY / UT
  * form: inside a chunk with cumulative decays g_r = prod_{s<=r} alpha_s,

@@ -18,7 +18,7 @@ import os
 import torch
 
 __all__ = [
-    "kda_conv_update", "kda_decode_step", "kda_prefill_chunked", "kda_prefill_workspace_size",
+    "kda_conv_update", "kda_decode_step", "kda_conv_decode_step", "kda_prefill_chunked", "kda_prefill_workspace_size",
     "mla_latent_decode", "mla_latent_decode_workspace_size", "mla_latent_decode_noalloc",
     "lad_device_error", "lad_version",
     "LadError", "LIB_PATH", "FLAG_SILU", "FLAG_L2NORM_QK", "FLAG_OUT_FP32", "MLA_SCALE",
@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
         "kda_conv_update": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_u, _c_vp], _c_int),
         "kda_decode_step": ([_c_vp, _c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                              _c_int, _c_f, _c_u, _c_vp], _c_int),
+        "kda_conv_decode_step": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
+                                  _c_int, _c_int, _c_f, _c_u, _c_vp], _c_int),
         "kda_prefill_chunked": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                                  _c_int, _c_int, _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
         "kda_prefill_workspace_size": ([_c_int] * 6, _c_sz),
@@ -75,12 +77,26 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-_lib = _load()
+_loaded = None
+
+
+def _L() -> ctypes.CDLL:
+    """The library, loaded on first use (so that building it never needs an old copy)."""
+    global _loaded
+    if _loaded is None:
+        _loaded = _load()
+    return _loaded
+
+
+def __getattr__(name):
+    if name == "_lib":
+        return _L()
+    raise AttributeError(name)
 
 
 def _check(fn: str, status: int) -> None:
     if status != 0:
-        raise LadError(fn, status, _lib.lad_last_error().decode(errors="replace"))
+        raise LadError(fn, status, _L().lad_last_error().decode(errors="replace"))
 
 
 def _stream(stream) -> int:
@@ -111,13 +127,13 @@ def _ptr(t):
 
 
 def lad_version() -> int:
-    return int(_lib.lad_version())
+    return int(_L().lad_version())
 
 
 def lad_device_error(stream=None) -> int:
     """Synchronises the stream, returns and clears the device error word (0 = no wait gave up)."""
     code = _c_int(0)
-    _check("lad_device_error", _lib.lad_device_error(_stream(stream), ctypes.byref(code)))
+    _check("lad_device_error", _L().lad_device_error(_stream(stream), ctypes.byref(code)))
     return int(code.value)
 
 
@@ -136,7 +152,7 @@ def kda_conv_update(x: torch.Tensor, conv_tail: torch.Tensor, w: torch.Tensor, y
         y = torch.empty_like(x)
     _contig(y, "y", bf)
     flags = FLAG_SILU if silu else 0
-    _check("kda_conv_update", _lib.kda_conv_update(x.data_ptr(), conv_tail.data_ptr(), w.data_ptr(), _ptr(bias),
+    _check("kda_conv_update", _L().kda_conv_update(x.data_ptr(), conv_tail.data_ptr(), w.data_ptr(), _ptr(bias),
                                                    y.data_ptr(), B, Cch, K, flags, _stream(stream)))
     return y
 
@@ -176,14 +192,42 @@ def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: to
         o = torch.empty((B, H, dv), device=S.device, dtype=odt)
     _contig(o, "o", odt)
     flags = (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
-    _check("kda_decode_step", _lib.kda_decode_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), sq, alpha.data_ptr(),
+    _check("kda_decode_step", _L().kda_decode_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), sq, alpha.data_ptr(),
                                                    beta.data_ptr(), S.data_ptr(), o.data_ptr(), B, H, dk, dv,
                                                    float(scale), flags, _stream(stream)))
     return o
 
 
+def kda_conv_decode_step(x: torch.Tensor, conv_tail: torch.Tensor, conv_w: torch.Tensor, alpha: torch.Tensor,
+                         beta: torch.Tensor, S: torch.Tensor, o: torch.Tensor | None = None,
+                         conv_bias: torch.Tensor | None = None, silu: bool = True, l2norm_qk: bool = True,
+                         scale: float = 1.0, out_fp32: bool = False, stream=None) -> torch.Tensor:
+    """Short conv + KDA step of one layer in one launch. x [B,3*H*128] raw token (q|k|v), conv_tail
+    [B,3,3*H*128] and S [B,H,128,128] updated in place; returns o [B,H,128]."""
+    bf = torch.bfloat16
+    _contig(x, "x", bf), _contig(conv_tail, "conv_tail", bf), _contig(conv_w, "conv_w", bf)
+    _contig(S, "S", torch.float32), _contig(alpha, "alpha", torch.float32), _contig(beta, "beta", torch.float32)
+    B, H, dk, dv = S.shape
+    K = conv_w.shape[1]
+    if x.shape != (B, 3 * H * dk) or conv_tail.shape != (B, K - 1, 3 * H * dk) or conv_w.shape != (3 * H * dk, K):
+        raise ValueError("kda_conv_decode_step: inconsistent conv shapes")
+    if alpha.numel() != B * H * dk or beta.numel() != B * H:
+        raise ValueError("alpha must be [B,H,dk] and beta [B,H]")
+    if conv_bias is not None:
+        _contig(conv_bias, "conv_bias", bf)
+    odt = torch.float32 if out_fp32 else bf
+    if o is None:
+        o = torch.empty((B, H, dv), device=S.device, dtype=odt)
+    _contig(o, "o", odt)
+    flags = (FLAG_SILU if silu else 0) | (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
+    _check("kda_conv_decode_step", _L().kda_conv_decode_step(
+        x.data_ptr(), conv_tail.data_ptr(), conv_w.data_ptr(), _ptr(conv_bias), alpha.data_ptr(), beta.data_ptr(),
+        S.data_ptr(), o.data_ptr(), B, H, dk, dv, K, float(scale), flags, _stream(stream)))
+    return o
+
+
 def kda_prefill_workspace_size(B: int, T: int, H: int, dk: int = 128, dv: int = 128, chunk: int = 64) -> int:
-    return int(_lib.kda_prefill_workspace_size(B, T, H, dk, dv, chunk))
+    return int(_L().kda_prefill_workspace_size(B, T, H, dk, dv, chunk))
 
 
 def kda_prefill_chunked(q, k, v, alpha, beta, S, o=None, chunk: int = 64, scale: float = 1.0,
@@ -205,7 +249,7 @@ def kda_prefill_chunked(q, k, v, alpha, beta, S, o=None, chunk: int = 64, scale:
     if workspace is None and ws > 0:
         workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
     flags = (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
-    _check("kda_prefill_chunked", _lib.kda_prefill_chunked(
+    _check("kda_prefill_chunked", _L().kda_prefill_chunked(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), alpha.data_ptr(), beta.data_ptr(), S.data_ptr(), o.data_ptr(),
         B, T, H, dk, dv, chunk, float(scale), flags, _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
@@ -213,7 +257,7 @@ def kda_prefill_chunked(q, k, v, alpha, beta, S, o=None, chunk: int = 64, scale:
 
 
 def mla_latent_decode_workspace_size(B: int, Hq: int = 64, d_latent: int = 512, num_sms: int = 0) -> int:
-    return int(_lib.mla_latent_decode_workspace_size(B, Hq, d_latent, num_sms))
+    return int(_L().mla_latent_decode_workspace_size(B, Hq, d_latent, num_sms))
 
 
 def mla_latent_decode(q: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tensor,
@@ -250,7 +294,7 @@ def mla_latent_decode(q: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tens
         workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
     flags = FLAG_OUT_FP32 if out_fp32 else 0
     seq_stride = cache.stride(0) if B > 1 else Lmax * D
-    _check("mla_latent_decode", _lib.mla_latent_decode(
+    _check("mla_latent_decode", _L().mla_latent_decode(
         q.data_ptr(), cache.data_ptr(), seq_stride, seq_lens.data_ptr(), _ptr(gate_logits), o.data_ptr(),
         _ptr(lse), B, Hq, d_latent, D - d_latent, Lmax, float(scale), flags, _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
@@ -284,7 +328,7 @@ def mla_latent_decode_noalloc(q: torch.Tensor, cache: torch.Tensor, seq_lens: to
     if lse is not None:
         _contig(lse, "lse", torch.float32)
     seq_stride = cache.stride(0) if B > 1 else cache.shape[1] * D
-    _check("mla_latent_decode_noalloc", _lib.mla_latent_decode_noalloc(
+    _check("mla_latent_decode_noalloc", _L().mla_latent_decode_noalloc(
         q.data_ptr(), cache.data_ptr(), seq_stride, seq_lens.data_ptr(), _ptr(gate_logits), o.data_ptr(),
         _ptr(lse), B, Hq, d_latent, D - d_latent, cache.shape[1], float(scale), FLAG_OUT_FP32 if out_fp32 else 0,
         _stream(stream)))

@@ -46,11 +46,21 @@ __device__ __forceinline__ void add4(float4 &acc, const float4 &x) {
     acc.w += x.w;
 }
 
-template <bool kOutF32>
+// The short convolution of one head's q, k and v channels, fused in front of the step (see
+// kda_conv_decode_step): raw token x [B][3 H 128], tails [B][3][3 H 128], taps [3 H 128][4].
+struct ConvIn {
+    const uint16_t *x;
+    uint16_t *tail;
+    const uint16_t *w;
+    const uint16_t *bias;
+    int silu;
+};
+
+template <bool kOutF32, bool kFusedConv>
 __global__ void __launch_bounds__(kThreads, 2)
 kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const uint16_t *__restrict__ v,
                   long long qkv_stride, const float *__restrict__ alpha, const float *__restrict__ beta,
-                  float *__restrict__ S, void *__restrict__ o, int H, float scale, int l2norm) {
+                  float *__restrict__ S, void *__restrict__ o, int H, float scale, int l2norm, ConvIn cv) {
     const int bh = blockIdx.x;
     const int b = bh / H;
     const int h = bh - b * H;
@@ -67,13 +77,46 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
     __shared__ float sq[kD], sk[kD], sv[kD], sa[kD];
     __shared__ float4 red_k[kWarps][kVec], red_q[kWarps][kVec];
 
-    const size_t row = static_cast<size_t>(b) * qkv_stride + static_cast<size_t>(h) * kD;
-    if (threadIdx.x < kD) {
-        const int i = threadIdx.x;
-        sq[i] = bf16_to_f32(q[row + i]);
-        sk[i] = bf16_to_f32(k[row + i]);
-        sv[i] = bf16_to_f32(v[row + i]);
-        sa[i] = alpha[static_cast<size_t>(bh) * kD + i];
+    if constexpr (kFusedConv) {
+        // y = taps . (tail, x) (+ bias), SiLU; kept in fp32; the tail shifts in place. Threads
+        // 0-127 take this head's q and k channels, threads 128-255 its v channels.
+        const size_t cch = static_cast<size_t>(3) * H * kD;
+        const uint16_t *xb = cv.x + static_cast<size_t>(b) * cch;
+        uint16_t *tb = cv.tail + static_cast<size_t>(b) * 3 * cch;
+        auto conv = [&](size_t c) -> float {
+            const uint16_t xr = xb[c], t0 = tb[c], t1 = tb[cch + c], t2 = tb[2 * cch + c];
+            const uint2 wv = *reinterpret_cast<const uint2 *>(cv.w + c * 4);
+            const float2 w01 = lad::dev::bf16x2_to_f32(wv.x), w23 = lad::dev::bf16x2_to_f32(wv.y);
+            float acc = w01.x * bf16_to_f32(t0);
+            acc = fmaf(w01.y, bf16_to_f32(t1), acc);
+            acc = fmaf(w23.x, bf16_to_f32(t2), acc);
+            acc = fmaf(w23.y, bf16_to_f32(xr), acc);
+            if (cv.bias) acc += bf16_to_f32(cv.bias[c]);
+            if (cv.silu) acc = acc / (1.f + expf(-acc));
+            tb[c] = t1;
+            tb[cch + c] = t2;
+            tb[2 * cch + c] = xr;
+            return acc;
+        };
+        const size_t hc = static_cast<size_t>(h) * kD;
+        if (threadIdx.x < kD) {
+            const int i = threadIdx.x;
+            sq[i] = conv(hc + i);
+            sk[i] = conv(static_cast<size_t>(H) * kD + hc + i);
+            sa[i] = alpha[static_cast<size_t>(bh) * kD + i];
+        } else {
+            const int i = threadIdx.x - kD;
+            sv[i] = conv(static_cast<size_t>(2) * H * kD + hc + i);
+        }
+    } else {
+        const size_t row = static_cast<size_t>(b) * qkv_stride + static_cast<size_t>(h) * kD;
+        if (threadIdx.x < kD) {
+            const int i = threadIdx.x;
+            sq[i] = bf16_to_f32(q[row + i]);
+            sk[i] = bf16_to_f32(k[row + i]);
+            sv[i] = bf16_to_f32(v[row + i]);
+            sa[i] = alpha[static_cast<size_t>(bh) * kD + i];
+        }
     }
     const float bt = beta[bh];
     __syncthreads();
@@ -176,11 +219,42 @@ extern "C" int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_b
     if (blocks > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "kda_decode_step: B*H too large");
     const int l2 = (flags & LAD_FLAG_L2NORM_QK) ? 1 : 0;
     cudaStream_t s = lad::as_stream(stream);
+    const ConvIn none{nullptr, nullptr, nullptr, nullptr, 0};
     if (f32)
-        kda_decode_kernel<true><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(q, k, v, stride, alpha, beta, S, o,
-                                                                                   H, scale, l2);
+        kda_decode_kernel<true, false><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(q, k, v, stride, alpha, beta,
+                                                                                          S, o, H, scale, l2, none);
     else
-        kda_decode_kernel<false><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(q, k, v, stride, alpha, beta, S,
-                                                                                    o, H, scale, l2);
+        kda_decode_kernel<false, false><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(q, k, v, stride, alpha, beta,
+                                                                                           S, o, H, scale, l2, none);
     return lad::check_launch("kda_decode_step");
+}
+
+extern "C" int kda_conv_decode_step(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 *conv_w,
+                                    const lad_bf16 *conv_bias, const float *alpha, const float *beta, float *S, void *o,
+                                    int B, int H, int dk, int dv, int K, float scale, unsigned flags, void *stream) {
+    using lad::set_error;
+    if (B < 0 || H < 0) return set_error(LAD_EINVAL, "kda_conv_decode_step: negative B or H");
+    if (dk != kD || dv != kD) return set_error(LAD_EUNSUPPORTED, "kda_conv_decode_step: dk = dv = 128 only");
+    if (K != 4) return set_error(LAD_EUNSUPPORTED, "kda_conv_decode_step: K = 4 only");
+    if (flags & ~(LAD_FLAG_OUT_FP32 | LAD_FLAG_L2NORM_QK | LAD_FLAG_SILU))
+        return set_error(LAD_EINVAL, "kda_conv_decode_step: unknown flags 0x%x", flags);
+    if (B == 0 || H == 0) return LAD_OK;
+    if (!x || !conv_tail || !conv_w || !alpha || !beta || !S || !o)
+        return set_error(LAD_EINVAL, "kda_conv_decode_step: null pointer");
+    if (!lad::aligned(S, 16) || !lad::aligned(conv_w, 8))
+        return set_error(LAD_EUNSUPPORTED, "kda_conv_decode_step: S 16-byte and conv_w 8-byte aligned");
+    const bool f32 = (flags & LAD_FLAG_OUT_FP32) != 0;
+    if (!lad::aligned(o, f32 ? 16 : 8)) return set_error(LAD_EUNSUPPORTED, "kda_conv_decode_step: o misaligned");
+    const long long blocks = static_cast<long long>(B) * H;
+    if (blocks > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "kda_conv_decode_step: B*H too large");
+    const int l2 = (flags & LAD_FLAG_L2NORM_QK) ? 1 : 0;
+    const ConvIn cv{x, conv_tail, conv_w, conv_bias, (flags & LAD_FLAG_SILU) ? 1 : 0};
+    cudaStream_t s = lad::as_stream(stream);
+    if (f32)
+        kda_decode_kernel<true, true><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
+            nullptr, nullptr, nullptr, 0, alpha, beta, S, o, H, scale, l2, cv);
+    else
+        kda_decode_kernel<false, true><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
+            nullptr, nullptr, nullptr, 0, alpha, beta, S, o, H, scale, l2, cv);
+    return lad::check_launch("kda_conv_decode_step");
 }

@@ -169,3 +169,67 @@ def test_conv_rejects_bad_width(lad, cuda_device):
     with pytest.raises(lad.LadError) as e:
         lad.kda_conv_update(inp["x"], inp["tail"], inp["w"])
     assert e.value.status == -2
+
+
+def _fused_oracle(inp, H, silu=True, bias=None):
+    """Conv (fp64, no bf16 rounding of its output) -> L2 norm -> one recurrent step."""
+    B = inp["x"].shape[0]
+    d = 128
+    y, tail = oracle.short_conv_step(f64(inp["x"]), f64(inp["tail"]), f64(inp["w"]),
+                                     None if bias is None else f64(bias), silu=silu)
+    q = oracle.l2norm(y[:, : H * d].reshape(B, 1, H, d))
+    k = oracle.l2norm(y[:, H * d: 2 * H * d].reshape(B, 1, H, d))
+    v = y[:, 2 * H * d:].reshape(B, 1, H, d)
+    o, S = oracle.kda_recurrent(q, k, v, f64(inp["alpha"])[:, None], f64(inp["beta"])[:, None], f64(inp["S"]),
+                                nthreads=oracle.max_threads())
+    return o[:, 0], S, tail
+
+
+def test_fused_conv_decode_b64(lad, cuda_device):
+    """kda_conv_decode_step on the 64 x 64-head layer: conv, L2 norm and the step in one launch."""
+    cfg = wl.CONFIGS["kda_decode_b64"]
+    inp = wl.kda_decode_inputs(cfg, cuda_device)
+    o_ref, S_ref, tail_ref = _fused_oracle(inp, cfg.H)
+    o = lad.kda_conv_decode_step(inp["x"], inp["tail"], inp["w"], inp["alpha"], inp["beta"], inp["S"],
+                                 out_fp32=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(f64(inp["tail"]), tail_ref)
+    assert rel_l2(o, o_ref) < 1e-4
+    assert rel_l2(inp["S"], S_ref) < TOL_STATE
+
+
+@pytest.mark.parametrize("B,H,silu,bias", [(1, 1, True, False), (3, 5, False, True)])
+def test_fused_conv_decode_variants(lad, cuda_device, B, H, silu, bias):
+    cfg = wl.KdaDecode("f", B=B, H=H, seed=31 + B)
+    inp = wl.kda_decode_inputs(cfg, cuda_device)
+    bvec = wl.normal_bf16((3 * H * 128,), 31, "bias", cuda_device) if bias else None
+    o_ref, S_ref, tail_ref = _fused_oracle(inp, H, silu=silu, bias=bvec)
+    o = lad.kda_conv_decode_step(inp["x"], inp["tail"], inp["w"], inp["alpha"], inp["beta"], inp["S"],
+                                 conv_bias=bvec, silu=silu, out_fp32=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(f64(inp["tail"]), tail_ref)
+    assert rel_l2(o, o_ref) < 1e-4 and rel_l2(inp["S"], S_ref) < TOL_STATE
+
+
+def test_fused_matches_two_calls(lad, cuda_device):
+    """The fused path keeps the conv output in fp32; the two-call path stores it as bf16. The two
+    kernels must differ by exactly what that rounding does in the oracle."""
+    cfg = wl.KdaDecode("t", B=8, seed=41)
+    a = wl.kda_decode_inputs(cfg, cuda_device)
+    b = {n: t.clone() for n, t in a.items()}
+    H, hd = cfg.H, cfg.H * 128
+    o_f, _, _ = _fused_oracle(a, H)
+    y, _ = oracle.short_conv_step(f64(a["x"]), f64(a["tail"]), f64(a["w"]), None, silu=True)
+    y16 = bf16_round(y)
+    o_2, _ = oracle.kda_recurrent(oracle.l2norm(y16[:, :hd].reshape(8, 1, H, 128)),
+                                  oracle.l2norm(y16[:, hd:2 * hd].reshape(8, 1, H, 128)),
+                                  y16[:, 2 * hd:].reshape(8, 1, H, 128), f64(a["alpha"])[:, None],
+                                  f64(a["beta"])[:, None], f64(a["S"]), nthreads=oracle.max_threads())
+    o1 = lad.kda_conv_decode_step(a["x"], a["tail"], a["w"], a["alpha"], a["beta"], a["S"], out_fp32=True)
+    yk = lad.kda_conv_update(b["x"], b["tail"], b["w"], silu=True)
+    o2 = lad.kda_decode_step(yk[:, :hd], yk[:, hd:2 * hd], yk[:, 2 * hd:], b["alpha"], b["beta"], b["S"],
+                             l2norm_qk=True, out_fp32=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a["tail"], b["tail"])
+    expected = rel_l2(o_2[:, 0], o_f)  # the effect of the bf16 conv output alone
+    assert abs(rel_l2(o2, o1) - expected) < 0.05 * expected
