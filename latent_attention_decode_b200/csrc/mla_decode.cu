@@ -360,6 +360,9 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             if (i == kBarSEmpty || i == kBarSEmpty + 1 || i == kBarPFull || i == kBarPFull + 1 || i == kBarWg ||
                 i == kBarWg + 1 || i == kBarOFree)
                 count = 4;  // one arrival per softmax warp
+            if ((i >= kBarEmpty && i < kBarEmpty + kStages) || i == kBarSFull || i == kBarSFull + 1 ||
+                i == kBarPEmpty || i == kBarPEmpty + 1 || i == kBarQEmpty || i == kBarDrain)
+                count = 2;  // one commit per MMA warp
             mbar_init(bar(i), count);
         }
         *abort_flag = 0;
@@ -427,9 +430,14 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                 }
             }
         }
-    } else if (warp == 1) {
-        // ================= MMA issuer (whole warp, elected lane issues) =================
+    } else if (warp == 1 || warp == 2) {
+        // ================= MMA issuers (warps 1 and 2, whole warps, elected lanes issue) =================
+        // A single warp issues a small tcgen05.mma only every ~28 cycles, below the tensor pipe's
+        // rate for these shapes, so two warps share the work: warp 1 issues GEMM1's even K-chunks
+        // and GEMM2's latent blocks 0-1, warp 2 the odd K-chunks and blocks 2-3. Each keeps its own
+        // accumulators, and every barrier an MMA completion arrives on expects both warps' commits.
         {
+            const int mi = warp - 1;
             int seq, tile0, nt, k = 0;
             uint32_t g = 0;
             bool ok = true;
@@ -458,9 +466,11 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int j = 2 * mi + jj;
                         tc_mma(tmem + kColO + 64 * j, a0 + (((2 * j) * kTChunkBytes + kk * 2048) >> 4),
                                b0 + ((kk * 256) >> 4), kIdesc2, kk == 0 ? acc0 : 1u);
+                    }
                 }
                 tc_commit(bar(kBarEmpty + s));
                 tc_commit(bar(kBarPEmpty + pb));
@@ -483,10 +493,10 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     const uint64_t cd = c_desc0 + ((s * kStageBytes) >> 4);
                     const uint32_t dS = tmem + kColS + sb * kSBufCols;
 #pragma unroll
-                    for (int c = 0; c < kNChunk; ++c) {
+                    for (int c = mi; c < kNChunk; c += 2) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            tc_mma(dS + (c & 1) * kTile, q_desc0 + ((c * kQChunkBytes + kk * 32) >> 4),
+                            tc_mma(dS + mi * kTile, q_desc0 + ((c * kQChunkBytes + kk * 32) >> 4),
                                    cd + ((c * kTChunkBytes + kk * 32) >> 4), kIdesc1, (c > 1 || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(bar(kBarSFull + sb));
