@@ -62,9 +62,12 @@ def _load():
             lib.lado_short_conv_step.argtypes = [ctypes.c_int] * 3 + [_dp, _dp, _dp, _dp, ctypes.c_int, _dp]
             lib.lado_mla_decode.argtypes = ([ctypes.c_int] * 4 + [ctypes.c_longlong, _dp, _up, _ip, _dp,
                                             ctypes.c_double, _dp, _dp, ctypes.c_int])
+            lib.lado_mla_decode_paged.argtypes = ([ctypes.c_int] * 7 + [_dp, _up, _ip, _ip, _dp,
+                                                  ctypes.c_double, _dp, _dp, ctypes.c_int])
             lib.lado_num_threads_available.argtypes = []
             for f in (lib.lado_kda_recurrent, lib.lado_kda_chunked, lib.lado_l2norm,
-                      lib.lado_short_conv_step, lib.lado_mla_decode, lib.lado_num_threads_available):
+                      lib.lado_short_conv_step, lib.lado_mla_decode, lib.lado_mla_decode_paged,
+                      lib.lado_num_threads_available):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -181,4 +184,31 @@ def mla_decode(q, cache_bits, seq_lens, gate=None, scale: float = 192 ** -0.5, d
                                  _ptr(cache_bits, _up), _ptr(lens, _ip), gptr, float(scale),
                                  _ptr(o), _ptr(lse), int(nthreads))
     _check(rc, "mla_decode")
+    return o, lse
+
+
+def mla_decode_paged(q, page_bits, block_table, seq_lens, gate=None, scale: float = 192 ** -0.5,
+                     d_latent: int = 512, nthreads: int = 1):
+    """mla_decode over a paged cache: page_bits uint16 bf16 bit patterns [num_pages, P, D];
+    row t of sequence b is row t % P of page block_table[b, t // P] (block_table int [B, n]).
+    Returns (o [B,H,d_latent], lse [B,H]) in float64."""
+    q = _f64(q)
+    page_bits = np.ascontiguousarray(page_bits, dtype=np.uint16)
+    B, H, D = q.shape
+    assert page_bits.ndim == 3 and page_bits.shape[2] == D
+    num_pages, P = page_bits.shape[0], page_bits.shape[1]
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    assert bt.ndim == 2 and bt.shape[0] == B
+    lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    assert lens.shape == (B,)
+    o = np.zeros((B, H, d_latent), dtype=np.float64)
+    lse = np.zeros((B, H), dtype=np.float64)
+    gptr = None
+    if gate is not None:
+        gate = _f64(gate)
+        gptr = _ptr(gate)
+    rc = _load().lado_mla_decode_paged(B, H, d_latent, D - d_latent, P, num_pages, bt.shape[1], _ptr(q),
+                                       _ptr(page_bits, _up), _ptr(bt, _ip), _ptr(lens, _ip), gptr, float(scale),
+                                       _ptr(o), _ptr(lse), int(nthreads))
+    _check(rc, "mla_decode_paged")
     return o, lse

@@ -310,10 +310,20 @@ int lado_short_conv_step(int B, int Cch, int K, const double *x, double *tail,
  * Layouts: q [B][H][Dc+Dr] (double); cache: bf16 bit patterns, row t of sequence b at
  * element offset b*seq_stride + t*(Dc+Dr); gate [B][H] or NULL; o [B][H][Dc]; lse [B][H] or NULL.
  */
-int lado_mla_decode(int B, int H, int Dc, int Dr, long long seq_stride,
-                    const double *q, const uint16_t *cache, const int *seq_lens,
-                    const double *gate, double scale, double *o, double *lse, int nthreads) {
-    if (B < 0 || H < 0 || Dc <= 0 || Dr < 0) return LADO_EINVAL;
+/* Row t of one sequence's cache: contiguous rows (bt == NULL), or the paged layout in which
+ * rows [j*P, (j+1)*P) of the sequence are page bt[j] of the pool, P rows per page. */
+static const uint16_t *mla_row(const uint16_t *base, const int *bt, int P, int D, int t) {
+    if (!bt) return base + (size_t)t * D;
+    return base + ((size_t)bt[t / P] * (size_t)P + (size_t)(t % P)) * (size_t)D;
+}
+
+/* Shared body of the contiguous and paged entry points. With block_table == NULL, sequence b's
+ * rows start at cache + b*seq_stride; otherwise cache is the page pool and row b of the block
+ * table (bt_stride entries) names its pages of P rows. */
+static int mla_decode_impl(int B, int H, int Dc, int Dr, const double *q, const uint16_t *cache,
+                           long long seq_stride, const int *block_table, int bt_stride, int P,
+                           const int *seq_lens, const double *gate, double scale, double *o, double *lse,
+                           int nthreads) {
     if (nthreads < 1) nthreads = 1;
     const int D = Dc + Dr;
     int err = 0;
@@ -334,10 +344,11 @@ int lado_mla_decode(int B, int H, int Dc, int Dr, long long seq_stride,
                 err = 1;
                 continue;
             }
-            const uint16_t *cb = cache + (size_t)b * (size_t)seq_stride;
+            const uint16_t *cb = block_table ? cache : cache + (size_t)b * (size_t)seq_stride;
+            const int *bt = block_table ? block_table + (size_t)b * (size_t)bt_stride : NULL;
             double m = -INFINITY;
             for (int t = 0; t < L; ++t) {
-                const uint16_t *ct = cb + (size_t)t * D;
+                const uint16_t *ct = mla_row(cb, bt, P, D, t);
                 double acc = 0.0;
                 for (int d = 0; d < D; ++d) acc += qh[d] * bf16_bits_to_double(ct[d]);
                 s[t] = scale * acc;
@@ -350,7 +361,7 @@ int lado_mla_decode(int B, int H, int Dc, int Dr, long long seq_stride,
             }
             for (int d = 0; d < Dc; ++d) oh[d] = 0.0;
             for (int t = 0; t < L; ++t) {
-                const uint16_t *ct = cb + (size_t)t * D;
+                const uint16_t *ct = mla_row(cb, bt, P, D, t);
                 double p = s[t] / z;
                 for (int d = 0; d < Dc; ++d) oh[d] += p * bf16_bits_to_double(ct[d]);
             }
@@ -363,4 +374,37 @@ int lado_mla_decode(int B, int H, int Dc, int Dr, long long seq_stride,
         }
     }
     return err ? LADO_ENOMEM : LADO_OK;
+}
+
+int lado_mla_decode(int B, int H, int Dc, int Dr, long long seq_stride,
+                    const double *q, const uint16_t *cache, const int *seq_lens,
+                    const double *gate, double scale, double *o, double *lse, int nthreads) {
+    if (B < 0 || H < 0 || Dc <= 0 || Dr < 0) return LADO_EINVAL;
+    return mla_decode_impl(B, H, Dc, Dr, q, cache, seq_stride, NULL, 0, 1, seq_lens, gate, scale, o, lse,
+                           nthreads);
+}
+
+/*
+ * The same attention over a paged cache, the layout serving engines keep the latent cache in
+ * ([P2] "How KDA and MLA split the work" and [P1] "How big is the cache per token, exactly?"
+ * give the row; the paging is storage only and changes no arithmetic): the pool holds
+ * num_pages pages of P rows (pages [num_pages][P][Dc+Dr], bf16 bit patterns) and row t of
+ * sequence b is row t % P of page block_table[b*bt_stride + t / P].
+ * Returns LADO_EINVAL if a sequence needs more than bt_stride pages or names a page outside
+ * [0, num_pages).
+ */
+int lado_mla_decode_paged(int B, int H, int Dc, int Dr, int P, int num_pages, int bt_stride,
+                          const double *q, const uint16_t *pages, const int *block_table, const int *seq_lens,
+                          const double *gate, double scale, double *o, double *lse, int nthreads) {
+    if (B < 0 || H < 0 || Dc <= 0 || Dr < 0 || P <= 0 || num_pages < 0 || bt_stride < 0) return LADO_EINVAL;
+    for (int b = 0; b < B; ++b) {
+        const long long L = seq_lens[b];
+        if (L < 0 || L > (long long)bt_stride * P) return LADO_EINVAL;
+        for (long long j = 0; j * P < L; ++j) {
+            const int pg = block_table[(size_t)b * bt_stride + (size_t)j];
+            if (pg < 0 || pg >= num_pages) return LADO_EINVAL;
+        }
+    }
+    return mla_decode_impl(B, H, Dc, Dr, q, pages, 0, block_table, bt_stride, P, seq_lens, gate, scale, o, lse,
+                           nthreads);
 }

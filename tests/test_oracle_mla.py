@@ -125,3 +125,60 @@ def test_threads_do_not_change_results(nthreads):
     o1, l1 = oracle.mla_decode(q, bits, lens, None, scale=0.2, d_latent=16, nthreads=1)
     on, ln = oracle.mla_decode(q, bits, lens, None, scale=0.2, d_latent=16, nthreads=nthreads)
     assert np.array_equal(o1, on) and np.array_equal(l1, ln)
+
+
+def _paginate(rng, bits, lens, P, extra_pages=3):
+    """Scatters each sequence's rows into pages of P rows at random pool positions; the pool's
+    unused rows hold NaN bit patterns. Returns (pool bits, block table)."""
+    B, L, D = bits.shape
+    per_seq = [(int(n) + P - 1) // P for n in lens]
+    n_pages = sum(per_seq) + extra_pages
+    perm = rng.permutation(n_pages)
+    pool = np.full((n_pages, P, D), 0x7FC0, np.uint16)
+    bt = np.full((B, max(max(per_seq), 1) + 1), -1, np.int32)
+    k = 0
+    for b in range(B):
+        for j in range(per_seq[b]):
+            pg = int(perm[k])
+            k += 1
+            bt[b, j] = pg
+            rows = bits[b, j * P:min((j + 1) * P, int(lens[b]))]
+            pool[pg, :rows.shape[0]] = rows
+    return pool, bt
+
+
+def test_paged_equals_contiguous_and_brute_force():
+    """The paged layout only moves rows: with pages scattered through a pool (unused rows NaN),
+    the result equals the contiguous cache's bit for bit, and a scipy softmax over the rows
+    gathered through the block table."""
+    rng = np.random.default_rng(6)
+    H, Dc, Dr, L, P = 3, 16, 8, 23, 4
+    c, bits = _cache(rng, 3, L, Dc + Dr)
+    q = rng.standard_normal((3, H, Dc + Dr))
+    gate = rng.standard_normal((3, H))
+    lens = np.array([23, 0, 9], np.int32)
+    pool, bt = _paginate(rng, bits, lens, P)
+    o_c, l_c = oracle.mla_decode(q, bits, lens, gate, scale=0.4, d_latent=Dc)
+    o_p, l_p = oracle.mla_decode_paged(q, pool, bt, lens, gate, scale=0.4, d_latent=Dc)
+    assert np.array_equal(o_p, o_c) and np.array_equal(l_p, l_c)
+    pool_f = torch.from_numpy(pool.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    for b in (0, 2):
+        rows = np.stack([pool_f[bt[b, t // P], t % P] for t in range(lens[b])])
+        s = 0.4 * q[b] @ rows.T
+        ref = softmax(s, axis=1) @ rows[:, :Dc] * expit(gate[b])[:, None]
+        np.testing.assert_allclose(o_p[b], ref, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(l_p[b], logsumexp(s, axis=1), rtol=1e-13)
+
+
+def test_paged_rejects_bad_block_table():
+    rng = np.random.default_rng(7)
+    c, bits = _cache(rng, 1, 8, 12)
+    q = rng.standard_normal((1, 2, 12))
+    lens = np.array([8], np.int32)
+    pool, bt = _paginate(rng, bits, lens, 4, extra_pages=0)
+    bad = bt.copy()
+    bad[0, 1] = pool.shape[0]
+    with pytest.raises(RuntimeError):
+        oracle.mla_decode_paged(q, pool, bad, lens, None, scale=0.5, d_latent=8)
+    with pytest.raises(RuntimeError):
+        oracle.mla_decode_paged(q, pool, bt[:, :1], lens, None, scale=0.5, d_latent=8)
