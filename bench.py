@@ -9,6 +9,7 @@ A step is one pass of the workload's hot path over one batch of synthetic input:
                               1,000,000 cached tokens per sequence
   kda_decode_b64              one KDA layer: kda_conv_update + kda_decode_step, 64 sequences x 64 heads
   mla_decode_b16              one gated MLA layer, 16 sequences, contexts uniform in [8192, 131072]
+  mla_decode_b16_paged        the same layer with the cache in 64-row pages of a shuffled pool
   kda_prefill_32k             kda_prefill_chunked, 1 x 32768 tokens x 64 heads, chunk 64
 
 Multi-GPU (torchrun, one process per GPU): the path shards by sequence with no exchange, so each
@@ -357,6 +358,38 @@ class MlaDecodeStep(Step):
         return {"mla_latent_decode": b, "step": b}
 
 
+class MlaPagedStep(MlaDecodeStep):
+    """The 16-sequence latent-attention workload with the cache in 64-row pages scattered through
+    a pool (seeded order), through mla_latent_decode_paged."""
+    name = "mla_decode_b16_paged"
+    page_size = 64
+
+    def __init__(self, lad, dev, rank, cfg: wl.MlaDecode | None = None):
+        super().__init__(lad, dev, rank, cfg)
+        self.pool, self.block_table = wl.paginate(self.cache, self.lens, self.page_size, self.cfg.seed)
+        del self.cache
+        torch.cuda.empty_cache()
+        self.dominant = "mla_latent_decode_paged"
+        self.config = dict(self.config, workload=self.name,
+                           paging=f"{self.page_size}-row pages, {self.pool.shape[0]} in a shuffled pool")
+
+    def run(self, timer=None):
+        if timer:
+            timer.begin("mla_latent_decode_paged")
+        self.lad.mla_latent_decode_paged(self.q, self.pool, self.block_table, self.lens, self.gate, o=self.o,
+                                         workspace=self.ws)
+        if timer:
+            timer.end("mla_latent_decode_paged")
+
+    def mla_bytes(self):
+        # the block table adds 4 bytes per page actually read
+        return super().mla_bytes() + 4 * sum(-(-int(n) // self.page_size) for n in self.lens.tolist())
+
+    def algorithmic_bytes(self):
+        b = self.mla_bytes()
+        return {"mla_latent_decode_paged": b, "step": b}
+
+
 class HybridStep(Step):
     name = "hybrid_8layer_1m"
 
@@ -458,6 +491,7 @@ WORKLOADS = {
     "hybrid_8layer_1m": HybridStep,
     "kda_decode_b64": KdaDecodeStep,
     "mla_decode_b16": MlaDecodeStep,
+    "mla_decode_b16_paged": MlaPagedStep,
     "kda_prefill_32k": PrefillStep,
 }
 
@@ -529,7 +563,7 @@ def cpu_oracle_rate(workload: str, budget_s: float = 20.0) -> dict:
     if workload == "kda_decode_b64":
         sec, sample = kda_layer_seconds(64)
         return {"value": 64 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": sample}
-    if workload == "mla_decode_b16":
+    if workload in ("mla_decode_b16", "mla_decode_b16_paged"):
         lens = wl.mla_seq_lens(wl.MlaDecode("mla", B=16, seed=1236)).tolist()
         sec, sample = mla_seconds(16, lens)
         return {"value": 16 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": sample}
@@ -571,7 +605,8 @@ def run_reference(args, rank, world):
 
 
 def _tokens(workload):
-    return {"hybrid_8layer_1m": 8, "kda_decode_b64": 64, "mla_decode_b16": 16, "kda_prefill_32k": 32768}[workload]
+    return {"hybrid_8layer_1m": 8, "kda_decode_b64": 64, "mla_decode_b16": 16, "mla_decode_b16_paged": 16,
+            "kda_prefill_32k": 32768}[workload]
 
 
 def main(argv=None) -> int:
@@ -654,7 +689,8 @@ def main(argv=None) -> int:
     dom_ms = timer.mean_ms(step.dominant)
     achieved = ab[step.dominant] / (dom_ms / 1000.0) / 1e9
     per_type = {}
-    for kname in ("kda_conv_decode_step", "kda_decode_step", "mla_latent_decode", "kda_prefill_chunked"):
+    for kname in ("kda_conv_decode_step", "kda_decode_step", "mla_latent_decode", "mla_latent_decode_paged",
+                  "kda_prefill_chunked"):
         km = timer.mean_ms(kname)
         if km is not None and kname in ab:
             gbs = ab[kname] / (km / 1000.0) / 1e9
@@ -665,8 +701,9 @@ def main(argv=None) -> int:
         per_type["kda_prefill_chunked"]["tflop_s"] = round(step.flops() / (dom_ms / 1000.0) / 1e12, 1)
     if isinstance(step, (MlaDecodeStep, HybridStep)):
         m = step if isinstance(step, MlaDecodeStep) else step.mla
-        km = timer.mean_ms("mla_latent_decode")
-        per_type["mla_latent_decode"]["mma_tflop_s"] = round(m.mla_flops() / (km / 1000.0) / 1e12, 1)
+        kname = m.dominant
+        km = timer.mean_ms(kname)
+        per_type[kname]["mma_tflop_s"] = round(m.mla_flops() / (km / 1000.0) / 1e12, 1)
 
     if rank == 0:
         cb = None

@@ -57,7 +57,9 @@ int lad_version(void);
 /*
  * Reads and clears the device-side error word that bounded waits set (see above), after
  * synchronising `stream`. *code receives 0 when no kernel gave up a wait, else a nonzero tag
- * naming the kernel and the wait. Returns LAD_OK or LAD_ECUDA.
+ * naming the kernel and the wait (0x101-0x104 latent decode, 0x201 chunked prefill), or 0x105
+ * when mla_latent_decode_paged met a block-table entry outside the pool. Returns LAD_OK or
+ * LAD_ECUDA.
  */
 int lad_device_error(void *stream, int *code);
 
@@ -171,7 +173,9 @@ size_t kda_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk
  *   o  *= sigmoid(gate_logits[b][h])        if gate_logits != NULL
  *   lse = log sum_t exp(s_t)                (natural log, before the gate) if lse_out != NULL
  * L == 0 gives o = 0 and lse = -inf. Scores and softmax are fp32; q.c and p.c run on the
- * tensor cores with bf16 operands and fp32 accumulation.
+ * tensor cores with bf16 operands and fp32 accumulation. Rows at or past L are read up to the
+ * next multiple of 32 (and below Lmax) but may hold anything, NaN included: they get exactly
+ * zero weight.
  *
  *   q           bf16 [B][Hq][d_latent + d_rope]
  *   cache       bf16, row t of sequence b at cache + b*cache_seq_stride + t*(d_latent+d_rope)
@@ -189,6 +193,31 @@ int mla_latent_decode(const lad_bf16 *q, const lad_bf16 *cache, long long cache_
 
 /* Workspace bytes mla_latent_decode needs; num_sms == 0 queries the current device. */
 size_t mla_latent_decode_workspace_size(int B, int Hq, int d_latent, int num_sms);
+
+/*
+ * mla_latent_decode_paged — mla_latent_decode over a paged latent cache, the layout serving
+ * engines keep it in ([P2] "How KDA and MLA split the work" and [P1] "How big is the cache per
+ * token, exactly?" define the row and the attention; paging moves rows and changes no
+ * arithmetic). Results equal mla_latent_decode's on the same rows.
+ *
+ *   kv_pages     bf16 [num_pages][page_size][d_latent + d_rope], a pool of pages
+ *   block_table  int32 [B][block_table_stride] device: rows [j*page_size, (j+1)*page_size) of
+ *                sequence b are page block_table[b*block_table_stride + j]; entries past
+ *                ceil(seq_lens[b] / page_size) are not read
+ *   seq_lens     int32 [B] device, each <= block_table_stride * page_size
+ *   q, gate_logits, o, lse_out, scale, flags, workspace: as for mla_latent_decode (the same
+ *                workspace size query)
+ * Supported: page_size a positive multiple of 32 (a 32-row tile never spans two pages);
+ * num_pages * page_size < 2^31; kv_pages 16-byte aligned. Rows of the last page past the length
+ * may hold anything (NaN included): they get exactly zero weight. A needed block-table entry
+ * outside [0, num_pages) (or past the stride) makes its rows read as zeros and sets device
+ * error 0x105 (lad_device_error); the launch itself still returns LAD_OK.
+ */
+int mla_latent_decode_paged(const lad_bf16 *q, const lad_bf16 *kv_pages, int num_pages, int page_size,
+                            const int *block_table, int block_table_stride, const int *seq_lens,
+                            const float *gate_logits, void *o, float *lse_out, int B, int Hq, int d_latent,
+                            int d_rope, float scale, unsigned flags, void *workspace, size_t ws_bytes,
+                            void *stream);
 
 /*
  * mla_latent_decode_noalloc — mla_latent_decode for callers that cannot allocate device memory

@@ -66,6 +66,8 @@ def _load() -> ctypes.CDLL:
         "mla_latent_decode": ([_c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int,
                                _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
         "mla_latent_decode_workspace_size": ([_c_int] * 4, _c_sz),
+        "mla_latent_decode_paged": ([_c_vp, _c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp,
+                                     _c_int, _c_int, _c_int, _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
         "mla_latent_decode_noalloc": ([_c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                                        _c_int, _c_int, _c_f, _c_u, _c_vp], _c_int),
         "mla_latent_decode_noalloc_max_batch": ([], _c_sz),
@@ -297,6 +299,47 @@ def mla_latent_decode(q: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tens
     _check("mla_latent_decode", _L().mla_latent_decode(
         q.data_ptr(), cache.data_ptr(), seq_stride, seq_lens.data_ptr(), _ptr(gate_logits), o.data_ptr(),
         _ptr(lse), B, Hq, d_latent, D - d_latent, Lmax, float(scale), flags, _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o
+
+
+def mla_latent_decode_paged(q: torch.Tensor, kv_pages: torch.Tensor, block_table: torch.Tensor,
+                            seq_lens: torch.Tensor, gate_logits: torch.Tensor | None = None,
+                            o: torch.Tensor | None = None, lse: torch.Tensor | None = None, scale: float = MLA_SCALE,
+                            d_latent: int = 512, out_fp32: bool = False, workspace: torch.Tensor | None = None,
+                            stream=None) -> torch.Tensor:
+    """Gated latent attention over a paged cache: kv_pages [num_pages, page_size, 576] bf16,
+    block_table int32 [B, n] (row t of sequence b is row t % page_size of page
+    block_table[b, t // page_size]), seq_lens int32 [B]. Returns o [B,Hq,d_latent]."""
+    bf = torch.bfloat16
+    _contig(q, "q", bf)
+    _contig(kv_pages, "kv_pages", bf)
+    B, Hq, D = q.shape
+    if kv_pages.dim() != 3 or kv_pages.shape[2] != D:
+        raise ValueError("kv_pages must be [num_pages, page_size, D]")
+    _contig(block_table, "block_table", torch.int32)
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, n]")
+    _contig(seq_lens, "seq_lens", torch.int32)
+    if seq_lens.shape != (B,):
+        raise ValueError("seq_lens must be [B]")
+    if gate_logits is not None:
+        _contig(gate_logits, "gate_logits", torch.float32)
+        if gate_logits.shape != (B, Hq):
+            raise ValueError("gate_logits must be [B,Hq]")
+    odt = torch.float32 if out_fp32 else bf
+    if o is None:
+        o = torch.empty((B, Hq, d_latent), device=q.device, dtype=odt)
+    _contig(o, "o", odt)
+    if lse is not None:
+        _contig(lse, "lse", torch.float32)
+    ws = mla_latent_decode_workspace_size(B, Hq, d_latent, 0)
+    if workspace is None and ws > 0:
+        workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
+    _check("mla_latent_decode_paged", _L().mla_latent_decode_paged(
+        q.data_ptr(), kv_pages.data_ptr(), kv_pages.shape[0], kv_pages.shape[1], block_table.data_ptr(),
+        block_table.shape[1], seq_lens.data_ptr(), _ptr(gate_logits), o.data_ptr(), _ptr(lse), B, Hq, d_latent,
+        D - d_latent, float(scale), FLAG_OUT_FP32 if out_fp32 else 0, _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
     return o
 

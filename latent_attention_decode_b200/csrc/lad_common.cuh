@@ -28,13 +28,14 @@ int device_sm_count();
 // Returned untyped; the caller casts it to the driver signature from <cuda.h>.
 void *tensor_map_encoder_raw();
 
-// Tags stored in the device error word when a bounded wait gives up.
+// Tags stored in the device error word when a bounded wait gives up (and one input check).
 enum DeviceErrorTag : int {
     kErrNone = 0,
     kErrMlaProducer = 0x101,
     kErrMlaMma = 0x102,
     kErrMlaSoftmax = 0x103,
     kErrMlaEpilogue = 0x104,
+    kErrMlaBlockTable = 0x105,  // a paged call met a block-table entry outside the pool (not a wait)
     kErrPrefill = 0x201,
 };
 

@@ -110,10 +110,6 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -304,9 +300,23 @@ struct Partials {
     long long *tile_prefix;  // [B + 1]
 };
 
+// Paged cache: row t of sequence b is row t % page_size of page block_table[b*bt_stride + t/page_size]
+// of a pool of num_pages pages (page_size a multiple of the 32-row tile, so a tile never spans
+// two pages). Unused by the contiguous variant.
+struct PagedCache {
+    const int *block_table;
+    int bt_stride;
+    int page_size;
+    int num_pages;
+    int oob_row;  // the pool map's row extent: a tile starting there reads as zeros
+};
+
+// kPaged: map_cache is 2-D over the page pool ([num_pages * page_size][576]) and each tile's row
+// comes from the block table; otherwise it is 3-D ([B][Lmax][576]).
+template <bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
 mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_constant__ CUtensorMap map_q,
-                 const int *__restrict__ seq_lens, int B, float score_scale_log2, Partials ws) {
+                 const int *__restrict__ seq_lens, int B, float score_scale_log2, Partials ws, PagedCache pc) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -391,6 +401,8 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             int seq, tile0, nt, k = 0;
             uint32_t g = 0;
             bool ok = true;
+            // paged: lane j holds block_table[seq][pg0 + j] (-1 past the table's row)
+            int pg_seq = -1, pg0 = 0, pg_lane = -1;
             while (ok && it.next(seq, tile0, nt)) {
                 if (k > 0 && !wait_bar(bar(kBarQEmpty), (k - 1) & 1, abort_flag, lad::kErrMlaProducer)) {
                     ok = false;
@@ -401,15 +413,38 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     tma_load_2d(sbase + kOffQ + c * kQChunkBytes, &map_q, c * kChunk, seq * kHq, bar(kBarQFull));
                 for (int i = 0; i < nt; ++i, ++g) {
                     const uint32_t s = g % kStages;
+                    int row = (tile0 + i) * kTile;
+                    if constexpr (kPaged) {
+                        // warp-uniform: every lane computes the same page index
+                        const int pi = row / pc.page_size;
+                        if (seq != pg_seq || pi < pg0 || pi >= pg0 + 32) {
+                            pg_seq = seq;
+                            pg0 = pi;
+                            const int j = pg0 + lane;
+                            pg_lane = j < pc.bt_stride ? pc.block_table[static_cast<long long>(seq) * pc.bt_stride + j]
+                                                       : -1;
+                        }
+                        const int page = __shfl_sync(0xffffffffu, pg_lane, pi - pg0);
+                        if (page >= 0 && page < pc.num_pages) {
+                            row = page * pc.page_size + (row - pi * pc.page_size);
+                        } else {
+                            // a row past the pool: TMA fills the tile with zeros; the call reports it
+                            row = pc.oob_row;
+                            if (lane == 0) atomicCAS(&g_mla_error, 0, lad::kErrMlaBlockTable);
+                        }
+                    }
                     if (!wait_bar(bar(kBarEmpty + s), ((g / kStages) & 1) ^ 1, abort_flag, lad::kErrMlaProducer)) {
                         ok = false;
                         break;
                     }
                     mbar_arrive_tx_elect(bar(kBarFull + s), kStageBytes);
                     const uint32_t dst = sbase + kOffStage + s * kStageBytes;
-                    for (int c = 0; c < kNChunk; ++c)
-                        tma_load_3d(dst + c * kTChunkBytes, &map_cache, c * kChunk, (tile0 + i) * kTile, seq,
-                                    bar(kBarFull + s));
+                    for (int c = 0; c < kNChunk; ++c) {
+                        if constexpr (kPaged)
+                            tma_load_2d(dst + c * kTChunkBytes, &map_cache, c * kChunk, row, bar(kBarFull + s));
+                        else
+                            tma_load_3d(dst + c * kTChunkBytes, &map_cache, c * kChunk, row, seq, bar(kBarFull + s));
+                    }
                 }
                 ++k;
             }
@@ -554,6 +589,17 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
 #pragma unroll
                     for (int t = 0; t < kTile; ++t)
                         if (tok0 + t >= len) x[t] = -INFINITY;
+                    // Rows past the length get weight 0, but 0 * (NaN or Inf) would still reach O:
+                    // zero their latent part in the stage (GEMM1 is done with it, GEMM2 waits for
+                    // P_full, which follows the proxy fence below).
+                    const int valid = len - tok0;
+                    uint8_t *stage = smem + kOffStage + (g % kStages) * kStageBytes;
+                    for (int idx = threadIdx.x - 128; idx < (kTile - valid) * 64; idx += 128) {
+                        const int rr = valid + (idx >> 6);
+                        const int c = (idx >> 3) & 7;
+                        *reinterpret_cast<uint4 *>(stage + c * kTChunkBytes + rr * 128 + (idx & 7) * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
                 }
                 // scores stay unscaled; the scale (with log2 e) is folded into the exponent below
                 float tmax = x[0];
@@ -804,6 +850,124 @@ int take_device_error_mla(cudaStream_t s, int *code) {
 }
 }  // namespace lad
 
+namespace {
+
+// Per-device one-time setup of the split kernels' shared-memory limit.
+int set_smem_attributes(const char *name) {
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return lad::set_error(LAD_ECUDA, "%s: %s", name, cudaGetErrorString(e));
+    if (dev < 0 || dev >= 64) return lad::set_error(LAD_EUNSUPPORTED, "%s: device %d", name, dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+        e = cudaFuncSetAttribute(mla_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(mla_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess)
+            return lad::set_error(LAD_ECUDA, "%s: smem attribute: %s", name, cudaGetErrorString(e));
+        done[dev] = true;
+    }
+    return LAD_OK;
+}
+
+// Checks shared by every entry point (B == 0 is handled by the caller after these).
+int check_common(const char *name, int B, int Hq, int d_latent, int d_rope, unsigned flags, float scale) {
+    using lad::set_error;
+    if (B < 0) return set_error(LAD_EINVAL, "%s: negative B", name);
+    if (Hq != kHq || d_latent != kDl || d_rope != kDr)
+        return set_error(LAD_EUNSUPPORTED, "%s: Hq = 64, d_latent = 512, d_rope = 64 only", name);
+    if (flags & ~LAD_FLAG_OUT_FP32) return set_error(LAD_EINVAL, "%s: unknown flags 0x%x", name, flags);
+    if (!(scale > 0.f) || scale == INFINITY) return set_error(LAD_EINVAL, "%s: scale must be positive", name);
+    return LAD_OK;
+}
+
+int check_pointers(const char *name, const void *q, const void *cache, const int *seq_lens, const void *o,
+                   unsigned flags) {
+    using lad::set_error;
+    if (!q || !cache || !seq_lens || !o) return set_error(LAD_EINVAL, "%s: null pointer", name);
+    if (!lad::aligned(q, 16) || !lad::aligned(cache, 16))
+        return set_error(LAD_EUNSUPPORTED, "%s: q and the cache must be 16-byte aligned", name);
+    if (!lad::aligned(o, (flags & LAD_FLAG_OUT_FP32) ? 16 : 8))
+        return set_error(LAD_EUNSUPPORTED, "%s: o misaligned", name);
+    return LAD_OK;
+}
+
+// Tiles of 32 rows x 64 columns (one 128-byte swizzle row each), 128-byte swizzle.
+int encode_cache_map(const char *name, CUtensorMap *map, const lad_bf16 *base, int rank, const cuuint64_t *dims,
+                     const cuuint64_t *strides) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return lad::set_error(LAD_ECUDA, "%s: cuTensorMapEncodeTiled unavailable", name);
+    const cuuint32_t box[3] = {kChunk, kTile, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<lad_bf16 *>(base), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return lad::set_error(LAD_ECUDA, "%s: cache tensor map failed (%d)", name, (int)r);
+    return LAD_OK;
+}
+
+// Contiguous cache [B][Lmax][576] with a sequence stride (elements).
+int encode_contiguous(const char *name, CUtensorMap *map, const lad_bf16 *cache, int B, int Lmax,
+                      long long seq_stride) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(Lmax),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDrow) * 2, static_cast<cuuint64_t>(seq_stride) * 2};
+    return encode_cache_map(name, map, cache, 3, dims, strides);
+}
+
+// Everything after the argument checks: the q map, the split kernel and the combine.
+int run_mla(const char *name, const CUtensorMap &map_cache, bool paged, const PagedCache &pc, const lad_bf16 *q,
+            const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B, float scale, unsigned flags,
+            uint8_t *ws, const WsLayout &wl, int G, void *stream) {
+    using lad::set_error;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return set_error(LAD_ECUDA, "%s: cuTensorMapEncodeTiled unavailable", name);
+    CUtensorMap map_q;
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(B) * kHq};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDrow) * 2};
+        const cuuint32_t box[2] = {kChunk, kHq};
+        const cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<lad_bf16 *>(q), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return set_error(LAD_ECUDA, "%s: q tensor map failed (%d)", name, (int)r);
+    }
+    int rc = set_smem_attributes(name);
+    if (rc != LAD_OK) return rc;
+    // Every slot the combine reads is written earlier in the same call (partials by their CTA's
+    // epilogue, the tile prefix by CTA 0), so nothing left over from a previous call is read.
+    Partials parts{reinterpret_cast<float *>(ws + wl.off_O), reinterpret_cast<float *>(ws + wl.off_m),
+                   reinterpret_cast<float *>(ws + wl.off_l), reinterpret_cast<long long *>(ws + wl.off_prefix)};
+    cudaStream_t s = lad::as_stream(stream);
+    const float score_scale_log2 = scale * 1.4426950408889634f;
+    if (paged)
+        mla_split_kernel<true><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B, score_scale_log2, parts,
+                                                                pc);
+    else
+        mla_split_kernel<false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B, score_scale_log2,
+                                                                 parts, pc);
+    rc = lad::check_launch(name);
+    if (rc != LAD_OK) return rc;
+    const dim3 cgrid(static_cast<unsigned>(B), kHq);
+    if (flags & LAD_FLAG_OUT_FP32)
+        mla_combine_kernel<true><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
+    else
+        mla_combine_kernel<false><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
+    return lad::check_launch(name);
+}
+
+int sm_count_checked(const char *name, int *G) {
+    *G = lad::device_sm_count();
+    if (*G <= 0) return lad::set_error(LAD_ECUDA, "%s: cannot query the SM count", name);
+    if (*G > kMaxSplitCtas) return lad::set_error(LAD_EUNSUPPORTED, "%s: more than %d SMs", name, kMaxSplitCtas);
+    return LAD_OK;
+}
+
+}  // namespace
+
 extern "C" size_t mla_latent_decode_workspace_size(int B, int Hq, int d_latent, int num_sms) {
     if (B < 0 || Hq != kHq || d_latent != kDl) return 0;
     const int G = num_sms > 0 ? num_sms : lad::device_sm_count();
@@ -816,76 +980,65 @@ extern "C" int mla_latent_decode(const lad_bf16 *q, const lad_bf16 *cache, long 
                                  int d_latent, int d_rope, int Lmax, float scale, unsigned flags, void *workspace,
                                  size_t ws_bytes, void *stream) {
     using lad::set_error;
-    if (B < 0 || Lmax < 0) return set_error(LAD_EINVAL, "mla_latent_decode: negative B or Lmax");
-    if (Hq != kHq || d_latent != kDl || d_rope != kDr)
-        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode: Hq = 64, d_latent = 512, d_rope = 64 only");
-    if (flags & ~LAD_FLAG_OUT_FP32) return set_error(LAD_EINVAL, "mla_latent_decode: unknown flags 0x%x", flags);
-    if (!(scale > 0.f) || scale == INFINITY) return set_error(LAD_EINVAL, "mla_latent_decode: scale must be positive");
+    const char *name = "mla_latent_decode";
+    int rc = check_common(name, B, Hq, d_latent, d_rope, flags, scale);
+    if (rc != LAD_OK) return rc;
+    if (Lmax < 0) return set_error(LAD_EINVAL, "%s: negative Lmax", name);
     if (B == 0) return LAD_OK;
-    if (!q || !cache || !seq_lens || !o) return set_error(LAD_EINVAL, "mla_latent_decode: null pointer");
+    rc = check_pointers(name, q, cache, seq_lens, o, flags);
+    if (rc != LAD_OK) return rc;
     if (Lmax == 0) Lmax = 1;  // every length is then 0; the tensor map still needs a non-empty extent
     if (cache_seq_stride < static_cast<long long>(Lmax) * kDrow || cache_seq_stride % 8 != 0)
-        return set_error(LAD_EINVAL, "mla_latent_decode: cache_seq_stride must be >= Lmax*576 and a multiple of 8");
-    if (!lad::aligned(q, 16) || !lad::aligned(cache, 16))
-        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode: q and cache must be 16-byte aligned");
-    const bool f32 = (flags & LAD_FLAG_OUT_FP32) != 0;
-    if (!lad::aligned(o, f32 ? 16 : 8)) return set_error(LAD_EUNSUPPORTED, "mla_latent_decode: o misaligned");
-    const int G = lad::device_sm_count();
-    if (G <= 0) return set_error(LAD_ECUDA, "mla_latent_decode: cannot query the SM count");
-    if (G > kMaxSplitCtas) return set_error(LAD_EUNSUPPORTED, "mla_latent_decode: more than %d SMs", kMaxSplitCtas);
+        return set_error(LAD_EINVAL, "%s: cache_seq_stride must be >= Lmax*576 and a multiple of 8", name);
+    int G = 0;
+    rc = sm_count_checked(name, &G);
+    if (rc != LAD_OK) return rc;
     const WsLayout wl = ws_layout(B, G);
     if (!workspace || ws_bytes < wl.total || !lad::aligned(workspace, 256))
-        return set_error(LAD_EWORKSPACE, "mla_latent_decode: workspace of %zu bytes (256-aligned) required",
-                         wl.total);
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return set_error(LAD_ECUDA, "mla_latent_decode: cuTensorMapEncodeTiled unavailable");
-
-    CUtensorMap map_cache, map_q;
-    {
-        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(Lmax),
-                                    static_cast<cuuint64_t>(B)};
-        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDrow) * 2,
-                                       static_cast<cuuint64_t>(cache_seq_stride) * 2};
-        const cuuint32_t box[3] = {kChunk, kTile, 1};
-        const cuuint32_t estr[3] = {1, 1, 1};
-        CUresult r = enc(&map_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<lad_bf16 *>(cache), dims, strides,
-                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return set_error(LAD_ECUDA, "mla_latent_decode: cache tensor map failed (%d)", (int)r);
-    }
-    {
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(B) * kHq};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDrow) * 2};
-        const cuuint32_t box[2] = {kChunk, kHq};
-        const cuuint32_t estr[2] = {1, 1};
-        CUresult r = enc(&map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<lad_bf16 *>(q), dims, strides, box,
-                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return set_error(LAD_ECUDA, "mla_latent_decode: q tensor map failed (%d)", (int)r);
-    }
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    Partials parts{reinterpret_cast<float *>(ws + wl.off_O), reinterpret_cast<float *>(ws + wl.off_m),
-                   reinterpret_cast<float *>(ws + wl.off_l), reinterpret_cast<long long *>(ws + wl.off_prefix)};
-
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(mla_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    });
-    if (attr_err != cudaSuccess)
-        return set_error(LAD_ECUDA, "mla_latent_decode: smem attribute: %s", cudaGetErrorString(attr_err));
-
-    cudaStream_t s = lad::as_stream(stream);
-    const float score_scale_log2 = scale * 1.4426950408889634f;
-    mla_split_kernel<<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B, score_scale_log2, parts);
-    int rc = lad::check_launch("mla_latent_decode (split)");
+        return set_error(LAD_EWORKSPACE, "%s: workspace of %zu bytes (256-aligned) required", name, wl.total);
+    CUtensorMap map_cache;
+    rc = encode_contiguous(name, &map_cache, cache, B, Lmax, cache_seq_stride);
     if (rc != LAD_OK) return rc;
-    const dim3 cgrid(static_cast<unsigned>(B), kHq);
-    if (f32)
-        mla_combine_kernel<true><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
-    else
-        mla_combine_kernel<false><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
-    return lad::check_launch("mla_latent_decode (combine)");
+    return run_mla(name, map_cache, false, PagedCache{}, q, seq_lens, gate_logits, o, lse_out, B, scale, flags,
+                   static_cast<uint8_t *>(workspace), wl, G, stream);
+}
+
+extern "C" int mla_latent_decode_paged(const lad_bf16 *q, const lad_bf16 *kv_pages, int num_pages, int page_size,
+                                       const int *block_table, int block_table_stride, const int *seq_lens,
+                                       const float *gate_logits, void *o, float *lse_out, int B, int Hq, int d_latent,
+                                       int d_rope, float scale, unsigned flags, void *workspace, size_t ws_bytes,
+                                       void *stream) {
+    using lad::set_error;
+    const char *name = "mla_latent_decode_paged";
+    int rc = check_common(name, B, Hq, d_latent, d_rope, flags, scale);
+    if (rc != LAD_OK) return rc;
+    if (num_pages < 0 || block_table_stride < 0) return set_error(LAD_EINVAL, "%s: negative size", name);
+    if (page_size <= 0 || page_size % kTile != 0)
+        return set_error(LAD_EUNSUPPORTED, "%s: page_size must be a positive multiple of %d", name, kTile);
+    if (static_cast<long long>(num_pages) * page_size > 0x7fffffffLL - page_size)
+        return set_error(LAD_EUNSUPPORTED, "%s: the pool holds more than 2^31 rows", name);
+    if (B == 0) return LAD_OK;
+    rc = check_pointers(name, q, kv_pages, seq_lens, o, flags);
+    if (rc != LAD_OK) return rc;
+    if (!block_table) return set_error(LAD_EINVAL, "%s: null block table", name);
+    int G = 0;
+    rc = sm_count_checked(name, &G);
+    if (rc != LAD_OK) return rc;
+    const WsLayout wl = ws_layout(B, G);
+    if (!workspace || ws_bytes < wl.total || !lad::aligned(workspace, 256))
+        return set_error(LAD_EWORKSPACE, "%s: workspace of %zu bytes (256-aligned) required", name, wl.total);
+    CUtensorMap map_cache;
+    // an empty pool still gets a one-row extent; every tile then reads as zeros
+    const int rows = num_pages > 0 ? num_pages * page_size : 1;
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(rows)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDrow) * 2};
+        rc = encode_cache_map(name, &map_cache, kv_pages, 2, dims, strides);
+        if (rc != LAD_OK) return rc;
+    }
+    const PagedCache pc{block_table, block_table_stride, page_size, num_pages, rows};
+    return run_mla(name, map_cache, true, pc, q, seq_lens, gate_logits, o, lse_out, B, scale, flags,
+                   static_cast<uint8_t *>(workspace), wl, G, stream);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -937,89 +1090,35 @@ extern "C" int mla_latent_decode_noalloc(const lad_bf16 *q, const lad_bf16 *cach
                                          int Hq, int d_latent, int d_rope, int Lmax, float scale, unsigned flags,
                                          void *stream) {
     using lad::set_error;
-    if (B < 0 || Lmax < 0) return set_error(LAD_EINVAL, "mla_latent_decode_noalloc: negative B or Lmax");
-    if (Hq != kHq || d_latent != kDl || d_rope != kDr)
-        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode_noalloc: Hq = 64, d_latent = 512, d_rope = 64 only");
-    if (flags & ~LAD_FLAG_OUT_FP32)
-        return set_error(LAD_EINVAL, "mla_latent_decode_noalloc: unknown flags 0x%x", flags);
-    if (!(scale > 0.f) || scale == INFINITY)
-        return set_error(LAD_EINVAL, "mla_latent_decode_noalloc: scale must be positive");
+    const char *name = "mla_latent_decode_noalloc";
+    int rc = check_common(name, B, Hq, d_latent, d_rope, flags, scale);
+    if (rc != LAD_OK) return rc;
+    if (Lmax < 0) return set_error(LAD_EINVAL, "%s: negative Lmax", name);
     if (B > kNoAllocMaxB)
         return set_error(LAD_EUNSUPPORTED,
-                         "mla_latent_decode_noalloc: B = %d exceeds the built-in scratch limit of %d sequences "
+                         "%s: B = %d exceeds the built-in scratch limit of %d sequences "
                          "(use mla_latent_decode with a workspace)",
-                         B, kNoAllocMaxB);
+                         name, B, kNoAllocMaxB);
     if (B == 0) return LAD_OK;
-    if (!q || !cache || !seq_lens || !o) return set_error(LAD_EINVAL, "mla_latent_decode_noalloc: null pointer");
+    rc = check_pointers(name, q, cache, seq_lens, o, flags);
+    if (rc != LAD_OK) return rc;
     if (Lmax == 0) Lmax = 1;
     if (cache_seq_stride < static_cast<long long>(Lmax) * kDrow || cache_seq_stride % 8 != 0)
-        return set_error(LAD_EINVAL,
-                         "mla_latent_decode_noalloc: cache_seq_stride must be >= Lmax*576 and a multiple of 8");
-    if (!lad::aligned(q, 16) || !lad::aligned(cache, 16))
-        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode_noalloc: q and cache must be 16-byte aligned");
-    const bool f32 = (flags & LAD_FLAG_OUT_FP32) != 0;
-    if (!lad::aligned(o, f32 ? 16 : 8)) return set_error(LAD_EUNSUPPORTED, "mla_latent_decode_noalloc: o misaligned");
+        return set_error(LAD_EINVAL, "%s: cache_seq_stride must be >= Lmax*576 and a multiple of 8", name);
     const int G = lad::device_sm_count();
-    if (G <= 0) return set_error(LAD_ECUDA, "mla_latent_decode_noalloc: cannot query the SM count");
+    if (G <= 0) return set_error(LAD_ECUDA, "%s: cannot query the SM count", name);
     if (G > kNoAllocMaxSms)
-        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode_noalloc: %d SMs exceed the built-in limit of %d", G,
-                         kNoAllocMaxSms);
+        return set_error(LAD_EUNSUPPORTED, "%s: %d SMs exceed the built-in limit of %d", name, G, kNoAllocMaxSms);
     const WsLayout wl = ws_layout(B, G);
     if (wl.total > kNoAllocScratchBytes)
-        return set_error(LAD_EUNSUPPORTED, "mla_latent_decode_noalloc: scratch of %zu bytes exceeds %zu", wl.total,
+        return set_error(LAD_EUNSUPPORTED, "%s: scratch of %zu bytes exceeds %zu", name, wl.total,
                          kNoAllocScratchBytes);
     uint8_t *ws = nullptr;
-    int rc = noalloc_scratch_ptr(&ws);
+    rc = noalloc_scratch_ptr(&ws);
     if (rc != LAD_OK) return rc;
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return set_error(LAD_ECUDA, "mla_latent_decode_noalloc: cuTensorMapEncodeTiled unavailable");
-
-    CUtensorMap map_cache, map_q;
-    {
-        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(Lmax),
-                                    static_cast<cuuint64_t>(B)};
-        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDrow) * 2,
-                                       static_cast<cuuint64_t>(cache_seq_stride) * 2};
-        const cuuint32_t box[3] = {kChunk, kTile, 1};
-        const cuuint32_t estr[3] = {1, 1, 1};
-        CUresult r = enc(&map_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<lad_bf16 *>(cache), dims, strides,
-                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS)
-            return set_error(LAD_ECUDA, "mla_latent_decode_noalloc: cache tensor map failed (%d)", (int)r);
-    }
-    {
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(B) * kHq};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDrow) * 2};
-        const cuuint32_t box[2] = {kChunk, kHq};
-        const cuuint32_t estr[2] = {1, 1};
-        CUresult r = enc(&map_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<lad_bf16 *>(q), dims, strides, box,
-                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS)
-            return set_error(LAD_ECUDA, "mla_latent_decode_noalloc: q tensor map failed (%d)", (int)r);
-    }
-    // Every slot the combine reads is written earlier in the same call (partials by their CTA's
-    // epilogue, the tile prefix by CTA 0), so nothing left over from a previous call is read and
-    // nothing needs clearing.
-    Partials parts{reinterpret_cast<float *>(ws + wl.off_O), reinterpret_cast<float *>(ws + wl.off_m),
-                   reinterpret_cast<float *>(ws + wl.off_l), reinterpret_cast<long long *>(ws + wl.off_prefix)};
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(mla_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    });
-    if (attr_err != cudaSuccess)
-        return set_error(LAD_ECUDA, "mla_latent_decode_noalloc: smem attribute: %s", cudaGetErrorString(attr_err));
-    cudaStream_t s = lad::as_stream(stream);
-    mla_split_kernel<<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B, scale * 1.4426950408889634f,
-                                                     parts);
-    rc = lad::check_launch("mla_latent_decode_noalloc (split)");
+    CUtensorMap map_cache;
+    rc = encode_contiguous(name, &map_cache, cache, B, Lmax, cache_seq_stride);
     if (rc != LAD_OK) return rc;
-    const dim3 cgrid(static_cast<unsigned>(B), kHq);
-    if (f32)
-        mla_combine_kernel<true><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
-    else
-        mla_combine_kernel<false><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
-    return lad::check_launch("mla_latent_decode_noalloc (combine)");
+    return run_mla(name, map_cache, false, PagedCache{}, q, seq_lens, gate_logits, o, lse_out, B, scale, flags, ws,
+                   wl, G, stream);
 }

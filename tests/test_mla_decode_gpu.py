@@ -88,6 +88,20 @@ def test_many_short_sequences(lad, cuda_device):
     assert np.all(np.isneginf(f64(lse)[~fin]))
 
 
+def test_nan_rows_past_length(lad, cuda_device):
+    """Rows past a sequence's length (in its last 32-row tile and beyond) may hold NaN: they get
+    exactly zero weight and must not reach the output."""
+    lens = [45, 64, 1]
+    q, cache, L, gate = _inputs(3, lens, 96, 8, cuda_device)
+    o_ref, lse_ref = _oracle(q, cache, L, gate)
+    for b, n in enumerate(lens):
+        cache[b, n:] = float("nan")
+    o, lse = _run(lad, q, cache, L, gate)
+    assert torch.isfinite(o).all()
+    assert rel_l2(o, o_ref) < TOL_OUT
+    np.testing.assert_allclose(f64(lse), lse_ref, rtol=0, atol=1e-3)
+
+
 def test_padded_cache_stride(lad, cuda_device):
     """The cache is a view into a larger allocation (sequence stride > Lmax rows)."""
     q, big, L, gate = _inputs(3, [50, 64, 10], 128, 5, cuda_device)

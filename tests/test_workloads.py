@@ -42,3 +42,16 @@ def test_large_draws_are_sliced_consistently():
     x = wl.normal_bf16((5, 3, 4), 9, "c")
     y = wl.normal_bf16((5, 3, 4), 9, "c")
     assert torch.equal(x, y) and x.dtype == torch.bfloat16
+
+
+def test_paginate_moves_rows_only():
+    c = wl.normal_bf16((3, 70, 8), 1, "c")
+    lens = torch.tensor([70, 0, 33], dtype=torch.int32)
+    pool, bt = wl.paginate(c, lens, 32, 5, spare_pages=2)
+    assert pool.shape == (3 + 2 + 2, 32, 8) and bt.shape == (3, 3)
+    used = bt[bt >= 0]
+    assert len(set(used.tolist())) == used.numel()   # no page used twice
+    for b in range(3):
+        for t in range(int(lens[b])):
+            assert torch.equal(pool[bt[b, t // 32], t % 32], c[b, t])
+    assert torch.isnan(pool[bt[2, 1], 1:].float()).all()   # past the length

@@ -241,6 +241,36 @@ def mla_inputs(cfg: MlaDecode, device="cpu", lmax: int | None = None) -> dict:
     }
 
 
+def paginate(cache: torch.Tensor, seq_lens: torch.Tensor, page_size: int, seed: int, spare_pages: int = 0):
+    """Moves a contiguous latent cache [B, Lmax, D] into a pool of pages of `page_size` rows placed
+    in a seeded random order, the way a serving engine's allocator scatters them. Rows of a page
+    past its sequence's length, and spare pages, hold NaN. Returns (pool [P, page_size, D],
+    block_table int32 [B, max pages], on the cache's device); unused table entries are -1."""
+    B, _, D = cache.shape
+    lens = [int(x) for x in seq_lens.tolist()]
+    per_seq = [(n + page_size - 1) // page_size for n in lens]
+    n_pages = sum(per_seq) + spare_pages
+    perm = np.random.default_rng(_seed(seed, "pages")).permutation(n_pages)
+    pool = torch.full((n_pages, page_size, D), float("nan"), dtype=cache.dtype, device=cache.device)
+    table = torch.full((B, max(max(per_seq, default=0), 1)), -1, dtype=torch.int32)
+    k = 0
+    for b in range(B):
+        n = per_seq[b]
+        if n == 0:
+            continue
+        pages = torch.from_numpy(perm[k:k + n].astype(np.int64))
+        k += n
+        table[b, :n] = pages.to(torch.int32)
+        rows = cache[b, :lens[b]]
+        full = lens[b] // page_size
+        dev_pages = pages.to(cache.device)
+        if full:
+            pool[dev_pages[:full]] = rows[:full * page_size].reshape(full, page_size, D)
+        if lens[b] > full * page_size:
+            pool[dev_pages[full], :lens[b] - full * page_size] = rows[full * page_size:]
+    return pool, table.to(cache.device)
+
+
 def to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact widening of a (bf16 or fp32) tensor to a float64 numpy array."""
     return t.detach().to("cpu").to(torch.float64).numpy()
