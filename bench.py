@@ -10,6 +10,7 @@ A step is one pass of the workload's hot path over one batch of synthetic input:
   kda_decode_b64              one KDA layer: kda_conv_update + kda_decode_step, 64 sequences x 64 heads
   mla_decode_b16              one gated MLA layer, 16 sequences, contexts uniform in [8192, 131072]
   mla_decode_b16_paged        the same layer with the cache in 64-row pages of a shuffled pool
+  kda_mtp_b64                 kda_decode_multi: 64 sequences x 64 heads, 4 tokens per state pass
   kda_prefill_32k             kda_prefill_chunked, 1 x 32768 tokens x 64 heads, chunk 64
 
 Multi-GPU (torchrun, one process per GPU): the path shards by sequence with no exchange, so each
@@ -299,6 +300,50 @@ class KdaDecodeStep(Step):
                          else _KdaLayer.bytes_decode(B) + _KdaLayer.bytes_conv(B))}
 
 
+class KdaMultiStep(Step):
+    """One KDA layer's multi-token pass: 64 sequences x 64 heads, 4 tokens per sequence (one
+    token plus three drafts, the verify step of multi-token prediction) through
+    kda_decode_multi, the state read once and written once."""
+    name = "kda_mtp_b64"
+
+    def __init__(self, lad, dev, rank, B=64, T=4):
+        cfg = wl.KdaScan("mtp", B=B, H=H, T=T, seed=1240 + 1000 * rank, state_std=0.02)
+        inp = wl.kda_scan_inputs(cfg, dev)
+        self.lad, self.B, self.T = lad, B, T
+        self.q, self.k, self.v = inp["q"], inp["k"], inp["v"]
+        self.alpha, self.beta, self.S = inp["alpha"], inp["beta"], inp["S0"]
+        self.o = torch.empty((B, T, H, D), device=dev, dtype=torch.bfloat16)
+        self.h_in = [t.cpu().pin_memory() for t in (self.q, self.k, self.v, self.alpha, self.beta)]
+        self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.tokens_per_step = B * T
+        self.launches_per_step = 1
+        self.dominant = "kda_decode_multi"
+        self.config = {"workload": self.name, "batch_per_gpu": B, "tokens_per_pass": T, "heads": H,
+                       "head_dim": D, "state": "fp32 128x128 per head, read and written once per pass",
+                       "l2": "inputs larger than L2 (268 MB of state per step)"}
+
+    def run(self, timer=None):
+        if timer:
+            timer.begin("kda_decode_multi")
+        self.lad.kda_decode_multi(self.q, self.k, self.v, self.alpha, self.beta, self.S, o=self.o)
+        if timer:
+            timer.end("kda_decode_multi")
+
+    def run_e2e(self):
+        for d, h in zip((self.q, self.k, self.v, self.alpha, self.beta), self.h_in):
+            d.copy_(h, non_blocking=True)
+        self.run()
+        self.h_o.copy_(self.o, non_blocking=True)
+
+    def e2e_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.h_in), self.h_o.numel() * 2
+
+    def algorithmic_bytes(self):
+        # per (b, h): state read + write; per token q, k, v (bf16), alpha (fp32), beta, o (bf16)
+        b = self.B * H * (2 * D * D * 4 + self.T * (3 * D * 2 + D * 4 + 4 + D * 2))
+        return {"kda_decode_multi": b, "step": b}
+
+
 class MlaDecodeStep(Step):
     name = "mla_decode_b16"
 
@@ -490,6 +535,7 @@ class PrefillStep(Step):
 WORKLOADS = {
     "hybrid_8layer_1m": HybridStep,
     "kda_decode_b64": KdaDecodeStep,
+    "kda_mtp_b64": KdaMultiStep,
     "mla_decode_b16": MlaDecodeStep,
     "mla_decode_b16_paged": MlaPagedStep,
     "kda_prefill_32k": PrefillStep,
@@ -563,6 +609,18 @@ def cpu_oracle_rate(workload: str, budget_s: float = 20.0) -> dict:
     if workload == "kda_decode_b64":
         sec, sample = kda_layer_seconds(64)
         return {"value": 64 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": sample}
+    if workload == "kda_mtp_b64":
+        # the oracle's recurrence over 4 tokens for a subset of sequences, all 64 heads
+        Bs = min(64, max(1, nth))
+        q = rng.standard_normal((Bs, 4, H, D))
+        S = 0.02 * rng.standard_normal((Bs, H, D, D))
+        a = np.full((Bs, 4, H, D), 0.9)
+        b = np.full((Bs, 4, H), 0.5)
+        t0 = time.perf_counter()
+        oracle.kda_recurrent(q, q, q, a, b, S, nthreads=nth)
+        sec = (time.perf_counter() - t0) * 64 / Bs
+        return {"value": 256 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle",
+                "sample": f"{Bs} of 64 sequences x 64 heads x 4 tokens, scaled to 64 sequences"}
     if workload in ("mla_decode_b16", "mla_decode_b16_paged"):
         lens = wl.mla_seq_lens(wl.MlaDecode("mla", B=16, seed=1236)).tolist()
         sec, sample = mla_seconds(16, lens)
@@ -605,8 +663,8 @@ def run_reference(args, rank, world):
 
 
 def _tokens(workload):
-    return {"hybrid_8layer_1m": 8, "kda_decode_b64": 64, "mla_decode_b16": 16, "mla_decode_b16_paged": 16,
-            "kda_prefill_32k": 32768}[workload]
+    return {"hybrid_8layer_1m": 8, "kda_decode_b64": 64, "kda_mtp_b64": 256, "mla_decode_b16": 16,
+            "mla_decode_b16_paged": 16, "kda_prefill_32k": 32768}[workload]
 
 
 def main(argv=None) -> int:
@@ -689,8 +747,8 @@ def main(argv=None) -> int:
     dom_ms = timer.mean_ms(step.dominant)
     achieved = ab[step.dominant] / (dom_ms / 1000.0) / 1e9
     per_type = {}
-    for kname in ("kda_conv_decode_step", "kda_decode_step", "mla_latent_decode", "mla_latent_decode_paged",
-                  "kda_prefill_chunked"):
+    for kname in ("kda_conv_decode_step", "kda_decode_step", "kda_decode_multi", "mla_latent_decode",
+                  "mla_latent_decode_paged", "kda_prefill_chunked"):
         km = timer.mean_ms(kname)
         if km is not None and kname in ab:
             gbs = ab[kname] / (km / 1000.0) / 1e9

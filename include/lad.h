@@ -47,6 +47,7 @@ typedef uint16_t lad_bf16; /* IEEE bfloat16 bit pattern */
 #define LAD_FLAG_SILU (1u << 0)      /* kda_conv_update: apply SiLU to the conv output */
 #define LAD_FLAG_L2NORM_QK (1u << 1) /* KDA calls: L2-normalise q and k per head in fp32 first */
 #define LAD_FLAG_OUT_FP32 (1u << 2)  /* KDA and MLA calls: write o as fp32 instead of bf16 */
+#define LAD_FLAG_KEEP_STATE (1u << 3) /* kda_decode_multi: read S but do not write it back */
 
 /* Description of the calling thread's most recent error ("" if none). */
 const char *lad_last_error(void);
@@ -114,6 +115,33 @@ int kda_conv_update(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 *w, c
 int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, long long qkv_batch_stride,
                     const float *alpha, const float *beta, float *S, void *o, int B, int H, int dk, int dv,
                     float scale, unsigned flags, void *stream);
+
+/*
+ * kda_decode_multi — kda_decode_step for T consecutive tokens per sequence in one pass over the
+ * state (read once, written once): the verification step of multi-token prediction, one token
+ * plus the drafts ([P1] "What does that mean for serving?": the serving recipe runs MTP with 3
+ * speculative tokens; [P2] "What is in the files": one MTP layer serves as the draft head;
+ * [P2] "The serving numbers are not one experiment": acceptance length 2.13-2.61). For
+ * t = 0 .. n_b - 1 the recurrence of
+ * kda_decode_step runs token by token (decay, delta write, readout after the write), so the
+ * result equals n_b calls of kda_decode_step, up to fp32 rounding order.
+ *
+ *   q, k, v   bf16 [B][T][H][dk]   (read)
+ *   alpha     fp32 [B][T][H][dk]; beta fp32 [B][T][H]
+ *   S         fp32 [B][H][dk][dv]  read; written with the state after the n_b tokens unless
+ *             flags & LAD_FLAG_KEEP_STATE
+ *   o         [B][T][H][dv] bf16 (fp32 with LAD_FLAG_OUT_FP32), or NULL for no outputs; only
+ *             positions t < n_b are written
+ *   n_tokens  int32 [B] device, or NULL for n_b = T: sequence b applies its first
+ *             n_b = clamp(n_tokens[b], 0, T) tokens
+ * A verify-then-commit cycle is one call with LAD_FLAG_KEEP_STATE (outputs for all drafts), then
+ * one call with n_tokens = the accepted counts and o = NULL (state committed).
+ * flags: LAD_FLAG_L2NORM_QK, LAD_FLAG_OUT_FP32, LAD_FLAG_KEEP_STATE.
+ * Supported: dk == dv == 128, 0 <= T <= 8; S 16-byte aligned. B, H or T == 0 is a no-op.
+ */
+int kda_decode_multi(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, const float *alpha, const float *beta,
+                     float *S, void *o, const int *n_tokens, int B, int T, int H, int dk, int dv, float scale,
+                     unsigned flags, void *stream);
 
 /*
  * kda_conv_decode_step — kda_conv_update and kda_decode_step of one KDA layer in one launch: the

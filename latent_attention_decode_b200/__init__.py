@@ -29,6 +29,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblad.so")
 FLAG_SILU = 1 << 0
 FLAG_L2NORM_QK = 1 << 1
 FLAG_OUT_FP32 = 1 << 2
+FLAG_KEEP_STATE = 1 << 3
 MLA_SCALE = 1.0 / math.sqrt(192.0)
 
 _c_vp = ctypes.c_void_p
@@ -60,6 +61,8 @@ def _load() -> ctypes.CDLL:
                              _c_int, _c_f, _c_u, _c_vp], _c_int),
         "kda_conv_decode_step": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                                   _c_int, _c_int, _c_f, _c_u, _c_vp], _c_int),
+        "kda_decode_multi": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
+                              _c_int, _c_int, _c_f, _c_u, _c_vp], _c_int),
         "kda_prefill_chunked": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                                  _c_int, _c_int, _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
         "kda_prefill_workspace_size": ([_c_int] * 6, _c_sz),
@@ -197,6 +200,44 @@ def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: to
     _check("kda_decode_step", _L().kda_decode_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), sq, alpha.data_ptr(),
                                                    beta.data_ptr(), S.data_ptr(), o.data_ptr(), B, H, dk, dv,
                                                    float(scale), flags, _stream(stream)))
+    return o
+
+
+def kda_decode_multi(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor,
+                     S: torch.Tensor, o: torch.Tensor | None = None, n_tokens: torch.Tensor | None = None,
+                     scale: float = 1.0, l2norm_qk: bool = False, out_fp32: bool = False, keep_state: bool = False,
+                     want_output: bool = True, stream=None) -> torch.Tensor | None:
+    """T KDA tokens per sequence in one pass over the state: q, k, v [B,T,H,128] bf16, alpha
+    [B,T,H,128] fp32, beta [B,T,H] fp32, S [B,H,128,128] fp32 (updated in place unless keep_state).
+    n_tokens (int32 [B], optional) limits sequence b to its first n_tokens[b] tokens. Returns
+    o [B,T,H,128] (positions past n_tokens[b] untouched), or None when want_output is False."""
+    bf = torch.bfloat16
+    _contig(S, "S", torch.float32)
+    B, H, dk, dv = S.shape
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _contig(t, name, bf)
+    T = q.shape[1] if q.dim() == 4 else -1
+    if q.shape != (B, T, H, dk) or k.shape != q.shape or v.shape != (B, T, H, dv):
+        raise ValueError("q, k, v must be [B,T,H,128]")
+    _contig(alpha, "alpha", torch.float32), _contig(beta, "beta", torch.float32)
+    if alpha.shape != (B, T, H, dk) or beta.shape != (B, T, H):
+        raise ValueError("alpha must be [B,T,H,dk] and beta [B,T,H]")
+    if n_tokens is not None:
+        _contig(n_tokens, "n_tokens", torch.int32)
+        if n_tokens.shape != (B,):
+            raise ValueError("n_tokens must be [B]")
+    odt = torch.float32 if out_fp32 else bf
+    if want_output:
+        if o is None:
+            o = torch.empty((B, T, H, dv), device=S.device, dtype=odt)
+        _contig(o, "o", odt)
+    else:
+        o = None
+    flags = ((FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
+             | (FLAG_KEEP_STATE if keep_state else 0))
+    _check("kda_decode_multi", _L().kda_decode_multi(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), alpha.data_ptr(), beta.data_ptr(), S.data_ptr(), _ptr(o),
+        _ptr(n_tokens), B, T, H, dk, dv, float(scale), flags, _stream(stream)))
     return o
 
 

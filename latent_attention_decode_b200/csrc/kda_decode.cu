@@ -195,6 +195,132 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
     }
 }
 
+// T tokens of the same recurrence per state pass (speculative verification: one token plus the
+// drafts). The state stays in the registers of K2's layout between tokens; each token costs one
+// shared-memory reduction of S'^T k and S'^T q (double-buffered, so one barrier per token).
+constexpr int kMaxMultiTokens = 8;
+
+template <bool kOutF32>
+__global__ void __launch_bounds__(kThreads, 2)
+kda_decode_multi_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
+                        const uint16_t *__restrict__ v, const float *__restrict__ alpha,
+                        const float *__restrict__ beta, float *__restrict__ S, void *__restrict__ o,
+                        const int *__restrict__ n_tokens, int B, int T, int H, float scale, int l2norm,
+                        int write_state) {
+    const int bh = blockIdx.x;
+    const int b = bh / H;
+    const int h = bh - b * H;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+
+    float4 *mine = reinterpret_cast<float4 *>(S + static_cast<size_t>(bh) * kD * kD) +
+                   static_cast<size_t>(warp * kRowsPerWarp) * kVec + lane;
+    float4 s[kRowsPerWarp];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) s[r] = __ldcs(mine + r * kVec);
+
+    __shared__ float sq[kMaxMultiTokens][kD], sk[kMaxMultiTokens][kD], sv[kMaxMultiTokens][kD],
+        sa[kMaxMultiTokens][kD];
+    __shared__ float sb[kMaxMultiTokens], s_rq[kMaxMultiTokens], s_rk[kMaxMultiTokens], s_qk[kMaxMultiTokens];
+    __shared__ float4 red_k[2][kWarps][kVec], red_q[2][kWarps][kVec];
+
+    int n = T;
+    if (n_tokens) n = min(max(n_tokens[b], 0), T);
+
+    // token t of (b, h): inputs at ((b*T + t)*H + h) rows of 128
+    for (int i = threadIdx.x; i < n * kD; i += kThreads) {
+        const int t = i / kD, c = i - t * kD;
+        const size_t row = (static_cast<size_t>(b) * T + t) * H + h;
+        sq[t][c] = bf16_to_f32(q[row * kD + c]);
+        sk[t][c] = bf16_to_f32(k[row * kD + c]);
+        sv[t][c] = bf16_to_f32(v[row * kD + c]);
+        sa[t][c] = alpha[row * kD + c];
+    }
+    if (threadIdx.x < n) sb[threadIdx.x] = beta[(static_cast<size_t>(b) * T + threadIdx.x) * H + h];
+    __syncthreads();
+    // warp t: the norms and q.k of token t
+    if (warp < n) {
+        float qq = 0.f, kk = 0.f, qk = 0.f;
+#pragma unroll
+        for (int i = lane; i < kD; i += 32) {
+            const float a = sq[warp][i], c = sk[warp][i];
+            qq = fmaf(a, a, qq);
+            kk = fmaf(c, c, kk);
+            qk = fmaf(a, c, qk);
+        }
+        qq = warp_sum(qq);
+        kk = warp_sum(kk);
+        qk = warp_sum(qk);
+        float rq = 1.f, rk = 1.f;
+        if (l2norm) {
+            rq = rsqrtf(qq + 1e-6f);
+            rk = rsqrtf(kk + 1e-6f);
+        }
+        if (lane == 0) {
+            s_rq[warp] = rq;
+            s_rk[warp] = rk;
+            s_qk[warp] = qk * rq * rk;
+        }
+    }
+    __syncthreads();
+
+    for (int t = 0; t < n; ++t) {
+        const float rq = s_rq[t], rk = s_rk[t];
+        float4 wk = make_float4(0.f, 0.f, 0.f, 0.f), wq = wk;
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            const int i = warp * kRowsPerWarp + r;
+            const float a = sa[t][i];
+            s[r].x *= a;
+            s[r].y *= a;
+            s[r].z *= a;
+            s[r].w *= a;
+            fma4(wk, sk[t][i] * rk, s[r]);
+            fma4(wq, sq[t][i] * rq, s[r]);
+        }
+        // buffer t&1 was last read before the previous token's barrier, which every warp has passed
+        red_k[t & 1][warp][lane] = wk;
+        red_q[t & 1][warp][lane] = wq;
+        __syncthreads();
+        float4 W = red_k[t & 1][0][lane], Q = red_q[t & 1][0][lane];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) {
+            add4(W, red_k[t & 1][w][lane]);
+            add4(Q, red_q[t & 1][w][lane]);
+        }
+        const float bt = sb[t];
+        const float4 vv = reinterpret_cast<const float4 *>(sv[t])[lane];
+        float4 u;
+        u.x = bt * (vv.x - W.x);
+        u.y = bt * (vv.y - W.y);
+        u.z = bt * (vv.z - W.z);
+        u.w = bt * (vv.w - W.w);
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) fma4(s[r], sk[t][warp * kRowsPerWarp + r] * rk, u);
+        if (o && warp == (t & (kWarps - 1))) {
+            const float qk = s_qk[t];
+            float4 ov;
+            ov.x = scale * fmaf(qk, u.x, Q.x);
+            ov.y = scale * fmaf(qk, u.y, Q.y);
+            ov.z = scale * fmaf(qk, u.z, Q.z);
+            ov.w = scale * fmaf(qk, u.w, Q.w);
+            const size_t orow = (static_cast<size_t>(b) * T + t) * H + h;
+            if constexpr (kOutF32) {
+                reinterpret_cast<float4 *>(static_cast<float *>(o) + orow * kD)[lane] = ov;
+            } else {
+                uint2 pk;
+                pk.x = static_cast<uint32_t>(f32_to_bf16(ov.x)) | (static_cast<uint32_t>(f32_to_bf16(ov.y)) << 16);
+                pk.y = static_cast<uint32_t>(f32_to_bf16(ov.z)) | (static_cast<uint32_t>(f32_to_bf16(ov.w)) << 16);
+                reinterpret_cast<uint2 *>(static_cast<uint16_t *>(o) + orow * kD)[lane] = pk;
+            }
+        }
+    }
+    if (write_state && n > 0) {
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) __stcs(mine + r * kVec, s[r]);
+    }
+}
+
 }  // namespace
 
 extern "C" int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, long long qkv_batch_stride,
@@ -257,4 +383,33 @@ extern "C" int kda_conv_decode_step(const lad_bf16 *x, lad_bf16 *conv_tail, cons
         kda_decode_kernel<false, true><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
             nullptr, nullptr, nullptr, 0, alpha, beta, S, o, H, scale, l2, cv);
     return lad::check_launch("kda_conv_decode_step");
+}
+
+extern "C" int kda_decode_multi(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, const float *alpha,
+                                const float *beta, float *S, void *o, const int *n_tokens, int B, int T, int H, int dk,
+                                int dv, float scale, unsigned flags, void *stream) {
+    using lad::set_error;
+    if (B < 0 || H < 0 || T < 0) return set_error(LAD_EINVAL, "kda_decode_multi: negative B, T or H");
+    if (dk != kD || dv != kD) return set_error(LAD_EUNSUPPORTED, "kda_decode_multi: dk = dv = 128 only");
+    if (T > kMaxMultiTokens)
+        return set_error(LAD_EUNSUPPORTED, "kda_decode_multi: at most %d tokens per call", kMaxMultiTokens);
+    if (flags & ~(LAD_FLAG_OUT_FP32 | LAD_FLAG_L2NORM_QK | LAD_FLAG_KEEP_STATE))
+        return set_error(LAD_EINVAL, "kda_decode_multi: unknown flags 0x%x", flags);
+    if (B == 0 || H == 0 || T == 0) return LAD_OK;
+    if (!q || !k || !v || !alpha || !beta || !S) return set_error(LAD_EINVAL, "kda_decode_multi: null pointer");
+    if (!lad::aligned(S, 16)) return set_error(LAD_EUNSUPPORTED, "kda_decode_multi: S must be 16-byte aligned");
+    const bool f32 = (flags & LAD_FLAG_OUT_FP32) != 0;
+    if (o && !lad::aligned(o, f32 ? 16 : 8)) return set_error(LAD_EUNSUPPORTED, "kda_decode_multi: o misaligned");
+    const long long blocks = static_cast<long long>(B) * H;
+    if (blocks > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "kda_decode_multi: B*H too large");
+    const int l2 = (flags & LAD_FLAG_L2NORM_QK) ? 1 : 0;
+    const int write_state = (flags & LAD_FLAG_KEEP_STATE) ? 0 : 1;
+    cudaStream_t s = lad::as_stream(stream);
+    if (f32)
+        kda_decode_multi_kernel<true><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
+            q, k, v, alpha, beta, S, o, n_tokens, B, T, H, scale, l2, write_state);
+    else
+        kda_decode_multi_kernel<false><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
+            q, k, v, alpha, beta, S, o, n_tokens, B, T, H, scale, l2, write_state);
+    return lad::check_launch("kda_decode_multi");
 }

@@ -25,7 +25,7 @@
 // cached byte crosses HBM once. P (bf16) goes through shared memory.
 //
 // Roles (256 threads): warp 0 issues TMA loads (q once per segment, then a 4-deep ring of
-// 36 KiB cache tiles), warp 1 owns TMEM and issues the MMAs, warps 4-7 run the online softmax
+// 36 KiB cache tiles), warp 1 owns TMEM, warps 1 and 2 issue the MMAs, warps 4-7 run the online softmax
 // (one head per lane, lanes 0-15 of each warp: the M = 64 accumulator occupies rows 16p..16p+15
 // of TMEM sub-partition p), rescale O when a head's running max grows by more than 2^8
 // (lazily, like FlashAttention-4), and write the segment's partial at its end.
