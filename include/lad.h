@@ -137,7 +137,8 @@ int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, lon
  * A verify-then-commit cycle is one call with LAD_FLAG_KEEP_STATE (outputs for all drafts), then
  * one call with n_tokens = the accepted counts and o = NULL (state committed).
  * flags: LAD_FLAG_L2NORM_QK, LAD_FLAG_OUT_FP32, LAD_FLAG_KEEP_STATE.
- * Supported: dk == dv == 128, 0 <= T <= 8; S 16-byte aligned. B, H or T == 0 is a no-op.
+ * Supported: dk == dv == 128, 0 <= T <= 8; S, q, k, v and alpha 16-byte aligned. B, H or T == 0
+ * is a no-op.
  */
 int kda_decode_multi(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, const float *alpha, const float *beta,
                      float *S, void *o, const int *n_tokens, int B, int T, int H, int dk, int dv, float scale,

@@ -13,6 +13,9 @@
 // column sums S'^T k and S'^T q are reduced across the row slices in shared memory. The state
 // is read once and written once: 128 KiB of HBM traffic per head against ~0.5 KiB of inputs,
 // so the kernel is HBM-bound and only needs enough bytes in flight per SM.
+#include <algorithm>
+#include <mutex>
+
 #include "lad_common.cuh"
 
 namespace {
@@ -196,129 +199,232 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
 }
 
 // T tokens of the same recurrence per state pass (speculative verification: one token plus the
-// drafts). The state stays in the registers of K2's layout between tokens; each token costs one
-// shared-memory reduction of S'^T k and S'^T q (double-buffered, so one barrier per token).
+// drafts). Each token adds a dependent chain (decay, column sums S'^T k and S'^T q across the
+// row slices, update) of a few microseconds per head; launched one head per CTA, the CTAs of an
+// SM would load, compute and store in step and leave HBM idle during the chains. So the kernel is
+// persistent (two CTAs per SM walk the heads with a stride of the grid) and prefetches: while
+// head i's tokens run in registers, each thread's cp.async copies bring its slice of head i+1's
+// state into its own slots of shared memory (read back by the same thread only, so no barrier
+// is needed for them), and head i+1's token inputs land by cp.async in the other of two input
+// buffers. Thread layout: warp w owns
+// columns 16w..16w+15 over all 128 rows; lane = (row group lane/4, float4 of columns lane%4) and
+// holds rows 8m + lane/4 (m = 0..15). A warp instruction then reads 8 rows x 64 contiguous bytes,
+// and the column sums S'^T k and S'^T q reduce over the 8 row groups with three shuffles: the
+// warps never wait for one another inside the token loop.
 constexpr int kMaxMultiTokens = 8;
+constexpr int kMultiCtasPerSm = 2;
+constexpr int kPiecesPerToken = 80;  // 16-byte pieces of one token's inputs: q 16, k 16, v 16, alpha 32
+
+// dynamic shared memory: state slots, per-token scalars, raw inputs, per-row factors
+constexpr int kMOffState = 0;                                   // [16 rows][256 threads] float4
+constexpr int kMOffScal = kMOffState + kRowsPerWarp * kThreads * 16;  // beta, 1/|q|, 1/|k|, q.k per token
+constexpr int kMOffBeta = kMOffScal + 4 * kMaxMultiTokens * 4;      // [2 buffers][8] beta
+constexpr int kMOffRaw = kMOffBeta + 2 * kMaxMultiTokens * 4;       // [2 buffers] per token: q,k,v bf16, alpha fp32
+constexpr int kRawTokenBytes = 3 * kD * 2 + kD * 4;                 // 1,280
+__host__ __device__ constexpr int multi_smem_bytes(int T) {
+    return kMOffRaw + 2 * T * kRawTokenBytes + T * kD * 16 + T * kD * 4;  // + per-row {alpha, k, q}, k
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// cp.async of head bh's token inputs (tokens 0..n-1) into one input buffer: piece p of token t
+// (16 bytes: q, k, v 8 bf16 each, alpha 4 fp32) and beta_t. The caller commits.
+__device__ __forceinline__ void prefetch_inputs(uint32_t raw_dst, uint32_t beta_dst, const uint16_t *q,
+                                                const uint16_t *k, const uint16_t *v, const float *alpha,
+                                                const float *beta, int bh, int H, int T, int n) {
+    const int b = bh / H, h = bh - b * H;
+    for (int p = threadIdx.x; p < n * kPiecesPerToken; p += kThreads) {
+        const int t = p / kPiecesPerToken, c = p - t * kPiecesPerToken;
+        const size_t row = ((static_cast<size_t>(b) * T + t) * H + h) * kD;
+        const uint32_t dst = raw_dst + t * kRawTokenBytes + (c < 48 ? (c >> 4) * 256 + (c & 15) * 16 : 768 + (c - 48) * 16);
+        if (c < 48) {
+            const uint16_t *src = c < 16 ? q : (c < 32 ? k : v);
+            cp_async16(dst, src + row + 8 * (c & 15));
+        } else {
+            cp_async16(dst, alpha + row + 4 * (c - 48));
+        }
+    }
+    if (threadIdx.x < n)
+        cp_async4(beta_dst + threadIdx.x * 4, beta + (static_cast<size_t>(b) * T + threadIdx.x) * H + h);
+}
 
 template <bool kOutF32>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kMultiCtasPerSm)
 kda_decode_multi_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
                         const uint16_t *__restrict__ v, const float *__restrict__ alpha,
                         const float *__restrict__ beta, float *__restrict__ S, void *__restrict__ o,
                         const int *__restrict__ n_tokens, int B, int T, int H, float scale, int l2norm,
                         int write_state) {
-    const int bh = blockIdx.x;
-    const int b = bh / H;
-    const int h = bh - b * H;
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int heads = B * H;
+    const uint32_t st_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + kMOffState)) + tid * 16;
+    const float4 *st = reinterpret_cast<const float4 *>(smem + kMOffState) + tid;
+    float *s_rq = reinterpret_cast<float *>(smem + kMOffScal);
+    float *s_rk = s_rq + kMaxMultiTokens, *s_qk = s_rk + kMaxMultiTokens;
+    const uint32_t raw_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + kMOffRaw));
+    const uint32_t beta_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + kMOffBeta));
+    float4 *rowf = reinterpret_cast<float4 *>(smem + kMOffRaw + 2 * T * kRawTokenBytes);  // [t][row]
+    float *rowk = reinterpret_cast<float *>(rowf + T * kD);  // [t][row]: k_i / |k| again, for the update
 
-    float4 *mine = reinterpret_cast<float4 *>(S + static_cast<size_t>(bh) * kD * kD) +
-                   static_cast<size_t>(warp * kRowsPerWarp) * kVec + lane;
-    float4 s[kRowsPerWarp];
+    auto n_of = [&](int bh) { return n_tokens ? min(max(n_tokens[bh / H], 0), T) : T; };
+    const int rsub = lane >> 2;  // row group: rows 8m + rsub
+    const int cq = lane & 3;     // float4 of columns 16*warp + 4*cq
+    // float4 index of (row 8m + rsub, this thread's columns) is m * 8 * kVec + thread_f4
+    const int thread_f4 = rsub * kVec + 4 * warp + cq;
+    auto prefetch_state = [&](int bh) {
+        const float4 *src = reinterpret_cast<const float4 *>(S + static_cast<size_t>(bh) * kD * kD) + thread_f4;
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) s[r] = __ldcs(mine + r * kVec);
+        for (int r = 0; r < kRowsPerWarp; ++r) cp_async16(st_base + r * kThreads * 16, src + r * 8 * kVec);
+        cp_async_commit();
+    };
 
-    __shared__ float sq[kMaxMultiTokens][kD], sk[kMaxMultiTokens][kD], sv[kMaxMultiTokens][kD],
-        sa[kMaxMultiTokens][kD];
-    __shared__ float sb[kMaxMultiTokens], s_rq[kMaxMultiTokens], s_rk[kMaxMultiTokens], s_qk[kMaxMultiTokens];
-    __shared__ float4 red_k[2][kWarps][kVec], red_q[2][kWarps][kVec];
+    int bh = blockIdx.x;
+    if (bh >= heads) return;
+    int n = n_of(bh);
+    prefetch_state(bh);
+    prefetch_inputs(raw_base, beta_base, q, k, v, alpha, beta, bh, H, T, n);
+    cp_async_commit();
 
-    int n = T;
-    if (n_tokens) n = min(max(n_tokens[b], 0), T);
-
-    // token t of (b, h): inputs at ((b*T + t)*H + h) rows of 128
-    for (int i = threadIdx.x; i < n * kD; i += kThreads) {
-        const int t = i / kD, c = i - t * kD;
-        const size_t row = (static_cast<size_t>(b) * T + t) * H + h;
-        sq[t][c] = bf16_to_f32(q[row * kD + c]);
-        sk[t][c] = bf16_to_f32(k[row * kD + c]);
-        sv[t][c] = bf16_to_f32(v[row * kD + c]);
-        sa[t][c] = alpha[row * kD + c];
-    }
-    if (threadIdx.x < n) sb[threadIdx.x] = beta[(static_cast<size_t>(b) * T + threadIdx.x) * H + h];
-    __syncthreads();
-    // warp t: the norms and q.k of token t
-    if (warp < n) {
-        float qq = 0.f, kk = 0.f, qk = 0.f;
-#pragma unroll
-        for (int i = lane; i < kD; i += 32) {
-            const float a = sq[warp][i], c = sk[warp][i];
-            qq = fmaf(a, a, qq);
-            kk = fmaf(c, c, kk);
-            qk = fmaf(a, c, qk);
-        }
-        qq = warp_sum(qq);
-        kk = warp_sum(kk);
-        qk = warp_sum(qk);
-        float rq = 1.f, rk = 1.f;
-        if (l2norm) {
-            rq = rsqrtf(qq + 1e-6f);
-            rk = rsqrtf(kk + 1e-6f);
-        }
-        if (lane == 0) {
-            s_rq[warp] = rq;
-            s_rk[warp] = rk;
-            s_qk[warp] = qk * rq * rk;
-        }
-    }
-    __syncthreads();
-
-    for (int t = 0; t < n; ++t) {
-        const float rq = s_rq[t], rk = s_rk[t];
-        float4 wk = make_float4(0.f, 0.f, 0.f, 0.f), wq = wk;
-#pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) {
-            const int i = warp * kRowsPerWarp + r;
-            const float a = sa[t][i];
-            s[r].x *= a;
-            s[r].y *= a;
-            s[r].z *= a;
-            s[r].w *= a;
-            fma4(wk, sk[t][i] * rk, s[r]);
-            fma4(wq, sq[t][i] * rq, s[r]);
-        }
-        // buffer t&1 was last read before the previous token's barrier, which every warp has passed
-        red_k[t & 1][warp][lane] = wk;
-        red_q[t & 1][warp][lane] = wq;
+    for (int it = 0; bh < heads; ++it) {
+        const int b = bh / H, h = bh - b * H;
+        const int buf = it & 1;
+        const uint8_t *raw = smem + kMOffRaw + buf * T * kRawTokenBytes;  // token t at t * kRawTokenBytes
+        const float *s_beta = reinterpret_cast<const float *>(smem + kMOffBeta) + buf * kMaxMultiTokens;
+        // 1. this head's state slots and inputs have landed (inputs are read by every thread)
+        cp_async_wait_all();
         __syncthreads();
-        float4 W = red_k[t & 1][0][lane], Q = red_q[t & 1][0][lane];
-#pragma unroll
-        for (int w = 1; w < kWarps; ++w) {
-            add4(W, red_k[t & 1][w][lane]);
-            add4(Q, red_q[t & 1][w][lane]);
-        }
-        const float bt = sb[t];
-        const float4 vv = reinterpret_cast<const float4 *>(sv[t])[lane];
-        float4 u;
-        u.x = bt * (vv.x - W.x);
-        u.y = bt * (vv.y - W.y);
-        u.z = bt * (vv.z - W.z);
-        u.w = bt * (vv.w - W.w);
-#pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) fma4(s[r], sk[t][warp * kRowsPerWarp + r] * rk, u);
-        if (o && warp == (t & (kWarps - 1))) {
-            const float qk = s_qk[t];
-            float4 ov;
-            ov.x = scale * fmaf(qk, u.x, Q.x);
-            ov.y = scale * fmaf(qk, u.y, Q.y);
-            ov.z = scale * fmaf(qk, u.z, Q.z);
-            ov.w = scale * fmaf(qk, u.w, Q.w);
-            const size_t orow = (static_cast<size_t>(b) * T + t) * H + h;
-            if constexpr (kOutF32) {
-                reinterpret_cast<float4 *>(static_cast<float *>(o) + orow * kD)[lane] = ov;
-            } else {
-                uint2 pk;
-                pk.x = static_cast<uint32_t>(f32_to_bf16(ov.x)) | (static_cast<uint32_t>(f32_to_bf16(ov.y)) << 16);
-                pk.y = static_cast<uint32_t>(f32_to_bf16(ov.z)) | (static_cast<uint32_t>(f32_to_bf16(ov.w)) << 16);
-                reinterpret_cast<uint2 *>(static_cast<uint16_t *>(o) + orow * kD)[lane] = pk;
+        // 2. warp t: the norms and q.k of token t
+        if (warp < n) {
+            const uint16_t *tq = reinterpret_cast<const uint16_t *>(raw + warp * kRawTokenBytes);
+            const uint2 xq = reinterpret_cast<const uint2 *>(tq)[lane];
+            const uint2 xk = reinterpret_cast<const uint2 *>(tq + kD)[lane];
+            const float2 q0 = lad::dev::bf16x2_to_f32(xq.x), q1 = lad::dev::bf16x2_to_f32(xq.y);
+            const float2 k0 = lad::dev::bf16x2_to_f32(xk.x), k1 = lad::dev::bf16x2_to_f32(xk.y);
+            float qq = q0.x * q0.x + q0.y * q0.y + q1.x * q1.x + q1.y * q1.y;
+            float kk = k0.x * k0.x + k0.y * k0.y + k1.x * k1.x + k1.y * k1.y;
+            float qk = q0.x * k0.x + q0.y * k0.y + q1.x * k1.x + q1.y * k1.y;
+            qq = warp_sum(qq);
+            kk = warp_sum(kk);
+            qk = warp_sum(qk);
+            float rq = 1.f, rk = 1.f;
+            if (l2norm) {
+                rq = rsqrtf(qq + 1e-6f);
+                rk = rsqrtf(kk + 1e-6f);
+            }
+            if (lane == 0) {
+                s_rq[warp] = rq;
+                s_rk[warp] = rk;
+                s_qk[warp] = qk * rq * rk;
             }
         }
-    }
-    if (write_state && n > 0) {
+        __syncthreads();
+        // 3. per-row factors {alpha_i, k_i / |k|, q_i / |q|} of every token
+        for (int e = tid; e < n * kD; e += kThreads) {
+            const int t = e >> 7, i = e & (kD - 1);
+            const uint16_t *tq = reinterpret_cast<const uint16_t *>(raw + t * kRawTokenBytes);
+            const float a = reinterpret_cast<const float *>(raw + t * kRawTokenBytes + 768)[i];
+            const float kn = bf16_to_f32(tq[kD + i]) * s_rk[t];
+            rowf[e] = make_float4(a, kn, bf16_to_f32(tq[i]) * s_rq[t], 0.f);
+            rowk[e] = kn;
+        }
+        // 4. this head's state: this thread's own slots
+        float4 s[kRowsPerWarp];
 #pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) __stcs(mine + r * kVec, s[r]);
+        for (int r = 0; r < kRowsPerWarp; ++r) s[r] = st[r * kThreads];
+        __syncthreads();
+        // 5. prefetch the next head: state into the same slots, inputs into the other buffer (its
+        //    last readers finished before the barrier at the end of the previous iteration)
+        const int nbh = bh + gridDim.x;
+        int nn = 0;
+        if (nbh < heads) {
+            nn = n_of(nbh);
+            prefetch_state(nbh);
+            prefetch_inputs(raw_base + (buf ^ 1) * T * kRawTokenBytes, beta_base + (buf ^ 1) * kMaxMultiTokens * 4, q,
+                            k, v, alpha, beta, nbh, H, T, nn);
+            cp_async_commit();
+        }
+        // 6. the tokens
+        for (int t = 0; t < n; ++t) {
+            const float4 *rf = rowf + t * kD + rsub;
+            float4 wk = make_float4(0.f, 0.f, 0.f, 0.f), wq = wk;
+            // two halves with a compiler fence between them, so that at most eight row-factor
+            // loads are hoisted at a time (all sixteen would not fit next to the state)
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                for (int mm = 0; mm < kRowsPerWarp / 2; ++mm) {
+                    const int m = half * (kRowsPerWarp / 2) + mm;
+                    const float4 f = rf[8 * m];
+                    s[m].x *= f.x;
+                    s[m].y *= f.x;
+                    s[m].z *= f.x;
+                    s[m].w *= f.x;
+                    fma4(wk, f.y, s[m]);
+                    fma4(wq, f.z, s[m]);
+                }
+                asm volatile("" ::: "memory");
+            }
+#pragma unroll
+            for (int x = 4; x < 32; x <<= 1) {
+                wk.x += __shfl_xor_sync(0xffffffffu, wk.x, x);
+                wk.y += __shfl_xor_sync(0xffffffffu, wk.y, x);
+                wk.z += __shfl_xor_sync(0xffffffffu, wk.z, x);
+                wk.w += __shfl_xor_sync(0xffffffffu, wk.w, x);
+                wq.x += __shfl_xor_sync(0xffffffffu, wq.x, x);
+                wq.y += __shfl_xor_sync(0xffffffffu, wq.y, x);
+                wq.z += __shfl_xor_sync(0xffffffffu, wq.z, x);
+                wq.w += __shfl_xor_sync(0xffffffffu, wq.w, x);
+            }
+            const float bt = s_beta[t];
+            const uint2 xv = reinterpret_cast<const uint2 *>(raw + t * kRawTokenBytes + 512)[4 * warp + cq];
+            const float2 v0 = lad::dev::bf16x2_to_f32(xv.x), v1 = lad::dev::bf16x2_to_f32(xv.y);
+            float4 u;
+            u.x = bt * (v0.x - wk.x);
+            u.y = bt * (v0.y - wk.y);
+            u.z = bt * (v1.x - wk.z);
+            u.w = bt * (v1.y - wk.w);
+#pragma unroll
+            for (int m = 0; m < kRowsPerWarp; ++m) fma4(s[m], rowk[t * kD + 8 * m + rsub], u);
+            if (o && rsub == 0) {
+                const float qk = s_qk[t];
+                float4 ov;
+                ov.x = scale * fmaf(qk, u.x, wq.x);
+                ov.y = scale * fmaf(qk, u.y, wq.y);
+                ov.z = scale * fmaf(qk, u.z, wq.z);
+                ov.w = scale * fmaf(qk, u.w, wq.w);
+                const size_t orow = ((static_cast<size_t>(b) * T + t) * H + h) * kD;
+                if constexpr (kOutF32) {
+                    reinterpret_cast<float4 *>(static_cast<float *>(o) + orow)[4 * warp + cq] = ov;
+                } else {
+                    uint2 pk;
+                    pk.x = static_cast<uint32_t>(f32_to_bf16(ov.x)) | (static_cast<uint32_t>(f32_to_bf16(ov.y)) << 16);
+                    pk.y = static_cast<uint32_t>(f32_to_bf16(ov.z)) | (static_cast<uint32_t>(f32_to_bf16(ov.w)) << 16);
+                    reinterpret_cast<uint2 *>(static_cast<uint16_t *>(o) + orow)[4 * warp + cq] = pk;
+                }
+            }
+        }
+        // 7. the new state
+        if (write_state && n > 0) {
+            float4 *dst = reinterpret_cast<float4 *>(S + static_cast<size_t>(bh) * kD * kD) + thread_f4;
+#pragma unroll
+            for (int r = 0; r < kRowsPerWarp; ++r) __stcs(dst + r * 8 * kVec, s[r]);
+        }
+        // raw, rowf and the scalars are rewritten next iteration: every thread must be done
+        __syncthreads();
+        bh = nbh;
+        n = nn;
     }
+    cp_async_wait_all();
 }
 
 }  // namespace
@@ -397,19 +503,44 @@ extern "C" int kda_decode_multi(const lad_bf16 *q, const lad_bf16 *k, const lad_
         return set_error(LAD_EINVAL, "kda_decode_multi: unknown flags 0x%x", flags);
     if (B == 0 || H == 0 || T == 0) return LAD_OK;
     if (!q || !k || !v || !alpha || !beta || !S) return set_error(LAD_EINVAL, "kda_decode_multi: null pointer");
-    if (!lad::aligned(S, 16)) return set_error(LAD_EUNSUPPORTED, "kda_decode_multi: S must be 16-byte aligned");
+    if (!lad::aligned(S, 16) || !lad::aligned(q, 16) || !lad::aligned(k, 16) || !lad::aligned(v, 16) ||
+        !lad::aligned(alpha, 16))
+        return set_error(LAD_EUNSUPPORTED, "kda_decode_multi: S, q, k, v and alpha must be 16-byte aligned");
     const bool f32 = (flags & LAD_FLAG_OUT_FP32) != 0;
     if (o && !lad::aligned(o, f32 ? 16 : 8)) return set_error(LAD_EUNSUPPORTED, "kda_decode_multi: o misaligned");
-    const long long blocks = static_cast<long long>(B) * H;
-    if (blocks > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "kda_decode_multi: B*H too large");
+    const long long heads = static_cast<long long>(B) * H;
+    if (heads > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "kda_decode_multi: B*H too large");
+    const int sms = lad::device_sm_count();
+    if (sms <= 0) return set_error(LAD_ECUDA, "kda_decode_multi: cannot query the SM count");
+    const int grid = static_cast<int>(std::min<long long>(heads, static_cast<long long>(kMultiCtasPerSm) * sms));
+    const int smem = multi_smem_bytes(T);
+    {
+        static std::mutex mu;
+        static bool done[64] = {};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess || dev < 0 || dev >= 64)
+            return set_error(LAD_ECUDA, "kda_decode_multi: cudaGetDevice: %s", cudaGetErrorString(e));
+        std::lock_guard<std::mutex> lock(mu);
+        if (!done[dev]) {
+            const int mx = multi_smem_bytes(kMaxMultiTokens);
+            e = cudaFuncSetAttribute(kda_decode_multi_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kda_decode_multi_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         mx);
+            if (e != cudaSuccess)
+                return set_error(LAD_ECUDA, "kda_decode_multi: smem attribute: %s", cudaGetErrorString(e));
+            done[dev] = true;
+        }
+    }
     const int l2 = (flags & LAD_FLAG_L2NORM_QK) ? 1 : 0;
     const int write_state = (flags & LAD_FLAG_KEEP_STATE) ? 0 : 1;
     cudaStream_t s = lad::as_stream(stream);
     if (f32)
-        kda_decode_multi_kernel<true><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
-            q, k, v, alpha, beta, S, o, n_tokens, B, T, H, scale, l2, write_state);
+        kda_decode_multi_kernel<true><<<grid, kThreads, smem, s>>>(q, k, v, alpha, beta, S, o, n_tokens, B, T, H,
+                                                                   scale, l2, write_state);
     else
-        kda_decode_multi_kernel<false><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
-            q, k, v, alpha, beta, S, o, n_tokens, B, T, H, scale, l2, write_state);
+        kda_decode_multi_kernel<false><<<grid, kThreads, smem, s>>>(q, k, v, alpha, beta, S, o, n_tokens, B, T, H,
+                                                                    scale, l2, write_state);
     return lad::check_launch("kda_decode_multi");
 }

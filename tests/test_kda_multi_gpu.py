@@ -53,14 +53,15 @@ def test_tokens_per_pass(lad, cuda_device, T, alpha_mode):
 
 
 def test_one_token_equals_decode_step(lad, cuda_device):
-    """T = 1 runs the same fp32 arithmetic in the same order as kda_decode_step."""
+    """T = 1 is kda_decode_step up to the fp32 summation order of the column sums."""
     cfg = wl.KdaScan("one", B=4, H=6, T=1, seed=50, state_std=0.02, alpha_mode="uniform")
     d = _dev(wl.kda_scan_inputs(cfg), cuda_device)
     S1, S2 = d["S0"].clone(), d["S0"].clone()
     o1 = _call(lad, d, S1, out_fp32=True)
     o2 = lad.kda_decode_step(d["q"][:, 0].contiguous(), d["k"][:, 0].contiguous(), d["v"][:, 0].contiguous(),
                              d["alpha"][:, 0].contiguous(), d["beta"][:, 0].contiguous(), S2, out_fp32=True)
-    assert torch.equal(o1[:, 0], o2) and torch.equal(S1, S2)
+    assert rel_l2(o1[:, 0], o2) < 1e-6
+    assert rel_l2(S1, S2) < 1e-6
 
 
 def test_l2norm_flag(lad, cuda_device):
