@@ -582,13 +582,22 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                 if (lane == 0) mbar_arrive(bar(kBarSEmpty + sb));
 
                 const int tok0 = (tile0 + i) * kTile;
-                float x[kTile];
+                // the 32 scores of head 16p + (lane % 16) are split over lanes l and l + 16: lane l
+                // keeps tokens 0-15 (it loaded the row), lane l + 16 receives tokens 16-31
+                const int hi = lane >> 4;
+                float xs[kTile / 2];
 #pragma unroll
-                for (int t = 0; t < kTile; ++t) x[t] = __uint_as_float(r[t]) + __uint_as_float(r2[t]);
+                for (int j = 0; j < kTile / 2; ++j) {
+                    const float a = __uint_as_float(r[j]) + __uint_as_float(r2[j]);
+                    const float b = __uint_as_float(r[16 + j]) + __uint_as_float(r2[16 + j]);
+                    const float from_low = __shfl_sync(0xffffffffu, b, lane & 15);
+                    xs[j] = hi ? from_low : a;
+                }
+                const int mytok0 = tok0 + 16 * hi;
                 if (tok0 + kTile > len) {
 #pragma unroll
-                    for (int t = 0; t < kTile; ++t)
-                        if (tok0 + t >= len) x[t] = -INFINITY;
+                    for (int j = 0; j < kTile / 2; ++j)
+                        if (mytok0 + j >= len) xs[j] = -INFINITY;
                     // Rows past the length get weight 0, but 0 * (NaN or Inf) would still reach O:
                     // zero their latent part in the stage (GEMM1 is done with it, GEMM2 waits for
                     // P_full, which follows the proxy fence below).
@@ -602,9 +611,13 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     }
                 }
                 // scores stay unscaled; the scale (with log2 e) is folded into the exponent below
-                float tmax = x[0];
+                float t8[8];
 #pragma unroll
-                for (int t = 1; t < kTile; ++t) tmax = fmaxf(tmax, x[t]);
+                for (int j = 0; j < 8; ++j) t8[j] = fmaxf(xs[j], xs[j + 8]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) t8[j] = fmaxf(t8[j], t8[j + 4]);
+                float tmax = fmaxf(fmaxf(t8[0], t8[2]), fmaxf(t8[1], t8[3]));
+                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
                 tmax *= score_scale_log2;
                 if (i == 0) {
                     m = -INFINITY;
@@ -620,15 +633,17 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     m = tmax;
                     need = true;
                 }
-                uint32_t pk[kTile / 2];
-                float psum = 0.f;
+                uint32_t pk[kTile / 4];
+                float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int t = 0; t < kTile; t += 2) {
-                    const float p0 = ex2(fmaf(x[t], score_scale_log2, -m));
-                    const float p1 = ex2(fmaf(x[t + 1], score_scale_log2, -m));
-                    psum += p0 + p1;  // the denominator keeps fp32 probabilities
-                    pk[t / 2] = lad::dev::f32x2_to_bf16x2(p0, p1);
+                for (int j = 0; j < kTile / 2; j += 2) {
+                    const float p0 = ex2(fmaf(xs[j], score_scale_log2, -m));
+                    const float p1 = ex2(fmaf(xs[j + 1], score_scale_log2, -m));
+                    ps[(j >> 1) & 3] += p0 + p1;  // the denominator keeps fp32 probabilities
+                    pk[j / 2] = lad::dev::f32x2_to_bf16x2(p0, p1);
                 }
+                float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                psum += __shfl_xor_sync(0xffffffffu, psum, 16);
                 l = l * f + psum;
 
                 const uint32_t pb = g & 1;
@@ -637,15 +652,15 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     break;
                 }
                 const uint32_t rb = g & 1;
-                if (owner) {
-                    // P[h][t], K-major without swizzle: 8x8 core matrices of 128 bytes;
-                    // head group h/8 at 512 B, token group t/8 at 128 B, row h%8 at 16 B.
-                    uint8_t *prow = smem + kOffP + pb * kPBytes + (h >> 3) * 512 + (h & 7) * 16;
-#pragma unroll
-                    for (int j = 0; j < kTile / 8; ++j)
-                        *reinterpret_cast<uint4 *>(prow + j * 128) =
-                            make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-                    rescale[rb * 64 + h] = f;
+                {
+                    // P[h][t], K-major without swizzle: 8x8 core matrices of 128 bytes; head group
+                    // h/8 at 512 B, token group t/8 at 128 B, row h%8 at 16 B. This lane's 16 tokens
+                    // are token groups 2*hi and 2*hi + 1.
+                    const int hh = 16 * p + (lane & 15);
+                    uint8_t *prow = smem + kOffP + pb * kPBytes + (hh >> 3) * 512 + (hh & 7) * 16 + 2 * hi * 128;
+                    *reinterpret_cast<uint4 *>(prow) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4 *>(prow + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    if (owner) rescale[rb * 64 + h] = f;
                 }
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 const int any = __any_sync(0xffffffffu, owner && need);
