@@ -25,7 +25,7 @@
 // cached byte crosses HBM once. P (bf16) goes through shared memory.
 //
 // Roles (256 threads): warp 0 issues TMA loads (q once per segment, then a 4-deep ring of
-// 36 KiB cache tiles), warp 1 owns TMEM, warps 1 and 2 issue the MMAs, warps 4-7 run the online softmax
+// 36 KiB cache tiles), warp 1 owns TMEM, warps 1 and 2 issue GEMM1, warp 3 GEMM2, warps 4-7 run the online softmax
 // (one head per lane, lanes 0-15 of each warp: the M = 64 accumulator occupies rows 16p..16p+15
 // of TMEM sub-partition p), rescale O when a head's running max grows by more than 2^8
 // (lazily, like FlashAttention-4), and write the segment's partial at its end.
@@ -370,9 +370,9 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             if (i == kBarSEmpty || i == kBarSEmpty + 1 || i == kBarPFull || i == kBarPFull + 1 || i == kBarWg ||
                 i == kBarWg + 1 || i == kBarOFree)
                 count = 4;  // one arrival per softmax warp
-            if ((i >= kBarEmpty && i < kBarEmpty + kStages) || i == kBarSFull || i == kBarSFull + 1 ||
-                i == kBarPEmpty || i == kBarPEmpty + 1 || i == kBarQEmpty || i == kBarDrain)
-                count = 2;  // one commit per MMA warp
+            if (i == kBarSFull || i == kBarSFull + 1 || i == kBarQEmpty)
+                count = 2;  // one commit per GEMM1 warp
+            if (i == kBarDrain) count = 3;  // every MMA warp
             mbar_init(bar(i), count);
         }
         *abort_flag = 0;
@@ -466,11 +466,10 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             }
         }
     } else if (warp == 1 || warp == 2) {
-        // ================= MMA issuers (warps 1 and 2, whole warps, elected lanes issue) =================
+        // ================= GEMM1 issuers (warps 1 and 2, whole warps, elected lanes issue) =================
         // A single warp issues a small tcgen05.mma only every ~28 cycles, below the tensor pipe's
-        // rate for these shapes, so two warps share the work: warp 1 issues GEMM1's even K-chunks
-        // and GEMM2's latent blocks 0-1, warp 2 the odd K-chunks and blocks 2-3. Each keeps its own
-        // accumulators, and every barrier an MMA completion arrives on expects both warps' commits.
+        // rate for these shapes, so two warps share GEMM1: warp 1 issues the even K chunks into one
+        // partial accumulator, warp 2 the odd ones into the other; S_full expects both commits.
         {
             const int mi = warp - 1;
             int seq, tile0, nt, k = 0;
@@ -478,39 +477,6 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             bool ok = true;
             const uint64_t q_desc0 = smem_desc(sbase + kOffQ, 16, 1024, kLayoutSw128);
             const uint64_t c_desc0 = smem_desc(sbase + kOffStage, 16, 1024, kLayoutSw128);
-            const uint64_t v_desc0 = smem_desc(sbase + kOffStage, kTChunkBytes, 1024, kLayoutSw128);
-            const uint64_t p_desc0 = smem_desc(sbase + kOffP, 128, 512, kLayoutNone);
-            // the previous tile's GEMM2 is issued after the current tile's GEMM1
-            bool have_prev = false;
-            uint32_t prev_g = 0;
-            bool prev_first = false;
-            int prev_seg = 0;
-            auto gemm2 = [&](uint32_t gg, bool first_of_seg, int seg) -> bool {
-                const uint32_t pb = gg & 1;
-                if (!wait_bar(bar(kBarPFull + pb), (gg >> 1) & 1, abort_flag, lad::kErrMlaMma)) return false;
-                if (first_of_seg && seg > 0 &&
-                    !wait_bar(bar(kBarOFree), (seg - 1) & 1, abort_flag, lad::kErrMlaMma))
-                    return false;
-                tc_fence_after();
-                const uint32_t s = gg % kStages;
-                // A = V^T: 128 latent dims (two 64-wide chunks, LBO apart) x 16 tokens (two 8-row groups)
-                const uint64_t a0 = v_desc0 + ((s * kStageBytes) >> 4);
-                // B = P: 64 heads (8-row core groups, SBO 512) x 16 tokens (two 8-token core columns, LBO 128)
-                const uint64_t b0 = p_desc0 + ((pb * kPBytes) >> 4);
-                const uint32_t acc0 = first_of_seg ? 0u : 1u;
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const int j = 2 * mi + jj;
-                        tc_mma(tmem + kColO + 64 * j, a0 + (((2 * j) * kTChunkBytes + kk * 2048) >> 4),
-                               b0 + ((kk * 256) >> 4), kIdesc2, kk == 0 ? acc0 : 1u);
-                    }
-                }
-                tc_commit(bar(kBarEmpty + s));
-                tc_commit(bar(kBarPEmpty + pb));
-                return true;
-            };
             while (ok && it.next(seq, tile0, nt)) {
                 if (!wait_bar(bar(kBarQFull), k & 1, abort_flag, lad::kErrMlaMma)) {
                     ok = false;
@@ -536,19 +502,55 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     }
                     tc_commit(bar(kBarSFull + sb));
                     if (i == nt - 1) tc_commit(bar(kBarQEmpty));
-                    if (have_prev && !gemm2(prev_g, prev_first, prev_seg)) {
-                        ok = false;
-                        break;
-                    }
-                    have_prev = true;
-                    prev_g = g;
-                    prev_first = (i == 0);
-                    prev_seg = k;
                 }
                 ++k;
             }
-            if (ok && have_prev) ok = gemm2(prev_g, prev_first, prev_seg);
             // drain every MMA this thread issued before TMEM is released
+            tc_commit(bar(kBarDrain));
+            const uint64_t tt = globaltimer_ns();
+            while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer_ns() - tt < kWaitLimitNs) {
+            }
+        }
+    } else if (warp == 3) {
+        // ================= GEMM2 issuer (warp 3, whole warp, elected lane issues) =================
+        // Issued as soon as a tile's P is ready, independently of the next tile's GEMM1, so that the
+        // tile's stage goes back to the TMA warp early: the ring is what keeps bytes in flight.
+        {
+            int seq, tile0, nt, k = 0;
+            uint32_t g = 0;
+            bool ok = true;
+            const uint64_t v_desc0 = smem_desc(sbase + kOffStage, kTChunkBytes, 1024, kLayoutSw128);
+            const uint64_t p_desc0 = smem_desc(sbase + kOffP, 128, 512, kLayoutNone);
+            while (ok && it.next(seq, tile0, nt)) {
+                for (int i = 0; i < nt; ++i, ++g) {
+                    const uint32_t pb = g & 1;
+                    if (!wait_bar(bar(kBarPFull + pb), (g >> 1) & 1, abort_flag, lad::kErrMlaMma)) {
+                        ok = false;
+                        break;
+                    }
+                    if (i == 0 && k > 0 && !wait_bar(bar(kBarOFree), (k - 1) & 1, abort_flag, lad::kErrMlaMma)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t s = g % kStages;
+                    // A = V^T: 128 latent dims (two 64-wide chunks, LBO apart) x 16 tokens (two 8-row groups)
+                    const uint64_t a0 = v_desc0 + ((s * kStageBytes) >> 4);
+                    // B = P: 64 heads (8-row core groups, SBO 512) x 16 tokens (two 8-token core columns, LBO 128)
+                    const uint64_t b0 = p_desc0 + ((pb * kPBytes) >> 4);
+                    const uint32_t acc0 = i == 0 ? 0u : 1u;
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            tc_mma(tmem + kColO + 64 * j, a0 + (((2 * j) * kTChunkBytes + kk * 2048) >> 4),
+                                   b0 + ((kk * 256) >> 4), kIdesc2, kk == 0 ? acc0 : 1u);
+                    }
+                    tc_commit(bar(kBarEmpty + s));
+                    tc_commit(bar(kBarPEmpty + pb));
+                }
+                ++k;
+            }
             tc_commit(bar(kBarDrain));
             const uint64_t tt = globaltimer_ns();
             while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer_ns() - tt < kWaitLimitNs) {
