@@ -64,9 +64,15 @@ def _load():
                                             ctypes.c_double, _dp, _dp, ctypes.c_int])
             lib.lado_mla_decode_paged.argtypes = ([ctypes.c_int] * 7 + [_dp, _up, _ip, _ip, _dp,
                                                   ctypes.c_double, _dp, _dp, ctypes.c_int])
+            lib.lado_rope.argtypes = [ctypes.c_int, ctypes.c_int, _dp, ctypes.POINTER(ctypes.c_longlong),
+                                      ctypes.c_double, ctypes.c_int, _dp]
+            lib.lado_round_bf16.argtypes = [ctypes.c_int, _dp, _up]
+            lib.lado_mla_cache_row.argtypes = [ctypes.c_int] * 3 + [_up, _up, ctypes.POINTER(ctypes.c_longlong),
+                                                                    ctypes.c_double, ctypes.c_int, _up]
             lib.lado_num_threads_available.argtypes = []
             for f in (lib.lado_kda_recurrent, lib.lado_kda_chunked, lib.lado_l2norm,
-                      lib.lado_short_conv_step, lib.lado_mla_decode, lib.lado_mla_decode_paged,
+                      lib.lado_short_conv_step, lib.lado_mla_decode, lib.lado_mla_decode_paged, lib.lado_rope,
+                      lib.lado_round_bf16, lib.lado_mla_cache_row,
                       lib.lado_num_threads_available):
                 f.restype = ctypes.c_int
             _lib = lib
@@ -212,3 +218,44 @@ def mla_decode_paged(q, page_bits, block_table, seq_lens, gate=None, scale: floa
                                        _ptr(o), _ptr(lse), int(nthreads))
     _check(rc, "mla_decode_paged")
     return o, lse
+
+
+def rope(x, positions, theta: float = 6.0e6, interleaved: bool = False):
+    """Rotary embedding of the last axis of x (even width D) by positions (one per row of the
+    leading axes, broadcast over any axes between). Returns float64 of x's shape."""
+    x = _f64(x)
+    D = x.shape[-1]
+    pos = np.asarray(positions, dtype=np.int64)
+    lead = x.shape[:-1]
+    pos = np.broadcast_to(pos.reshape(pos.shape + (1,) * (len(lead) - pos.ndim)), lead)
+    flat = np.ascontiguousarray(x.reshape(-1, D))
+    pflat = np.ascontiguousarray(pos.reshape(-1))
+    out = np.empty_like(flat)
+    rc = _load().lado_rope(flat.shape[0], D, _ptr(flat), pflat.ctypes.data_as(ctypes.POINTER(ctypes.c_longlong)),
+                           float(theta), int(bool(interleaved)), _ptr(out))
+    _check(rc, "rope")
+    return out.reshape(x.shape)
+
+
+def round_bf16_bits(x) -> np.ndarray:
+    """bf16 bit patterns of float64 values, rounded once to nearest, ties to even."""
+    x = np.ascontiguousarray(_f64(x))
+    out = np.empty(x.shape, dtype=np.uint16)
+    _check(_load().lado_round_bf16(x.size, _ptr(x), _ptr(out, _up)), "round_bf16")
+    return out
+
+
+def mla_cache_row(c_kv_bits, k_pe_bits, positions, theta: float = 6.0e6, interleaved: bool = False) -> np.ndarray:
+    """New latent-cache rows (bf16 bits [n, Dc + Dr]): the latent as given, the RoPE key turned
+    to its position and rounded to bf16 once. c_kv_bits [n, Dc], k_pe_bits [n, Dr] uint16."""
+    c = np.ascontiguousarray(c_kv_bits, dtype=np.uint16)
+    k = np.ascontiguousarray(k_pe_bits, dtype=np.uint16)
+    n, Dc = c.shape
+    Dr = k.shape[1]
+    pos = np.ascontiguousarray(positions, dtype=np.int64)
+    out = np.empty((n, Dc + Dr), dtype=np.uint16)
+    rc = _load().lado_mla_cache_row(n, Dc, Dr, _ptr(c, _up), _ptr(k, _up),
+                                    pos.ctypes.data_as(ctypes.POINTER(ctypes.c_longlong)), float(theta),
+                                    int(bool(interleaved)), _ptr(out, _up))
+    _check(rc, "mla_cache_row")
+    return out

@@ -408,3 +408,94 @@ int lado_mla_decode_paged(int B, int H, int Dc, int Dr, int P, int num_pages, in
     return mla_decode_impl(B, H, Dc, Dr, q, pages, 0, block_table, bt_stride, P, seq_lens, gate, scale, o, lse,
                            nthreads);
 }
+
+/*
+ * Rotary position embedding of the 64-wide RoPE part of a latent-attention query or key ([P2]
+ * "Context: 1M in the claims, 262,144 in the config": position enters the model only in the MLA
+ * layers, through 64 of each head's 192 query-key dimensions; rope_theta = 6,000,000 with no
+ * scaling). The pages do not say how dimensions pair up; the two usual pairings are offered:
+ *   interleaved == 0 (rotate-half): pair i is (x[i], x[i + D/2]), i < D/2
+ *   interleaved == 1:               pair i is (x[2i], x[2i + 1])
+ * Pair i turns by the angle p * theta^(-2i/D):  (a, b) -> (a cos - b sin, b cos + a sin).
+ * x, out: [n][D] (out may alias x); positions: [n]; D even.
+ */
+int lado_rope(int n, int D, const double *x, const long long *positions, double theta, int interleaved,
+              double *out) {
+    if (n < 0 || D <= 0 || (D & 1) || !(theta > 0.0)) return LADO_EINVAL;
+    const int half = D / 2;
+    for (int r = 0; r < n; ++r) {
+        const double *xr = x + (size_t)r * D;
+        double *yr = out + (size_t)r * D;
+        double tmp[1024];
+        if (D > 1024) return LADO_EINVAL;
+        for (int d = 0; d < D; ++d) tmp[d] = xr[d];
+        for (int i = 0; i < half; ++i) {
+            const double ang = (double)positions[r] * pow(theta, -2.0 * i / D);
+            const double c = cos(ang), sn = sin(ang);
+            const int ia = interleaved ? 2 * i : i;
+            const int ib = interleaved ? 2 * i + 1 : i + half;
+            const double a = tmp[ia], b = tmp[ib];
+            yr[ia] = a * c - b * sn;
+            yr[ib] = b * c + a * sn;
+        }
+    }
+    return LADO_OK;
+}
+
+/* IEEE binary64 -> bfloat16 bit pattern, rounded once, to nearest with ties to even: the two
+ * bf16 neighbours of |v| are multiples of the spacing 2^(e-8) of 8-bit significands in v's binade
+ * (2^-133 below the normal range); the nearer one wins, a tie goes to the even significand. */
+static uint16_t double_to_bf16_bits(double v) {
+    if (v != v) return 0x7FC0u;
+    const uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    const double a = fabs(v);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80u);
+    int e;
+    frexp(a, &e); /* a = m * 2^e, m in [0.5, 1) */
+    int q = e - 8;
+    if (q < -133) q = -133;
+    const double ulp = ldexp(1.0, q);
+    const double lo = floor(a / ulp) * ulp, hi = lo + ulp;
+    const double dlo = a - lo, dhi = hi - a;
+    double r;
+    if (dlo < dhi)
+        r = lo;
+    else if (dhi < dlo)
+        r = hi;
+    else
+        r = (fmod(lo / ulp, 2.0) == 0.0) ? lo : hi;
+    if (r >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7F80u);
+    const float f = (float)r; /* exact: r has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(sign | (u >> 16));
+}
+
+/* For tests: the bf16 rounding above, applied to n values. */
+int lado_round_bf16(int n, const double *x, uint16_t *out) {
+    if (n < 0) return LADO_EINVAL;
+    for (int i = 0; i < n; ++i) out[i] = double_to_bf16_bits(x[i]);
+    return LADO_OK;
+}
+
+/*
+ * A new latent-cache row for each of n tokens ([P1] "How big is the cache per token, exactly?":
+ * the row is the 512-wide compressed latent followed by the 64-wide RoPE key, in bf16): the latent
+ * is stored as given, the RoPE key is turned to its position (lado_rope, fp64) and rounded to
+ * bf16 once. c_kv: [n][Dc] bf16 bits; k_pe: [n][Dr] bf16 bits; out: [n][Dc + Dr] bf16 bits.
+ */
+int lado_mla_cache_row(int n, int Dc, int Dr, const uint16_t *c_kv, const uint16_t *k_pe, const long long *positions,
+                       double theta, int interleaved, uint16_t *out) {
+    if (n < 0 || Dc < 0 || Dr <= 0 || Dr > 1024 || (Dr & 1)) return LADO_EINVAL;
+    double x[1024], y[1024];
+    for (int r = 0; r < n; ++r) {
+        uint16_t *o = out + (size_t)r * (Dc + Dr);
+        memcpy(o, c_kv + (size_t)r * Dc, sizeof(uint16_t) * (size_t)Dc);
+        for (int d = 0; d < Dr; ++d) x[d] = bf16_bits_to_double(k_pe[(size_t)r * Dr + d]);
+        const int rc = lado_rope(1, Dr, x, positions + r, theta, interleaved, y);
+        if (rc != LADO_OK) return rc;
+        for (int d = 0; d < Dr; ++d) o[Dc + d] = double_to_bf16_bits(y[d]);
+    }
+    return LADO_OK;
+}
