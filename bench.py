@@ -10,6 +10,7 @@ A step is one pass of the workload's hot path over one batch of synthetic input:
   kda_decode_b64              one KDA layer: kda_conv_update + kda_decode_step, 64 sequences x 64 heads
   mla_decode_b16              one gated MLA layer, 16 sequences, contexts uniform in [8192, 131072]
   mla_decode_b16_paged        the same layer with the cache in 64-row pages of a shuffled pool
+  mla_decode_b16_paged_rope   the paged layer with RoPE in the kernels: append the new rows, then attend
   kda_mtp_b64                 kda_decode_multi: 64 sequences x 64 heads, 4 tokens per state pass
   kda_prefill_32k             kda_prefill_chunked, 1 x 32768 tokens x 64 heads, chunk 64
 
@@ -435,6 +436,37 @@ class MlaPagedStep(MlaDecodeStep):
         return {"mla_latent_decode_paged": b, "step": b}
 
 
+class MlaPagedRopeStep(MlaPagedStep):
+    """The paged 16-sequence layer as an engine runs it: append each sequence's new row (latent +
+    RoPE key turned to its position, mla_cache_append) and attend with the query's RoPE part
+    turned inside the kernel (mla_latent_decode_paged_rope), both at position len - 1."""
+    name = "mla_decode_b16_paged_rope"
+
+    def __init__(self, lad, dev, rank, cfg: wl.MlaDecode | None = None):
+        super().__init__(lad, dev, rank, cfg)
+        B, s = self.cfg.B, self.cfg.seed
+        self.c_kv = wl.normal_bf16((B, wl.D_LATENT), s, "mla_ckv", dev)
+        self.k_pe = wl.normal_bf16((B, wl.D_ROPE), s, "mla_kpe", dev)
+        self.pos = (self.lens - 1).contiguous()
+        self.launches_per_step = 3
+        self.dominant = "mla_latent_decode_paged_rope"
+        self.config = dict(self.config, workload=self.name, rope="theta 6e6, rotate-half pairing, in-kernel")
+
+    def run(self, timer=None):
+        self.lad.mla_cache_append(self.c_kv, self.k_pe, self.pos, self.pool, block_table=self.block_table)
+        if timer:
+            timer.begin("mla_latent_decode_paged_rope")
+        self.lad.mla_latent_decode_paged_rope(self.q, self.pos, self.pool, self.block_table, self.lens, self.gate,
+                                              o=self.o, workspace=self.ws)
+        if timer:
+            timer.end("mla_latent_decode_paged_rope")
+
+    def algorithmic_bytes(self):
+        b = self.mla_bytes()
+        append = self.cfg.B * (wl.D_LATENT * 2 + wl.D_ROPE * 2 + 4 + wl.D_ROW * 2 + 4)
+        return {"mla_latent_decode_paged_rope": b, "step": b + append}
+
+
 class HybridStep(Step):
     name = "hybrid_8layer_1m"
 
@@ -538,6 +570,7 @@ WORKLOADS = {
     "kda_mtp_b64": KdaMultiStep,
     "mla_decode_b16": MlaDecodeStep,
     "mla_decode_b16_paged": MlaPagedStep,
+    "mla_decode_b16_paged_rope": MlaPagedRopeStep,
     "kda_prefill_32k": PrefillStep,
 }
 
@@ -621,7 +654,7 @@ def cpu_oracle_rate(workload: str, budget_s: float = 20.0) -> dict:
         sec = (time.perf_counter() - t0) * 64 / Bs
         return {"value": 256 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle",
                 "sample": f"{Bs} of 64 sequences x 64 heads x 4 tokens, scaled to 64 sequences"}
-    if workload in ("mla_decode_b16", "mla_decode_b16_paged"):
+    if workload in ("mla_decode_b16", "mla_decode_b16_paged", "mla_decode_b16_paged_rope"):
         lens = wl.mla_seq_lens(wl.MlaDecode("mla", B=16, seed=1236)).tolist()
         sec, sample = mla_seconds(16, lens)
         return {"value": 16 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": sample}
@@ -664,7 +697,7 @@ def run_reference(args, rank, world):
 
 def _tokens(workload):
     return {"hybrid_8layer_1m": 8, "kda_decode_b64": 64, "kda_mtp_b64": 256, "mla_decode_b16": 16,
-            "mla_decode_b16_paged": 16, "kda_prefill_32k": 32768}[workload]
+            "mla_decode_b16_paged": 16, "mla_decode_b16_paged_rope": 16, "kda_prefill_32k": 32768}[workload]
 
 
 def main(argv=None) -> int:
@@ -748,7 +781,7 @@ def main(argv=None) -> int:
     achieved = ab[step.dominant] / (dom_ms / 1000.0) / 1e9
     per_type = {}
     for kname in ("kda_conv_decode_step", "kda_decode_step", "kda_decode_multi", "mla_latent_decode",
-                  "mla_latent_decode_paged", "kda_prefill_chunked"):
+                  "mla_latent_decode_paged", "mla_latent_decode_paged_rope", "kda_prefill_chunked"):
         km = timer.mean_ms(kname)
         if km is not None and kname in ab:
             gbs = ab[kname] / (km / 1000.0) / 1e9

@@ -48,6 +48,7 @@ typedef uint16_t lad_bf16; /* IEEE bfloat16 bit pattern */
 #define LAD_FLAG_L2NORM_QK (1u << 1) /* KDA calls: L2-normalise q and k per head in fp32 first */
 #define LAD_FLAG_OUT_FP32 (1u << 2)  /* KDA and MLA calls: write o as fp32 instead of bf16 */
 #define LAD_FLAG_KEEP_STATE (1u << 3) /* kda_decode_multi: read S but do not write it back */
+#define LAD_FLAG_ROPE_INTERLEAVED (1u << 4) /* RoPE calls: pair dims (2i, 2i+1) instead of (i, i+32) */
 
 /* Description of the calling thread's most recent error ("" if none). */
 const char *lad_last_error(void);
@@ -58,9 +59,9 @@ int lad_version(void);
 /*
  * Reads and clears the device-side error word that bounded waits set (see above), after
  * synchronising `stream`. *code receives 0 when no kernel gave up a wait, else a nonzero tag
- * naming the kernel and the wait (0x101-0x104 latent decode, 0x201 chunked prefill), or 0x105
- * when mla_latent_decode_paged met a block-table entry outside the pool. Returns LAD_OK or
- * LAD_ECUDA.
+ * naming the kernel and the wait (0x101-0x104 latent decode, 0x201 chunked prefill), 0x105 when
+ * a paged decode met a block-table entry outside the pool, or 0x301 when mla_cache_append had a
+ * position with no row to write. Returns LAD_OK or LAD_ECUDA.
  */
 int lad_device_error(void *stream, int *code);
 
@@ -247,6 +248,47 @@ int mla_latent_decode_paged(const lad_bf16 *q, const lad_bf16 *kv_pages, int num
                             const float *gate_logits, void *o, float *lse_out, int B, int Hq, int d_latent,
                             int d_rope, float scale, unsigned flags, void *workspace, size_t ws_bytes,
                             void *stream);
+
+/*
+ * mla_latent_decode_paged_rope — mla_latent_decode_paged with RoPE applied to the query inside
+ * the kernel. [P2] "Context: 1M in the claims, 262,144 in the config": position enters only the
+ * MLA layers, through 64 of each head's 192 query-key dimensions, with rope_theta 6e6 and no
+ * scaling. q's last d_rope = 64 values per head arrive not yet turned; the kernel turns them to
+ * positions[b] (the query token's position, normally seq_lens[b] - 1) before the scores. The
+ * pairing is not on the pages: dims (i, i + 32) by default, (2i, 2i + 1) with
+ * LAD_FLAG_ROPE_INTERLEAVED; pair i turns by positions[b] * rope_theta^(-2i/64) (angle and sines in
+ * fp64, the turned values rounded to bf16 once). The cache rows are expected turned already, as
+ * mla_cache_append writes them.
+ *   positions  int32 [B] device; rope_theta > 1
+ *   the rest   as for mla_latent_decode_paged; flags: LAD_FLAG_OUT_FP32, LAD_FLAG_ROPE_INTERLEAVED
+ */
+int mla_latent_decode_paged_rope(const lad_bf16 *q, const int *positions, float rope_theta, const lad_bf16 *kv_pages,
+                                 int num_pages, int page_size, const int *block_table, int block_table_stride,
+                                 const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B,
+                                 int Hq, int d_latent, int d_rope, float scale, unsigned flags, void *workspace,
+                                 size_t ws_bytes, void *stream);
+
+/*
+ * mla_cache_append — writes one new latent-cache row per sequence: [P1] "How big is the cache per
+ * token, exactly?" (a row is the 512-wide compressed latent followed by the 64-wide RoPE key, bf16),
+ * with the RoPE key turned to the token's position here ([P2] "Context: 1M in the claims, 262,144
+ * in the config"; pairing and angles as in mla_latent_decode_paged_rope, computed in fp64, each
+ * turned value rounded to bf16 once; the latent is stored as given).
+ *   c_kv       bf16 [B][d_latent], 16-byte aligned    the compressed latent (after its norm)
+ *   k_pe       bf16 [B][d_rope]                        the RoPE key, not yet turned
+ *   positions  int32 [B] device                        row index of the new token in its sequence
+ *   cache      bf16, 16-byte aligned: with block_table == NULL the contiguous cache of
+ *              mla_latent_decode (row t of sequence b at b*cache_seq_stride + t*576, t < Lmax);
+ *              otherwise the page pool of mla_latent_decode_paged (num_pages pages of page_size
+ *              rows; row t of sequence b in page block_table[b*block_table_stride + t/page_size])
+ * A position with no row to write (negative, >= Lmax, past the block table or naming a page outside
+ * the pool) writes nothing and sets device error 0x301 (lad_device_error).
+ * flags: LAD_FLAG_ROPE_INTERLEAVED. Supported: d_latent == 512, d_rope == 64; rope_theta > 1.
+ */
+int mla_cache_append(const lad_bf16 *c_kv, const lad_bf16 *k_pe, const int *positions, lad_bf16 *cache,
+                     long long cache_seq_stride, int Lmax, const int *block_table, int block_table_stride,
+                     int num_pages, int page_size, int B, int d_latent, int d_rope, float rope_theta, unsigned flags,
+                     void *stream);
 
 /*
  * mla_latent_decode_noalloc — mla_latent_decode for callers that cannot allocate device memory

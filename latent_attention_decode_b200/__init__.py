@@ -30,6 +30,8 @@ FLAG_SILU = 1 << 0
 FLAG_L2NORM_QK = 1 << 1
 FLAG_OUT_FP32 = 1 << 2
 FLAG_KEEP_STATE = 1 << 3
+FLAG_ROPE_INTERLEAVED = 1 << 4
+ROPE_THETA = 6.0e6
 MLA_SCALE = 1.0 / math.sqrt(192.0)
 
 _c_vp = ctypes.c_void_p
@@ -69,6 +71,11 @@ def _load() -> ctypes.CDLL:
         "mla_latent_decode": ([_c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int,
                                _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
         "mla_latent_decode_workspace_size": ([_c_int] * 4, _c_sz),
+        "mla_latent_decode_paged_rope": ([_c_vp, _c_vp, _c_f, _c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp,
+                                          _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_f, _c_u, _c_vp, _c_sz,
+                                          _c_vp], _c_int),
+        "mla_cache_append": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_ll, _c_int, _c_vp, _c_int, _c_int, _c_int, _c_int,
+                              _c_int, _c_int, _c_f, _c_u, _c_vp], _c_int),
         "mla_latent_decode_paged": ([_c_vp, _c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp, _c_vp, _c_vp,
                                      _c_int, _c_int, _c_int, _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
         "mla_latent_decode_noalloc": ([_c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
@@ -383,6 +390,79 @@ def mla_latent_decode_paged(q: torch.Tensor, kv_pages: torch.Tensor, block_table
         D - d_latent, float(scale), FLAG_OUT_FP32 if out_fp32 else 0, _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
     return o
+
+
+def mla_latent_decode_paged_rope(q: torch.Tensor, positions: torch.Tensor, kv_pages: torch.Tensor,
+                                 block_table: torch.Tensor, seq_lens: torch.Tensor,
+                                 gate_logits: torch.Tensor | None = None, o: torch.Tensor | None = None,
+                                 lse: torch.Tensor | None = None, scale: float = MLA_SCALE,
+                                 rope_theta: float = ROPE_THETA, interleaved: bool = False, d_latent: int = 512,
+                                 out_fp32: bool = False, workspace: torch.Tensor | None = None,
+                                 stream=None) -> torch.Tensor:
+    """mla_latent_decode_paged with q's RoPE part (last 64 values per head) turned to positions[b]
+    inside the kernel. positions int32 [B]."""
+    bf = torch.bfloat16
+    _contig(q, "q", bf)
+    _contig(kv_pages, "kv_pages", bf)
+    B, Hq, D = q.shape
+    if kv_pages.dim() != 3 or kv_pages.shape[2] != D:
+        raise ValueError("kv_pages must be [num_pages, page_size, D]")
+    _contig(block_table, "block_table", torch.int32)
+    _contig(seq_lens, "seq_lens", torch.int32)
+    _contig(positions, "positions", torch.int32)
+    if block_table.dim() != 2 or block_table.shape[0] != B or seq_lens.shape != (B,) or positions.shape != (B,):
+        raise ValueError("block_table must be [B, n]; seq_lens and positions [B]")
+    if gate_logits is not None:
+        _contig(gate_logits, "gate_logits", torch.float32)
+    odt = torch.float32 if out_fp32 else bf
+    if o is None:
+        o = torch.empty((B, Hq, d_latent), device=q.device, dtype=odt)
+    _contig(o, "o", odt)
+    if lse is not None:
+        _contig(lse, "lse", torch.float32)
+    ws = mla_latent_decode_workspace_size(B, Hq, d_latent, 0)
+    if workspace is None and ws > 0:
+        workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
+    flags = (FLAG_OUT_FP32 if out_fp32 else 0) | (FLAG_ROPE_INTERLEAVED if interleaved else 0)
+    _check("mla_latent_decode_paged_rope", _L().mla_latent_decode_paged_rope(
+        q.data_ptr(), positions.data_ptr(), float(rope_theta), kv_pages.data_ptr(), kv_pages.shape[0],
+        kv_pages.shape[1], block_table.data_ptr(), block_table.shape[1], seq_lens.data_ptr(), _ptr(gate_logits),
+        o.data_ptr(), _ptr(lse), B, Hq, d_latent, D - d_latent, float(scale), flags, _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o
+
+
+def mla_cache_append(c_kv: torch.Tensor, k_pe: torch.Tensor, positions: torch.Tensor, cache: torch.Tensor,
+                     block_table: torch.Tensor | None = None, rope_theta: float = ROPE_THETA,
+                     interleaved: bool = False, stream=None) -> None:
+    """Writes row positions[b] of every sequence: [c_kv[b] ; k_pe[b] turned to positions[b]].
+    cache is the contiguous [B, Lmax, 576] cache (block_table None) or a page pool
+    [num_pages, page_size, 576] with block_table int32 [B, n]."""
+    bf = torch.bfloat16
+    _contig(c_kv, "c_kv", bf), _contig(k_pe, "k_pe", bf), _contig(positions, "positions", torch.int32)
+    B, Dc = c_kv.shape
+    Dr = k_pe.shape[1]
+    if k_pe.shape != (B, Dr) or positions.shape != (B,):
+        raise ValueError("c_kv [B, 512], k_pe [B, 64], positions [B]")
+    flags = FLAG_ROPE_INTERLEAVED if interleaved else 0
+    if block_table is None:
+        _cuda(cache, "cache", bf)
+        if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != Dc + Dr or cache.stride(2) != 1 \
+                or cache.stride(1) != Dc + Dr:
+            raise ValueError("cache must be [B, Lmax, 576] with contiguous rows")
+        seq_stride = cache.stride(0) if B > 1 else cache.shape[1] * (Dc + Dr)
+        rc = _L().mla_cache_append(c_kv.data_ptr(), k_pe.data_ptr(), positions.data_ptr(), cache.data_ptr(),
+                                   seq_stride, cache.shape[1], None, 0, 0, 0, B, Dc, Dr, float(rope_theta), flags,
+                                   _stream(stream))
+    else:
+        _contig(cache, "cache", bf)
+        _contig(block_table, "block_table", torch.int32)
+        if cache.dim() != 3 or cache.shape[2] != Dc + Dr or block_table.dim() != 2 or block_table.shape[0] != B:
+            raise ValueError("cache must be [num_pages, page_size, 576] and block_table [B, n]")
+        rc = _L().mla_cache_append(c_kv.data_ptr(), k_pe.data_ptr(), positions.data_ptr(), cache.data_ptr(), 0, 0,
+                                   block_table.data_ptr(), block_table.shape[1], cache.shape[0], cache.shape[1], B,
+                                   Dc, Dr, float(rope_theta), flags, _stream(stream))
+    _check("mla_cache_append", rc)
 
 
 def mla_latent_decode_noalloc(q: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tensor,

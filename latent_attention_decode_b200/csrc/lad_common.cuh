@@ -36,12 +36,17 @@ enum DeviceErrorTag : int {
     kErrMlaSoftmax = 0x103,
     kErrMlaEpilogue = 0x104,
     kErrMlaBlockTable = 0x105,  // a paged call met a block-table entry outside the pool (not a wait)
+    kErrCacheAppend = 0x301,    // mla_cache_append: a position with no row to write (not a wait)
     kErrPrefill = 0x201,
 };
 
 // Host-side readers of the per-module device error words (each clears its word).
 int take_device_error_mla(cudaStream_t s, int *code);
 int take_device_error_prefill(cudaStream_t s, int *code);
+int take_device_error_cache(cudaStream_t s, int *code);
+
+// pow(theta, -2i/d) for the d/2 RoPE pairs, on the host (the oracle computes them the same way)
+void rope_inverse_frequencies(double theta, int d_rope, double *out);
 
 }  // namespace lad
 

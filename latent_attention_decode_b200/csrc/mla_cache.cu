@@ -1,0 +1,130 @@
+// Appending decode tokens to the latent cache, with the RoPE key turned to its position here.
+//
+// Sources: "Ling-3.1-flash and the 7:1 hybrid: how much KV cache does a 560B model need at 1M
+// tokens?", section "How big is the cache per token, exactly?" (a cached row is the 512-wide
+// compressed latent followed by the 64-wide RoPE key, 576 bf16 values); "Ling-3.1-flash: a 560B
+// hybrid-attention MoE, counted from its safetensors headers", section "Context: 1M in the
+// claims, 262,144 in the config" (position enters only through RoPE on 64 of the 192 query-key
+// dimensions of the MLA layers; rope_theta 6e6, no scaling).
+//
+// One CTA of 64 threads per new token: the latent row moves as 64 16-byte pieces; threads 0-31
+// each turn one pair of the RoPE key, in fp64 (angle = position x inverse frequency, the
+// frequencies computed on the host), and round each result to bf16 once.
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "lad_common.cuh"
+
+namespace {
+
+constexpr int kDl = 512, kDr = 64, kDrow = kDl + kDr;
+
+__device__ int g_cache_error = 0;
+
+struct AppendArgs {
+    const uint16_t *c_kv;   // [B][512]
+    const uint16_t *k_pe;   // [B][64], not yet turned
+    const int *positions;   // [B]
+    uint16_t *cache;        // contiguous [B][Lmax][576] (block_table == nullptr) or a page pool
+    long long seq_stride;   // contiguous: elements between sequences
+    int Lmax;               // contiguous: rows per sequence
+    const int *block_table; // paged: [B][bt_stride]
+    int bt_stride, page_size, num_pages;
+    int interleaved;
+    double inv_freq[kDr / 2];
+};
+
+__global__ void __launch_bounds__(64) mla_cache_append_kernel(const __grid_constant__ AppendArgs a) {
+    const int b = blockIdx.x, t = threadIdx.x;
+    const int pos = a.positions[b];
+    uint16_t *dst = nullptr;
+    if (a.block_table) {
+        if (pos >= 0 && pos / a.page_size < a.bt_stride) {
+            const int page = a.block_table[static_cast<long long>(b) * a.bt_stride + pos / a.page_size];
+            if (page >= 0 && page < a.num_pages)
+                dst = a.cache + (static_cast<long long>(page) * a.page_size + pos % a.page_size) * kDrow;
+        }
+    } else if (pos >= 0 && pos < a.Lmax) {
+        dst = a.cache + static_cast<long long>(b) * a.seq_stride + static_cast<long long>(pos) * kDrow;
+    }
+    if (!dst) {
+        if (t == 0) atomicCAS(&g_cache_error, 0, lad::kErrCacheAppend);
+        return;
+    }
+    reinterpret_cast<uint4 *>(dst)[t] = reinterpret_cast<const uint4 *>(a.c_kv + static_cast<size_t>(b) * kDl)[t];
+    if (t < kDr / 2) {
+        const int ia = a.interleaved ? 2 * t : t, ib = a.interleaved ? 2 * t + 1 : t + kDr / 2;
+        const uint16_t *k = a.k_pe + static_cast<size_t>(b) * kDr;
+        const double x = static_cast<double>(lad::dev::bf16_to_f32(k[ia]));
+        const double y = static_cast<double>(lad::dev::bf16_to_f32(k[ib]));
+        double s, c;
+        sincos(static_cast<double>(pos) * a.inv_freq[t], &s, &c);
+        // separate roundings (no fused multiply-add), as a plain fp64 evaluation does
+        const double u = __dsub_rn(__dmul_rn(x, c), __dmul_rn(y, s));
+        const double w = __dadd_rn(__dmul_rn(y, c), __dmul_rn(x, s));
+        dst[kDl + ia] = __bfloat16_as_ushort(__double2bfloat16(u));
+        dst[kDl + ib] = __bfloat16_as_ushort(__double2bfloat16(w));
+    }
+}
+
+}  // namespace
+
+namespace lad {
+int take_device_error_cache(cudaStream_t s, int *code) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_cache_error, sizeof v, 0, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return set_error(LAD_ECUDA, "lad_device_error: %s", cudaGetErrorString(e));
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_cache_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return set_error(LAD_ECUDA, "lad_device_error: %s", cudaGetErrorString(e));
+    }
+    *code = v;
+    return LAD_OK;
+}
+
+void rope_inverse_frequencies(double theta, int d_rope, double *out) {
+    for (int i = 0; i < d_rope / 2; ++i) out[i] = std::pow(theta, -2.0 * i / d_rope);
+}
+}  // namespace lad
+
+extern "C" int mla_cache_append(const lad_bf16 *c_kv, const lad_bf16 *k_pe, const int *positions, lad_bf16 *cache,
+                                long long cache_seq_stride, int Lmax, const int *block_table, int block_table_stride,
+                                int num_pages, int page_size, int B, int d_latent, int d_rope, float rope_theta,
+                                unsigned flags, void *stream) {
+    using lad::set_error;
+    const char *name = "mla_cache_append";
+    if (B < 0) return set_error(LAD_EINVAL, "%s: negative B", name);
+    if (d_latent != kDl || d_rope != kDr) return set_error(LAD_EUNSUPPORTED, "%s: d_latent = 512, d_rope = 64 only", name);
+    if (flags & ~LAD_FLAG_ROPE_INTERLEAVED) return set_error(LAD_EINVAL, "%s: unknown flags 0x%x", name, flags);
+    if (!(rope_theta > 1.f) || rope_theta == INFINITY) return set_error(LAD_EINVAL, "%s: rope_theta must be > 1", name);
+    if (B == 0) return LAD_OK;
+    if (!c_kv || !k_pe || !positions || !cache) return set_error(LAD_EINVAL, "%s: null pointer", name);
+    if (!lad::aligned(c_kv, 16) || !lad::aligned(cache, 16))
+        return set_error(LAD_EUNSUPPORTED, "%s: c_kv and the cache must be 16-byte aligned", name);
+    AppendArgs a{};
+    a.c_kv = reinterpret_cast<const uint16_t *>(c_kv);
+    a.k_pe = reinterpret_cast<const uint16_t *>(k_pe);
+    a.positions = positions;
+    a.cache = reinterpret_cast<uint16_t *>(cache);
+    a.interleaved = (flags & LAD_FLAG_ROPE_INTERLEAVED) ? 1 : 0;
+    if (block_table) {
+        if (page_size <= 0 || num_pages < 0 || block_table_stride < 0)
+            return set_error(LAD_EINVAL, "%s: page_size > 0, num_pages and block_table_stride >= 0", name);
+        a.block_table = block_table;
+        a.bt_stride = block_table_stride;
+        a.page_size = page_size;
+        a.num_pages = num_pages;
+    } else {
+        if (Lmax < 0 || cache_seq_stride < static_cast<long long>(Lmax) * kDrow || cache_seq_stride % 8 != 0)
+            return set_error(LAD_EINVAL, "%s: cache_seq_stride must be >= Lmax*576 and a multiple of 8", name);
+        a.seq_stride = cache_seq_stride;
+        a.Lmax = Lmax;
+    }
+    lad::rope_inverse_frequencies(static_cast<double>(rope_theta), kDr, a.inv_freq);
+    mla_cache_append_kernel<<<B, 64, 0, lad::as_stream(stream)>>>(a);
+    return lad::check_launch(name);
+}

@@ -87,7 +87,8 @@ enum Bar : int {
     kBarWg = kBarPEmpty + 2,           // [2] softmax warps exchanged their rescale decisions
     kBarOFree = kBarWg + 2,            // epilogue has read O
     kBarQFull = kBarOFree + 1,         // q of a segment landed
-    kBarQEmpty = kBarQFull + 1,        // GEMM1s of a segment done with q
+    kBarQRoped = kBarQFull + 1,        // (RoPE variant) q's RoPE part turned to the query position
+    kBarQEmpty = kBarQRoped + 1,       // GEMM1s of a segment done with q
     kBarDrain = kBarQEmpty + 1,        // final MMA drain
     kNumBars = kBarDrain + 1,
 };
@@ -311,12 +312,22 @@ struct PagedCache {
     int oob_row;  // the pool map's row extent: a tile starting there reads as zeros
 };
 
+// RoPE variant: q arrives with its 64-wide RoPE part not yet turned; sequence b's query sits at
+// position positions[b]. Pair i (dims i and i + 32, or 2i and 2i + 1 when interleaved) turns by
+// positions[b] * inv_freq[i] (inverse frequencies computed on the host).
+struct RopeQ {
+    const int *positions;
+    int interleaved;
+    double inv_freq[kDr / 2];
+};
+
 // kPaged: map_cache is 2-D over the page pool ([num_pages * page_size][576]) and each tile's row
 // comes from the block table; otherwise it is 3-D ([B][Lmax][576]).
-template <bool kPaged>
+template <bool kPaged, bool kRopeQ>
 __global__ void __launch_bounds__(kThreads, 1)
 mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_constant__ CUtensorMap map_q,
-                 const int *__restrict__ seq_lens, int B, float score_scale_log2, Partials ws, PagedCache pc) {
+                 const int *__restrict__ seq_lens, int B, float score_scale_log2, Partials ws, PagedCache pc,
+                 const __grid_constant__ RopeQ rq) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -478,7 +489,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             const uint64_t q_desc0 = smem_desc(sbase + kOffQ, 16, 1024, kLayoutSw128);
             const uint64_t c_desc0 = smem_desc(sbase + kOffStage, 16, 1024, kLayoutSw128);
             while (ok && it.next(seq, tile0, nt)) {
-                if (!wait_bar(bar(kBarQFull), k & 1, abort_flag, lad::kErrMlaMma)) {
+                if (!wait_bar(bar(kRopeQ ? kBarQRoped : kBarQFull), k & 1, abort_flag, lad::kErrMlaMma)) {
                     ok = false;
                     break;
                 }
@@ -522,6 +533,33 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             const uint64_t v_desc0 = smem_desc(sbase + kOffStage, kTChunkBytes, 1024, kLayoutSw128);
             const uint64_t p_desc0 = smem_desc(sbase + kOffP, 128, 512, kLayoutNone);
             while (ok && it.next(seq, tile0, nt)) {
+                if constexpr (kRopeQ) {
+                    // turn the RoPE part (q dims 512..575: the last 64-dim chunk, one 128-byte
+                    // swizzled row per head) to the query position; lane i takes pair i of all heads
+                    if (!wait_bar(bar(kBarQFull), k & 1, abort_flag, lad::kErrMlaMma)) {
+                        ok = false;
+                        break;
+                    }
+                    double sd, cd;
+                    sincos(static_cast<double>(rq.positions[seq]) * rq.inv_freq[lane], &sd, &cd);
+                    const float c = static_cast<float>(cd), sn = static_cast<float>(sd);
+                    const int ia = rq.interleaved ? 2 * lane : lane;
+                    const int ib = rq.interleaved ? 2 * lane + 1 : lane + kDr / 2;
+                    uint16_t *qr = reinterpret_cast<uint16_t *>(smem + kOffQ + (kNChunk - 1) * kQChunkBytes);
+#pragma unroll 4
+                    for (int hh = 0; hh < kHq; ++hh) {
+                        // element d of head hh's row: 16-byte chunk (d / 8) xor (hh % 8), slot d % 8
+                        uint16_t *row = qr + hh * 64;
+                        const int oa = (((ia >> 3) ^ (hh & 7)) << 3) + (ia & 7);
+                        const int ob = (((ib >> 3) ^ (hh & 7)) << 3) + (ib & 7);
+                        const float x = lad::dev::bf16_to_f32(row[oa]), y = lad::dev::bf16_to_f32(row[ob]);
+                        row[oa] = lad::dev::f32_to_bf16(x * c - y * sn);
+                        row[ob] = lad::dev::f32_to_bf16(y * c + x * sn);
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(kBarQRoped));
+                }
                 for (int i = 0; i < nt; ++i, ++g) {
                     const uint32_t pb = g & 1;
                     if (!wait_bar(bar(kBarPFull + pb), (g >> 1) & 1, abort_flag, lad::kErrMlaMma)) {
@@ -879,9 +917,14 @@ int set_smem_attributes(const char *name) {
     if (dev < 0 || dev >= 64) return lad::set_error(LAD_EUNSUPPORTED, "%s: device %d", name, dev);
     std::lock_guard<std::mutex> lock(mu);
     if (!done[dev]) {
-        e = cudaFuncSetAttribute(mla_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        e = cudaFuncSetAttribute(mla_split_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemBytes);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(mla_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            e = cudaFuncSetAttribute(mla_split_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(mla_split_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kSmemBytes);
         if (e != cudaSuccess)
             return lad::set_error(LAD_ECUDA, "%s: smem attribute: %s", name, cudaGetErrorString(e));
         done[dev] = true;
@@ -935,9 +978,9 @@ int encode_contiguous(const char *name, CUtensorMap *map, const lad_bf16 *cache,
 }
 
 // Everything after the argument checks: the q map, the split kernel and the combine.
-int run_mla(const char *name, const CUtensorMap &map_cache, bool paged, const PagedCache &pc, const lad_bf16 *q,
-            const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B, float scale, unsigned flags,
-            uint8_t *ws, const WsLayout &wl, int G, void *stream) {
+int run_mla(const char *name, const CUtensorMap &map_cache, bool paged, const PagedCache &pc, const RopeQ *rope,
+            const lad_bf16 *q, const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B,
+            float scale, unsigned flags, uint8_t *ws, const WsLayout &wl, int G, void *stream) {
     using lad::set_error;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return set_error(LAD_ECUDA, "%s: cuTensorMapEncodeTiled unavailable", name);
@@ -960,12 +1003,16 @@ int run_mla(const char *name, const CUtensorMap &map_cache, bool paged, const Pa
                    reinterpret_cast<float *>(ws + wl.off_l), reinterpret_cast<long long *>(ws + wl.off_prefix)};
     cudaStream_t s = lad::as_stream(stream);
     const float score_scale_log2 = scale * 1.4426950408889634f;
-    if (paged)
-        mla_split_kernel<true><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B, score_scale_log2, parts,
-                                                                pc);
+    const RopeQ none{};
+    if (rope)
+        mla_split_kernel<true, true><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B, score_scale_log2,
+                                                                      parts, pc, *rope);
+    else if (paged)
+        mla_split_kernel<true, false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
+                                                                       score_scale_log2, parts, pc, none);
     else
-        mla_split_kernel<false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B, score_scale_log2,
-                                                                 parts, pc);
+        mla_split_kernel<false, false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
+                                                                        score_scale_log2, parts, pc, none);
     rc = lad::check_launch(name);
     if (rc != LAD_OK) return rc;
     const dim3 cgrid(static_cast<unsigned>(B), kHq);
@@ -1016,18 +1063,17 @@ extern "C" int mla_latent_decode(const lad_bf16 *q, const lad_bf16 *cache, long 
     CUtensorMap map_cache;
     rc = encode_contiguous(name, &map_cache, cache, B, Lmax, cache_seq_stride);
     if (rc != LAD_OK) return rc;
-    return run_mla(name, map_cache, false, PagedCache{}, q, seq_lens, gate_logits, o, lse_out, B, scale, flags,
-                   static_cast<uint8_t *>(workspace), wl, G, stream);
+    return run_mla(name, map_cache, false, PagedCache{}, nullptr, q, seq_lens, gate_logits, o, lse_out, B, scale,
+                   flags, static_cast<uint8_t *>(workspace), wl, G, stream);
 }
 
-extern "C" int mla_latent_decode_paged(const lad_bf16 *q, const lad_bf16 *kv_pages, int num_pages, int page_size,
-                                       const int *block_table, int block_table_stride, const int *seq_lens,
-                                       const float *gate_logits, void *o, float *lse_out, int B, int Hq, int d_latent,
-                                       int d_rope, float scale, unsigned flags, void *workspace, size_t ws_bytes,
-                                       void *stream) {
+namespace {
+int run_paged(const char *name, const lad_bf16 *q, const lad_bf16 *kv_pages, int num_pages, int page_size,
+              const int *block_table, int block_table_stride, const int *seq_lens, const float *gate_logits, void *o,
+              float *lse_out, int B, int Hq, int d_latent, int d_rope, float scale, unsigned flags,
+              unsigned extra_flags, const RopeQ *rope, void *workspace, size_t ws_bytes, void *stream) {
     using lad::set_error;
-    const char *name = "mla_latent_decode_paged";
-    int rc = check_common(name, B, Hq, d_latent, d_rope, flags, scale);
+    int rc = check_common(name, B, Hq, d_latent, d_rope, flags & ~extra_flags, scale);
     if (rc != LAD_OK) return rc;
     if (num_pages < 0 || block_table_stride < 0) return set_error(LAD_EINVAL, "%s: negative size", name);
     if (page_size <= 0 || page_size % kTile != 0)
@@ -1054,8 +1100,38 @@ extern "C" int mla_latent_decode_paged(const lad_bf16 *q, const lad_bf16 *kv_pag
         if (rc != LAD_OK) return rc;
     }
     const PagedCache pc{block_table, block_table_stride, page_size, num_pages, rows};
-    return run_mla(name, map_cache, true, pc, q, seq_lens, gate_logits, o, lse_out, B, scale, flags,
-                   static_cast<uint8_t *>(workspace), wl, G, stream);
+    return run_mla(name, map_cache, true, pc, rope, q, seq_lens, gate_logits, o, lse_out, B, scale,
+                   flags & ~extra_flags, static_cast<uint8_t *>(workspace), wl, G, stream);
+}
+}  // namespace
+
+extern "C" int mla_latent_decode_paged(const lad_bf16 *q, const lad_bf16 *kv_pages, int num_pages, int page_size,
+                                       const int *block_table, int block_table_stride, const int *seq_lens,
+                                       const float *gate_logits, void *o, float *lse_out, int B, int Hq, int d_latent,
+                                       int d_rope, float scale, unsigned flags, void *workspace, size_t ws_bytes,
+                                       void *stream) {
+    return run_paged("mla_latent_decode_paged", q, kv_pages, num_pages, page_size, block_table, block_table_stride,
+                     seq_lens, gate_logits, o, lse_out, B, Hq, d_latent, d_rope, scale, flags, 0u, nullptr, workspace,
+                     ws_bytes, stream);
+}
+
+extern "C" int mla_latent_decode_paged_rope(const lad_bf16 *q, const int *positions, float rope_theta,
+                                            const lad_bf16 *kv_pages, int num_pages, int page_size,
+                                            const int *block_table, int block_table_stride, const int *seq_lens,
+                                            const float *gate_logits, void *o, float *lse_out, int B, int Hq,
+                                            int d_latent, int d_rope, float scale, unsigned flags, void *workspace,
+                                            size_t ws_bytes, void *stream) {
+    const char *name = "mla_latent_decode_paged_rope";
+    if (B > 0 && !positions) return lad::set_error(LAD_EINVAL, "%s: null positions", name);
+    if (!(rope_theta > 1.f) || rope_theta == INFINITY)
+        return lad::set_error(LAD_EINVAL, "%s: rope_theta must be > 1", name);
+    RopeQ rq{};
+    rq.positions = positions;
+    rq.interleaved = (flags & LAD_FLAG_ROPE_INTERLEAVED) ? 1 : 0;
+    if (d_rope == kDr) lad::rope_inverse_frequencies(static_cast<double>(rope_theta), kDr, rq.inv_freq);
+    return run_paged(name, q, kv_pages, num_pages, page_size, block_table, block_table_stride, seq_lens, gate_logits,
+                     o, lse_out, B, Hq, d_latent, d_rope, scale, flags, LAD_FLAG_ROPE_INTERLEAVED, &rq, workspace,
+                     ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1136,6 +1212,6 @@ extern "C" int mla_latent_decode_noalloc(const lad_bf16 *q, const lad_bf16 *cach
     CUtensorMap map_cache;
     rc = encode_contiguous(name, &map_cache, cache, B, Lmax, cache_seq_stride);
     if (rc != LAD_OK) return rc;
-    return run_mla(name, map_cache, false, PagedCache{}, q, seq_lens, gate_logits, o, lse_out, B, scale, flags, ws,
-                   wl, G, stream);
+    return run_mla(name, map_cache, false, PagedCache{}, nullptr, q, seq_lens, gate_logits, o, lse_out, B, scale,
+                   flags, ws, wl, G, stream);
 }
