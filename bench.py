@@ -111,6 +111,26 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def kernel_traffic(kernel: str, units: float | None) -> dict | None:
+    """DRAM bytes of one launch of `kernel` from the ncu capture recorded in profiles/traffic.json,
+    scaled by units (cached rows, heads, token-heads) to this launch; None when there is no capture
+    or the kernel's source has changed since it was taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if units is None or not os.path.exists(p):
+        return None
+    with open(p) as f:
+        e = json.load(f)["kernels"].get(kernel)
+    if not e:
+        return None
+    with open(os.path.join(ROOT, e["source"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != e["sha256"]:
+            return None
+    scale = units / e["units"]
+    return {"bytes": int(round((e["read"] + e["write"]) * scale)), "scaled_from": e["capture"],
+            "scale": round(scale, 6), "profile": e["profile"]}
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
 
@@ -183,6 +203,10 @@ class Step:
     tokens_per_step = 0          # decode tokens (or prefill tokens) one step produces on this GPU
     launches_per_step = 0        # library kernels one step launches
     dominant = ""                # name of the roofline kernel
+
+    def dominant_units(self):
+        """Units of the dominant kernel's work per launch, in the unit profiles/traffic.json uses."""
+        return None
     dominant_unit = "GB/s"
     dominant_bound = "hbm"
     config: dict = {}
@@ -293,6 +317,9 @@ class KdaDecodeStep(Step):
     def e2e_bytes(self):
         return self.layer.h2d_bytes(), self.layer.d2h_bytes()
 
+    def dominant_units(self):
+        return self.layer.B * H
+
     def algorithmic_bytes(self):
         B = self.layer.B
         return {"kda_decode_step": _KdaLayer.bytes_decode(B), "kda_conv_update": _KdaLayer.bytes_conv(B),
@@ -338,6 +365,9 @@ class KdaMultiStep(Step):
 
     def e2e_bytes(self):
         return sum(t.numel() * t.element_size() for t in self.h_in), self.h_o.numel() * 2
+
+    def dominant_units(self):
+        return self.B * H if self.T == 4 else None
 
     def algorithmic_bytes(self):
         # per (b, h): state read + write; per token q, k, v (bf16), alpha (fp32), beta, o (bf16)
@@ -398,6 +428,9 @@ class MlaDecodeStep(Step):
 
     def mla_flops(self):
         return 2 * self.cfg.Hq * (wl.D_ROW + wl.D_LATENT) * self.total_len
+
+    def dominant_units(self):
+        return self.total_len
 
     def algorithmic_bytes(self):
         b = self.mla_bytes()
@@ -477,6 +510,7 @@ class HybridStep(Step):
         self.tokens_per_step = B
         self.launches_per_step = (1 if _KdaLayer.fused else 2) * kda_layers + self.mla.launches_per_step
         self.dominant = "mla_latent_decode"
+        self.dominant_units = lambda: self.mla.total_len
         self.config = {"workload": self.name, "batch_per_gpu": B, "layers": f"{kda_layers} KDA + 1 gated MLA",
                        "kda_path": "fused conv+step" if _KdaLayer.fused else "conv, then step",
                        "mla_context": ctx, "heads": H, "head_dim": D,
@@ -548,6 +582,9 @@ class PrefillStep(Step):
 
     def e2e_bytes(self):
         return sum(t.numel() * t.element_size() for t in self.h_in), self.h_o.numel() * 2
+
+    def dominant_units(self):
+        return self.cfg.B * self.cfg.T * self.cfg.H
 
     def algorithmic_bytes(self):
         c = self.cfg
@@ -801,6 +838,7 @@ def main(argv=None) -> int:
         if world == 1 and not args.no_cpu_baseline:
             cb = cpu_oracle_rate(args.workload)
         hb, db = step.e2e_bytes()
+        traffic = kernel_traffic(step.dominant, step.dominant_units())
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -811,7 +849,8 @@ def main(argv=None) -> int:
             "step_gb_s": ab["step"] / (ms / 1000.0) / 1e9,
             "roofline": {"kernel": step.dominant, "bound": step.dominant_bound, "achieved": achieved,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                         "traffic": None, "peak_source": f"{peaks['source']} hbm_gbs (copy)",
+                         "traffic": traffic["bytes"] if traffic else None,
+                         "traffic_source": traffic, "peak_source": f"{peaks['source']} hbm_gbs (copy)",
                          "algorithmic_bytes_per_launch": ab[step.dominant]},
             "cpu_baseline": cb,
             "e2e": {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": hb * world,
