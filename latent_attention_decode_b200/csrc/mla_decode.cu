@@ -791,7 +791,6 @@ mla_combine_kernel(const int *__restrict__ seq_lens, int B, int G, const float *
     const int b = blockIdx.x, h = blockIdx.y;
     const int d = 4 * threadIdx.x;
     __shared__ int s_c[2];
-    __shared__ unsigned char s_valid[kMaxSplitCtas];  // CTA c0 + i has a non-empty tile range
     const long long total = ws.tile_prefix[B];
     const long long lo = ws.tile_prefix[b], hi = ws.tile_prefix[b + 1];
     if (threadIdx.x == 0) {
@@ -811,24 +810,51 @@ mla_combine_kernel(const int *__restrict__ seq_lens, int B, int G, const float *
     }
     __syncthreads();
     const int c0 = s_c[0], c1 = s_c[1];
-    // with fewer tiles than CTAs some CTAs own no tiles and wrote no partial
-    for (int c = c0 + static_cast<int>(threadIdx.x); c <= c1; c += blockDim.x)
-        s_valid[c - c0] = split_point(total, G, c) < split_point(total, G, c + 1);
+    // Per covering CTA its partial's weight, in shared memory: 0 for a CTA that owns no tiles (with
+    // fewer tiles than CTAs) and so wrote no partial. Then every thread runs over the partials with
+    // independent loads.
+    __shared__ float s_w[kMaxSplitCtas];
+    __shared__ float s_red[4];
+    const int nc = c1 - c0 + 1;
+    float mx = -INFINITY;
+    for (int i = static_cast<int>(threadIdx.x); i < nc; i += blockDim.x) {
+        const int c = c0 + i;
+        const bool valid = split_point(total, G, c) < split_point(total, G, c + 1);
+        const float mc = valid ? ws.m[(static_cast<long long>(c) + b) * kHq + h] : -INFINITY;
+        s_w[i] = mc;
+        mx = fmaxf(mx, mc);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = mx;
     __syncthreads();
+    const float M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+    float ls = 0.f;
+    for (int i = static_cast<int>(threadIdx.x); i < nc; i += blockDim.x) {
+        const float mc = s_w[i];
+        const float w = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+        s_w[i] = w;
+        if (w != 0.f) ls = fmaf(w, ws.l[(static_cast<long long>(c0 + i) + b) * kHq + h], ls);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    __syncthreads();  // s_red is reused below; s_w is complete
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = ls;
+    __syncthreads();
+    const float Lsum = (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float M = -INFINITY, Lsum = 0.f;
-    for (int c = c0; c <= c1; ++c)
-        if (s_valid[c - c0]) M = fmaxf(M, ws.m[(static_cast<long long>(c) + b) * kHq + h]);
-    for (int c = c0; c <= c1; ++c) {
-        if (!s_valid[c - c0]) continue;
-        const long long slot = static_cast<long long>(c) + b;
-        const float w = exp2f(ws.m[slot * kHq + h] - M);
-        Lsum += w * ws.l[slot * kHq + h];
-        const float4 v = *reinterpret_cast<const float4 *>(ws.O + (slot * kHq + h) * kDl + d);
-        acc.x = fmaf(w, v.x, acc.x);
-        acc.y = fmaf(w, v.y, acc.y);
-        acc.z = fmaf(w, v.z, acc.z);
-        acc.w = fmaf(w, v.w, acc.w);
+    const float *Ob = ws.O + (static_cast<long long>(c0 + b) * kHq + h) * kDl + d;
+    const long long slot_stride = static_cast<long long>(kHq) * kDl;
+#pragma unroll 4
+    for (int i = 0; i < nc; ++i) {
+        const float w = s_w[i];
+        if (w != 0.f) {
+            const float4 v = *reinterpret_cast<const float4 *>(Ob + i * slot_stride);
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
     }
     float sc = (Lsum > 0.f) ? 1.f / Lsum : 0.f;
     if (gate) sc *= 1.f / (1.f + expf(-gate[b * kHq + h]));
