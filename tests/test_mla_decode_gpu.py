@@ -148,3 +148,18 @@ def test_million_token_context_sampled(lad, cuda_device):
     o_ref, lse_ref = _oracle(q, cache, L, gate, seqs=[1], heads=heads)
     assert rel_l2(o[1, heads], o_ref[0]) < TOL_OUT
     np.testing.assert_allclose(f64(lse[1, heads]), lse_ref[0], rtol=0, atol=1e-3)
+
+
+@pytest.mark.slow
+def test_hybrid_launch_8x1m_sampled(lad, cuda_device):
+    """The 8-layer hybrid step's latent decode exactly as bench.py launches it: 8 sequences of
+    1,000,000 cached rows drawn with the bench's seed; eight heads (one per head group of each
+    TMEM sub-partition) of two sequences, the first and the last, against the oracle."""
+    cfg = wl.MlaDecode("mla", B=8, seed=1238, fixed_len=1_000_000)
+    inp = wl.mla_inputs(cfg, cuda_device)
+    o, lse = _run(lad, inp["q"], inp["cache"], inp["seq_lens"], inp["gate"], out_fp32=False)
+    seqs, heads = [0, 7], [0, 9, 18, 27, 36, 45, 54, 63]
+    o_ref, lse_ref = _oracle(inp["q"], inp["cache"], inp["seq_lens"], inp["gate"], seqs=seqs, heads=heads)
+    got = o[seqs][:, heads]
+    assert rel_l2(got, bf16_round(o_ref)) < TOL_OUT
+    np.testing.assert_allclose(f64(lse[seqs][:, heads]), lse_ref, rtol=0, atol=1e-3)
