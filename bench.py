@@ -522,10 +522,26 @@ class HybridStep(Step):
         self.mla.run(timer)
 
     def run_e2e(self):
-        for layer in self.kda:
-            layer.h2d()
-        self.mla.h2d()
-        self.run()
+        # Every layer's token inputs are known when the step starts: they go up on a copy stream,
+        # layer by layer, and each layer waits only for its own copy, so later copies overlap
+        # earlier layers. Outputs come back on the compute stream at the end.
+        cur = torch.cuda.current_stream()
+        if not hasattr(self, "_copy_stream"):
+            self._copy_stream = torch.cuda.Stream()
+        cs = self._copy_stream
+        cs.wait_stream(cur)   # the previous step's kernels are done with these buffers
+        events = []
+        with torch.cuda.stream(cs):
+            for part in (*self.kda, self.mla):
+                part.h2d()
+                e = torch.cuda.Event()
+                e.record(cs)
+                events.append(e)
+        for layer, e in zip(self.kda, events):
+            cur.wait_event(e)
+            layer.run()
+        cur.wait_event(events[-1])
+        self.mla.run()
         for layer in self.kda:
             layer.d2h()
         self.mla.d2h()
