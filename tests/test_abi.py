@@ -47,3 +47,32 @@ def test_host_side_validation(lib):
     assert lib.kda_conv_update(16, 16, 16, None, 32, 1, 16, 4, 0x80, None) == -1
     assert lib.kda_conv_update(16, 16, 16, None, 16, 1, 16, 4, 0, None) == -1  # y aliases x
     assert lad.lad_version() >= 100
+
+
+def test_host_side_validation_of_the_newer_calls(lib):
+    """Each of these returns before any CUDA call (no GPU here)."""
+    # kda_decode_multi: more than 8 tokens, unknown flag, head size, empty work
+    assert lib.kda_decode_multi(16, 16, 16, 16, 16, 16, None, None, 1, 9, 1, 128, 128, 1.0, 0, None) == -2
+    assert lib.kda_decode_multi(16, 16, 16, 16, 16, 16, None, None, 1, 4, 1, 128, 128, 1.0, 0x100, None) == -1
+    assert lib.kda_decode_multi(16, 16, 16, 16, 16, 16, None, None, 1, 4, 1, 64, 64, 1.0, 0, None) == -2
+    assert lib.kda_decode_multi(None, None, None, None, None, None, None, None, 0, 4, 1, 128, 128, 1.0, 0, None) == 0
+    assert lib.kda_decode_multi(None, 16, 16, 16, 16, 16, None, None, 1, 4, 1, 128, 128, 1.0, 0, None) == -1
+    # mla_latent_decode_paged: page size not a multiple of 32, head count, scale
+    args = (16, 16, 4, 48, 16, 1, 16, None, 16, None, 1, 64, 512, 64, 0.1, 0, 16, 1 << 20, None)
+    assert lib.mla_latent_decode_paged(*args) == -2 and b"multiple of 32" in lib.lad_last_error()
+    bad_h = list(args); bad_h[3] = 64; bad_h[11] = 32
+    assert lib.mla_latent_decode_paged(*bad_h) == -2
+    bad_s = list(args); bad_s[3] = 64; bad_s[14] = -1.0
+    assert lib.mla_latent_decode_paged(*bad_s) == -1
+    # mla_latent_decode_paged_rope: rope_theta must exceed 1, positions required
+    r = (16, 16, 1.0, 16, 4, 64, 16, 1, 16, None, 16, None, 1, 64, 512, 64, 0.1, 0, 16, 1 << 20, None)
+    assert lib.mla_latent_decode_paged_rope(*r) == -1 and b"rope_theta" in lib.lad_last_error()
+    r2 = list(r); r2[1] = None; r2[2] = 6.0e6
+    assert lib.mla_latent_decode_paged_rope(*r2) == -1 and b"positions" in lib.lad_last_error()
+    # mla_cache_append: unknown flag, widths, theta, contiguous stride too small, empty batch
+    a = [16, 16, 16, 16, 576 * 8, 8, None, 0, 0, 0, 1, 512, 64, 6.0e6, 0, None]
+    assert lib.mla_cache_append(*(a[:14] + [0x40] + a[15:])) == -1
+    assert lib.mla_cache_append(*(a[:11] + [256] + a[12:])) == -2
+    assert lib.mla_cache_append(*(a[:13] + [0.5] + a[14:])) == -1
+    assert lib.mla_cache_append(*(a[:4] + [576] + a[5:])) == -1 and b"cache_seq_stride" in lib.lad_last_error()
+    assert lib.mla_cache_append(*(a[:10] + [0] + a[11:])) == 0
