@@ -38,7 +38,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "lad_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace {
 
@@ -96,161 +96,40 @@ constexpr int kOffScalars = kNumBars * 8;  // inside the barrier region: tmem ba
 
 __device__ int g_mla_error = 0;
 
-// ------------------------------------------------------------------------------------------
-// PTX wrappers
-// ------------------------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait for the phase of `bar` with parity `parity`. Returns false if the CTA is
-// aborting (this wait ran out, or another role's did).
-__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag, int tag) {
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicCAS(&g_mla_error, 0, tag);
-            return false;
-        }
-    }
-}
-
-// Called by whole warps; the result is made warp-uniform so that every lane takes the same path
-// (the issue helpers rely on the warp staying converged).
+// Bounded waits: lad::ptx::wait_bar with this module's device error word (see lad_common.cuh).
+// Called by whole warps; the result is warp-uniform, so every lane takes the same path (the issue
+// helpers rely on the warp staying converged).
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag, int tag) {
-    const bool r = mbar_try_wait(bar, parity) || wait_bar_slow(bar, parity, abort_flag, tag);
-    return __all_sync(0xffffffffu, r);
+    return lad::ptx::wait_bar(bar, parity, abort_flag, &g_mla_error, tag);
 }
 
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// The issue helpers below are executed by a whole, converged warp; `elect.sync` picks one lane
+// The issue helpers (lad::ptx) are executed by a whole, converged warp; `elect.sync` picks one lane
 // (the same lowest lane every time) that actually issues. Keeping the warp converged lets the
 // descriptors and addresses live in uniform registers, which tcgen05.mma and TMA read directly.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z, uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-        "[%5];\n\t}" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-        : "memory");
+using lad::ptx::ex2_approx;
+using lad::ptx::kLayoutNone;
+using lad::ptx::kLayoutSw128;
+using lad::ptx::mbar_arrive;
+using lad::ptx::mbar_arrive_tx_elect;
+using lad::ptx::mbar_init;
+using lad::ptx::mbar_try_wait;
+using lad::ptx::smem_desc;
+using lad::ptx::smem_u32;
+using lad::ptx::tc_commit;
+using lad::ptx::tc_fence_after;
+using lad::ptx::tc_fence_before;
+using lad::ptx::tmem_ld32u;
+using lad::ptx::tmem_st32u;
+using lad::ptx::tmem_wait_ld;
+using lad::ptx::tmem_wait_st;
+
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    lad::ptx::tc_mma_f16(d, a, b, idesc, acc);
 }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-        "@e cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];\n\t}" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_tx_elect(uint32_t bar, uint32_t bytes) {
-    asm volatile(
-        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-        "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(bar),
-        "r"(bytes)
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Warp-wide: the elected lane commits (the same lane that issued the MMAs).
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
-        : "memory");
-}
-
-// Warp-wide: D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (bf16 in, fp32 accumulate),
-// issued by the elected lane.
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-#define LAD_TMEM_LD32(taddr, r)                                                                                      \
-    asm volatile(                                                                                                    \
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18," \
-        "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                                              \
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),           \
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),     \
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),   \
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])    \
-        : "r"(taddr))
-
-#define LAD_TMEM_ST32(taddr, r)                                                                                      \
-    asm volatile(                                                                                                    \
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17," \
-        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),                              \
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),         \
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), \
-        "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]),            \
-        "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])                                      \
-        : "memory")
-
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// ------------------------------------------------------------------------------------------
-// UMMA descriptors
-// ------------------------------------------------------------------------------------------
-// Shared-memory matrix descriptor: start address, leading / stride byte offsets (16-byte
-// units), descriptor version 1, layout type in bits 61..63.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
-    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
-    d |= static_cast<uint64_t>(1u) << 46;  // version
-    d |= static_cast<uint64_t>(layout & 7u) << 61;
-    return d;
-}
-constexpr uint32_t kLayoutSw128 = 2;
-constexpr uint32_t kLayoutNone = 0;
-
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, majors, N >> 3, M >> 4.
+// bf16 operands, fp32 accumulator; majors (0 K-major, 1 MN-major)
 constexpr uint32_t make_idesc(int M, int N, int a_mn_major, int b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn_major) << 15) |
-           (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
-           (static_cast<uint32_t>(M >> 4) << 24);
+    return lad::ptx::make_idesc(M, N, lad::ptx::kFmtBf16, a_mn_major, b_mn_major);
 }
 constexpr uint32_t kIdesc1 = make_idesc(64, kTile, 0, 0);   // S = q . C^T
 constexpr uint32_t kIdesc2 = make_idesc(128, kHq, 1, 0);    // O^T += V^T . P^T
@@ -421,7 +300,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                 }
                 mbar_arrive_tx_elect(bar(kBarQFull), kQBytes);
                 for (int c = 0; c < kNChunk; ++c)
-                    tma_load_2d(sbase + kOffQ + c * kQChunkBytes, &map_q, c * kChunk, seq * kHq, bar(kBarQFull));
+                    lad::ptx::tma_load_2d_elect(sbase + kOffQ + c * kQChunkBytes, &map_q, c * kChunk, seq * kHq, bar(kBarQFull));
                 for (int i = 0; i < nt; ++i, ++g) {
                     const uint32_t s = g % kStages;
                     int row = (tile0 + i) * kTile;
@@ -452,9 +331,9 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     const uint32_t dst = sbase + kOffStage + s * kStageBytes;
                     for (int c = 0; c < kNChunk; ++c) {
                         if constexpr (kPaged)
-                            tma_load_2d(dst + c * kTChunkBytes, &map_cache, c * kChunk, row, bar(kBarFull + s));
+                            lad::ptx::tma_load_2d_elect(dst + c * kTChunkBytes, &map_cache, c * kChunk, row, bar(kBarFull + s));
                         else
-                            tma_load_3d(dst + c * kTChunkBytes, &map_cache, c * kChunk, row, seq, bar(kBarFull + s));
+                            lad::ptx::tma_load_3d_elect(dst + c * kTChunkBytes, &map_cache, c * kChunk, row, seq, bar(kBarFull + s));
                     }
                 }
                 ++k;
@@ -614,8 +493,8 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                 }
                 tc_fence_after();
                 uint32_t r[kTile], r2[kTile];
-                LAD_TMEM_LD32(tmem + lane_addr + kColS + sb * kSBufCols, r);
-                LAD_TMEM_LD32(tmem + lane_addr + kColS + sb * kSBufCols + kTile, r2);
+                tmem_ld32u(tmem + lane_addr + kColS + sb * kSBufCols, r);
+                tmem_ld32u(tmem + lane_addr + kColS + sb * kSBufCols + kTile, r2);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
@@ -669,7 +548,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     m = tmax;
                     f = 0.f;
                 } else if (tmax > m + 8.f) {
-                    f = ex2(m - tmax);
+                    f = ex2_approx(m - tmax);
                     m = tmax;
                     need = true;
                 }
@@ -677,8 +556,8 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                 float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int j = 0; j < kTile / 2; j += 2) {
-                    const float p0 = ex2(fmaf(xs[j], score_scale_log2, -m));
-                    const float p1 = ex2(fmaf(xs[j + 1], score_scale_log2, -m));
+                    const float p0 = ex2_approx(fmaf(xs[j], score_scale_log2, -m));
+                    const float p1 = ex2_approx(fmaf(xs[j + 1], score_scale_log2, -m));
                     ps[(j >> 1) & 3] += p0 + p1;  // the denominator keeps fp32 probabilities
                     pk[j / 2] = lad::dev::f32x2_to_bf16x2(p0, p1);
                 }
@@ -727,12 +606,12 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                         for (int half = 0; half < 2; ++half) {
                             uint32_t o[32];
                             const uint32_t ta = tmem + lane_addr + kColO + 64 * j + 32 * half;
-                            LAD_TMEM_LD32(ta, o);
+                            tmem_ld32u(ta, o);
                             tmem_wait_ld();
 #pragma unroll
                             for (int c = 0; c < 32; ++c)
                                 o[c] = __float_as_uint(__uint_as_float(o[c]) * rescale[rb * 64 + 32 * half + c]);
-                            LAD_TMEM_ST32(ta, o);
+                            tmem_st32u(ta, o);
                         }
                     }
                     tmem_wait_st();
@@ -756,7 +635,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
 #pragma unroll 1
                         for (int half = 0; half < 2; ++half) {
                             uint32_t o[32];
-                            LAD_TMEM_LD32(tmem + lane_addr + kColO + 64 * j + 32 * half, o);
+                            tmem_ld32u(tmem + lane_addr + kColO + 64 * j + 32 * half, o);
                             tmem_wait_ld();
 #pragma unroll
                             for (int c = 0; c < 32; ++c) Od[(32 * half + c) * kDl + d] = __uint_as_float(o[c]);
