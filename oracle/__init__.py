@@ -69,10 +69,11 @@ def _load():
             lib.lado_round_bf16.argtypes = [ctypes.c_int, _dp, _up]
             lib.lado_mla_cache_row.argtypes = [ctypes.c_int] * 3 + [_up, _up, ctypes.POINTER(ctypes.c_longlong),
                                                                     ctypes.c_double, ctypes.c_int, _up]
+            lib.lado_gated_rmsnorm.argtypes = [ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, ctypes.c_double, _dp]
             lib.lado_num_threads_available.argtypes = []
             for f in (lib.lado_kda_recurrent, lib.lado_kda_chunked, lib.lado_l2norm,
                       lib.lado_short_conv_step, lib.lado_mla_decode, lib.lado_mla_decode_paged, lib.lado_rope,
-                      lib.lado_round_bf16, lib.lado_mla_cache_row,
+                      lib.lado_round_bf16, lib.lado_mla_cache_row, lib.lado_gated_rmsnorm,
                       lib.lado_num_threads_available):
                 f.restype = ctypes.c_int
             _lib = lib
@@ -259,3 +260,21 @@ def mla_cache_row(c_kv_bits, k_pe_bits, positions, theta: float = 6.0e6, interle
                                     int(bool(interleaved)), _ptr(out, _up))
     _check(rc, "mla_cache_row")
     return out
+
+
+def gated_rmsnorm(o, g, w=None, eps: float = 1e-5):
+    """KDA output gate: per row of the last axis, o / sqrt(mean(o^2) + eps) * w * sigmoid(g)."""
+    o = np.ascontiguousarray(_f64(o))
+    g = np.ascontiguousarray(_f64(g))
+    assert g.shape == o.shape
+    D = o.shape[-1]
+    flat_o, flat_g = o.reshape(-1, D), g.reshape(-1, D)
+    out = np.empty_like(flat_o)
+    wp = None
+    if w is not None:
+        w = np.ascontiguousarray(_f64(w))
+        assert w.shape == (D,)
+        wp = _ptr(w)
+    rc = _load().lado_gated_rmsnorm(flat_o.shape[0], D, _ptr(flat_o), _ptr(flat_g), wp, float(eps), _ptr(out))
+    _check(rc, "gated_rmsnorm")
+    return out.reshape(o.shape)

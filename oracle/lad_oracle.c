@@ -499,3 +499,27 @@ int lado_mla_cache_row(int n, int Dc, int Dr, const uint16_t *c_kv, const uint16
     }
     return LADO_OK;
 }
+
+/*
+ * Output gate of a KDA head, the epilogue of the decode step ([P2] "How KDA and MLA split the
+ * work": besides q, k, v and the decay, each KDA layer projects an output gate, full-rank). The
+ * page does not give its form; the reading is the gated RMSNorm of the published KDA: per head,
+ *   out = o / sqrt(mean(o^2) + eps) * w * sigmoid(g)
+ * over the head's D output values (w per channel, shared by the heads; w == NULL means 1).
+ * o, g, out: [n][D]; w: [D] or NULL.
+ */
+int lado_gated_rmsnorm(int n, int D, const double *o, const double *g, const double *w, double eps, double *out) {
+    if (n < 0 || D <= 0 || !(eps >= 0.0)) return LADO_EINVAL;
+    for (int r = 0; r < n; ++r) {
+        const double *orow = o + (size_t)r * D;
+        const double *grow = g + (size_t)r * D;
+        double ss = 0.0;
+        for (int d = 0; d < D; ++d) ss += orow[d] * orow[d];
+        const double inv = 1.0 / sqrt(ss / D + eps);
+        for (int d = 0; d < D; ++d) {
+            const double wd = w ? w[d] : 1.0;
+            out[(size_t)r * D + d] = orow[d] * inv * wd / (1.0 + exp(-grow[d]));
+        }
+    }
+    return LADO_OK;
+}
