@@ -11,6 +11,7 @@ A step is one pass of the workload's hot path over one batch of synthetic input:
   mla_decode_b16              one gated MLA layer, 16 sequences, contexts uniform in [8192, 131072]
   mla_decode_b16_paged        the same layer with the cache in 64-row pages of a shuffled pool
   mla_decode_b16_paged_rope   the paged layer with RoPE in the kernels: append the new rows, then attend
+  kda_decode_b64_gated        the same layer with the output gate fused (kda_conv_decode_step_gated)
   kda_mtp_b64                 kda_decode_multi: 64 sequences x 64 heads, 4 tokens per state pass
   kda_prefill_32k             kda_prefill_chunked, 1 x 32768 tokens x 64 heads, chunk 64
 
@@ -328,6 +329,46 @@ class KdaDecodeStep(Step):
                          else _KdaLayer.bytes_decode(B) + _KdaLayer.bytes_conv(B))}
 
 
+class KdaGatedStep(KdaDecodeStep):
+    """The 64 x 64-head KDA layer with the output gate (gated RMSNorm) fused into the step:
+    kda_conv_decode_step_gated."""
+    name = "kda_decode_b64_gated"
+
+    def __init__(self, lad, dev, rank, B=64):
+        super().__init__(lad, dev, rank, B)
+        L = self.layer
+        self.gate = wl.normal_bf16((B, H, D), 1235 + 1000 * rank, "kda_gate", dev, std=2.0)
+        self.norm_w = torch.ones(D, device=dev, dtype=torch.float32)
+        self.h_gate = self.gate.cpu().pin_memory()
+        self.dominant = "kda_conv_decode_step_gated"
+        self.launches_per_step = 1
+        self.config = dict(self.config, workload=self.name, kda_path="fused conv+step+output gate")
+
+    def run(self, timer=None):
+        L = self.layer
+        if timer:
+            timer.begin("kda_conv_decode_step_gated")
+        L.lad.kda_conv_decode_step_gated(L.x, L.tail, L.w, L.alpha, L.beta, L.S, self.gate, self.norm_w, o=L.o)
+        if timer:
+            timer.end("kda_conv_decode_step_gated")
+
+    def run_e2e(self):
+        self.layer.h2d()
+        self.gate.copy_(self.h_gate, non_blocking=True)
+        self.run()
+        self.layer.d2h()
+
+    def e2e_bytes(self):
+        return self.layer.h2d_bytes() + self.h_gate.numel() * 2, self.layer.d2h_bytes()
+
+    def dominant_units(self):
+        return None
+
+    def algorithmic_bytes(self):
+        b = _KdaLayer.bytes_fused(self.layer.B) + self.layer.B * H * D * 2 + D * 4
+        return {"kda_conv_decode_step_gated": b, "step": b}
+
+
 class KdaMultiStep(Step):
     """One KDA layer's multi-token pass: 64 sequences x 64 heads, 4 tokens per sequence (one
     token plus three drafts, the verify step of multi-token prediction) through
@@ -620,6 +661,7 @@ class PrefillStep(Step):
 WORKLOADS = {
     "hybrid_8layer_1m": HybridStep,
     "kda_decode_b64": KdaDecodeStep,
+    "kda_decode_b64_gated": KdaGatedStep,
     "kda_mtp_b64": KdaMultiStep,
     "mla_decode_b16": MlaDecodeStep,
     "mla_decode_b16_paged": MlaPagedStep,
@@ -692,7 +734,7 @@ def cpu_oracle_rate(workload: str, budget_s: float = 20.0) -> dict:
         total_units_tokens = H * float(sum(lens))
         return dt * total_units_tokens / (units * L), f"{units} heads x {L} cached tokens of 1 sequence"
 
-    if workload == "kda_decode_b64":
+    if workload in ("kda_decode_b64", "kda_decode_b64_gated"):
         sec, sample = kda_layer_seconds(64)
         return {"value": 64 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": sample}
     if workload == "kda_mtp_b64":
@@ -749,7 +791,7 @@ def run_reference(args, rank, world):
 
 
 def _tokens(workload):
-    return {"hybrid_8layer_1m": 8, "kda_decode_b64": 64, "kda_mtp_b64": 256, "mla_decode_b16": 16,
+    return {"hybrid_8layer_1m": 8, "kda_decode_b64": 64, "kda_decode_b64_gated": 64, "kda_mtp_b64": 256, "mla_decode_b16": 16,
             "mla_decode_b16_paged": 16, "mla_decode_b16_paged_rope": 16, "kda_prefill_32k": 32768}[workload]
 
 
@@ -833,7 +875,8 @@ def main(argv=None) -> int:
     dom_ms = timer.mean_ms(step.dominant)
     achieved = ab[step.dominant] / (dom_ms / 1000.0) / 1e9
     per_type = {}
-    for kname in ("kda_conv_decode_step", "kda_decode_step", "kda_decode_multi", "mla_latent_decode",
+    for kname in ("kda_conv_decode_step", "kda_conv_decode_step_gated", "kda_decode_step", "kda_decode_multi",
+                  "mla_latent_decode",
                   "mla_latent_decode_paged", "mla_latent_decode_paged_rope", "kda_prefill_chunked"):
         km = timer.mean_ms(kname)
         if km is not None and kname in ab:

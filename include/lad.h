@@ -118,6 +118,24 @@ int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, lon
                     float scale, unsigned flags, void *stream);
 
 /*
+ * kda_conv_decode_step_gated — kda_conv_decode_step with the head's output gate applied to o in
+ * the same kernel. [P2] "How KDA and MLA split the work": each KDA layer also projects an output
+ * gate (a full-rank 4096 -> 8192 projection, one value per output channel). The page does not give
+ * the gate's form; the reading is the gated RMSNorm of the published KDA, per head over its dv
+ * outputs:
+ *   o <- o / sqrt(mean(o^2) + eps) * norm_w * sigmoid(gate)
+ *   gate    bf16 [B][H][dv], 8-byte aligned       gate logits for this token (read)
+ *   norm_w  fp32 [dv] or NULL (all ones), 16-byte aligned   per-channel weight, shared by heads
+ *   eps     finite, >= 0
+ * The other arguments, flags and limits are kda_conv_decode_step's; `scale` scales o before the
+ * norm (so it only matters through eps).
+ */
+int kda_conv_decode_step_gated(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 *conv_w,
+                               const lad_bf16 *conv_bias, const float *alpha, const float *beta, float *S,
+                               const lad_bf16 *gate, const float *norm_w, float eps, void *o, int B, int H, int dk,
+                               int dv, int K, float scale, unsigned flags, void *stream);
+
+/*
  * kda_decode_multi — kda_decode_step for T consecutive tokens per sequence in one pass over the
  * state (read once, written once): the verification step of multi-token prediction, one token
  * plus the drafts ([P1] "What does that mean for serving?": the serving recipe runs MTP with 3

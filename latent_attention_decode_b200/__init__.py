@@ -63,6 +63,8 @@ def _load() -> ctypes.CDLL:
                              _c_int, _c_f, _c_u, _c_vp], _c_int),
         "kda_conv_decode_step": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                                   _c_int, _c_int, _c_f, _c_u, _c_vp], _c_int),
+        "kda_conv_decode_step_gated": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_f, _c_vp,
+                                        _c_int, _c_int, _c_int, _c_int, _c_int, _c_f, _c_u, _c_vp], _c_int),
         "kda_decode_multi": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                               _c_int, _c_int, _c_f, _c_u, _c_vp], _c_int),
         "kda_prefill_chunked": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
@@ -207,6 +209,41 @@ def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: to
     _check("kda_decode_step", _L().kda_decode_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), sq, alpha.data_ptr(),
                                                    beta.data_ptr(), S.data_ptr(), o.data_ptr(), B, H, dk, dv,
                                                    float(scale), flags, _stream(stream)))
+    return o
+
+
+def kda_conv_decode_step_gated(x: torch.Tensor, conv_tail: torch.Tensor, conv_w: torch.Tensor, alpha: torch.Tensor,
+                               beta: torch.Tensor, S: torch.Tensor, gate: torch.Tensor,
+                               norm_w: torch.Tensor | None = None, eps: float = 1e-5, o: torch.Tensor | None = None,
+                               conv_bias: torch.Tensor | None = None, silu: bool = True, l2norm_qk: bool = True,
+                               scale: float = 1.0, out_fp32: bool = False, stream=None) -> torch.Tensor:
+    """kda_conv_decode_step with the output gate (gated RMSNorm) fused: gate bf16 [B,H,128] logits,
+    norm_w fp32 [128] (or None). Returns o [B,H,128]."""
+    bf = torch.bfloat16
+    _contig(x, "x", bf), _contig(conv_tail, "conv_tail", bf), _contig(conv_w, "conv_w", bf)
+    _contig(S, "S", torch.float32), _contig(alpha, "alpha", torch.float32), _contig(beta, "beta", torch.float32)
+    _contig(gate, "gate", bf)
+    B, H, dk, dv = S.shape
+    K = conv_w.shape[1]
+    if x.shape != (B, 3 * H * dk) or conv_tail.shape != (B, K - 1, 3 * H * dk) or conv_w.shape != (3 * H * dk, K):
+        raise ValueError("kda_conv_decode_step_gated: inconsistent conv shapes")
+    if alpha.numel() != B * H * dk or beta.numel() != B * H or gate.shape != (B, H, dv):
+        raise ValueError("alpha must be [B,H,dk], beta [B,H], gate [B,H,dv]")
+    if norm_w is not None:
+        _contig(norm_w, "norm_w", torch.float32)
+        if norm_w.shape != (dv,):
+            raise ValueError("norm_w must be [dv]")
+    if conv_bias is not None:
+        _contig(conv_bias, "conv_bias", bf)
+    odt = torch.float32 if out_fp32 else bf
+    if o is None:
+        o = torch.empty((B, H, dv), device=S.device, dtype=odt)
+    _contig(o, "o", odt)
+    flags = ((FLAG_SILU if silu else 0) | (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0))
+    _check("kda_conv_decode_step_gated", _L().kda_conv_decode_step_gated(
+        x.data_ptr(), conv_tail.data_ptr(), conv_w.data_ptr(), _ptr(conv_bias), alpha.data_ptr(), beta.data_ptr(),
+        S.data_ptr(), gate.data_ptr(), _ptr(norm_w), float(eps), o.data_ptr(), B, H, dk, dv, K, float(scale), flags,
+        _stream(stream)))
     return o
 
 

@@ -49,6 +49,14 @@ __device__ __forceinline__ void add4(float4 &acc, const float4 &x) {
     acc.w += x.w;
 }
 
+// Output gate of the head (kda_conv_decode_step_gated), applied to o in the epilogue:
+// o <- o / sqrt(mean(o^2) + eps) * w * sigmoid(g), g [B][H][128] bf16, w [128] fp32 or null.
+struct GateIn {
+    const uint16_t *g;
+    const float *w;
+    float eps;
+};
+
 // The short convolution of one head's q, k and v channels, fused in front of the step (see
 // kda_conv_decode_step): raw token x [B][3 H 128], tails [B][3][3 H 128], taps [3 H 128][4].
 struct ConvIn {
@@ -63,7 +71,8 @@ template <bool kOutF32, bool kFusedConv>
 __global__ void __launch_bounds__(kThreads, 2)
 kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const uint16_t *__restrict__ v,
                   long long qkv_stride, const float *__restrict__ alpha, const float *__restrict__ beta,
-                  float *__restrict__ S, void *__restrict__ o, int H, float scale, int l2norm, ConvIn cv) {
+                  float *__restrict__ S, void *__restrict__ o, int H, float scale, int l2norm, ConvIn cv,
+                  GateIn gi) {
     const int bh = blockIdx.x;
     const int b = bh / H;
     const int h = bh - b * H;
@@ -79,6 +88,8 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
 
     __shared__ float sq[kD], sk[kD], sv[kD], sa[kD];
     __shared__ float4 red_k[kWarps][kVec], red_q[kWarps][kVec];
+    __shared__ uint2 s_gate[kVec];   // output gate logits, 4 bf16 per lane of warp 0
+    __shared__ float4 s_gw[kVec];    // norm weight, 4 per lane of warp 0
 
     if constexpr (kFusedConv) {
         // y = taps . (tail, x) (+ bias), SiLU; kept in fp32; the tail shifts in place. Threads
@@ -143,6 +154,15 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
     }
     qk *= rq * rk;
 
+    // the gate's inputs are fetched here, to land during the decay and the column sums
+    if (gi.g) {
+        if (threadIdx.x < kVec)
+            s_gate[threadIdx.x] = reinterpret_cast<const uint2 *>(gi.g + static_cast<size_t>(bh) * kD)[threadIdx.x];
+        else if (threadIdx.x < 2 * kVec)
+            s_gw[threadIdx.x - kVec] = gi.w ? reinterpret_cast<const float4 *>(gi.w)[threadIdx.x - kVec]
+                                            : make_float4(1.f, 1.f, 1.f, 1.f);
+    }
+
     // S' = Diag(alpha) S and this warp's share of S'^T k and S'^T q.
     float4 wk = make_float4(0.f, 0.f, 0.f, 0.f), wq = wk;
 #pragma unroll
@@ -187,6 +207,18 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
         ov.y = scale * fmaf(qk, u.y, Q.y);
         ov.z = scale * fmaf(qk, u.z, Q.z);
         ov.w = scale * fmaf(qk, u.w, Q.w);
+        if (gi.g) {
+            // gated RMSNorm over the head's 128 outputs (4 per lane)
+            const float ss = warp_sum(ov.x * ov.x + ov.y * ov.y + ov.z * ov.z + ov.w * ov.w);
+            const float inv = rsqrtf(ss * (1.f / kD) + gi.eps);
+            const uint2 gw = s_gate[lane];
+            const float2 g01 = lad::dev::bf16x2_to_f32(gw.x), g23 = lad::dev::bf16x2_to_f32(gw.y);
+            const float4 w4 = s_gw[lane];
+            ov.x *= inv * w4.x / (1.f + __expf(-g01.x));
+            ov.y *= inv * w4.y / (1.f + __expf(-g01.y));
+            ov.z *= inv * w4.z / (1.f + __expf(-g23.x));
+            ov.w *= inv * w4.w / (1.f + __expf(-g23.y));
+        }
         if constexpr (kOutF32) {
             reinterpret_cast<float4 *>(static_cast<float *>(o) + static_cast<size_t>(bh) * kD)[lane] = ov;
         } else {
@@ -454,41 +486,65 @@ extern "C" int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_b
     const ConvIn none{nullptr, nullptr, nullptr, nullptr, 0};
     if (f32)
         kda_decode_kernel<true, false><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(q, k, v, stride, alpha, beta,
-                                                                                          S, o, H, scale, l2, none);
+                                                                                          S, o, H, scale, l2, none,
+                                                                                          GateIn{});
     else
         kda_decode_kernel<false, false><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(q, k, v, stride, alpha, beta,
-                                                                                           S, o, H, scale, l2, none);
+                                                                                           S, o, H, scale, l2, none,
+                                                                                           GateIn{});
     return lad::check_launch("kda_decode_step");
 }
 
-extern "C" int kda_conv_decode_step(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 *conv_w,
-                                    const lad_bf16 *conv_bias, const float *alpha, const float *beta, float *S, void *o,
-                                    int B, int H, int dk, int dv, int K, float scale, unsigned flags, void *stream) {
+namespace {
+int conv_decode(const char *name, const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 *conv_w,
+                const lad_bf16 *conv_bias, const float *alpha, const float *beta, float *S, const GateIn &gi, void *o,
+                int B, int H, int dk, int dv, int K, float scale, unsigned flags, void *stream) {
     using lad::set_error;
-    if (B < 0 || H < 0) return set_error(LAD_EINVAL, "kda_conv_decode_step: negative B or H");
-    if (dk != kD || dv != kD) return set_error(LAD_EUNSUPPORTED, "kda_conv_decode_step: dk = dv = 128 only");
-    if (K != 4) return set_error(LAD_EUNSUPPORTED, "kda_conv_decode_step: K = 4 only");
+    if (B < 0 || H < 0) return set_error(LAD_EINVAL, "%s: negative B or H", name);
+    if (dk != kD || dv != kD) return set_error(LAD_EUNSUPPORTED, "%s: dk = dv = 128 only", name);
+    if (K != 4) return set_error(LAD_EUNSUPPORTED, "%s: K = 4 only", name);
     if (flags & ~(LAD_FLAG_OUT_FP32 | LAD_FLAG_L2NORM_QK | LAD_FLAG_SILU))
-        return set_error(LAD_EINVAL, "kda_conv_decode_step: unknown flags 0x%x", flags);
+        return set_error(LAD_EINVAL, "%s: unknown flags 0x%x", name, flags);
     if (B == 0 || H == 0) return LAD_OK;
-    if (!x || !conv_tail || !conv_w || !alpha || !beta || !S || !o)
-        return set_error(LAD_EINVAL, "kda_conv_decode_step: null pointer");
+    if (!x || !conv_tail || !conv_w || !alpha || !beta || !S || !o) return set_error(LAD_EINVAL, "%s: null pointer", name);
     if (!lad::aligned(S, 16) || !lad::aligned(conv_w, 8))
-        return set_error(LAD_EUNSUPPORTED, "kda_conv_decode_step: S 16-byte and conv_w 8-byte aligned");
+        return set_error(LAD_EUNSUPPORTED, "%s: S 16-byte and conv_w 8-byte aligned", name);
     const bool f32 = (flags & LAD_FLAG_OUT_FP32) != 0;
-    if (!lad::aligned(o, f32 ? 16 : 8)) return set_error(LAD_EUNSUPPORTED, "kda_conv_decode_step: o misaligned");
+    if (!lad::aligned(o, f32 ? 16 : 8)) return set_error(LAD_EUNSUPPORTED, "%s: o misaligned", name);
+    if (gi.g && (!lad::aligned(gi.g, 8) || (gi.w && !lad::aligned(gi.w, 16))))
+        return set_error(LAD_EUNSUPPORTED, "%s: gate 8-byte and norm weight 16-byte aligned", name);
     const long long blocks = static_cast<long long>(B) * H;
-    if (blocks > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "kda_conv_decode_step: B*H too large");
+    if (blocks > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "%s: B*H too large", name);
     const int l2 = (flags & LAD_FLAG_L2NORM_QK) ? 1 : 0;
     const ConvIn cv{x, conv_tail, conv_w, conv_bias, (flags & LAD_FLAG_SILU) ? 1 : 0};
     cudaStream_t s = lad::as_stream(stream);
     if (f32)
         kda_decode_kernel<true, true><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
-            nullptr, nullptr, nullptr, 0, alpha, beta, S, o, H, scale, l2, cv);
+            nullptr, nullptr, nullptr, 0, alpha, beta, S, o, H, scale, l2, cv, gi);
     else
         kda_decode_kernel<false, true><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
-            nullptr, nullptr, nullptr, 0, alpha, beta, S, o, H, scale, l2, cv);
-    return lad::check_launch("kda_conv_decode_step");
+            nullptr, nullptr, nullptr, 0, alpha, beta, S, o, H, scale, l2, cv, gi);
+    return lad::check_launch(name);
+}
+}  // namespace
+
+extern "C" int kda_conv_decode_step(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 *conv_w,
+                                    const lad_bf16 *conv_bias, const float *alpha, const float *beta, float *S, void *o,
+                                    int B, int H, int dk, int dv, int K, float scale, unsigned flags, void *stream) {
+    return conv_decode("kda_conv_decode_step", x, conv_tail, conv_w, conv_bias, alpha, beta, S, GateIn{}, o, B, H, dk,
+                       dv, K, scale, flags, stream);
+}
+
+extern "C" int kda_conv_decode_step_gated(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 *conv_w,
+                                          const lad_bf16 *conv_bias, const float *alpha, const float *beta, float *S,
+                                          const lad_bf16 *gate, const float *norm_w, float eps, void *o, int B, int H,
+                                          int dk, int dv, int K, float scale, unsigned flags, void *stream) {
+    const char *name = "kda_conv_decode_step_gated";
+    if (B > 0 && H > 0 && !gate) return lad::set_error(LAD_EINVAL, "%s: null gate", name);
+    if (!(eps >= 0.f) || eps == INFINITY) return lad::set_error(LAD_EINVAL, "%s: eps must be finite and >= 0", name);
+    return conv_decode(name, x, conv_tail, conv_w, conv_bias, alpha, beta, S,
+                       GateIn{reinterpret_cast<const uint16_t *>(gate), norm_w, eps}, o, B, H, dk, dv, K, scale, flags,
+                       stream);
 }
 
 extern "C" int kda_decode_multi(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, const float *alpha,

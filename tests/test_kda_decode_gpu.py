@@ -233,3 +233,25 @@ def test_fused_matches_two_calls(lad, cuda_device):
     assert torch.equal(a["tail"], b["tail"])
     expected = rel_l2(o_2[:, 0], o_f)  # the effect of the bf16 conv output alone
     assert abs(rel_l2(o2, o1) - expected) < 0.05 * expected
+
+
+@pytest.mark.parametrize("B,H,with_w", [(64, 64, True), (3, 5, False)])
+def test_fused_gated_output(lad, cuda_device, B, H, with_w):
+    """kda_conv_decode_step_gated: the output gate (gated RMSNorm over each head's 128 outputs)
+    fused into the step; the state and tails are those of the ungated call, bit for bit."""
+    cfg = wl.KdaDecode("gate", B=B, H=H, seed=50 + B)
+    a = wl.kda_decode_inputs(cfg, cuda_device)
+    b = {n: t.clone() for n, t in a.items()}
+    gate = wl.normal_bf16((B, H, 128), 50, "gate", cuda_device, std=2.0)
+    w = (wl.normal((128,), 50, "normw", cuda_device) * 0.2 + 1.0) if with_w else None
+    o_ref, S_ref, tail_ref = _fused_oracle(a, H)
+    want = oracle.gated_rmsnorm(o_ref, f64(gate), None if w is None else f64(w), eps=1e-5)
+    o = lad.kda_conv_decode_step_gated(a["x"], a["tail"], a["w"], a["alpha"], a["beta"], a["S"], gate, w,
+                                       eps=1e-5, out_fp32=True)
+    lad.kda_conv_decode_step(b["x"], b["tail"], b["w"], b["alpha"], b["beta"], b["S"], out_fp32=True)
+    torch.cuda.synchronize()
+    assert rel_l2(o, want) < 1e-4
+    assert torch.equal(a["S"], b["S"]) and torch.equal(a["tail"], b["tail"])
+    assert np.array_equal(f64(a["tail"]), tail_ref) and rel_l2(a["S"], S_ref) < TOL_STATE
+    o16 = lad.kda_conv_decode_step_gated(b["x"], b["tail"], b["w"], b["alpha"], b["beta"], b["S"].clone(), gate, w)
+    assert o16.dtype == torch.bfloat16
