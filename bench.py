@@ -558,8 +558,14 @@ class HybridStep(Step):
                        "l2": "inputs larger than L2 (9.2 GB latent cache + 235 MB KDA state per step)"}
 
     def run(self, timer=None):
+        # the seven KDA layers are timed as one bracket (short kernels: see KernelTimer)
+        kname = "kda_conv_decode_step" if _KdaLayer.fused else None
+        if timer and kname:
+            timer.begin(kname, count=len(self.kda))
         for layer in self.kda:
-            layer.run(timer)
+            layer.run(None if kname else timer)
+        if timer and kname:
+            timer.end(kname)
         self.mla.run(timer)
 
     def run_e2e(self):
@@ -671,15 +677,17 @@ WORKLOADS = {
 
 
 class KernelTimer:
-    """CUDA events around each launch of named kernels, on the current (launching) stream."""
+    """CUDA events around each launch of named kernels, on the current (launching) stream. A pair
+    may bracket `count` back-to-back launches of the same kernel (then it is timed per launch as
+    the bracket's time / count), which keeps the events' own cost out of short kernels."""
 
     def __init__(self):
         self.pairs: dict[str, list] = {}
 
-    def begin(self, name):
+    def begin(self, name, count: int = 1):
         e = torch.cuda.Event(enable_timing=True)
         e.record()
-        self.pairs.setdefault(name, []).append([e, None])
+        self.pairs.setdefault(name, []).append([e, None, count])
 
     def end(self, name):
         e = torch.cuda.Event(enable_timing=True)
@@ -690,7 +698,7 @@ class KernelTimer:
         ps = self.pairs.get(name)
         if not ps:
             return None
-        return sum(a.elapsed_time(b) for a, b in ps) / len(ps)
+        return sum(a.elapsed_time(b) for a, b, _ in ps) / sum(n for _, _, n in ps)
 
 
 # ---------------------------------------------------------------------------------------------
