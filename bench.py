@@ -362,7 +362,7 @@ class KdaGatedStep(KdaDecodeStep):
         return self.layer.h2d_bytes() + self.h_gate.numel() * 2, self.layer.d2h_bytes()
 
     def dominant_units(self):
-        return None
+        return self.layer.B * H
 
     def algorithmic_bytes(self):
         b = _KdaLayer.bytes_fused(self.layer.B) + self.layer.B * H * D * 2 + D * 4
