@@ -18,13 +18,13 @@
 //
 // Per chunk (two warpgroups; warp 0 issues the MMAs, converged, elect.sync):
 //   1. load q, k, alpha, v, beta; running products g; write the operand tiles
-//   2. MMA  [Qt; Kt] Kh^T  (M = 128: rows 0-63 give Qt Kh^T, rows 64-127 give Kt Kh^T)
-//   3. lower(Qt Kh^T) -> operand; A -> fp32 scratch; T = (I + A)^-1 by 16x16 blocked forward
-//      substitution on the CUDA cores; Tb -> operand
-//   4. MMA  W^T = Kt^T Tb^T,  U' = Tb V;   W -> operand
-//   5. MMA  X = W S0;  U = U' - X -> operand
-//   6. MMA  O = Qt S0 + lower(Qt Kh^T) U;  S += Kh^T U
-//   7. O -> HBM; S <- Diag(g_last) S in TMEM, and -> next chunk's S0 operand (HBM after the last)
+//   2. MMA  [Qt; Kt] Kh^T  (M = 128: rows 0-63 give Qt Kh^T, rows 64-127 give Kt Kh^T), and
+//           Y = Kt S0 (it needs no T: W S0 = Tb (Kt S0), so W itself is never formed)
+//   3. lower(Qt Kh^T) -> operand; A -> fp32 scratch; Y -> operand; T = (I + A)^-1 by 16x16
+//      blocked forward substitution on the CUDA cores; Tb -> operand
+//   4. MMA  U' = Tb V,  X = Tb Y;  U = U' - X -> operand
+//   5. MMA  O = Qt S0 + lower(Qt Kh^T) U;  S += Kh^T U
+//   6. O -> HBM; S <- Diag(g_last) S in TMEM, and -> next chunk's S0 operand (HBM after the last)
 // Every operand tile is K-major fp32 with the 128-byte swizzle (tf32 operands read MN-major
 // would need a different swizzle; storing the transposes instead keeps one layout): the tiles
 // that a contraction needs "the other way round" (Kt^T, Kh^T, V^T / U^T, S0^T) are written
@@ -57,7 +57,7 @@ constexpr uint32_t kOffXQK = 0;        // [Qt; Kt]: 128 rows (tokens) x 128 (d_k
 constexpr uint32_t kOffTT = 8192;      //   Tb [64 r][64 s] in the Kt half of XQK blocks 0-1 (stride 16 KiB)
 constexpr uint32_t kOffQM = 40960;     //   lower(Qt Kh^T) [64][64] in the Kt half of blocks 2-3
 constexpr uint32_t kOffKH = 65536;     // Kh [64 tokens][128 d_k], stride 8 KiB; then A/T scratch; then W
-constexpr uint32_t kOffKTT = 98304;    // Kt^T [128 d_k][64 tokens], stride 16 KiB
+constexpr uint32_t kOffYT = 98304;     // Y^T = (Kt S0)^T [64 d_v][64 tokens], stride 8 KiB
 constexpr uint32_t kOffKHT = 131072;   // Kh^T [128 d_k][64 tokens], stride 16 KiB
 constexpr uint32_t kOffVT = 163840;    // V^T, then U^T: [64 d_v][64 tokens], stride 8 KiB
 constexpr uint32_t kOffSOT = 180224;   // S0^T [64 d_v][128 d_k], stride 8 KiB
@@ -66,8 +66,8 @@ constexpr uint32_t kStr16 = 16384, kStr8 = 8192;
 constexpr uint32_t kMiscBeta = 0, kMiscRq = 256, kMiscRk = 512, kMiscGc = 768, kMiscBar = 1280, kMiscTmem = 1288,
                    kMiscAbort = 1292, kMiscTmaBar = 1296, kMiscOct = 2048;  // s_oct: [8 octets][128] fp32
 // Raw inputs of the next chunk, TMA-staged over tiles that are dead once a chunk's last MMA has
-// completed (Kt^T, Kh^T and U^T): alpha [64][128] fp32, q and k [64][128] bf16, v [64][64] bf16.
-constexpr uint32_t kOffStA = kOffKTT;            // 32 KiB
+// completed (Y^T, Kh^T and U^T): alpha [64][128] fp32, q and k [64][128] bf16, v [64][64] bf16.
+constexpr uint32_t kOffStA = kOffYT;             // 32 KiB
 constexpr uint32_t kOffStQ = kOffStA + 32768;    // 16 KiB
 constexpr uint32_t kOffStK = kOffStQ + 16384;    // 16 KiB
 constexpr uint32_t kOffStV = kOffStK + 16384;    // 8 KiB, ends inside the V^T tile
@@ -77,9 +77,9 @@ constexpr uint32_t kSmemBytes = kOffMisc + kMiscOct + 8 * 128 * 4 + 1024;  // + 
 // TMEM columns (fp32)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc1 = 0;    // M=128 x 64: [Qt Kh^T ; Kt Kh^T]
-constexpr uint32_t kColWT = 64;     // M=128 x 64: W^T (rows d_k, columns r)
+constexpr uint32_t kColY = 64;      // M=64 x 64: Y = Kt S0
 constexpr uint32_t kColU = 128;     // M=64 x 64: U' = Tb V
-constexpr uint32_t kColX = 192;     // M=64 x 64: W S0
+constexpr uint32_t kColX = 192;     // M=64 x 64: Tb Y = W S0
 constexpr uint32_t kColO = 256;     // M=64 x 64
 constexpr uint32_t kColS = 320;     // M=128 x 64: state master (rows d_k)
 
@@ -317,30 +317,30 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
             float vv[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) vv[r] = bf16_to_f32(sv[(r0 + r) * kDvh + j]);
-            __syncthreads();  // the staging area is read; Kt^T, Kh^T and V^T overwrite it
+            __syncthreads();  // the staging area is read; Kh^T and V^T overwrite it
 #pragma unroll
             for (int r = 0; r < 16; r += 4) st_tile4(sm + kOffVT, j, r0 + r, kStr8, vv[r], vv[r + 1], vv[r + 2], vv[r + 3]);
-            // Kt^T and Kh^T: thread -> channel i (row), tokens of half th, from the tiles above
+            // Kh^T: thread -> channel i (row), tokens of half th, from the tile above
             const int i = tid & (kDk - 1), th = tid >> 7;
-#pragma unroll 2
+#pragma unroll 4
             for (int r = (kC / 2) * th; r < (kC / 2) * (th + 1); r += 4) {
-                float kt[4], kh[4];
+                float kh[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    kt[u] = *reinterpret_cast<const float *>(sm + kOffXQK + sw128_off32(kC + r + u, i, kStr16));
+                for (int u = 0; u < 4; ++u)
                     kh[u] = *reinterpret_cast<const float *>(sm + kOffKH + sw128_off32(r + u, i, kStr8));
-                }
-                st_tile4(sm + kOffKTT, i, r, kStr16, kt[0], kt[1], kt[2], kt[3]);
                 st_tile4(sm + kOffKHT, i, r, kStr16, kh[0], kh[1], kh[2], kh[3]);
             }
         }
 
-        // ---- 2. [Qt; Kt] Kh^T ----
+        // ---- 2. [Qt; Kt] Kh^T and Y = Kt S0 (Kt: rows 64-127 of the [Qt; Kt] tile) ----
         ok = mma_sync([&] {
 #pragma unroll
-            for (int j = 0; j < kDk / 8; ++j)
+            for (int j = 0; j < kDk / 8; ++j) {
+                const uint64_t sot = kdesc(d0 + (kOffSOT >> 4), kStr8, j);
                 tc_mma_tf32(tmem + kColAcc1, kdesc(d0 + (kOffXQK >> 4), kStr16, j), kdesc(d0 + (kOffKH >> 4), kStr8, j),
                             kIdesc128, j > 0);
+                tc_mma_tf32(tmem + kColY, kdesc(d0 + ((kOffXQK + kC * 128) >> 4), kStr16, j), sot, kIdesc64, j > 0);
+            }
         });
         if (!ok) break;
 
@@ -365,6 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
                 for (int j = 0; j < 32; j += 4)
                     dst[j / 4] = make_float4(c0 + j < r ? br * x[j] : 0.f, c0 + j + 1 < r ? br * x[j + 1] : 0.f,
                                              c0 + j + 2 < r ? br * x[j + 2] : 0.f, c0 + j + 3 < r ? br * x[j + 3] : 0.f);
+            }
+            // Y [token][d_v] (M = 64 rows: lanes 0-15) -> Y^T operand
+            float y[32];
+            tmem_ld32(tmem + lane_base + kColY + 32 * cg, y);
+            tmem_wait_ld();
+            if (lane < 16) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) st_tile1(sm + kOffYT, 32 * cg + j, row64, kStr8, y[j]);
             }
         }
         __syncthreads();
@@ -441,31 +449,14 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
             }
         }
 
-        // ---- 4. W^T = Kt^T Tb^T (M = 128 d_k),  U' = Tb V (B = V^T) ----
+        // ---- 4. U' = Tb V (B = V^T),  X = Tb Y (B = Y^T);  U = U' - X -> U^T operand ----
         ok = mma_sync([&] {
 #pragma unroll
             for (int j = 0; j < kC / 8; ++j) {
                 const uint64_t tt = kdesc(d0 + (kOffTT >> 4), kStr16, j);
-                tc_mma_tf32(tmem + kColWT, kdesc(d0 + (kOffKTT >> 4), kStr16, j), tt, kIdesc128, j > 0);
                 tc_mma_tf32(tmem + kColU, tt, kdesc(d0 + (kOffVT >> 4), kStr8, j), kIdesc64, j > 0);
+                tc_mma_tf32(tmem + kColX, tt, kdesc(d0 + (kOffYT >> 4), kStr8, j), kIdesc64, j > 0);
             }
-        });
-        if (!ok) break;
-        // W [r][d_k] -> operand in the Kh slot: this thread has W^T row row128 (= d_k), 32 tokens
-        {
-            float w[32];
-            tmem_ld32(tmem + lane_base + kColWT + 32 * cg, w);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) st_tile1(sm + kOffKH, 32 * cg + j, row128, kStr8, w[j]);
-        }
-
-        // ---- 5. X = W S0 (B = S0^T);  U = U' - X -> U^T operand ----
-        ok = mma_sync([&] {
-#pragma unroll
-            for (int j = 0; j < kDk / 8; ++j)
-                tc_mma_tf32(tmem + kColX, kdesc(d0 + (kOffKH >> 4), kStr8, j), kdesc(d0 + (kOffSOT >> 4), kStr8, j),
-                            kIdesc64, j > 0);
         });
         if (!ok) break;
         {
@@ -479,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
             }
         }
 
-        // ---- 6. O = Qt S0 + lower(Qt Kh^T) U;  S += Kh^T U ----
+        // ---- 5. O = Qt S0 + lower(Qt Kh^T) U;  S += Kh^T U ----
         ok = mma_sync([&] {
 #pragma unroll
             for (int j = 0; j < kDk / 8; ++j)
@@ -494,8 +485,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
         });
         if (!ok) break;
 
-        // ---- 7. O -> HBM; S <- Diag(g_last) S (TMEM), S^T -> operand (HBM after the last chunk) ----
-        if (ch + 1 < nchunks) {  // Kt^T, Kh^T, U^T are dead now
+        // ---- 6. O -> HBM; S <- Diag(g_last) S (TMEM), S^T -> operand (HBM after the last chunk) ----
+        if (ch + 1 < nchunks) {  // Y^T, Kh^T, U^T are dead now
             if (tid == 0) stage(ch + 1);
             pending = 1;
         }
