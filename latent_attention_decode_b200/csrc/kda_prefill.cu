@@ -19,11 +19,12 @@
 // Per chunk (two warpgroups; warp 0 issues the MMAs, converged, elect.sync):
 //   1. load q, k, alpha, v, beta; running products g; write the operand tiles
 //   2. MMA  [Qt; Kt] Kh^T  (M = 128: rows 0-63 give Qt Kh^T, rows 64-127 give Kt Kh^T), and
-//           Y = Kt S0 (it needs no T: W S0 = Tb (Kt S0), so W itself is never formed)
+//           Y = Kt S0 (it needs no T: W S0 = Tb (Kt S0), so W itself is never formed); then
+//           O = Qt S0 is issued without waiting, to run during step 3
 //   3. lower(Qt Kh^T) -> operand; A -> fp32 scratch; Y -> operand; T = (I + A)^-1 by 16x16
 //      blocked forward substitution on the CUDA cores; Tb -> operand
 //   4. MMA  U' = Tb V,  X = Tb Y;  U = U' - X -> operand
-//   5. MMA  O = Qt S0 + lower(Qt Kh^T) U;  S += Kh^T U
+//   5. MMA  O += lower(Qt Kh^T) U;  S += Kh^T U
 //   6. O -> HBM; S <- Diag(g_last) S in TMEM, and -> next chunk's S0 operand (HBM after the last)
 // Every operand tile is K-major fp32 with the 128-byte swizzle (tf32 operands read MN-major
 // would need a different swizzle; storing the transposes instead keeps one layout): the tiles
@@ -343,6 +344,15 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
             }
         });
         if (!ok) break;
+        // O = Qt S0 needs nothing of this chunk's solve and Qt and S0^T stay put until the chunk ends:
+        // issued now, it runs while the CUDA cores solve; the commit after step 5's MMAs covers it
+        if (warp == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < kDk / 8; ++j)
+                tc_mma_tf32(tmem + kColO, kdesc(d0 + (kOffXQK >> 4), kStr16, j), kdesc(d0 + (kOffSOT >> 4), kStr8, j),
+                            kIdesc64, j > 0);
+        }
 
         // ---- 3a. lower(Qt Kh^T) -> QM (rows 0-63); A = strict_lower(diag(beta) Kt Kh^T) -> fp32
         //          scratch (rows 64-127); each thread has 32 of the 64 columns of its row ----
@@ -400,13 +410,52 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
             }
         }
         __syncthreads();
-        // block rows 1..3: T_ij = -T_ii * sum_{k=j}^{i-1} A_ik T_kj; a thread computes a 1x4 strip
+        // Off-diagonal blocks: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj = -sum_k M_ik T_kj with
+        // M_ik = T_ii A_ik, which needs only the diagonal blocks: all six M blocks in one pass (kept in
+        // A's place), then one pass per block row. A thread computes 1x4 strips (row rr, columns cc).
+        {
+            // M_ik for (i, k) = (1,0), (2,0), (2,1), (3,0), (3,1), (3,2): 6 blocks x 64 strips
+            float4 m[2];
+            int mi[2], mk[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int e = tid + h * kThreads;
+                m[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+                mi[h] = -1;
+                if (e < 6 * 64) {
+                    const int blk = e >> 6, rr = (e >> 2) & 15, cc = (e & 3) * 4;
+                    const int i = blk == 0 ? 1 : (blk < 3 ? 2 : 3);
+                    const int k = blk == 0 ? 0 : (blk < 3 ? blk - 1 : blk - 3);
+                    mi[h] = i;
+                    mk[h] = k;
+#pragma unroll
+                    for (int ss = 0; ss < 16; ++ss) {
+                        const float t = Tpl[(16 * i + rr) * 64 + 16 * i + ss];
+                        const float4 a4 = *reinterpret_cast<const float4 *>(Apl + (16 * i + ss) * 64 + 16 * k + cc);
+                        m[h].x = fmaf(t, a4.x, m[h].x);
+                        m[h].y = fmaf(t, a4.y, m[h].y);
+                        m[h].z = fmaf(t, a4.z, m[h].z);
+                        m[h].w = fmaf(t, a4.w, m[h].w);
+                    }
+                }
+            }
+            __syncthreads();  // every read of A is done: the M blocks replace it
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int e = tid + h * kThreads;
+                if (mi[h] >= 0) {
+                    const int rr = (e >> 2) & 15, cc = (e & 3) * 4;
+                    *reinterpret_cast<float4 *>(Apl + (16 * mi[h] + rr) * 64 + 16 * mk[h] + cc) = m[h];
+                }
+            }
+            __syncthreads();
+        }
 #pragma unroll 1
         for (int bi = 1; bi < 4; ++bi) {
-            const bool act = tid < bi * 64;
-            const int bj = tid >> 6, rr = (tid >> 2) & 15, cc = (tid & 3) * 4;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (act) {
+            // block row bi: blocks bj < bi, one strip per thread (bi * 64 threads)
+            if (tid < bi * 64) {
+                const int bj = tid >> 6, rr = (tid >> 2) & 15, cc = (tid & 3) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int kb = bj; kb < bi; ++kb) {
 #pragma unroll
                     for (int ss = 0; ss < 16; ++ss) {
@@ -418,24 +467,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
                         acc.w = fmaf(a, t4.w, acc.w);
                     }
                 }
+                *reinterpret_cast<float4 *>(Tpl + (16 * bi + rr) * 64 + 16 * bj + cc) =
+                    make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
             }
-            __syncthreads();
-            if (act) *reinterpret_cast<float4 *>(Tpl + (16 * bi + rr) * 64 + 16 * bj + cc) = acc;  // R_j, for now
-            __syncthreads();
-            float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (act) {
-#pragma unroll
-                for (int ss = 0; ss < 16; ++ss) {
-                    const float t = Tpl[(16 * bi + rr) * 64 + 16 * bi + ss];
-                    const float4 r4 = *reinterpret_cast<const float4 *>(Tpl + (16 * bi + ss) * 64 + 16 * bj + cc);
-                    out.x = fmaf(-t, r4.x, out.x);
-                    out.y = fmaf(-t, r4.y, out.y);
-                    out.z = fmaf(-t, r4.z, out.z);
-                    out.w = fmaf(-t, r4.w, out.w);
-                }
-            }
-            __syncthreads();
-            if (act) *reinterpret_cast<float4 *>(Tpl + (16 * bi + rr) * 64 + 16 * bj + cc) = out;
             __syncthreads();
         }
         // Tb = T diag(beta) -> operand tile (thread -> row tid/4, 16 columns)
@@ -470,12 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
             }
         }
 
-        // ---- 5. O = Qt S0 + lower(Qt Kh^T) U;  S += Kh^T U ----
+        // ---- 5. O += lower(Qt Kh^T) U;  S += Kh^T U ----
         ok = mma_sync([&] {
-#pragma unroll
-            for (int j = 0; j < kDk / 8; ++j)
-                tc_mma_tf32(tmem + kColO, kdesc(d0 + (kOffXQK >> 4), kStr16, j), kdesc(d0 + (kOffSOT >> 4), kStr8, j),
-                            kIdesc64, j > 0);
 #pragma unroll
             for (int j = 0; j < kC / 8; ++j) {
                 const uint64_t ut = kdesc(d0 + (kOffVT >> 4), kStr8, j);
