@@ -206,15 +206,25 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
     }
 
     // the next chunk's raw inputs, staged by TMA (thread 0); rows past T read as zeros
-    auto stage = [&](int chunk) {
+    // One barrier phase per chunk's staging, expecting all its bytes at once: alpha (over Y^T, dead
+    // once step 4's MMAs are complete) goes first, q, k and v (over Kh^T and U^T) after step 5.
+    auto stage_alpha = [&](int chunk) {
         fence_async_smem();
         mbar_arrive_tx_raw(tma_bar, kStageTx);
+        tma_load_3d(sbase + kOffStA, &maps.alpha, h * kDk, chunk * kC, b, tma_bar);
+    };
+    auto stage_qkv = [&](int chunk) {
+        fence_async_smem();
         const int t = chunk * kC;
-        tma_load_3d(sbase + kOffStA, &maps.alpha, h * kDk, t, b, tma_bar);
         tma_load_3d(sbase + kOffStQ, &maps.q, h * kDk, t, b, tma_bar);
         tma_load_3d(sbase + kOffStK, &maps.k, h * kDk, t, b, tma_bar);
         tma_load_3d(sbase + kOffStV, &maps.v, h * kDv + half * kDvh, t, b, tma_bar);
     };
+    auto stage = [&](int chunk) {
+        stage_alpha(chunk);
+        stage_qkv(chunk);
+    };
+    int qkv_owed = -1;  // a chunk whose alpha is staged but whose q, k, v are not yet
     uint32_t tma_phase = 0;
     int pending = 0;  // a staging copy is in flight
     const int nchunks = (p.T + kC - 1) / kC;
@@ -398,15 +408,20 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
                 for (int ss = 0; ss < rr; ++ss) acc -= Apl[(base + rr) * 64 + base + ss] * t[ss];
                 t[rr] = acc;
             }
+            const float bc = s_beta[base + c];
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) Tpl[(base + rr) * 64 + base + c] = t[rr];
+            for (int rr = 0; rr < 16; ++rr) {
+                Tpl[(base + rr) * 64 + base + c] = t[rr];
+                st_tile1(sm + kOffTT, base + rr, base + c, kStr16, t[rr] * bc);  // Tb = T diag(beta)
+            }
         } else {
-            // zero the blocks above the diagonal: (bi, bj) with bi < bj, 4 floats per store
+            // zero the blocks above the diagonal, in T and in the Tb operand: (bi, bj) with bi < bj
             for (int e = tid - kC; e < 6 * 64; e += kThreads - kC) {
                 const int blk = e >> 6, rr = (e >> 2) & 15, cc = (e & 3) * 4;
                 const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
                 const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
                 *reinterpret_cast<float4 *>(Tpl + (16 * bi + rr) * 64 + 16 * bj + cc) = make_float4(0.f, 0.f, 0.f, 0.f);
+                st_tile4(sm + kOffTT, 16 * bi + rr, 16 * bj + cc, kStr16, 0.f, 0.f, 0.f, 0.f);
             }
         }
         __syncthreads();
@@ -469,20 +484,12 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
                 }
                 *reinterpret_cast<float4 *>(Tpl + (16 * bi + rr) * 64 + 16 * bj + cc) =
                     make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+                const int c = 16 * bj + cc;
+                st_tile4(sm + kOffTT, 16 * bi + rr, c, kStr16, -acc.x * s_beta[c], -acc.y * s_beta[c + 1],
+                         -acc.z * s_beta[c + 2], -acc.w * s_beta[c + 3]);
             }
             __syncthreads();
         }
-        // Tb = T diag(beta) -> operand tile (thread -> row tid/4, 16 columns)
-        {
-            const int r = tid >> 2, jc = (tid & 3) * 16;
-#pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-                const float4 t4 = *reinterpret_cast<const float4 *>(Tpl + r * 64 + jc + j);
-                st_tile4(sm + kOffTT, r, jc + j, kStr16, t4.x * s_beta[jc + j], t4.y * s_beta[jc + j + 1],
-                         t4.z * s_beta[jc + j + 2], t4.w * s_beta[jc + j + 3]);
-            }
-        }
-
         // ---- 4. U' = Tb V (B = V^T),  X = Tb Y (B = Y^T);  U = U' - X -> U^T operand ----
         ok = mma_sync([&] {
 #pragma unroll
@@ -493,6 +500,11 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
             }
         });
         if (!ok) break;
+        if (ch + 1 < nchunks) {  // Y^T is dead now: the next chunk's alpha can come in
+            if (tid == 0) stage_alpha(ch + 1);
+            pending = 1;
+            qkv_owed = ch + 1;
+        }
         {
             float u[32], x[32];
             tmem_ld32(tmem + lane_base + kColU + 32 * cg, u);
@@ -516,9 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
         if (!ok) break;
 
         // ---- 6. O -> HBM; S <- Diag(g_last) S (TMEM), S^T -> operand (HBM after the last chunk) ----
-        if (ch + 1 < nchunks) {  // Y^T, Kh^T, U^T are dead now
-            if (tid == 0) stage(ch + 1);
-            pending = 1;
+        if (qkv_owed >= 0) {  // Kh^T and U^T are dead now
+            if (tid == 0) stage_qkv(qkv_owed);
+            qkv_owed = -1;
         }
         {
             float ov[32];
@@ -566,6 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
 
     // drain: a staging copy still in flight (after an abort) lands, and every MMA this CTA
     // issued completes, before shared memory and TMEM are released
+    if (tid == 0 && qkv_owed >= 0) stage_qkv(qkv_owed);  // the phase expects those bytes too
     if (tid == 0 && pending) {
         const uint64_t t0 = lad::dev::globaltimer_ns();
         while (!mbar_try_wait(tma_bar, tma_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
