@@ -36,6 +36,7 @@ _lib = None
 _dp = ctypes.POINTER(ctypes.c_double)
 _ip = ctypes.POINTER(ctypes.c_int)
 _up = ctypes.POINTER(ctypes.c_uint16)
+_bp = ctypes.POINTER(ctypes.c_uint8)
 
 
 def build(force: bool = False) -> str:
@@ -70,10 +71,20 @@ def _load():
             lib.lado_mla_cache_row.argtypes = [ctypes.c_int] * 3 + [_up, _up, ctypes.POINTER(ctypes.c_longlong),
                                                                     ctypes.c_double, ctypes.c_int, _up]
             lib.lado_gated_rmsnorm.argtypes = [ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, ctypes.c_double, _dp]
+            lib.lado_e4m3_decode.argtypes = [ctypes.c_int, _bp, _dp]
+            lib.lado_e4m3_encode.argtypes = [ctypes.c_int, _dp, _bp]
+            lib.lado_mla_decode_fp8.argtypes = ([ctypes.c_int] * 4 + [ctypes.c_longlong, _dp, _bp, ctypes.c_double,
+                                                _ip, _dp, ctypes.c_double, _dp, _dp, ctypes.c_int])
+            lib.lado_mla_decode_paged_fp8.argtypes = ([ctypes.c_int] * 7 + [_dp, _bp, ctypes.c_double, _ip, _ip, _dp,
+                                                      ctypes.c_double, _dp, _dp, ctypes.c_int])
+            lib.lado_mla_cache_row_fp8.argtypes = ([ctypes.c_int] * 3 + [_up, _up, ctypes.POINTER(ctypes.c_longlong),
+                                                   ctypes.c_double, ctypes.c_int, ctypes.c_double, _bp])
             lib.lado_num_threads_available.argtypes = []
             for f in (lib.lado_kda_recurrent, lib.lado_kda_chunked, lib.lado_l2norm,
                       lib.lado_short_conv_step, lib.lado_mla_decode, lib.lado_mla_decode_paged, lib.lado_rope,
                       lib.lado_round_bf16, lib.lado_mla_cache_row, lib.lado_gated_rmsnorm,
+                      lib.lado_e4m3_decode, lib.lado_e4m3_encode, lib.lado_mla_decode_fp8,
+                      lib.lado_mla_decode_paged_fp8, lib.lado_mla_cache_row_fp8,
                       lib.lado_num_threads_available):
                 f.restype = ctypes.c_int
             _lib = lib
@@ -221,6 +232,70 @@ def mla_decode_paged(q, page_bits, block_table, seq_lens, gate=None, scale: floa
     return o, lse
 
 
+def e4m3_decode(codes) -> np.ndarray:
+    """float64 values of E4M3 codes (uint8, any shape)."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, dtype=np.float64)
+    _check(_load().lado_e4m3_decode(c.size, _ptr(c, _bp), _ptr(out)), "e4m3_decode")
+    return out
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest E4M3 codes of float64 values (ties to even, saturating at +-448, NaN to 0x7F)."""
+    x = np.ascontiguousarray(_f64(x))
+    out = np.empty(x.shape, dtype=np.uint8)
+    _check(_load().lado_e4m3_encode(x.size, _ptr(x), _ptr(out, _bp)), "e4m3_encode")
+    return out
+
+
+def mla_decode_fp8(q, cache_codes, kv_scale: float, seq_lens, gate=None, scale: float = 192 ** -0.5,
+                   d_latent: int = 512, nthreads: int = 1):
+    """mla_decode over an FP8 cache: cache_codes uint8 E4M3 codes [B,Lmax,D], each element worth
+    kv_scale * E4M3(code). Returns (o [B,H,d_latent], lse [B,H]) in float64."""
+    q = _f64(q)
+    codes = np.ascontiguousarray(cache_codes, dtype=np.uint8)
+    B, H, D = q.shape
+    assert codes.ndim == 3 and codes.shape[0] == B and codes.shape[2] == D
+    lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    assert lens.shape == (B,) and (lens <= codes.shape[1]).all()
+    o = np.zeros((B, H, d_latent), dtype=np.float64)
+    lse = np.zeros((B, H), dtype=np.float64)
+    gptr = None
+    if gate is not None:
+        gate = _f64(gate)
+        gptr = _ptr(gate)
+    rc = _load().lado_mla_decode_fp8(B, H, d_latent, D - d_latent, codes.shape[1] * D, _ptr(q), _ptr(codes, _bp),
+                                     float(kv_scale), _ptr(lens, _ip), gptr, float(scale), _ptr(o), _ptr(lse),
+                                     int(nthreads))
+    _check(rc, "mla_decode_fp8")
+    return o, lse
+
+
+def mla_decode_paged_fp8(q, page_codes, kv_scale: float, block_table, seq_lens, gate=None,
+                         scale: float = 192 ** -0.5, d_latent: int = 512, nthreads: int = 1):
+    """mla_decode_paged over an FP8 page pool: page_codes uint8 E4M3 codes [num_pages, P, D]."""
+    q = _f64(q)
+    codes = np.ascontiguousarray(page_codes, dtype=np.uint8)
+    B, H, D = q.shape
+    assert codes.ndim == 3 and codes.shape[2] == D
+    num_pages, P = codes.shape[0], codes.shape[1]
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    assert bt.ndim == 2 and bt.shape[0] == B
+    lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    assert lens.shape == (B,)
+    o = np.zeros((B, H, d_latent), dtype=np.float64)
+    lse = np.zeros((B, H), dtype=np.float64)
+    gptr = None
+    if gate is not None:
+        gate = _f64(gate)
+        gptr = _ptr(gate)
+    rc = _load().lado_mla_decode_paged_fp8(B, H, d_latent, D - d_latent, P, num_pages, bt.shape[1], _ptr(q),
+                                           _ptr(codes, _bp), float(kv_scale), _ptr(bt, _ip), _ptr(lens, _ip), gptr,
+                                           float(scale), _ptr(o), _ptr(lse), int(nthreads))
+    _check(rc, "mla_decode_paged_fp8")
+    return o, lse
+
+
 def rope(x, positions, theta: float = 6.0e6, interleaved: bool = False):
     """Rotary embedding of the last axis of x (even width D) by positions (one per row of the
     leading axes, broadcast over any axes between). Returns float64 of x's shape."""
@@ -243,6 +318,23 @@ def round_bf16_bits(x) -> np.ndarray:
     x = np.ascontiguousarray(_f64(x))
     out = np.empty(x.shape, dtype=np.uint16)
     _check(_load().lado_round_bf16(x.size, _ptr(x), _ptr(out, _up)), "round_bf16")
+    return out
+
+
+def mla_cache_row_fp8(c_kv_bits, k_pe_bits, positions, kv_scale: float, theta: float = 6.0e6,
+                      interleaved: bool = False) -> np.ndarray:
+    """New FP8 latent-cache rows (E4M3 codes [n, Dc + Dr]): each element of the row that
+    mla_cache_row would round to bf16 is divided by kv_scale in fp32 and rounded to E4M3."""
+    c = np.ascontiguousarray(c_kv_bits, dtype=np.uint16)
+    k = np.ascontiguousarray(k_pe_bits, dtype=np.uint16)
+    n, Dc = c.shape
+    Dr = k.shape[1]
+    pos = np.ascontiguousarray(positions, dtype=np.int64)
+    out = np.empty((n, Dc + Dr), dtype=np.uint8)
+    rc = _load().lado_mla_cache_row_fp8(n, Dc, Dr, _ptr(c, _up), _ptr(k, _up),
+                                        pos.ctypes.data_as(ctypes.POINTER(ctypes.c_longlong)), float(theta),
+                                        int(bool(interleaved)), float(kv_scale), _ptr(out, _bp))
+    _check(rc, "mla_cache_row_fp8")
     return out
 
 

@@ -312,16 +312,91 @@ int lado_short_conv_step(int B, int Cch, int K, const double *x, double *tail,
  */
 /* Row t of one sequence's cache: contiguous rows (bt == NULL), or the paged layout in which
  * rows [j*P, (j+1)*P) of the sequence are page bt[j] of the pool, P rows per page. */
-static const uint16_t *mla_row(const uint16_t *base, const int *bt, int P, int D, int t) {
-    if (!bt) return base + (size_t)t * D;
-    return base + ((size_t)bt[t / P] * (size_t)P + (size_t)(t % P)) * (size_t)D;
+static size_t mla_row(const int *bt, int P, int D, int t) {
+    if (!bt) return (size_t)t * D;
+    return ((size_t)bt[t / P] * (size_t)P + (size_t)(t % P)) * (size_t)D;
+}
+
+/*
+ * FP8 latent cache ([P1] "How big is the cache per token, exactly?": 2 bytes per element in
+ * bf16, an FP8 cache halves that; [P2] "Does 292 GiB fit on four Hopper GPUs?": an FP8 cache
+ * doubles the tokens that fit). The FP8 the pages name is E4M3 ([P2] "What is in the files": the
+ * release's E4M3 weights carry one fp32 scale per 128x128 block). E4M3: 1 sign bit, 4 exponent
+ * bits with bias 7, 3 mantissa bits; exponent field 0 holds the subnormals m/8 * 2^-6; there is
+ * no infinity, and exponent and mantissa all ones (0x7F, 0xFF) is NaN, so the largest finite
+ * value is 1.75 * 2^8 = 448. The pages give no scale for the cache; the reading here is one fp32
+ * scale per cache: an element's value is scale * E4M3(code).
+ */
+static double e4m3_to_double(uint8_t c) {
+    const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        v = NAN;
+    else if (e == 0)
+        v = ldexp((double)m, -9); /* m/8 * 2^-6 */
+    else
+        v = ldexp(8.0 + m, e - 10); /* (1 + m/8) * 2^(e-7) */
+    return sign ? -v : v;
+}
+
+/* Nearest E4M3 code of v, ties to the even code, magnitudes beyond 448 clamped to 448 (a
+ * saturating conversion), NaN to 0x7F. The candidates in v's binade are multiples of the spacing
+ * of 4-bit significands there, 2^(e-4) for |v| = m * 2^e, m in [0.5, 1); below 2^-6 the spacing
+ * stays at the subnormal step 2^-9. A multiple k of the spacing maps to its code directly: the
+ * code's low 7 bits, read as an integer, count steps of the spacing within the format. */
+static uint8_t double_to_e4m3(double v) {
+    if (v != v) return 0x7Fu;
+    const uint8_t sign = signbit(v) ? 0x80u : 0u;
+    const double a = fabs(v);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7Eu);
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);
+    int q = e - 4;
+    if (q < -9) q = -9;
+    const double ulp = ldexp(1.0, q);
+    const double klo = floor(a / ulp), khi = klo + 1.0;
+    const double dlo = a - klo * ulp, dhi = khi * ulp - a;
+    double k;
+    if (dlo < dhi)
+        k = klo;
+    else if (dhi < dlo)
+        k = khi;
+    else
+        k = (fmod(klo, 2.0) == 0.0) ? klo : khi;
+    const double r = k * ulp; /* <= 448: 448 is a multiple of its binade's spacing 32 */
+    if (r == 0.0) return sign;
+    /* r = j * 2^-9 for j < 8 (subnormal codes j), else r = (8 + m) * 2^(E-10) with E >= 1 */
+    if (r < ldexp(1.0, -6)) return (uint8_t)(sign | (uint8_t)(r * 512.0));
+    int E;
+    const double f = frexp(r, &E); /* r = f * 2^E, f in [0.5, 1): exponent field E + 6 */
+    const int m = (int)(f * 16.0) - 8;
+    return (uint8_t)(sign | (uint8_t)(((E + 6) << 3) | m));
+}
+
+int lado_e4m3_decode(int n, const uint8_t *c, double *out) {
+    if (n < 0) return LADO_EINVAL;
+    for (int i = 0; i < n; ++i) out[i] = e4m3_to_double(c[i]);
+    return LADO_OK;
+}
+
+int lado_e4m3_encode(int n, const double *x, uint8_t *out) {
+    if (n < 0) return LADO_EINVAL;
+    for (int i = 0; i < n; ++i) out[i] = double_to_e4m3(x[i]);
+    return LADO_OK;
+}
+
+/* Element d of a cache row: bf16 bits (fp8 == 0) or an E4M3 code times the cache's scale. */
+static double cache_elem(const void *cache, int fp8, double kv_scale, size_t i) {
+    if (fp8) return kv_scale * e4m3_to_double(((const uint8_t *)cache)[i]);
+    return bf16_bits_to_double(((const uint16_t *)cache)[i]);
 }
 
 /* Shared body of the contiguous and paged entry points. With block_table == NULL, sequence b's
  * rows start at cache + b*seq_stride; otherwise cache is the page pool and row b of the block
  * table (bt_stride entries) names its pages of P rows. */
-static int mla_decode_impl(int B, int H, int Dc, int Dr, const double *q, const uint16_t *cache,
-                           long long seq_stride, const int *block_table, int bt_stride, int P,
+static int mla_decode_impl(int B, int H, int Dc, int Dr, const double *q, const void *cache, int fp8,
+                           double kv_scale, long long seq_stride, const int *block_table, int bt_stride, int P,
                            const int *seq_lens, const double *gate, double scale, double *o, double *lse,
                            int nthreads) {
     if (nthreads < 1) nthreads = 1;
@@ -344,13 +419,13 @@ static int mla_decode_impl(int B, int H, int Dc, int Dr, const double *q, const 
                 err = 1;
                 continue;
             }
-            const uint16_t *cb = block_table ? cache : cache + (size_t)b * (size_t)seq_stride;
+            const size_t cb = block_table ? 0 : (size_t)b * (size_t)seq_stride;
             const int *bt = block_table ? block_table + (size_t)b * (size_t)bt_stride : NULL;
             double m = -INFINITY;
             for (int t = 0; t < L; ++t) {
-                const uint16_t *ct = mla_row(cb, bt, P, D, t);
+                const size_t ct = cb + mla_row(bt, P, D, t);
                 double acc = 0.0;
-                for (int d = 0; d < D; ++d) acc += qh[d] * bf16_bits_to_double(ct[d]);
+                for (int d = 0; d < D; ++d) acc += qh[d] * cache_elem(cache, fp8, kv_scale, ct + (size_t)d);
                 s[t] = scale * acc;
                 if (s[t] > m) m = s[t];
             }
@@ -361,9 +436,9 @@ static int mla_decode_impl(int B, int H, int Dc, int Dr, const double *q, const 
             }
             for (int d = 0; d < Dc; ++d) oh[d] = 0.0;
             for (int t = 0; t < L; ++t) {
-                const uint16_t *ct = mla_row(cb, bt, P, D, t);
+                const size_t ct = cb + mla_row(bt, P, D, t);
                 double p = s[t] / z;
-                for (int d = 0; d < Dc; ++d) oh[d] += p * bf16_bits_to_double(ct[d]);
+                for (int d = 0; d < Dc; ++d) oh[d] += p * cache_elem(cache, fp8, kv_scale, ct + (size_t)d);
             }
             if (gate) {
                 double sg = 1.0 / (1.0 + exp(-gate[(size_t)b * H + h]));
@@ -380,8 +455,18 @@ int lado_mla_decode(int B, int H, int Dc, int Dr, long long seq_stride,
                     const double *q, const uint16_t *cache, const int *seq_lens,
                     const double *gate, double scale, double *o, double *lse, int nthreads) {
     if (B < 0 || H < 0 || Dc <= 0 || Dr < 0) return LADO_EINVAL;
-    return mla_decode_impl(B, H, Dc, Dr, q, cache, seq_stride, NULL, 0, 1, seq_lens, gate, scale, o, lse,
+    return mla_decode_impl(B, H, Dc, Dr, q, cache, 0, 1.0, seq_stride, NULL, 0, 1, seq_lens, gate, scale, o, lse,
                            nthreads);
+}
+
+/* The same attention over an FP8 cache: E4M3 codes, row t of sequence b at byte offset
+ * b*seq_stride + t*(Dc+Dr), each element worth kv_scale * E4M3(code). */
+int lado_mla_decode_fp8(int B, int H, int Dc, int Dr, long long seq_stride, const double *q, const uint8_t *cache,
+                        double kv_scale, const int *seq_lens, const double *gate, double scale, double *o,
+                        double *lse, int nthreads) {
+    if (B < 0 || H < 0 || Dc <= 0 || Dr < 0) return LADO_EINVAL;
+    return mla_decode_impl(B, H, Dc, Dr, q, cache, 1, kv_scale, seq_stride, NULL, 0, 1, seq_lens, gate, scale, o,
+                           lse, nthreads);
 }
 
 /*
@@ -393,10 +478,8 @@ int lado_mla_decode(int B, int H, int Dc, int Dr, long long seq_stride,
  * Returns LADO_EINVAL if a sequence needs more than bt_stride pages or names a page outside
  * [0, num_pages).
  */
-int lado_mla_decode_paged(int B, int H, int Dc, int Dr, int P, int num_pages, int bt_stride,
-                          const double *q, const uint16_t *pages, const int *block_table, const int *seq_lens,
-                          const double *gate, double scale, double *o, double *lse, int nthreads) {
-    if (B < 0 || H < 0 || Dc <= 0 || Dr < 0 || P <= 0 || num_pages < 0 || bt_stride < 0) return LADO_EINVAL;
+static int check_block_table(int B, int P, int num_pages, int bt_stride, const int *block_table,
+                             const int *seq_lens) {
     for (int b = 0; b < B; ++b) {
         const long long L = seq_lens[b];
         if (L < 0 || L > (long long)bt_stride * P) return LADO_EINVAL;
@@ -405,8 +488,28 @@ int lado_mla_decode_paged(int B, int H, int Dc, int Dr, int P, int num_pages, in
             if (pg < 0 || pg >= num_pages) return LADO_EINVAL;
         }
     }
-    return mla_decode_impl(B, H, Dc, Dr, q, pages, 0, block_table, bt_stride, P, seq_lens, gate, scale, o, lse,
-                           nthreads);
+    return LADO_OK;
+}
+
+int lado_mla_decode_paged(int B, int H, int Dc, int Dr, int P, int num_pages, int bt_stride,
+                          const double *q, const uint16_t *pages, const int *block_table, const int *seq_lens,
+                          const double *gate, double scale, double *o, double *lse, int nthreads) {
+    if (B < 0 || H < 0 || Dc <= 0 || Dr < 0 || P <= 0 || num_pages < 0 || bt_stride < 0) return LADO_EINVAL;
+    const int rc = check_block_table(B, P, num_pages, bt_stride, block_table, seq_lens);
+    if (rc != LADO_OK) return rc;
+    return mla_decode_impl(B, H, Dc, Dr, q, pages, 0, 1.0, 0, block_table, bt_stride, P, seq_lens, gate, scale, o,
+                           lse, nthreads);
+}
+
+/* The paged attention over an FP8 page pool (E4M3 codes [num_pages][P][Dc+Dr], scale kv_scale). */
+int lado_mla_decode_paged_fp8(int B, int H, int Dc, int Dr, int P, int num_pages, int bt_stride, const double *q,
+                              const uint8_t *pages, double kv_scale, const int *block_table, const int *seq_lens,
+                              const double *gate, double scale, double *o, double *lse, int nthreads) {
+    if (B < 0 || H < 0 || Dc <= 0 || Dr < 0 || P <= 0 || num_pages < 0 || bt_stride < 0) return LADO_EINVAL;
+    const int rc = check_block_table(B, P, num_pages, bt_stride, block_table, seq_lens);
+    if (rc != LADO_OK) return rc;
+    return mla_decode_impl(B, H, Dc, Dr, q, pages, 1, kv_scale, 0, block_table, bt_stride, P, seq_lens, gate, scale,
+                           o, lse, nthreads);
 }
 
 /*
@@ -496,6 +599,36 @@ int lado_mla_cache_row(int n, int Dc, int Dr, const uint16_t *c_kv, const uint16
         const int rc = lado_rope(1, Dr, x, positions + r, theta, interleaved, y);
         if (rc != LADO_OK) return rc;
         for (int d = 0; d < Dr; ++d) o[Dc + d] = double_to_bf16_bits(y[d]);
+    }
+    return LADO_OK;
+}
+
+/*
+ * A new FP8 latent-cache row for each of n tokens: the bf16 row of lado_mla_cache_row before its
+ * final rounding (the latent as given, the RoPE key turned in fp64), each element x stored as
+ * the E4M3 code of x / kv_scale. The quotient is taken in fp32, the precision the code is decided
+ * in on the GPU: x rounded to fp32 (exact for the bf16 latent), divided by fp32(kv_scale) with
+ * one rounding to nearest, then rounded once more to E4M3 (double_to_e4m3).
+ * out: [n][Dc + Dr] E4M3 codes.
+ */
+int lado_mla_cache_row_fp8(int n, int Dc, int Dr, const uint16_t *c_kv, const uint16_t *k_pe,
+                           const long long *positions, double theta, int interleaved, double kv_scale, uint8_t *out) {
+    if (n < 0 || Dc < 0 || Dr <= 0 || Dr > 1024 || (Dr & 1) || !(kv_scale > 0.0)) return LADO_EINVAL;
+    const float s = (float)kv_scale;
+    double x[1024], y[1024];
+    for (int r = 0; r < n; ++r) {
+        uint8_t *o = out + (size_t)r * (Dc + Dr);
+        for (int d = 0; d < Dc; ++d) {
+            const float v = (float)bf16_bits_to_double(c_kv[(size_t)r * Dc + d]);
+            o[d] = double_to_e4m3((double)(v / s));
+        }
+        for (int d = 0; d < Dr; ++d) x[d] = bf16_bits_to_double(k_pe[(size_t)r * Dr + d]);
+        const int rc = lado_rope(1, Dr, x, positions + r, theta, interleaved, y);
+        if (rc != LADO_OK) return rc;
+        for (int d = 0; d < Dr; ++d) {
+            const float v = (float)y[d];
+            o[Dc + d] = double_to_e4m3((double)(v / s));
+        }
     }
     return LADO_OK;
 }

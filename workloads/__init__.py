@@ -244,14 +244,16 @@ def mla_inputs(cfg: MlaDecode, device="cpu", lmax: int | None = None) -> dict:
 def paginate(cache: torch.Tensor, seq_lens: torch.Tensor, page_size: int, seed: int, spare_pages: int = 0):
     """Moves a contiguous latent cache [B, Lmax, D] into a pool of pages of `page_size` rows placed
     in a seeded random order, the way a serving engine's allocator scatters them. Rows of a page
-    past its sequence's length, and spare pages, hold NaN. Returns (pool [P, page_size, D],
-    block_table int32 [B, max pages], on the cache's device); unused table entries are -1."""
+    past its sequence's length, and spare pages, hold NaN (for a uint8 cache of E4M3 codes, the
+    NaN code 0x7F). Returns (pool [P, page_size, D], block_table int32 [B, max pages], on the
+    cache's device); unused table entries are -1."""
     B, _, D = cache.shape
+    fill = 0x7F if cache.dtype == torch.uint8 else float("nan")
     lens = [int(x) for x in seq_lens.tolist()]
     per_seq = [(n + page_size - 1) // page_size for n in lens]
     n_pages = sum(per_seq) + spare_pages
     perm = np.random.default_rng(_seed(seed, "pages")).permutation(n_pages)
-    pool = torch.full((n_pages, page_size, D), float("nan"), dtype=cache.dtype, device=cache.device)
+    pool = torch.full((n_pages, page_size, D), fill, dtype=cache.dtype, device=cache.device)
     table = torch.full((B, max(max(per_seq, default=0), 1)), -1, dtype=torch.int32)
     k = 0
     for b in range(B):
