@@ -11,6 +11,8 @@ A step is one pass of the workload's hot path over one batch of synthetic input:
   mla_decode_b16              one gated MLA layer, 16 sequences, contexts uniform in [8192, 131072]
   mla_decode_b16_paged        the same layer with the cache in 64-row pages of a shuffled pool
   mla_decode_b16_paged_rope   the paged layer with RoPE in the kernels: append the new rows, then attend
+  mla_decode_b16_fp8          mla_decode_b16 over an FP8 (E4M3) cache, one fp32 scale (mla_latent_decode_fp8)
+  mla_decode_b16_paged_rope_fp8  the engine step of mla_decode_b16_paged_rope over FP8 pages
   kda_decode_b64_gated        the same layer with the output gate fused (kda_conv_decode_step_gated)
   kda_mtp_b64                 kda_decode_multi: 64 sequences x 64 heads, 4 tokens per state pass
   kda_prefill_32k             kda_prefill_chunked, 1 x 32768 tokens x 64 heads, chunk 64
@@ -544,6 +546,78 @@ class MlaPagedRopeStep(MlaPagedStep):
         return {"mla_latent_decode_paged_rope": b, "step": b + append}
 
 
+class MlaFp8Step(MlaDecodeStep):
+    """The 16-sequence latent-attention workload over an FP8 (E4M3) cache with one fp32 scale,
+    through mla_latent_decode_fp8; the cache holds half the bytes of the bf16 one."""
+    name = "mla_decode_b16_fp8"
+
+    def __init__(self, lad, dev, rank, cfg: wl.MlaDecode | None = None):
+        super().__init__(lad, dev, rank, cfg)
+        del self.cache
+        torch.cuda.empty_cache()
+        self.cache8 = wl.mla_fp8_cache(self.cfg, dev)
+        self.kv_scale = wl.KV_SCALE_FP8
+        self.dominant = "mla_latent_decode_fp8"
+        self.config = dict(self.config, workload=self.name, cache_row="512 latent + 64 rope, E4M3 codes",
+                           kv_scale=f"one fp32 scale per cache ({self.kv_scale})")
+
+    def run(self, timer=None):
+        if timer:
+            timer.begin("mla_latent_decode_fp8")
+        self.lad.mla_latent_decode_fp8(self.q, self.cache8, self.kv_scale, self.lens, self.gate, o=self.o,
+                                       workspace=self.ws)
+        if timer:
+            timer.end("mla_latent_decode_fp8")
+
+    def mla_bytes(self):
+        B, Hq = self.cfg.B, self.cfg.Hq
+        return self.total_len * wl.D_ROW + B * Hq * (wl.D_ROW * 2 + 4 + wl.D_LATENT * 2) + B * 4
+
+    def algorithmic_bytes(self):
+        b = self.mla_bytes()
+        return {"mla_latent_decode_fp8": b, "step": b}
+
+
+class MlaPagedRopeFp8Step(MlaFp8Step):
+    """The engine step of mla_decode_b16_paged_rope over a pool of FP8 pages: mla_cache_append_fp8
+    writes each sequence's new row at len - 1, then mla_latent_decode_paged_fp8 attends with the
+    query's RoPE part turned in the kernel."""
+    name = "mla_decode_b16_paged_rope_fp8"
+    page_size = 64
+
+    def __init__(self, lad, dev, rank, cfg: wl.MlaDecode | None = None):
+        super().__init__(lad, dev, rank, cfg)
+        self.pool, self.block_table = wl.paginate(self.cache8, self.lens, self.page_size, self.cfg.seed)
+        del self.cache8
+        torch.cuda.empty_cache()
+        B, s = self.cfg.B, self.cfg.seed
+        self.c_kv = wl.normal_bf16((B, wl.D_LATENT), s, "mla_ckv", dev)
+        self.k_pe = wl.normal_bf16((B, wl.D_ROPE), s, "mla_kpe", dev)
+        self.pos = (self.lens - 1).contiguous()
+        self.launches_per_step = 3
+        self.dominant = "mla_latent_decode_paged_fp8"
+        self.config = dict(self.config, workload=self.name, rope="theta 6e6, rotate-half pairing, in-kernel",
+                           paging=f"{self.page_size}-row pages, {self.pool.shape[0]} in a shuffled pool")
+
+    def run(self, timer=None):
+        self.lad.mla_cache_append_fp8(self.c_kv, self.k_pe, self.pos, self.pool, self.kv_scale,
+                                      block_table=self.block_table)
+        if timer:
+            timer.begin("mla_latent_decode_paged_fp8")
+        self.lad.mla_latent_decode_paged_fp8(self.q, self.pool, self.kv_scale, self.block_table, self.lens,
+                                             positions=self.pos, gate_logits=self.gate, o=self.o, workspace=self.ws)
+        if timer:
+            timer.end("mla_latent_decode_paged_fp8")
+
+    def mla_bytes(self):
+        return super().mla_bytes() + 4 * sum(-(-int(n) // self.page_size) for n in self.lens.tolist())
+
+    def algorithmic_bytes(self):
+        b = self.mla_bytes()
+        append = self.cfg.B * (wl.D_LATENT * 2 + wl.D_ROPE * 2 + 4 + wl.D_ROW + 4)
+        return {"mla_latent_decode_paged_fp8": b, "step": b + append}
+
+
 class HybridStep(Step):
     name = "hybrid_8layer_1m"
 
@@ -678,6 +752,8 @@ WORKLOADS = {
     "mla_decode_b16": MlaDecodeStep,
     "mla_decode_b16_paged": MlaPagedStep,
     "mla_decode_b16_paged_rope": MlaPagedRopeStep,
+    "mla_decode_b16_fp8": MlaFp8Step,
+    "mla_decode_b16_paged_rope_fp8": MlaPagedRopeFp8Step,
     "kda_prefill_32k": PrefillStep,
 }
 
@@ -736,12 +812,18 @@ def cpu_oracle_rate(workload: str, budget_s: float = 20.0) -> dict:
         dt = time.perf_counter() - t0
         return dt * B / Bs, f"{Bs} of {B} sequences x 64 heads, one token"
 
-    def mla_seconds(B, lens):
+    def mla_seconds(B, lens, fp8=False):
         # units = (sequence, head); sample `nth` heads of the longest sequence over its whole context
         L = int(max(lens))
         units = min(nth, H)
-        cache = (rng.standard_normal((1, L, wl.D_ROW)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
         qs = rng.standard_normal((1, units, wl.D_ROW))
+        if fp8:
+            codes = rng.integers(0, 0x7F, (1, L, wl.D_ROW), dtype=np.uint8)
+            t0 = time.perf_counter()
+            oracle.mla_decode_fp8(qs, codes, wl.KV_SCALE_FP8, np.array([L], np.int32), None, nthreads=nth)
+            dt = time.perf_counter() - t0
+            return dt * H * float(sum(lens)) / (units * L), f"{units} heads x {L} cached tokens of 1 sequence"
+        cache = (rng.standard_normal((1, L, wl.D_ROW)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
         t0 = time.perf_counter()
         oracle.mla_decode(qs, cache, np.array([L], np.int32), None, nthreads=nth)
         dt = time.perf_counter() - t0
@@ -763,9 +845,10 @@ def cpu_oracle_rate(workload: str, budget_s: float = 20.0) -> dict:
         sec = (time.perf_counter() - t0) * 64 / Bs
         return {"value": 256 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle",
                 "sample": f"{Bs} of 64 sequences x 64 heads x 4 tokens, scaled to 64 sequences"}
-    if workload in ("mla_decode_b16", "mla_decode_b16_paged", "mla_decode_b16_paged_rope"):
+    if workload in ("mla_decode_b16", "mla_decode_b16_paged", "mla_decode_b16_paged_rope", "mla_decode_b16_fp8",
+                    "mla_decode_b16_paged_rope_fp8"):
         lens = wl.mla_seq_lens(wl.MlaDecode("mla", B=16, seed=1236)).tolist()
-        sec, sample = mla_seconds(16, lens)
+        sec, sample = mla_seconds(16, lens, fp8=workload.endswith("fp8"))
         return {"value": 16 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": sample}
     if workload == "hybrid_8layer_1m":
         ks, s1 = kda_layer_seconds(8)
@@ -806,7 +889,8 @@ def run_reference(args, rank, world):
 
 def _tokens(workload):
     return {"hybrid_8layer_1m": 8, "kda_decode_b64": 64, "kda_decode_b64_gated": 64, "kda_mtp_b64": 256, "mla_decode_b16": 16,
-            "mla_decode_b16_paged": 16, "mla_decode_b16_paged_rope": 16, "kda_prefill_32k": 32768}[workload]
+            "mla_decode_b16_paged": 16, "mla_decode_b16_paged_rope": 16, "mla_decode_b16_fp8": 16,
+            "mla_decode_b16_paged_rope_fp8": 16, "kda_prefill_32k": 32768}[workload]
 
 
 def main(argv=None) -> int:
@@ -891,7 +975,8 @@ def main(argv=None) -> int:
     per_type = {}
     for kname in ("kda_conv_decode_step", "kda_conv_decode_step_gated", "kda_decode_step", "kda_decode_multi",
                   "mla_latent_decode",
-                  "mla_latent_decode_paged", "mla_latent_decode_paged_rope", "kda_prefill_chunked"):
+                  "mla_latent_decode_paged", "mla_latent_decode_paged_rope", "mla_latent_decode_fp8",
+                  "mla_latent_decode_paged_fp8", "kda_prefill_chunked"):
         km = timer.mean_ms(kname)
         if km is not None and kname in ab:
             gbs = ab[kname] / (km / 1000.0) / 1e9
@@ -915,7 +1000,9 @@ def main(argv=None) -> int:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16 inputs, fp32 state and accumulation", "data": "synthetic",
+            "vs_baseline": None, "dtype": ("e4m3 cache widened to bf16, bf16 query, fp32 accumulation"
+                                           if args.workload.endswith("fp8") else
+                                           "bf16 inputs, fp32 state and accumulation"), "data": "synthetic",
             "config": {**step.config, "global_batch": int(round(tokens)) if not isinstance(step, PrefillStep)
                        else world * step.cfg.B, "parallelism": f"sequence-sharded x{world}, no exchange"},
             "per_layer_type": per_type,

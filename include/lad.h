@@ -59,7 +59,8 @@ int lad_version(void);
 /*
  * Reads and clears the device-side error word that bounded waits set (see above), after
  * synchronising `stream`. *code receives 0 when no kernel gave up a wait, else a nonzero tag
- * naming the kernel and the wait (0x101-0x104 latent decode, 0x201 chunked prefill), 0x105 when
+ * naming the kernel and the wait (0x101-0x104 and 0x107 latent decode, 0x201 chunked prefill),
+ * 0x106 when an FP8-cache decode met a query value beyond the f16 range, 0x105 when
  * a paged decode met a block-table entry outside the pool, or 0x301 when mla_cache_append had a
  * position with no row to write. Returns LAD_OK or LAD_ECUDA.
  */
@@ -307,6 +308,61 @@ int mla_cache_append(const lad_bf16 *c_kv, const lad_bf16 *k_pe, const int *posi
                      long long cache_seq_stride, int Lmax, const int *block_table, int block_table_stride,
                      int num_pages, int page_size, int B, int d_latent, int d_rope, float rope_theta, unsigned flags,
                      void *stream);
+
+/*
+ * FP8 latent cache. [P1] "How big is the cache per token, exactly?": the bf16 cache takes 2 bytes
+ * per element and an FP8 cache would halve it; [P2] "Does 292 GiB fit on four Hopper GPUs?": an
+ * FP8 cache doubles the tokens that fit. The FP8 the pages use is E4M3 ([P2] "What is in the
+ * files", with one fp32 scale per weight block); for the cache they give no scale, and the
+ * reading here is one fp32 scale per cache: element = kv_scale * E4M3(code). E4M3: sign, 4
+ * exponent bits (bias 7), 3 mantissa bits, largest finite 448, 0x7F / 0xFF NaN, no infinity.
+ *
+ * mla_latent_decode_fp8 — mla_latent_decode over an FP8 cache. The codes are widened to f16
+ * exactly on chip and the query is converted bf16 -> f16 (exact for |q| <= 65504 outside the f16
+ * subnormal range; a larger |q| sets device error 0x106), so the tensor cores run q.c and p.c on
+ * f16 operands with fp32 accumulation (P in f16); kv_scale is applied to the fp32 scores and to
+ * the normalised output. A bounded wait of the widening warps that gives up sets 0x107.
+ *   cache             E4M3 codes, row t of sequence b at cache + b*cache_seq_stride + t*576 (bytes)
+ *   cache_seq_stride  bytes between sequences (>= Lmax*576, multiple of 16)
+ *   kv_scale          > 0, finite
+ *   the rest          as for mla_latent_decode (same workspace size query); rows at or past
+ *                     seq_lens[b] are never read; rows at or past Lmax read as zeros
+ * Supported: as mla_latent_decode; cache and q 16-byte aligned.
+ */
+int mla_latent_decode_fp8(const lad_bf16 *q, const uint8_t *cache, long long cache_seq_stride, float kv_scale,
+                          const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B, int Hq,
+                          int d_latent, int d_rope, int Lmax, float scale, unsigned flags, void *workspace,
+                          size_t ws_bytes, void *stream);
+
+/*
+ * mla_latent_decode_paged_fp8 — mla_latent_decode_paged over a pool of FP8 pages, with the
+ * query's RoPE part turned in the kernel when positions != NULL (as mla_latent_decode_paged_rope;
+ * rope_theta is then > 1 and LAD_FLAG_ROPE_INTERLEAVED selects the pairing) or arriving turned
+ * when positions == NULL (rope_theta ignored).
+ *   kv_pages   E4M3 codes [num_pages][page_size][576], 16-byte aligned
+ *   kv_scale   > 0, finite
+ *   the rest   as for mla_latent_decode_paged (block table, limits, device error 0x105)
+ */
+int mla_latent_decode_paged_fp8(const lad_bf16 *q, const int *positions, float rope_theta, const uint8_t *kv_pages,
+                                float kv_scale, int num_pages, int page_size, const int *block_table,
+                                int block_table_stride, const int *seq_lens, const float *gate_logits, void *o,
+                                float *lse_out, int B, int Hq, int d_latent, int d_rope, float scale, unsigned flags,
+                                void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * mla_cache_append_fp8 — mla_cache_append into an FP8 cache: each element x of the new row (the
+ * latent as given, the RoPE key turned in fp64) is stored as the E4M3 code of x / kv_scale, the
+ * quotient taken in fp32 (x rounded to fp32 first; one IEEE division) and rounded to nearest
+ * even, saturating at +-448 (NaN stays NaN).
+ *   cache       E4M3 codes, 16-byte aligned; contiguous (cache_seq_stride in bytes, multiple
+ *               of 16) or a page pool, as for mla_cache_append
+ *   kv_scale    > 0, finite
+ *   the rest    as for mla_cache_append (device error 0x301 for a position with no row)
+ */
+int mla_cache_append_fp8(const lad_bf16 *c_kv, const lad_bf16 *k_pe, const int *positions, uint8_t *cache,
+                         long long cache_seq_stride, int Lmax, const int *block_table, int block_table_stride,
+                         int num_pages, int page_size, int B, int d_latent, int d_rope, float rope_theta,
+                         float kv_scale, unsigned flags, void *stream);
 
 /*
  * mla_latent_decode_noalloc — mla_latent_decode for callers that cannot allocate device memory

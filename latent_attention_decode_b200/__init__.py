@@ -18,10 +18,14 @@ import os
 import torch
 
 __all__ = [
-    "kda_conv_update", "kda_decode_step", "kda_conv_decode_step", "kda_prefill_chunked", "kda_prefill_workspace_size",
-    "mla_latent_decode", "mla_latent_decode_workspace_size", "mla_latent_decode_noalloc",
+    "kda_conv_update", "kda_decode_step", "kda_conv_decode_step", "kda_conv_decode_step_gated", "kda_decode_multi",
+    "kda_prefill_chunked", "kda_prefill_workspace_size",
+    "mla_latent_decode", "mla_latent_decode_workspace_size", "mla_latent_decode_paged",
+    "mla_latent_decode_paged_rope", "mla_cache_append", "mla_latent_decode_fp8", "mla_latent_decode_paged_fp8",
+    "mla_cache_append_fp8", "mla_latent_decode_noalloc",
     "lad_device_error", "lad_version",
-    "LadError", "LIB_PATH", "FLAG_SILU", "FLAG_L2NORM_QK", "FLAG_OUT_FP32", "MLA_SCALE",
+    "LadError", "LIB_PATH", "FLAG_SILU", "FLAG_L2NORM_QK", "FLAG_OUT_FP32", "FLAG_KEEP_STATE",
+    "FLAG_ROPE_INTERLEAVED", "MLA_SCALE", "ROPE_THETA",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblad.so")
@@ -83,6 +87,13 @@ def _load() -> ctypes.CDLL:
         "mla_latent_decode_noalloc": ([_c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                                        _c_int, _c_int, _c_f, _c_u, _c_vp], _c_int),
         "mla_latent_decode_noalloc_max_batch": ([], _c_sz),
+        "mla_latent_decode_fp8": ([_c_vp, _c_vp, _c_ll, _c_f, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
+                                   _c_int, _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
+        "mla_latent_decode_paged_fp8": ([_c_vp, _c_vp, _c_f, _c_vp, _c_f, _c_int, _c_int, _c_vp, _c_int, _c_vp,
+                                         _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_f, _c_u, _c_vp,
+                                         _c_sz, _c_vp], _c_int),
+        "mla_cache_append_fp8": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_ll, _c_int, _c_vp, _c_int, _c_int, _c_int, _c_int,
+                                  _c_int, _c_int, _c_f, _c_f, _c_u, _c_vp], _c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -500,6 +511,120 @@ def mla_cache_append(c_kv: torch.Tensor, k_pe: torch.Tensor, positions: torch.Te
                                    block_table.data_ptr(), block_table.shape[1], cache.shape[0], cache.shape[1], B,
                                    Dc, Dr, float(rope_theta), flags, _stream(stream))
     _check("mla_cache_append", rc)
+
+
+def _codes(t: torch.Tensor, name: str) -> torch.Tensor:
+    """An E4M3 cache as uint8 codes (torch.float8_e4m3fn tensors are viewed, not converted)."""
+    if t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    return _cuda(t, name, torch.uint8)
+
+
+def _mla_common(q, seq_lens, gate_logits, o, lse, d_latent, out_fp32, workspace):
+    bf = torch.bfloat16
+    _contig(q, "q", bf)
+    B, Hq, D = q.shape
+    _contig(seq_lens, "seq_lens", torch.int32)
+    if seq_lens.shape != (B,):
+        raise ValueError("seq_lens must be [B]")
+    if gate_logits is not None:
+        _contig(gate_logits, "gate_logits", torch.float32)
+        if gate_logits.shape != (B, Hq):
+            raise ValueError("gate_logits must be [B,Hq]")
+    odt = torch.float32 if out_fp32 else bf
+    if o is None:
+        o = torch.empty((B, Hq, d_latent), device=q.device, dtype=odt)
+    _contig(o, "o", odt)
+    if lse is not None:
+        _contig(lse, "lse", torch.float32)
+    ws = mla_latent_decode_workspace_size(B, Hq, d_latent, 0)
+    if workspace is None and ws > 0:
+        workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return B, Hq, D, o, workspace, ws_bytes
+
+
+def mla_latent_decode_fp8(q: torch.Tensor, cache: torch.Tensor, kv_scale: float, seq_lens: torch.Tensor,
+                          gate_logits: torch.Tensor | None = None, o: torch.Tensor | None = None,
+                          lse: torch.Tensor | None = None, scale: float = MLA_SCALE, d_latent: int = 512,
+                          out_fp32: bool = False, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """mla_latent_decode over an FP8 cache: cache [B,Lmax,576] E4M3 codes (uint8 or
+    float8_e4m3fn, rows contiguous), every element worth kv_scale * E4M3(code)."""
+    cache = _codes(cache, "cache")
+    B, Hq, D, o, workspace, ws_bytes = _mla_common(q, seq_lens, gate_logits, o, lse, d_latent, out_fp32, workspace)
+    if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != D or cache.stride(2) != 1 \
+            or cache.stride(1) != D:
+        raise ValueError("cache must be [B,Lmax,D] with contiguous rows")
+    Lmax = cache.shape[1]
+    seq_stride = cache.stride(0) if B > 1 else Lmax * D
+    _check("mla_latent_decode_fp8", _L().mla_latent_decode_fp8(
+        q.data_ptr(), cache.data_ptr(), seq_stride, float(kv_scale), seq_lens.data_ptr(), _ptr(gate_logits),
+        o.data_ptr(), _ptr(lse), B, Hq, d_latent, D - d_latent, Lmax, float(scale),
+        FLAG_OUT_FP32 if out_fp32 else 0, _ptr(workspace), ws_bytes, _stream(stream)))
+    return o
+
+
+def mla_latent_decode_paged_fp8(q: torch.Tensor, kv_pages: torch.Tensor, kv_scale: float, block_table: torch.Tensor,
+                                seq_lens: torch.Tensor, positions: torch.Tensor | None = None,
+                                gate_logits: torch.Tensor | None = None, o: torch.Tensor | None = None,
+                                lse: torch.Tensor | None = None, scale: float = MLA_SCALE,
+                                rope_theta: float = ROPE_THETA, interleaved: bool = False, d_latent: int = 512,
+                                out_fp32: bool = False, workspace: torch.Tensor | None = None,
+                                stream=None) -> torch.Tensor:
+    """mla_latent_decode_paged over a pool of FP8 pages [num_pages, page_size, 576] (E4M3 codes);
+    with positions (int32 [B]) q's RoPE part is turned in the kernel, as mla_latent_decode_paged_rope."""
+    kv_pages = _codes(kv_pages, "kv_pages")
+    _contig(kv_pages, "kv_pages")
+    B, Hq, D, o, workspace, ws_bytes = _mla_common(q, seq_lens, gate_logits, o, lse, d_latent, out_fp32, workspace)
+    if kv_pages.dim() != 3 or kv_pages.shape[2] != D:
+        raise ValueError("kv_pages must be [num_pages, page_size, D]")
+    _contig(block_table, "block_table", torch.int32)
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, n]")
+    if positions is not None:
+        _contig(positions, "positions", torch.int32)
+        if positions.shape != (B,):
+            raise ValueError("positions must be [B]")
+    flags = (FLAG_OUT_FP32 if out_fp32 else 0) | (FLAG_ROPE_INTERLEAVED if interleaved else 0)
+    _check("mla_latent_decode_paged_fp8", _L().mla_latent_decode_paged_fp8(
+        q.data_ptr(), _ptr(positions), float(rope_theta), kv_pages.data_ptr(), float(kv_scale), kv_pages.shape[0],
+        kv_pages.shape[1], block_table.data_ptr(), block_table.shape[1], seq_lens.data_ptr(), _ptr(gate_logits),
+        o.data_ptr(), _ptr(lse), B, Hq, d_latent, D - d_latent, float(scale), flags, _ptr(workspace), ws_bytes,
+        _stream(stream)))
+    return o
+
+
+def mla_cache_append_fp8(c_kv: torch.Tensor, k_pe: torch.Tensor, positions: torch.Tensor, cache: torch.Tensor,
+                         kv_scale: float, block_table: torch.Tensor | None = None, rope_theta: float = ROPE_THETA,
+                         interleaved: bool = False, stream=None) -> None:
+    """mla_cache_append into an FP8 cache (E4M3 codes, uint8 or float8_e4m3fn): each element x of
+    the new row is stored as the code of x / kv_scale."""
+    bf = torch.bfloat16
+    cache = _codes(cache, "cache")
+    _contig(c_kv, "c_kv", bf), _contig(k_pe, "k_pe", bf), _contig(positions, "positions", torch.int32)
+    B, Dc = c_kv.shape
+    Dr = k_pe.shape[1]
+    if k_pe.shape != (B, Dr) or positions.shape != (B,):
+        raise ValueError("c_kv [B, 512], k_pe [B, 64], positions [B]")
+    flags = FLAG_ROPE_INTERLEAVED if interleaved else 0
+    if block_table is None:
+        if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != Dc + Dr or cache.stride(2) != 1 \
+                or cache.stride(1) != Dc + Dr:
+            raise ValueError("cache must be [B, Lmax, 576] with contiguous rows")
+        seq_stride = cache.stride(0) if B > 1 else cache.shape[1] * (Dc + Dr)
+        rc = _L().mla_cache_append_fp8(c_kv.data_ptr(), k_pe.data_ptr(), positions.data_ptr(), cache.data_ptr(),
+                                       seq_stride, cache.shape[1], None, 0, 0, 0, B, Dc, Dr, float(rope_theta),
+                                       float(kv_scale), flags, _stream(stream))
+    else:
+        _contig(cache, "cache")
+        _contig(block_table, "block_table", torch.int32)
+        if cache.dim() != 3 or cache.shape[2] != Dc + Dr or block_table.dim() != 2 or block_table.shape[0] != B:
+            raise ValueError("cache must be [num_pages, page_size, 576] and block_table [B, n]")
+        rc = _L().mla_cache_append_fp8(c_kv.data_ptr(), k_pe.data_ptr(), positions.data_ptr(), cache.data_ptr(), 0,
+                                       0, block_table.data_ptr(), block_table.shape[1], cache.shape[0],
+                                       cache.shape[1], B, Dc, Dr, float(rope_theta), float(kv_scale), flags,
+                                       _stream(stream))
+    _check("mla_cache_append_fp8", rc)
 
 
 def mla_latent_decode_noalloc(q: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tensor,

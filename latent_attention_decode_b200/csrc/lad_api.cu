@@ -56,7 +56,7 @@ void *tensor_map_encoder_raw() {
 
 extern "C" const char *lad_last_error(void) { return lad::g_last_error; }
 
-extern "C" int lad_version(void) { return 101; }
+extern "C" int lad_version(void) { return 102; }
 
 extern "C" int lad_device_error(void *stream, int *code) {
     if (!code) return lad::set_error(LAD_EINVAL, "lad_device_error: code is NULL");

@@ -36,6 +36,8 @@ enum DeviceErrorTag : int {
     kErrMlaSoftmax = 0x103,
     kErrMlaEpilogue = 0x104,
     kErrMlaBlockTable = 0x105,  // a paged call met a block-table entry outside the pool (not a wait)
+    kErrMlaQRange = 0x106,      // FP8-cache call: a query value beyond the f16 range (not a wait)
+    kErrMlaConvert = 0x107,     // FP8-cache call: the widening warps gave up a wait
     kErrCacheAppend = 0x301,    // mla_cache_append: a position with no row to write (not a wait)
     kErrPrefill = 0x201,
 };

@@ -30,6 +30,16 @@
 // of TMEM sub-partition p), rescale O when a head's running max grows by more than 2^8
 // (lazily, like FlashAttention-4), and write the segment's partial at its end.
 //
+// FP8 cache variant (kFp8): rows are 576 E4M3 codes with one fp32 scale for the whole cache. Four
+// more warps (8-11) load each tile's codes from global memory straight into registers, two tiles
+// ahead (no shared-memory staging: the kernel is bound by shared-memory traffic, not by HBM),
+// and write them widened into the same swizzled operand layout and 4-deep ring the TMA fills for
+// a bf16 cache; the producer warp then loads only q. The tensor cores run on f16
+// operands (kind::f16 takes A and B of one type): an E4M3 pair becomes an f16 pair in one
+// conversion (bf16 would take four), every E4M3 value is exact in f16, the query is converted
+// bf16 -> f16 in place once per segment (exact within the f16 range; a larger |q| is reported),
+// and P is written as f16. The scale folds into the score scale and the combine's normalisation.
+//
 // Every wait on an mbarrier is bounded (see lad_common.cuh); a wait that runs out records a tag
 // in the device error word, raises an abort flag the other roles see, and the CTA drains its
 // own copies and MMAs, frees TMEM and returns.
@@ -52,8 +62,9 @@ constexpr int kDrow = kDl + kDr;   // 576 bf16 per cached row
 constexpr int kChunk = 64;         // bf16 per 128-byte swizzle row
 constexpr int kNChunk = kDrow / kChunk;  // 9
 constexpr int kTile = 32;          // cached rows per tile
-constexpr int kStages = 4;
+constexpr int kStages = 4;            // bf16 ring fed by TMA
 constexpr int kThreads = 256;
+constexpr int kThreadsF8 = 384;       // + 4 converter warps
 constexpr int kMaxSplitCtas = 1024;  // one split CTA per SM; the combine tracks at most this many
 
 constexpr int kQChunkBytes = kHq * 128;                 // 8 KiB: 64 heads x 64 dims
@@ -90,7 +101,8 @@ enum Bar : int {
     kBarQRoped = kBarQFull + 1,        // (RoPE variant) q's RoPE part turned to the query position
     kBarQEmpty = kBarQRoped + 1,       // GEMM1s of a segment done with q
     kBarDrain = kBarQEmpty + 1,        // final MMA drain
-    kNumBars = kBarDrain + 1,
+    kBarQF16 = kBarDrain + 1,          // (FP8) q converted to f16
+    kNumBars = kBarQF16 + 1,
 };
 constexpr int kOffScalars = kNumBars * 8;  // inside the barrier region: tmem base, abort flag, ...
 
@@ -106,7 +118,10 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 // The issue helpers (lad::ptx) are executed by a whole, converged warp; `elect.sync` picks one lane
 // (the same lowest lane every time) that actually issues. Keeping the warp converged lets the
 // descriptors and addresses live in uniform registers, which tcgen05.mma and TMA read directly.
+using lad::ptx::e4m3x2_to_f16x2;
+using lad::ptx::f32x2_to_f16x2;
 using lad::ptx::ex2_approx;
+using lad::ptx::fence_async_smem;
 using lad::ptx::kLayoutNone;
 using lad::ptx::kLayoutSw128;
 using lad::ptx::mbar_arrive;
@@ -133,6 +148,9 @@ constexpr uint32_t make_idesc(int M, int N, int a_mn_major, int b_mn_major) {
 }
 constexpr uint32_t kIdesc1 = make_idesc(64, kTile, 0, 0);   // S = q . C^T
 constexpr uint32_t kIdesc2 = make_idesc(128, kHq, 1, 0);    // O^T += V^T . P^T
+// the same with f16 operands (FP8 cache)
+constexpr uint32_t kIdesc1F16 = lad::ptx::make_idesc(64, kTile, lad::ptx::kFmtF16, 0, 0);
+constexpr uint32_t kIdesc2F16 = lad::ptx::make_idesc(128, kHq, lad::ptx::kFmtF16, 1, 0);
 
 // ------------------------------------------------------------------------------------------
 // work split
@@ -200,13 +218,75 @@ struct RopeQ {
     double inv_freq[kDr / 2];
 };
 
+// FP8 cache: E4M3 codes, row t of sequence b at base + b * seq_stride + t * 576 (contiguous,
+// rows past Lmax read as zeros) or in the page pool at base (paged, rows located as above).
+struct Fp8Cache {
+    const uint8_t *base;
+    long long seq_stride;  // bytes
+    int Lmax;
+};
+
+// Walks the tiles of a CTA's range in order for the FP8 widening warps: per tile, the address of its
+// first row and how many of its rows hold codes to read (0 at or past the length, past Lmax, or in
+// a page outside the pool, which is reported). next() is warp-uniform: every lane of a warp calls it.
+template <bool kPaged>
+struct Fp8Cursor {
+    SegIter it;
+    const int *seq_lens;
+    Fp8Cache f8;
+    PagedCache pc;
+    int seq, tile0, nt, i, len;
+    bool more;
+    int pseq, pg0, pg_lane;  // paged: lane j holds block_table[seq][pg0 + j]
+
+    __device__ Fp8Cursor(const SegIter &it_, const int *lens, const Fp8Cache &f, const PagedCache &p)
+        : it(it_), seq_lens(lens), f8(f), pc(p), seq(0), tile0(0), nt(0), i(0), len(0), more(true), pseq(-1), pg0(0),
+          pg_lane(-1) {}
+
+    __device__ bool next(int lane, const uint8_t *&row0, int &nrows) {
+        while (more && i >= nt) {
+            more = it.next(seq, tile0, nt);
+            i = 0;
+            if (more) len = seq_lens[seq];
+        }
+        if (!more) return false;
+        const int t_row = (tile0 + i) * kTile;
+        ++i;
+        const int lim = kPaged ? len : min(len, f8.Lmax);
+        nrows = max(0, min(kTile, lim - t_row));
+        if constexpr (kPaged) {
+            // 32 block-table entries per load, one per lane
+            const int pi = t_row / pc.page_size;
+            if (seq != pseq || pi < pg0 || pi >= pg0 + 32) {
+                pseq = seq;
+                pg0 = pi;
+                const int j = pg0 + lane;
+                pg_lane = j < pc.bt_stride ? pc.block_table[static_cast<long long>(seq) * pc.bt_stride + j] : -1;
+            }
+            const int page = __shfl_sync(0xffffffffu, pg_lane, pi - pg0);
+            if (page >= 0 && page < pc.num_pages) {
+                row0 = f8.base + (static_cast<long long>(page) * pc.page_size + (t_row - pi * pc.page_size)) * kDrow;
+            } else {
+                if (nrows > 0 && lane == 0) atomicCAS(&g_mla_error, 0, lad::kErrMlaBlockTable);
+                row0 = nullptr;
+                nrows = 0;
+            }
+        } else {
+            row0 = f8.base + seq * f8.seq_stride + static_cast<long long>(t_row) * kDrow;
+        }
+        return true;
+    }
+};
+
 // kPaged: map_cache is 2-D over the page pool ([num_pages * page_size][576]) and each tile's row
-// comes from the block table; otherwise it is 3-D ([B][Lmax][576]).
-template <bool kPaged, bool kRopeQ>
-__global__ void __launch_bounds__(kThreads, 1)
+// comes from the block table; otherwise it is 3-D ([B][Lmax][576]). kFp8: map_cache is unused and
+// the cache is read through f8.
+template <bool kPaged, bool kRopeQ, bool kFp8>
+__global__ void __launch_bounds__(kFp8 ? kThreadsF8 : kThreads, 1)
 mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_constant__ CUtensorMap map_q,
                  const int *__restrict__ seq_lens, int B, float score_scale_log2, Partials ws, PagedCache pc,
-                 const __grid_constant__ RopeQ rq) {
+                 const __grid_constant__ RopeQ rq, Fp8Cache f8) {
+    constexpr int NSt = kStages;  // depth of the operand ring
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -262,6 +342,8 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                 count = 4;  // one arrival per softmax warp
             if (i == kBarSFull || i == kBarSFull + 1 || i == kBarQEmpty)
                 count = 2;  // one commit per GEMM1 warp
+            if (kFp8 && ((i >= kBarFull && i < kBarFull + NSt) || i == kBarQF16))
+                count = 4;  // one arrival per converter warp
             if (i == kBarDrain) count = 3;  // every MMA warp
             mbar_init(bar(i), count);
         }
@@ -301,8 +383,9 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                 mbar_arrive_tx_elect(bar(kBarQFull), kQBytes);
                 for (int c = 0; c < kNChunk; ++c)
                     lad::ptx::tma_load_2d_elect(sbase + kOffQ + c * kQChunkBytes, &map_q, c * kChunk, seq * kHq, bar(kBarQFull));
-                for (int i = 0; i < nt; ++i, ++g) {
-                    const uint32_t s = g % kStages;
+                // (FP8 cache: the widening warps load the tiles themselves)
+                for (int i = 0; i < (kFp8 ? 0 : nt); ++i, ++g) {
+                    const uint32_t s = g % NSt;
                     int row = (tile0 + i) * kTile;
                     if constexpr (kPaged) {
                         // warp-uniform: every lane computes the same page index
@@ -323,7 +406,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                             if (lane == 0) atomicCAS(&g_mla_error, 0, lad::kErrMlaBlockTable);
                         }
                     }
-                    if (!wait_bar(bar(kBarEmpty + s), ((g / kStages) & 1) ^ 1, abort_flag, lad::kErrMlaProducer)) {
+                    if (!wait_bar(bar(kBarEmpty + s), ((g / NSt) & 1) ^ 1, abort_flag, lad::kErrMlaProducer)) {
                         ok = false;
                         break;
                     }
@@ -331,9 +414,11 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     const uint32_t dst = sbase + kOffStage + s * kStageBytes;
                     for (int c = 0; c < kNChunk; ++c) {
                         if constexpr (kPaged)
-                            lad::ptx::tma_load_2d_elect(dst + c * kTChunkBytes, &map_cache, c * kChunk, row, bar(kBarFull + s));
+                            lad::ptx::tma_load_2d_elect(dst + c * kTChunkBytes, &map_cache, c * kChunk, row,
+                                                        bar(kBarFull + s));
                         else
-                            lad::ptx::tma_load_3d_elect(dst + c * kTChunkBytes, &map_cache, c * kChunk, row, seq, bar(kBarFull + s));
+                            lad::ptx::tma_load_3d_elect(dst + c * kTChunkBytes, &map_cache, c * kChunk, row, seq,
+                                                        bar(kBarFull + s));
                     }
                 }
                 ++k;
@@ -341,11 +426,10 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             if (!ok) {
                 // drain: every load this thread issued completes on its full barrier
                 const uint32_t issued = g;
-                for (uint32_t j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
-                    const uint32_t s = j % kStages;
+                for (uint32_t j = (issued > NSt ? issued - NSt : 0); j < issued; ++j) {
+                    const uint32_t s = j % NSt;
                     const uint64_t tt = globaltimer_ns();
-                    while (!mbar_try_wait(bar(kBarFull + s), (j / kStages) & 1) &&
-                           globaltimer_ns() - tt < kWaitLimitNs) {
+                    while (!mbar_try_wait(bar(kBarFull + s), (j / NSt) & 1) && globaltimer_ns() - tt < kWaitLimitNs) {
                     }
                 }
                 if (k > 0) {
@@ -368,14 +452,15 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             const uint64_t q_desc0 = smem_desc(sbase + kOffQ, 16, 1024, kLayoutSw128);
             const uint64_t c_desc0 = smem_desc(sbase + kOffStage, 16, 1024, kLayoutSw128);
             while (ok && it.next(seq, tile0, nt)) {
-                if (!wait_bar(bar(kRopeQ ? kBarQRoped : kBarQFull), k & 1, abort_flag, lad::kErrMlaMma)) {
+                if (!wait_bar(bar(kFp8 ? kBarQF16 : (kRopeQ ? kBarQRoped : kBarQFull)), k & 1, abort_flag,
+                              lad::kErrMlaMma)) {
                     ok = false;
                     break;
                 }
                 for (int i = 0; i < nt; ++i, ++g) {
-                    const uint32_t s = g % kStages;
+                    const uint32_t s = g % NSt;
                     const uint32_t sb = g & 1;
-                    if (!wait_bar(bar(kBarFull + s), (g / kStages) & 1, abort_flag, lad::kErrMlaMma) ||
+                    if (!wait_bar(bar(kBarFull + s), (g / NSt) & 1, abort_flag, lad::kErrMlaMma) ||
                         !wait_bar(bar(kBarSEmpty + sb), ((g >> 1) & 1) ^ 1, abort_flag, lad::kErrMlaMma)) {
                         ok = false;
                         break;
@@ -388,7 +473,8 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             tc_mma(dS + mi * kTile, q_desc0 + ((c * kQChunkBytes + kk * 32) >> 4),
-                                   cd + ((c * kTChunkBytes + kk * 32) >> 4), kIdesc1, (c > 1 || kk > 0) ? 1u : 0u);
+                                   cd + ((c * kTChunkBytes + kk * 32) >> 4), kFp8 ? kIdesc1F16 : kIdesc1,
+                                   (c > 1 || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(bar(kBarSFull + sb));
                     if (i == nt - 1) tc_commit(bar(kBarQEmpty));
@@ -450,7 +536,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t s = g % kStages;
+                    const uint32_t s = g % NSt;
                     // A = V^T: 128 latent dims (two 64-wide chunks, LBO apart) x 16 tokens (two 8-row groups)
                     const uint64_t a0 = v_desc0 + ((s * kStageBytes) >> 4);
                     // B = P: 64 heads (8-row core groups, SBO 512) x 16 tokens (two 8-token core columns, LBO 128)
@@ -461,7 +547,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
                             tc_mma(tmem + kColO + 64 * j, a0 + (((2 * j) * kTChunkBytes + kk * 2048) >> 4),
-                                   b0 + ((kk * 256) >> 4), kIdesc2, kk == 0 ? acc0 : 1u);
+                                   b0 + ((kk * 256) >> 4), kFp8 ? kIdesc2F16 : kIdesc2, kk == 0 ? acc0 : 1u);
                     }
                     tc_commit(bar(kBarEmpty + s));
                     tc_commit(bar(kBarPEmpty + pb));
@@ -473,7 +559,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer_ns() - tt < kWaitLimitNs) {
             }
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 8) {
         // ================= softmax, rescale and epilogue (warps 4..7) =================
         const int p = warp & 3;                 // TMEM sub-partition
         const bool owner = lane < 16;           // this lane owns head 16p + lane
@@ -517,11 +603,13 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
 #pragma unroll
                     for (int j = 0; j < kTile / 2; ++j)
                         if (mytok0 + j >= len) xs[j] = -INFINITY;
+                }
+                if (!kFp8 && tok0 + kTile > len) {  // (the FP8 converter already wrote those rows as zeros)
                     // Rows past the length get weight 0, but 0 * (NaN or Inf) would still reach O:
                     // zero their latent part in the stage (GEMM1 is done with it, GEMM2 waits for
                     // P_full, which follows the proxy fence below).
                     const int valid = len - tok0;
-                    uint8_t *stage = smem + kOffStage + (g % kStages) * kStageBytes;
+                    uint8_t *stage = smem + kOffStage + (g % NSt) * kStageBytes;
                     for (int idx = threadIdx.x - 128; idx < (kTile - valid) * 64; idx += 128) {
                         const int rr = valid + (idx >> 6);
                         const int c = (idx >> 3) & 7;
@@ -559,7 +647,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                     const float p0 = ex2_approx(fmaf(xs[j], score_scale_log2, -m));
                     const float p1 = ex2_approx(fmaf(xs[j + 1], score_scale_log2, -m));
                     ps[(j >> 1) & 3] += p0 + p1;  // the denominator keeps fp32 probabilities
-                    pk[j / 2] = lad::dev::f32x2_to_bf16x2(p0, p1);
+                    pk[j / 2] = kFp8 ? f32x2_to_f16x2(p0, p1) : lad::dev::f32x2_to_bf16x2(p0, p1);
                 }
                 float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
                 psum += __shfl_xor_sync(0xffffffffu, psum, 16);
@@ -653,6 +741,99 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
             ++k;
         }
         (void)ok;
+    } else if constexpr (kFp8) {
+        // ================= FP8 widening (warps 8..11) =================
+        // Per segment, q (bf16, turned in the RoPE variant) becomes f16 in place. Per tile, thread
+        // (r, jj) holds codes 16jj..16jj+15 of row r of each of the 9 64-wide chunks (9 x 16 bytes),
+        // loaded two tiles ahead into one of two register sets, and writes them widened as two
+        // 16-byte pieces of the swizzled f16 row. Rows at or past the length (or Lmax, or in a page
+        // outside the pool) are not loaded and become zeros.
+        const int ct = static_cast<int>(threadIdx.x) - 256;
+        const int r = ct >> 2, jj = ct & 3;
+        const uint32_t o0 = static_cast<uint32_t>(r * 128 + (((2 * jj) ^ (r & 7)) << 4));
+        const uint32_t o1 = static_cast<uint32_t>(r * 128 + (((2 * jj + 1) ^ (r & 7)) << 4));
+        // The load cursor runs two tiles ahead of the conversion (two register sets).
+        Fp8Cursor<kPaged> cl(it, seq_lens, f8, pc);
+        auto load_next = [&](uint4 (&buf)[kNChunk]) {
+            const uint8_t *p = nullptr;
+            int n = 0;
+            if (!cl.next(lane, p, n)) n = 0;
+            const uint8_t *src = r < n ? p + r * kDrow + jj * 16 : nullptr;
+#pragma unroll
+            for (int c = 0; c < kNChunk; ++c) {
+                if (src) {
+                    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(buf[c].x), "=r"(buf[c].y), "=r"(buf[c].z), "=r"(buf[c].w)
+                                 : "l"(src + c * kChunk));
+                } else {
+                    buf[c] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+        };
+        auto widen = [&](const uint4 (&buf)[kNChunk], uint8_t *dst) {
+#pragma unroll
+            for (int c = 0; c < kNChunk; ++c) {
+                const uint4 in = buf[c];
+                *reinterpret_cast<uint4 *>(dst + c * kTChunkBytes + o0) =
+                    make_uint4(e4m3x2_to_f16x2(in.x), e4m3x2_to_f16x2(in.x >> 16), e4m3x2_to_f16x2(in.y),
+                               e4m3x2_to_f16x2(in.y >> 16));
+                *reinterpret_cast<uint4 *>(dst + c * kTChunkBytes + o1) =
+                    make_uint4(e4m3x2_to_f16x2(in.z), e4m3x2_to_f16x2(in.z >> 16), e4m3x2_to_f16x2(in.w),
+                               e4m3x2_to_f16x2(in.w >> 16));
+            }
+        };
+        uint4 bufA[kNChunk], bufB[kNChunk];
+        load_next(bufA);
+        load_next(bufB);
+        int seq, tile0, nt, k = 0;
+        uint32_t g = 0;
+        bool ok = true;
+        while (ok && it.next(seq, tile0, nt)) {
+            if (!wait_bar(bar(kRopeQ ? kBarQRoped : kBarQFull), k & 1, abort_flag, lad::kErrMlaConvert)) {
+                ok = false;
+                break;
+            }
+            {
+                uint4 *qv = reinterpret_cast<uint4 *>(smem + kOffQ);
+                bool over = false;
+#pragma unroll 2
+                for (int i = ct; i < kQBytes / 16; i += 128) {
+                    const uint4 w = qv[i];
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                    uint32_t hs[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float lo = __uint_as_float(ws[u] << 16), hi = __uint_as_float(ws[u] & 0xffff0000u);
+                        over |= fabsf(lo) > 65504.f || fabsf(hi) > 65504.f;
+                        hs[u] = f32x2_to_f16x2(lo, hi);
+                    }
+                    qv[i] = make_uint4(hs[0], hs[1], hs[2], hs[3]);
+                }
+                if (__any_sync(0xffffffffu, over) && lane == 0) atomicCAS(&g_mla_error, 0, lad::kErrMlaQRange);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarQF16));
+            }
+            ++k;
+            for (int i = 0; i < nt; ++i, ++g) {
+                const uint32_t s = g % NSt;
+                if (!wait_bar(bar(kBarEmpty + s), ((g / NSt) & 1) ^ 1, abort_flag, lad::kErrMlaConvert)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *dst = smem + kOffStage + s * kStageBytes;
+                if (g & 1) {
+                    widen(bufB, dst);
+                    load_next(bufB);
+                } else {
+                    widen(bufA, dst);
+                    load_next(bufA);
+                }
+                fence_async_smem();  // the tensor core (async proxy) reads what these stores wrote
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarFull + s));
+            }
+        }
     }
 
     tc_fence_before();
@@ -666,7 +847,7 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
 template <bool kOutF32>
 __global__ void __launch_bounds__(128)
 mla_combine_kernel(const int *__restrict__ seq_lens, int B, int G, const float *__restrict__ gate,
-                   Partials ws, void *__restrict__ out, float *__restrict__ lse_out) {
+                   Partials ws, void *__restrict__ out, float *__restrict__ lse_out, float value_scale) {
     const int b = blockIdx.x, h = blockIdx.y;
     const int d = 4 * threadIdx.x;
     __shared__ int s_c[2];
@@ -735,7 +916,7 @@ mla_combine_kernel(const int *__restrict__ seq_lens, int B, int G, const float *
             acc.w = fmaf(w, v.w, acc.w);
         }
     }
-    float sc = (Lsum > 0.f) ? 1.f / Lsum : 0.f;
+    float sc = (Lsum > 0.f) ? value_scale / Lsum : 0.f;
     if (gate) sc *= 1.f / (1.f + expf(-gate[b * kHq + h]));
     acc.x *= sc;
     acc.y *= sc;
@@ -822,14 +1003,18 @@ int set_smem_attributes(const char *name) {
     if (dev < 0 || dev >= 64) return lad::set_error(LAD_EUNSUPPORTED, "%s: device %d", name, dev);
     std::lock_guard<std::mutex> lock(mu);
     if (!done[dev]) {
-        e = cudaFuncSetAttribute(mla_split_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(mla_split_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(mla_split_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kSmemBytes);
+        const void *kernels[] = {
+            reinterpret_cast<const void *>(mla_split_kernel<false, false, false>),
+            reinterpret_cast<const void *>(mla_split_kernel<true, false, false>),
+            reinterpret_cast<const void *>(mla_split_kernel<true, true, false>),
+            reinterpret_cast<const void *>(mla_split_kernel<false, false, true>),
+            reinterpret_cast<const void *>(mla_split_kernel<true, false, true>),
+            reinterpret_cast<const void *>(mla_split_kernel<true, true, true>),
+        };
+        for (const void *k : kernels) {
+            e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            if (e != cudaSuccess) break;
+        }
         if (e != cudaSuccess)
             return lad::set_error(LAD_ECUDA, "%s: smem attribute: %s", name, cudaGetErrorString(e));
         done[dev] = true;
@@ -882,10 +1067,12 @@ int encode_contiguous(const char *name, CUtensorMap *map, const lad_bf16 *cache,
     return encode_cache_map(name, map, cache, 3, dims, strides);
 }
 
-// Everything after the argument checks: the q map, the split kernel and the combine.
+// Everything after the argument checks: the q map, the split kernel and the combine. f8 non-null:
+// the cache is FP8 (map_cache unused), every element worth kv_scale times its code.
 int run_mla(const char *name, const CUtensorMap &map_cache, bool paged, const PagedCache &pc, const RopeQ *rope,
             const lad_bf16 *q, const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B,
-            float scale, unsigned flags, uint8_t *ws, const WsLayout &wl, int G, void *stream) {
+            float scale, unsigned flags, uint8_t *ws, const WsLayout &wl, int G, void *stream,
+            const Fp8Cache *f8 = nullptr, float kv_scale = 1.f) {
     using lad::set_error;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return set_error(LAD_ECUDA, "%s: cuTensorMapEncodeTiled unavailable", name);
@@ -907,24 +1094,37 @@ int run_mla(const char *name, const CUtensorMap &map_cache, bool paged, const Pa
     Partials parts{reinterpret_cast<float *>(ws + wl.off_O), reinterpret_cast<float *>(ws + wl.off_m),
                    reinterpret_cast<float *>(ws + wl.off_l), reinterpret_cast<long long *>(ws + wl.off_prefix)};
     cudaStream_t s = lad::as_stream(stream);
-    const float score_scale_log2 = scale * 1.4426950408889634f;
+    const float score_scale_log2 = scale * kv_scale * 1.4426950408889634f;
     const RopeQ none{};
-    if (rope)
-        mla_split_kernel<true, true><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B, score_scale_log2,
-                                                                      parts, pc, *rope);
-    else if (paged)
-        mla_split_kernel<true, false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
-                                                                       score_scale_log2, parts, pc, none);
-    else
-        mla_split_kernel<false, false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
-                                                                        score_scale_log2, parts, pc, none);
+    const RopeQ &rq = rope ? *rope : none;
+    const Fp8Cache fc = f8 ? *f8 : Fp8Cache{};
+    if (f8) {
+        if (rope)
+            mla_split_kernel<true, true, true><<<G, kThreadsF8, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
+                                                                                 score_scale_log2, parts, pc, rq, fc);
+        else if (paged)
+            mla_split_kernel<true, false, true><<<G, kThreadsF8, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
+                                                                                  score_scale_log2, parts, pc, rq, fc);
+        else
+            mla_split_kernel<false, false, true><<<G, kThreadsF8, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
+                                                                                   score_scale_log2, parts, pc, rq, fc);
+    } else if (rope) {
+        mla_split_kernel<true, true, false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
+                                                                            score_scale_log2, parts, pc, rq, fc);
+    } else if (paged) {
+        mla_split_kernel<true, false, false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
+                                                                             score_scale_log2, parts, pc, rq, fc);
+    } else {
+        mla_split_kernel<false, false, false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
+                                                                              score_scale_log2, parts, pc, rq, fc);
+    }
     rc = lad::check_launch(name);
     if (rc != LAD_OK) return rc;
     const dim3 cgrid(static_cast<unsigned>(B), kHq);
     if (flags & LAD_FLAG_OUT_FP32)
-        mla_combine_kernel<true><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
+        mla_combine_kernel<true><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out, kv_scale);
     else
-        mla_combine_kernel<false><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out);
+        mla_combine_kernel<false><<<cgrid, 128, 0, s>>>(seq_lens, B, G, gate_logits, parts, o, lse_out, kv_scale);
     return lad::check_launch(name);
 }
 
@@ -973,10 +1173,11 @@ extern "C" int mla_latent_decode(const lad_bf16 *q, const lad_bf16 *cache, long 
 }
 
 namespace {
-int run_paged(const char *name, const lad_bf16 *q, const lad_bf16 *kv_pages, int num_pages, int page_size,
+int run_paged(const char *name, const lad_bf16 *q, const void *kv_pages, int num_pages, int page_size,
               const int *block_table, int block_table_stride, const int *seq_lens, const float *gate_logits, void *o,
               float *lse_out, int B, int Hq, int d_latent, int d_rope, float scale, unsigned flags,
-              unsigned extra_flags, const RopeQ *rope, void *workspace, size_t ws_bytes, void *stream) {
+              unsigned extra_flags, const RopeQ *rope, void *workspace, size_t ws_bytes, void *stream,
+              bool fp8 = false, float kv_scale = 1.f) {
     using lad::set_error;
     int rc = check_common(name, B, Hq, d_latent, d_rope, flags & ~extra_flags, scale);
     if (rc != LAD_OK) return rc;
@@ -996,17 +1197,20 @@ int run_paged(const char *name, const lad_bf16 *q, const lad_bf16 *kv_pages, int
     if (!workspace || ws_bytes < wl.total || !lad::aligned(workspace, 256))
         return set_error(LAD_EWORKSPACE, "%s: workspace of %zu bytes (256-aligned) required", name, wl.total);
     CUtensorMap map_cache;
+    std::memset(&map_cache, 0, sizeof map_cache);
     // an empty pool still gets a one-row extent; every tile then reads as zeros
     const int rows = num_pages > 0 ? num_pages * page_size : 1;
-    {
+    if (!fp8) {
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDrow), static_cast<cuuint64_t>(rows)};
         const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDrow) * 2};
-        rc = encode_cache_map(name, &map_cache, kv_pages, 2, dims, strides);
+        rc = encode_cache_map(name, &map_cache, static_cast<const lad_bf16 *>(kv_pages), 2, dims, strides);
         if (rc != LAD_OK) return rc;
     }
     const PagedCache pc{block_table, block_table_stride, page_size, num_pages, rows};
+    const Fp8Cache f8{static_cast<const uint8_t *>(kv_pages), 0, 0};
     return run_mla(name, map_cache, true, pc, rope, q, seq_lens, gate_logits, o, lse_out, B, scale,
-                   flags & ~extra_flags, static_cast<uint8_t *>(workspace), wl, G, stream);
+                   flags & ~extra_flags, static_cast<uint8_t *>(workspace), wl, G, stream, fp8 ? &f8 : nullptr,
+                   kv_scale);
 }
 }  // namespace
 
@@ -1037,6 +1241,69 @@ extern "C" int mla_latent_decode_paged_rope(const lad_bf16 *q, const int *positi
     return run_paged(name, q, kv_pages, num_pages, page_size, block_table, block_table_stride, seq_lens, gate_logits,
                      o, lse_out, B, Hq, d_latent, d_rope, scale, flags, LAD_FLAG_ROPE_INTERLEAVED, &rq, workspace,
                      ws_bytes, stream);
+}
+
+// ------------------------------------------------------------------------------------------
+// FP8 (E4M3) cache: the same attention with every cached element worth kv_scale * E4M3(code).
+// ------------------------------------------------------------------------------------------
+namespace {
+int check_kv_scale(const char *name, float kv_scale) {
+    if (!(kv_scale > 0.f) || kv_scale == INFINITY)
+        return lad::set_error(LAD_EINVAL, "%s: kv_scale must be positive and finite", name);
+    return LAD_OK;
+}
+}  // namespace
+
+extern "C" int mla_latent_decode_fp8(const lad_bf16 *q, const uint8_t *cache, long long cache_seq_stride,
+                                     float kv_scale, const int *seq_lens, const float *gate_logits, void *o,
+                                     float *lse_out, int B, int Hq, int d_latent, int d_rope, int Lmax, float scale,
+                                     unsigned flags, void *workspace, size_t ws_bytes, void *stream) {
+    using lad::set_error;
+    const char *name = "mla_latent_decode_fp8";
+    int rc = check_common(name, B, Hq, d_latent, d_rope, flags, scale);
+    if (rc == LAD_OK) rc = check_kv_scale(name, kv_scale);
+    if (rc != LAD_OK) return rc;
+    if (Lmax < 0) return set_error(LAD_EINVAL, "%s: negative Lmax", name);
+    if (B == 0) return LAD_OK;
+    rc = check_pointers(name, q, cache, seq_lens, o, flags);
+    if (rc != LAD_OK) return rc;
+    if (cache_seq_stride < static_cast<long long>(Lmax) * kDrow || cache_seq_stride % 16 != 0)
+        return set_error(LAD_EINVAL, "%s: cache_seq_stride must be >= Lmax*576 and a multiple of 16", name);
+    int G = 0;
+    rc = sm_count_checked(name, &G);
+    if (rc != LAD_OK) return rc;
+    const WsLayout wl = ws_layout(B, G);
+    if (!workspace || ws_bytes < wl.total || !lad::aligned(workspace, 256))
+        return set_error(LAD_EWORKSPACE, "%s: workspace of %zu bytes (256-aligned) required", name, wl.total);
+    CUtensorMap unused;
+    std::memset(&unused, 0, sizeof unused);
+    const Fp8Cache f8{cache, cache_seq_stride, Lmax};
+    return run_mla(name, unused, false, PagedCache{}, nullptr, q, seq_lens, gate_logits, o, lse_out, B, scale, flags,
+                   static_cast<uint8_t *>(workspace), wl, G, stream, &f8, kv_scale);
+}
+
+extern "C" int mla_latent_decode_paged_fp8(const lad_bf16 *q, const int *positions, float rope_theta,
+                                           const uint8_t *kv_pages, float kv_scale, int num_pages, int page_size,
+                                           const int *block_table, int block_table_stride, const int *seq_lens,
+                                           const float *gate_logits, void *o, float *lse_out, int B, int Hq,
+                                           int d_latent, int d_rope, float scale, unsigned flags, void *workspace,
+                                           size_t ws_bytes, void *stream) {
+    const char *name = "mla_latent_decode_paged_fp8";
+    int rc = check_kv_scale(name, kv_scale);
+    if (rc != LAD_OK) return rc;
+    if (!positions)
+        return run_paged(name, q, kv_pages, num_pages, page_size, block_table, block_table_stride, seq_lens,
+                         gate_logits, o, lse_out, B, Hq, d_latent, d_rope, scale, flags, 0u, nullptr, workspace,
+                         ws_bytes, stream, true, kv_scale);
+    if (!(rope_theta > 1.f) || rope_theta == INFINITY)
+        return lad::set_error(LAD_EINVAL, "%s: rope_theta must be > 1", name);
+    RopeQ rq{};
+    rq.positions = positions;
+    rq.interleaved = (flags & LAD_FLAG_ROPE_INTERLEAVED) ? 1 : 0;
+    if (d_rope == kDr) lad::rope_inverse_frequencies(static_cast<double>(rope_theta), kDr, rq.inv_freq);
+    return run_paged(name, q, kv_pages, num_pages, page_size, block_table, block_table_stride, seq_lens, gate_logits,
+                     o, lse_out, B, Hq, d_latent, d_rope, scale, flags, LAD_FLAG_ROPE_INTERLEAVED, &rq, workspace,
+                     ws_bytes, stream, true, kv_scale);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -140,6 +140,28 @@ __device__ __forceinline__ void tma_load_3d_elect(uint32_t dst, const void *map,
         : "memory");
 }
 
+// Two E4M3 codes (the first in the low byte) to an f16 pair (the first in the low half): one
+// conversion, exact (every E4M3 value is an f16 normal or zero; NaN stays NaN).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(static_cast<uint16_t>(two_codes)));
+    return r;
+}
+
+// Two floats to an f16 pair (lo in the low half), rounded to nearest even.
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two floats to E4M3 codes (a in the low byte), rounded to nearest even, saturating at +-448.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float a, float b) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+    return r;
+}
+
 // 2^x, the MUFU approximation (flushes subnormals); softmax exponents in log2 units.
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
@@ -227,6 +249,7 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N, uint32_t ab_form
            (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);
 }
+constexpr uint32_t kFmtF16 = 0;
 constexpr uint32_t kFmtBf16 = 1;
 constexpr uint32_t kFmtTf32 = 2;
 

@@ -386,9 +386,10 @@ int lado_e4m3_encode(int n, const double *x, uint8_t *out) {
     return LADO_OK;
 }
 
-/* Element d of a cache row: bf16 bits (fp8 == 0) or an E4M3 code times the cache's scale. */
-static double cache_elem(const void *cache, int fp8, double kv_scale, size_t i) {
-    if (fp8) return kv_scale * e4m3_to_double(((const uint8_t *)cache)[i]);
+/* Element i of the cache: bf16 bits (fp8_value == NULL), or an E4M3 code looked up in
+ * fp8_value[code] = kv_scale * E4M3(code) (filled once per call from e4m3_to_double). */
+static double cache_elem(const void *cache, const double *fp8_value, size_t i) {
+    if (fp8_value) return fp8_value[((const uint8_t *)cache)[i]];
     return bf16_bits_to_double(((const uint16_t *)cache)[i]);
 }
 
@@ -402,6 +403,9 @@ static int mla_decode_impl(int B, int H, int Dc, int Dr, const double *q, const 
     if (nthreads < 1) nthreads = 1;
     const int D = Dc + Dr;
     int err = 0;
+    double fp8_table[256];
+    for (int c = 0; c < 256; ++c) fp8_table[c] = kv_scale * e4m3_to_double((uint8_t)c);
+    const double *fp8_value = fp8 ? fp8_table : NULL;
 #pragma omp parallel for num_threads(nthreads) collapse(2) schedule(dynamic)
     for (int b = 0; b < B; ++b) {
         for (int h = 0; h < H; ++h) {
@@ -425,7 +429,7 @@ static int mla_decode_impl(int B, int H, int Dc, int Dr, const double *q, const 
             for (int t = 0; t < L; ++t) {
                 const size_t ct = cb + mla_row(bt, P, D, t);
                 double acc = 0.0;
-                for (int d = 0; d < D; ++d) acc += qh[d] * cache_elem(cache, fp8, kv_scale, ct + (size_t)d);
+                for (int d = 0; d < D; ++d) acc += qh[d] * cache_elem(cache, fp8_value, ct + (size_t)d);
                 s[t] = scale * acc;
                 if (s[t] > m) m = s[t];
             }
@@ -438,7 +442,7 @@ static int mla_decode_impl(int B, int H, int Dc, int Dr, const double *q, const 
             for (int t = 0; t < L; ++t) {
                 const size_t ct = cb + mla_row(bt, P, D, t);
                 double p = s[t] / z;
-                for (int d = 0; d < Dc; ++d) oh[d] += p * cache_elem(cache, fp8, kv_scale, ct + (size_t)d);
+                for (int d = 0; d < Dc; ++d) oh[d] += p * cache_elem(cache, fp8_value, ct + (size_t)d);
             }
             if (gate) {
                 double sg = 1.0 / (1.0 + exp(-gate[(size_t)b * H + h]));

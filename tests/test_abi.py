@@ -76,3 +76,39 @@ def test_host_side_validation_of_the_newer_calls(lib):
     assert lib.mla_cache_append(*(a[:13] + [0.5] + a[14:])) == -1
     assert lib.mla_cache_append(*(a[:4] + [576] + a[5:])) == -1 and b"cache_seq_stride" in lib.lad_last_error()
     assert lib.mla_cache_append(*(a[:10] + [0] + a[11:])) == 0
+
+
+def test_host_side_validation_of_the_fp8_calls(lib):
+    """FP8 cache calls: kv_scale, stride and alignment checks return before any CUDA call."""
+    # mla_latent_decode_fp8(q, cache, stride, kv_scale, lens, gate, o, lse, B, Hq, Dl, Dr, Lmax, scale, flags, ws,
+    #                       ws_bytes, stream)
+    d = [16, 16, 576 * 8, 0.5, 16, None, 16, None, 1, 64, 512, 64, 8, 0.1, 0, 16, 1 << 20, None]
+    bad = list(d); bad[3] = 0.0
+    assert lib.mla_latent_decode_fp8(*bad) == -1 and b"kv_scale" in lib.lad_last_error()
+    bad = list(d); bad[3] = float("inf")
+    assert lib.mla_latent_decode_fp8(*bad) == -1
+    bad = list(d); bad[2] = 576 * 8 + 8  # bytes between sequences must be a multiple of 16
+    assert lib.mla_latent_decode_fp8(*bad) == -1 and b"multiple of 16" in lib.lad_last_error()
+    bad = list(d); bad[1] = 24  # the cache must be 16-byte aligned
+    assert lib.mla_latent_decode_fp8(*bad) == -2
+    bad = list(d); bad[8] = 0
+    assert lib.mla_latent_decode_fp8(*bad) == 0
+    # mla_latent_decode_paged_fp8(q, positions, theta, pages, kv_scale, num_pages, page_size, bt, bt_stride, lens,
+    #                             gate, o, lse, B, Hq, Dl, Dr, scale, flags, ws, ws_bytes, stream)
+    p = [16, None, 6.0e6, 16, 0.5, 4, 48, 16, 1, 16, None, 16, None, 1, 64, 512, 64, 0.1, 0, 16, 1 << 20, None]
+    assert lib.mla_latent_decode_paged_fp8(*p) == -2 and b"multiple of 32" in lib.lad_last_error()
+    bad = list(p); bad[6] = 64; bad[4] = -1.0
+    assert lib.mla_latent_decode_paged_fp8(*bad) == -1 and b"kv_scale" in lib.lad_last_error()
+    bad = list(p); bad[6] = 64; bad[1] = 16; bad[2] = 0.5
+    assert lib.mla_latent_decode_paged_fp8(*bad) == -1 and b"rope_theta" in lib.lad_last_error()
+    bad = list(p); bad[6] = 64; bad[18] = 1 << 4  # the interleaved pairing needs positions
+    assert lib.mla_latent_decode_paged_fp8(*bad) == -1
+    # mla_cache_append_fp8(c_kv, k_pe, positions, cache, stride, Lmax, bt, bt_stride, num_pages, page_size, B, Dl,
+    #                      Dr, theta, kv_scale, flags, stream)
+    a = [16, 16, 16, 16, 576 * 8, 8, None, 0, 0, 0, 1, 512, 64, 6.0e6, 0.5, 0, None]
+    bad = list(a); bad[14] = 0.0
+    assert lib.mla_cache_append_fp8(*bad) == -1 and b"kv_scale" in lib.lad_last_error()
+    bad = list(a); bad[4] = 576 * 8 + 8
+    assert lib.mla_cache_append_fp8(*bad) == -1 and b"multiple of 16" in lib.lad_last_error()
+    bad = list(a); bad[10] = 0
+    assert lib.mla_cache_append_fp8(*bad) == 0

@@ -86,6 +86,28 @@ def normal_bf16(shape, seed: int, name: str, device="cpu", std: float = 1.0) -> 
     return out
 
 
+E4M3_CODE_STD = 32.0
+KV_SCALE_FP8 = 1.0 / E4M3_CODE_STD
+
+
+def e4m3_codes(shape, seed: int, name: str, device="cpu", std: float = E4M3_CODE_STD) -> torch.Tensor:
+    """E4M3 codes (uint8) of N(0, std^2) draws, cast by torch's float8_e4m3fn conversion (round to
+    nearest even), drawn slice by slice along dim 0. With std = 32 the draws stay far inside the
+    format's +-448; with kv_scale = 1/32 a cache of these codes holds elements distributed like the
+    bf16 cache's N(0, 1)."""
+    shape = tuple(int(s) for s in shape)
+    out = torch.empty(shape, device=device, dtype=torch.uint8)
+    g = _gen(seed, name, device)
+    rows = shape[0]
+    per_row = int(np.prod(shape[1:])) if len(shape) > 1 else 1
+    step_rows = max(1, (1 << 27) // max(per_row, 1))
+    for r in range(0, rows, step_rows):
+        m = min(step_rows, rows - r)
+        chunk = torch.randn((m,) + shape[1:], generator=g, device=device, dtype=torch.float32).mul_(std)
+        out[r:r + m] = chunk.to(torch.float8_e4m3fn).view(torch.uint8)
+    return out
+
+
 def unit_sphere_bf16(shape, seed: int, name: str, device="cpu") -> torch.Tensor:
     """Directions uniform on the unit sphere over the last axis (Gaussian / its length), bf16."""
     x = normal(shape, seed, name, device).double()
@@ -239,6 +261,12 @@ def mla_inputs(cfg: MlaDecode, device="cpu", lmax: int | None = None) -> dict:
         "seq_lens": lens.to(device),
         "gate": normal((cfg.B, cfg.Hq), s, "mla_gate", device),
     }
+
+
+def mla_fp8_cache(cfg: MlaDecode, device="cpu", lmax: int | None = None) -> torch.Tensor:
+    """The FP8 latent cache of an MLA workload: E4M3 codes [B, Lmax, 576] (kv_scale KV_SCALE_FP8)."""
+    L = int(mla_seq_lens(cfg).max().item()) if lmax is None else int(lmax)
+    return e4m3_codes((cfg.B, L, D_ROW), cfg.seed, "mla_cache_fp8", device)
 
 
 def paginate(cache: torch.Tensor, seq_lens: torch.Tensor, page_size: int, seed: int, spare_pages: int = 0):
