@@ -67,6 +67,20 @@ int lad_version(void);
 int lad_device_error(void *stream, int *code);
 
 /*
+ * lad_check_bounded_wait — a check of the failure handling above that faults nothing: it launches
+ * one CTA of two warps on `stream` whose barrier waits can never complete (nothing arrives on
+ * them). Warp 0's wait runs out after the bounded-wait limit (about 1 s), records tag 0x401 and
+ * raises the CTA's abort flag; warp 1, whose wait starts half a limit later, then returns at once
+ * instead of reaching its own limit; the kernel returns and the context stays usable.
+ * Synchronises `stream`.
+ *   tag      receives the recorded device error tag (0x401 expected)
+ *   results  int[4]: warp 0's wait result (0 = gave up), warp 1's wait result (0), milliseconds
+ *            warp 1 waited (about half the limit), the abort flag (1)
+ * Returns LAD_OK, LAD_EINVAL (null output) or LAD_ECUDA.
+ */
+int lad_check_bounded_wait(int *tag, int *results, void *stream);
+
+/*
  * kda_conv_update — one decode step of the short causal depthwise convolution in front of
  * the KDA recurrence. [P2] "How KDA and MLA split the work": q, k and v come through a short
  * causal convolution of width 4; [P2] "Does 292 GiB fit on four Hopper GPUs?": the layer keeps

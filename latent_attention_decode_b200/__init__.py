@@ -23,7 +23,7 @@ __all__ = [
     "mla_latent_decode", "mla_latent_decode_workspace_size", "mla_latent_decode_paged",
     "mla_latent_decode_paged_rope", "mla_cache_append", "mla_latent_decode_fp8", "mla_latent_decode_paged_fp8",
     "mla_cache_append_fp8", "mla_latent_decode_noalloc",
-    "lad_device_error", "lad_version",
+    "lad_device_error", "lad_check_bounded_wait", "lad_version",
     "LadError", "LIB_PATH", "FLAG_SILU", "FLAG_L2NORM_QK", "FLAG_OUT_FP32", "FLAG_KEEP_STATE",
     "FLAG_ROPE_INTERLEAVED", "MLA_SCALE", "ROPE_THETA",
 ]
@@ -62,6 +62,7 @@ def _load() -> ctypes.CDLL:
         "lad_last_error": ([], ctypes.c_char_p),
         "lad_version": ([], _c_int),
         "lad_device_error": ([_c_vp, ctypes.POINTER(_c_int)], _c_int),
+        "lad_check_bounded_wait": ([ctypes.POINTER(_c_int), ctypes.POINTER(_c_int), _c_vp], _c_int),
         "kda_conv_update": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_u, _c_vp], _c_int),
         "kda_decode_step": ([_c_vp, _c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                              _c_int, _c_f, _c_u, _c_vp], _c_int),
@@ -160,6 +161,15 @@ def lad_device_error(stream=None) -> int:
     code = _c_int(0)
     _check("lad_device_error", _L().lad_device_error(_stream(stream), ctypes.byref(code)))
     return int(code.value)
+
+
+def lad_check_bounded_wait(stream=None) -> tuple[int, list[int]]:
+    """Runs the library's bounded-wait check (a barrier wait that can never complete; about 1 s).
+    Returns (tag, [warp 0 result, warp 1 result, ms warp 1 waited, abort flag])."""
+    tag = _c_int(0)
+    res = (_c_int * 4)()
+    _check("lad_check_bounded_wait", _L().lad_check_bounded_wait(ctypes.byref(tag), res, _stream(stream)))
+    return tag.value, list(res)
 
 
 def kda_conv_update(x: torch.Tensor, conv_tail: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None,

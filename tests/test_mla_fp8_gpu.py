@@ -99,6 +99,46 @@ def test_power_of_two_scale_equals_bf16_kernel(lad, cuda_device):
     assert rel_l2(o8, ob) < TOL_OUT
 
 
+def test_many_short_sequences(lad, cuda_device):
+    """More sequences than SMs: a CTA's share spans several segments, so the widening warps' load
+    cursor crosses sequences two tiles ahead of the conversion, and q is converted per segment."""
+    rng = np.random.default_rng(29)
+    lens = rng.integers(0, 200, size=400).tolist()
+    q, codes, L, gate = _inputs(lens, 200, 29, cuda_device)
+    o, lse = _run(lad, q, codes, L, gate, wl.KV_SCALE_FP8)
+    o_ref, lse_ref = _oracle(q, codes, L, gate, wl.KV_SCALE_FP8)
+    _check(o, lse, o_ref, lse_ref)
+
+
+def test_all_lengths_zero(lad, cuda_device):
+    q, codes, L, gate = _inputs([0, 0, 0], 8, 30, cuda_device)
+    o, lse = _run(lad, q, codes, L, gate, wl.KV_SCALE_FP8)
+    assert torch.count_nonzero(o) == 0 and torch.isinf(lse).all()
+
+
+def test_paged_many_sequences_and_bad_entry(lad, cuda_device):
+    """300 sequences in one shuffled pool of 32-row pages; then one table entry naming no page:
+    its rows read as zeros, device error 0x105, the other sequences unaffected."""
+    rng = np.random.default_rng(31)
+    lens = rng.integers(0, 400, size=300).tolist()
+    q, codes, L, gate = _inputs(lens, 400, 31, cuda_device)
+    pool, bt = wl.paginate(codes, L, 32, 31)
+    o = lad.mla_latent_decode_paged_fp8(q, pool, wl.KV_SCALE_FP8, bt, L, gate_logits=gate, out_fp32=True)
+    assert lad.lad_device_error() == 0
+    o_ref, _ = oracle.mla_decode_paged_fp8(f64(q), pool.cpu().numpy(), wl.KV_SCALE_FP8, bt.cpu().numpy(),
+                                           L.cpu().numpy(), f64(gate), scale=wl.MLA_SCALE,
+                                           nthreads=oracle.max_threads())
+    assert rel_l2(o, o_ref) < TOL_OUT
+    b0 = int(np.argmax(np.asarray(lens) > 64))  # a sequence with a second page
+    bad = bt.clone()
+    bad[b0, 1] = pool.shape[0] + 5
+    o2 = lad.mla_latent_decode_paged_fp8(q, pool, wl.KV_SCALE_FP8, bad, L, gate_logits=gate, out_fp32=True)
+    assert lad.lad_device_error() == 0x105
+    keep = [b for b in range(len(lens)) if b != b0]
+    assert rel_l2(o2[keep], o_ref[keep]) < TOL_OUT
+    assert torch.isfinite(o2[b0]).all()
+
+
 @pytest.mark.parametrize("page_size", [32, 128])
 def test_paged_scattered_pages(lad, cuda_device, page_size):
     lens = [1, 31, 33, 257, 0, 64, 200]
