@@ -211,14 +211,21 @@ int kda_conv_decode_step(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 
  *   beta         fp32 [B][T][H]
  *   S            fp32 [B][H][dk][dv]  initial state in, final state out
  *   o            [B][T][H][dv] bf16, or fp32 if flags & LAD_FLAG_OUT_FP32
- *   workspace    device scratch of ws_bytes >= kda_prefill_workspace_size(...) (may be NULL
- *                when that size is 0)
+ *   workspace    NULL, or device scratch of ws_bytes >= kda_prefill_workspace_size(...),
+ *                1 KiB aligned: with it the call runs two kernels per segment of up to 128
+ *                chunks (every chunk's state-independent operands in parallel, written to the
+ *                workspace as one 145 KiB record per (sequence, head, chunk); then the state
+ *                chain alone); without it, one kernel that does both per chunk. Same results
+ *                within rounding.
  * Supported: dk == dv == 128, chunk == 64; flags LAD_FLAG_L2NORM_QK, LAD_FLAG_OUT_FP32.
  * alpha must keep prod(alpha) over one chunk above ~1e-30 per channel (fp32 range of 1/g).
  */
 int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, const float *alpha,
                         const float *beta, float *S, void *o, int B, int T, int H, int dk, int dv, int chunk,
                         float scale, unsigned flags, void *workspace, size_t ws_bytes, void *stream);
+/* Workspace bytes of kda_prefill_chunked's two-kernel path: B * H * min(ceil(T / 64), 128) records
+ * of 145 KiB (about 1.19 GB for one sequence of 64 heads and 8,192 tokens or more); 0 for
+ * unsupported shapes. */
 size_t kda_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk);
 
 /*

@@ -339,8 +339,11 @@ def kda_prefill_workspace_size(B: int, T: int, H: int, dk: int = 128, dv: int = 
 
 
 def kda_prefill_chunked(q, k, v, alpha, beta, S, o=None, chunk: int = 64, scale: float = 1.0,
-                        l2norm_qk: bool = False, out_fp32: bool = False, workspace=None, stream=None):
-    """KDA over T tokens in chunks: q,k,alpha [B,T,H,128], v [B,T,H,128], beta [B,T,H]; S in/out."""
+                        l2norm_qk: bool = False, out_fp32: bool = False, workspace=None, split: bool = True,
+                        stream=None):
+    """KDA over T tokens in chunks: q,k,alpha [B,T,H,128], v [B,T,H,128], beta [B,T,H]; S in/out.
+    split=True runs the two-kernel path with a workspace (allocated here unless given); split=False
+    passes no workspace, which selects the single-kernel path."""
     bf = torch.bfloat16
     _contig(q, "q", bf), _contig(k, "k", bf), _contig(v, "v", bf)
     _contig(alpha, "alpha", torch.float32), _contig(beta, "beta", torch.float32), _contig(S, "S", torch.float32)
@@ -354,7 +357,9 @@ def kda_prefill_chunked(q, k, v, alpha, beta, S, o=None, chunk: int = 64, scale:
         o = torch.empty((B, T, H, dv), device=q.device, dtype=odt)
     _contig(o, "o", odt)
     ws = kda_prefill_workspace_size(B, T, H, dk, dv, chunk)
-    if workspace is None and ws > 0:
+    if not split:
+        workspace = None
+    elif workspace is None and ws > 0:
         workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
     flags = (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
     _check("kda_prefill_chunked", _L().kda_prefill_chunked(

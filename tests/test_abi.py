@@ -112,3 +112,15 @@ def test_host_side_validation_of_the_fp8_calls(lib):
     assert lib.mla_cache_append_fp8(*bad) == -1 and b"multiple of 16" in lib.lad_last_error()
     bad = list(a); bad[10] = 0
     assert lib.mla_cache_append_fp8(*bad) == 0
+
+
+def test_prefill_workspace_size(lib):
+    """The two-kernel prefill path's workspace: one 145 KiB record per (sequence, head, chunk) of a
+    segment of at most 128 chunks; zero for shapes the call does not support."""
+    rec = 145 * 1024
+    assert lib.kda_prefill_workspace_size(1, 32768, 64, 128, 128, 64) == 64 * 128 * rec
+    assert lib.kda_prefill_workspace_size(2, 100, 3, 128, 128, 64) == 2 * 3 * 2 * rec
+    assert lib.kda_prefill_workspace_size(1, 1, 1, 128, 128, 64) == rec
+    assert lib.kda_prefill_workspace_size(1, 0, 64, 128, 128, 64) == 0
+    assert lib.kda_prefill_workspace_size(1, 64, 64, 64, 128, 64) == 0
+    assert lib.kda_prefill_workspace_size(1, 64, 64, 128, 128, 32) == 0

@@ -4,6 +4,8 @@ token-by-token recurrence.
 Outputs are held to the 2e-3 relative-L2 output budget (they come out near 3e-4: tf32 operands).
 The final state is held to 2e-3 as well: its chunk updates are tf32 contractions, so the 1e-4
 figure of the fp32 decode path does not apply (see the kernel header).
+Both paths are checked: the two-kernel path (a workspace: every chunk's operands in parallel, then
+the state chain, segment by segment) and the single-kernel path (no workspace).
 """
 import numpy as np
 import pytest
@@ -33,44 +35,47 @@ def _oracle(inp, scale=1.0, l2=False, heads=None):
     return oracle.kda_recurrent(q, k, v, a, b, S0, scale=scale, nthreads=oracle.max_threads())
 
 
-def _run(lad, inp, dev, scale=1.0, l2=False, out_fp32=True):
+def _run(lad, inp, dev, scale=1.0, l2=False, out_fp32=True, split=True):
     t = {n: inp[n].to(dev) for n in ("q", "k", "v", "alpha", "beta")}
     S = inp["S0"].to(dev).clone()
     o = lad.kda_prefill_chunked(t["q"], t["k"], t["v"], t["alpha"], t["beta"], S, scale=scale, l2norm_qk=l2,
-                                out_fp32=out_fp32)
+                                out_fp32=out_fp32, split=split)
     assert lad.lad_device_error() == 0
     return o, S
 
 
+@pytest.mark.parametrize("split", [True, False])
 @pytest.mark.parametrize("B,H,T", [(1, 2, 64), (2, 3, 200), (1, 1, 1), (1, 2, 63), (1, 2, 65), (1, 4, 256)])
-def test_prefill_shapes(lad, cuda_device, B, H, T):
+def test_prefill_shapes(lad, cuda_device, B, H, T, split):
     """One chunk, several chunks with a ragged tail, a single token, one short of / one past a chunk."""
     cfg = wl.KdaScan("p", B=B, H=H, T=T, seed=100 + T, state_std=0.02, alpha_mode="uniform")
     inp = wl.kda_scan_inputs(cfg)
     o_ref, S_ref = _oracle(inp, scale=0.7)
-    o, S = _run(lad, inp, cuda_device, scale=0.7)
+    o, S = _run(lad, inp, cuda_device, scale=0.7, split=split)
     assert rel_l2(o, o_ref) < TOL_OUT
     assert rel_l2(S, S_ref) < TOL_PREFILL_STATE
 
 
-def test_prefill_clamped_decays_zero_state(lad, cuda_device):
+@pytest.mark.parametrize("split", [True, False])
+def test_prefill_clamped_decays_zero_state(lad, cuda_device, split):
     """The workload recipe: alpha mostly on the 0.9 clamp, zero initial state, bf16 output too."""
     cfg = wl.KdaScan("p", B=1, H=2, T=300, seed=7)
     inp = wl.kda_scan_inputs(cfg)
     o_ref, S_ref = _oracle(inp)
-    o, S = _run(lad, inp, cuda_device)
+    o, S = _run(lad, inp, cuda_device, split=split)
     assert rel_l2(o, o_ref) < TOL_OUT and rel_l2(S, S_ref) < TOL_PREFILL_STATE
-    o16, _ = _run(lad, inp, cuda_device, out_fp32=False)
+    o16, _ = _run(lad, inp, cuda_device, out_fp32=False, split=split)
     assert rel_l2(o16, bf16_round(o_ref)) < TOL_OUT
 
 
-def test_prefill_l2norm_flag(lad, cuda_device):
+@pytest.mark.parametrize("split", [True, False])
+def test_prefill_l2norm_flag(lad, cuda_device, split):
     cfg = wl.KdaScan("p", B=1, H=2, T=130, seed=9, state_std=0.02, alpha_mode="uniform")
     inp = wl.kda_scan_inputs(cfg)
     inp["q"] = wl.normal_bf16(inp["q"].shape, 9, "qraw", std=2.0)
     inp["k"] = wl.normal_bf16(inp["k"].shape, 9, "kraw", std=0.3)
     o_ref, S_ref = _oracle(inp, l2=True)
-    o, S = _run(lad, inp, cuda_device, l2=True)
+    o, S = _run(lad, inp, cuda_device, l2=True, split=split)
     assert rel_l2(o, o_ref) < TOL_OUT and rel_l2(S, S_ref) < TOL_PREFILL_STATE
 
 
@@ -87,6 +92,18 @@ def test_prefill_matches_decode_steps(lad, cuda_device):
     torch.cuda.synchronize()
     assert rel_l2(o_p, torch.stack(outs, 1)) < TOL_OUT
     assert rel_l2(S_p, S) < TOL_PREFILL_STATE
+
+
+def test_prefill_several_segments(lad, cuda_device):
+    """The two-kernel path works through 128-chunk segments, the state passing between them in HBM:
+    8,292 tokens are three segments (the last one ragged); agrees with the single-kernel path too."""
+    cfg = wl.KdaScan("p", B=1, H=2, T=2 * 128 * 64 + 100, seed=13, state_std=0.02, alpha_mode="uniform")
+    inp = wl.kda_scan_inputs(cfg)
+    o_ref, S_ref = _oracle(inp)
+    o, S = _run(lad, inp, cuda_device)
+    assert rel_l2(o, o_ref) < TOL_OUT and rel_l2(S, S_ref) < TOL_PREFILL_STATE
+    o1, S1 = _run(lad, inp, cuda_device, split=False)
+    assert rel_l2(o, o1) < TOL_OUT and rel_l2(S, S1) < TOL_PREFILL_STATE
 
 
 def test_prefill_empty_sequence_keeps_state(lad, cuda_device):
