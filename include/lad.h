@@ -212,11 +212,11 @@ int kda_conv_decode_step(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 
  *   S            fp32 [B][H][dk][dv]  initial state in, final state out
  *   o            [B][T][H][dv] bf16, or fp32 if flags & LAD_FLAG_OUT_FP32
  *   workspace    NULL, or device scratch of ws_bytes >= kda_prefill_workspace_size(...),
- *                1 KiB aligned: with it the call runs two kernels per segment of up to 128
- *                chunks (every chunk's state-independent operands in parallel, written to the
- *                workspace as one 145 KiB record per (sequence, head, chunk); then the state
- *                chain alone); without it, one kernel that does both per chunk. Same results
- *                within rounding.
+ *                16-byte aligned (else LAD_EWORKSPACE): with it the call runs two kernels per
+ *                segment of up to 128 chunks (every chunk's state-independent operands in
+ *                parallel, written to the workspace as one 145 KiB record per (sequence, head,
+ *                chunk); then the state chain alone); without it, one kernel that does both per
+ *                chunk. Same results within rounding.
  * Supported: dk == dv == 128, chunk == 64; flags LAD_FLAG_L2NORM_QK, LAD_FLAG_OUT_FP32.
  * alpha must keep prod(alpha) over one chunk above ~1e-30 per channel (fp32 range of 1/g).
  */

@@ -1247,7 +1247,10 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
     const long long ctas = 2LL * B * H;
     if (ctas > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "kda_prefill_chunked: B*H too large");
     const size_t ws_need = kda_prefill_workspace_size(B, T, H, dk, dv, chunk);
-    const bool split = workspace != nullptr && ws_bytes >= ws_need && lad::aligned(workspace, 1024);
+    const bool split = workspace != nullptr;
+    if (split && (ws_bytes < ws_need || !lad::aligned(workspace, 16)))
+        return set_error(LAD_EWORKSPACE, "kda_prefill_chunked: workspace of %zu bytes (16-byte aligned) required, or NULL",
+                         ws_need);
     if (split && static_cast<long long>(B) * H * kSegChunks > 0x7fffffffLL)
         return set_error(LAD_EUNSUPPORTED, "kda_prefill_chunked: B*H too large");
     static std::once_flag attr_once;

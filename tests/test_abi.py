@@ -124,3 +124,12 @@ def test_prefill_workspace_size(lib):
     assert lib.kda_prefill_workspace_size(1, 0, 64, 128, 128, 64) == 0
     assert lib.kda_prefill_workspace_size(1, 64, 64, 64, 128, 64) == 0
     assert lib.kda_prefill_workspace_size(1, 64, 64, 128, 128, 32) == 0
+
+
+def test_prefill_workspace_given_too_small(lib):
+    """A workspace that is given must hold kda_prefill_workspace_size bytes (NULL selects the
+    single-kernel path instead); the check comes before any CUDA call."""
+    rc = lib.kda_prefill_chunked(16, 16, 16, 16, 16, 16, 16, 1, 64, 1, 128, 128, 64, 1.0, 0, 16, 100, None)
+    assert rc == -4 and b"workspace" in lib.lad_last_error()
+    rc = lib.kda_prefill_chunked(16, 16, 16, 16, 16, 16, 16, 1, 64, 1, 128, 128, 64, 1.0, 0, 24, 1 << 20, None)
+    assert rc == -4  # misaligned
