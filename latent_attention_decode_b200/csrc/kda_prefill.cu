@@ -969,14 +969,17 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-// scan shared memory
-constexpr uint32_t kSW = 0, kSQ = 32768, kSKHT = 65536, kSP = 98304, kSU = 114688, kSG = 131072;
-constexpr uint32_t kSSOT = 135168;   // S0^T [64 d_v][128 d_k], stride 8 KiB
-constexpr uint32_t kSUT = 167936;    // U^T [64 d_v][64 tok], stride 8 KiB
-constexpr uint32_t kSMisc = 184320;  // beta unused; bars, tmem slot, abort flag
+// scan shared memory: W and Qt (single buffer), then two buffers of Kh^T, P and g_last (the
+// second batch's operands arrive a whole chunk ahead), S0^T, U^T; U' goes straight to registers
+constexpr uint32_t kSW = 0, kSQ = 32768;
+constexpr uint32_t kSKP0 = 65536, kSKPBytes = 50176;  // a buffer: Kh^T 32 KiB, P 16 KiB, g_last 512 B (+pad)
+constexpr uint32_t kSKHT = 0, kSP = 32768, kSG = 49152;  // offsets inside a buffer
+constexpr uint32_t kSSOT = kSKP0 + 2 * kSKPBytes;   // 165,888: S0^T [64 d_v][128 d_k], stride 8 KiB
+constexpr uint32_t kSUT = kSSOT + 32768;            // U^T [64 d_v][64 tok], stride 8 KiB
+constexpr uint32_t kSMisc = kSUT + 16384;           // bars, tmem slot, abort flag
 constexpr uint32_t kSSmemBytes = kSMisc + 2048 + 1024;
-constexpr uint32_t kSBar1Tx = 65536;           // W, Qt
-constexpr uint32_t kSBar2Tx = 32768 + 16384 + 16384 + 512;  // Kh^T, P, U' half, g_last
+constexpr uint32_t kSBar1Tx = 65536;                // W, Qt
+constexpr uint32_t kSBar2Tx = 32768 + 16384 + 512;  // Kh^T, P, g_last
 constexpr uint32_t kSColX = 0, kSColO = 64, kSColS = 128;
 constexpr uint32_t kSTmemCols = 256;
 
@@ -992,9 +995,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_scan_kernel(SplitArgs
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
     const uint32_t bar = sbase + kSMisc;
-    const uint32_t bar1 = sbase + kSMisc + 8, bar2 = sbase + kSMisc + 16;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kSMisc + 24);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kSMisc + 28);
+    const uint32_t bar1 = sbase + kSMisc + 8;
+    auto bar2 = [&](int j) { return sbase + kSMisc + 16 + 8u * static_cast<uint32_t>(j); };  // per buffer
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kSMisc + 32);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kSMisc + 36);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int sp = warp & 3, cg = warp >> 2;
@@ -1010,7 +1014,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_scan_kernel(SplitArgs
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(bar1, 1);
-        mbar_init(bar2, 1);
+        mbar_init(bar2(0), 1);
+        mbar_init(bar2(1), 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -1019,7 +1024,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_scan_kernel(SplitArgs
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    uint32_t phase = 0, ph1 = 0, ph2 = 0;
+    uint32_t phase = 0, ph1 = 0, ph2[2] = {0, 0};
     bool ok = true;
 
     auto mma_sync = [&](auto &&issue) {
@@ -1043,21 +1048,23 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_scan_kernel(SplitArgs
         bulk_g2s(sbase + kSW, rec + kItW, 32768, bar1);
         bulk_g2s(sbase + kSQ, rec + kItQ, 32768, bar1);
     };
-    auto load2 = [&](int i) {  // Kh^T, P, this CTA's half of U', g_last
+    auto load2 = [&](int i) {  // Kh^T, P, g_last of chunk i into buffer i % 2
         const uint8_t *rec = recs + static_cast<size_t>(i) * kItemBytes;
+        const uint32_t buf = sbase + kSKP0 + (i & 1) * kSKPBytes;
         fence_async_smem();
-        mbar_arrive_tx_raw(bar2, kSBar2Tx);
-        bulk_g2s(sbase + kSKHT, rec + kItKHT, 32768, bar2);
-        bulk_g2s(sbase + kSP, rec + kItP, 16384, bar2);
-        bulk_g2s(sbase + kSU, rec + kItU + half * 16384, 16384, bar2);
-        bulk_g2s(sbase + kSG, rec + kItG, 512, bar2);
+        mbar_arrive_tx_raw(bar2(i & 1), kSBar2Tx);
+        bulk_g2s(buf + kSKHT, rec + kItKHT, 32768, bar2(i & 1));
+        bulk_g2s(buf + kSP, rec + kItP, 16384, bar2(i & 1));
+        bulk_g2s(buf + kSG, rec + kItG, 512, bar2(i & 1));
     };
-    int pend1 = 0, pend2 = 0;
+    int pend1 = 0, pend2[2] = {0, 0};
     if (tid == 0) {
         load1(0);
         load2(0);
+        if (p.nseg > 1) load2(1);
     }
-    pend1 = pend2 = 1;
+    pend1 = pend2[0] = 1;
+    pend2[1] = p.nseg > 1 ? 1 : 0;
 
     // ---- the state entering the segment: TMEM master (row = key channel) and the S0^T operand ----
     {
@@ -1083,6 +1090,17 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_scan_kernel(SplitArgs
         const int n = min(kC, p.T - t0);
         const size_t tok0 = (static_cast<size_t>(b) * p.T + t0) * p.H + h;
         const size_t tstride = static_cast<size_t>(p.H);
+        // this chunk's U' (rows of this thread, 32 of this CTA's d_v columns) straight into registers
+        float4 up[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) up[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane < 16) {  // rows 0-63 of the M = 64 accumulator sit in lanes 0-15
+            const float4 *src = reinterpret_cast<const float4 *>(recs + static_cast<size_t>(i) * kItemBytes + kItU +
+                                                                 half * 16384) +
+                                (row64 * 64 + 32 * cg) / 4;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) up[j] = src[j];
+        }
         {
             const bool w = wait_bar(bar1, ph1, abort_flag, &g_prefill_error, lad::kErrPrefill);
             ph1 ^= 1;
@@ -1104,23 +1122,29 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_scan_kernel(SplitArgs
             if (tid == 0) load1(i + 1);
             pend1 = 1;
         }
+        const int kb = i & 1;
+        const uint32_t kp = kSKP0 + static_cast<uint32_t>(kb) * kSKPBytes;
         {
-            const bool w = wait_bar(bar2, ph2, abort_flag, &g_prefill_error, lad::kErrPrefill);
-            ph2 ^= 1;
-            pend2 = 0;
+            const bool w = wait_bar(bar2(kb), ph2[kb], abort_flag, &g_prefill_error, lad::kErrPrefill);
+            ph2[kb] ^= 1;
+            pend2[kb] = 0;
             ok = __syncthreads_and(w) != 0;
             if (!ok) break;
         }
-        const float gc = reinterpret_cast<const float *>(sm + kSG)[row128];
+        const float gc = reinterpret_cast<const float *>(sm + kp + kSG)[row128];
         // ---- U = U' - X -> U^T operand ----
         {
             float x[32];
             tmem_ld32(tmem + lane_base + kSColX + 32 * cg, x);
             tmem_wait_ld();
             if (lane < 16) {
-                const float *up = reinterpret_cast<const float *>(sm + kSU) + row64 * 64 + 32 * cg;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) st_tile1(sm + kSUT, 32 * cg + j, row64, kStr8, up[j] - x[j]);
+                for (int j = 0; j < 8; ++j) {
+                    st_tile1(sm + kSUT, 32 * cg + 4 * j, row64, kStr8, up[j].x - x[4 * j]);
+                    st_tile1(sm + kSUT, 32 * cg + 4 * j + 1, row64, kStr8, up[j].y - x[4 * j + 1]);
+                    st_tile1(sm + kSUT, 32 * cg + 4 * j + 2, row64, kStr8, up[j].z - x[4 * j + 2]);
+                    st_tile1(sm + kSUT, 32 * cg + 4 * j + 3, row64, kStr8, up[j].w - x[4 * j + 3]);
+                }
             }
         }
         // ---- O += P U;  S += Kh^T U ----
@@ -1128,14 +1152,14 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_scan_kernel(SplitArgs
 #pragma unroll
             for (int j = 0; j < kC / 8; ++j) {
                 const uint64_t ut = kdesc(d0 + (kSUT >> 4), kStr8, j);
-                tc_mma_tf32(tmem + kSColO, kdesc(d0 + (kSP >> 4), kStr8, j), ut, kIdesc64, 1);
-                tc_mma_tf32(tmem + kSColS, kdesc(d0 + (kSKHT >> 4), kStr16, j), ut, kIdesc128, 1);
+                tc_mma_tf32(tmem + kSColO, kdesc(d0 + ((kp + kSP) >> 4), kStr8, j), ut, kIdesc64, 1);
+                tc_mma_tf32(tmem + kSColS, kdesc(d0 + ((kp + kSKHT) >> 4), kStr16, j), ut, kIdesc128, 1);
             }
         });
         if (!ok) break;
-        if (i + 1 < p.nseg) {
-            if (tid == 0) load2(i + 1);
-            pend2 = 1;
+        if (i + 2 < p.nseg) {  // this buffer is free again: chunk i + 2's operands
+            if (tid == 0) load2(i + 2);
+            pend2[kb] = 1;
         }
         // ---- O -> HBM; S <- Diag(g_last) S, S^T -> operand (HBM after the segment's last chunk) ----
         {
@@ -1185,8 +1209,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_scan_kernel(SplitArgs
         const uint64_t t0 = lad::dev::globaltimer_ns();
         while (pend1 && !mbar_try_wait(bar1, ph1) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
         }
-        while (pend2 && !mbar_try_wait(bar2, ph2) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
-        }
+        for (int j = 0; j < 2; ++j)
+            while (pend2[j] && !mbar_try_wait(bar2(j), ph2[j]) &&
+                   lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+            }
     }
     if (warp == 0) {
         tc_commit(bar);
