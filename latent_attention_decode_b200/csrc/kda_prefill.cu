@@ -851,7 +851,18 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
                          bf16_to_f32(sv[(r0 + r + 1) * kDv + j]), bf16_to_f32(sv[(r0 + r + 2) * kDv + j]),
                          bf16_to_f32(sv[(r0 + r + 3) * kDv + j]));
         }
+        // ---- MMA 1: [Qt; Kt] Kh^T, issued now; the transposes below only read its operands ----
+        fence_async_smem();
+        tc_fence_before();
         __syncthreads();  // the staging area is read: Kh^T and Kt^T go over it
+        if (warp == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < kDk / 8; ++j)
+                tc_mma_tf32(tmem + kPColAcc1, kdesc(d0 + (kPXQK >> 4), kStr16, j), kdesc(d0 + (kPKH >> 4), kStr8, j),
+                            kIdesc128, j > 0);
+            tc_commit(bar);
+        }
         {
             // Kh^T from Kh, Kt^T from the Kt rows of [Qt; Kt]: thread -> channel i, tokens of half th
             const int i = tid & (kDk - 1), th = tid >> 7;
@@ -867,15 +878,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
                 st_tile4(sm + kPKTT, i, r, kStr16, kt[0], kt[1], kt[2], kt[3]);
             }
         }
-
-        // ---- MMA 1: [Qt; Kt] Kh^T ----
-        ok = mma_sync([&] {
-#pragma unroll
-            for (int j = 0; j < kDk / 8; ++j)
-                tc_mma_tf32(tmem + kPColAcc1, kdesc(d0 + (kPXQK >> 4), kStr16, j), kdesc(d0 + (kPKH >> 4), kStr8, j),
-                            kIdesc128, j > 0);
-        });
-        if (!ok) break;
+        {
+            const bool w = wait_bar(bar, phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            phase ^= 1;
+            tc_fence_after();
+            ok = __syncthreads_and(w) != 0;
+            if (!ok) break;
+        }
         // Kh^T, Qt and g_last are final: out to the record
         copy_out(rec + kItKHT, sm + kPKHT, 32768, tid);
 #pragma unroll
