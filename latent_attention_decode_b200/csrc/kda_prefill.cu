@@ -658,10 +658,20 @@ struct SplitArgs {
     int l2norm, out_f32;
 };
 
-__device__ __forceinline__ void copy_out(uint8_t *dst, const uint8_t *src, uint32_t bytes, int tid) {
-    for (uint32_t i = 16u * tid; i < bytes; i += 16u * kThreads)
-        *reinterpret_cast<uint4 *>(dst + i) = *reinterpret_cast<const uint4 *>(src + i);
+// Bulk copy shared -> global by one thread, in the thread's current bulk group; both addresses
+// 16-byte aligned, bytes a multiple of 16. The shared source must not change until
+// bulk_wait_read has seen the group through.
+__device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+                 "r"(src), "r"(bytes)
+                 : "memory");
 }
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {  // all but the newest N groups have read their source
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // One CTA per SM walks the segment's (sequence, head, chunk) items; the next item's raw inputs are
 // staged (alpha once Kh^T has been written out, q, k, v once the second MMA batch is complete).
@@ -760,6 +770,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
         uint8_t *rec = p.ws + static_cast<size_t>(item) * kItemBytes;
 
         if (tid < kC) s_beta[tid] = (tid < n) ? p.beta[tok0 + tid * tstride] : 0.f;
+        if (tid == 0) bulk_wait_read<0>();  // the previous item's W and U' have left [Qt; Kt]
         {
             const bool w = wait_bar(tma_bar, tma_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
             tma_phase ^= 1;
@@ -878,6 +889,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
                 st_tile4(sm + kPKTT, i, r, kStr16, kt[0], kt[1], kt[2], kt[3]);
             }
         }
+        fence_async_smem();  // the transposes are read by the bulk store below
         {
             const bool w = wait_bar(bar, phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
             phase ^= 1;
@@ -885,11 +897,14 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
             ok = __syncthreads_and(w) != 0;
             if (!ok) break;
         }
-        // Kh^T, Qt and g_last are final: out to the record
-        copy_out(rec + kItKHT, sm + kPKHT, 32768, tid);
+        // Kh^T, Qt and g_last are final: out to the record by bulk stores (group 1)
+        if (tid == 0) {
+            bulk_s2g(rec + kItKHT, sbase + kPKHT, 32768);
 #pragma unroll
-        for (int blk = 0; blk < 4; ++blk) copy_out(rec + kItQ + blk * 8192, sm + kPXQK + blk * kStr16, 8192, tid);
-        if (tid < 32) reinterpret_cast<float4 *>(rec + kItG)[tid] = reinterpret_cast<const float4 *>(s_gc)[tid];
+            for (int blk = 0; blk < 4; ++blk) bulk_s2g(rec + kItQ + blk * 8192, sbase + kPXQK + blk * kStr16, 8192);
+            bulk_s2g(rec + kItG, smem_u32(s_gc), 512);
+            bulk_commit();
+        }
         // ---- lower(Qt Kh^T) -> P tile (rows 0-63); A = strict_lower(diag(beta) Kt Kh^T) -> scratch ----
         {
             float x[32];
@@ -912,13 +927,18 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
                                              c0 + j + 2 < r ? br * x[j + 2] : 0.f, c0 + j + 3 < r ? br * x[j + 3] : 0.f);
             }
         }
-        __syncthreads();  // Kh^T copied out: the next item's alpha can come in over it
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_s2g(rec + kItP, sbase + kPP, 16384);  // group 2
+            bulk_commit();
+            bulk_wait_read<1>();  // group 1 has read Kh^T: the next item's alpha can come in over it
+        }
         if (next < nitems) {
             if (tid == 0) stage_alpha(next);
             pending = 1;
             qkv_owed = next;
         }
-        copy_out(rec + kItP, sm + kPP, 16384, tid);
         // ---- T = (I + A)^-1, Tb -> operand ----
         solve_tb(Apl, Tpl, s_beta, sm + kPTT, tid);
         // ---- MMA 2: W = Tb Kt (B = Kt^T), U' = Tb V (B = V^T) ----
@@ -931,12 +951,16 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
             }
         });
         if (!ok) break;
+        if (tid == 0) bulk_wait_read<0>();  // P (and Qt) read out: the staging area and XQK are free
         if (qkv_owed >= 0) {  // Kt^T and P are done with: q, k, v of the next item
             if (tid == 0) stage_qkv(qkv_owed);
             qkv_owed = -1;
         }
-        // ---- W (tf32-rounded operand layout) and U' (plain fp32, per d_v half) -> record ----
+        __syncthreads();
+        // ---- W (tf32-rounded operand layout) and U' (plain fp32, per d_v half) -> shared memory over
+        //      [Qt; Kt], then -> record by one bulk store (group 3) ----
         {
+            float *ush = reinterpret_cast<float *>(sm + kPXQK + 32768);  // U' [2 halves][64 tok][64]
 #pragma unroll 1
             for (int part = 0; part < 2; ++part) {
                 const int c0 = 32 * cg + 64 * part;  // columns c0 .. c0 + 31
@@ -947,18 +971,22 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
                 if (lane < 16) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
-                        *reinterpret_cast<float4 *>(rec + kItW + sw128_off32(row64, c0 + j, 8192)) =
-                            make_float4(round_tf32(w[j]), round_tf32(w[j + 1]), round_tf32(w[j + 2]),
-                                        round_tf32(w[j + 3]));
+                        st_tile4(sm + kPXQK, row64, c0 + j, kStr8, w[j], w[j + 1], w[j + 2], w[j + 3]);
                         const int hv = c0 >> 6, cc = (c0 & 63) + j;
-                        *reinterpret_cast<float4 *>(rec + kItU + ((hv * 64 + row64) * 64 + cc) * 4) =
+                        *reinterpret_cast<float4 *>(ush + (hv * 64 + row64) * 64 + cc) =
                             make_float4(u[j], u[j + 1], u[j + 2], u[j + 3]);
                     }
                 }
             }
         }
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        if (tid == 0) {
+            bulk_s2g(rec + kItW, sbase + kPXQK, 32768);
+            bulk_s2g(rec + kItU, sbase + kPXQK + 32768, 32768);
+            bulk_commit();
+        }
     }
     if (tid == 0 && qkv_owed >= 0) stage_qkv(qkv_owed);
     if (tid == 0 && pending) {
@@ -966,6 +994,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
         while (!mbar_try_wait(tma_bar, tma_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
         }
     }
+    if (tid == 0) bulk_wait_all();  // every record write has landed
     if (warp == 0) {
         tc_commit(bar);
         const uint64_t t0 = lad::dev::globaltimer_ns();
