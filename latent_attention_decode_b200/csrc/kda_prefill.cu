@@ -16,7 +16,12 @@
 // d_v columns of S are independent, so a CTA owns one (sequence, head, half of d_v) and walks
 // its chunks in order: 128 CTAs for one sequence of 64 heads.
 //
-// Per chunk (two warpgroups; warp 0 issues the MMAs, converged, elect.sync):
+// Two paths. With a workspace, two kernels per segment of up to 128 chunks: the prep kernel
+// computes every chunk's state-independent operands (W, Tb V, Qt, Kh^T, lower(Qt Kh^T), g_last)
+// in parallel into a record per chunk, and the scan kernel runs only the state chain, two MMA
+// batches per chunk (see "Split path" below). Without one, the single kernel does both, per chunk:
+//
+// Single kernel, per chunk (two warpgroups; warp 0 issues the MMAs, converged, elect.sync):
 //   1. load q, k, alpha, v, beta; running products g; write the operand tiles
 //   2. MMA  [Qt; Kt] Kh^T  (M = 128: rows 0-63 give Qt Kh^T, rows 64-127 give Kt Kh^T), and
 //           Y = Kt S0 (it needs no T: W S0 = Tb (Kt S0), so W itself is never formed); then
