@@ -39,7 +39,7 @@ typedef uint16_t lad_bf16; /* IEEE bfloat16 bit pattern */
 /* status codes */
 #define LAD_OK 0
 #define LAD_EINVAL (-1)        /* null pointer, negative or inconsistent size */
-#define LAD_EUNSUPPORTED (-2)  /* a size or alignment this build does not implement */
+#define LAD_EUNSUPPORTED (-2)  /* a size or alignment the library does not implement */
 #define LAD_ECUDA (-3)         /* a CUDA runtime error (launch, attribute, device query) */
 #define LAD_EWORKSPACE (-4)    /* workspace missing or smaller than the query returned */
 
