@@ -702,7 +702,8 @@ class PrefillStep(Step):
         self.h_in = [t.cpu().pin_memory() for t in (self.q, self.k, self.v, self.alpha, self.beta)]
         self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
         self.tokens_per_step = cfg.B * cfg.T
-        self.launches_per_step = 1
+        # the two-kernel path (a workspace is given): prep + scan per segment of up to 128 chunks
+        self.launches_per_step = 2 * math.ceil(math.ceil(cfg.T / cfg.chunk) / 128)
         self.dominant = "kda_prefill_chunked"
         self.config = {"workload": self.name, "batch_per_gpu": cfg.B, "seq_len": cfg.T, "heads": cfg.H,
                        "chunk": cfg.chunk, "l2": f"inputs larger than L2 ({self.algorithmic_bytes()['step'] / 1e9:.2f} GB per step)"}
@@ -738,8 +739,9 @@ class PrefillStep(Step):
         c = self.cfg
         chunks = c.B * c.H * math.ceil(c.T / c.chunk)
         C = c.chunk
-        # multiply-adds per chunk-head: [Qt; Kt] Kh^T (2 C C D), W^T = Kt^T Tb^T (C C D), U' = Tb V (C C D),
+        # multiply-adds per chunk-head: [Qt; Kt] Kh^T (2 C C D), W = Tb Kt (C C D), U' = Tb V (C C D),
         # X = W S0 (C D D), O = Qt S0 (C D D) + lower(Qt Kh^T) U (C C D), S += Kh^T U (D D C)
+        # (the single kernel forms Tb (Kt S0) instead of (Tb Kt) S0: the same count)
         per_chunk = 2 * (2 * C * C * D + C * C * D + C * C * D + C * D * D + C * D * D + C * C * D + D * D * C)
         return chunks * per_chunk
 
