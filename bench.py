@@ -11,6 +11,7 @@ A step is one pass of the workload's hot path over one batch of synthetic input:
   mla_decode_b16              one gated MLA layer, 16 sequences, contexts uniform in [8192, 131072]
   mla_decode_b16_paged        the same layer with the cache in 64-row pages of a shuffled pool
   mla_decode_b16_paged_rope   the paged layer with RoPE in the kernels: append the new rows, then attend
+  mla_mtp_b16                 mla_decode_b16 with 4 query tokens per sequence (mla_latent_decode_multi)
   mla_decode_b16_fp8          mla_decode_b16 over an FP8 (E4M3) cache, one fp32 scale (mla_latent_decode_fp8)
   mla_decode_b16_paged_rope_fp8  the engine step of mla_decode_b16_paged_rope over FP8 pages
   kda_decode_b64_gated        the same layer with the output gate fused (kda_conv_decode_step_gated)
@@ -546,6 +547,49 @@ class MlaPagedRopeStep(MlaPagedStep):
         return {"mla_latent_decode_paged_rope": b, "step": b + append}
 
 
+class MlaMultiStep(MlaDecodeStep):
+    """The 16-sequence latent-attention workload as a multi-token verify step: 4 query tokens per
+    sequence (a token and 3 drafts, the pages' MTP setting), token j attending the first
+    len - 3 + j rows, through mla_latent_decode_multi. Algorithmic bytes count the cache once."""
+    name = "mla_mtp_b16"
+    T = 4
+
+    def __init__(self, lad, dev, rank, cfg: wl.MlaDecode | None = None):
+        super().__init__(lad, dev, rank, cfg)
+        B, H, T, s = self.cfg.B, self.cfg.Hq, self.T, self.cfg.seed
+        self.q = wl.normal_bf16((B, T, H, wl.D_ROW), s, "mla_q_mtp", dev)
+        self.gate = wl.normal((B, T, H), s, "mla_gate_mtp", dev)
+        self.o = torch.empty((B, T, H, wl.D_LATENT), device=dev, dtype=torch.bfloat16)
+        self.ws = torch.empty(lad.mla_latent_decode_multi_workspace_size(B, T, H, wl.D_LATENT, 0), device=dev,
+                              dtype=torch.uint8)
+        self.h_q = self.q.cpu().pin_memory()
+        self.h_gate = self.gate.cpu().pin_memory()
+        self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.tokens_per_step = B * T
+        self.launches_per_step = 3
+        self.dominant = "mla_latent_decode_multi"
+        self.config = dict(self.config, workload=self.name, query_tokens_per_sequence=T,
+                           causal="token j attends rows 0 .. len - T + j")
+
+    def run(self, timer=None):
+        if timer:
+            timer.begin("mla_latent_decode_multi")
+        self.lad.mla_latent_decode_multi(self.q, self.cache, self.lens, self.gate, o=self.o, workspace=self.ws)
+        if timer:
+            timer.end("mla_latent_decode_multi")
+
+    def mla_bytes(self):
+        B, H, T = self.cfg.B, self.cfg.Hq, self.T
+        return self.total_len * wl.D_ROW * 2 + B * T * H * (wl.D_ROW * 2 + 4 + wl.D_LATENT * 2) + B * 4
+
+    def mla_flops(self):
+        return self.T * super().mla_flops()
+
+    def algorithmic_bytes(self):
+        b = self.mla_bytes()
+        return {"mla_latent_decode_multi": b, "step": b}
+
+
 class MlaFp8Step(MlaDecodeStep):
     """The 16-sequence latent-attention workload over an FP8 (E4M3) cache with one fp32 scale,
     through mla_latent_decode_fp8; the cache holds half the bytes of the bf16 one."""
@@ -754,6 +798,7 @@ WORKLOADS = {
     "mla_decode_b16": MlaDecodeStep,
     "mla_decode_b16_paged": MlaPagedStep,
     "mla_decode_b16_paged_rope": MlaPagedRopeStep,
+    "mla_mtp_b16": MlaMultiStep,
     "mla_decode_b16_fp8": MlaFp8Step,
     "mla_decode_b16_paged_rope_fp8": MlaPagedRopeFp8Step,
     "kda_prefill_32k": PrefillStep,
@@ -848,9 +893,12 @@ def cpu_oracle_rate(workload: str, budget_s: float = 20.0) -> dict:
         return {"value": 256 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle",
                 "sample": f"{Bs} of 64 sequences x 64 heads x 4 tokens, scaled to 64 sequences"}
     if workload in ("mla_decode_b16", "mla_decode_b16_paged", "mla_decode_b16_paged_rope", "mla_decode_b16_fp8",
-                    "mla_decode_b16_paged_rope_fp8"):
+                    "mla_decode_b16_paged_rope_fp8", "mla_mtp_b16"):
         lens = wl.mla_seq_lens(wl.MlaDecode("mla", B=16, seed=1236)).tolist()
         sec, sample = mla_seconds(16, lens, fp8=workload.endswith("fp8"))
+        if workload == "mla_mtp_b16":  # four query tokens per sequence: four attentions over (nearly) the rows
+            return {"value": 64 / (4 * sec), "unit": "tokens/s", "cores": nth, "kind": "oracle",
+                    "sample": sample + ", x4 query tokens"}
         return {"value": 16 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": sample}
     if workload == "hybrid_8layer_1m":
         ks, s1 = kda_layer_seconds(8)
@@ -892,7 +940,7 @@ def run_reference(args, rank, world):
 def _tokens(workload):
     return {"hybrid_8layer_1m": 8, "kda_decode_b64": 64, "kda_decode_b64_gated": 64, "kda_mtp_b64": 256, "mla_decode_b16": 16,
             "mla_decode_b16_paged": 16, "mla_decode_b16_paged_rope": 16, "mla_decode_b16_fp8": 16,
-            "mla_decode_b16_paged_rope_fp8": 16, "kda_prefill_32k": 32768}[workload]
+            "mla_decode_b16_paged_rope_fp8": 16, "mla_mtp_b16": 64, "kda_prefill_32k": 32768}[workload]
 
 
 def main(argv=None) -> int:
@@ -978,7 +1026,7 @@ def main(argv=None) -> int:
     for kname in ("kda_conv_decode_step", "kda_conv_decode_step_gated", "kda_decode_step", "kda_decode_multi",
                   "mla_latent_decode",
                   "mla_latent_decode_paged", "mla_latent_decode_paged_rope", "mla_latent_decode_fp8",
-                  "mla_latent_decode_paged_fp8", "kda_prefill_chunked"):
+                  "mla_latent_decode_paged_fp8", "mla_latent_decode_multi", "kda_prefill_chunked"):
         km = timer.mean_ms(kname)
         if km is not None and kname in ab:
             gbs = ab[kname] / (km / 1000.0) / 1e9

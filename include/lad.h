@@ -331,6 +331,25 @@ int mla_cache_append(const lad_bf16 *c_kv, const lad_bf16 *k_pe, const int *posi
                      void *stream);
 
 /*
+ * mla_latent_decode_multi — the MLA half of a multi-token step (speculative-decoding verify, [P1]
+ * "What does that mean for serving?" / [P2] "What is in the files": an MTP layer drafts 3 tokens).
+ * T query tokens per sequence: the last T of sequence b's seq_lens[b] cached rows are the tokens'
+ * own rows (appended first), and token j (0-based) attends rows 0 .. seq_lens[b] - T + j, a
+ * causal reading the pages leave open. T = 1 is mla_latent_decode.
+ *   q           bf16 [B][T][Hq][576]
+ *   gate_logits fp32 [B][T][Hq] or NULL;  o [B][T][Hq][d_latent];  lse_out fp32 [B][T][Hq] or NULL
+ *   cache, cache_seq_stride, seq_lens, Lmax, scale, flags: as for mla_latent_decode
+ *   workspace   ws_bytes >= mla_latent_decode_multi_workspace_size(B, T, Hq, d_latent, 0), 256-aligned
+ * Each token is attended as a sequence of its own over the shared rows (the cache is read once per
+ * token from HBM or L2). Tokens with no row to attend (seq_lens[b] - T + j < 0) give o = 0, lse = -inf.
+ */
+int mla_latent_decode_multi(const lad_bf16 *q, const lad_bf16 *cache, long long cache_seq_stride,
+                            const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B, int T,
+                            int Hq, int d_latent, int d_rope, int Lmax, float scale, unsigned flags, void *workspace,
+                            size_t ws_bytes, void *stream);
+size_t mla_latent_decode_multi_workspace_size(int B, int T, int Hq, int d_latent, int num_sms);
+
+/*
  * FP8 latent cache. [P1] "How big is the cache per token, exactly?": the bf16 cache takes 2 bytes
  * per element and an FP8 cache would halve it; [P2] "Does 292 GiB fit on four Hopper GPUs?": an
  * FP8 cache doubles the tokens that fit. The FP8 the pages use is E4M3 ([P2] "What is in the

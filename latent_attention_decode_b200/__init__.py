@@ -21,7 +21,8 @@ __all__ = [
     "kda_conv_update", "kda_decode_step", "kda_conv_decode_step", "kda_conv_decode_step_gated", "kda_decode_multi",
     "kda_prefill_chunked", "kda_prefill_workspace_size",
     "mla_latent_decode", "mla_latent_decode_workspace_size", "mla_latent_decode_paged",
-    "mla_latent_decode_paged_rope", "mla_cache_append", "mla_latent_decode_fp8", "mla_latent_decode_paged_fp8",
+    "mla_latent_decode_paged_rope", "mla_cache_append", "mla_latent_decode_multi",
+    "mla_latent_decode_multi_workspace_size", "mla_latent_decode_fp8", "mla_latent_decode_paged_fp8",
     "mla_cache_append_fp8", "mla_latent_decode_noalloc",
     "lad_device_error", "lad_check_bounded_wait", "lad_version",
     "LadError", "LIB_PATH", "FLAG_SILU", "FLAG_L2NORM_QK", "FLAG_OUT_FP32", "FLAG_KEEP_STATE",
@@ -88,6 +89,9 @@ def _load() -> ctypes.CDLL:
         "mla_latent_decode_noalloc": ([_c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                                        _c_int, _c_int, _c_f, _c_u, _c_vp], _c_int),
         "mla_latent_decode_noalloc_max_batch": ([], _c_sz),
+        "mla_latent_decode_multi": ([_c_vp, _c_vp, _c_ll, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int,
+                                     _c_int, _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
+        "mla_latent_decode_multi_workspace_size": ([_c_int] * 5, _c_sz),
         "mla_latent_decode_fp8": ([_c_vp, _c_vp, _c_ll, _c_f, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                                    _c_int, _c_int, _c_f, _c_u, _c_vp, _c_sz, _c_vp], _c_int),
         "mla_latent_decode_paged_fp8": ([_c_vp, _c_vp, _c_f, _c_vp, _c_f, _c_int, _c_int, _c_vp, _c_int, _c_vp,
@@ -557,6 +561,48 @@ def _mla_common(q, seq_lens, gate_logits, o, lse, d_latent, out_fp32, workspace)
         workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     return B, Hq, D, o, workspace, ws_bytes
+
+
+def mla_latent_decode_multi_workspace_size(B: int, T: int, Hq: int = 64, d_latent: int = 512, num_sms: int = 0) -> int:
+    return int(_L().mla_latent_decode_multi_workspace_size(B, T, Hq, d_latent, num_sms))
+
+
+def mla_latent_decode_multi(q: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tensor,
+                            gate_logits: torch.Tensor | None = None, o: torch.Tensor | None = None,
+                            lse: torch.Tensor | None = None, scale: float = MLA_SCALE, d_latent: int = 512,
+                            out_fp32: bool = False, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Multi-token step: q [B,T,Hq,576]; the last T of seq_lens[b] cached rows are the tokens' own, token j
+    attends rows 0 .. seq_lens[b] - T + j. Returns o [B,T,Hq,d_latent]; fills lse [B,T,Hq] when given."""
+    bf = torch.bfloat16
+    _contig(q, "q", bf)
+    _cuda(cache, "cache", bf)
+    B, T, Hq, D = q.shape
+    if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != D or cache.stride(2) != 1 \
+            or cache.stride(1) != D:
+        raise ValueError("cache must be [B,Lmax,D] with contiguous rows")
+    Lmax = cache.shape[1]
+    _contig(seq_lens, "seq_lens", torch.int32)
+    if seq_lens.shape != (B,):
+        raise ValueError("seq_lens must be [B]")
+    if gate_logits is not None:
+        _contig(gate_logits, "gate_logits", torch.float32)
+        if gate_logits.shape != (B, T, Hq):
+            raise ValueError("gate_logits must be [B,T,Hq]")
+    odt = torch.float32 if out_fp32 else bf
+    if o is None:
+        o = torch.empty((B, T, Hq, d_latent), device=q.device, dtype=odt)
+    _contig(o, "o", odt)
+    if lse is not None:
+        _contig(lse, "lse", torch.float32)
+    ws = mla_latent_decode_multi_workspace_size(B, T, Hq, d_latent, 0)
+    if workspace is None and ws > 0:
+        workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
+    seq_stride = cache.stride(0) if B > 1 else Lmax * D
+    _check("mla_latent_decode_multi", _L().mla_latent_decode_multi(
+        q.data_ptr(), cache.data_ptr(), seq_stride, seq_lens.data_ptr(), _ptr(gate_logits), o.data_ptr(), _ptr(lse),
+        B, T, Hq, d_latent, D - d_latent, Lmax, float(scale), FLAG_OUT_FP32 if out_fp32 else 0, _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o
 
 
 def mla_latent_decode_fp8(q: torch.Tensor, cache: torch.Tensor, kv_scale: float, seq_lens: torch.Tensor,

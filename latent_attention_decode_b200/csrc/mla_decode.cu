@@ -280,12 +280,14 @@ struct Fp8Cursor {
 
 // kPaged: map_cache is 2-D over the page pool ([num_pages * page_size][576]) and each tile's row
 // comes from the block table; otherwise it is 3-D ([B][Lmax][576]). kFp8: map_cache is unused and
-// the cache is read through f8.
+// the cache is read through f8. cache_group: consecutive sequences that read one cached sequence
+// (the query tokens of a multi-token step; 1 otherwise): sequence s reads cached sequence
+// s / cache_group of the contiguous map.
 template <bool kPaged, bool kRopeQ, bool kFp8>
 __global__ void __launch_bounds__(kFp8 ? kThreadsF8 : kThreads, 1)
 mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_constant__ CUtensorMap map_q,
                  const int *__restrict__ seq_lens, int B, float score_scale_log2, Partials ws, PagedCache pc,
-                 const __grid_constant__ RopeQ rq, Fp8Cache f8) {
+                 const __grid_constant__ RopeQ rq, Fp8Cache f8, int cache_group) {
     constexpr int NSt = kStages;  // depth of the operand ring
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -417,8 +419,8 @@ mla_split_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_con
                             lad::ptx::tma_load_2d_elect(dst + c * kTChunkBytes, &map_cache, c * kChunk, row,
                                                         bar(kBarFull + s));
                         else
-                            lad::ptx::tma_load_3d_elect(dst + c * kTChunkBytes, &map_cache, c * kChunk, row, seq,
-                                                        bar(kBarFull + s));
+                            lad::ptx::tma_load_3d_elect(dst + c * kTChunkBytes, &map_cache, c * kChunk, row,
+                                                        seq / cache_group, bar(kBarFull + s));
                     }
                 }
                 ++k;
@@ -1072,7 +1074,7 @@ int encode_contiguous(const char *name, CUtensorMap *map, const lad_bf16 *cache,
 int run_mla(const char *name, const CUtensorMap &map_cache, bool paged, const PagedCache &pc, const RopeQ *rope,
             const lad_bf16 *q, const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B,
             float scale, unsigned flags, uint8_t *ws, const WsLayout &wl, int G, void *stream,
-            const Fp8Cache *f8 = nullptr, float kv_scale = 1.f) {
+            const Fp8Cache *f8 = nullptr, float kv_scale = 1.f, int cache_group = 1) {
     using lad::set_error;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return set_error(LAD_ECUDA, "%s: cuTensorMapEncodeTiled unavailable", name);
@@ -1101,22 +1103,22 @@ int run_mla(const char *name, const CUtensorMap &map_cache, bool paged, const Pa
     if (f8) {
         if (rope)
             mla_split_kernel<true, true, true><<<G, kThreadsF8, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
-                                                                                 score_scale_log2, parts, pc, rq, fc);
+                                                                                 score_scale_log2, parts, pc, rq, fc, cache_group);
         else if (paged)
             mla_split_kernel<true, false, true><<<G, kThreadsF8, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
-                                                                                  score_scale_log2, parts, pc, rq, fc);
+                                                                                  score_scale_log2, parts, pc, rq, fc, cache_group);
         else
             mla_split_kernel<false, false, true><<<G, kThreadsF8, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
-                                                                                   score_scale_log2, parts, pc, rq, fc);
+                                                                                   score_scale_log2, parts, pc, rq, fc, cache_group);
     } else if (rope) {
         mla_split_kernel<true, true, false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
-                                                                            score_scale_log2, parts, pc, rq, fc);
+                                                                            score_scale_log2, parts, pc, rq, fc, cache_group);
     } else if (paged) {
         mla_split_kernel<true, false, false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
-                                                                             score_scale_log2, parts, pc, rq, fc);
+                                                                             score_scale_log2, parts, pc, rq, fc, cache_group);
     } else {
         mla_split_kernel<false, false, false><<<G, kThreads, kSmemBytes, s>>>(map_cache, map_q, seq_lens, B,
-                                                                              score_scale_log2, parts, pc, rq, fc);
+                                                                              score_scale_log2, parts, pc, rq, fc, cache_group);
     }
     rc = lad::check_launch(name);
     if (rc != LAD_OK) return rc;
@@ -1241,6 +1243,71 @@ extern "C" int mla_latent_decode_paged_rope(const lad_bf16 *q, const int *positi
     return run_paged(name, q, kv_pages, num_pages, page_size, block_table, block_table_stride, seq_lens, gate_logits,
                      o, lse_out, B, Hq, d_latent, d_rope, scale, flags, LAD_FLAG_ROPE_INTERLEAVED, &rq, workspace,
                      ws_bytes, stream);
+}
+
+// ------------------------------------------------------------------------------------------
+// Multi-token step (the T query tokens of a speculative-decoding verify): the last T of a
+// sequence's L cached rows are the T tokens' own rows, and token j attends rows 0 .. L - T + j.
+// Every token is a sequence of its own to the split kernel (cache_group = T: T consecutive
+// ones read one cached sequence), with its length written by a small kernel into the workspace.
+// ------------------------------------------------------------------------------------------
+namespace {
+__global__ void mla_multi_lens_kernel(const int *__restrict__ seq_lens, int B, int T, int *__restrict__ vlens) {
+    const int v = blockIdx.x * blockDim.x + threadIdx.x;
+    if (v < B * T) {
+        const int b = v / T, j = v - b * T;
+        const int L = seq_lens[b] - (T - 1 - j);
+        vlens[v] = L > 0 ? L : 0;
+    }
+}
+
+size_t multi_ws_bytes(int BT, int G) {
+    return ws_layout(BT, G).total + align_up(static_cast<size_t>(BT) * sizeof(int), 256);
+}
+}  // namespace
+
+extern "C" size_t mla_latent_decode_multi_workspace_size(int B, int T, int Hq, int d_latent, int num_sms) {
+    if (B < 0 || T < 1 || Hq != kHq || d_latent != kDl || static_cast<long long>(B) * T > 0x7fffffffLL) return 0;
+    const int G = num_sms > 0 ? num_sms : lad::device_sm_count();
+    if (G <= 0) return 0;
+    return multi_ws_bytes(B * T, G);
+}
+
+extern "C" int mla_latent_decode_multi(const lad_bf16 *q, const lad_bf16 *cache, long long cache_seq_stride,
+                                       const int *seq_lens, const float *gate_logits, void *o, float *lse_out, int B,
+                                       int T, int Hq, int d_latent, int d_rope, int Lmax, float scale, unsigned flags,
+                                       void *workspace, size_t ws_bytes, void *stream) {
+    using lad::set_error;
+    const char *name = "mla_latent_decode_multi";
+    int rc = check_common(name, B, Hq, d_latent, d_rope, flags, scale);
+    if (rc != LAD_OK) return rc;
+    if (T < 1) return set_error(LAD_EINVAL, "%s: T must be at least 1", name);
+    if (static_cast<long long>(B) * T > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "%s: B*T too large", name);
+    if (Lmax < 0) return set_error(LAD_EINVAL, "%s: negative Lmax", name);
+    if (B == 0) return LAD_OK;
+    rc = check_pointers(name, q, cache, seq_lens, o, flags);
+    if (rc != LAD_OK) return rc;
+    if (Lmax == 0) Lmax = 1;
+    if (cache_seq_stride < static_cast<long long>(Lmax) * kDrow || cache_seq_stride % 8 != 0)
+        return set_error(LAD_EINVAL, "%s: cache_seq_stride must be >= Lmax*576 and a multiple of 8", name);
+    int G = 0;
+    rc = sm_count_checked(name, &G);
+    if (rc != LAD_OK) return rc;
+    const int BT = B * T;
+    const WsLayout wl = ws_layout(BT, G);
+    if (!workspace || ws_bytes < multi_ws_bytes(BT, G) || !lad::aligned(workspace, 256))
+        return set_error(LAD_EWORKSPACE, "%s: workspace of %zu bytes (256-aligned) required", name,
+                         multi_ws_bytes(BT, G));
+    int *vlens = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + wl.total);
+    cudaStream_t s = lad::as_stream(stream);
+    mla_multi_lens_kernel<<<(BT + 255) / 256, 256, 0, s>>>(seq_lens, B, T, vlens);
+    rc = lad::check_launch(name);
+    if (rc != LAD_OK) return rc;
+    CUtensorMap map_cache;
+    rc = encode_contiguous(name, &map_cache, cache, B, Lmax, cache_seq_stride);
+    if (rc != LAD_OK) return rc;
+    return run_mla(name, map_cache, false, PagedCache{}, nullptr, q, vlens, gate_logits, o, lse_out, BT, scale, flags,
+                   static_cast<uint8_t *>(workspace), wl, G, stream, nullptr, 1.f, T);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -133,3 +133,18 @@ def test_prefill_workspace_given_too_small(lib):
     assert rc == -4 and b"workspace" in lib.lad_last_error()
     rc = lib.kda_prefill_chunked(16, 16, 16, 16, 16, 16, 16, 1, 64, 1, 128, 128, 64, 1.0, 0, 24, 1 << 20, None)
     assert rc == -4  # misaligned
+
+
+def test_multi_token_mla_host_checks(lib):
+    # mla_latent_decode_multi(q, cache, stride, lens, gate, o, lse, B, T, Hq, Dl, Dr, Lmax, scale, flags, ws, ws_bytes,
+    #                         stream)
+    a = [16, 16, 576 * 8, 16, None, 16, None, 1, 4, 64, 512, 64, 8, 0.1, 0, 16, 1 << 20, None]
+    bad = list(a); bad[8] = 0
+    assert lib.mla_latent_decode_multi(*bad) == -1 and b"T must be" in lib.lad_last_error()
+    bad = list(a); bad[9] = 32
+    assert lib.mla_latent_decode_multi(*bad) == -2
+    bad = list(a); bad[7] = 0
+    assert lib.mla_latent_decode_multi(*bad) == 0
+    assert lib.mla_latent_decode_multi_workspace_size(2, 4, 64, 512, 10) == \
+        lib.mla_latent_decode_workspace_size(8, 64, 512, 10) + 256
+    assert lib.mla_latent_decode_multi_workspace_size(2, 0, 64, 512, 10) == 0
