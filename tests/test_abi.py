@@ -148,3 +148,15 @@ def test_multi_token_mla_host_checks(lib):
     assert lib.mla_latent_decode_multi_workspace_size(2, 4, 64, 512, 10) == \
         lib.mla_latent_decode_workspace_size(8, 64, 512, 10) + 256
     assert lib.mla_latent_decode_multi_workspace_size(2, 0, 64, 512, 10) == 0
+
+
+def test_binding_covers_every_declared_call(lib):
+    """Every call include/lad.h declares has a Python wrapper of the same name in the binding
+    (argument marshalling only), except the error-string accessor and the no-alloc batch limit,
+    which the binding uses internally."""
+    import latent_attention_decode_b200 as lad
+    internal = {"lad_last_error", "mla_latent_decode_noalloc_max_batch"}
+    missing = [n for n in _declared() if n not in internal and not callable(getattr(lad, n, None))]
+    assert not missing, missing
+    for n in lad.__all__:
+        assert hasattr(lad, n), n
