@@ -834,105 +834,163 @@ class KernelTimer:
 # CPU oracle timing (the reference arm and the cpu_baseline key)
 # ---------------------------------------------------------------------------------------------
 
-def cpu_oracle_rate(workload: str, budget_s: float = 20.0) -> dict:
-    """Times the fp64 oracle on a bounded sample of the workload; returns tokens/s for the
-    whole workload step estimated from the sample, with the sample described."""
-    import oracle
-    nth = oracle.max_threads()
-    rng = np.random.default_rng(0)
+class OracleSample:
+    """One bounded sample of a workload step for the fp64 oracle on `nth` host threads.
 
-    def kda_layer_seconds(B):
-        # one KDA decode layer (conv + step) for B sequences, all 64 heads
-        Bs = min(B, max(1, nth))
-        x = rng.standard_normal((Bs, 3 * H * D))
-        tail = rng.standard_normal((Bs, 3, 3 * H * D))
-        w = 0.5 * rng.standard_normal((3 * H * D, 4))
-        q = rng.standard_normal((Bs, 1, H, D))
-        S = 0.02 * rng.standard_normal((Bs, H, D, D))
-        a = np.full((Bs, 1, H, D), 0.9)
-        b = np.full((Bs, 1, H), 0.5)
-        t0 = time.perf_counter()
-        y, _ = oracle.short_conv_step(x, tail, w, None, True)
-        qn = oracle.l2norm(y[:, : H * D].reshape(Bs, 1, H, D))
-        kn = oracle.l2norm(y[:, H * D: 2 * H * D].reshape(Bs, 1, H, D))
-        oracle.kda_recurrent(qn, kn, y[:, 2 * H * D:].reshape(Bs, 1, H, D), a, b, S, nthreads=nth)
-        dt = time.perf_counter() - t0
-        return dt * B / Bs, f"{Bs} of {B} sequences x 64 heads, one token"
+    The sample is a list of parts, each an oracle call over a subset of the step's units (some
+    of a layer's sequences, some heads over a context) with the factor that scales its time to
+    the whole step; the sample's size follows `nth`, so one thread runs a proportionally smaller
+    sample. run() returns the estimated seconds of one whole workload step."""
 
-    def mla_seconds(B, lens, fp8=False):
-        # units = (sequence, head); sample `nth` heads of the longest sequence over its whole context
-        L = int(max(lens))
-        units = min(nth, H)
-        qs = rng.standard_normal((1, units, wl.D_ROW))
-        if fp8:
-            codes = rng.integers(0, 0x7F, (1, L, wl.D_ROW), dtype=np.uint8)
+    def __init__(self, workload: str, nth: int):
+        import oracle
+        self.oracle, self.nth = oracle, nth
+        rng = np.random.default_rng(0)
+        self.parts: list[tuple] = []   # (callable, factor)
+        desc = []
+
+        def kda_layer(B):
+            Bs = min(B, max(1, nth))
+            x = rng.standard_normal((Bs, 3 * H * D))
+            tail = rng.standard_normal((Bs, 3, 3 * H * D))
+            w = 0.5 * rng.standard_normal((3 * H * D, 4))
+            S = 0.02 * rng.standard_normal((Bs, H, D, D))
+            a = np.full((Bs, 1, H, D), 0.9)
+            b = np.full((Bs, 1, H), 0.5)
+
+            def run():
+                y, _ = oracle.short_conv_step(x, tail, w, None, True)
+                qn = oracle.l2norm(y[:, : H * D].reshape(Bs, 1, H, D))
+                kn = oracle.l2norm(y[:, H * D: 2 * H * D].reshape(Bs, 1, H, D))
+                oracle.kda_recurrent(qn, kn, y[:, 2 * H * D:].reshape(Bs, 1, H, D), a, b, S.copy(), nthreads=nth)
+            return run, B / Bs, f"{Bs} of {B} sequences x 64 heads, one token"
+
+        def mla(lens, fp8=False):
+            # (sequence, head) units: `units` heads of the longest sequence over its whole context
+            L = int(max(lens))
+            units = min(max(1, nth), H)
+            qs = rng.standard_normal((1, units, wl.D_ROW))
+            ln = np.array([L], np.int32)
+            if fp8:
+                codes = rng.integers(0, 0x7F, (1, L, wl.D_ROW), dtype=np.uint8)
+
+                def run():
+                    oracle.mla_decode_fp8(qs, codes, wl.KV_SCALE_FP8, ln, None, nthreads=nth)
+            else:
+                cache = (rng.standard_normal((1, L, wl.D_ROW)).astype(np.float32).view(np.uint32) >> 16).astype(
+                    np.uint16)
+
+                def run():
+                    oracle.mla_decode(qs, cache, ln, None, nthreads=nth)
+            return run, H * float(sum(lens)) / (units * L), f"{units} heads x {L} cached tokens of 1 sequence"
+
+        if workload in ("kda_decode_b64", "kda_decode_b64_gated"):
+            f, k, d = kda_layer(64)
+            self.parts.append((f, k))
+            desc.append(d)
+        elif workload == "kda_mtp_b64":
+            Bs = min(64, max(1, nth))
+            q = rng.standard_normal((Bs, 4, H, D))
+            S = 0.02 * rng.standard_normal((Bs, H, D, D))
+            a = np.full((Bs, 4, H, D), 0.9)
+            b = np.full((Bs, 4, H), 0.5)
+            self.parts.append((lambda: oracle.kda_recurrent(q, q, q, a, b, S.copy(), nthreads=nth), 64 / Bs))
+            desc.append(f"{Bs} of 64 sequences x 64 heads x 4 tokens")
+        elif workload in ("mla_decode_b16", "mla_decode_b16_paged", "mla_decode_b16_paged_rope",
+                          "mla_decode_b16_fp8", "mla_decode_b16_paged_rope_fp8"):
+            lens = wl.mla_seq_lens(wl.MlaDecode("mla", B=16, seed=1236)).tolist()
+            f, k, d = mla(lens, fp8=workload.endswith("fp8"))
+            self.parts.append((f, k))
+            desc.append(d)
+        elif workload == "mla_mtp_b16":  # four query tokens: four attentions over (nearly) the rows
+            lens = wl.mla_seq_lens(wl.MlaDecode("mla", B=16, seed=1236)).tolist()
+            f, k, d = mla(lens)
+            self.parts.append((f, 4 * k))
+            desc.append(d + ", x4 query tokens")
+        elif workload == "hybrid_8layer_1m":
+            f, k, d1 = kda_layer(8)
+            self.parts.append((f, 7 * k))
+            g, m, d2 = mla([1_000_000] * 8)
+            self.parts.append((g, m))
+            desc.append(f"KDA layer: {d1} (x7 layers); MLA: {d2}")
+        elif workload == "kda_prefill_32k":
+            T, Hs = 1024, min(max(1, nth), H)
+            q = rng.standard_normal((1, T, Hs, D))
+            a = np.full((1, T, Hs, D), 0.95)
+            b = np.full((1, T, Hs), 0.5)
+            S = np.zeros((1, Hs, D, D))
+            self.parts.append((lambda: oracle.kda_recurrent(q, q, q, a, b, S.copy(), nthreads=nth),
+                               (32768 / T) * (64 / Hs)))
+            desc.append(f"{Hs} heads x {T} tokens")
+        else:
+            raise ValueError(workload)
+        self.sample = "; ".join(desc) + "; scaled to the whole step"
+
+    def run(self) -> float:
+        est = 0.0
+        for f, k in self.parts:
             t0 = time.perf_counter()
-            oracle.mla_decode_fp8(qs, codes, wl.KV_SCALE_FP8, np.array([L], np.int32), None, nthreads=nth)
-            dt = time.perf_counter() - t0
-            return dt * H * float(sum(lens)) / (units * L), f"{units} heads x {L} cached tokens of 1 sequence"
-        cache = (rng.standard_normal((1, L, wl.D_ROW)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
-        t0 = time.perf_counter()
-        oracle.mla_decode(qs, cache, np.array([L], np.int32), None, nthreads=nth)
-        dt = time.perf_counter() - t0
-        total_units_tokens = H * float(sum(lens))
-        return dt * total_units_tokens / (units * L), f"{units} heads x {L} cached tokens of 1 sequence"
+            f()
+            est += (time.perf_counter() - t0) * k
+        return est
 
-    if workload in ("kda_decode_b64", "kda_decode_b64_gated"):
-        sec, sample = kda_layer_seconds(64)
-        return {"value": 64 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": sample}
-    if workload == "kda_mtp_b64":
-        # the oracle's recurrence over 4 tokens for a subset of sequences, all 64 heads
-        Bs = min(64, max(1, nth))
-        q = rng.standard_normal((Bs, 4, H, D))
-        S = 0.02 * rng.standard_normal((Bs, H, D, D))
-        a = np.full((Bs, 4, H, D), 0.9)
-        b = np.full((Bs, 4, H), 0.5)
-        t0 = time.perf_counter()
-        oracle.kda_recurrent(q, q, q, a, b, S, nthreads=nth)
-        sec = (time.perf_counter() - t0) * 64 / Bs
-        return {"value": 256 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle",
-                "sample": f"{Bs} of 64 sequences x 64 heads x 4 tokens, scaled to 64 sequences"}
-    if workload in ("mla_decode_b16", "mla_decode_b16_paged", "mla_decode_b16_paged_rope", "mla_decode_b16_fp8",
-                    "mla_decode_b16_paged_rope_fp8", "mla_mtp_b16"):
-        lens = wl.mla_seq_lens(wl.MlaDecode("mla", B=16, seed=1236)).tolist()
-        sec, sample = mla_seconds(16, lens, fp8=workload.endswith("fp8"))
-        if workload == "mla_mtp_b16":  # four query tokens per sequence: four attentions over (nearly) the rows
-            return {"value": 64 / (4 * sec), "unit": "tokens/s", "cores": nth, "kind": "oracle",
-                    "sample": sample + ", x4 query tokens"}
-        return {"value": 16 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": sample}
-    if workload == "hybrid_8layer_1m":
-        ks, s1 = kda_layer_seconds(8)
-        ms, s2 = mla_seconds(8, [1_000_000] * 8)
-        sec = 7 * ks + ms
-        return {"value": 8 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle",
-                "sample": f"KDA layer: {s1} (x7 layers); MLA: {s2}; scaled to 8 sequences x 64 heads"}
-    if workload == "kda_prefill_32k":
-        T = 1024
-        q = rng.standard_normal((1, T, nth, D))
-        a = np.full((1, T, nth, D), 0.95)
-        b = np.full((1, T, nth), 0.5)
-        S = np.zeros((1, nth, D, D))
-        t0 = time.perf_counter()
-        oracle.kda_recurrent(q, q, q, a, b, S, nthreads=nth)
-        dt = time.perf_counter() - t0
-        sec = dt * (32768 / T) * (64 / nth)
-        return {"value": 32768 / sec, "unit": "tokens/s", "cores": nth, "kind": "oracle",
-                "sample": f"{nth} heads x {T} tokens, scaled to 64 heads x 32768 tokens"}
-    raise ValueError(workload)
+
+def cpu_oracle_rate(workload: str, nth: int | None = None, repeats: int = 3) -> dict:
+    """The fp64 oracle's rate (tokens/s of the whole workload step) from the median of `repeats`
+    timed samples after one untimed one, on `nth` threads (default: all host cores)."""
+    import oracle
+    nth = oracle.max_threads() if nth is None else nth
+    smp = OracleSample(workload, nth)
+    smp.run()
+    est = [smp.run() for _ in range(repeats)]
+    med = statistics.median(est)
+    return {"value": _tokens(workload) / med, "unit": "tokens/s", "cores": nth, "kind": "oracle",
+            "sample": smp.sample, "repeats": repeats,
+            "spread": round((max(est) - min(est)) / med, 4)}
+
+
+def cpu_baseline(workload: str) -> dict:
+    """The all-core oracle rate, with the single-thread rate beside it."""
+    cb = cpu_oracle_rate(workload)
+    one = cpu_oracle_rate(workload, nth=1)
+    cb["single_thread"] = {"value": one["value"], "unit": one["unit"], "sample": one["sample"],
+                           "repeats": one["repeats"]}
+    return cb
 
 
 # ---------------------------------------------------------------------------------------------
 
 def run_reference(args, rank, world):
+    """The oracle as the reference arm: W untimed and K timed steps, each step one bounded sample
+    of the workload (OracleSample) on all host cores; ms_per_step is the median wall time of a
+    sample, value the tokens/s of the whole workload step the samples estimate."""
     if rank != 0:
         return 0
-    cb = cpu_oracle_rate(args.workload)
-    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * _tokens(args.workload) / cb["value"],
+    import oracle
+    nth = oracle.max_threads()
+    smp = OracleSample(args.workload, nth)
+    for _ in range(args.warmup):
+        smp.run()
+    wall, est = [], []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        est.append(smp.run())
+        wall.append(time.perf_counter() - t0)
+    step_s = statistics.median(est)
+    value = _tokens(args.workload) / step_s
+    one = cpu_oracle_rate(args.workload, nth=1)
+    cb = {"value": value, "unit": "tokens/s", "cores": nth, "kind": "oracle", "sample": smp.sample,
+          "repeats": args.steps, "single_thread": {"value": one["value"], "unit": one["unit"],
+                                                    "sample": one["sample"], "repeats": one["repeats"]}}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.median(wall),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "implementation": "fp64 CPU oracle (plain C, OpenMP over heads)"},
+            "config": {"workload": args.workload, "implementation": "fp64 CPU oracle (plain C, OpenMP over heads)",
+                       "step": "one bounded sample of the workload step (see cpu_baseline.sample); value is the "
+                               "whole step's tokens over the step time the samples estimate (median)",
+                       "estimated_ms_per_workload_step": 1000.0 * step_s},
             "cpu_baseline": cb,
-            "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -941,6 +999,65 @@ def _tokens(workload):
     return {"hybrid_8layer_1m": 8, "kda_decode_b64": 64, "kda_decode_b64_gated": 64, "kda_mtp_b64": 256, "mla_decode_b16": 16,
             "mla_decode_b16_paged": 16, "mla_decode_b16_paged_rope": 16, "mla_decode_b16_fp8": 16,
             "mla_decode_b16_paged_rope_fp8": 16, "mla_mtp_b16": 64, "kda_prefill_32k": 32768}[workload]
+
+
+def time_device(step, steps: int, warmup: int, local: int, dev):
+    """W untimed steps, then device events around exactly K steps (per-kernel events inside), with
+    the SM clock sampled meanwhile; the step time is the max over ranks."""
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    barrier(local)
+    timer = KernelTimer()
+    clocks = ClockSampler(physical_gpu_index(local))
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    barrier(local)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step.run(timer)
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(local)
+    clk = clocks.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, dev)
+    return ms, timer, clk
+
+
+# configs 1-3 of the workload list, timed after the headline in the same process: the single
+# KDA decode layer (64 x 64 heads), the 16-sequence MLA layer, and the 32K-token prefill
+PER_CONFIG = (("kda_decode_b64", "config 1: KDA decode layer, 64 sequences x 64 heads, conv fused"),
+              ("mla_decode_b16", "config 2: gated MLA decode, 16 sequences, contexts uniform in [8192, 131072]"),
+              ("kda_prefill_32k", "config 3: KDA chunked prefill, 1 x 32768 tokens x 64 heads, chunk 64"))
+
+
+def per_config_lines(lad, dev, rank, local, steps: int, warmup: int, peaks: dict) -> dict:
+    out = {}
+    for name, what in PER_CONFIG:
+        step = WORKLOADS[name](lad, dev, rank)
+        torch.cuda.synchronize()
+        ms, timer, clk = time_device(step, steps, warmup, local, dev)
+        km = timer.mean_ms(step.dominant)
+        ab = step.algorithmic_bytes()
+        gbs = ab[step.dominant] / (km / 1000.0) / 1e9
+        e = {"what": what, "kernel": step.dominant, "ms_per_step": round(ms, 4), "ms_per_launch": round(km, 4),
+             "tokens_per_s": step.tokens_per_step / (ms / 1000.0), "gb_s": round(gbs, 1),
+             "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "steps": steps, "warmup": warmup,
+             "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]}}
+        if isinstance(step, PrefillStep):
+            tf = step.flops() / (km / 1000.0) / 1e12
+            peak_tf32 = peaks["bf16_tflops"] * 1.1 / 2.25
+            e.update({"tflop_s": round(tf, 1), "frac_of_tf32_peak": round(tf / peak_tf32, 4)})
+        if isinstance(step, MlaDecodeStep):
+            e["mma_tflop_s"] = round(step.mla_flops() / (km / 1000.0) / 1e12, 1)
+        out[name] = e
+        del step
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
 
 
 def main(argv=None) -> int:
@@ -954,6 +1071,8 @@ def main(argv=None) -> int:
     ap.add_argument("--seq-len", type=int, default=32768, help="tokens of the kda_prefill_32k workload")
     ap.add_argument("--unfused-conv", action="store_true",
                     help="KDA layers as kda_conv_update + kda_decode_step instead of kda_conv_decode_step")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per_config timings of configs 1-3 after the default workload")
     args = ap.parse_args(argv)
     _KdaLayer.fused = not args.unfused_conv
     if args.warmup < 3:
@@ -977,29 +1096,7 @@ def main(argv=None) -> int:
         step = WORKLOADS[args.workload](lad, dev, rank)
     torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
-        step.run()
-    torch.cuda.synchronize()
-    barrier(local)
-
-    # timed region: device events around exactly K steps, clocks sampled meanwhile
-    timer = KernelTimer()
-    clocks = ClockSampler(physical_gpu_index(local))
-    clocks.start()
-    time.sleep(0.3)
-    torch.cuda.synchronize()
-    barrier(local)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(args.steps):
-        step.run(timer)
-    t1.record()
-    torch.cuda.synchronize()
-    barrier(local)
-    clk = clocks.stop()
-    ms = t0.elapsed_time(t1) / args.steps
-    ms = max_over_ranks(ms, dev)
+    ms, timer, clk = time_device(step, args.steps, args.warmup, local, dev)
 
     # end to end through the public API: pinned host inputs in, outputs back, every step
     for _ in range(3):
@@ -1041,10 +1138,8 @@ def main(argv=None) -> int:
         km = timer.mean_ms(kname)
         per_type[kname]["mma_tflop_s"] = round(m.mla_flops() / (km / 1000.0) / 1e12, 1)
 
+    line = None
     if rank == 0:
-        cb = None
-        if world == 1 and not args.no_cpu_baseline:
-            cb = cpu_oracle_rate(args.workload)
         hb, db = step.e2e_bytes()
         traffic = kernel_traffic(step.dominant, step.dominant_units())
         line = {
@@ -1062,7 +1157,7 @@ def main(argv=None) -> int:
                          "traffic": traffic["bytes"] if traffic else None,
                          "traffic_source": traffic, "peak_source": f"{peaks['source']} hbm_gbs (copy)",
                          "algorithmic_bytes_per_launch": ab[step.dominant]},
-            "cpu_baseline": cb,
+            "cpu_baseline": None,
             "e2e": {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": hb * world,
                     "d2h_bytes_per_step": db * world},
             "gpu_launches": step.launches_per_step * args.steps,
@@ -1080,6 +1175,18 @@ def main(argv=None) -> int:
                                 "peak_source": f"{peaks['source']} bf16_tflops (burst) x 1.1/2.25 (nominal tf32/bf16)",
                                 "algorithmic_flops_per_launch": step.flops(),
                                 "tensor_pipe_active_pct": traffic.get("tensor_pipe_active_pct") if traffic else None}
+
+    # configs 1-3 (single GPU), after the headline, when the default workload runs alone; their
+    # launches are not counted in gpu_launches, which covers the headline's timed region only
+    if world == 1 and args.workload == DEFAULT_WORKLOAD and not args.no_per_config:
+        del step
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        line["per_config"] = per_config_lines(lad, dev, rank, local, min(args.steps, 10), args.warmup, peaks)
+
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.workload)
         print(json.dumps(line), flush=True)
 
     if world > 1:

@@ -9,9 +9,12 @@
  *        (ai.thesatyajit.com)
  *
  * Conventions shared by every call:
- *   - All tensor pointers are DEVICE pointers owned by the caller. The library keeps no state
- *     between calls and allocates no device memory; where scratch space is needed the caller
- *     passes a workspace whose size a *_workspace_size() query returns.
+ *   - All tensor pointers are DEVICE pointers owned by the caller. No call allocates device
+ *     memory; where scratch space is needed the caller passes a workspace whose size a
+ *     *_workspace_size() query returns. The library's only device-resident state is fixed-size
+ *     and compiled in: one error word per kernel module (set by bounded waits and device-side
+ *     input checks, read and cleared by lad_device_error()) and the scratch array of
+ *     mla_latent_decode_noalloc (below).
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Every
  *     call only enqueues work on that stream and returns; results are ready when the stream
  *     reaches that point.
@@ -417,7 +420,9 @@ int mla_cache_append_fp8(const lad_bf16 *c_kv, const lad_bf16 *k_pe, const int *
  *   - B must not exceed mla_latent_decode_noalloc_max_batch() (32); larger B returns
  *     LAD_EUNSUPPORTED with a message. The device must have at most 160 SMs.
  *   - The first call on a device looks up the array's device address (with that device
- *     current); make that first call before any stream capture.
+ *     current) and keeps it for the life of the process; make that first call before any stream
+ *     capture, and do not reset the device (cudaDeviceReset) while the library is in use: a new
+ *     primary context would leave the kept address stale.
  *   - All calls share the one array: calls whose kernels may overlap on the GPU (different
  *     streams, or different host threads) race and give undefined results. Serialise them.
  *   - The array keeps the last call's contents; nothing in it needs to start at zero.

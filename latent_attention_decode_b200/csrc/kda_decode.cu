@@ -67,165 +67,224 @@ struct ConvIn {
     int silu;
 };
 
-template <bool kOutF32, bool kFusedConv>
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// kPair (small batches): a CTA updates two heads, bh = blockIdx.x and bh + gridDim.x. With one
+// head per CTA and B * H between one and two times the resident CTAs (8 x 64 heads on 296 slots),
+// the CTAs of the second wave start only as the first wave's finish, and the waves load, reduce
+// and store in step, so HBM idles between the phases. Here the second head's state is copied
+// into shared memory (cp.async, each thread its own 16-byte slots, read back by the same thread
+// only) while the first head is loaded into registers, so every state byte of the launch is
+// requested at once; the second head then runs from shared memory while the first head's
+// stores drain.
+constexpr int kPairSmemBytes = kRowsPerWarp * kThreads * 16;  // 64 KiB of state slots
+
+template <bool kOutF32, bool kFusedConv, bool kPair>
 __global__ void __launch_bounds__(kThreads, 2)
 kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const uint16_t *__restrict__ v,
                   long long qkv_stride, const float *__restrict__ alpha, const float *__restrict__ beta,
                   float *__restrict__ S, void *__restrict__ o, int H, float scale, int l2norm, ConvIn cv,
-                  GateIn gi) {
-    const int bh = blockIdx.x;
-    const int b = bh / H;
-    const int h = bh - b * H;
+                  GateIn gi, int units) {
+    constexpr int kUnits = kPair ? 2 : 1;
+    extern __shared__ __align__(16) uint8_t pair_slots[];  // kPair: the second head's state
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
+    const int bh0 = blockIdx.x;
+    const int bh1 = kPair ? bh0 + static_cast<int>(gridDim.x) : units;
+    const bool has1 = kPair && bh1 < units;  // uniform over the CTA
 
+    auto state_of = [&](int bh) {
+        return reinterpret_cast<float4 *>(S + static_cast<size_t>(bh) * kD * kD) +
+               static_cast<size_t>(warp * kRowsPerWarp) * kVec + lane;
+    };
     // Issue the 16 state loads first so their latency overlaps everything below.
-    float4 *mine = reinterpret_cast<float4 *>(S + static_cast<size_t>(bh) * kD * kD) +
-                   static_cast<size_t>(warp * kRowsPerWarp) * kVec + lane;
     float4 s[kRowsPerWarp];
+    {
+        const float4 *mine = state_of(bh0);
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) s[r] = __ldcs(mine + r * kVec);
+        for (int r = 0; r < kRowsPerWarp; ++r) s[r] = __ldcs(mine + r * kVec);
+    }
+    const uint32_t slot_base = static_cast<uint32_t>(__cvta_generic_to_shared(pair_slots)) + threadIdx.x * 16;
+    if (has1) {
+        const float4 *src = state_of(bh1);
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) cp_async16(slot_base + r * kThreads * 16, src + r * kVec);
+        cp_async_commit();
+    }
 
-    __shared__ float sq[kD], sk[kD], sv[kD], sa[kD];
+    __shared__ float sq[kUnits][kD], sk[kUnits][kD], sv[kUnits][kD], sa[kUnits][kD];
     __shared__ float4 red_k[kWarps][kVec], red_q[kWarps][kVec];
     __shared__ uint2 s_gate[kVec];   // output gate logits, 4 bf16 per lane of warp 0
     __shared__ float4 s_gw[kVec];    // norm weight, 4 per lane of warp 0
 
-    if constexpr (kFusedConv) {
-        // y = taps . (tail, x) (+ bias), SiLU; kept in fp32; the tail shifts in place. Threads
-        // 0-127 take this head's q and k channels, threads 128-255 its v channels.
-        const size_t cch = static_cast<size_t>(3) * H * kD;
-        const uint16_t *xb = cv.x + static_cast<size_t>(b) * cch;
-        uint16_t *tb = cv.tail + static_cast<size_t>(b) * 3 * cch;
-        auto conv = [&](size_t c) -> float {
-            const uint16_t xr = xb[c], t0 = tb[c], t1 = tb[cch + c], t2 = tb[2 * cch + c];
-            const uint2 wv = *reinterpret_cast<const uint2 *>(cv.w + c * 4);
-            const float2 w01 = lad::dev::bf16x2_to_f32(wv.x), w23 = lad::dev::bf16x2_to_f32(wv.y);
-            float acc = w01.x * bf16_to_f32(t0);
-            acc = fmaf(w01.y, bf16_to_f32(t1), acc);
-            acc = fmaf(w23.x, bf16_to_f32(t2), acc);
-            acc = fmaf(w23.y, bf16_to_f32(xr), acc);
-            if (cv.bias) acc += bf16_to_f32(cv.bias[c]);
-            if (cv.silu) acc = acc / (1.f + expf(-acc));
-            tb[c] = t1;
-            tb[cch + c] = t2;
-            tb[2 * cch + c] = xr;
-            return acc;
-        };
-        const size_t hc = static_cast<size_t>(h) * kD;
-        if (threadIdx.x < kD) {
-            const int i = threadIdx.x;
-            sq[i] = conv(hc + i);
-            sk[i] = conv(static_cast<size_t>(H) * kD + hc + i);
-            sa[i] = alpha[static_cast<size_t>(bh) * kD + i];
+    // this head's q, k, v (through the fused conv, or as given) and alpha into slot u
+    auto inputs = [&](int u, int bh) {
+        const int b = bh / H, h = bh - b * H;
+        if constexpr (kFusedConv) {
+            // y = taps . (tail, x) (+ bias), SiLU; kept in fp32; the tail shifts in place. Threads
+            // 0-127 take this head's q and k channels, threads 128-255 its v channels.
+            const size_t cch = static_cast<size_t>(3) * H * kD;
+            const uint16_t *xb = cv.x + static_cast<size_t>(b) * cch;
+            uint16_t *tb = cv.tail + static_cast<size_t>(b) * 3 * cch;
+            auto conv = [&](size_t c) -> float {
+                const uint16_t xr = xb[c], t0 = tb[c], t1 = tb[cch + c], t2 = tb[2 * cch + c];
+                const uint2 wv = *reinterpret_cast<const uint2 *>(cv.w + c * 4);
+                const float2 w01 = lad::dev::bf16x2_to_f32(wv.x), w23 = lad::dev::bf16x2_to_f32(wv.y);
+                float acc = w01.x * bf16_to_f32(t0);
+                acc = fmaf(w01.y, bf16_to_f32(t1), acc);
+                acc = fmaf(w23.x, bf16_to_f32(t2), acc);
+                acc = fmaf(w23.y, bf16_to_f32(xr), acc);
+                if (cv.bias) acc += bf16_to_f32(cv.bias[c]);
+                if (cv.silu) acc = acc / (1.f + expf(-acc));
+                tb[c] = t1;
+                tb[cch + c] = t2;
+                tb[2 * cch + c] = xr;
+                return acc;
+            };
+            const size_t hc = static_cast<size_t>(h) * kD;
+            if (threadIdx.x < kD) {
+                const int i = threadIdx.x;
+                sq[u][i] = conv(hc + i);
+                sk[u][i] = conv(static_cast<size_t>(H) * kD + hc + i);
+                sa[u][i] = alpha[static_cast<size_t>(bh) * kD + i];
+            } else {
+                const int i = threadIdx.x - kD;
+                sv[u][i] = conv(static_cast<size_t>(2) * H * kD + hc + i);
+            }
         } else {
-            const int i = threadIdx.x - kD;
-            sv[i] = conv(static_cast<size_t>(2) * H * kD + hc + i);
+            const size_t row = static_cast<size_t>(b) * qkv_stride + static_cast<size_t>(h) * kD;
+            if (threadIdx.x < kD) {
+                const int i = threadIdx.x;
+                sq[u][i] = bf16_to_f32(q[row + i]);
+                sk[u][i] = bf16_to_f32(k[row + i]);
+                sv[u][i] = bf16_to_f32(v[row + i]);
+                sa[u][i] = alpha[static_cast<size_t>(bh) * kD + i];
+            }
         }
-    } else {
-        const size_t row = static_cast<size_t>(b) * qkv_stride + static_cast<size_t>(h) * kD;
-        if (threadIdx.x < kD) {
-            const int i = threadIdx.x;
-            sq[i] = bf16_to_f32(q[row + i]);
-            sk[i] = bf16_to_f32(k[row + i]);
-            sv[i] = bf16_to_f32(v[row + i]);
-            sa[i] = alpha[static_cast<size_t>(bh) * kD + i];
+    };
+
+    // one head's update from the state in s (slot u of the inputs); ends with the new state
+    // stored and o written
+    auto update = [&](int u, int bh) {
+        const float bt = beta[bh];
+        // q.k, and the inverse norms when normalising; each warp reduces them itself.
+        float qq = 0.f, kk = 0.f, qk = 0.f;
+#pragma unroll
+        for (int i = lane; i < kD; i += 32) {
+            const float a = sq[u][i], c = sk[u][i];
+            qq = fmaf(a, a, qq);
+            kk = fmaf(c, c, kk);
+            qk = fmaf(a, c, qk);
         }
-    }
-    const float bt = beta[bh];
-    __syncthreads();
+        qq = warp_sum(qq);
+        kk = warp_sum(kk);
+        qk = warp_sum(qk);
+        float rq = 1.f, rk = 1.f;
+        if (l2norm) {
+            rq = rsqrtf(qq + 1e-6f);
+            rk = rsqrtf(kk + 1e-6f);
+        }
+        qk *= rq * rk;
 
-    // q.k, and the inverse norms when normalising; each warp reduces them itself.
-    float qq = 0.f, kk = 0.f, qk = 0.f;
-#pragma unroll
-    for (int i = lane; i < kD; i += 32) {
-        const float a = sq[i], c = sk[i];
-        qq = fmaf(a, a, qq);
-        kk = fmaf(c, c, kk);
-        qk = fmaf(a, c, qk);
-    }
-    qq = warp_sum(qq);
-    kk = warp_sum(kk);
-    qk = warp_sum(qk);
-    float rq = 1.f, rk = 1.f;
-    if (l2norm) {
-        rq = rsqrtf(qq + 1e-6f);
-        rk = rsqrtf(kk + 1e-6f);
-    }
-    qk *= rq * rk;
-
-    // the gate's inputs are fetched here, to land during the decay and the column sums
-    if (gi.g) {
-        if (threadIdx.x < kVec)
-            s_gate[threadIdx.x] = reinterpret_cast<const uint2 *>(gi.g + static_cast<size_t>(bh) * kD)[threadIdx.x];
-        else if (threadIdx.x < 2 * kVec)
-            s_gw[threadIdx.x - kVec] = gi.w ? reinterpret_cast<const float4 *>(gi.w)[threadIdx.x - kVec]
-                                            : make_float4(1.f, 1.f, 1.f, 1.f);
-    }
-
-    // S' = Diag(alpha) S and this warp's share of S'^T k and S'^T q.
-    float4 wk = make_float4(0.f, 0.f, 0.f, 0.f), wq = wk;
-#pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-        const int i = warp * kRowsPerWarp + r;
-        const float a = sa[i];
-        s[r].x *= a;
-        s[r].y *= a;
-        s[r].z *= a;
-        s[r].w *= a;
-        fma4(wk, sk[i] * rk, s[r]);
-        fma4(wq, sq[i] * rq, s[r]);
-    }
-    red_k[warp][lane] = wk;
-    red_q[warp][lane] = wq;
-    __syncthreads();
-    float4 W = red_k[0][lane], Q = red_q[0][lane];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) {
-        add4(W, red_k[w][lane]);
-        add4(Q, red_q[w][lane]);
-    }
-
-    // u = beta (v - S'^T k), then the write S = S' + k u^T.
-    const float4 vv = reinterpret_cast<const float4 *>(sv)[lane];
-    float4 u;
-    u.x = bt * (vv.x - W.x);
-    u.y = bt * (vv.y - W.y);
-    u.z = bt * (vv.z - W.z);
-    u.w = bt * (vv.w - W.w);
-#pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-        const int i = warp * kRowsPerWarp + r;
-        fma4(s[r], sk[i] * rk, u);
-        __stcs(mine + r * kVec, s[r]);
-    }
-
-    // o = scale S^T q = scale (S'^T q + (k.q) u)
-    if (warp == 0) {
-        float4 ov;
-        ov.x = scale * fmaf(qk, u.x, Q.x);
-        ov.y = scale * fmaf(qk, u.y, Q.y);
-        ov.z = scale * fmaf(qk, u.z, Q.z);
-        ov.w = scale * fmaf(qk, u.w, Q.w);
+        // the gate's inputs are fetched here, to land during the decay and the column sums
         if (gi.g) {
-            // gated RMSNorm over the head's 128 outputs (4 per lane)
-            const float ss = warp_sum(ov.x * ov.x + ov.y * ov.y + ov.z * ov.z + ov.w * ov.w);
-            const float inv = rsqrtf(ss * (1.f / kD) + gi.eps);
-            const uint2 gw = s_gate[lane];
-            const float2 g01 = lad::dev::bf16x2_to_f32(gw.x), g23 = lad::dev::bf16x2_to_f32(gw.y);
-            const float4 w4 = s_gw[lane];
-            ov.x *= inv * w4.x / (1.f + __expf(-g01.x));
-            ov.y *= inv * w4.y / (1.f + __expf(-g01.y));
-            ov.z *= inv * w4.z / (1.f + __expf(-g23.x));
-            ov.w *= inv * w4.w / (1.f + __expf(-g23.y));
+            if (threadIdx.x < kVec)
+                s_gate[threadIdx.x] =
+                    reinterpret_cast<const uint2 *>(gi.g + static_cast<size_t>(bh) * kD)[threadIdx.x];
+            else if (threadIdx.x < 2 * kVec)
+                s_gw[threadIdx.x - kVec] = gi.w ? reinterpret_cast<const float4 *>(gi.w)[threadIdx.x - kVec]
+                                                : make_float4(1.f, 1.f, 1.f, 1.f);
         }
-        if constexpr (kOutF32) {
-            reinterpret_cast<float4 *>(static_cast<float *>(o) + static_cast<size_t>(bh) * kD)[lane] = ov;
-        } else {
-            uint2 pk;
-            pk.x = static_cast<uint32_t>(f32_to_bf16(ov.x)) | (static_cast<uint32_t>(f32_to_bf16(ov.y)) << 16);
-            pk.y = static_cast<uint32_t>(f32_to_bf16(ov.z)) | (static_cast<uint32_t>(f32_to_bf16(ov.w)) << 16);
-            reinterpret_cast<uint2 *>(static_cast<uint16_t *>(o) + static_cast<size_t>(bh) * kD)[lane] = pk;
+
+        // S' = Diag(alpha) S and this warp's share of S'^T k and S'^T q.
+        float4 wk = make_float4(0.f, 0.f, 0.f, 0.f), wq = wk;
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            const int i = warp * kRowsPerWarp + r;
+            const float a = sa[u][i];
+            s[r].x *= a;
+            s[r].y *= a;
+            s[r].z *= a;
+            s[r].w *= a;
+            fma4(wk, sk[u][i] * rk, s[r]);
+            fma4(wq, sq[u][i] * rq, s[r]);
+        }
+        red_k[warp][lane] = wk;
+        red_q[warp][lane] = wq;
+        __syncthreads();
+        float4 W = red_k[0][lane], Q = red_q[0][lane];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) {
+            add4(W, red_k[w][lane]);
+            add4(Q, red_q[w][lane]);
+        }
+
+        // u = beta (v - S'^T k), then the write S = S' + k u^T.
+        const float4 vv = reinterpret_cast<const float4 *>(sv[u])[lane];
+        float4 uu;
+        uu.x = bt * (vv.x - W.x);
+        uu.y = bt * (vv.y - W.y);
+        uu.z = bt * (vv.z - W.z);
+        uu.w = bt * (vv.w - W.w);
+        float4 *mine = state_of(bh);
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            const int i = warp * kRowsPerWarp + r;
+            fma4(s[r], sk[u][i] * rk, uu);
+            __stcs(mine + r * kVec, s[r]);
+        }
+
+        // o = scale S^T q = scale (S'^T q + (k.q) u)
+        if (warp == 0) {
+            float4 ov;
+            ov.x = scale * fmaf(qk, uu.x, Q.x);
+            ov.y = scale * fmaf(qk, uu.y, Q.y);
+            ov.z = scale * fmaf(qk, uu.z, Q.z);
+            ov.w = scale * fmaf(qk, uu.w, Q.w);
+            if (gi.g) {
+                // gated RMSNorm over the head's 128 outputs (4 per lane)
+                const float ss = warp_sum(ov.x * ov.x + ov.y * ov.y + ov.z * ov.z + ov.w * ov.w);
+                const float inv = rsqrtf(ss * (1.f / kD) + gi.eps);
+                const uint2 gw = s_gate[lane];
+                const float2 g01 = lad::dev::bf16x2_to_f32(gw.x), g23 = lad::dev::bf16x2_to_f32(gw.y);
+                const float4 w4 = s_gw[lane];
+                ov.x *= inv * w4.x / (1.f + __expf(-g01.x));
+                ov.y *= inv * w4.y / (1.f + __expf(-g01.y));
+                ov.z *= inv * w4.z / (1.f + __expf(-g23.x));
+                ov.w *= inv * w4.w / (1.f + __expf(-g23.y));
+            }
+            if constexpr (kOutF32) {
+                reinterpret_cast<float4 *>(static_cast<float *>(o) + static_cast<size_t>(bh) * kD)[lane] = ov;
+            } else {
+                uint2 pk;
+                pk.x = static_cast<uint32_t>(f32_to_bf16(ov.x)) | (static_cast<uint32_t>(f32_to_bf16(ov.y)) << 16);
+                pk.y = static_cast<uint32_t>(f32_to_bf16(ov.z)) | (static_cast<uint32_t>(f32_to_bf16(ov.w)) << 16);
+                reinterpret_cast<uint2 *>(static_cast<uint16_t *>(o) + static_cast<size_t>(bh) * kD)[lane] = pk;
+            }
+        }
+    };
+
+    inputs(0, bh0);
+    if (has1) inputs(1 % kUnits, bh1);
+    __syncthreads();
+    update(0, bh0);
+    if constexpr (kPair) {
+        if (has1) {
+            // the second head: this thread's own slots (no barrier needed to read them), then a
+            // barrier before the reduction buffers and the gate inputs are reused
+            cp_async_wait_all();
+            const float4 *slots = reinterpret_cast<const float4 *>(pair_slots) + threadIdx.x;
+#pragma unroll
+            for (int r = 0; r < kRowsPerWarp; ++r) s[r] = slots[r * kThreads];
+            __syncthreads();
+            update(1, bh1);
         }
     }
 }
@@ -257,14 +316,6 @@ __host__ __device__ constexpr int multi_smem_bytes(int T) {
     return kMOffRaw + 2 * T * kRawTokenBytes + T * kD * 16 + T * kD * 4;  // + per-row {alpha, k, q}, k
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // cp.async of head bh's token inputs (tokens 0..n-1) into one input buffer: piece p of token t
 // (16 bytes: q, k, v 8 bf16 each, alpha 4 fp32) and beta_t. The caller commits.
@@ -461,6 +512,42 @@ kda_decode_multi_kernel(const uint16_t *__restrict__ q, const uint16_t *__restri
 
 }  // namespace
 
+namespace {
+// One head per CTA, or two (kPair) when B * H is between one and two times the resident CTAs:
+// then every CTA is resident at once and all state bytes are requested together.
+template <bool kOutF32, bool kFusedConv>
+int launch_decode(const char *name, const uint16_t *q, const uint16_t *k, const uint16_t *v, long long stride,
+                  const float *alpha, const float *beta, float *S, void *o, int units, int H, float scale, int l2,
+                  const ConvIn &cv, const GateIn &gi, cudaStream_t s) {
+    const int sms = lad::device_sm_count();
+    const long long slots = 2LL * (sms > 0 ? sms : 0);
+    if (sms > 0 && units > slots && units <= 2 * slots) {
+        static std::mutex mu;
+        static bool done[64] = {};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess || dev < 0 || dev >= 64)
+            return lad::set_error(LAD_ECUDA, "%s: cudaGetDevice: %s", name, cudaGetErrorString(e));
+        {
+            std::lock_guard<std::mutex> lock(mu);
+            if (!done[dev]) {
+                e = cudaFuncSetAttribute(kda_decode_kernel<kOutF32, kFusedConv, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes);
+                if (e != cudaSuccess)
+                    return lad::set_error(LAD_ECUDA, "%s: smem attribute: %s", name, cudaGetErrorString(e));
+                done[dev] = true;
+            }
+        }
+        kda_decode_kernel<kOutF32, kFusedConv, true><<<static_cast<unsigned>(slots), kThreads, kPairSmemBytes, s>>>(
+            q, k, v, stride, alpha, beta, S, o, H, scale, l2, cv, gi, units);
+    } else {
+        kda_decode_kernel<kOutF32, kFusedConv, false><<<static_cast<unsigned>(units), kThreads, 0, s>>>(
+            q, k, v, stride, alpha, beta, S, o, H, scale, l2, cv, gi, units);
+    }
+    return lad::check_launch(name);
+}
+}  // namespace
+
 extern "C" int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, long long qkv_batch_stride,
                                const float *alpha, const float *beta, float *S, void *o, int B, int H, int dk,
                                int dv, float scale, unsigned flags, void *stream) {
@@ -484,15 +571,13 @@ extern "C" int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_b
     const int l2 = (flags & LAD_FLAG_L2NORM_QK) ? 1 : 0;
     cudaStream_t s = lad::as_stream(stream);
     const ConvIn none{nullptr, nullptr, nullptr, nullptr, 0};
-    if (f32)
-        kda_decode_kernel<true, false><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(q, k, v, stride, alpha, beta,
-                                                                                          S, o, H, scale, l2, none,
-                                                                                          GateIn{});
-    else
-        kda_decode_kernel<false, false><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(q, k, v, stride, alpha, beta,
-                                                                                           S, o, H, scale, l2, none,
-                                                                                           GateIn{});
-    return lad::check_launch("kda_decode_step");
+    const uint16_t *qq = reinterpret_cast<const uint16_t *>(q), *kk = reinterpret_cast<const uint16_t *>(k),
+                   *vv = reinterpret_cast<const uint16_t *>(v);
+    const int units = static_cast<int>(blocks);
+    return f32 ? launch_decode<true, false>("kda_decode_step", qq, kk, vv, stride, alpha, beta, S, o, units, H, scale,
+                                            l2, none, GateIn{}, s)
+               : launch_decode<false, false>("kda_decode_step", qq, kk, vv, stride, alpha, beta, S, o, units, H, scale,
+                                             l2, none, GateIn{}, s);
 }
 
 namespace {
@@ -518,13 +603,11 @@ int conv_decode(const char *name, const lad_bf16 *x, lad_bf16 *conv_tail, const 
     const int l2 = (flags & LAD_FLAG_L2NORM_QK) ? 1 : 0;
     const ConvIn cv{x, conv_tail, conv_w, conv_bias, (flags & LAD_FLAG_SILU) ? 1 : 0};
     cudaStream_t s = lad::as_stream(stream);
-    if (f32)
-        kda_decode_kernel<true, true><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
-            nullptr, nullptr, nullptr, 0, alpha, beta, S, o, H, scale, l2, cv, gi);
-    else
-        kda_decode_kernel<false, true><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(
-            nullptr, nullptr, nullptr, 0, alpha, beta, S, o, H, scale, l2, cv, gi);
-    return lad::check_launch(name);
+    const int units = static_cast<int>(blocks);
+    return f32 ? launch_decode<true, true>(name, nullptr, nullptr, nullptr, 0, alpha, beta, S, o, units, H, scale, l2,
+                                           cv, gi, s)
+               : launch_decode<false, true>(name, nullptr, nullptr, nullptr, 0, alpha, beta, S, o, units, H, scale, l2,
+                                            cv, gi, s);
 }
 }  // namespace
 

@@ -6,6 +6,9 @@ Tolerances (relative L2 = ||got - want|| / ||want||):
 - outputs the kernel writes as bf16 are compared with the oracle's fp64 result, so one bf16
   rounding (relative 2^-9 per element, ~1.7e-3 RMS on N(0,1) data) is inside the 2e-3 budget;
   where an output can also be requested as fp32, the fp32 path is held to a tighter bound.
+- besides the norm over a whole tensor, max_rel_l2 takes the norm per unit (per head of a
+  sequence, say) and returns the worst unit, so that a fault confined to a few units is not
+  diluted by the rest of the tensor; it is applied with the same budgets.
 """
 import numpy as np
 import torch
@@ -32,3 +35,17 @@ def bf16_round(x: np.ndarray) -> np.ndarray:
     """Round fp64 values to bf16 (to nearest even) through fp32, as the kernels' stores do."""
     return torch.from_numpy(np.asarray(x, dtype=np.float64)).to(torch.float32).to(torch.bfloat16).to(
         torch.float64).numpy()
+
+
+def max_rel_l2(got, want, lead: int) -> float:
+    """The largest relative L2 over the units that the first `lead` axes index (for example
+    lead=2 on [B, H, ...]: one norm per (sequence, head)); units whose reference is all zero are
+    measured by their absolute error."""
+    g, w = f64(got), f64(want)
+    assert g.shape == w.shape, (g.shape, w.shape)
+    n = int(np.prod(g.shape[:lead])) if lead else 1
+    g, w = g.reshape(n, -1), w.reshape(n, -1)
+    den = np.linalg.norm(w, axis=1)
+    num = np.linalg.norm(g - w, axis=1)
+    r = np.where(den > 0, num / np.where(den > 0, den, 1.0), num)
+    return float(r.max()) if r.size else 0.0

@@ -73,3 +73,29 @@ def test_measured_peaks_and_token_counts():
     for w in bench.WORKLOADS:
         assert bench._tokens(w) > 0, w
     assert bench.DEFAULT_WORKLOAD in bench.WORKLOADS
+
+
+def test_oracle_sample_scales_to_the_whole_step():
+    """The oracle's bounded sample for the prefill workload: one thread runs 1 head x 1024 tokens,
+    and the estimate scales it by 32 (tokens) x 64 (heads) to the 32,768-token step."""
+    smp = bench.OracleSample("kda_prefill_32k", nth=1)
+    assert len(smp.parts) == 1 and abs(smp.parts[0][1] - 32 * 64) < 1e-9
+    assert "1 heads x 1024 tokens" in smp.sample
+    est = smp.run()
+    assert est > 0
+    r = bench.cpu_oracle_rate("kda_prefill_32k", nth=1, repeats=3)
+    assert r["repeats"] == 3 and r["cores"] == 1 and r["value"] > 0 and r["spread"] >= 0
+
+
+def test_reference_arm_reports_the_samples_it_ran(capsys):
+    """--impl reference: K timed steps, each one bounded sample; ms_per_step is a sample's wall
+    time, so ms_per_step x steps is the time the timed samples actually took."""
+    import time
+    t0 = time.perf_counter()
+    assert bench.main(["--impl", "reference", "--workload", "kda_prefill_32k", "--steps", "3", "--warmup", "3"]) == 0
+    wall = time.perf_counter() - t0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 3 and line["warmup"] == 3
+    assert line["ms_per_step"] * line["steps"] / 1000.0 < wall
+    assert line["cpu_baseline"]["single_thread"]["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import workloads as wl
-from tests.parity import TOL_OUT, TOL_STATE, bf16_round, f64, rel_l2
+from tests.parity import TOL_OUT, TOL_STATE, bf16_round, f64, max_rel_l2, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -121,6 +121,7 @@ def test_decode_b64_conv_then_step(lad, cuda_device):
     assert np.all(np.abs(yg - y_ref16) <= np.abs(y_ref16) * 2.0 ** -7 + 1e-30)
     assert rel_l2(o, o_ref[:, 0]) < 1e-4
     assert rel_l2(inp["S"], S_ref) < TOL_STATE
+    assert max_rel_l2(o, o_ref[:, 0], 2) < 1e-4 and max_rel_l2(inp["S"], S_ref, 2) < TOL_STATE
 
 
 @pytest.mark.parametrize("B,H", [(1, 1), (3, 7), (256, 64)])
@@ -196,6 +197,68 @@ def test_fused_conv_decode_b64(lad, cuda_device):
     assert np.array_equal(f64(inp["tail"]), tail_ref)
     assert rel_l2(o, o_ref) < 1e-4
     assert rel_l2(inp["S"], S_ref) < TOL_STATE
+    assert max_rel_l2(o, o_ref, 2) < 1e-4 and max_rel_l2(inp["S"], S_ref, 2) < TOL_STATE
+
+
+def _slots():
+    """Resident CTAs of the single-token kernel: two per SM."""
+    return 2 * torch.cuda.get_device_properties(0).multi_processor_count
+
+
+def test_fused_conv_decode_b8_paired(lad, cuda_device):
+    """The hybrid's KDA layer at full size, 8 sequences x 64 heads: 512 heads are more than the
+    resident CTAs, so each CTA updates two heads (the second from shared memory). Every element
+    of o, the state and the tails against the oracle; the ungated, gated and two-call forms."""
+    cfg = wl.KdaDecode("kda_b8", B=8, seed=1238)
+    assert _slots() < cfg.B * cfg.H <= 2 * _slots()
+    a = wl.kda_decode_inputs(cfg, cuda_device)
+    g = {n: t.clone() for n, t in a.items()}
+    c = {n: t.clone() for n, t in a.items()}
+    orig = {n: f64(t) for n, t in a.items()}
+    o_ref, S_ref, tail_ref = _fused_oracle(a, cfg.H)
+    o = lad.kda_conv_decode_step(a["x"], a["tail"], a["w"], a["alpha"], a["beta"], a["S"], out_fp32=True)
+    gate = wl.normal_bf16((8, 64, 128), 52, "gate", cuda_device, std=2.0)
+    og = lad.kda_conv_decode_step_gated(g["x"], g["tail"], g["w"], g["alpha"], g["beta"], g["S"], gate, None,
+                                        eps=1e-5, out_fp32=True)
+    hd = cfg.H * 128
+    y = lad.kda_conv_update(c["x"], c["tail"], c["w"], silu=True)
+    o2 = lad.kda_decode_step(y[:, :hd], y[:, hd:2 * hd], y[:, 2 * hd:], c["alpha"], c["beta"], c["S"],
+                             l2norm_qk=True, out_fp32=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(f64(a["tail"]), tail_ref)
+    assert rel_l2(o, o_ref) < 1e-4 and max_rel_l2(o, o_ref, 2) < 1e-4
+    assert rel_l2(a["S"], S_ref) < TOL_STATE and max_rel_l2(a["S"], S_ref, 2) < TOL_STATE
+    want_g = oracle.gated_rmsnorm(o_ref, f64(gate), None, eps=1e-5)
+    assert max_rel_l2(og, want_g, 2) < 1e-4 and torch.equal(g["S"], a["S"])
+    # the two-call path sees the conv output rounded to bf16: the oracle of that, per head
+    y16 = bf16_round(oracle.short_conv_step(orig["x"], orig["tail"], orig["w"], None, silu=True)[0])
+    qr = oracle.l2norm(y16[:, :hd].reshape(8, 1, 64, 128))
+    kr = oracle.l2norm(y16[:, hd:2 * hd].reshape(8, 1, 64, 128))
+    o2_ref, S2_ref = oracle.kda_recurrent(qr, kr, y16[:, 2 * hd:].reshape(8, 1, 64, 128), orig["alpha"][:, None],
+                                          orig["beta"][:, None], orig["S"], nthreads=oracle.max_threads())
+    assert max_rel_l2(o2, o2_ref[:, 0], 2) < 1e-4 and max_rel_l2(c["S"], S2_ref, 2) < TOL_STATE
+
+
+@pytest.mark.parametrize("extra", ["one_past", "half", "all_paired", "one_more_than_paired"])
+def test_paired_launch_boundaries(lad, cuda_device, extra):
+    """Head counts around the switch between one and two heads per CTA (one head per sequence so
+    that any count is reachable): just above the resident CTAs, in between, exactly twice (every
+    CTA paired), and one more (back to one head per CTA)."""
+    n = _slots()
+    B = {"one_past": n + 1, "half": n + n // 2 + 1, "all_paired": 2 * n, "one_more_than_paired": 2 * n + 1}[extra]
+    cfg = wl.KdaDecode("pb", B=B, H=1, seed=60)
+    inp = wl.kda_decode_inputs(cfg, cuda_device)
+    q = wl.unit_sphere_bf16((B, 1, 128), 61, "q", cuda_device)
+    k = wl.unit_sphere_bf16((B, 1, 128), 61, "k", cuda_device)
+    v = wl.normal_bf16((B, 1, 128), 61, "v", cuda_device)
+    S0 = f64(inp["S"])
+    o = lad.kda_decode_step(q, k, v, inp["alpha"], inp["beta"], inp["S"], out_fp32=True)
+    torch.cuda.synchronize()
+    o_ref, S_ref = oracle.kda_recurrent(f64(q)[:, None], f64(k)[:, None], f64(v)[:, None],
+                                        f64(inp["alpha"])[:, None], f64(inp["beta"])[:, None], S0,
+                                        nthreads=oracle.max_threads())
+    assert max_rel_l2(o, o_ref[:, 0], 2) < 1e-5
+    assert max_rel_l2(inp["S"], S_ref, 2) < TOL_STATE
 
 
 @pytest.mark.parametrize("B,H,silu,bias", [(1, 1, True, False), (3, 5, False, True)])

@@ -13,7 +13,7 @@ import torch
 
 import oracle
 import workloads as wl
-from tests.parity import TOL_OUT, bf16_round, f64, rel_l2
+from tests.parity import TOL_OUT, bf16_round, f64, max_rel_l2, rel_l2
 
 pytestmark = pytest.mark.gpu
 TOL_PREFILL_STATE = 2e-3
@@ -115,12 +115,20 @@ def test_prefill_empty_sequence_keeps_state(lad, cuda_device):
 
 @pytest.mark.slow
 def test_prefill_32k_full_size_sampled(lad, cuda_device):
-    """The 32,768-token, 64-head workload at full size; two heads checked over every token."""
+    """The 32,768-token, 64-head workload at full size; eight heads checked over every token, each
+    head's outputs and final state on its own as well as together. The measured errors are
+    printed (run with -s to see them)."""
     cfg = wl.CONFIGS["kda_prefill_32k"]
     inp = wl.kda_scan_inputs(cfg, cuda_device)
     o, S = _run(lad, inp, cuda_device, out_fp32=True)
-    heads = [5, 60]
+    heads = [0, 5, 17, 26, 38, 45, 60, 63]
     cpu = {n: inp[n].cpu() for n in inp}
     o_ref, S_ref = _oracle(cpu, heads=heads)
-    assert rel_l2(o[:, :, heads], o_ref) < TOL_OUT
-    assert rel_l2(S[:, heads], S_ref) < TOL_PREFILL_STATE
+    og, Sg = o[:, :, heads].permute(0, 2, 1, 3), S[:, heads]
+    oref = o_ref.transpose(0, 2, 1, 3)
+    errs = {"o": rel_l2(og, oref), "o_max_head": max_rel_l2(og, oref, 2), "S": rel_l2(Sg, S_ref),
+            "S_max_head": max_rel_l2(Sg, S_ref, 2)}
+    print("prefill 32k measured relative L2:", errs)
+    assert errs["o"] < TOL_OUT and errs["o_max_head"] < TOL_OUT
+    assert errs["S"] < TOL_PREFILL_STATE and errs["S_max_head"] < TOL_PREFILL_STATE
+    assert torch.isfinite(o).all()

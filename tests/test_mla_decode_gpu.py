@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import workloads as wl
-from tests.parity import TOL_OUT, bf16_round, f64, rel_l2
+from tests.parity import TOL_OUT, bf16_round, f64, max_rel_l2, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -134,6 +134,7 @@ def test_decode_b16_full_size_sampled(lad, cuda_device):
     seqs = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 3, 11})
     o_ref, lse_ref = _oracle(inp["q"], inp["cache"], inp["seq_lens"], inp["gate"], seqs=seqs)
     assert rel_l2(o[seqs], o_ref) < TOL_OUT
+    assert max_rel_l2(o[seqs], o_ref, 2) < TOL_OUT   # every (sequence, head) on its own
     np.testing.assert_allclose(f64(lse[seqs]), lse_ref, rtol=0, atol=1e-3)
 
 
@@ -153,13 +154,15 @@ def test_million_token_context_sampled(lad, cuda_device):
 @pytest.mark.slow
 def test_hybrid_launch_8x1m_sampled(lad, cuda_device):
     """The 8-layer hybrid step's latent decode exactly as bench.py launches it: 8 sequences of
-    1,000,000 cached rows drawn with the bench's seed; eight heads (one per head group of each
-    TMEM sub-partition) of two sequences, the first and the last, against the oracle."""
+    1,000,000 cached rows drawn with the bench's seed; every head of the first sequence and eight
+    heads (one per head group of each TMEM sub-partition) of the last, against the oracle, each
+    (sequence, head) on its own as well as together."""
     cfg = wl.MlaDecode("mla", B=8, seed=1238, fixed_len=1_000_000)
     inp = wl.mla_inputs(cfg, cuda_device)
     o, lse = _run(lad, inp["q"], inp["cache"], inp["seq_lens"], inp["gate"], out_fp32=False)
-    seqs, heads = [0, 7], [0, 9, 18, 27, 36, 45, 54, 63]
-    o_ref, lse_ref = _oracle(inp["q"], inp["cache"], inp["seq_lens"], inp["gate"], seqs=seqs, heads=heads)
-    got = o[seqs][:, heads]
-    assert rel_l2(got, bf16_round(o_ref)) < TOL_OUT
-    np.testing.assert_allclose(f64(lse[seqs][:, heads]), lse_ref, rtol=0, atol=1e-3)
+    for seqs, heads in (([0], list(range(64))), ([7], [0, 9, 18, 27, 36, 45, 54, 63])):
+        o_ref, lse_ref = _oracle(inp["q"], inp["cache"], inp["seq_lens"], inp["gate"], seqs=seqs, heads=heads)
+        got = o[seqs][:, heads]
+        assert rel_l2(got, bf16_round(o_ref)) < TOL_OUT
+        assert max_rel_l2(got, bf16_round(o_ref), 2) < TOL_OUT
+        np.testing.assert_allclose(f64(lse[seqs][:, heads]), lse_ref, rtol=0, atol=1e-3)

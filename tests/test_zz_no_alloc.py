@@ -58,11 +58,35 @@ def test_noalloc_matches_workspace_entry_point(cuda_device):
         assert rel_l2(lse_n[fin], lse_w[fin]) < TOL_OUT
 
 
+def test_noalloc_python_wrapper(cuda_device):
+    """The binding's own marshalling (shape checks, the single-sequence stride, d_rope = D - 512)
+    with caller-allocated o and lse, including B = 1, against the workspace entry point."""
+    import latent_attention_decode_b200 as lad
+    for lens, lmax, seed in (([777], 800, 41), ([5, 0, 1200, 64], 1300, 42)):
+        q, cache, L, gate = _inputs(lens, lmax, seed, cuda_device)
+        B = len(lens)
+        o_n = torch.empty((B, 64, 512), device=cuda_device, dtype=torch.float32)
+        lse_n = torch.empty((B, 64), device=cuda_device, dtype=torch.float32)
+        out = lad.mla_latent_decode_noalloc(q, cache, L, gate, o=o_n, lse=lse_n, out_fp32=True)
+        assert out.data_ptr() == o_n.data_ptr()
+        lse_w = torch.empty_like(lse_n)
+        o_w = lad.mla_latent_decode(q, cache, L, gate, lse=lse_w, out_fp32=True)
+        torch.cuda.synchronize()
+        assert lad.lad_device_error() == 0
+        assert rel_l2(o_n, o_w) < TOL_OUT
+        fin = torch.isfinite(lse_w)
+        assert torch.equal(fin, torch.isfinite(lse_n))
+        assert rel_l2(lse_n[fin], lse_w[fin]) < TOL_OUT
+
+
 def test_noalloc_rejects_batch_over_limit(cuda_device):
     import latent_attention_decode_b200 as lad
     lim = lad._lib.mla_latent_decode_noalloc_max_batch()
     q, cache, L, gate = _inputs([8] * (lim + 1), 8, 3, cuda_device)
+    o = torch.full((lim + 1, 64, 512), 7.0, device=cuda_device, dtype=torch.bfloat16)
     f = lad._lib.mla_latent_decode_noalloc
-    rc = f(q.data_ptr(), cache.data_ptr(), cache.stride(0), L.data_ptr(), gate.data_ptr(), q.data_ptr(), None,
+    rc = f(q.data_ptr(), cache.data_ptr(), cache.stride(0), L.data_ptr(), gate.data_ptr(), o.data_ptr(), None,
            lim + 1, 64, 512, 64, 8, wl.MLA_SCALE, 0, None)
     assert rc == -2 and b"scratch limit" in lad._lib.lad_last_error()
+    torch.cuda.synchronize()
+    assert bool((o == 7.0).all())  # rejected before any launch: o untouched
