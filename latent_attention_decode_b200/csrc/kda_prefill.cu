@@ -612,56 +612,218 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
 
 
 // ------------------------------------------------------------------------------------------
-// Split path: the chunk-local, state-independent part of every chunk in parallel (prep), then
-// the state chain alone (scan). With S0 the state entering a chunk:
-//   X = W S0,  O = scale (Qt S0 + P (U' - X)),  S = Diag(g_last) (S0 + Kh^T (U' - X))
-// where W = Tb Kt, U' = Tb V and P = lower(Qt Kh^T) depend only on the chunk's own inputs. The
-// scan then runs two MMA batches per chunk instead of three, and none of the chunk's operand
-// formation or the (I + A)^-1 solve stays on the serial chain; the price is the per-chunk
-// operands' round trip through HBM (one record per (sequence, head, chunk)).
+// Split path (a workspace is given): the chunk-local, state-independent part of every chunk in
+// parallel (prep), then the state chain alone (chain), segment by segment. With S0 the state
+// entering a chunk, U' = Tb V, W = Tb Kt and P = lower(Qt Kh^T):
+//   X = W S0,  U = U' - X,  O = scale (Qt S0 + P U),  S = Diag(g_last) S0 + Kg^T U
+// with Kg = K * g_last / g (the chunk's decay folded into the key). The chain holds S^T (rows d_v,
+// columns d_k) as its fp32 master in tensor memory and runs, per chunk, two tensor-core batches:
+//   [X^T | O^T]  = S0^T [W; Qt]^T           M = 128 (d_v), N = 128 (64 W + 64 Qt rows), K = 128
+//   S^T += U^T Kg,  O^T += U^T P^T          M = 128, N = 128 and 64, K = 64 (tokens)
+// Every operand is fp16 (kind::f16, fp32 accumulation): its rounding unit is that of tf32 and it
+// runs at twice tf32's rate with half the bytes; each tile is stored once, rows as formed, and
+// the tensor cores read it K-major or MN-major as a contraction needs (no transposed copies).
+// U' is formed from the bf16 values with Tb split into bf16 hi + lo (two MMAs): V enters exactly
+// as given. Values whose magnitude leaves the fp16 range (65504) would overflow: with unit-norm
+// keys that needs a chunk's decay product below about 1.5e-5.
 // ------------------------------------------------------------------------------------------
 
-// Record of one (sequence, head, chunk) in the workspace. The four tiles are stored exactly as
-// their shared-memory operand tiles (K-major, tf32-rounded fp32, 128-byte swizzle, 1 KiB aligned),
-// so the scan copies them byte for byte.
-constexpr uint32_t kItW = 0;          // W = Tb Kt [64 tok][128 d_k]: 4 blocks x 8 KiB
-constexpr uint32_t kItQ = 32768;      // Qt [64 tok][128 d_k]: 4 blocks x 8 KiB
-constexpr uint32_t kItKHT = 65536;    // Kh^T [128 d_k][64 tok]: 2 blocks x 16 KiB
-constexpr uint32_t kItP = 98304;      // lower(Qt Kh^T) [64][64]: 2 blocks x 8 KiB
-constexpr uint32_t kItU = 114688;     // U' = Tb V, plain fp32 [2 d_v halves][64 tok][64]
-constexpr uint32_t kItG = 147456;     // g_last [128] fp32
-constexpr uint32_t kItemBytes = 148480;  // 145 KiB
-constexpr int kSegChunks = 128;          // chunks per segment (prep then scan), bounds the workspace
+// Record of one (sequence, head, chunk) in the workspace: the three fp16 tiles and g_last, laid
+// out exactly as the chain's shared-memory operands (one bulk copy), then U' for direct loads.
+constexpr uint32_t kRQW = 0;           // [W; Qt]: 128 rows x 128 d_k fp16, K-major SW128, 2 blocks x 16 KiB
+constexpr uint32_t kRKG = 32768;       // Kg [64 tok][128 d_k] fp16, SW128, 2 blocks x 8 KiB (read MN-major)
+constexpr uint32_t kRP = 49152;        // P = lower(Qt Kh^T) [64 r][64 s] fp16, K-major SW128, 8 KiB
+constexpr uint32_t kRG = 57344;        // g_last [128] fp32
+constexpr uint32_t kRTiles = 57856;    // the four above: one bulk copy
+constexpr uint32_t kRUP = 57856;       // U' [64 tok][128 d_v] fp32, plain row-major
+constexpr uint32_t kRecBytes = 90624;  // 708 lines of 128 bytes
+#ifndef LAD_PREFILL_SEG_CHUNKS
+#define LAD_PREFILL_SEG_CHUNKS 128
+#endif
+constexpr int kSegChunks = LAD_PREFILL_SEG_CHUNKS;  // chunks per segment (prep, then chain)
 
-// prep shared memory
-constexpr uint32_t kPStA = 0, kPStQ = 32768, kPStK = 49152, kPStV = 65536;  // raw staging (80 KiB)
-constexpr uint32_t kPKHT = 0;        // Kh^T [128][64], stride 16 KiB (over the staged alpha)
-constexpr uint32_t kPKTT = 32768;    // Kt^T [128][64], stride 16 KiB (over the staged q, k)
-constexpr uint32_t kPP = 65536;      // P [64][64], stride 8 KiB (over the staged v)
-constexpr uint32_t kPXQK = 81920;    // [Qt; Kt] 128 x 128, stride 16 KiB
-constexpr uint32_t kPTT = kPXQK + 8192;  // Tb in the Kt half of XQK blocks 0-1
-constexpr uint32_t kPKH = 147456;    // Kh [64][128], stride 8 KiB; then the A / T scratch
-constexpr uint32_t kPVT = 180224;    // V^T [128 d_v][64 tok], stride 16 KiB
-constexpr uint32_t kPMisc = 212992;
-constexpr uint32_t kPStageTx = 32768 + 16384 + 16384 + 16384;
-constexpr uint32_t kPSmemBytes = kPMisc + kMiscOct + 8 * 128 * 4 + 1024;
+// fp16 / bf16 SW128 tiles: 64 two-byte columns per 128-byte row, blocks of 64 columns
+__device__ __forceinline__ uint32_t sw128_off16(int row, int col, uint32_t block_bytes) {
+    const int cc = col & 63;
+    return static_cast<uint32_t>(col >> 6) * block_bytes + static_cast<uint32_t>(row) * 128u +
+           static_cast<uint32_t>(((cc >> 3) ^ (row & 7)) << 4) + static_cast<uint32_t>((cc & 7) << 1);
+}
 
-constexpr uint32_t kPColAcc1 = 0;    // M=128 x 64: [Qt Kh^T ; Kt Kh^T]
-constexpr uint32_t kPColW = 64;      // M=64 x 128: W = Tb Kt
-constexpr uint32_t kPColU = 192;     // M=64 x 128: U' = Tb V
-constexpr uint32_t kIdesc64x128 = make_idesc(64, 128, kFmtTf32, 0, 0);
+// K-major SW128 descriptor of a 16-bit tile for k-step j (16 elements of K per MMA)
+__device__ __forceinline__ uint64_t kdesc16(uint64_t base_desc, uint32_t block_bytes, int j) {
+    return base_desc + ((static_cast<uint32_t>(j >> 2) * block_bytes + static_cast<uint32_t>(j & 3) * 32u) >> 4);
+}
 
-struct SplitArgs {
-    const uint16_t *q, *k, *v;
-    const float *alpha, *beta;
-    float *S;
-    void *o;
-    uint8_t *ws;        // records of this segment, [B*H][nseg]
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
+}
+
+constexpr uint32_t kIdescA = make_idesc(128, 64, kFmtF16, 0, 0);     // [Kt; Qt] Kh^T
+constexpr uint32_t kIdescW = make_idesc(64, 128, kFmtF16, 0, 1);     // W = Tb Kt (Kt read MN-major)
+constexpr uint32_t kIdescU = make_idesc(128, 64, kFmtBf16, 1, 0);    // U'^T = V^T Tb^T (V read MN-major)
+constexpr uint32_t kIdescXO = make_idesc(128, 128, kFmtF16, 0, 0);   // [X^T | O^T] = S^T [W; Qt]^T
+constexpr uint32_t kIdescS = make_idesc(128, 128, kFmtF16, 0, 1);    // S^T += U^T Kg (Kg read MN-major)
+constexpr uint32_t kIdescO = make_idesc(128, 64, kFmtF16, 0, 0);     // O^T += U^T P^T
+
+struct PrepArgs {
+    const float *beta;
+    uint8_t *ws;  // this segment's records, [B*H][nseg]
     int B, T, H;
-    int c0, nseg;       // the segment: chunks c0 .. c0 + nseg - 1
-    float scale;
-    int l2norm, out_f32;
+    int c0, nseg;  // the segment: chunks c0 .. c0 + nseg - 1
+    int l2norm;
 };
+
+struct PrepMaps {
+    CUtensorMap q, k, alpha;  // 3-D [B][T][H*128], boxes of 128 channels x 64 tokens, no swizzle
+    CUtensorMap v;            // the same view of v, boxes of 64 channels x 64 tokens, 128-byte swizzle
+};
+
+// prep shared memory (offsets from a 1024-aligned base); the record's tiles sit as in the record
+constexpr uint32_t kPQW = kRQW, kPKG = kRKG, kPP = kRP, kPG = kRG;  // [0, 57856)
+constexpr uint32_t kPKH = 58368;    // Kh [64 tok][128 d_k] fp16 K-major, 2 blocks x 8 KiB
+constexpr uint32_t kPTB = 74752;    // Tb [64 r][64 s] fp16 K-major
+constexpr uint32_t kPTBH = 82944;   // Tb, bf16 high part
+constexpr uint32_t kPTBL = 91136;   // Tb, bf16 low part (Tb - hi)
+constexpr uint32_t kPV = 99328;     // v [64 tok][128 d_v] bf16 as two SW128 boxes of 64 d_v (TMA)
+constexpr uint32_t kPSQ = 115712;   // q [64 tok][128] bf16, plain (TMA)
+constexpr uint32_t kPSK = 132096;   // k, the same
+constexpr uint32_t kPSA = 148480;   // alpha [64 tok][128] fp32, plain (TMA)
+constexpr int kAS = 68;             // row stride (floats) of the A / T scratch (68: fewer bank conflicts)
+constexpr uint32_t kPA = 181248;    // A [64][kAS] fp32
+constexpr uint32_t kPT = kPA + 64 * kAS * 4;   // T [64][kAS] fp32
+constexpr uint32_t kPMisc = kPT + 64 * kAS * 4;
+constexpr uint32_t kPmBeta = 0, kPmRq = 256, kPmRk = 512, kPmOct = 768, kPmBar = 768 + 4096, kPmTmem = kPmBar + 16,
+                   kPmAbort = kPmBar + 20;
+constexpr uint32_t kPSmemBytes = kPMisc + kPmBar + 32 + 1024;
+constexpr uint32_t kPStageQKA = 16384 + 16384 + 32768;
+constexpr uint32_t kPStageTx = kPStageQKA + 16384;
+constexpr uint32_t kPColA = 0, kPColW = 64, kPColU = 192, kPTmemCols = 256;
+
+// element (r, s) of the three Tb tiles, four consecutive s at once (s % 4 == 0)
+__device__ __forceinline__ void put_tb4(uint8_t *tb16, uint8_t *tbh, uint8_t *tbl, int r, int s, float a, float b,
+                                        float c, float d) {
+    const uint32_t off = sw128_off16(r, s, 8192);
+    *reinterpret_cast<uint2 *>(tb16 + off) = make_uint2(f32x2_to_f16x2(a, b), f32x2_to_f16x2(c, d));
+    const uint32_t h0 = bf16x2_rn(a, b), h1 = bf16x2_rn(c, d);
+    *reinterpret_cast<uint2 *>(tbh + off) = make_uint2(h0, h1);
+    const float2 fa = lad::dev::bf16x2_to_f32(h0), fc = lad::dev::bf16x2_to_f32(h1);
+    *reinterpret_cast<uint2 *>(tbl + off) = make_uint2(bf16x2_rn(a - fa.x, b - fa.y), bf16x2_rn(c - fc.x, d - fc.y));
+}
+
+__device__ __forceinline__ void put_tb1(uint8_t *tb16, uint8_t *tbh, uint8_t *tbl, int r, int s, float a) {
+    const uint32_t off = sw128_off16(r, s, 8192);
+    *reinterpret_cast<__half *>(tb16 + off) = __float2half_rn(a);
+    const __nv_bfloat16 h = __float2bfloat16_rn(a);
+    *reinterpret_cast<__nv_bfloat16 *>(tbh + off) = h;
+    *reinterpret_cast<__nv_bfloat16 *>(tbl + off) = __float2bfloat16_rn(a - __bfloat162float(h));
+}
+
+// T = (I + A)^-1 for A strictly lower triangular [64][64] (fp32, row stride kAS), by 16x16 blocks:
+// the diagonal blocks by forward substitution (one thread per column), then M_ik = T_ii A_ik for
+// the six blocks below the diagonal (written over A), then T_ij = -sum_k M_ik T_kj one block row at
+// a time. T goes to sT; Tb = T diag(beta) to the three operand tiles as each block is final.
+// Called by all kThreads threads; contains block-wide barriers.
+__device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_beta, uint8_t *tb16, uint8_t *tbh,
+                                          uint8_t *tbl, int tid) {
+    if (tid < kC) {
+        const int i0 = 16 * (tid >> 4), c = tid & 15;
+        float t[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc = (r == c) ? 1.f : 0.f;
+#pragma unroll
+            for (int s = 0; s < r; ++s) acc = fmaf(-sA[(i0 + r) * kAS + i0 + s], t[s], acc);
+            t[r] = acc;
+        }
+        const float bc = s_beta[i0 + c];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            sT[(i0 + r) * kAS + i0 + c] = t[r];
+            put_tb1(tb16, tbh, tbl, i0 + r, i0 + c, t[r] * bc);
+        }
+    } else {
+        // zero the six blocks above the diagonal of the three tiles: 6 blocks x 16 rows x 2 chunks
+        for (int e = tid - kC; e < 6 * 32; e += kThreads - kC) {
+            const int blk = e >> 5, rr = (e >> 1) & 15, hf = e & 1;
+            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+            const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            const uint32_t off = sw128_off16(16 * bi + rr, 16 * bj + 8 * hf, 8192);
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(tb16 + off) = z;
+            *reinterpret_cast<uint4 *>(tbh + off) = z;
+            *reinterpret_cast<uint4 *>(tbl + off) = z;
+        }
+    }
+    __syncthreads();
+    {
+        // M_ik for (i, k) = (1,0), (2,0), (2,1), (3,0), (3,1), (3,2): 6 blocks x 64 strips of 1x4
+        float4 m[2];
+        int mi[2], mk[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int e = tid + h * kThreads;
+            m[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+            mi[h] = -1;
+            mk[h] = 0;
+            if (e < 6 * 64) {
+                const int blk = e >> 6, rr = (e >> 2) & 15, cc = (e & 3) * 4;
+                const int i = blk == 0 ? 1 : (blk < 3 ? 2 : 3);
+                const int k = blk == 0 ? 0 : (blk < 3 ? blk - 1 : blk - 3);
+                mi[h] = i;
+                mk[h] = k;
+#pragma unroll
+                for (int ss = 0; ss < 16; ++ss) {
+                    const float tv = sT[(16 * i + rr) * kAS + 16 * i + ss];
+                    const float4 a4 = *reinterpret_cast<const float4 *>(sA + (16 * i + ss) * kAS + 16 * k + cc);
+                    m[h].x = fmaf(tv, a4.x, m[h].x);
+                    m[h].y = fmaf(tv, a4.y, m[h].y);
+                    m[h].z = fmaf(tv, a4.z, m[h].z);
+                    m[h].w = fmaf(tv, a4.w, m[h].w);
+                }
+            }
+        }
+        __syncthreads();  // every read of A is done: the M blocks replace it
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int e = tid + h * kThreads;
+            if (mi[h] >= 0) {
+                const int rr = (e >> 2) & 15, cc = (e & 3) * 4;
+                *reinterpret_cast<float4 *>(sA + (16 * mi[h] + rr) * kAS + 16 * mk[h] + cc) = m[h];
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll 1
+    for (int bi = 1; bi < 4; ++bi) {
+        if (tid < bi * 64) {
+            const int bj = tid >> 6, rr = (tid >> 2) & 15, cc = (tid & 3) * 4;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int kb = bj; kb < bi; ++kb) {
+#pragma unroll
+                for (int ss = 0; ss < 16; ++ss) {
+                    const float a = sA[(16 * bi + rr) * kAS + 16 * kb + ss];
+                    const float4 t4 = *reinterpret_cast<const float4 *>(sT + (16 * kb + ss) * kAS + 16 * bj + cc);
+                    acc.x = fmaf(a, t4.x, acc.x);
+                    acc.y = fmaf(a, t4.y, acc.y);
+                    acc.z = fmaf(a, t4.z, acc.z);
+                    acc.w = fmaf(a, t4.w, acc.w);
+                }
+            }
+            const int r = 16 * bi + rr, c = 16 * bj + cc;
+            *reinterpret_cast<float4 *>(sT + r * kAS + c) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+            put_tb4(tb16, tbh, tbl, r, c, -acc.x * s_beta[c], -acc.y * s_beta[c + 1], -acc.z * s_beta[c + 2],
+                    -acc.w * s_beta[c + 3]);
+        }
+        __syncthreads();
+    }
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
 
 // Bulk copy shared -> global by one thread, in the thread's current bulk group; both addresses
 // 16-byte aligned, bytes a multiple of 16. The shared source must not change until
@@ -672,95 +834,86 @@ __device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {  // all but the newest N groups have read their source
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// One CTA per SM walks the segment's (sequence, head, chunk) items; the next item's raw inputs are
-// staged (alpha once Kh^T has been written out, q, k, v once the second MMA batch is complete).
-__global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs p,
-                                                                      const __grid_constant__ Maps maps) {
+// One CTA per SM walks the segment's (sequence, head, chunk) items. The next item's q, k and alpha
+// are staged (TMA) once the current item's operand tiles are formed, its v once the current
+// item's last MMAs (which read v) are complete; the record leaves by one bulk store (tiles) and
+// direct stores (U').
+__global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p, const __grid_constant__ PrepMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
-    float *s_beta = reinterpret_cast<float *>(sm + kPMisc + kMiscBeta);
-    float *s_rq = reinterpret_cast<float *>(sm + kPMisc + kMiscRq);
-    float *s_rk = reinterpret_cast<float *>(sm + kPMisc + kMiscRk);
-    float *s_gc = reinterpret_cast<float *>(sm + kPMisc + kMiscGc);
-    float *s_oct = reinterpret_cast<float *>(sm + kPMisc + kMiscOct);
-    const uint32_t bar = sbase + kPMisc + kMiscBar;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kPMisc + kMiscTmem);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kPMisc + kMiscAbort);
-    const uint32_t tma_bar = sbase + kPMisc + kMiscTmaBar;
-    float *Apl = reinterpret_cast<float *>(sm + kPKH);
-    float *Tpl = reinterpret_cast<float *>(sm + kPKH + 64 * 64 * 4);
+    float *s_beta = reinterpret_cast<float *>(sm + kPMisc + kPmBeta);
+    float *s_rq = reinterpret_cast<float *>(sm + kPMisc + kPmRq);
+    float *s_rk = reinterpret_cast<float *>(sm + kPMisc + kPmRk);
+    float *s_oct = reinterpret_cast<float *>(sm + kPMisc + kPmOct);
+    float *s_g = reinterpret_cast<float *>(sm + kPG);
+    float *sA = reinterpret_cast<float *>(sm + kPA);
+    float *sT = reinterpret_cast<float *>(sm + kPT);
+    const uint32_t stage_bar = sbase + kPMisc + kPmBar;
+    const uint32_t mma_bar = stage_bar + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kPMisc + kPmTmem);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kPMisc + kPmAbort);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int sp = warp & 3, cg = warp >> 2;
     const uint32_t lane_base = static_cast<uint32_t>(32 * sp) << 16;
-    const int row128 = 32 * sp + lane;
-    const int row64 = 16 * sp + lane;
-    const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);
     const int nitems = p.B * p.H * p.nseg;
 
     if (tid == 0) {
-        mbar_init(bar, 1);
-        mbar_init(tma_bar, 1);
+        mbar_init(stage_bar, 1);
+        mbar_init(mma_bar, 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kPTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    uint32_t phase = 0, tma_phase = 0;
+    uint32_t stage_phase = 0, mma_phase = 0;
     bool ok = true;
 
-    auto mma_sync = [&](auto &&issue) {
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (warp == 0) {
-            tc_fence_after();
-            issue();
-            tc_commit(bar);
-        }
-        const bool w = wait_bar(bar, phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
-        phase ^= 1;
-        tc_fence_after();
-        return __syncthreads_and(w) != 0;
-    };
-    // item -> (b, h, chunk); items of one (b, h) are consecutive
+    // item -> (b, h, chunk); the items of one (b, h) are consecutive
     auto coords = [&](int item, int &b, int &h, int &ch) {
         const int bh = item / p.nseg;
         ch = p.c0 + (item - bh * p.nseg);
         b = bh / p.H;
         h = bh - b * p.H;
     };
-    auto stage_alpha = [&](int item) {
+    auto stage_qka = [&](int item) {
         int b, h, ch;
         coords(item, b, h, ch);
         fence_async_smem();
-        mbar_arrive_tx_raw(tma_bar, kPStageTx);
-        tma_load_3d(sbase + kPStA, &maps.alpha, h * kDk, ch * kC, b, tma_bar);
+        mbar_arrive_tx_raw(stage_bar, kPStageTx);
+        tma_load_3d(sbase + kPSQ, &maps.q, h * kDk, ch * kC, b, stage_bar);
+        tma_load_3d(sbase + kPSK, &maps.k, h * kDk, ch * kC, b, stage_bar);
+        tma_load_3d(sbase + kPSA, &maps.alpha, h * kDk, ch * kC, b, stage_bar);
     };
-    auto stage_qkv = [&](int item) {
+    auto stage_v = [&](int item) {
         int b, h, ch;
         coords(item, b, h, ch);
         fence_async_smem();
-        tma_load_3d(sbase + kPStQ, &maps.q, h * kDk, ch * kC, b, tma_bar);
-        tma_load_3d(sbase + kPStK, &maps.k, h * kDk, ch * kC, b, tma_bar);
-        tma_load_3d(sbase + kPStV, &maps.v, h * kDv, ch * kC, b, tma_bar);
+        tma_load_3d(sbase + kPV, &maps.v, h * kDv, ch * kC, b, stage_bar);
+        tma_load_3d(sbase + kPV + 8192, &maps.v, h * kDv + 64, ch * kC, b, stage_bar);
     };
-    int pending = 0, qkv_owed = -1;
+    auto mma_wait = [&]() {
+        const bool w = wait_bar(mma_bar, mma_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
+        mma_phase ^= 1;
+        tc_fence_after();
+        return __syncthreads_and(w) != 0;
+    };
+    const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);  // K-major SW128 at offset 0
+
+    int pending = 0;   // a staging phase is in flight
+    int v_owed = -1;   // an item whose q, k and alpha are staged but whose v is not yet
     int item = blockIdx.x;
     if (item < nitems) {
         if (tid == 0) {
-            stage_alpha(item);
-            stage_qkv(item);
+            stage_qka(item);
+            stage_v(item);
         }
         pending = 1;
     }
@@ -771,21 +924,21 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
         const int t0 = ch * kC;
         const int n = min(kC, p.T - t0);
         const size_t tok0 = (static_cast<size_t>(b) * p.T + t0) * p.H + h;
-        const size_t tstride = static_cast<size_t>(p.H);
-        uint8_t *rec = p.ws + static_cast<size_t>(item) * kItemBytes;
+        uint8_t *rec = p.ws + static_cast<size_t>(item) * kRecBytes;
 
-        if (tid < kC) s_beta[tid] = (tid < n) ? p.beta[tok0 + tid * tstride] : 0.f;
-        if (tid == 0) bulk_wait_read<0>();  // the previous item's W and U' have left [Qt; Kt]
+        if (tid < kC) s_beta[tid] = (tid < n) ? p.beta[tok0 + static_cast<size_t>(tid) * p.H] : 0.f;
+        if (tid == 0) bulk_wait_read0();  // the previous item's tiles have left for its record
         {
-            const bool w = wait_bar(tma_bar, tma_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
-            tma_phase ^= 1;
+            const bool w = wait_bar(stage_bar, stage_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            stage_phase ^= 1;
             pending = 0;
             ok = __syncthreads_and(w) != 0;
             if (!ok) break;
         }
+        const uint16_t *sq = reinterpret_cast<const uint16_t *>(sm + kPSQ);
+        const uint16_t *sk = reinterpret_cast<const uint16_t *>(sm + kPSK);
+        const float *sa = reinterpret_cast<const float *>(sm + kPSA);
         if (p.l2norm) {
-            const uint16_t *sq = reinterpret_cast<const uint16_t *>(sm + kPStQ);
-            const uint16_t *sk = reinterpret_cast<const uint16_t *>(sm + kPStK);
 #pragma unroll 1
             for (int r = warp; r < kC; r += kThreads / 32) {
                 const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + 4 * lane);
@@ -808,14 +961,11 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
             s_rq[tid] = 1.f;
             s_rk[tid] = 1.f;
         }
-        __syncthreads();
 
-        // ---- running decay and the operand tiles (warp w: tokens 8w..8w+7; lane l: channels 4l..) ----
+        // ---- running decay and the operand tiles: warp w takes tokens 8w .. 8w+7, lane l the key
+        //      channels 4l .. 4l+3; the products over earlier token octets come through shared memory ----
         {
             const int o = warp, c4 = 4 * lane;
-            const float *sa = reinterpret_cast<const float *>(sm + kPStA);
-            const uint16_t *sq = reinterpret_cast<const uint16_t *>(sm + kPStQ);
-            const uint16_t *sk = reinterpret_cast<const uint16_t *>(sm + kPStK);
             float4 gl[8];
             float4 run = make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
@@ -831,21 +981,27 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
             }
             *reinterpret_cast<float4 *>(s_oct + o * kDk + c4) = run;
             __syncthreads();
-            float4 excl = make_float4(1.f, 1.f, 1.f, 1.f);
-            for (int oo = 0; oo < o; ++oo) {
+            float4 excl = make_float4(1.f, 1.f, 1.f, 1.f), all = excl;  // before octet o; all octets
+#pragma unroll
+            for (int oo = 0; oo < kThreads / 32; ++oo) {
                 const float4 y = *reinterpret_cast<const float4 *>(s_oct + oo * kDk + c4);
-                excl.x *= y.x;
-                excl.y *= y.y;
-                excl.z *= y.z;
-                excl.w *= y.w;
+                if (oo < o) {
+                    excl.x *= y.x;
+                    excl.y *= y.y;
+                    excl.z *= y.z;
+                    excl.w *= y.w;
+                }
+                all.x *= y.x;
+                all.y *= y.y;
+                all.z *= y.z;
+                all.w *= y.w;
             }
-            if (o == kThreads / 32 - 1)
-                *reinterpret_cast<float4 *>(s_gc + c4) =
-                    make_float4(excl.x * run.x, excl.y * run.y, excl.z * run.z, excl.w * run.w);
+            if (o == 0) *reinterpret_cast<float4 *>(s_g + c4) = all;  // g_last, for the record
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int r = 8 * o + u;
-                const float gg[4] = {excl.x * gl[u].x, excl.y * gl[u].y, excl.z * gl[u].z, excl.w * gl[u].w};
+                const float g[4] = {excl.x * gl[u].x, excl.y * gl[u].y, excl.z * gl[u].z, excl.w * gl[u].w};
+                const float ga[4] = {all.x, all.y, all.z, all.w};
                 const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + c4);
                 const uint2 kw = *reinterpret_cast<const uint2 *>(sk + r * kDk + c4);
                 const float2 q0 = lad::dev::bf16x2_to_f32(qw.x), q1 = lad::dev::bf16x2_to_f32(qw.y);
@@ -853,420 +1009,402 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_prep_kernel(SplitArgs
                 const float rq = s_rq[r], rk = s_rk[r];
                 const float qv[4] = {q0.x * rq, q0.y * rq, q1.x * rq, q1.y * rq};
                 const float kv[4] = {k0.x * rk, k0.y * rk, k1.x * rk, k1.y * rk};
-                st_tile4(sm + kPXQK, r, c4, kStr16, qv[0] * gg[0], qv[1] * gg[1], qv[2] * gg[2], qv[3] * gg[3]);
-                st_tile4(sm + kPXQK, kC + r, c4, kStr16, kv[0] * gg[0], kv[1] * gg[1], kv[2] * gg[2], kv[3] * gg[3]);
-                st_tile4(sm + kPKH, r, c4, kStr8, __fdividef(kv[0], gg[0]), __fdividef(kv[1], gg[1]),
-                         __fdividef(kv[2], gg[2]), __fdividef(kv[3], gg[3]));
+                float kh[4], kg[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    kh[e] = __fdividef(kv[e], g[e]);
+                    kg[e] = kh[e] * ga[e];
+                }
+                const uint32_t off = sw128_off16(r, c4, 8192);                 // 64-row tiles (Kh, Kg)
+                const uint32_t offq = sw128_off16(kC + r, c4, 16384);          // row 64 + r of [Kt; Qt]
+                const uint32_t offk = sw128_off16(r, c4, 16384);               // row r of [Kt; Qt]
+                *reinterpret_cast<uint2 *>(sm + kPQW + offk) =
+                    make_uint2(f32x2_to_f16x2(kv[0] * g[0], kv[1] * g[1]), f32x2_to_f16x2(kv[2] * g[2], kv[3] * g[3]));
+                *reinterpret_cast<uint2 *>(sm + kPQW + offq) =
+                    make_uint2(f32x2_to_f16x2(qv[0] * g[0], qv[1] * g[1]), f32x2_to_f16x2(qv[2] * g[2], qv[3] * g[3]));
+                *reinterpret_cast<uint2 *>(sm + kPKH + off) =
+                    make_uint2(f32x2_to_f16x2(kh[0], kh[1]), f32x2_to_f16x2(kh[2], kh[3]));
+                *reinterpret_cast<uint2 *>(sm + kPKG + off) =
+                    make_uint2(f32x2_to_f16x2(kg[0], kg[1]), f32x2_to_f16x2(kg[2], kg[3]));
             }
-            // V^T [128 d_v][64 tok]: thread -> value column j = tid % 128, tokens 32 * (tid / 128) .. + 31
-            const uint16_t *sv = reinterpret_cast<const uint16_t *>(sm + kPStV);
-            const int j = tid & 127, r0 = 32 * (tid >> 7);
-#pragma unroll 2
-            for (int r = 0; r < 32; r += 4)
-                st_tile4(sm + kPVT, j, r0 + r, kStr16, bf16_to_f32(sv[(r0 + r) * kDv + j]),
-                         bf16_to_f32(sv[(r0 + r + 1) * kDv + j]), bf16_to_f32(sv[(r0 + r + 2) * kDv + j]),
-                         bf16_to_f32(sv[(r0 + r + 3) * kDv + j]));
         }
-        // ---- MMA 1: [Qt; Kt] Kh^T, issued now; the transposes below only read its operands ----
+        // ---- [Kt; Qt] Kh^T: rows 0-63 give Kt Kh^T, rows 64-127 Qt Kh^T ----
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();  // the staging area is read: Kh^T and Kt^T go over it
+        __syncthreads();  // q, k and alpha of this item are read: the next item's come in
+        if (next < nitems) {
+            if (tid == 0) stage_qka(next);
+            pending = 1;
+            v_owed = next;
+        }
         if (warp == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int j = 0; j < kDk / 8; ++j)
-                tc_mma_tf32(tmem + kPColAcc1, kdesc(d0 + (kPXQK >> 4), kStr16, j), kdesc(d0 + (kPKH >> 4), kStr8, j),
-                            kIdesc128, j > 0);
-            tc_commit(bar);
+            for (int j = 0; j < kDk / 16; ++j)
+                tc_mma_f16(tmem + kPColA, kdesc16(d0 + (kPQW >> 4), 16384, j), kdesc16(d0 + (kPKH >> 4), 8192, j),
+                           kIdescA, j > 0);
+            tc_commit(mma_bar);
         }
-        {
-            // Kh^T from Kh, Kt^T from the Kt rows of [Qt; Kt]: thread -> channel i, tokens of half th
-            const int i = tid & (kDk - 1), th = tid >> 7;
-#pragma unroll 2
-            for (int r = (kC / 2) * th; r < (kC / 2) * (th + 1); r += 4) {
-                float kh[4], kt[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    kh[u] = *reinterpret_cast<const float *>(sm + kPKH + sw128_off32(r + u, i, kStr8));
-                    kt[u] = *reinterpret_cast<const float *>(sm + kPXQK + sw128_off32(kC + r + u, i, kStr16));
-                }
-                st_tile4(sm + kPKHT, i, r, kStr16, kh[0], kh[1], kh[2], kh[3]);
-                st_tile4(sm + kPKTT, i, r, kStr16, kt[0], kt[1], kt[2], kt[3]);
-            }
-        }
-        fence_async_smem();  // the transposes are read by the bulk store below
-        {
-            const bool w = wait_bar(bar, phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
-            phase ^= 1;
-            tc_fence_after();
-            ok = __syncthreads_and(w) != 0;
-            if (!ok) break;
-        }
-        // Kh^T, Qt and g_last are final: out to the record by bulk stores (group 1)
-        if (tid == 0) {
-            bulk_s2g(rec + kItKHT, sbase + kPKHT, 32768);
-#pragma unroll
-            for (int blk = 0; blk < 4; ++blk) bulk_s2g(rec + kItQ + blk * 8192, sbase + kPXQK + blk * kStr16, 8192);
-            bulk_s2g(rec + kItG, smem_u32(s_gc), 512);
-            bulk_commit();
-        }
-        // ---- lower(Qt Kh^T) -> P tile (rows 0-63); A = strict_lower(diag(beta) Kt Kh^T) -> scratch ----
+        ok = mma_wait();
+        if (!ok) break;
+        // ---- A = strict_lower(diag(beta) Kt Kh^T) -> fp32 scratch; P = lower(Qt Kh^T) -> fp16 tile ----
         {
             float x[32];
-            tmem_ld32(tmem + lane_base + kPColAcc1 + 32 * cg, x);
+            tmem_ld32(tmem + lane_base + kPColA + 32 * cg, x);
             tmem_wait_ld();
-            const int c0 = 32 * cg;
-            if (row128 < kC) {
-                const int r = row128;
-#pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    st_tile4(sm + kPP, r, c0 + j, kStr8, c0 + j <= r ? x[j] : 0.f, c0 + j + 1 <= r ? x[j + 1] : 0.f,
-                             c0 + j + 2 <= r ? x[j + 2] : 0.f, c0 + j + 3 <= r ? x[j + 3] : 0.f);
-            } else {
-                const int r = row128 - kC;
+            const int row = 32 * sp + lane, c0 = 32 * cg;
+            if (row < kC) {
+                const int r = row;
                 const float br = s_beta[r];
-                float4 *dst = reinterpret_cast<float4 *>(Apl + r * 64 + c0);
+                float4 *dst = reinterpret_cast<float4 *>(sA + r * kAS + c0);
 #pragma unroll
                 for (int j = 0; j < 32; j += 4)
                     dst[j / 4] = make_float4(c0 + j < r ? br * x[j] : 0.f, c0 + j + 1 < r ? br * x[j + 1] : 0.f,
                                              c0 + j + 2 < r ? br * x[j + 2] : 0.f, c0 + j + 3 < r ? br * x[j + 3] : 0.f);
-            }
-        }
-        fence_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            bulk_s2g(rec + kItP, sbase + kPP, 16384);  // group 2
-            bulk_commit();
-            bulk_wait_read<1>();  // group 1 has read Kh^T: the next item's alpha can come in over it
-        }
-        if (next < nitems) {
-            if (tid == 0) stage_alpha(next);
-            pending = 1;
-            qkv_owed = next;
-        }
-        // ---- T = (I + A)^-1, Tb -> operand ----
-        solve_tb(Apl, Tpl, s_beta, sm + kPTT, tid);
-        // ---- MMA 2: W = Tb Kt (B = Kt^T), U' = Tb V (B = V^T) ----
-        ok = mma_sync([&] {
+            } else {
+                const int r = row - kC;
 #pragma unroll
-            for (int j = 0; j < kC / 8; ++j) {
-                const uint64_t tt = kdesc(d0 + (kPTT >> 4), kStr16, j);
-                tc_mma_tf32(tmem + kPColW, tt, kdesc(d0 + (kPKTT >> 4), kStr16, j), kIdesc64x128, j > 0);
-                tc_mma_tf32(tmem + kPColU, tt, kdesc(d0 + (kPVT >> 4), kStr16, j), kIdesc64x128, j > 0);
-            }
-        });
-        if (!ok) break;
-        if (tid == 0) bulk_wait_read<0>();  // P (and Qt) read out: the staging area and XQK are free
-        if (qkv_owed >= 0) {  // Kt^T and P are done with: q, k, v of the next item
-            if (tid == 0) stage_qkv(qkv_owed);
-            qkv_owed = -1;
-        }
-        __syncthreads();
-        // ---- W (tf32-rounded operand layout) and U' (plain fp32, per d_v half) -> shared memory over
-        //      [Qt; Kt], then -> record by one bulk store (group 3) ----
-        {
-            float *ush = reinterpret_cast<float *>(sm + kPXQK + 32768);  // U' [2 halves][64 tok][64]
-#pragma unroll 1
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 32 * cg + 64 * part;  // columns c0 .. c0 + 31
-                float w[32], u[32];
-                tmem_ld32(tmem + lane_base + kPColW + c0, w);
-                tmem_ld32(tmem + lane_base + kPColU + c0, u);
-                tmem_wait_ld();
-                if (lane < 16) {
+                for (int j = 0; j < 32; j += 8) {
+                    float y[8];
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        st_tile4(sm + kPXQK, row64, c0 + j, kStr8, w[j], w[j + 1], w[j + 2], w[j + 3]);
-                        const int hv = c0 >> 6, cc = (c0 & 63) + j;
-                        *reinterpret_cast<float4 *>(ush + (hv * 64 + row64) * 64 + cc) =
-                            make_float4(u[j], u[j + 1], u[j + 2], u[j + 3]);
-                    }
+                    for (int e = 0; e < 8; ++e) y[e] = (c0 + j + e <= r) ? x[j + e] : 0.f;
+                    *reinterpret_cast<uint4 *>(sm + kPP + sw128_off16(r, c0 + j, 8192)) =
+                        make_uint4(f32x2_to_f16x2(y[0], y[1]), f32x2_to_f16x2(y[2], y[3]), f32x2_to_f16x2(y[4], y[5]),
+                                   f32x2_to_f16x2(y[6], y[7]));
                 }
             }
         }
-        fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0) {
-            bulk_s2g(rec + kItW, sbase + kPXQK, 32768);
-            bulk_s2g(rec + kItU, sbase + kPXQK + 32768, 32768);
-            bulk_commit();
-        }
-    }
-    if (tid == 0 && qkv_owed >= 0) stage_qkv(qkv_owed);
-    if (tid == 0 && pending) {
-        const uint64_t t0 = lad::dev::globaltimer_ns();
-        while (!mbar_try_wait(tma_bar, tma_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
-        }
-    }
-    if (tid == 0) bulk_wait_all();  // every record write has landed
-    if (warp == 0) {
-        tc_commit(bar);
-        const uint64_t t0 = lad::dev::globaltimer_ns();
-        while (!mbar_try_wait(bar, phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
-}
-
-// scan shared memory: W and Qt (single buffer), then two buffers of Kh^T, P and g_last (the
-// second batch's operands arrive a whole chunk ahead), S0^T, U^T; U' goes straight to registers
-constexpr uint32_t kSW = 0, kSQ = 32768;
-constexpr uint32_t kSKP0 = 65536, kSKPBytes = 50176;  // a buffer: Kh^T 32 KiB, P 16 KiB, g_last 512 B (+pad)
-constexpr uint32_t kSKHT = 0, kSP = 32768, kSG = 49152;  // offsets inside a buffer
-constexpr uint32_t kSSOT = kSKP0 + 2 * kSKPBytes;   // 165,888: S0^T [64 d_v][128 d_k], stride 8 KiB
-constexpr uint32_t kSUT = kSSOT + 32768;            // U^T [64 d_v][64 tok], stride 8 KiB
-constexpr uint32_t kSMisc = kSUT + 16384;           // bars, tmem slot, abort flag
-constexpr uint32_t kSSmemBytes = kSMisc + 2048 + 1024;
-constexpr uint32_t kSBar1Tx = 65536;                // W, Qt
-constexpr uint32_t kSBar2Tx = 32768 + 16384 + 512;  // Kh^T, P, g_last
-constexpr uint32_t kSColX = 0, kSColO = 64, kSColS = 128;
-constexpr uint32_t kSTmemCols = 256;
-
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-
-// One CTA per (sequence, head, half of d_v) walks the segment's chunks with the state in TMEM.
-__global__ void __launch_bounds__(kThreads, 1) kda_prefill_scan_kernel(SplitArgs p) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t sbase = smem_u32(sm);
-    const uint32_t bar = sbase + kSMisc;
-    const uint32_t bar1 = sbase + kSMisc + 8;
-    auto bar2 = [&](int j) { return sbase + kSMisc + 16 + 8u * static_cast<uint32_t>(j); };  // per buffer
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kSMisc + 32);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kSMisc + 36);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int sp = warp & 3, cg = warp >> 2;
-    const uint32_t lane_base = static_cast<uint32_t>(32 * sp) << 16;
-    const int row128 = 32 * sp + lane;
-    const int row64 = 16 * sp + lane;
-    const int half = blockIdx.x & 1;
-    const int bh = blockIdx.x >> 1;
-    const int b = bh / p.H, h = bh - b * p.H;
-    const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);
-    const uint8_t *recs = p.ws + static_cast<size_t>(bh) * p.nseg * kItemBytes;
-
-    if (tid == 0) {
-        mbar_init(bar, 1);
-        mbar_init(bar1, 1);
-        mbar_init(bar2(0), 1);
-        mbar_init(bar2(1), 1);
-        *abort_flag = 0;
-        mbar_fence_init();
-    }
-    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kSTmemCols);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    uint32_t phase = 0, ph1 = 0, ph2[2] = {0, 0};
-    bool ok = true;
-
-    auto mma_sync = [&](auto &&issue) {
+        // ---- T = (I + A)^-1, Tb = T diag(beta) -> the fp16 tile and its bf16 hi / lo split ----
+        solve_tb16(sA, sT, s_beta, sm + kPTB, sm + kPTBH, sm + kPTBL, tid);
+        // ---- W = Tb Kt (Kt: rows 0-63 of [Kt; Qt], read MN-major); U'^T = V^T (Tb_hi + Tb_lo)^T ----
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         if (warp == 0) {
             tc_fence_after();
-            issue();
-            tc_commit(bar);
-        }
-        const bool w = wait_bar(bar, phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
-        phase ^= 1;
-        tc_fence_after();
-        return __syncthreads_and(w) != 0;
-    };
-    auto load1 = [&](int i) {  // W, Qt of chunk i of the segment
-        const uint8_t *rec = recs + static_cast<size_t>(i) * kItemBytes;
-        fence_async_smem();
-        mbar_arrive_tx_raw(bar1, kSBar1Tx);
-        bulk_g2s(sbase + kSW, rec + kItW, 32768, bar1);
-        bulk_g2s(sbase + kSQ, rec + kItQ, 32768, bar1);
-    };
-    auto load2 = [&](int i) {  // Kh^T, P, g_last of chunk i into buffer i % 2
-        const uint8_t *rec = recs + static_cast<size_t>(i) * kItemBytes;
-        const uint32_t buf = sbase + kSKP0 + (i & 1) * kSKPBytes;
-        fence_async_smem();
-        mbar_arrive_tx_raw(bar2(i & 1), kSBar2Tx);
-        bulk_g2s(buf + kSKHT, rec + kItKHT, 32768, bar2(i & 1));
-        bulk_g2s(buf + kSP, rec + kItP, 16384, bar2(i & 1));
-        bulk_g2s(buf + kSG, rec + kItG, 512, bar2(i & 1));
-    };
-    int pend1 = 0, pend2[2] = {0, 0};
-    if (tid == 0) {
-        load1(0);
-        load2(0);
-        if (p.nseg > 1) load2(1);
-    }
-    pend1 = pend2[0] = 1;
-    pend2[1] = p.nseg > 1 ? 1 : 0;
-
-    // ---- the state entering the segment: TMEM master (row = key channel) and the S0^T operand ----
-    {
-        const float *S0 = p.S + (static_cast<size_t>(bh) * kDk + row128) * kDv + half * kDvh + 32 * cg;
-        float v[32];
+            const uint64_t kt0 = smem_desc(sbase + kPQW, 16384, 1024, kLayoutSw128);  // MN chunks 16 KiB apart
+            const uint64_t v0 = smem_desc(sbase + kPV, 8192, 1024, kLayoutSw128);     // MN chunks 8 KiB apart
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(S0 + j);
-            v[j] = x.x;
-            v[j + 1] = x.y;
-            v[j + 2] = x.z;
-            v[j + 3] = x.w;
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) st_tile1(sm + kSSOT, 32 * cg + j, row128, kStr8, v[j]);
-        tmem_st32(tmem + lane_base + kSColS + 32 * cg, v);
-        tmem_wait_st();
-    }
-
-    for (int i = 0; i < p.nseg && ok; ++i) {
-        const int ch = p.c0 + i;
-        const int t0 = ch * kC;
-        const int n = min(kC, p.T - t0);
-        const size_t tok0 = (static_cast<size_t>(b) * p.T + t0) * p.H + h;
-        const size_t tstride = static_cast<size_t>(p.H);
-        // this chunk's U' (rows of this thread, 32 of this CTA's d_v columns) straight into registers
-        float4 up[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) up[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (lane < 16) {  // rows 0-63 of the M = 64 accumulator sit in lanes 0-15
-            const float4 *src = reinterpret_cast<const float4 *>(recs + static_cast<size_t>(i) * kItemBytes + kItU +
-                                                                 half * 16384) +
-                                (row64 * 64 + 32 * cg) / 4;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) up[j] = src[j];
-        }
-        {
-            const bool w = wait_bar(bar1, ph1, abort_flag, &g_prefill_error, lad::kErrPrefill);
-            ph1 ^= 1;
-            pend1 = 0;
-            ok = __syncthreads_and(w) != 0;
-            if (!ok) break;
-        }
-        // ---- X = W S0,  O = Qt S0 ----
-        ok = mma_sync([&] {
-#pragma unroll
-            for (int j = 0; j < kDk / 8; ++j) {
-                const uint64_t sot = kdesc(d0 + (kSSOT >> 4), kStr8, j);
-                tc_mma_tf32(tmem + kSColX, kdesc(d0 + (kSW >> 4), kStr8, j), sot, kIdesc64, j > 0);
-                tc_mma_tf32(tmem + kSColO, kdesc(d0 + (kSQ >> 4), kStr8, j), sot, kIdesc64, j > 0);
+            for (int j = 0; j < kC / 16; ++j) {
+                tc_mma_f16(tmem + kPColW, kdesc16(d0 + (kPTB >> 4), 8192, j), kt0 + ((j * 2048) >> 4), kIdescW, j > 0);
+                tc_mma_f16(tmem + kPColU, v0 + ((j * 2048) >> 4), kdesc16(d0 + (kPTBH >> 4), 8192, j), kIdescU, j > 0);
             }
-        });
+#pragma unroll
+            for (int j = 0; j < kC / 16; ++j)
+                tc_mma_f16(tmem + kPColU, v0 + ((j * 2048) >> 4), kdesc16(d0 + (kPTBL >> 4), 8192, j), kIdescU, 1);
+            tc_commit(mma_bar);
+        }
+        ok = mma_wait();
         if (!ok) break;
-        if (i + 1 < p.nseg) {
-            if (tid == 0) load1(i + 1);
-            pend1 = 1;
+        if (v_owed >= 0) {  // v is read: the next item's comes in
+            if (tid == 0) stage_v(v_owed);
+            v_owed = -1;
         }
-        const int kb = i & 1;
-        const uint32_t kp = kSKP0 + static_cast<uint32_t>(kb) * kSKPBytes;
+        // ---- W -> rows 0-63 of [W; Qt] (over Kt); U' -> the record ----
         {
-            const bool w = wait_bar(bar2(kb), ph2[kb], abort_flag, &g_prefill_error, lad::kErrPrefill);
-            ph2[kb] ^= 1;
-            pend2[kb] = 0;
-            ok = __syncthreads_and(w) != 0;
-            if (!ok) break;
-        }
-        const float gc = reinterpret_cast<const float *>(sm + kp + kSG)[row128];
-        // ---- U = U' - X -> U^T operand ----
-        {
-            float x[32];
-            tmem_ld32(tmem + lane_base + kSColX + 32 * cg, x);
-            tmem_wait_ld();
-            if (lane < 16) {
+            // M = 64: row 16 sp + i sits in lane i (< 16) of sub-partition sp; the loads are
+            // collective, so the whole warp issues them and lanes 0-15 keep the rows
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    st_tile1(sm + kSUT, 32 * cg + 4 * j, row64, kStr8, up[j].x - x[4 * j]);
-                    st_tile1(sm + kSUT, 32 * cg + 4 * j + 1, row64, kStr8, up[j].y - x[4 * j + 1]);
-                    st_tile1(sm + kSUT, 32 * cg + 4 * j + 2, row64, kStr8, up[j].z - x[4 * j + 2]);
-                    st_tile1(sm + kSUT, 32 * cg + 4 * j + 3, row64, kStr8, up[j].w - x[4 * j + 3]);
-                }
-            }
-        }
-        // ---- O += P U;  S += Kh^T U ----
-        ok = mma_sync([&] {
-#pragma unroll
-            for (int j = 0; j < kC / 8; ++j) {
-                const uint64_t ut = kdesc(d0 + (kSUT >> 4), kStr8, j);
-                tc_mma_tf32(tmem + kSColO, kdesc(d0 + ((kp + kSP) >> 4), kStr8, j), ut, kIdesc64, 1);
-                tc_mma_tf32(tmem + kSColS, kdesc(d0 + ((kp + kSKHT) >> 4), kStr16, j), ut, kIdesc128, 1);
-            }
-        });
-        if (!ok) break;
-        if (i + 2 < p.nseg) {  // this buffer is free again: chunk i + 2's operands
-            if (tid == 0) load2(i + 2);
-            pend2[kb] = 1;
-        }
-        // ---- O -> HBM; S <- Diag(g_last) S, S^T -> operand (HBM after the segment's last chunk) ----
-        {
-            float ov[32];
-            tmem_ld32(tmem + lane_base + kSColO + 32 * cg, ov);
-            tmem_wait_ld();
-            if (lane < 16 && row64 < n) {
-                const size_t orow = (tok0 + row64 * tstride) * kDv + half * kDvh + 32 * cg;
-                if (p.out_f32) {
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow);
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        dst[j / 4] = make_float4(p.scale * ov[j], p.scale * ov[j + 1], p.scale * ov[j + 2],
-                                                 p.scale * ov[j + 3]);
-                } else {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) + orow);
+            for (int part = 0; part < 2; ++part) {
+                const int c0 = 64 * cg + 32 * part;
+                float w[32];
+                tmem_ld32(tmem + lane_base + kPColW + c0, w);
+                tmem_wait_ld();
+                if (lane < 16) {
+                    const int r = 16 * sp + lane;
 #pragma unroll
                     for (int j = 0; j < 32; j += 8)
-                        dst[j / 8] = make_uint4(lad::dev::f32x2_to_bf16x2(p.scale * ov[j], p.scale * ov[j + 1]),
-                                                lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 2], p.scale * ov[j + 3]),
-                                                lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 4], p.scale * ov[j + 5]),
-                                                lad::dev::f32x2_to_bf16x2(p.scale * ov[j + 6], p.scale * ov[j + 7]));
+                        *reinterpret_cast<uint4 *>(sm + kPQW + sw128_off16(r, c0 + j, 16384)) =
+                            make_uint4(f32x2_to_f16x2(w[j], w[j + 1]), f32x2_to_f16x2(w[j + 2], w[j + 3]),
+                                       f32x2_to_f16x2(w[j + 4], w[j + 5]), f32x2_to_f16x2(w[j + 6], w[j + 7]));
                 }
             }
-            float sv[32];
-            tmem_ld32(tmem + lane_base + kSColS + 32 * cg, sv);
+            float u[32];
+            tmem_ld32(tmem + lane_base + kPColU + 32 * cg, u);
             tmem_wait_ld();
+            float *up = reinterpret_cast<float *>(rec + kRUP) + 32 * sp + lane;  // column d_v
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                sv[j] *= gc;
-                st_tile1(sm + kSSOT, 32 * cg + j, row128, kStr8, sv[j]);
-            }
-            tmem_st32(tmem + lane_base + kSColS + 32 * cg, sv);
-            if (i == p.nseg - 1) {
-                float *Sout = p.S + (static_cast<size_t>(bh) * kDk + row128) * kDv + half * kDvh + 32 * cg;
-#pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4 *>(Sout + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
-            }
-            tmem_wait_st();
+            for (int j = 0; j < 32; ++j) up[(32 * cg + j) * kDv] = u[j];
         }
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
-    }
-    // drain: copies still in flight (after an abort) land, MMAs complete, before release
-    if (tid == 0) {
-        const uint64_t t0 = lad::dev::globaltimer_ns();
-        while (pend1 && !mbar_try_wait(bar1, ph1) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+        if (tid == 0) {
+            bulk_s2g(rec, sbase + kPQW, kRTiles);
+            bulk_commit();
         }
-        for (int j = 0; j < 2; ++j)
-            while (pend2[j] && !mbar_try_wait(bar2(j), ph2[j]) &&
-                   lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
-            }
     }
-    if (warp == 0) {
-        tc_commit(bar);
+    // drain: a staging copy still in flight (after an abort) lands, the record stores complete and
+    // every MMA this CTA issued completes, before shared memory and TMEM are released
+    if (tid == 0 && v_owed >= 0) stage_v(v_owed);  // the staging phase expects those bytes too
+    if (tid == 0 && pending) {
         const uint64_t t0 = lad::dev::globaltimer_ns();
-        while (!mbar_try_wait(bar, phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+        while (!mbar_try_wait(stage_bar, stage_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+        }
+    }
+    if (tid == 0) bulk_wait_all();
+    if (warp == 0) {
+        tc_commit(mma_bar);
+        const uint64_t t0 = lad::dev::globaltimer_ns();
+        while (!mbar_try_wait(mma_bar, mma_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, kSTmemCols);
+    if (warp == 0) tmem_dealloc(tmem, kPTmemCols);
+}
+
+struct ChainArgs {
+    float *S;
+    void *o;
+    const uint8_t *ws;  // this segment's records, [B*H][nseg]
+    int B, T, H;
+    int c0, nseg;
+    float scale;
+    int out_f32;
+};
+
+// chain shared memory (offsets from a 1024-aligned base)
+constexpr uint32_t kCS16 = 0;            // S^T [128 d_v][128 d_k] fp16, K-major SW128, 2 blocks x 16 KiB
+constexpr uint32_t kCU16 = 32768;        // U^T [128 d_v][64 tok] fp16, K-major SW128, 16 KiB
+constexpr uint32_t kCRec = 49152;        // two record buffers (the tiles and g_last of a chunk)
+constexpr uint32_t kCRecStride = 58368;  // 57 KiB each (1024-aligned)
+constexpr uint32_t kCMisc = kCRec + 2 * kCRecStride;
+constexpr uint32_t kCSmemBytes = kCMisc + 64 + 1024;
+// TMEM: the fp32 master S^T (128 lanes = d_v, 128 columns = d_k) and two [X^T | O^T] buffers
+constexpr uint32_t kCColS = 0, kCColXO = 128, kCTmemCols = 512;
+
+// One CTA per (sequence, head) walks the segment's chunks with the state master in tensor memory.
+__global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    const uint32_t rec_bar0 = sbase + kCMisc, mma_bar = sbase + kCMisc + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kCMisc + 24);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kCMisc + 28);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int sp = warp & 3, cg = warp >> 2;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * sp) << 16;
+    const int dv = 32 * sp + lane;  // this thread's row of S^T: a value column
+    const int bh = blockIdx.x;
+    const int b = bh / p.H, h = bh - b * p.H;
+    const uint8_t *recs = p.ws + static_cast<size_t>(bh) * p.nseg * kRecBytes;
+    const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);
+
+    if (tid == 0) {
+        mbar_init(rec_bar0, 1);
+        mbar_init(rec_bar0 + 8, 1);
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kCTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto load_rec = [&](int i) {  // chunk i's tiles into buffer i % 2
+        const uint32_t bar = rec_bar0 + 8u * static_cast<uint32_t>(i & 1);
+        mbar_arrive_tx_raw(bar, kRTiles);
+        bulk_g2s(sbase + kCRec + static_cast<uint32_t>(i & 1) * kCRecStride, recs + static_cast<size_t>(i) * kRecBytes,
+                 kRTiles, bar);
+    };
+    uint32_t pend = p.nseg > 1 ? 3u : 1u;  // bit j: a copy into buffer j is in flight
+    if (tid == 0) {
+        load_rec(0);
+        if (p.nseg > 1) load_rec(1);
+    }
+
+    // U' of chunk i for this thread's value column and tokens 32 cg .. 32 cg + 31
+    auto load_up = [&](float (&u)[32], int i) {
+        const float *src = reinterpret_cast<const float *>(recs + static_cast<size_t>(i) * kRecBytes + kRUP) + dv;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) u[j] = __ldcg(src + (32 * cg + j) * kDv);
+    };
+    // the outputs of chunk i (O^T in buffer i % 2, columns 64-127), scaled
+    auto store_o = [&](int i) {
+        float x[32];
+        tmem_ld32(tmem + lane_base + kCColXO + static_cast<uint32_t>(i & 1) * 128 + 64 + 32 * cg, x);
+        tmem_wait_ld();
+        const int t0 = (p.c0 + i) * kC;
+        const int n = min(kC, p.T - t0);
+        const size_t row0 = (static_cast<size_t>(b) * p.T + t0) * p.H + h;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int t = 32 * cg + j;
+            if (t < n) {
+                const size_t at = (row0 + static_cast<size_t>(t) * p.H) * kDv + dv;
+                if (p.out_f32)
+                    static_cast<float *>(p.o)[at] = p.scale * x[j];
+                else
+                    static_cast<uint16_t *>(p.o)[at] = lad::dev::f32_to_bf16(p.scale * x[j]);
+            }
+        }
+    };
+
+    // ---- the state entering the segment: master S^T and its fp16 copy ----
+    {
+        const float *S0 = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int c0 = 64 * cg + 32 * part;
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = S0[static_cast<size_t>(c0 + j) * kDv];
+            tmem_st32(tmem + lane_base + kCColS + c0, v);
+#pragma unroll
+            for (int j = 0; j < 32; j += 8)
+                *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, c0 + j, 16384)) =
+                    make_uint4(f32x2_to_f16x2(v[j], v[j + 1]), f32x2_to_f16x2(v[j + 2], v[j + 3]),
+                               f32x2_to_f16x2(v[j + 4], v[j + 5]), f32x2_to_f16x2(v[j + 6], v[j + 7]));
+        }
+        tmem_wait_st();
+    }
+    float up[32], upn[32];
+    load_up(up, 0);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    uint32_t rph = 0, mph = 0;  // rph bit j: the phase buffer j's barrier waits for next
+    bool ok = true;
+    auto mma_wait = [&]() {
+        const bool w = wait_bar(mma_bar, mph, abort_flag, &g_prefill_error, lad::kErrPrefill);
+        mph ^= 1;
+        tc_fence_after();
+        return __syncthreads_and(w) != 0;
+    };
+    for (int i = 0; i < p.nseg && ok; ++i) {
+        const int buf = i & 1;
+        const uint32_t rs = kCRec + static_cast<uint32_t>(buf) * kCRecStride;  // offset of the record tiles
+        const float *gl = reinterpret_cast<const float *>(sm + rs + kRG);
+        const uint32_t xo = tmem + kCColXO + static_cast<uint32_t>(buf) * 128;
+        {
+            const bool w =
+                wait_bar(rec_bar0 + 8u * buf, (rph >> buf) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            rph ^= 1u << buf;
+            pend &= ~(1u << buf);
+            ok = __syncthreads_and(w) != 0;
+            if (!ok) break;
+        }
+        // ---- [X^T | O^T] = S^T [W; Qt]^T ----
+        if (warp == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < kDk / 16; ++j)
+                tc_mma_f16(xo, kdesc16(d0 + (kCS16 >> 4), 16384, j), kdesc16(d0 + ((rs + kRQW) >> 4), 16384, j),
+                           kIdescXO, j > 0);
+            tc_commit(mma_bar);
+        }
+        // ---- while it runs: the master takes the chunk's decay (column d_k times g_last[d_k]), the
+        //      previous chunk's outputs leave, the next chunk's U' comes into registers ----
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int c0 = 64 * cg + 32 * part;
+            float s[32];
+            tmem_ld32(tmem + lane_base + kCColS + c0, s);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s[j] *= gl[c0 + j];
+            tmem_st32(tmem + lane_base + kCColS + c0, s);
+        }
+        tmem_wait_st();
+        if (i > 0) store_o(i - 1);
+        if (i + 1 < p.nseg) load_up(upn, i + 1);
+        ok = mma_wait();
+        if (!ok) break;
+        // ---- U = U' - X -> the U^T operand (row d_v, this thread's 32 tokens) ----
+        {
+            float x[32];
+            tmem_ld32(xo + lane_base + 32 * cg, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; j += 8)
+                *reinterpret_cast<uint4 *>(sm + kCU16 + sw128_off16(dv, 32 * cg + j, 16384)) =
+                    make_uint4(f32x2_to_f16x2(up[j] - x[j], up[j + 1] - x[j + 1]),
+                               f32x2_to_f16x2(up[j + 2] - x[j + 2], up[j + 3] - x[j + 3]),
+                               f32x2_to_f16x2(up[j + 4] - x[j + 4], up[j + 5] - x[j + 5]),
+                               f32x2_to_f16x2(up[j + 6] - x[j + 6], up[j + 7] - x[j + 7]));
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // ---- S^T += U^T Kg (Kg read MN-major);  O^T += U^T P^T ----
+        if (warp == 0) {
+            tc_fence_after();
+            const uint64_t kg0 = smem_desc(sbase + rs + kRKG, 8192, 1024, kLayoutSw128);
+#pragma unroll
+            for (int j = 0; j < kC / 16; ++j) {
+                const uint64_t ua = kdesc16(d0 + (kCU16 >> 4), 16384, j);
+                tc_mma_f16(tmem + kCColS, ua, kg0 + ((j * 2048) >> 4), kIdescS, 1);
+                tc_mma_f16(xo + 64, ua, kdesc16(d0 + ((rs + kRP) >> 4), 8192, j), kIdescO, 1);
+            }
+            tc_commit(mma_bar);
+        }
+        ok = mma_wait();
+        if (!ok) break;
+        // ---- the buffer is free: chunk i + 2's record comes in; chunk i's is dropped from L2 ----
+        if (i + 2 < p.nseg) {
+            if (tid == 0) load_rec(i + 2);
+            pend |= 1u << buf;
+        }
+        if (warp == 1) {
+            const uint8_t *r = recs + static_cast<size_t>(i) * kRecBytes;
+            for (uint32_t l = lane; l < kRecBytes / 128; l += 32)
+                asm volatile("discard.global.L2 [%0], 128;" ::"l"(r + l * 128) : "memory");
+        }
+        // ---- the new state: its fp16 copy for the next chunk, or the state out after the last ----
+        const bool last = i == p.nseg - 1;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int c0 = 64 * cg + 32 * part;
+            float s[32];
+            tmem_ld32(tmem + lane_base + kCColS + c0, s);
+            tmem_wait_ld();
+            if (last) {
+                float *Sout = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) Sout[static_cast<size_t>(c0 + j) * kDv] = s[j];
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; j += 8)
+                    *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, c0 + j, 16384)) =
+                        make_uint4(f32x2_to_f16x2(s[j], s[j + 1]), f32x2_to_f16x2(s[j + 2], s[j + 3]),
+                                   f32x2_to_f16x2(s[j + 4], s[j + 5]), f32x2_to_f16x2(s[j + 6], s[j + 7]));
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) up[j] = upn[j];
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (last) store_o(i);
+    }
+    // drain: record copies still in flight (after an abort) land and every MMA this CTA issued
+    // completes, before shared memory and TMEM are released
+    if (tid == 0) {
+        const uint64_t t0 = lad::dev::globaltimer_ns();
+        for (int j = 0; j < 2; ++j)
+            while (((pend >> j) & 1u) && !mbar_try_wait(rec_bar0 + 8u * j, (rph >> j) & 1u) &&
+                   lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+            }
+    }
+    if (warp == 0) {
+        tc_commit(mma_bar);
+        const uint64_t t0 = lad::dev::globaltimer_ns();
+        while (!mbar_try_wait(mma_bar, mph) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kCTmemCols);
 }
 
 }  // namespace
@@ -1292,7 +1430,7 @@ extern "C" size_t kda_prefill_workspace_size(int B, int T, int H, int dk, int dv
     if (B <= 0 || T <= 0 || H <= 0 || dk != kDk || dv != kDv || chunk != kC) return 0;
     const long long nch = (static_cast<long long>(T) + kC - 1) / kC;
     const long long seg = nch < kSegChunks ? nch : kSegChunks;
-    return static_cast<size_t>(B) * static_cast<size_t>(H) * static_cast<size_t>(seg) * kItemBytes;
+    return static_cast<size_t>(B) * static_cast<size_t>(H) * static_cast<size_t>(seg) * kRecBytes;
 }
 
 extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, const float *alpha,
@@ -1317,8 +1455,8 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
     if (ctas > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "kda_prefill_chunked: B*H too large");
     const size_t ws_need = kda_prefill_workspace_size(B, T, H, dk, dv, chunk);
     const bool split = workspace != nullptr;
-    if (split && (ws_bytes < ws_need || !lad::aligned(workspace, 16)))
-        return set_error(LAD_EWORKSPACE, "kda_prefill_chunked: workspace of %zu bytes (16-byte aligned) required, or NULL",
+    if (split && (ws_bytes < ws_need || !lad::aligned(workspace, 256)))
+        return set_error(LAD_EWORKSPACE, "kda_prefill_chunked: workspace of %zu bytes (256-byte aligned) required, or NULL",
                          ws_need);
     if (split && static_cast<long long>(B) * H * kSegChunks > 0x7fffffffLL)
         return set_error(LAD_EUNSUPPORTED, "kda_prefill_chunked: B*H too large");
@@ -1327,11 +1465,11 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
     std::call_once(attr_once, [] {
         attr_err = cudaFuncSetAttribute(kda_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(kda_prefill_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            attr_err = cudaFuncSetAttribute(kda_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             kPSmemBytes);
         if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(kda_prefill_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            kSSmemBytes);
+            attr_err = cudaFuncSetAttribute(kda_chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            kCSmemBytes);
     });
     if (attr_err != cudaSuccess)
         return set_error(LAD_ECUDA, "kda_prefill_chunked: smem attribute: %s", cudaGetErrorString(attr_err));
@@ -1340,8 +1478,7 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
            (flags & LAD_FLAG_L2NORM_QK) ? 1 : 0, f32 ? 1 : 0};
     auto enc = reinterpret_cast<EncodeTiledFn>(lad::tensor_map_encoder_raw());
     if (!enc) return set_error(LAD_ECUDA, "kda_prefill_chunked: cuTensorMapEncodeTiled unavailable");
-    Maps maps;
-    auto make = [&](CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int box0) -> int {
+    auto make = [&](CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int box0, bool sw128) -> int {
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(H) * kDk, static_cast<cuuint64_t>(T),
                                     static_cast<cuuint64_t>(B)};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * kDk * esize,
@@ -1349,34 +1486,41 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
         const cuuint32_t box[3] = {static_cast<cuuint32_t>(box0), static_cast<cuuint32_t>(kC), 1};
         const cuuint32_t estr[3] = {1, 1, 1};
         CUresult r = enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                         sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         return r == CUDA_SUCCESS ? LAD_OK : set_error(LAD_ECUDA, "kda_prefill_chunked: tensor map failed (%d)", (int)r);
     };
-    int rc = make(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk);
-    if (rc == LAD_OK) rc = make(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk);
-    if (rc == LAD_OK) rc = make(&maps.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDk);
-    if (rc == LAD_OK) rc = make(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, split ? kDv : kDvh);
-    if (rc != LAD_OK) return rc;
     cudaStream_t st = lad::as_stream(stream);
     if (!split) {
+        Maps maps;
+        int rc = make(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk, false);
+        if (rc == LAD_OK) rc = make(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk, false);
+        if (rc == LAD_OK) rc = make(&maps.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDk, false);
+        if (rc == LAD_OK) rc = make(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDvh, false);
+        if (rc != LAD_OK) return rc;
         kda_prefill_kernel<<<static_cast<unsigned>(ctas), kThreads, kSmemBytes, st>>>(a, maps);
         return lad::check_launch("kda_prefill_chunked");
     }
     // split path, segment by segment: every chunk's operands of the segment (prep), then the chain
+    PrepMaps pm;
+    int rc = make(&pm.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk, false);
+    if (rc == LAD_OK) rc = make(&pm.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk, false);
+    if (rc == LAD_OK) rc = make(&pm.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDk, false);
+    if (rc == LAD_OK) rc = make(&pm.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, true);
+    if (rc != LAD_OK) return rc;
     const int nch = (T + kC - 1) / kC;
     const int sms = lad::device_sm_count();
     if (sms <= 0) return set_error(LAD_ECUDA, "kda_prefill_chunked: cannot query the SM count");
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
     for (int c0 = 0; c0 < nch; c0 += kSegChunks) {
         const int nseg = nch - c0 < kSegChunks ? nch - c0 : kSegChunks;
-        SplitArgs sa{a.q, a.k, a.v, alpha, beta, S, o, static_cast<uint8_t *>(workspace), B, T, H, c0, nseg,
-                     scale, a.l2norm, a.out_f32};
         const long long items = static_cast<long long>(B) * H * nseg;
         const unsigned pg = static_cast<unsigned>(items < sms ? items : sms);
-        kda_prefill_prep_kernel<<<pg, kThreads, kPSmemBytes, st>>>(sa, maps);
+        kda_chunk_prep_kernel<<<pg, kThreads, kPSmemBytes, st>>>(PrepArgs{beta, ws, B, T, H, c0, nseg, a.l2norm}, pm);
         rc = lad::check_launch("kda_prefill_chunked");
         if (rc != LAD_OK) return rc;
-        kda_prefill_scan_kernel<<<static_cast<unsigned>(ctas), kThreads, kSSmemBytes, st>>>(sa);
+        kda_chunk_chain_kernel<<<static_cast<unsigned>(B * H), kThreads, kCSmemBytes, st>>>(
+            ChainArgs{S, o, ws, B, T, H, c0, nseg, scale, a.out_f32});
         rc = lad::check_launch("kda_prefill_chunked");
         if (rc != LAD_OK) return rc;
     }

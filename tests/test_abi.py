@@ -115,9 +115,10 @@ def test_host_side_validation_of_the_fp8_calls(lib):
 
 
 def test_prefill_workspace_size(lib):
-    """The two-kernel prefill path's workspace: one 145 KiB record per (sequence, head, chunk) of a
-    segment of at most 128 chunks; zero for shapes the call does not support."""
-    rec = 145 * 1024
+    """The two-kernel prefill path's workspace: one 90,624-byte record (fp16 operand tiles, g_last
+    and U') per (sequence, head, chunk) of a segment of at most 128 chunks; zero for shapes the call
+    does not support."""
+    rec = 90624
     assert lib.kda_prefill_workspace_size(1, 32768, 64, 128, 128, 64) == 64 * 128 * rec
     assert lib.kda_prefill_workspace_size(2, 100, 3, 128, 128, 64) == 2 * 3 * 2 * rec
     assert lib.kda_prefill_workspace_size(1, 1, 1, 128, 128, 64) == rec

@@ -107,8 +107,9 @@ def test_decode_b64_conv_then_step(lad, cuda_device):
     qr = oracle.l2norm(y_ref16[:, : H * d].reshape(B, 1, H, d))
     kr = oracle.l2norm(y_ref16[:, H * d: 2 * H * d].reshape(B, 1, H, d))
     vr = y_ref16[:, 2 * H * d:].reshape(B, 1, H, d)
+    S0 = f64(inp["S"])
     o_ref, S_ref = oracle.kda_recurrent(qr, kr, vr, f64(inp["alpha"])[:, None], f64(inp["beta"])[:, None],
-                                        f64(inp["S"]), nthreads=oracle.max_threads())
+                                        S0, nthreads=oracle.max_threads())
 
     y = lad.kda_conv_update(inp["x"], inp["tail"], inp["w"], silu=True)
     o = lad.kda_decode_step(y[:, : H * d], y[:, H * d: 2 * H * d], y[:, 2 * H * d:], inp["alpha"], inp["beta"],
@@ -121,7 +122,14 @@ def test_decode_b64_conv_then_step(lad, cuda_device):
     assert np.all(np.abs(yg - y_ref16) <= np.abs(y_ref16) * 2.0 ** -7 + 1e-30)
     assert rel_l2(o, o_ref[:, 0]) < 1e-4
     assert rel_l2(inp["S"], S_ref) < TOL_STATE
-    assert max_rel_l2(o, o_ref[:, 0], 2) < 1e-4 and max_rel_l2(inp["S"], S_ref, 2) < TOL_STATE
+    # per head, against the oracle fed the exact bf16 conv output the step consumed (the rounded
+    # fp64 conv output above can differ from it by one bf16 step in a few channels, which moves a
+    # single head's o by a few 1e-4)
+    q2 = oracle.l2norm(yg[:, : H * d].reshape(B, 1, H, d))
+    k2 = oracle.l2norm(yg[:, H * d: 2 * H * d].reshape(B, 1, H, d))
+    o2, S2 = oracle.kda_recurrent(q2, k2, yg[:, 2 * H * d:].reshape(B, 1, H, d), f64(inp["alpha"])[:, None],
+                                  f64(inp["beta"])[:, None], S0, nthreads=oracle.max_threads())
+    assert max_rel_l2(o, o2[:, 0], 2) < 1e-4 and max_rel_l2(inp["S"], S2, 2) < TOL_STATE
 
 
 @pytest.mark.parametrize("B,H", [(1, 1), (3, 7), (256, 64)])
