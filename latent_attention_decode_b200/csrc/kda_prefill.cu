@@ -711,111 +711,104 @@ __device__ __forceinline__ void put_tb4(uint8_t *tb16, uint8_t *tbh, uint8_t *tb
     *reinterpret_cast<uint2 *>(tbl + off) = make_uint2(bf16x2_rn(a - fa.x, b - fa.y), bf16x2_rn(c - fc.x, d - fc.y));
 }
 
-__device__ __forceinline__ void put_tb1(uint8_t *tb16, uint8_t *tbh, uint8_t *tbl, int r, int s, float a) {
-    const uint32_t off = sw128_off16(r, s, 8192);
-    *reinterpret_cast<__half *>(tb16 + off) = __float2half_rn(a);
-    const __nv_bfloat16 h = __float2bfloat16_rn(a);
-    *reinterpret_cast<__nv_bfloat16 *>(tbh + off) = h;
-    *reinterpret_cast<__nv_bfloat16 *>(tbl + off) = __float2bfloat16_rn(a - __bfloat162float(h));
-}
 
-// T = (I + A)^-1 for A strictly lower triangular [64][64] (fp32, row stride kAS), by 16x16 blocks:
-// the diagonal blocks by forward substitution (one thread per column), then M_ik = T_ii A_ik for
-// the six blocks below the diagonal (written over A), then T_ij = -sum_k M_ik T_kj one block row at
-// a time. T goes to sT; Tb = T diag(beta) to the three operand tiles as each block is final.
-// Called by all kThreads threads; contains block-wide barriers.
+// T = (I + A)^-1 for A strictly lower triangular [64][64] (fp32, row stride kAS), by recursive
+// doubling over 16x16 blocks: (1) the four diagonal blocks by forward substitution, one thread per
+// column; (2) in each 32x32 diagonal block, T_{2p+1,2p} = -T_{2p+1,2p+1} A_{2p+1,2p} T_{2p,2p};
+// (3) the lower-left 32x32 block, -T_hi A_{hi,lo} T_lo. The products A T of (2) and (3) are parked in
+// A's upper triangle, which holds no data. Then Tb = T diag(beta) goes to the three operand tiles
+// (fp16, and the bf16 hi / lo split). Called by all kThreads threads; contains block-wide barriers.
 __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_beta, uint8_t *tb16, uint8_t *tbh,
                                           uint8_t *tbl, int tid) {
     if (tid < kC) {
+        // column c of (I + A_ii)^-1: t_r = [r == c] - sum_{c <= s < r} A_rs t_s
         const int i0 = 16 * (tid >> 4), c = tid & 15;
         float t[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            float acc = (r == c) ? 1.f : 0.f;
+            float acc = 0.f;
 #pragma unroll
-            for (int s = 0; s < r; ++s) acc = fmaf(-sA[(i0 + r) * kAS + i0 + s], t[s], acc);
-            t[r] = acc;
+            for (int s2 = 0; s2 < r; ++s2) acc = fmaf(sA[(i0 + r) * kAS + i0 + s2], t[s2], acc);
+            t[r] = r < c ? 0.f : (r == c ? 1.f : -acc);
         }
-        const float bc = s_beta[i0 + c];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            sT[(i0 + r) * kAS + i0 + c] = t[r];
-            put_tb1(tb16, tbh, tbl, i0 + r, i0 + c, t[r] * bc);
-        }
-    } else {
-        // zero the six blocks above the diagonal of the three tiles: 6 blocks x 16 rows x 2 chunks
-        for (int e = tid - kC; e < 6 * 32; e += kThreads - kC) {
-            const int blk = e >> 5, rr = (e >> 1) & 15, hf = e & 1;
-            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-            const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            const uint32_t off = sw128_off16(16 * bi + rr, 16 * bj + 8 * hf, 8192);
-            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4 *>(tb16 + off) = z;
-            *reinterpret_cast<uint4 *>(tbh + off) = z;
-            *reinterpret_cast<uint4 *>(tbl + off) = z;
-        }
+        for (int r = 0; r < 16; ++r) sT[(i0 + r) * kAS + i0 + c] = t[r];
     }
     __syncthreads();
-    {
-        // M_ik for (i, k) = (1,0), (2,0), (2,1), (3,0), (3,1), (3,2): 6 blocks x 64 strips of 1x4
-        float4 m[2];
-        int mi[2], mk[2];
+    // (2a) Y_p = A_{2p+1,2p} T_{2p,2p} into A at rows 32p .. 32p+15, columns 32p+16 .. 32p+31
+    if (tid < 128) {
+        const int q0 = 32 * (tid >> 6), rr = (tid >> 2) & 15, cc = (tid & 3) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int e = tid + h * kThreads;
-            m[h] = make_float4(0.f, 0.f, 0.f, 0.f);
-            mi[h] = -1;
-            mk[h] = 0;
-            if (e < 6 * 64) {
-                const int blk = e >> 6, rr = (e >> 2) & 15, cc = (e & 3) * 4;
-                const int i = blk == 0 ? 1 : (blk < 3 ? 2 : 3);
-                const int k = blk == 0 ? 0 : (blk < 3 ? blk - 1 : blk - 3);
-                mi[h] = i;
-                mk[h] = k;
-#pragma unroll
-                for (int ss = 0; ss < 16; ++ss) {
-                    const float tv = sT[(16 * i + rr) * kAS + 16 * i + ss];
-                    const float4 a4 = *reinterpret_cast<const float4 *>(sA + (16 * i + ss) * kAS + 16 * k + cc);
-                    m[h].x = fmaf(tv, a4.x, m[h].x);
-                    m[h].y = fmaf(tv, a4.y, m[h].y);
-                    m[h].z = fmaf(tv, a4.z, m[h].z);
-                    m[h].w = fmaf(tv, a4.w, m[h].w);
-                }
-            }
+        for (int s2 = 0; s2 < 16; ++s2) {
+            const float a = sA[(q0 + 16 + rr) * kAS + q0 + s2];
+            const float4 t4 = *reinterpret_cast<const float4 *>(sT + (q0 + s2) * kAS + q0 + cc);
+            acc.x = fmaf(a, t4.x, acc.x);
+            acc.y = fmaf(a, t4.y, acc.y);
+            acc.z = fmaf(a, t4.z, acc.z);
+            acc.w = fmaf(a, t4.w, acc.w);
         }
-        __syncthreads();  // every read of A is done: the M blocks replace it
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int e = tid + h * kThreads;
-            if (mi[h] >= 0) {
-                const int rr = (e >> 2) & 15, cc = (e & 3) * 4;
-                *reinterpret_cast<float4 *>(sA + (16 * mi[h] + rr) * kAS + 16 * mk[h] + cc) = m[h];
-            }
-        }
-        __syncthreads();
+        *reinterpret_cast<float4 *>(sA + (q0 + rr) * kAS + q0 + 16 + cc) = acc;
     }
-#pragma unroll 1
-    for (int bi = 1; bi < 4; ++bi) {
-        if (tid < bi * 64) {
-            const int bj = tid >> 6, rr = (tid >> 2) & 15, cc = (tid & 3) * 4;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int kb = bj; kb < bi; ++kb) {
+    __syncthreads();
+    // (2b) T_{2p+1,2p} = -T_{2p+1,2p+1} Y_p
+    if (tid < 128) {
+        const int q0 = 32 * (tid >> 6), rr = (tid >> 2) & 15, cc = (tid & 3) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int ss = 0; ss < 16; ++ss) {
-                    const float a = sA[(16 * bi + rr) * kAS + 16 * kb + ss];
-                    const float4 t4 = *reinterpret_cast<const float4 *>(sT + (16 * kb + ss) * kAS + 16 * bj + cc);
-                    acc.x = fmaf(a, t4.x, acc.x);
-                    acc.y = fmaf(a, t4.y, acc.y);
-                    acc.z = fmaf(a, t4.z, acc.z);
-                    acc.w = fmaf(a, t4.w, acc.w);
-                }
-            }
-            const int r = 16 * bi + rr, c = 16 * bj + cc;
-            *reinterpret_cast<float4 *>(sT + r * kAS + c) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-            put_tb4(tb16, tbh, tbl, r, c, -acc.x * s_beta[c], -acc.y * s_beta[c + 1], -acc.z * s_beta[c + 2],
-                    -acc.w * s_beta[c + 3]);
+        for (int s2 = 0; s2 < 16; ++s2) {
+            const float t = sT[(q0 + 16 + rr) * kAS + q0 + 16 + s2];
+            const float4 y4 = *reinterpret_cast<const float4 *>(sA + (q0 + s2) * kAS + q0 + 16 + cc);
+            acc.x = fmaf(t, y4.x, acc.x);
+            acc.y = fmaf(t, y4.y, acc.y);
+            acc.z = fmaf(t, y4.z, acc.z);
+            acc.w = fmaf(t, y4.w, acc.w);
         }
-        __syncthreads();
+        *reinterpret_cast<float4 *>(sT + (q0 + 16 + rr) * kAS + q0 + cc) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    __syncthreads();
+    // (3a) R = A_{hi,lo} T_lo (32 x 32) into A at rows 0 .. 31, columns 32 .. 63; T_lo is lower
+    //      triangular, so only s >= cc contributes
+    {
+        const int rr = tid >> 3, cc = (tid & 7) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int s2 = cc; s2 < 32; ++s2) {
+            const float a = sA[(32 + rr) * kAS + s2];
+            const float4 t4 = *reinterpret_cast<const float4 *>(sT + s2 * kAS + cc);
+            acc.x = fmaf(a, t4.x, acc.x);
+            acc.y = fmaf(a, t4.y, acc.y);
+            acc.z = fmaf(a, t4.z, acc.z);
+            acc.w = fmaf(a, t4.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(sA + rr * kAS + 32 + cc) = acc;
+    }
+    __syncthreads();
+    // (3b) T[32 + rr][0 .. 31] = -T_hi R; T_hi is lower triangular, so only s <= rr contributes
+    {
+        const int rr = tid >> 3, cc = (tid & 7) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int s2 = 0; s2 <= rr; ++s2) {
+            const float t = sT[(32 + rr) * kAS + 32 + s2];
+            const float4 r4 = *reinterpret_cast<const float4 *>(sA + s2 * kAS + 32 + cc);
+            acc.x = fmaf(t, r4.x, acc.x);
+            acc.y = fmaf(t, r4.y, acc.y);
+            acc.z = fmaf(t, r4.z, acc.z);
+            acc.w = fmaf(t, r4.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(sT + (32 + rr) * kAS + cc) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    __syncthreads();
+    // Tb = T diag(beta): 64 rows x 16 quads of columns, four quads per thread; zero above the
+    // diagonal blocks (T holds nothing there)
+#pragma unroll
+    for (int e = tid; e < kC * 16; e += kThreads) {
+        const int r = e >> 4, c = (e & 15) * 4;
+        float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if ((c >> 4) <= (r >> 4)) t4 = *reinterpret_cast<const float4 *>(sT + r * kAS + c);
+        put_tb4(tb16, tbh, tbl, r, c, t4.x * s_beta[c], t4.y * s_beta[c + 1], t4.z * s_beta[c + 2],
+                t4.w * s_beta[c + 3]);
     }
 }
 
@@ -910,6 +903,15 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
     int pending = 0;   // a staging phase is in flight
     int v_owed = -1;   // an item whose q, k and alpha are staged but whose v is not yet
     int item = blockIdx.x;
+    // beta of an item (threads 0-63, one token each, strided by H in memory): loaded one item ahead
+    auto load_beta = [&](int it) -> float {
+        if (tid >= kC || it >= nitems) return 0.f;
+        int b, h, ch;
+        coords(it, b, h, ch);
+        const int t = ch * kC + tid;
+        return t < p.T ? p.beta[(static_cast<size_t>(b) * p.T + t) * p.H + h] : 0.f;
+    };
+    float beta_next = load_beta(item);
     if (item < nitems) {
         if (tid == 0) {
             stage_qka(item);
@@ -923,10 +925,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
         const int next = item + static_cast<int>(gridDim.x);
         const int t0 = ch * kC;
         const int n = min(kC, p.T - t0);
-        const size_t tok0 = (static_cast<size_t>(b) * p.T + t0) * p.H + h;
         uint8_t *rec = p.ws + static_cast<size_t>(item) * kRecBytes;
 
-        if (tid < kC) s_beta[tid] = (tid < n) ? p.beta[tok0 + static_cast<size_t>(tid) * p.H] : 0.f;
+        if (tid < kC) s_beta[tid] = beta_next;
+        beta_next = load_beta(next);
         if (tid == 0) bulk_wait_read0();  // the previous item's tiles have left for its record
         {
             const bool w = wait_bar(stage_bar, stage_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
@@ -1172,13 +1174,21 @@ constexpr uint32_t kCS16 = 0;            // S^T [128 d_v][128 d_k] fp16, K-major
 constexpr uint32_t kCU16 = 32768;        // U^T [128 d_v][64 tok] fp16, K-major SW128, 16 KiB
 constexpr uint32_t kCRec = 49152;        // two record buffers (the tiles and g_last of a chunk)
 constexpr uint32_t kCRecStride = 58368;  // 57 KiB each (1024-aligned)
-constexpr uint32_t kCMisc = kCRec + 2 * kCRecStride;
+constexpr uint32_t kCO = kCRec + 2 * kCRecStride;  // O [64 tok][128 d_v] bf16 or fp32, plain (TMA store)
+constexpr uint32_t kCMisc = kCO + 32768;
 constexpr uint32_t kCSmemBytes = kCMisc + 64 + 1024;
 // TMEM: the fp32 master S^T (128 lanes = d_v, 128 columns = d_k) and two [X^T | O^T] buffers
 constexpr uint32_t kCColS = 0, kCColXO = 128, kCTmemCols = 512;
 
 // One CTA per (sequence, head) walks the segment's chunks with the state master in tensor memory.
-__global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs p) {
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs p, const __grid_constant__ CUtensorMap omap) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -1226,25 +1236,26 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
 #pragma unroll
         for (int j = 0; j < 32; ++j) u[j] = __ldcg(src + (32 * cg + j) * kDv);
     };
-    // the outputs of chunk i (O^T in buffer i % 2, columns 64-127), scaled
-    auto store_o = [&](int i) {
+    // the outputs of chunk i (O^T in buffer i % 2, columns 64-127), scaled, into the O tile
+    // [token][d_v] (a TMA store takes it out; rows past T are not written)
+    auto stage_o = [&](int i) {
         float x[32];
         tmem_ld32(tmem + lane_base + kCColXO + static_cast<uint32_t>(i & 1) * 128 + 64 + 32 * cg, x);
         tmem_wait_ld();
-        const int t0 = (p.c0 + i) * kC;
-        const int n = min(kC, p.T - t0);
-        const size_t row0 = (static_cast<size_t>(b) * p.T + t0) * p.H + h;
+        if (p.out_f32) {
+            float *od = reinterpret_cast<float *>(sm + kCO) + dv;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int t = 32 * cg + j;
-            if (t < n) {
-                const size_t at = (row0 + static_cast<size_t>(t) * p.H) * kDv + dv;
-                if (p.out_f32)
-                    static_cast<float *>(p.o)[at] = p.scale * x[j];
-                else
-                    static_cast<uint16_t *>(p.o)[at] = lad::dev::f32_to_bf16(p.scale * x[j]);
-            }
+            for (int j = 0; j < 32; ++j) od[(32 * cg + j) * kDv] = p.scale * x[j];
+        } else {
+            uint16_t *od = reinterpret_cast<uint16_t *>(sm + kCO) + dv;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) od[(32 * cg + j) * kDv] = lad::dev::f32_to_bf16(p.scale * x[j]);
         }
+        fence_async_smem();
+    };
+    auto store_o = [&](int i) {  // one thread, after a barrier that follows stage_o
+        tma_store_3d(&omap, sbase + kCO, h * kDv, (p.c0 + i) * kC, b);
+        bulk_commit();
     };
 
     // ---- the state entering the segment: master S^T and its fp16 copy ----
@@ -1288,6 +1299,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
         {
             const bool w =
                 wait_bar(rec_bar0 + 8u * buf, (rph >> buf) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            if (tid == 0) bulk_wait_read0();  // the previous outputs have left the O tile
             rph ^= 1u << buf;
             pend &= ~(1u << buf);
             ok = __syncthreads_and(w) != 0;
@@ -1315,10 +1327,11 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
             tmem_st32(tmem + lane_base + kCColS + c0, s);
         }
         tmem_wait_st();
-        if (i > 0) store_o(i - 1);
+        if (i > 0) stage_o(i - 1);
         if (i + 1 < p.nseg) load_up(upn, i + 1);
         ok = mma_wait();
         if (!ok) break;
+        if (i > 0 && tid == 0) store_o(i - 1);
         // ---- U = U' - X -> the U^T operand (row d_v, this thread's 32 tokens) ----
         {
             float x[32];
@@ -1354,11 +1367,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
             if (tid == 0) load_rec(i + 2);
             pend |= 1u << buf;
         }
-        if (warp == 1) {
-            const uint8_t *r = recs + static_cast<size_t>(i) * kRecBytes;
-            for (uint32_t l = lane; l < kRecBytes / 128; l += 32)
-                asm volatile("discard.global.L2 [%0], 128;" ::"l"(r + l * 128) : "memory");
-        }
         // ---- the new state: its fp16 copy for the next chunk, or the state out after the last ----
         const bool last = i == p.nseg - 1;
 #pragma unroll
@@ -1384,7 +1392,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (last) store_o(i);
+        if (last) {
+            if (tid == 0) bulk_wait_read0();
+            __syncthreads();
+            stage_o(i);
+            __syncthreads();
+            if (tid == 0) store_o(i);
+        }
     }
     // drain: record copies still in flight (after an abort) land and every MMA this CTA issued
     // completes, before shared memory and TMEM are released
@@ -1395,6 +1409,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
                    lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
             }
     }
+    if (tid == 0) bulk_wait_all();  // the output stores have completed
     if (warp == 0) {
         tc_commit(mma_bar);
         const uint64_t t0 = lad::dev::globaltimer_ns();
@@ -1507,6 +1522,10 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
     if (rc == LAD_OK) rc = make(&pm.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk, false);
     if (rc == LAD_OK) rc = make(&pm.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDk, false);
     if (rc == LAD_OK) rc = make(&pm.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, true);
+    CUtensorMap omap;
+    if (rc == LAD_OK)
+        rc = make(&omap, o, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 ? 4 : 2, kDv,
+                  false);
     if (rc != LAD_OK) return rc;
     const int nch = (T + kC - 1) / kC;
     const int sms = lad::device_sm_count();
@@ -1520,7 +1539,7 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
         rc = lad::check_launch("kda_prefill_chunked");
         if (rc != LAD_OK) return rc;
         kda_chunk_chain_kernel<<<static_cast<unsigned>(B * H), kThreads, kCSmemBytes, st>>>(
-            ChainArgs{S, o, ws, B, T, H, c0, nseg, scale, a.out_f32});
+            ChainArgs{S, o, ws, B, T, H, c0, nseg, scale, a.out_f32}, omap);
         rc = lad::check_launch("kda_prefill_chunked");
         if (rc != LAD_OK) return rc;
     }
