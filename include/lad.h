@@ -62,7 +62,8 @@ int lad_version(void);
 /*
  * Reads and clears the device-side error word that bounded waits set (see above), after
  * synchronising `stream`. *code receives 0 when no kernel gave up a wait, else a nonzero tag
- * naming the kernel and the wait (0x101-0x104 and 0x107 latent decode, 0x201 chunked prefill),
+ * naming the kernel and the wait (0x101-0x104 and 0x107 latent decode, 0x201 chunked prefill,
+ * 0x501 the KDA decode step's copy of a second head's state, taken at small batch),
  * 0x106 when an FP8-cache decode met a query value beyond the f16 range, 0x105 when
  * a paged decode met a block-table entry outside the pool, or 0x301 when mla_cache_append had a
  * position with no row to write. Returns LAD_OK or LAD_ECUDA.

@@ -16,9 +16,11 @@
 #include <algorithm>
 #include <mutex>
 
-#include "lad_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace {
+
+__device__ int g_kda_error = 0;
 
 using lad::dev::bf16_to_f32;
 using lad::dev::f32_to_bf16;
@@ -79,11 +81,12 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // kPair (small batches): a CTA updates two heads, bh = blockIdx.x and bh + gridDim.x. With one
 // head per CTA and B * H between one and two times the resident CTAs (8 x 64 heads on 296 slots),
 // the CTAs of the second wave start only as the first wave's finish, and the waves load, reduce
-// and store in step, so HBM idles between the phases. Here the second head's state is copied
-// into shared memory (cp.async, each thread its own 16-byte slots, read back by the same thread
-// only) while the first head is loaded into registers, so every state byte of the launch is
-// requested at once; the second head then runs from shared memory while the first head's
-// stores drain.
+// and store in step, so HBM idles between the phases. Here the second head's 64 KiB state comes
+// into shared memory by one bulk copy (the copy engine, not the load/store units, which the
+// first head's 16 loads per thread keep busy) while the first head is loaded into registers, so
+// every state byte of the launch is requested at once; the second head then runs from shared
+// memory while the first head's stores drain. The copy's wait is bounded: if it runs out, the
+// second head is left untouched and device error 0x501 is recorded.
 constexpr int kPairSmemBytes = kRowsPerWarp * kThreads * 16;  // 64 KiB of state slots
 
 template <bool kOutF32, bool kFusedConv, bool kPair>
@@ -111,12 +114,19 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) s[r] = __ldcs(mine + r * kVec);
     }
-    const uint32_t slot_base = static_cast<uint32_t>(__cvta_generic_to_shared(pair_slots)) + threadIdx.x * 16;
-    if (has1) {
-        const float4 *src = state_of(bh1);
-#pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) cp_async16(slot_base + r * kThreads * 16, src + r * kVec);
-        cp_async_commit();
+    __shared__ __align__(8) uint64_t pair_bar;
+    __shared__ int pair_abort;
+    const uint32_t bar = static_cast<uint32_t>(__cvta_generic_to_shared(&pair_bar));
+    if (has1 && threadIdx.x == 0) {
+        pair_abort = 0;
+        lad::ptx::mbar_init(bar, 1);
+        lad::ptx::mbar_fence_init();
+        lad::ptx::mbar_arrive_tx_raw(bar, kD * kD * 4);
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                static_cast<uint32_t>(__cvta_generic_to_shared(pair_slots))),
+            "l"(reinterpret_cast<uint64_t>(S + static_cast<size_t>(bh1) * kD * kD)), "r"(kD * kD * 4), "r"(bar)
+            : "memory");
     }
 
     __shared__ float sq[kUnits][kD], sk[kUnits][kD], sv[kUnits][kD], sa[kUnits][kD];
@@ -277,14 +287,22 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
     update(0, bh0);
     if constexpr (kPair) {
         if (has1) {
-            // the second head: this thread's own slots (no barrier needed to read them), then a
-            // barrier before the reduction buffers and the gate inputs are reused
-            cp_async_wait_all();
-            const float4 *slots = reinterpret_cast<const float4 *>(pair_slots) + threadIdx.x;
+            // the second head from shared memory (the state's own layout: this thread's rows and
+            // float4 of columns), then a barrier before the reduction buffers and gate inputs are reused
+            const bool landed = lad::ptx::wait_bar(bar, 0, &pair_abort, &g_kda_error, lad::kErrKdaPair);
+            const float4 *rows = reinterpret_cast<const float4 *>(pair_slots) +
+                                 static_cast<size_t>(warp * kRowsPerWarp) * kVec + lane;
 #pragma unroll
-            for (int r = 0; r < kRowsPerWarp; ++r) s[r] = slots[r * kThreads];
-            __syncthreads();
-            update(1, bh1);
+            for (int r = 0; r < kRowsPerWarp; ++r) s[r] = rows[r * kVec];
+            if (__syncthreads_and(landed)) {
+                update(1, bh1);
+            } else if (threadIdx.x == 0) {
+                // the copy may still be in flight: give it one more bounded wait before the CTA
+                // (and its shared memory) goes away
+                const uint64_t t0 = lad::dev::globaltimer_ns();
+                while (!lad::ptx::mbar_try_wait(bar, 0) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+                }
+            }
         }
     }
 }
@@ -511,6 +529,23 @@ kda_decode_multi_kernel(const uint16_t *__restrict__ q, const uint16_t *__restri
 }
 
 }  // namespace
+
+namespace lad {
+int take_device_error_kda(cudaStream_t s, int *code) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_kda_error, sizeof v, 0, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return set_error(LAD_ECUDA, "lad_device_error: %s", cudaGetErrorString(e));
+    if (v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_kda_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return set_error(LAD_ECUDA, "lad_device_error: %s", cudaGetErrorString(e));
+    }
+    *code = v;
+    return LAD_OK;
+}
+}  // namespace lad
 
 namespace {
 // One head per CTA, or two (kPair) when B * H is between one and two times the resident CTAs:

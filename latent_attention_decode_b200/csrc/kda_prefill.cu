@@ -614,12 +614,19 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
 // ------------------------------------------------------------------------------------------
 // Split path (a workspace is given): the chunk-local, state-independent part of every chunk in
 // parallel (prep), then the state chain alone (chain), segment by segment. With S0 the state
-// entering a chunk, U' = Tb V, W = Tb Kt and P = lower(Qt Kh^T):
+// entering a chunk, U' = Tb V, W = Tb Kt, P = lower(Qt Kh^T) and Kg = K * g_last / g (the chunk's
+// decay folded into the key), the chunk form
 //   X = W S0,  U = U' - X,  O = scale (Qt S0 + P U),  S = Diag(g_last) S0 + Kg^T U
-// with Kg = K * g_last / g (the chunk's decay folded into the key). The chain holds S^T (rows d_v,
-// columns d_k) as its fp32 master in tensor memory and runs, per chunk, two tensor-core batches:
-//   [X^T | O^T]  = S0^T [W; Qt]^T           M = 128 (d_v), N = 128 (64 W + 64 Qt rows), K = 128
-//   S^T += U^T Kg,  O^T += U^T P^T          M = 128, N = 128 and 64, K = 64 (tokens)
+// regroups by what multiplies S0:
+//   S = Diag(g_last) S0 + Kg^T U' + N S0,        N = -Kg^T W
+//   O = scale (Qe S0 + P U'),                     Qe = Qt - P W
+// The prep computes N, Qe, Kg, P and U' (all chunk-local); the chain then holds S^T (rows d_v,
+// columns d_k) as an fp32 master in tensor memory and runs one tensor-core batch per chunk
+// (M = 128 value rows):
+//   S^T <- S^T Diag(g_last) (threads, fp32)  +  U'^T Kg  +  S0^T N^T
+//   O^T  = U'^T P^T + S0^T Qe^T
+// so the state makes one trip through the threads per chunk (fp32 master -> fp16 operand copy,
+// and the decay), the decay itself never rounded to fp16.
 // Every operand is fp16 (kind::f16, fp32 accumulation): its rounding unit is that of tf32 and it
 // runs at twice tf32's rate with half the bytes; each tile is stored once, rows as formed, and
 // the tensor cores read it K-major or MN-major as a contraction needs (no transposed copies).
@@ -628,14 +635,14 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
 // keys that needs a chunk's decay product below about 1.5e-5.
 // ------------------------------------------------------------------------------------------
 
-// Record of one (sequence, head, chunk) in the workspace: the three fp16 tiles and g_last, laid
-// out exactly as the chain's shared-memory operands (one bulk copy), then U' for direct loads.
-constexpr uint32_t kRQW = 0;           // [W; Qt]: 128 rows x 128 d_k fp16, K-major SW128, 2 blocks x 16 KiB
-constexpr uint32_t kRKG = 32768;       // Kg [64 tok][128 d_k] fp16, SW128, 2 blocks x 8 KiB (read MN-major)
-constexpr uint32_t kRP = 49152;        // P = lower(Qt Kh^T) [64 r][64 s] fp16, K-major SW128, 8 KiB
-constexpr uint32_t kRG = 57344;        // g_last [128] fp32
-constexpr uint32_t kRTiles = 57856;    // the four above: one bulk copy
-constexpr uint32_t kRUP = 57856;       // U' [64 tok][128 d_v] fp32, plain row-major
+// Record of one (sequence, head, chunk) in the workspace: the chain's operand tiles (fp16, SW128)
+// and g_last, laid out exactly as in the chain's shared memory (one bulk copy).
+constexpr uint32_t kRN = 0;            // N [128 d_k'][128 d_k], K-major: 2 blocks x 16 KiB
+constexpr uint32_t kRQE = 32768;       // Qe [64 tok][128 d_k], K-major: 2 blocks x 8 KiB
+constexpr uint32_t kRKG = 49152;       // Kg [64 tok][128 d_k]: 2 blocks x 8 KiB (read MN-major)
+constexpr uint32_t kRP = 65536;        // P [64 r][64 s], K-major: 8 KiB
+constexpr uint32_t kRU = 73728;        // U'^T [128 d_v][64 tok], K-major: 16 KiB
+constexpr uint32_t kRG = 90112;        // g_last [128] fp32
 constexpr uint32_t kRecBytes = 90624;  // 708 lines of 128 bytes
 #ifndef LAD_PREFILL_SEG_CHUNKS
 #define LAD_PREFILL_SEG_CHUNKS 128
@@ -662,9 +669,11 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
 constexpr uint32_t kIdescA = make_idesc(128, 64, kFmtF16, 0, 0);     // [Kt; Qt] Kh^T
 constexpr uint32_t kIdescW = make_idesc(64, 128, kFmtF16, 0, 1);     // W = Tb Kt (Kt read MN-major)
 constexpr uint32_t kIdescU = make_idesc(128, 64, kFmtBf16, 1, 0);    // U'^T = V^T Tb^T (V read MN-major)
-constexpr uint32_t kIdescXO = make_idesc(128, 128, kFmtF16, 0, 0);   // [X^T | O^T] = S^T [W; Qt]^T
-constexpr uint32_t kIdescS = make_idesc(128, 128, kFmtF16, 0, 1);    // S^T += U^T Kg (Kg read MN-major)
-constexpr uint32_t kIdescO = make_idesc(128, 64, kFmtF16, 0, 0);     // O^T += U^T P^T
+constexpr uint32_t kIdescN = make_idesc(128, 128, kFmtF16, 1, 1);    // Kg^T W (both read MN-major)
+constexpr uint32_t kIdescPW = make_idesc(64, 128, kFmtF16, 0, 1);    // P W (W read MN-major)
+constexpr uint32_t kIdescSU = make_idesc(128, 128, kFmtF16, 0, 1);   // S^T += U'^T Kg (Kg read MN-major)
+constexpr uint32_t kIdescSN = make_idesc(128, 128, kFmtF16, 0, 0);   // S^T += S0^T N^T
+constexpr uint32_t kIdescO = make_idesc(128, 64, kFmtF16, 0, 0);     // O^T = U'^T P^T + S0^T Qe^T
 
 struct PrepArgs {
     const float *beta;
@@ -679,10 +688,17 @@ struct PrepMaps {
     CUtensorMap v;            // the same view of v, boxes of 64 channels x 64 tokens, 128-byte swizzle
 };
 
-// prep shared memory (offsets from a 1024-aligned base); the record's tiles sit as in the record
-constexpr uint32_t kPQW = kRQW, kPKG = kRKG, kPP = kRP, kPG = kRG;  // [0, 57856)
-constexpr uint32_t kPKH = 58368;    // Kh [64 tok][128 d_k] fp16 K-major, 2 blocks x 8 KiB
-constexpr uint32_t kPTB = 74752;    // Tb [64 r][64 s] fp16 K-major
+// prep shared memory (offsets from a 1024-aligned base). Regions are reused once their first
+// contents are dead: Kh (after the first MMA batch) holds U'^T, the Tb tiles (after the second)
+// hold Qe, the A / T scratch (after the solve) holds N. The record leaves by bulk stores from
+// where its tiles sit.
+constexpr uint32_t kPQW = 0;        // [Kt; Qt]: 128 rows x 128 d_k fp16, K-major, 2 blocks x 16 KiB;
+                                    //   rows 0-63 become W once Kt is read
+constexpr uint32_t kPKH = 32768;    // Kh [64 tok][128 d_k], 2 blocks x 8 KiB; then U'^T [128 d_v][64 tok]
+constexpr uint32_t kPKG = 49152;    // Kg [64 tok][128 d_k], 2 blocks x 8 KiB (record)
+constexpr uint32_t kPP = 65536;     // P [64][64] (record)
+constexpr uint32_t kPG = 73728;     // g_last [128] fp32 (record)
+constexpr uint32_t kPTB = 74752;    // Tb [64 r][64 s] fp16 K-major; then (with TBH) Qe [64][128], 2 x 8 KiB
 constexpr uint32_t kPTBH = 82944;   // Tb, bf16 high part
 constexpr uint32_t kPTBL = 91136;   // Tb, bf16 low part (Tb - hi)
 constexpr uint32_t kPV = 99328;     // v [64 tok][128 d_v] bf16 as two SW128 boxes of 64 d_v (TMA)
@@ -690,7 +706,7 @@ constexpr uint32_t kPSQ = 115712;   // q [64 tok][128] bf16, plain (TMA)
 constexpr uint32_t kPSK = 132096;   // k, the same
 constexpr uint32_t kPSA = 148480;   // alpha [64 tok][128] fp32, plain (TMA)
 constexpr int kAS = 68;             // row stride (floats) of the A / T scratch (68: fewer bank conflicts)
-constexpr uint32_t kPA = 181248;    // A [64][kAS] fp32
+constexpr uint32_t kPA = 181248;    // A [64][kAS] fp32; then (with T) N [128][128] fp16, 2 x 16 KiB
 constexpr uint32_t kPT = kPA + 64 * kAS * 4;   // T [64][kAS] fp32
 constexpr uint32_t kPMisc = kPT + 64 * kAS * 4;
 constexpr uint32_t kPmBeta = 0, kPmRq = 256, kPmRk = 512, kPmOct = 768, kPmBar = 768 + 4096, kPmTmem = kPmBar + 16,
@@ -698,7 +714,8 @@ constexpr uint32_t kPmBeta = 0, kPmRq = 256, kPmRk = 512, kPmOct = 768, kPmBar =
 constexpr uint32_t kPSmemBytes = kPMisc + kPmBar + 32 + 1024;
 constexpr uint32_t kPStageQKA = 16384 + 16384 + 32768;
 constexpr uint32_t kPStageTx = kPStageQKA + 16384;
-constexpr uint32_t kPColA = 0, kPColW = 64, kPColU = 192, kPTmemCols = 256;
+// TMEM columns: [Kt; Qt] Kh^T, W, U'^T, Kg^T W, P W
+constexpr uint32_t kPColA = 0, kPColW = 64, kPColU = 192, kPColN = 256, kPColPW = 384, kPTmemCols = 512;
 
 // element (r, s) of the three Tb tiles, four consecutive s at once (s % 4 == 0)
 __device__ __forceinline__ void put_tb4(uint8_t *tb16, uint8_t *tbh, uint8_t *tbl, int r, int s, float a, float b,
@@ -1104,7 +1121,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
             if (tid == 0) stage_v(v_owed);
             v_owed = -1;
         }
-        // ---- W -> rows 0-63 of [W; Qt] (over Kt); U' -> the record ----
+        // ---- W -> rows 0-63 of [W; Qt] (over Kt); U'^T -> fp16 tile (over Kh) ----
         {
             // M = 64: row 16 sp + i sits in lane i (< 16) of sub-partition sp; the loads are
             // collective, so the whole warp issues them and lanes 0-15 keep the rows
@@ -1126,15 +1143,80 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
             float u[32];
             tmem_ld32(tmem + lane_base + kPColU + 32 * cg, u);
             tmem_wait_ld();
-            float *up = reinterpret_cast<float *>(rec + kRUP) + 32 * sp + lane;  // column d_v
+            const int dv = 32 * sp + lane;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) up[(32 * cg + j) * kDv] = u[j];
+            for (int j = 0; j < 32; j += 8)
+                *reinterpret_cast<uint4 *>(sm + kPKH + sw128_off16(dv, 32 * cg + j, 16384)) =
+                    make_uint4(f32x2_to_f16x2(u[j], u[j + 1]), f32x2_to_f16x2(u[j + 2], u[j + 3]),
+                               f32x2_to_f16x2(u[j + 4], u[j + 5]), f32x2_to_f16x2(u[j + 6], u[j + 7]));
+        }
+        // ---- Kg^T W (both read MN-major) and P W ----
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) {
+            tc_fence_after();
+            const uint64_t kg0 = smem_desc(sbase + kPKG, 8192, 1024, kLayoutSw128);  // MN chunks 8 KiB apart
+            const uint64_t w0 = smem_desc(sbase + kPQW, 16384, 1024, kLayoutSw128);  // MN chunks 16 KiB apart
+#pragma unroll
+            for (int j = 0; j < kC / 16; ++j) {
+                const uint64_t wj = w0 + ((j * 2048) >> 4);
+                tc_mma_f16(tmem + kPColN, kg0 + ((j * 2048) >> 4), wj, kIdescN, j > 0);
+                tc_mma_f16(tmem + kPColPW, kdesc16(d0 + (kPP >> 4), 8192, j), wj, kIdescPW, j > 0);
+            }
+            tc_commit(mma_bar);
+        }
+        ok = mma_wait();
+        if (!ok) break;
+        // ---- N = -Kg^T W -> fp16 tile (over the A / T scratch); Qe = Qt - P W -> fp16 tile (over Tb) ----
+        {
+            const int row = 32 * sp + lane;  // d_k' of N
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int c0 = 64 * cg + 32 * part;
+                float x[32];
+                tmem_ld32(tmem + lane_base + kPColN + c0, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; j += 8)
+                    *reinterpret_cast<uint4 *>(sm + kPA + sw128_off16(row, c0 + j, 16384)) =
+                        make_uint4(f32x2_to_f16x2(-x[j], -x[j + 1]), f32x2_to_f16x2(-x[j + 2], -x[j + 3]),
+                                   f32x2_to_f16x2(-x[j + 4], -x[j + 5]), f32x2_to_f16x2(-x[j + 6], -x[j + 7]));
+            }
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int c0 = 64 * cg + 32 * part;
+                float x[32];
+                tmem_ld32(tmem + lane_base + kPColPW + c0, x);  // M = 64: rows in lanes 0-15
+                tmem_wait_ld();
+                if (lane < 16) {
+                    const int r = 16 * sp + lane;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        const uint4 qv = *reinterpret_cast<const uint4 *>(sm + kPQW + sw128_off16(kC + r, c0 + j, 16384));
+                        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                        uint32_t ow[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 qf = __half22float2(*reinterpret_cast<const __half2 *>(&qw[e]));
+                            ow[e] = f32x2_to_f16x2(qf.x - x[j + 2 * e], qf.y - x[j + 2 * e + 1]);
+                        }
+                        *reinterpret_cast<uint4 *>(sm + kPTB + sw128_off16(r, c0 + j, 8192)) =
+                            make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    }
+                }
+            }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {
-            bulk_s2g(rec, sbase + kPQW, kRTiles);
+            bulk_s2g(rec + kRN, sbase + kPA, 32768);
+            bulk_s2g(rec + kRQE, sbase + kPTB, 16384);
+            bulk_s2g(rec + kRKG, sbase + kPKG, 16384);
+            bulk_s2g(rec + kRP, sbase + kPP, 8192);
+            bulk_s2g(rec + kRU, sbase + kPKH, 16384);
+            bulk_s2g(rec + kRG, sbase + kPG, 512);
             bulk_commit();
         }
     }
@@ -1170,17 +1252,16 @@ struct ChainArgs {
 };
 
 // chain shared memory (offsets from a 1024-aligned base)
-constexpr uint32_t kCS16 = 0;            // S^T [128 d_v][128 d_k] fp16, K-major SW128, 2 blocks x 16 KiB
-constexpr uint32_t kCU16 = 32768;        // U^T [128 d_v][64 tok] fp16, K-major SW128, 16 KiB
-constexpr uint32_t kCRec = 49152;        // two record buffers (the tiles and g_last of a chunk)
-constexpr uint32_t kCRecStride = 58368;  // 57 KiB each (1024-aligned)
-constexpr uint32_t kCO = kCRec + 2 * kCRecStride;  // O [64 tok][128 d_v] bf16 or fp32, plain (TMA store)
-constexpr uint32_t kCMisc = kCO + 32768;
-constexpr uint32_t kCSmemBytes = kCMisc + 64 + 1024;
-// TMEM: the fp32 master S^T (128 lanes = d_v, 128 columns = d_k) and two [X^T | O^T] buffers
-constexpr uint32_t kCColS = 0, kCColXO = 128, kCTmemCols = 512;
+constexpr uint32_t kCS16 = 0;            // S0^T [128 d_v][128 d_k] fp16, K-major SW128, 2 blocks x 16 KiB
+constexpr uint32_t kCRec = 32768;        // two record buffers, each one record (kRecBytes)
+constexpr uint32_t kCRecStride = 91136;  // 89 KiB (1024-aligned); the barriers sit in buffer 0's slack
+constexpr uint32_t kCO = kCRec + 2 * kCRecStride;  // O [64 tok][128 d_v] bf16 (or 32 tokens x fp32), plain
+constexpr uint32_t kCMisc = kCRec + kRecBytes;     // inside buffer 0's last 512 bytes
+constexpr uint32_t kCSmemBytes = kCO + 16384 + 1024;
+static_assert(kCMisc + 64 <= kCRec + kCRecStride, "chain barriers must fit in the record slack");
+// TMEM: the fp32 master S^T (128 lanes = d_v, 128 columns = d_k) and two O^T buffers of 64 columns
+constexpr uint32_t kCColS = 0, kCColO = 128, kCTmemCols = 256;
 
-// One CTA per (sequence, head) walks the segment's chunks with the state master in tensor memory.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int x, int y, int z) {
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
                      reinterpret_cast<uint64_t>(map)),
@@ -1188,7 +1269,11 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
                  : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs p, const __grid_constant__ CUtensorMap omap) {
+// One CTA per (sequence, head) walks the segment's chunks with the state master in tensor memory.
+// omap: the outputs o as a 3-D tensor [B][T][H * 128] (bf16, or fp32 with LAD_FLAG_OUT_FP32),
+// boxes of 128 channels x 64 tokens (32 for fp32, which stores a chunk in two halves).
+__global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs p,
+                                                                     const __grid_constant__ CUtensorMap omap) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -1218,73 +1303,94 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    auto load_rec = [&](int i) {  // chunk i's tiles into buffer i % 2
+    auto load_rec = [&](int i) {  // chunk i's record into buffer i % 2
         const uint32_t bar = rec_bar0 + 8u * static_cast<uint32_t>(i & 1);
-        mbar_arrive_tx_raw(bar, kRTiles);
-        bulk_g2s(sbase + kCRec + static_cast<uint32_t>(i & 1) * kCRecStride, recs + static_cast<size_t>(i) * kRecBytes,
-                 kRTiles, bar);
+        mbar_arrive_tx_raw(bar, kRecBytes);
+        bulk_g2s(sbase + kCRec + static_cast<uint32_t>(i & 1) * kCRecStride,
+                 recs + static_cast<size_t>(i) * kRecBytes, kRecBytes, bar);
     };
     uint32_t pend = p.nseg > 1 ? 3u : 1u;  // bit j: a copy into buffer j is in flight
+    uint32_t rph = 0, mph = 0;             // rph bit j: the phase buffer j's barrier waits for next
     if (tid == 0) {
         load_rec(0);
         if (p.nseg > 1) load_rec(1);
     }
-
-    // U' of chunk i for this thread's value column and tokens 32 cg .. 32 cg + 31
-    auto load_up = [&](float (&u)[32], int i) {
-        const float *src = reinterpret_cast<const float *>(recs + static_cast<size_t>(i) * kRecBytes + kRUP) + dv;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) u[j] = __ldcg(src + (32 * cg + j) * kDv);
+    auto rec_wait = [&](int i) {
+        const int j = i & 1;
+        const bool w = wait_bar(rec_bar0 + 8u * j, (rph >> j) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
+        rph ^= 1u << j;
+        pend &= ~(1u << j);
+        return __syncthreads_and(w) != 0;
     };
-    // the outputs of chunk i (O^T in buffer i % 2, columns 64-127), scaled, into the O tile
-    // [token][d_v] (a TMA store takes it out; rows past T are not written)
-    auto stage_o = [&](int i) {
+    auto gl_of = [&](int i) {  // g_last of chunk i (its record buffer)
+        return reinterpret_cast<const float *>(sm + kCRec + static_cast<uint32_t>(i & 1) * kCRecStride + kRG);
+    };
+    // O of chunk i (O^T in buffer i % 2), scaled, through the O tile and TMA stores; called by all
+    // threads after a barrier that follows the MMAs of chunk i and the previous store's read
+    auto store_o = [&](int i) {
         float x[32];
-        tmem_ld32(tmem + lane_base + kCColXO + static_cast<uint32_t>(i & 1) * 128 + 64 + 32 * cg, x);
+        tmem_ld32(tmem + lane_base + kCColO + static_cast<uint32_t>(i & 1) * 64 + 32 * cg, x);
         tmem_wait_ld();
-        if (p.out_f32) {
-            float *od = reinterpret_cast<float *>(sm + kCO) + dv;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) od[(32 * cg + j) * kDv] = p.scale * x[j];
-        } else {
+        const int t0 = (p.c0 + i) * kC;
+        if (!p.out_f32) {
             uint16_t *od = reinterpret_cast<uint16_t *>(sm + kCO) + dv;
 #pragma unroll
             for (int j = 0; j < 32; ++j) od[(32 * cg + j) * kDv] = lad::dev::f32_to_bf16(p.scale * x[j]);
+            fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tma_store_3d(&omap, sbase + kCO, h * kDv, t0, b);
+                bulk_commit();
+            }
+        } else {
+            // fp32: 32 tokens (16 KiB) at a time, the two column halves one after the other
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                if (cg == half) {
+                    float *od = reinterpret_cast<float *>(sm + kCO) + dv;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) od[j * kDv] = p.scale * x[j];
+                    fence_async_smem();
+                }
+                __syncthreads();
+                if (tid == 0) {
+                    tma_store_3d(&omap, sbase + kCO, h * kDv, t0 + 32 * half, b);
+                    bulk_commit();
+                    bulk_wait_read0();
+                }
+                __syncthreads();
+            }
         }
-        fence_async_smem();
-    };
-    auto store_o = [&](int i) {  // one thread, after a barrier that follows stage_o
-        tma_store_3d(&omap, sbase + kCO, h * kDv, (p.c0 + i) * kC, b);
-        bulk_commit();
     };
 
-    // ---- the state entering the segment: master S^T and its fp16 copy ----
-    {
+    // ---- the state entering the segment: the fp16 copy (S0^T), and the master scaled by chunk
+    //      0's decay, ready for chunk 0's contraction ----
+    bool ok = rec_wait(0);
+    if (ok) {
         const float *S0 = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
+        const float *gl = gl_of(0);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
             const int c0 = 64 * cg + 32 * part;
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = S0[static_cast<size_t>(c0 + j) * kDv];
-            tmem_st32(tmem + lane_base + kCColS + c0, v);
 #pragma unroll
             for (int j = 0; j < 32; j += 8)
                 *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, c0 + j, 16384)) =
                     make_uint4(f32x2_to_f16x2(v[j], v[j + 1]), f32x2_to_f16x2(v[j + 2], v[j + 3]),
                                f32x2_to_f16x2(v[j + 4], v[j + 5]), f32x2_to_f16x2(v[j + 6], v[j + 7]));
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= gl[c0 + j];
+            tmem_st32(tmem + lane_base + kCColS + c0, v);
         }
         tmem_wait_st();
     }
-    float up[32], upn[32];
-    load_up(up, 0);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
-    uint32_t rph = 0, mph = 0;  // rph bit j: the phase buffer j's barrier waits for next
-    bool ok = true;
     auto mma_wait = [&]() {
         const bool w = wait_bar(mma_bar, mph, abort_flag, &g_prefill_error, lad::kErrPrefill);
         mph ^= 1;
@@ -1292,124 +1398,80 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
         return __syncthreads_and(w) != 0;
     };
     for (int i = 0; i < p.nseg && ok; ++i) {
-        const int buf = i & 1;
-        const uint32_t rs = kCRec + static_cast<uint32_t>(buf) * kCRecStride;  // offset of the record tiles
-        const float *gl = reinterpret_cast<const float *>(sm + rs + kRG);
-        const uint32_t xo = tmem + kCColXO + static_cast<uint32_t>(buf) * 128;
-        {
-            const bool w =
-                wait_bar(rec_bar0 + 8u * buf, (rph >> buf) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
-            if (tid == 0) bulk_wait_read0();  // the previous outputs have left the O tile
-            rph ^= 1u << buf;
-            pend &= ~(1u << buf);
-            ok = __syncthreads_and(w) != 0;
-            if (!ok) break;
-        }
-        // ---- [X^T | O^T] = S^T [W; Qt]^T ----
-        if (warp == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < kDk / 16; ++j)
-                tc_mma_f16(xo, kdesc16(d0 + (kCS16 >> 4), 16384, j), kdesc16(d0 + ((rs + kRQW) >> 4), 16384, j),
-                           kIdescXO, j > 0);
-            tc_commit(mma_bar);
-        }
-        // ---- while it runs: the master takes the chunk's decay (column d_k times g_last[d_k]), the
-        //      previous chunk's outputs leave, the next chunk's U' comes into registers ----
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int c0 = 64 * cg + 32 * part;
-            float s[32];
-            tmem_ld32(tmem + lane_base + kCColS + c0, s);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s[j] *= gl[c0 + j];
-            tmem_st32(tmem + lane_base + kCColS + c0, s);
-        }
-        tmem_wait_st();
-        if (i > 0) stage_o(i - 1);
-        if (i + 1 < p.nseg) load_up(upn, i + 1);
-        ok = mma_wait();
-        if (!ok) break;
-        if (i > 0 && tid == 0) store_o(i - 1);
-        // ---- U = U' - X -> the U^T operand (row d_v, this thread's 32 tokens) ----
-        {
-            float x[32];
-            tmem_ld32(xo + lane_base + 32 * cg, x);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; j += 8)
-                *reinterpret_cast<uint4 *>(sm + kCU16 + sw128_off16(dv, 32 * cg + j, 16384)) =
-                    make_uint4(f32x2_to_f16x2(up[j] - x[j], up[j + 1] - x[j + 1]),
-                               f32x2_to_f16x2(up[j + 2] - x[j + 2], up[j + 3] - x[j + 3]),
-                               f32x2_to_f16x2(up[j + 4] - x[j + 4], up[j + 5] - x[j + 5]),
-                               f32x2_to_f16x2(up[j + 6] - x[j + 6], up[j + 7] - x[j + 7]));
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        // ---- S^T += U^T Kg (Kg read MN-major);  O^T += U^T P^T ----
+        const uint32_t rs = kCRec + static_cast<uint32_t>(i & 1) * kCRecStride;  // this chunk's record
+        const uint32_t od = tmem + kCColO + static_cast<uint32_t>(i & 1) * 64;
+        // ---- S^T += U'^T Kg + S0^T N^T;  O^T = U'^T P^T + S0^T Qe^T ----
         if (warp == 0) {
             tc_fence_after();
             const uint64_t kg0 = smem_desc(sbase + rs + kRKG, 8192, 1024, kLayoutSw128);
 #pragma unroll
             for (int j = 0; j < kC / 16; ++j) {
-                const uint64_t ua = kdesc16(d0 + (kCU16 >> 4), 16384, j);
-                tc_mma_f16(tmem + kCColS, ua, kg0 + ((j * 2048) >> 4), kIdescS, 1);
-                tc_mma_f16(xo + 64, ua, kdesc16(d0 + ((rs + kRP) >> 4), 8192, j), kIdescO, 1);
+                const uint64_t ua = kdesc16(d0 + ((rs + kRU) >> 4), 16384, j);
+                tc_mma_f16(tmem + kCColS, ua, kg0 + ((j * 2048) >> 4), kIdescSU, 1);
+                tc_mma_f16(od, ua, kdesc16(d0 + ((rs + kRP) >> 4), 8192, j), kIdescO, j > 0);
+            }
+#pragma unroll
+            for (int j = 0; j < kDk / 16; ++j) {
+                const uint64_t sa = kdesc16(d0 + (kCS16 >> 4), 16384, j);
+                tc_mma_f16(tmem + kCColS, sa, kdesc16(d0 + ((rs + kRN) >> 4), 16384, j), kIdescSN, 1);
+                tc_mma_f16(od, sa, kdesc16(d0 + ((rs + kRQE) >> 4), 8192, j), kIdescO, 1);
             }
             tc_commit(mma_bar);
         }
+        // ---- while they run: the previous chunk's outputs leave ----
+        if (i > 0) store_o(i - 1);
         ok = mma_wait();
         if (!ok) break;
-        // ---- the buffer is free: chunk i + 2's record comes in; chunk i's is dropped from L2 ----
+        // ---- the buffer is free: chunk i + 2's record comes in ----
         if (i + 2 < p.nseg) {
             if (tid == 0) load_rec(i + 2);
-            pend |= 1u << buf;
+            pend |= 1u << (i & 1);
         }
-        // ---- the new state: its fp16 copy for the next chunk, or the state out after the last ----
         const bool last = i == p.nseg - 1;
+        if (!last) {
+            ok = rec_wait(i + 1);  // the next chunk's decay
+            if (!ok) break;
+        }
+        // ---- the new state: its fp16 copy and the next chunk's decay (or the state out) ----
+        const float *gn = last ? nullptr : gl_of(i + 1);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
             const int c0 = 64 * cg + 32 * part;
-            float s[32];
-            tmem_ld32(tmem + lane_base + kCColS + c0, s);
+            float v[32];
+            tmem_ld32(tmem + lane_base + kCColS + c0, v);
             tmem_wait_ld();
             if (last) {
                 float *Sout = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) Sout[static_cast<size_t>(c0 + j) * kDv] = s[j];
+                for (int j = 0; j < 32; ++j) Sout[static_cast<size_t>(c0 + j) * kDv] = v[j];
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; j += 8)
                     *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, c0 + j, 16384)) =
-                        make_uint4(f32x2_to_f16x2(s[j], s[j + 1]), f32x2_to_f16x2(s[j + 2], s[j + 3]),
-                                   f32x2_to_f16x2(s[j + 4], s[j + 5]), f32x2_to_f16x2(s[j + 6], s[j + 7]));
+                        make_uint4(f32x2_to_f16x2(v[j], v[j + 1]), f32x2_to_f16x2(v[j + 2], v[j + 3]),
+                                   f32x2_to_f16x2(v[j + 4], v[j + 5]), f32x2_to_f16x2(v[j + 6], v[j + 7]));
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] *= gn[c0 + j];
+                tmem_st32(tmem + lane_base + kCColS + c0, v);
             }
         }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) up[j] = upn[j];
+        tmem_wait_st();
+        if (tid == 0) bulk_wait_read0();  // the previous outputs have left the O tile
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (last) {
-            if (tid == 0) bulk_wait_read0();
-            __syncthreads();
-            stage_o(i);
-            __syncthreads();
-            if (tid == 0) store_o(i);
-        }
+        if (last) store_o(i);
     }
-    // drain: record copies still in flight (after an abort) land and every MMA this CTA issued
-    // completes, before shared memory and TMEM are released
+    // drain: record copies still in flight (after an abort) land, the output stores complete and
+    // every MMA this CTA issued completes, before shared memory and TMEM are released
     if (tid == 0) {
         const uint64_t t0 = lad::dev::globaltimer_ns();
         for (int j = 0; j < 2; ++j)
             while (((pend >> j) & 1u) && !mbar_try_wait(rec_bar0 + 8u * j, (rph >> j) & 1u) &&
                    lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
             }
+        bulk_wait_all();
     }
-    if (tid == 0) bulk_wait_all();  // the output stores have completed
     if (warp == 0) {
         tc_commit(mma_bar);
         const uint64_t t0 = lad::dev::globaltimer_ns();
@@ -1493,12 +1555,13 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
            (flags & LAD_FLAG_L2NORM_QK) ? 1 : 0, f32 ? 1 : 0};
     auto enc = reinterpret_cast<EncodeTiledFn>(lad::tensor_map_encoder_raw());
     if (!enc) return set_error(LAD_ECUDA, "kda_prefill_chunked: cuTensorMapEncodeTiled unavailable");
-    auto make = [&](CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int box0, bool sw128) -> int {
+    auto make = [&](CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int box0, bool sw128,
+                    int box1 = kC) -> int {
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(H) * kDk, static_cast<cuuint64_t>(T),
                                     static_cast<cuuint64_t>(B)};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * kDk * esize,
                                        static_cast<cuuint64_t>(T) * H * kDk * esize};
-        const cuuint32_t box[3] = {static_cast<cuuint32_t>(box0), static_cast<cuuint32_t>(kC), 1};
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(box0), static_cast<cuuint32_t>(box1), 1};
         const cuuint32_t estr[3] = {1, 1, 1};
         CUresult r = enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -1525,7 +1588,7 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
     CUtensorMap omap;
     if (rc == LAD_OK)
         rc = make(&omap, o, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 ? 4 : 2, kDv,
-                  false);
+                  false, f32 ? kC / 2 : kC);
     if (rc != LAD_OK) return rc;
     const int nch = (T + kC - 1) / kC;
     const int sms = lad::device_sm_count();

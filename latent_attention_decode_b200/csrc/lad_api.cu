@@ -63,13 +63,15 @@ extern "C" int lad_device_error(void *stream, int *code) {
     cudaStream_t s = lad::as_stream(stream);
     cudaError_t e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return lad::set_error(LAD_ECUDA, "lad_device_error: %s", cudaGetErrorString(e));
-    int c1 = 0, c2 = 0, c3 = 0;
+    int c1 = 0, c2 = 0, c3 = 0, c4 = 0;
     int rc = lad::take_device_error_mla(s, &c1);
     if (rc != LAD_OK) return rc;
     rc = lad::take_device_error_prefill(s, &c2);
     if (rc != LAD_OK) return rc;
     rc = lad::take_device_error_cache(s, &c3);
     if (rc != LAD_OK) return rc;
-    *code = c1 ? c1 : (c2 ? c2 : c3);
+    rc = lad::take_device_error_kda(s, &c4);
+    if (rc != LAD_OK) return rc;
+    *code = c1 ? c1 : (c2 ? c2 : (c3 ? c3 : c4));
     return LAD_OK;
 }

@@ -40,12 +40,14 @@ enum DeviceErrorTag : int {
     kErrMlaConvert = 0x107,     // FP8-cache call: the widening warps gave up a wait
     kErrCacheAppend = 0x301,    // mla_cache_append: a position with no row to write (not a wait)
     kErrPrefill = 0x201,
+    kErrKdaPair = 0x501,        // KDA decode, two heads per CTA: the second head's state copy never landed
 };
 
 // Host-side readers of the per-module device error words (each clears its word).
 int take_device_error_mla(cudaStream_t s, int *code);
 int take_device_error_prefill(cudaStream_t s, int *code);
 int take_device_error_cache(cudaStream_t s, int *code);
+int take_device_error_kda(cudaStream_t s, int *code);
 
 // pow(theta, -2i/d) for the d/2 RoPE pairs, on the host (the oracle computes them the same way)
 void rope_inverse_frequencies(double theta, int d_rope, double *out);
