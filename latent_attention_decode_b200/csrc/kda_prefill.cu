@@ -738,15 +738,25 @@ __device__ __forceinline__ void put_tb4(uint8_t *tb16, uint8_t *tbh, uint8_t *tb
 __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_beta, uint8_t *tb16, uint8_t *tbh,
                                           uint8_t *tbl, int tid) {
     if (tid < kC) {
-        // column c of (I + A_ii)^-1: t_r = [r == c] - sum_{c <= s < r} A_rs t_s
+        // column c of (I + A_ii)^-1: t_r = [r == c] - sum_{s < r} A_rs t_s (t_s = 0 for s < c); a
+        // row of the block comes in four 16-byte loads, and two partial sums halve the FMA chain
         const int i0 = 16 * (tid >> 4), c = tid & 15;
         float t[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            float acc = 0.f;
+            const float4 *arow = reinterpret_cast<const float4 *>(sA + (i0 + r) * kAS + i0);
+            float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int s2 = 0; s2 < r; ++s2) acc = fmaf(sA[(i0 + r) * kAS + i0 + s2], t[s2], acc);
-            t[r] = r < c ? 0.f : (r == c ? 1.f : -acc);
+            for (int q4 = 0; q4 < 4; ++q4) {
+                if (4 * q4 < r) {
+                    const float4 a = arow[q4];
+                    acc0 = fmaf(a.x, t[4 * q4], acc0);
+                    if (4 * q4 + 1 < r) acc1 = fmaf(a.y, t[4 * q4 + 1], acc1);
+                    if (4 * q4 + 2 < r) acc0 = fmaf(a.z, t[4 * q4 + 2], acc0);
+                    if (4 * q4 + 3 < r) acc1 = fmaf(a.w, t[4 * q4 + 3], acc1);
+                }
+            }
+            t[r] = r < c ? 0.f : (r == c ? 1.f : -(acc0 + acc1));
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) sT[(i0 + r) * kAS + i0 + c] = t[r];
