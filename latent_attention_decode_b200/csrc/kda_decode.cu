@@ -87,7 +87,11 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // every state byte of the launch is requested at once; the second head then runs from shared
 // memory while the first head's stores drain. The copy's wait is bounded: if it runs out, the
 // second head is left untouched and device error 0x501 is recorded.
-constexpr int kPairSmemBytes = kRowsPerWarp * kThreads * 16;  // 64 KiB of state slots
+// dynamic shared memory of the paired kernel: the second head's 64 KiB state, then its copy's
+// mbarrier and abort flag, the whole region aligned to 128 bytes by hand (the dynamic region
+// starts wherever the static shared variables end, which need not be 16-byte aligned)
+constexpr int kPairStateBytes = kD * kD * 4;
+constexpr int kPairSmemBytes = kPairStateBytes + 16 + 128;
 
 template <bool kOutF32, bool kFusedConv, bool kPair>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -96,7 +100,7 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
                   float *__restrict__ S, void *__restrict__ o, int H, float scale, int l2norm, ConvIn cv,
                   GateIn gi, int units) {
     constexpr int kUnits = kPair ? 2 : 1;
-    extern __shared__ __align__(16) uint8_t pair_slots[];  // kPair: the second head's state
+    extern __shared__ uint8_t pair_raw[];  // kPair: the second head's state (aligned below)
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int bh0 = blockIdx.x;
@@ -114,11 +118,12 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) s[r] = __ldcs(mine + r * kVec);
     }
-    __shared__ __align__(8) uint64_t pair_bar;
-    __shared__ int pair_abort;
-    const uint32_t bar = static_cast<uint32_t>(__cvta_generic_to_shared(&pair_bar));
+    uint8_t *pair_slots =
+        reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(pair_raw) + 127) & ~static_cast<uintptr_t>(127));
+    const uint32_t bar = static_cast<uint32_t>(__cvta_generic_to_shared(pair_slots + kPairStateBytes));
+    volatile int *pair_abort = reinterpret_cast<volatile int *>(pair_slots + kPairStateBytes + 8);
     if (has1 && threadIdx.x == 0) {
-        pair_abort = 0;
+        *pair_abort = 0;
         lad::ptx::mbar_init(bar, 1);
         lad::ptx::mbar_fence_init();
         lad::ptx::mbar_arrive_tx_raw(bar, kD * kD * 4);
@@ -289,7 +294,7 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
         if (has1) {
             // the second head from shared memory (the state's own layout: this thread's rows and
             // float4 of columns), then a barrier before the reduction buffers and gate inputs are reused
-            const bool landed = lad::ptx::wait_bar(bar, 0, &pair_abort, &g_kda_error, lad::kErrKdaPair);
+            const bool landed = lad::ptx::wait_bar(bar, 0, pair_abort, &g_kda_error, lad::kErrKdaPair);
             const float4 *rows = reinterpret_cast<const float4 *>(pair_slots) +
                                  static_cast<size_t>(warp * kRowsPerWarp) * kVec + lane;
 #pragma unroll

@@ -1266,7 +1266,8 @@ constexpr uint32_t kCS16 = 0;            // S0^T [128 d_v][128 d_k] fp16, K-majo
 constexpr uint32_t kCRec = 32768;        // two record buffers, each one record (kRecBytes)
 constexpr uint32_t kCRecStride = 91136;  // 89 KiB (1024-aligned); the barriers sit in buffer 0's slack
 constexpr uint32_t kCO = kCRec + 2 * kCRecStride;  // O [64 tok][128 d_v] bf16 (or 32 tokens x fp32), plain
-constexpr uint32_t kCMisc = kCRec + kRecBytes;     // inside buffer 0's last 512 bytes
+constexpr uint32_t kCMisc = kCRec + kRecBytes;     // inside buffer 0's last 512 bytes: 2 record
+                                                   // barriers, state and output MMA barriers, TMEM slot, abort
 constexpr uint32_t kCSmemBytes = kCO + 16384 + 1024;
 static_assert(kCMisc + 64 <= kCRec + kCRecStride, "chain barriers must fit in the record slack");
 // TMEM: the fp32 master S^T (128 lanes = d_v, 128 columns = d_k) and two O^T buffers of 64 columns
@@ -1282,19 +1283,26 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
 // One CTA per (sequence, head) walks the segment's chunks with the state master in tensor memory.
 // omap: the outputs o as a 3-D tensor [B][T][H * 128] (bf16, or fp32 with LAD_FLAG_OUT_FP32),
 // boxes of 128 channels x 64 tokens (32 for fp32, which stores a chunk in two halves).
-__global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs p,
-                                                                     const __grid_constant__ CUtensorMap omap) {
+// Warps 0-7 own the master's rows (warp w: lanes 32 (w % 4) .., columns half w / 4); warp 8 issues
+// the MMAs and the record copies: per chunk the state part first (its own commit, which the master
+// pass waits for), then the output part, whose completion warp 8 waits for before the iteration's
+// closing barrier (so the next iteration may read those outputs without a wait of its own).
+constexpr int kChainThreads = kThreads + 32;
+
+__global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(ChainArgs p,
+                                                                          const __grid_constant__ CUtensorMap omap) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
-    const uint32_t rec_bar0 = sbase + kCMisc, mma_bar = sbase + kCMisc + 16;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kCMisc + 24);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kCMisc + 28);
+    const uint32_t rec_bar0 = sbase + kCMisc, mbar_s = sbase + kCMisc + 16, mbar_o = sbase + kCMisc + 24;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kCMisc + 32);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kCMisc + 36);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int sp = warp & 3, cg = warp >> 2;
+    const bool issuer = warp == kThreads / 32;  // warp 8
+    const int sp = warp & 3, cg = (warp >> 2) & 1;
     const uint32_t lane_base = static_cast<uint32_t>(32 * sp) << 16;
-    const int dv = 32 * sp + lane;  // this thread's row of S^T: a value column
+    const int dv = 32 * sp + lane;  // this thread's row of S^T: a value column (warps 0-7)
     const int bh = blockIdx.x;
     const int b = bh / p.H, h = bh - b * p.H;
     const uint8_t *recs = p.ws + static_cast<size_t>(bh) * p.nseg * kRecBytes;
@@ -1303,7 +1311,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
     if (tid == 0) {
         mbar_init(rec_bar0, 1);
         mbar_init(rec_bar0 + 8, 1);
-        mbar_init(mma_bar, 1);
+        mbar_init(mbar_s, 1);
+        mbar_init(mbar_o, 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -1313,30 +1322,29 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    auto load_rec = [&](int i) {  // chunk i's record into buffer i % 2
+    auto load_rec = [&](int i) {  // chunk i's record into buffer i % 2 (one thread)
         const uint32_t bar = rec_bar0 + 8u * static_cast<uint32_t>(i & 1);
         mbar_arrive_tx_raw(bar, kRecBytes);
         bulk_g2s(sbase + kCRec + static_cast<uint32_t>(i & 1) * kCRecStride,
                  recs + static_cast<size_t>(i) * kRecBytes, kRecBytes, bar);
     };
-    uint32_t pend = p.nseg > 1 ? 3u : 1u;  // bit j: a copy into buffer j is in flight
-    uint32_t rph = 0, mph = 0;             // rph bit j: the phase buffer j's barrier waits for next
-    if (tid == 0) {
+    uint32_t pend = p.nseg > 1 ? 3u : 1u;  // bit j: a copy into buffer j is in flight (issuer's view)
+    if (issuer && lane == 0) {
         load_rec(0);
         if (p.nseg > 1) load_rec(1);
     }
-    auto rec_wait = [&](int i) {
+    // waits by the calling warp (bounded; warp-uniform result); chunk i's record has landed
+    auto rec_ready = [&](int i) {
         const int j = i & 1;
-        const bool w = wait_bar(rec_bar0 + 8u * j, (rph >> j) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
-        rph ^= 1u << j;
-        pend &= ~(1u << j);
-        return __syncthreads_and(w) != 0;
+        return wait_bar(rec_bar0 + 8u * j, static_cast<uint32_t>(i >> 1) & 1u, abort_flag, &g_prefill_error,
+                        lad::kErrPrefill);
     };
     auto gl_of = [&](int i) {  // g_last of chunk i (its record buffer)
         return reinterpret_cast<const float *>(sm + kCRec + static_cast<uint32_t>(i & 1) * kCRecStride + kRG);
     };
-    // O of chunk i (O^T in buffer i % 2), scaled, through the O tile and TMA stores; called by all
-    // threads after a barrier that follows the MMAs of chunk i and the previous store's read
+    auto bar256 = []() { asm volatile("bar.sync 1, 256;" ::: "memory"); };  // warps 0-7 only
+    // O of chunk i (O^T in buffer i % 2, complete), scaled, through the O tile and TMA stores;
+    // warps 0-7, the previous store having read the tile
     auto store_o = [&](int i) {
         float x[32];
         tmem_ld32(tmem + lane_base + kCColO + static_cast<uint32_t>(i & 1) * 64 + 32 * cg, x);
@@ -1347,7 +1355,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
 #pragma unroll
             for (int j = 0; j < 32; ++j) od[(32 * cg + j) * kDv] = lad::dev::f32_to_bf16(p.scale * x[j]);
             fence_async_smem();
-            __syncthreads();
+            bar256();
             if (tid == 0) {
                 tma_store_3d(&omap, sbase + kCO, h * kDv, t0, b);
                 bulk_commit();
@@ -1362,132 +1370,144 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_chain_kernel(ChainArgs 
                     for (int j = 0; j < 32; ++j) od[j * kDv] = p.scale * x[j];
                     fence_async_smem();
                 }
-                __syncthreads();
+                bar256();
                 if (tid == 0) {
                     tma_store_3d(&omap, sbase + kCO, h * kDv, t0 + 32 * half, b);
                     bulk_commit();
                     bulk_wait_read0();
                 }
-                __syncthreads();
+                bar256();
             }
         }
     };
 
     // ---- the state entering the segment: the fp16 copy (S0^T), and the master scaled by chunk
     //      0's decay, ready for chunk 0's contraction ----
-    bool ok = rec_wait(0);
-    if (ok) {
-        const float *S0 = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
-        const float *gl = gl_of(0);
+    bool ok = true;
+    if (!issuer) {
+        ok = rec_ready(0);
+        if (ok) {
+            const float *S0 = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
+            const float *gl = gl_of(0);
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int c0 = 64 * cg + 32 * part;
-            float v[32];
+            for (int part = 0; part < 2; ++part) {
+                const int c0 = 64 * cg + 32 * part;
+                float v[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = S0[static_cast<size_t>(c0 + j) * kDv];
-#pragma unroll
-            for (int j = 0; j < 32; j += 8)
-                *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, c0 + j, 16384)) =
-                    make_uint4(f32x2_to_f16x2(v[j], v[j + 1]), f32x2_to_f16x2(v[j + 2], v[j + 3]),
-                               f32x2_to_f16x2(v[j + 4], v[j + 5]), f32x2_to_f16x2(v[j + 6], v[j + 7]));
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= gl[c0 + j];
-            tmem_st32(tmem + lane_base + kCColS + c0, v);
-        }
-        tmem_wait_st();
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    auto mma_wait = [&]() {
-        const bool w = wait_bar(mma_bar, mph, abort_flag, &g_prefill_error, lad::kErrPrefill);
-        mph ^= 1;
-        tc_fence_after();
-        return __syncthreads_and(w) != 0;
-    };
-    for (int i = 0; i < p.nseg && ok; ++i) {
-        const uint32_t rs = kCRec + static_cast<uint32_t>(i & 1) * kCRecStride;  // this chunk's record
-        const uint32_t od = tmem + kCColO + static_cast<uint32_t>(i & 1) * 64;
-        // ---- S^T += U'^T Kg + S0^T N^T;  O^T = U'^T P^T + S0^T Qe^T ----
-        if (warp == 0) {
-            tc_fence_after();
-            const uint64_t kg0 = smem_desc(sbase + rs + kRKG, 8192, 1024, kLayoutSw128);
-#pragma unroll
-            for (int j = 0; j < kC / 16; ++j) {
-                const uint64_t ua = kdesc16(d0 + ((rs + kRU) >> 4), 16384, j);
-                tc_mma_f16(tmem + kCColS, ua, kg0 + ((j * 2048) >> 4), kIdescSU, 1);
-                tc_mma_f16(od, ua, kdesc16(d0 + ((rs + kRP) >> 4), 8192, j), kIdescO, j > 0);
-            }
-#pragma unroll
-            for (int j = 0; j < kDk / 16; ++j) {
-                const uint64_t sa = kdesc16(d0 + (kCS16 >> 4), 16384, j);
-                tc_mma_f16(tmem + kCColS, sa, kdesc16(d0 + ((rs + kRN) >> 4), 16384, j), kIdescSN, 1);
-                tc_mma_f16(od, sa, kdesc16(d0 + ((rs + kRQE) >> 4), 8192, j), kIdescO, 1);
-            }
-            tc_commit(mma_bar);
-        }
-        // ---- while they run: the previous chunk's outputs leave ----
-        if (i > 0) store_o(i - 1);
-        ok = mma_wait();
-        if (!ok) break;
-        // ---- the buffer is free: chunk i + 2's record comes in ----
-        if (i + 2 < p.nseg) {
-            if (tid == 0) load_rec(i + 2);
-            pend |= 1u << (i & 1);
-        }
-        const bool last = i == p.nseg - 1;
-        if (!last) {
-            ok = rec_wait(i + 1);  // the next chunk's decay
-            if (!ok) break;
-        }
-        // ---- the new state: its fp16 copy and the next chunk's decay (or the state out) ----
-        const float *gn = last ? nullptr : gl_of(i + 1);
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int c0 = 64 * cg + 32 * part;
-            float v[32];
-            tmem_ld32(tmem + lane_base + kCColS + c0, v);
-            tmem_wait_ld();
-            if (last) {
-                float *Sout = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) Sout[static_cast<size_t>(c0 + j) * kDv] = v[j];
-            } else {
+                for (int j = 0; j < 32; ++j) v[j] = S0[static_cast<size_t>(c0 + j) * kDv];
 #pragma unroll
                 for (int j = 0; j < 32; j += 8)
                     *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, c0 + j, 16384)) =
                         make_uint4(f32x2_to_f16x2(v[j], v[j + 1]), f32x2_to_f16x2(v[j + 2], v[j + 3]),
                                    f32x2_to_f16x2(v[j + 4], v[j + 5]), f32x2_to_f16x2(v[j + 6], v[j + 7]));
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] *= gn[c0 + j];
+                for (int j = 0; j < 32; ++j) v[j] *= gl[c0 + j];
                 tmem_st32(tmem + lane_base + kCColS + c0, v);
             }
+            tmem_wait_st();
         }
-        tmem_wait_st();
-        if (tid == 0) bulk_wait_read0();  // the previous outputs have left the O tile
+    }
+    fence_async_smem();
+    tc_fence_before();
+    ok = __syncthreads_and(ok) != 0;
+    tc_fence_after();
+
+    for (int i = 0; i < p.nseg && ok; ++i) {
+        const uint32_t rs = kCRec + static_cast<uint32_t>(i & 1) * kCRecStride;  // this chunk's record
+        const uint32_t od = tmem + kCColO + static_cast<uint32_t>(i & 1) * 64;
+        const bool last = i == p.nseg - 1;
+        bool w = true;
+        if (issuer) {
+            // ---- S^T += U'^T Kg + S0^T N^T (commit: the master pass may start);
+            //      O^T = U'^T P^T + S0^T Qe^T (commit: waited for here) ----
+            tc_fence_after();
+            const uint64_t kg0 = smem_desc(sbase + rs + kRKG, 8192, 1024, kLayoutSw128);
+            const uint64_t ua0 = d0 + ((rs + kRU) >> 4), sa0 = d0 + (kCS16 >> 4);
+#pragma unroll
+            for (int j = 0; j < kC / 16; ++j)
+                tc_mma_f16(tmem + kCColS, kdesc16(ua0, 16384, j), kg0 + ((j * 2048) >> 4), kIdescSU, 1);
+#pragma unroll
+            for (int j = 0; j < kDk / 16; ++j)
+                tc_mma_f16(tmem + kCColS, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRN) >> 4), 16384, j),
+                           kIdescSN, 1);
+            tc_commit(mbar_s);
+#pragma unroll
+            for (int j = 0; j < kC / 16; ++j)
+                tc_mma_f16(od, kdesc16(ua0, 16384, j), kdesc16(d0 + ((rs + kRP) >> 4), 8192, j), kIdescO, j > 0);
+#pragma unroll
+            for (int j = 0; j < kDk / 16; ++j)
+                tc_mma_f16(od, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRQE) >> 4), 8192, j), kIdescO, 1);
+            tc_commit(mbar_o);
+            // every MMA of the chunk is complete: its record buffer takes chunk i + 2's
+            w = wait_bar(mbar_o, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            if (w && i + 2 < p.nseg) {
+                if (lane == 0) load_rec(i + 2);
+                pend |= 1u << (i & 1);
+            }
+        } else {
+            // ---- while they run: the previous chunk's outputs leave ----
+            if (i > 0) store_o(i - 1);
+            w = wait_bar(mbar_s, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            if (w && !last) w = rec_ready(i + 1);  // the next chunk's decay
+            tc_fence_after();
+            if (w) {
+                // ---- the new state: its fp16 copy and the next chunk's decay (or the state out) ----
+                float v[64];
+                tmem_ld32(tmem + lane_base + kCColS + 64 * cg, *reinterpret_cast<float(*)[32]>(v));
+                tmem_ld32(tmem + lane_base + kCColS + 64 * cg + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                tmem_wait_ld();
+                if (last) {
+                    float *Sout = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) Sout[static_cast<size_t>(64 * cg + j) * kDv] = v[j];
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; j += 8)
+                        *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, 64 * cg + j, 16384)) =
+                            make_uint4(f32x2_to_f16x2(v[j], v[j + 1]), f32x2_to_f16x2(v[j + 2], v[j + 3]),
+                                       f32x2_to_f16x2(v[j + 4], v[j + 5]), f32x2_to_f16x2(v[j + 6], v[j + 7]));
+                    const float4 *gn = reinterpret_cast<const float4 *>(gl_of(i + 1) + 64 * cg);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float4 g4 = gn[j];
+                        v[4 * j] *= g4.x;
+                        v[4 * j + 1] *= g4.y;
+                        v[4 * j + 2] *= g4.z;
+                        v[4 * j + 3] *= g4.w;
+                    }
+                    tmem_st32(tmem + lane_base + kCColS + 64 * cg, *reinterpret_cast<float(*)[32]>(v));
+                    tmem_st32(tmem + lane_base + kCColS + 64 * cg + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                    tmem_wait_st();
+                }
+            }
+            if (tid == 0) bulk_wait_read0();  // the previous outputs have left the O tile
+        }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
-        if (last) store_o(i);
+        ok = __syncthreads_and(w) != 0;
+        tc_fence_after();
+        if (ok && last && !issuer) store_o(i);
     }
     // drain: record copies still in flight (after an abort) land, the output stores complete and
     // every MMA this CTA issued completes, before shared memory and TMEM are released
-    if (tid == 0) {
+    if (issuer && lane == 0) {
         const uint64_t t0 = lad::dev::globaltimer_ns();
-        for (int j = 0; j < 2; ++j)
-            while (((pend >> j) & 1u) && !mbar_try_wait(rec_bar0 + 8u * j, (rph >> j) & 1u) &&
+        for (int j = 0; j < 2; ++j) {
+            // the last copy into buffer j was for chunk nseg - 1 - ((nseg - 1 - j) & 1) ... wait on the
+            // phase of the newest chunk that used buffer j
+            const int newest = ((p.nseg - 1) & 1) == j ? p.nseg - 1 : p.nseg - 2;
+            if (newest < 0) continue;
+            while (((pend >> j) & 1u) && !mbar_try_wait(rec_bar0 + 8u * j, static_cast<uint32_t>(newest >> 1) & 1u) &&
                    lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
             }
-        bulk_wait_all();
-    }
-    if (warp == 0) {
-        tc_commit(mma_bar);
-        const uint64_t t0 = lad::dev::globaltimer_ns();
-        while (!mbar_try_wait(mma_bar, mph) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+        }
+        tc_commit(mbar_o);  // a fresh completion covering every MMA issued
+        const uint64_t t1 = lad::dev::globaltimer_ns();
+        while (!mbar_try_wait(mbar_o, static_cast<uint32_t>(p.nseg) & 1u) &&
+               lad::dev::globaltimer_ns() - t1 < lad::dev::kWaitLimitNs) {
         }
     }
+    if (tid == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1611,7 +1631,7 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
         kda_chunk_prep_kernel<<<pg, kThreads, kPSmemBytes, st>>>(PrepArgs{beta, ws, B, T, H, c0, nseg, a.l2norm}, pm);
         rc = lad::check_launch("kda_prefill_chunked");
         if (rc != LAD_OK) return rc;
-        kda_chunk_chain_kernel<<<static_cast<unsigned>(B * H), kThreads, kCSmemBytes, st>>>(
+        kda_chunk_chain_kernel<<<static_cast<unsigned>(B * H), kChainThreads, kCSmemBytes, st>>>(
             ChainArgs{S, o, ws, B, T, H, c0, nseg, scale, a.out_f32}, omap);
         rc = lad::check_launch("kda_prefill_chunked");
         if (rc != LAD_OK) return rc;
