@@ -1490,22 +1490,28 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
     }
     // drain: record copies still in flight (after an abort) land, the output stores complete and
     // every MMA this CTA issued completes, before shared memory and TMEM are released
-    if (issuer && lane == 0) {
-        const uint64_t t0 = lad::dev::globaltimer_ns();
-        for (int j = 0; j < 2; ++j) {
-            // the last copy into buffer j was for chunk nseg - 1 - ((nseg - 1 - j) & 1) ... wait on the
-            // phase of the newest chunk that used buffer j
-            const int newest = ((p.nseg - 1) & 1) == j ? p.nseg - 1 : p.nseg - 2;
-            if (newest < 0) continue;
-            while (((pend >> j) & 1u) && !mbar_try_wait(rec_bar0 + 8u * j, static_cast<uint32_t>(newest >> 1) & 1u) &&
-                   lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+    if (issuer) {
+        if (lane == 0) {
+            const uint64_t t0 = lad::dev::globaltimer_ns();
+            for (int j = 0; j < 2; ++j) {
+                // wait on the phase of the newest chunk that used buffer j
+                const int newest = ((p.nseg - 1) & 1) == j ? p.nseg - 1 : p.nseg - 2;
+                if (newest < 0) continue;
+                while (((pend >> j) & 1u) &&
+                       !mbar_try_wait(rec_bar0 + 8u * j, static_cast<uint32_t>(newest >> 1) & 1u) &&
+                       lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+                }
             }
         }
-        tc_commit(mbar_o);  // a fresh completion covering every MMA issued
-        const uint64_t t1 = lad::dev::globaltimer_ns();
-        while (!mbar_try_wait(mbar_o, static_cast<uint32_t>(p.nseg) & 1u) &&
-               lad::dev::globaltimer_ns() - t1 < lad::dev::kWaitLimitNs) {
+        __syncwarp();
+        tc_commit(mbar_o);  // warp-wide (elect.sync): a fresh completion covering every MMA issued
+        if (lane == 0) {
+            const uint64_t t1 = lad::dev::globaltimer_ns();
+            while (!mbar_try_wait(mbar_o, static_cast<uint32_t>(p.nseg) & 1u) &&
+                   lad::dev::globaltimer_ns() - t1 < lad::dev::kWaitLimitNs) {
+            }
         }
+        __syncwarp();
     }
     if (tid == 0) bulk_wait_all();
     tc_fence_before();
