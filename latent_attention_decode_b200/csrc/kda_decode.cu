@@ -139,48 +139,91 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
     __shared__ uint2 s_gate[kVec];   // output gate logits, 4 bf16 per lane of warp 0
     __shared__ float4 s_gw[kVec];    // norm weight, 4 per lane of warp 0
 
-    // this head's q, k, v (through the fused conv, or as given) and alpha into slot u
-    auto inputs = [&](int u, int bh) {
-        const int b = bh / H, h = bh - b * H;
+    // the heads' q, k, v (through the fused conv, or as given) and alpha into their slots. With the
+    // fused conv, every input of every conv this thread does (q and k channels for threads 0-127, v
+    // channels for 128-255, of each of the CTA's heads) is loaded first, and only then are the
+    // outputs computed and the tails shifted: a tail store must not come between two convs' loads,
+    // or each conv would wait a full memory round trip behind the state stream
+    auto inputs = [&]() {
+        const int nheads = has1 ? 2 : 1;
         if constexpr (kFusedConv) {
-            // y = taps . (tail, x) (+ bias), SiLU; kept in fp32; the tail shifts in place. Threads
-            // 0-127 take this head's q and k channels, threads 128-255 its v channels.
             const size_t cch = static_cast<size_t>(3) * H * kD;
-            const uint16_t *xb = cv.x + static_cast<size_t>(b) * cch;
-            uint16_t *tb = cv.tail + static_cast<size_t>(b) * 3 * cch;
-            auto conv = [&](size_t c) -> float {
-                const uint16_t xr = xb[c], t0 = tb[c], t1 = tb[cch + c], t2 = tb[2 * cch + c];
-                const uint2 wv = *reinterpret_cast<const uint2 *>(cv.w + c * 4);
-                const float2 w01 = lad::dev::bf16x2_to_f32(wv.x), w23 = lad::dev::bf16x2_to_f32(wv.y);
-                float acc = w01.x * bf16_to_f32(t0);
-                acc = fmaf(w01.y, bf16_to_f32(t1), acc);
-                acc = fmaf(w23.x, bf16_to_f32(t2), acc);
-                acc = fmaf(w23.y, bf16_to_f32(xr), acc);
-                if (cv.bias) acc += bf16_to_f32(cv.bias[c]);
-                if (cv.silu) acc = acc / (1.f + expf(-acc));
-                tb[c] = t1;
-                tb[cch + c] = t2;
-                tb[2 * cch + c] = xr;
-                return acc;
-            };
-            const size_t hc = static_cast<size_t>(h) * kD;
-            if (threadIdx.x < kD) {
-                const int i = threadIdx.x;
-                sq[u][i] = conv(hc + i);
-                sk[u][i] = conv(static_cast<size_t>(H) * kD + hc + i);
-                sa[u][i] = alpha[static_cast<size_t>(bh) * kD + i];
-            } else {
-                const int i = threadIdx.x - kD;
-                sv[u][i] = conv(static_cast<size_t>(2) * H * kD + hc + i);
+            const bool qk = threadIdx.x < kD;
+            const int i = qk ? threadIdx.x : threadIdx.x - kD;
+            uint16_t xr[kUnits][2], t0[kUnits][2], t1[kUnits][2], t2[kUnits][2], bs[kUnits][2];
+            uint2 wv[kUnits][2];
+            float al[kUnits];
+            size_t chan[kUnits][2];
+#pragma unroll
+            for (int u = 0; u < kUnits; ++u) {
+                if (u < nheads) {
+                    const int bh = u == 0 ? bh0 : bh1;
+                    const int b = bh / H, h = bh - b * H;
+                    const size_t hc = static_cast<size_t>(h) * kD;
+                    const uint16_t *xb = cv.x + static_cast<size_t>(b) * cch;
+                    const uint16_t *tb = cv.tail + static_cast<size_t>(b) * 3 * cch;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        if (j == 0 || qk) {
+                            const size_t c = qk ? static_cast<size_t>(j) * H * kD + hc + i
+                                                : static_cast<size_t>(2) * H * kD + hc + i;
+                            chan[u][j] = static_cast<size_t>(b) * cch + c;
+                            xr[u][j] = xb[c];
+                            t0[u][j] = tb[c];
+                            t1[u][j] = tb[cch + c];
+                            t2[u][j] = tb[2 * cch + c];
+                            wv[u][j] = *reinterpret_cast<const uint2 *>(cv.w + c * 4);
+                            bs[u][j] = cv.bias ? cv.bias[c] : static_cast<uint16_t>(0);
+                        }
+                    }
+                    al[u] = qk ? alpha[static_cast<size_t>(bh) * kD + i] : 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kUnits; ++u) {
+                if (u < nheads) {
+                    const int b = (u == 0 ? bh0 : bh1) / H;
+                    uint16_t *tb = cv.tail + static_cast<size_t>(b) * 3 * cch;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        if (j == 0 || qk) {
+                            // y = taps . (tail, x) (+ bias), SiLU; kept in fp32; the tail shifts in place
+                            const float2 w01 = lad::dev::bf16x2_to_f32(wv[u][j].x),
+                                         w23 = lad::dev::bf16x2_to_f32(wv[u][j].y);
+                            float acc = w01.x * bf16_to_f32(t0[u][j]);
+                            acc = fmaf(w01.y, bf16_to_f32(t1[u][j]), acc);
+                            acc = fmaf(w23.x, bf16_to_f32(t2[u][j]), acc);
+                            acc = fmaf(w23.y, bf16_to_f32(xr[u][j]), acc);
+                            if (cv.bias) acc += bf16_to_f32(bs[u][j]);
+                            if (cv.silu) acc = acc / (1.f + expf(-acc));
+                            const size_t c = chan[u][j] - static_cast<size_t>(b) * cch;
+                            tb[c] = t1[u][j];
+                            tb[cch + c] = t2[u][j];
+                            tb[2 * cch + c] = xr[u][j];
+                            if (!qk)
+                                sv[u][i] = acc;
+                            else if (j == 0)
+                                sq[u][i] = acc;
+                            else
+                                sk[u][i] = acc;
+                        }
+                    }
+                    if (qk) sa[u][i] = al[u];
+                }
             }
         } else {
-            const size_t row = static_cast<size_t>(b) * qkv_stride + static_cast<size_t>(h) * kD;
-            if (threadIdx.x < kD) {
-                const int i = threadIdx.x;
-                sq[u][i] = bf16_to_f32(q[row + i]);
-                sk[u][i] = bf16_to_f32(k[row + i]);
-                sv[u][i] = bf16_to_f32(v[row + i]);
-                sa[u][i] = alpha[static_cast<size_t>(bh) * kD + i];
+#pragma unroll
+            for (int u = 0; u < kUnits; ++u) {
+                if (u < nheads && threadIdx.x < kD) {
+                    const int bh = u == 0 ? bh0 : bh1;
+                    const int b = bh / H, h = bh - b * H;
+                    const size_t row = static_cast<size_t>(b) * qkv_stride + static_cast<size_t>(h) * kD;
+                    const int i = threadIdx.x;
+                    sq[u][i] = bf16_to_f32(q[row + i]);
+                    sk[u][i] = bf16_to_f32(k[row + i]);
+                    sv[u][i] = bf16_to_f32(v[row + i]);
+                    sa[u][i] = alpha[static_cast<size_t>(bh) * kD + i];
+                }
             }
         }
     };
@@ -286,8 +329,7 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
         }
     };
 
-    inputs(0, bh0);
-    if (has1) inputs(1 % kUnits, bh1);
+    inputs();
     __syncthreads();
     update(0, bh0);
     if constexpr (kPair) {

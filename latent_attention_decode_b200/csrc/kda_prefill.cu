@@ -1285,8 +1285,9 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
 // boxes of 128 channels x 64 tokens (32 for fp32, which stores a chunk in two halves).
 // Warps 0-7 own the master's rows (warp w: lanes 32 (w % 4) .., columns half w / 4); warp 8 issues
 // the MMAs and the record copies: per chunk the state part first (its own commit, which the master
-// pass waits for), then the output part, whose completion warp 8 waits for before the iteration's
-// closing barrier (so the next iteration may read those outputs without a wait of its own).
+// pass waits for), then the output part. The master pass keeps the new state's fp16 copy in
+// registers and writes it over S0's only once the output MMAs (which read S0's) are complete; warp 8
+// waits for them too before reusing the record buffer.
 constexpr int kChainThreads = kThreads + 32;
 
 __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(ChainArgs p,
@@ -1450,35 +1451,43 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
             w = wait_bar(mbar_s, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
             if (w && !last) w = rec_ready(i + 1);  // the next chunk's decay
             tc_fence_after();
+            uint32_t hv[32];  // the new state's fp16 copy, held until the output MMAs have read S0
             if (w) {
                 // ---- the new state: its fp16 copy and the next chunk's decay (or the state out) ----
-                float v[64];
-                tmem_ld32(tmem + lane_base + kCColS + 64 * cg, *reinterpret_cast<float(*)[32]>(v));
-                tmem_ld32(tmem + lane_base + kCColS + 64 * cg + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-                tmem_wait_ld();
-                if (last) {
-                    float *Sout = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) Sout[static_cast<size_t>(64 * cg + j) * kDv] = v[j];
-                } else {
+                for (int part = 0; part < 2; ++part) {
+                    const int c0 = 64 * cg + 32 * part;
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + kCColS + c0, v);
+                    tmem_wait_ld();
+                    if (last) {
+                        float *Sout = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
 #pragma unroll
-                    for (int j = 0; j < 64; j += 8)
-                        *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, 64 * cg + j, 16384)) =
-                            make_uint4(f32x2_to_f16x2(v[j], v[j + 1]), f32x2_to_f16x2(v[j + 2], v[j + 3]),
-                                       f32x2_to_f16x2(v[j + 4], v[j + 5]), f32x2_to_f16x2(v[j + 6], v[j + 7]));
-                    const float4 *gn = reinterpret_cast<const float4 *>(gl_of(i + 1) + 64 * cg);
+                        for (int j = 0; j < 32; ++j) Sout[static_cast<size_t>(c0 + j) * kDv] = v[j];
+                    } else {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float4 g4 = gn[j];
-                        v[4 * j] *= g4.x;
-                        v[4 * j + 1] *= g4.y;
-                        v[4 * j + 2] *= g4.z;
-                        v[4 * j + 3] *= g4.w;
+                        for (int j = 0; j < 16; ++j) hv[16 * part + j] = f32x2_to_f16x2(v[2 * j], v[2 * j + 1]);
+                        const float4 *gn = reinterpret_cast<const float4 *>(gl_of(i + 1) + c0);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float4 g4 = gn[j];
+                            v[4 * j] *= g4.x;
+                            v[4 * j + 1] *= g4.y;
+                            v[4 * j + 2] *= g4.z;
+                            v[4 * j + 3] *= g4.w;
+                        }
+                        tmem_st32(tmem + lane_base + kCColS + c0, v);
                     }
-                    tmem_st32(tmem + lane_base + kCColS + 64 * cg, *reinterpret_cast<float(*)[32]>(v));
-                    tmem_st32(tmem + lane_base + kCColS + 64 * cg + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-                    tmem_wait_st();
                 }
+                tmem_wait_st();
+            }
+            // the output MMAs read S0's fp16 copy: it is overwritten only once they are complete
+            if (w) w = wait_bar(mbar_o, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            if (w && !last) {
+#pragma unroll
+                for (int j = 0; j < 64; j += 8)
+                    *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, 64 * cg + j, 16384)) =
+                        make_uint4(hv[j / 2], hv[j / 2 + 1], hv[j / 2 + 2], hv[j / 2 + 3]);
             }
             if (tid == 0) bulk_wait_read0();  // the previous outputs have left the O tile
         }
