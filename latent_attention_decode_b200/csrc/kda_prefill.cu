@@ -676,6 +676,7 @@ constexpr uint32_t kIdescSN = make_idesc(128, 128, kFmtF16, 0, 0);   // S^T += S
 constexpr uint32_t kIdescO = make_idesc(128, 64, kFmtF16, 0, 0);     // O^T = U'^T P^T + S0^T Qe^T
 
 struct PrepArgs {
+    const uint16_t *v;  // [B][T][H][128] bf16 (the prep reads it through registers)
     const float *beta;
     uint8_t *ws;  // this segment's records, [B*H][nseg]
     int B, T, H;
@@ -685,7 +686,6 @@ struct PrepArgs {
 
 struct PrepMaps {
     CUtensorMap q, k, alpha;  // 3-D [B][T][H*128], boxes of 128 channels x 64 tokens, no swizzle
-    CUtensorMap v;            // the same view of v, boxes of 64 channels x 64 tokens, 128-byte swizzle
 };
 
 // prep shared memory (offsets from a 1024-aligned base). Regions are reused once their first
@@ -701,7 +701,7 @@ constexpr uint32_t kPG = 73728;     // g_last [128] fp32 (record)
 constexpr uint32_t kPTB = 74752;    // Tb [64 r][64 s] fp16 K-major; then (with TBH) Qe [64][128], 2 x 8 KiB
 constexpr uint32_t kPTBH = 82944;   // Tb, bf16 high part
 constexpr uint32_t kPTBL = 91136;   // Tb, bf16 low part (Tb - hi)
-constexpr uint32_t kPV = 99328;     // v [64 tok][128 d_v] bf16 as two SW128 boxes of 64 d_v (TMA)
+constexpr uint32_t kPV = 99328;     // v [64 tok][128 d_v] bf16, two SW128 blocks of 64 d_v (MN-major operand)
 constexpr uint32_t kPSQ = 115712;   // q [64 tok][128] bf16, plain (TMA)
 constexpr uint32_t kPSK = 132096;   // k, the same
 constexpr uint32_t kPSA = 148480;   // alpha [64 tok][128] fp32, plain (TMA)
@@ -709,11 +709,12 @@ constexpr int kAS = 68;             // row stride (floats) of the A / T scratch 
 constexpr uint32_t kPA = 181248;    // A [64][kAS] fp32; then (with T) N [128][128] fp16, 2 x 16 KiB
 constexpr uint32_t kPT = kPA + 64 * kAS * 4;   // T [64][kAS] fp32
 constexpr uint32_t kPMisc = kPT + 64 * kAS * 4;
-constexpr uint32_t kPmBeta = 0, kPmRq = 256, kPmRk = 512, kPmOct = 768, kPmBar = 768 + 4096, kPmTmem = kPmBar + 16,
-                   kPmAbort = kPmBar + 20;
+constexpr int kPThreads = 512;      // 16 warps: the CUDA-core phases are latency-bound
+constexpr int kPWarps = kPThreads / 32;
+constexpr uint32_t kPmBeta = 0, kPmRq = 256, kPmRk = 512, kPmOct = 768, kPmBar = 768 + kPWarps * 128 * 4,
+                   kPmTmem = kPmBar + 16, kPmAbort = kPmBar + 20;
 constexpr uint32_t kPSmemBytes = kPMisc + kPmBar + 32 + 1024;
-constexpr uint32_t kPStageQKA = 16384 + 16384 + 32768;
-constexpr uint32_t kPStageTx = kPStageQKA + 16384;
+constexpr uint32_t kPStageTx = 16384 + 16384 + 32768;  // q, k, alpha (v comes through registers)
 // TMEM columns: [Kt; Qt] Kh^T, W, U'^T, Kg^T W, P W
 constexpr uint32_t kPColA = 0, kPColW = 64, kPColU = 192, kPColN = 256, kPColPW = 384, kPTmemCols = 512;
 
@@ -734,7 +735,7 @@ __device__ __forceinline__ void put_tb4(uint8_t *tb16, uint8_t *tbh, uint8_t *tb
 // column; (2) in each 32x32 diagonal block, T_{2p+1,2p} = -T_{2p+1,2p+1} A_{2p+1,2p} T_{2p,2p};
 // (3) the lower-left 32x32 block, -T_hi A_{hi,lo} T_lo. The products A T of (2) and (3) are parked in
 // A's upper triangle, which holds no data. Then Tb = T diag(beta) goes to the three operand tiles
-// (fp16, and the bf16 hi / lo split). Called by all kThreads threads; contains block-wide barriers.
+// (fp16, and the bf16 hi / lo split). Called by all kPThreads threads; contains block-wide barriers.
 __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_beta, uint8_t *tb16, uint8_t *tbh,
                                           uint8_t *tbl, int tid) {
     if (tid < kC) {
@@ -762,80 +763,64 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
         for (int r = 0; r < 16; ++r) sT[(i0 + r) * kAS + i0 + c] = t[r];
     }
     __syncthreads();
-    // (2a) Y_p = A_{2p+1,2p} T_{2p,2p} into A at rows 32p .. 32p+15, columns 32p+16 .. 32p+31
-    if (tid < 128) {
-        const int q0 = 32 * (tid >> 6), rr = (tid >> 2) & 15, cc = (tid & 3) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2) {
-            const float a = sA[(q0 + 16 + rr) * kAS + q0 + s2];
-            const float4 t4 = *reinterpret_cast<const float4 *>(sT + (q0 + s2) * kAS + q0 + cc);
-            acc.x = fmaf(a, t4.x, acc.x);
-            acc.y = fmaf(a, t4.y, acc.y);
-            acc.z = fmaf(a, t4.z, acc.z);
-            acc.w = fmaf(a, t4.w, acc.w);
-        }
-        *reinterpret_cast<float4 *>(sA + (q0 + rr) * kAS + q0 + 16 + cc) = acc;
-    }
-    __syncthreads();
-    // (2b) T_{2p+1,2p} = -T_{2p+1,2p+1} Y_p
-    if (tid < 128) {
-        const int q0 = 32 * (tid >> 6), rr = (tid >> 2) & 15, cc = (tid & 3) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2) {
-            const float t = sT[(q0 + 16 + rr) * kAS + q0 + 16 + s2];
-            const float4 y4 = *reinterpret_cast<const float4 *>(sA + (q0 + s2) * kAS + q0 + 16 + cc);
-            acc.x = fmaf(t, y4.x, acc.x);
-            acc.y = fmaf(t, y4.y, acc.y);
-            acc.z = fmaf(t, y4.z, acc.z);
-            acc.w = fmaf(t, y4.w, acc.w);
-        }
-        *reinterpret_cast<float4 *>(sT + (q0 + 16 + rr) * kAS + q0 + cc) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-    }
-    __syncthreads();
-    // (3a) R = A_{hi,lo} T_lo (32 x 32) into A at rows 0 .. 31, columns 32 .. 63; T_lo is lower
-    //      triangular, so only s >= cc contributes
+    // (2a) Y_p = A_{2p+1,2p} T_{2p,2p} into A at rows 32p .. 32p+15, columns 32p+16 .. 32p+31:
+    //      one element per thread (2 blocks x 16 x 16)
     {
-        const int rr = tid >> 3, cc = (tid & 7) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const int q0 = 32 * (tid >> 8), rr = (tid >> 4) & 15, cc = tid & 15;
+        float acc = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2) acc = fmaf(sA[(q0 + 16 + rr) * kAS + q0 + s2], sT[(q0 + s2) * kAS + q0 + cc], acc);
+        sA[(q0 + rr) * kAS + q0 + 16 + cc] = acc;
+    }
+    __syncthreads();
+    // (2b) T_{2p+1,2p} = -T_{2p+1,2p+1} Y_p (T_{2p+1,2p+1} lower triangular: s <= rr)
+    {
+        const int q0 = 32 * (tid >> 8), rr = (tid >> 4) & 15, cc = tid & 15;
+        float acc = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2)
+            if (s2 <= rr) acc = fmaf(sT[(q0 + 16 + rr) * kAS + q0 + 16 + s2], sA[(q0 + s2) * kAS + q0 + 16 + cc], acc);
+        sT[(q0 + 16 + rr) * kAS + q0 + cc] = -acc;
+    }
+    __syncthreads();
+    // (3a) R = A_{hi,lo} T_lo (32 x 32) into A at rows 0 .. 31, columns 32 .. 63; a thread takes one
+    //      row and a pair of columns; T_lo is lower triangular, so only s >= cc contributes
+    {
+        const int rr = tid >> 4, cc = (tid & 15) * 2;
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll 8
         for (int s2 = cc; s2 < 32; ++s2) {
             const float a = sA[(32 + rr) * kAS + s2];
-            const float4 t4 = *reinterpret_cast<const float4 *>(sT + s2 * kAS + cc);
-            acc.x = fmaf(a, t4.x, acc.x);
-            acc.y = fmaf(a, t4.y, acc.y);
-            acc.z = fmaf(a, t4.z, acc.z);
-            acc.w = fmaf(a, t4.w, acc.w);
+            const float2 t2 = *reinterpret_cast<const float2 *>(sT + s2 * kAS + cc);
+            acc.x = fmaf(a, t2.x, acc.x);
+            acc.y = fmaf(a, t2.y, acc.y);
         }
-        *reinterpret_cast<float4 *>(sA + rr * kAS + 32 + cc) = acc;
+        *reinterpret_cast<float2 *>(sA + rr * kAS + 32 + cc) = acc;
     }
     __syncthreads();
     // (3b) T[32 + rr][0 .. 31] = -T_hi R; T_hi is lower triangular, so only s <= rr contributes
     {
-        const int rr = tid >> 3, cc = (tid & 7) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const int rr = tid >> 4, cc = (tid & 15) * 2;
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll 8
         for (int s2 = 0; s2 <= rr; ++s2) {
             const float t = sT[(32 + rr) * kAS + 32 + s2];
-            const float4 r4 = *reinterpret_cast<const float4 *>(sA + s2 * kAS + 32 + cc);
-            acc.x = fmaf(t, r4.x, acc.x);
-            acc.y = fmaf(t, r4.y, acc.y);
-            acc.z = fmaf(t, r4.z, acc.z);
-            acc.w = fmaf(t, r4.w, acc.w);
+            const float2 r2 = *reinterpret_cast<const float2 *>(sA + s2 * kAS + 32 + cc);
+            acc.x = fmaf(t, r2.x, acc.x);
+            acc.y = fmaf(t, r2.y, acc.y);
         }
-        *reinterpret_cast<float4 *>(sT + (32 + rr) * kAS + cc) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        *reinterpret_cast<float2 *>(sT + (32 + rr) * kAS + cc) = make_float2(-acc.x, -acc.y);
     }
     __syncthreads();
-    // Tb = T diag(beta): 64 rows x 16 quads of columns, four quads per thread; zero above the
+    // Tb = T diag(beta): 64 rows x 16 quads of columns, two quads per thread; zero above the
     // diagonal blocks (T holds nothing there)
 #pragma unroll
-    for (int e = tid; e < kC * 16; e += kThreads) {
+    for (int e = tid; e < kC * 16; e += kPThreads) {
         const int r = e >> 4, c = (e & 15) * 4;
         float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
         if ((c >> 4) <= (r >> 4)) t4 = *reinterpret_cast<const float4 *>(sT + r * kAS + c);
-        put_tb4(tb16, tbh, tbl, r, c, t4.x * s_beta[c], t4.y * s_beta[c + 1], t4.z * s_beta[c + 2],
-                t4.w * s_beta[c + 3]);
+        const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + c);
+        put_tb4(tb16, tbh, tbl, r, c, t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
     }
 }
 
@@ -857,11 +842,12 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// One CTA per SM walks the segment's (sequence, head, chunk) items. The next item's q, k and alpha
-// are staged (TMA) once the current item's operand tiles are formed, its v once the current
-// item's last MMAs (which read v) are complete; the record leaves by one bulk store (tiles) and
-// direct stores (U').
-__global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p, const __grid_constant__ PrepMaps maps) {
+// One CTA per SM walks the segment's (sequence, head, chunk) items with 16 warps. The next item's
+// q, k and alpha are staged (TMA) once the current item's operand tiles are formed; its v comes
+// into registers (32 bytes a thread) at the start of the current item and into the v tile (the
+// 128-byte swizzled MN-major operand layout) once the current item's last reader of that tile is
+// complete; beta is prefetched into a register the same way. The record leaves by bulk stores.
+__global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p, const __grid_constant__ PrepMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -878,7 +864,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kPMisc + kPmAbort);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int sp = warp & 3, cg = warp >> 2;
+    const int sp = warp & 3, qd = warp >> 2;  // TMEM sub-partition; quarter of an accumulator's columns
     const uint32_t lane_base = static_cast<uint32_t>(32 * sp) << 16;
     const int nitems = p.B * p.H * p.nseg;
 
@@ -912,12 +898,27 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
         tma_load_3d(sbase + kPSK, &maps.k, h * kDk, ch * kC, b, stage_bar);
         tma_load_3d(sbase + kPSA, &maps.alpha, h * kDk, ch * kC, b, stage_bar);
     };
-    auto stage_v = [&](int item) {
+    // v of an item: thread t holds 16-byte pieces 2t and 2t + 1 (piece p: token p / 16, values
+    // 8 (p % 16) .. + 7); tokens past T read as zero
+    auto load_v = [&](int it, uint4 (&vr)[2]) {
+        vr[0] = vr[1] = make_uint4(0u, 0u, 0u, 0u);
+        if (it >= nitems) return;
         int b, h, ch;
-        coords(item, b, h, ch);
-        fence_async_smem();
-        tma_load_3d(sbase + kPV, &maps.v, h * kDv, ch * kC, b, stage_bar);
-        tma_load_3d(sbase + kPV + 8192, &maps.v, h * kDv + 64, ch * kC, b, stage_bar);
+        coords(it, b, h, ch);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int pc = 2 * tid + e, tok = pc >> 4, t = ch * kC + tok;
+            if (t < p.T)
+                vr[e] = __ldcs(reinterpret_cast<const uint4 *>(p.v + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * kDv) +
+                               (pc & 15));
+        }
+    };
+    auto put_v = [&](const uint4 (&vr)[2]) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int pc = 2 * tid + e, tok = pc >> 4, c16 = pc & 15;
+            *reinterpret_cast<uint4 *>(sm + kPV + (c16 >> 3) * 8192 + tok * 128 + (((c16 & 7) ^ (tok & 7)) << 4)) = vr[e];
+        }
     };
     auto mma_wait = [&]() {
         const bool w = wait_bar(mma_bar, mma_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
@@ -927,8 +928,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
     };
     const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);  // K-major SW128 at offset 0
 
-    int pending = 0;   // a staging phase is in flight
-    int v_owed = -1;   // an item whose q, k and alpha are staged but whose v is not yet
+    int pending = 0;  // a staging phase is in flight
     int item = blockIdx.x;
     // beta of an item (threads 0-63, one token each, strided by H in memory): loaded one item ahead
     auto load_beta = [&](int it) -> float {
@@ -939,12 +939,12 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
         return t < p.T ? p.beta[(static_cast<size_t>(b) * p.T + t) * p.H + h] : 0.f;
     };
     float beta_next = load_beta(item);
+    uint4 v_next[2];
+    load_v(item, v_next);
     if (item < nitems) {
-        if (tid == 0) {
-            stage_qka(item);
-            stage_v(item);
-        }
+        if (tid == 0) stage_qka(item);
         pending = 1;
+        put_v(v_next);  // the first item's v; the barrier after the staging wait publishes it
     }
     for (; item < nitems && ok; item += gridDim.x) {
         int b, h, ch;
@@ -956,6 +956,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
 
         if (tid < kC) s_beta[tid] = beta_next;
         beta_next = load_beta(next);
+        load_v(next, v_next);
         if (tid == 0) bulk_wait_read0();  // the previous item's tiles have left for its record
         {
             const bool w = wait_bar(stage_bar, stage_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
@@ -969,7 +970,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
         const float *sa = reinterpret_cast<const float *>(sm + kPSA);
         if (p.l2norm) {
 #pragma unroll 1
-            for (int r = warp; r < kC; r += kThreads / 32) {
+            for (int r = warp; r < kC; r += kPWarps) {
                 const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + 4 * lane);
                 const uint2 kw = *reinterpret_cast<const uint2 *>(sk + r * kDk + 4 * lane);
                 const float2 q0 = lad::dev::bf16x2_to_f32(qw.x), q1 = lad::dev::bf16x2_to_f32(qw.y);
@@ -991,15 +992,15 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
             s_rk[tid] = 1.f;
         }
 
-        // ---- running decay and the operand tiles: warp w takes tokens 8w .. 8w+7, lane l the key
-        //      channels 4l .. 4l+3; the products over earlier token octets come through shared memory ----
+        // ---- running decay and the operand tiles: warp w takes tokens 4w .. 4w+3, lane l the key
+        //      channels 4l .. 4l+3; the products over earlier token quartets come through shared memory ----
         {
             const int o = warp, c4 = 4 * lane;
-            float4 gl[8];
+            float4 gl[4];
             float4 run = make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int r = 8 * o + u;
+            for (int u = 0; u < 4; ++u) {
+                const int r = 4 * o + u;
                 const float4 a = (r < n) ? *reinterpret_cast<const float4 *>(sa + r * kDk + c4)
                                          : make_float4(1.f, 1.f, 1.f, 1.f);
                 run.x *= a.x;
@@ -1010,9 +1011,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
             }
             *reinterpret_cast<float4 *>(s_oct + o * kDk + c4) = run;
             __syncthreads();
-            float4 excl = make_float4(1.f, 1.f, 1.f, 1.f), all = excl;  // before octet o; all octets
+            float4 excl = make_float4(1.f, 1.f, 1.f, 1.f), all = excl;  // before quartet o; all of them
 #pragma unroll
-            for (int oo = 0; oo < kThreads / 32; ++oo) {
+            for (int oo = 0; oo < kPWarps; ++oo) {
                 const float4 y = *reinterpret_cast<const float4 *>(s_oct + oo * kDk + c4);
                 if (oo < o) {
                     excl.x *= y.x;
@@ -1027,8 +1028,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
             }
             if (o == 0) *reinterpret_cast<float4 *>(s_g + c4) = all;  // g_last, for the record
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int r = 8 * o + u;
+            for (int u = 0; u < 4; ++u) {
+                const int r = 4 * o + u;
                 const float g[4] = {excl.x * gl[u].x, excl.y * gl[u].y, excl.z * gl[u].z, excl.w * gl[u].w};
                 const float ga[4] = {all.x, all.y, all.z, all.w};
                 const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + c4);
@@ -1064,7 +1065,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
         if (next < nitems) {
             if (tid == 0) stage_qka(next);
             pending = 1;
-            v_owed = next;
         }
         if (warp == 0) {
             tc_fence_after();
@@ -1076,24 +1076,25 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
         }
         ok = mma_wait();
         if (!ok) break;
-        // ---- A = strict_lower(diag(beta) Kt Kh^T) -> fp32 scratch; P = lower(Qt Kh^T) -> fp16 tile ----
+        // ---- A = strict_lower(diag(beta) Kt Kh^T) -> fp32 scratch; P = lower(Qt Kh^T) -> fp16 tile;
+        //      a thread takes 16 of a row's 64 columns ----
         {
-            float x[32];
-            tmem_ld32(tmem + lane_base + kPColA + 32 * cg, x);
+            float x[16];
+            tmem_ld16(tmem + lane_base + kPColA + 16 * qd, x);
             tmem_wait_ld();
-            const int row = 32 * sp + lane, c0 = 32 * cg;
+            const int row = 32 * sp + lane, c0 = 16 * qd;
             if (row < kC) {
                 const int r = row;
                 const float br = s_beta[r];
                 float4 *dst = reinterpret_cast<float4 *>(sA + r * kAS + c0);
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)
+                for (int j = 0; j < 16; j += 4)
                     dst[j / 4] = make_float4(c0 + j < r ? br * x[j] : 0.f, c0 + j + 1 < r ? br * x[j + 1] : 0.f,
                                              c0 + j + 2 < r ? br * x[j + 2] : 0.f, c0 + j + 3 < r ? br * x[j + 3] : 0.f);
             } else {
                 const int r = row - kC;
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
+                for (int j = 0; j < 16; j += 8) {
                     float y[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) y[e] = (c0 + j + e <= r) ? x[j + e] : 0.f;
@@ -1127,17 +1128,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
         }
         ok = mma_wait();
         if (!ok) break;
-        if (v_owed >= 0) {  // v is read: the next item's comes in
-            if (tid == 0) stage_v(v_owed);
-            v_owed = -1;
-        }
+        put_v(v_next);  // the v tile is read: the next item's goes in (published by the barriers below)
         // ---- W -> rows 0-63 of [W; Qt] (over Kt); U'^T -> fp16 tile (over Kh) ----
         {
             // M = 64: row 16 sp + i sits in lane i (< 16) of sub-partition sp; the loads are
             // collective, so the whole warp issues them and lanes 0-15 keep the rows
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * cg + 32 * part;
+            {
+                const int c0 = 32 * qd;
                 float w[32];
                 tmem_ld32(tmem + lane_base + kPColW + c0, w);
                 tmem_wait_ld();
@@ -1150,13 +1147,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
                                        f32x2_to_f16x2(w[j + 4], w[j + 5]), f32x2_to_f16x2(w[j + 6], w[j + 7]));
                 }
             }
-            float u[32];
-            tmem_ld32(tmem + lane_base + kPColU + 32 * cg, u);
+            float u[16];
+            tmem_ld16(tmem + lane_base + kPColU + 16 * qd, u);
             tmem_wait_ld();
             const int dv = 32 * sp + lane;
 #pragma unroll
-            for (int j = 0; j < 32; j += 8)
-                *reinterpret_cast<uint4 *>(sm + kPKH + sw128_off16(dv, 32 * cg + j, 16384)) =
+            for (int j = 0; j < 16; j += 8)
+                *reinterpret_cast<uint4 *>(sm + kPKH + sw128_off16(dv, 16 * qd + j, 16384)) =
                     make_uint4(f32x2_to_f16x2(u[j], u[j + 1]), f32x2_to_f16x2(u[j + 2], u[j + 3]),
                                f32x2_to_f16x2(u[j + 4], u[j + 5]), f32x2_to_f16x2(u[j + 6], u[j + 7]));
         }
@@ -1180,40 +1177,31 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
         if (!ok) break;
         // ---- N = -Kg^T W -> fp16 tile (over the A / T scratch); Qe = Qt - P W -> fp16 tile (over Tb) ----
         {
-            const int row = 32 * sp + lane;  // d_k' of N
+            const int row = 32 * sp + lane, c0 = 32 * qd;  // d_k' of N; 32 columns
+            float x[32];
+            tmem_ld32(tmem + lane_base + kPColN + c0, x);
+            tmem_wait_ld();
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * cg + 32 * part;
-                float x[32];
-                tmem_ld32(tmem + lane_base + kPColN + c0, x);
-                tmem_wait_ld();
+            for (int j = 0; j < 32; j += 8)
+                *reinterpret_cast<uint4 *>(sm + kPA + sw128_off16(row, c0 + j, 16384)) =
+                    make_uint4(f32x2_to_f16x2(-x[j], -x[j + 1]), f32x2_to_f16x2(-x[j + 2], -x[j + 3]),
+                               f32x2_to_f16x2(-x[j + 4], -x[j + 5]), f32x2_to_f16x2(-x[j + 6], -x[j + 7]));
+            tmem_ld32(tmem + lane_base + kPColPW + c0, x);  // M = 64: rows in lanes 0-15
+            tmem_wait_ld();
+            if (lane < 16) {
+                const int r = 16 * sp + lane;
 #pragma unroll
-                for (int j = 0; j < 32; j += 8)
-                    *reinterpret_cast<uint4 *>(sm + kPA + sw128_off16(row, c0 + j, 16384)) =
-                        make_uint4(f32x2_to_f16x2(-x[j], -x[j + 1]), f32x2_to_f16x2(-x[j + 2], -x[j + 3]),
-                                   f32x2_to_f16x2(-x[j + 4], -x[j + 5]), f32x2_to_f16x2(-x[j + 6], -x[j + 7]));
-            }
+                for (int j = 0; j < 32; j += 8) {
+                    const uint4 qv = *reinterpret_cast<const uint4 *>(sm + kPQW + sw128_off16(kC + r, c0 + j, 16384));
+                    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                    uint32_t ow[4];
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * cg + 32 * part;
-                float x[32];
-                tmem_ld32(tmem + lane_base + kPColPW + c0, x);  // M = 64: rows in lanes 0-15
-                tmem_wait_ld();
-                if (lane < 16) {
-                    const int r = 16 * sp + lane;
-#pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        const uint4 qv = *reinterpret_cast<const uint4 *>(sm + kPQW + sw128_off16(kC + r, c0 + j, 16384));
-                        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-                        uint32_t ow[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 qf = __half22float2(*reinterpret_cast<const __half2 *>(&qw[e]));
-                            ow[e] = f32x2_to_f16x2(qf.x - x[j + 2 * e], qf.y - x[j + 2 * e + 1]);
-                        }
-                        *reinterpret_cast<uint4 *>(sm + kPTB + sw128_off16(r, c0 + j, 8192)) =
-                            make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 qf = __half22float2(*reinterpret_cast<const __half2 *>(&qw[e]));
+                        ow[e] = f32x2_to_f16x2(qf.x - x[j + 2 * e], qf.y - x[j + 2 * e + 1]);
                     }
+                    *reinterpret_cast<uint4 *>(sm + kPTB + sw128_off16(r, c0 + j, 8192)) =
+                        make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
             }
         }
@@ -1232,7 +1220,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_prep_kernel(PrepArgs p,
     }
     // drain: a staging copy still in flight (after an abort) lands, the record stores complete and
     // every MMA this CTA issued completes, before shared memory and TMEM are released
-    if (tid == 0 && v_owed >= 0) stage_v(v_owed);  // the staging phase expects those bytes too
     if (tid == 0 && pending) {
         const uint64_t t0 = lad::dev::globaltimer_ns();
         while (!mbar_try_wait(stage_bar, stage_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
@@ -1629,7 +1616,6 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
     int rc = make(&pm.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk, false);
     if (rc == LAD_OK) rc = make(&pm.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk, false);
     if (rc == LAD_OK) rc = make(&pm.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDk, false);
-    if (rc == LAD_OK) rc = make(&pm.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, true);
     CUtensorMap omap;
     if (rc == LAD_OK)
         rc = make(&omap, o, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 ? 4 : 2, kDv,
@@ -1643,7 +1629,8 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
         const int nseg = nch - c0 < kSegChunks ? nch - c0 : kSegChunks;
         const long long items = static_cast<long long>(B) * H * nseg;
         const unsigned pg = static_cast<unsigned>(items < sms ? items : sms);
-        kda_chunk_prep_kernel<<<pg, kThreads, kPSmemBytes, st>>>(PrepArgs{beta, ws, B, T, H, c0, nseg, a.l2norm}, pm);
+        kda_chunk_prep_kernel<<<pg, kPThreads, kPSmemBytes, st>>>(PrepArgs{a.v, beta, ws, B, T, H, c0, nseg, a.l2norm},
+                                                                   pm);
         rc = lad::check_launch("kda_prefill_chunked");
         if (rc != LAD_OK) return rc;
         kda_chunk_chain_kernel<<<static_cast<unsigned>(B * H), kChainThreads, kCSmemBytes, st>>>(
