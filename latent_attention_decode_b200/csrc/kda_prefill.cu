@@ -661,9 +661,11 @@ __device__ __forceinline__ uint64_t kdesc16(uint64_t base_desc, uint32_t block_b
     return base_desc + ((static_cast<uint32_t>(j >> 2) * block_bytes + static_cast<uint32_t>(j & 3) * 32u) >> 4);
 }
 
+// two floats to a bf16 pair (lo in the low half), rounded to nearest even, in one conversion
 __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
-    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
-           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
 }
 
 constexpr uint32_t kIdescA = make_idesc(128, 64, kFmtF16, 0, 0);     // [Kt; Qt] Kh^T
@@ -711,9 +713,12 @@ constexpr uint32_t kPT = kPA + 64 * kAS * 4;   // T [64][kAS] fp32
 constexpr uint32_t kPMisc = kPT + 64 * kAS * 4;
 constexpr int kPThreads = 512;      // 16 warps: the CUDA-core phases are latency-bound
 constexpr int kPWarps = kPThreads / 32;
+constexpr int kPStageTid = 32;  // issues the input staging (warp 0 issues the MMAs)
+constexpr int kPBulkTid = 64;   // issues the record's bulk stores, in four groups an item, and waits on them
 constexpr uint32_t kPmBeta = 0, kPmRq = 256, kPmRk = 512, kPmOct = 768, kPmBar = 768 + kPWarps * 128 * 4,
-                   kPmTmem = kPmBar + 16, kPmAbort = kPmBar + 20;
-constexpr uint32_t kPSmemBytes = kPMisc + kPmBar + 32 + 1024;
+                   kPmTmem = kPmBar + 16, kPmAbort = kPmBar + 20, kPmRg = kPmBar + 32;
+constexpr uint32_t kPSmemBytes = kPMisc + kPmRg + 512 + 1024;
+static_assert(kPSmemBytes <= 232448, "prep shared memory over the per-block limit");
 constexpr uint32_t kPStageTx = 16384 + 16384 + 32768;  // q, k, alpha (v comes through registers)
 // TMEM columns: [Kt; Qt] Kh^T, W, U'^T, Kg^T W, P W
 constexpr uint32_t kPColA = 0, kPColW = 64, kPColU = 192, kPColN = 256, kPColPW = 384, kPTmemCols = 512;
@@ -731,13 +736,19 @@ __device__ __forceinline__ void put_tb4(uint8_t *tb16, uint8_t *tbh, uint8_t *tb
 
 
 // T = (I + A)^-1 for A strictly lower triangular [64][64] (fp32, row stride kAS), by recursive
-// doubling over 16x16 blocks: (1) the four diagonal blocks by forward substitution, one thread per
-// column; (2) in each 32x32 diagonal block, T_{2p+1,2p} = -T_{2p+1,2p+1} A_{2p+1,2p} T_{2p,2p};
-// (3) the lower-left 32x32 block, -T_hi A_{hi,lo} T_lo. The products A T of (2) and (3) are parked in
-// A's upper triangle, which holds no data. Then Tb = T diag(beta) goes to the three operand tiles
-// (fp16, and the bf16 hi / lo split). Called by all kPThreads threads; contains block-wide barriers.
+// doubling over 16x16 blocks, and Tb = T diag(beta) into the three operand tiles (fp16, and the
+// bf16 hi / lo split):
+//   (0) the four diagonal blocks by forward substitution, one thread per column;
+//   (1) in each 32x32 diagonal block, T_{2p+1,2p} = -T_{2p+1,2p+1} A_{2p+1,2p} T_{2p,2p};
+//   (2) the lower-left 32x32 block, -T_hi A_{hi,lo} T_lo.
+// The products A T of (1) and (2) are parked in A's upper triangle, which holds no data; the blocks
+// of T above its diagonal blocks are zeroed in (1), so that (2) runs over whole 32x32 blocks. Steps
+// (1) and (2) run on warps 0-3 (a row, or a row pair, and four columns a thread); in (2) warps 4-15
+// write the rows of Tb that are final already. Called by all kPThreads threads; contains block-wide
+// barriers.
 __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_beta, uint8_t *tb16, uint8_t *tbh,
                                           uint8_t *tbl, int tid) {
+    const int warp = tid >> 5, lane = tid & 31;
     if (tid < kC) {
         // column c of (I + A_ii)^-1: t_r = [r == c] - sum_{s < r} A_rs t_s (t_s = 0 for s < c); a
         // row of the block comes in four 16-byte loads, and two partial sums halve the FMA chain
@@ -760,67 +771,99 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
             t[r] = r < c ? 0.f : (r == c ? 1.f : -(acc0 + acc1));
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sT[(i0 + r) * kAS + i0 + c] = t[r];
+        for (int r = 0; r < 16; ++r) sT[(i0 + r) * kAS + i0 + c] = t[r];  // zeros above the diagonal too
     }
     __syncthreads();
-    // (2a) Y_p = A_{2p+1,2p} T_{2p,2p} into A at rows 32p .. 32p+15, columns 32p+16 .. 32p+31:
-    //      one element per thread (2 blocks x 16 x 16)
-    {
-        const int q0 = 32 * (tid >> 8), rr = (tid >> 4) & 15, cc = tid & 15;
-        float acc = 0.f;
+    // (1a) Y_p = A_{2p+1,2p} T_{2p,2p} into A at rows 32p .. 32p+15, columns 32p+16 .. 32p+31
+    const int q0 = 32 * (warp >> 1), rr = 8 * (warp & 1) + (lane >> 2), cc = 4 * (lane & 3);
+    if (warp < 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2) acc = fmaf(sA[(q0 + 16 + rr) * kAS + q0 + s2], sT[(q0 + s2) * kAS + q0 + cc], acc);
-        sA[(q0 + rr) * kAS + q0 + 16 + cc] = acc;
-    }
-    __syncthreads();
-    // (2b) T_{2p+1,2p} = -T_{2p+1,2p+1} Y_p (T_{2p+1,2p+1} lower triangular: s <= rr)
-    {
-        const int q0 = 32 * (tid >> 8), rr = (tid >> 4) & 15, cc = tid & 15;
-        float acc = 0.f;
-#pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2)
-            if (s2 <= rr) acc = fmaf(sT[(q0 + 16 + rr) * kAS + q0 + 16 + s2], sA[(q0 + s2) * kAS + q0 + 16 + cc], acc);
-        sT[(q0 + 16 + rr) * kAS + q0 + cc] = -acc;
-    }
-    __syncthreads();
-    // (3a) R = A_{hi,lo} T_lo (32 x 32) into A at rows 0 .. 31, columns 32 .. 63; a thread takes one
-    //      row and a pair of columns; T_lo is lower triangular, so only s >= cc contributes
-    {
-        const int rr = tid >> 4, cc = (tid & 15) * 2;
-        float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 8
-        for (int s2 = cc; s2 < 32; ++s2) {
-            const float a = sA[(32 + rr) * kAS + s2];
-            const float2 t2 = *reinterpret_cast<const float2 *>(sT + s2 * kAS + cc);
-            acc.x = fmaf(a, t2.x, acc.x);
-            acc.y = fmaf(a, t2.y, acc.y);
+        for (int s2 = 0; s2 < 16; ++s2) {
+            const float a = sA[(q0 + 16 + rr) * kAS + q0 + s2];
+            const float4 t = *reinterpret_cast<const float4 *>(sT + (q0 + s2) * kAS + q0 + cc);
+            acc.x = fmaf(a, t.x, acc.x);
+            acc.y = fmaf(a, t.y, acc.y);
+            acc.z = fmaf(a, t.z, acc.z);
+            acc.w = fmaf(a, t.w, acc.w);
         }
-        *reinterpret_cast<float2 *>(sA + rr * kAS + 32 + cc) = acc;
+        *reinterpret_cast<float4 *>(sA + (q0 + rr) * kAS + q0 + 16 + cc) = acc;
     }
     __syncthreads();
-    // (3b) T[32 + rr][0 .. 31] = -T_hi R; T_hi is lower triangular, so only s <= rr contributes
-    {
-        const int rr = tid >> 4, cc = (tid & 15) * 2;
-        float2 acc = make_float2(0.f, 0.f);
-#pragma unroll 8
-        for (int s2 = 0; s2 <= rr; ++s2) {
-            const float t = sT[(32 + rr) * kAS + 32 + s2];
-            const float2 r2 = *reinterpret_cast<const float2 *>(sA + s2 * kAS + 32 + cc);
-            acc.x = fmaf(t, r2.x, acc.x);
-            acc.y = fmaf(t, r2.y, acc.y);
-        }
-        *reinterpret_cast<float2 *>(sT + (32 + rr) * kAS + cc) = make_float2(-acc.x, -acc.y);
-    }
-    __syncthreads();
-    // Tb = T diag(beta): 64 rows x 16 quads of columns, two quads per thread; zero above the
-    // diagonal blocks (T holds nothing there)
+    // (1b) T_{2p+1,2p} = -T_{2p+1,2p+1} Y_p; T_{2p,2p+1} = 0
+    if (warp < 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int e = tid; e < kC * 16; e += kPThreads) {
-        const int r = e >> 4, c = (e & 15) * 4;
-        float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if ((c >> 4) <= (r >> 4)) t4 = *reinterpret_cast<const float4 *>(sT + r * kAS + c);
-        const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + c);
-        put_tb4(tb16, tbh, tbl, r, c, t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
+        for (int s2 = 0; s2 < 16; ++s2) {
+            const float t = sT[(q0 + 16 + rr) * kAS + q0 + 16 + s2];
+            const float4 y = *reinterpret_cast<const float4 *>(sA + (q0 + s2) * kAS + q0 + 16 + cc);
+            acc.x = fmaf(t, y.x, acc.x);
+            acc.y = fmaf(t, y.y, acc.y);
+            acc.z = fmaf(t, y.z, acc.z);
+            acc.w = fmaf(t, y.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(sT + (q0 + 16 + rr) * kAS + q0 + cc) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        *reinterpret_cast<float4 *>(sT + (q0 + rr) * kAS + q0 + 16 + cc) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+    // thread (warps 0-3) of steps (2a) / (2b): rows r2, r2 + 1 of a 32-row block, columns c2 .. c2 + 3
+    const int r2 = 2 * (tid >> 3), c2 = 4 * (tid & 7);
+    // (2a) R = A_{hi,lo} T_lo into A at rows 0 .. 31, columns 32 .. 63. Warps 4-15: Tb rows 0-31
+    //      (T_lo times beta; zero right of column 31)
+    if (warp < 4) {
+        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+#pragma unroll 8
+        for (int s = 0; s < 32; ++s) {
+            const float a0 = sA[(32 + r2) * kAS + s], a1 = sA[(33 + r2) * kAS + s];
+            const float4 t = *reinterpret_cast<const float4 *>(sT + s * kAS + c2);
+            acc0.x = fmaf(a0, t.x, acc0.x);
+            acc0.y = fmaf(a0, t.y, acc0.y);
+            acc0.z = fmaf(a0, t.z, acc0.z);
+            acc0.w = fmaf(a0, t.w, acc0.w);
+            acc1.x = fmaf(a1, t.x, acc1.x);
+            acc1.y = fmaf(a1, t.y, acc1.y);
+            acc1.z = fmaf(a1, t.z, acc1.z);
+            acc1.w = fmaf(a1, t.w, acc1.w);
+        }
+        *reinterpret_cast<float4 *>(sA + r2 * kAS + 32 + c2) = acc0;
+        *reinterpret_cast<float4 *>(sA + (r2 + 1) * kAS + 32 + c2) = acc1;
+    } else {
+        for (int e = tid - 128; e < 32 * 16; e += kPThreads - 128) {
+            const int r = e >> 4, c = (e & 15) * 4;
+            float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c < 32) t4 = *reinterpret_cast<const float4 *>(sT + r * kAS + c);
+            const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + c);
+            put_tb4(tb16, tbh, tbl, r, c, t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
+        }
+    }
+    __syncthreads();
+    // (2b) T[32 + r][0 .. 31] = -T_hi R, times beta, straight into Tb (T_hi is lower triangular: a
+    //      warp's rows end at 8 warp + 7). Warps 4-15: Tb rows 32-63, columns 32-63 (T_hi times beta)
+    if (warp < 4) {
+        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+#pragma unroll 8
+        for (int s = 0; s < 8 * warp + 8; ++s) {
+            const float t0 = sT[(32 + r2) * kAS + 32 + s], t1 = sT[(33 + r2) * kAS + 32 + s];
+            const float4 y = *reinterpret_cast<const float4 *>(sA + s * kAS + 32 + c2);
+            acc0.x = fmaf(t0, y.x, acc0.x);
+            acc0.y = fmaf(t0, y.y, acc0.y);
+            acc0.z = fmaf(t0, y.z, acc0.z);
+            acc0.w = fmaf(t0, y.w, acc0.w);
+            acc1.x = fmaf(t1, y.x, acc1.x);
+            acc1.y = fmaf(t1, y.y, acc1.y);
+            acc1.z = fmaf(t1, y.z, acc1.z);
+            acc1.w = fmaf(t1, y.w, acc1.w);
+        }
+        const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + c2);
+        put_tb4(tb16, tbh, tbl, 32 + r2, c2, -acc0.x * b4.x, -acc0.y * b4.y, -acc0.z * b4.z, -acc0.w * b4.w);
+        put_tb4(tb16, tbh, tbl, 33 + r2, c2, -acc1.x * b4.x, -acc1.y * b4.y, -acc1.z * b4.z, -acc1.w * b4.w);
+    } else {
+        for (int e = tid - 128; e < 32 * 8; e += kPThreads - 128) {
+            const int r = 32 + (e >> 3), c = 32 + (e & 7) * 4;
+            const float4 t4 = *reinterpret_cast<const float4 *>(sT + r * kAS + c);
+            const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + c);
+            put_tb4(tb16, tbh, tbl, r, c, t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
+        }
     }
 }
 
@@ -840,6 +883,7 @@ __device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // One CTA per SM walks the segment's (sequence, head, chunk) items with 16 warps. The next item's
@@ -854,7 +898,9 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
     float *s_beta = reinterpret_cast<float *>(sm + kPMisc + kPmBeta);
     float *s_rq = reinterpret_cast<float *>(sm + kPMisc + kPmRq);
     float *s_rk = reinterpret_cast<float *>(sm + kPMisc + kPmRk);
-    float *s_oct = reinterpret_cast<float *>(sm + kPMisc + kPmOct);
+    float *s_oct = reinterpret_cast<float *>(sm + kPMisc + kPmOct);  // per quartet: forward products
+    float *s_suf = reinterpret_cast<float *>(sm + kPTBL);           //   backward ones (Tb_lo is dead here)
+    float *s_rg = reinterpret_cast<float *>(sm + kPMisc + kPmRg);    // 1 / g_last
     float *s_g = reinterpret_cast<float *>(sm + kPG);
     float *sA = reinterpret_cast<float *>(sm + kPA);
     float *sT = reinterpret_cast<float *>(sm + kPT);
@@ -942,7 +988,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
     uint4 v_next[2];
     load_v(item, v_next);
     if (item < nitems) {
-        if (tid == 0) stage_qka(item);
+        if (tid == kPStageTid) stage_qka(item);
         pending = 1;
         put_v(v_next);  // the first item's v; the barrier after the staging wait publishes it
     }
@@ -957,7 +1003,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         if (tid < kC) s_beta[tid] = beta_next;
         beta_next = load_beta(next);
         load_v(next, v_next);
-        if (tid == 0) bulk_wait_read0();  // the previous item's tiles have left for its record
+        if (tid == kPBulkTid) bulk_wait_read1();  // the previous item's Kg, g, P, U'^T have left
         {
             const bool w = wait_bar(stage_bar, stage_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
             stage_phase ^= 1;
@@ -992,46 +1038,61 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
             s_rk[tid] = 1.f;
         }
 
-        // ---- running decay and the operand tiles: warp w takes tokens 4w .. 4w+3, lane l the key
-        //      channels 4l .. 4l+3; the products over earlier token quartets come through shared memory ----
+        // ---- running decays and the operand tiles. Per key channel, g_r = prod_{s <= r} alpha_s and
+        //      R_r = prod_{s > r} alpha_s (so Kg = K R = K g_last / g and Kh = Kg / g_last: one
+        //      reciprocal per channel, none per element). Warp w takes tokens 4w .. 4w+3, lane l the
+        //      channels 4l .. 4l+3; the 16 quartet products of a channel are scanned both ways by
+        //      threads 0-127, one channel each ----
         {
             const int o = warp, c4 = 4 * lane;
-            float4 gl[4];
-            float4 run = make_float4(1.f, 1.f, 1.f, 1.f);
+            float4 fw[4], bw[4];
+            {
+                float4 a4[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int r = 4 * o + u;
-                const float4 a = (r < n) ? *reinterpret_cast<const float4 *>(sa + r * kDk + c4)
-                                         : make_float4(1.f, 1.f, 1.f, 1.f);
-                run.x *= a.x;
-                run.y *= a.y;
-                run.z *= a.z;
-                run.w *= a.w;
-                gl[u] = run;
-            }
-            *reinterpret_cast<float4 *>(s_oct + o * kDk + c4) = run;
-            __syncthreads();
-            float4 excl = make_float4(1.f, 1.f, 1.f, 1.f), all = excl;  // before quartet o; all of them
-#pragma unroll
-            for (int oo = 0; oo < kPWarps; ++oo) {
-                const float4 y = *reinterpret_cast<const float4 *>(s_oct + oo * kDk + c4);
-                if (oo < o) {
-                    excl.x *= y.x;
-                    excl.y *= y.y;
-                    excl.z *= y.z;
-                    excl.w *= y.w;
+                for (int u = 0; u < 4; ++u) {
+                    const int r = 4 * o + u;
+                    a4[u] = (r < n) ? *reinterpret_cast<const float4 *>(sa + r * kDk + c4) : make_float4(1.f, 1.f, 1.f, 1.f);
                 }
-                all.x *= y.x;
-                all.y *= y.y;
-                all.z *= y.z;
-                all.w *= y.w;
+                float4 run = make_float4(1.f, 1.f, 1.f, 1.f);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    run = make_float4(run.x * a4[u].x, run.y * a4[u].y, run.z * a4[u].z, run.w * a4[u].w);
+                    fw[u] = run;  // prod over the quartet's tokens up to u
+                }
+                run = make_float4(1.f, 1.f, 1.f, 1.f);
+#pragma unroll
+                for (int u = 3; u >= 0; --u) {
+                    bw[u] = run;  // prod over the quartet's tokens after u
+                    run = make_float4(run.x * a4[u].x, run.y * a4[u].y, run.z * a4[u].z, run.w * a4[u].w);
+                }
             }
-            if (o == 0) *reinterpret_cast<float4 *>(s_g + c4) = all;  // g_last, for the record
+            *reinterpret_cast<float4 *>(s_oct + o * kDk + c4) = fw[3];
+            __syncthreads();
+            if (tid < kDk) {
+                float y[kPWarps];
+#pragma unroll
+                for (int oo = 0; oo < kPWarps; ++oo) y[oo] = s_oct[oo * kDk + tid];
+                float pre = 1.f, suf = 1.f;
+#pragma unroll
+                for (int oo = 0; oo < kPWarps; ++oo) {
+                    s_oct[oo * kDk + tid] = pre;  // before quartet oo
+                    pre *= y[oo];
+                    s_suf[(kPWarps - 1 - oo) * kDk + tid] = suf;  // after quartet 15 - oo
+                    suf *= y[kPWarps - 1 - oo];
+                }
+                s_g[tid] = pre;  // g_last, for the record
+                s_rg[tid] = __frcp_rn(pre);
+            }
+            __syncthreads();
+            const float4 ex = *reinterpret_cast<const float4 *>(s_oct + o * kDk + c4);
+            const float4 sx = *reinterpret_cast<const float4 *>(s_suf + o * kDk + c4);
+            const float4 rg = *reinterpret_cast<const float4 *>(s_rg + c4);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int r = 4 * o + u;
-                const float g[4] = {excl.x * gl[u].x, excl.y * gl[u].y, excl.z * gl[u].z, excl.w * gl[u].w};
-                const float ga[4] = {all.x, all.y, all.z, all.w};
+                const float g[4] = {ex.x * fw[u].x, ex.y * fw[u].y, ex.z * fw[u].z, ex.w * fw[u].w};
+                const float R[4] = {sx.x * bw[u].x, sx.y * bw[u].y, sx.z * bw[u].z, sx.w * bw[u].w};
+                const float rgl[4] = {rg.x, rg.y, rg.z, rg.w};
                 const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + c4);
                 const uint2 kw = *reinterpret_cast<const uint2 *>(sk + r * kDk + c4);
                 const float2 q0 = lad::dev::bf16x2_to_f32(qw.x), q1 = lad::dev::bf16x2_to_f32(qw.y);
@@ -1042,8 +1103,8 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
                 float kh[4], kg[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    kh[e] = __fdividef(kv[e], g[e]);
-                    kg[e] = kh[e] * ga[e];
+                    kg[e] = kv[e] * R[e];
+                    kh[e] = kg[e] * rgl[e];
                 }
                 const uint32_t off = sw128_off16(r, c4, 8192);                 // 64-row tiles (Kh, Kg)
                 const uint32_t offq = sw128_off16(kC + r, c4, 16384);          // row 64 + r of [Kt; Qt]
@@ -1063,8 +1124,13 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         tc_fence_before();
         __syncthreads();  // q, k and alpha of this item are read: the next item's come in
         if (next < nitems) {
-            if (tid == 0) stage_qka(next);
+            if (tid == kPStageTid) stage_qka(next);
             pending = 1;
+        }
+        if (tid == kPBulkTid) {  // the record's Kg and g_last are final
+            bulk_s2g(rec + kRKG, sbase + kPKG, 16384);
+            bulk_s2g(rec + kRG, sbase + kPG, 512);
+            bulk_commit();
         }
         if (warp == 0) {
             tc_fence_after();
@@ -1074,6 +1140,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
                            kIdescA, j > 0);
             tc_commit(mma_bar);
         }
+        if (tid == kPBulkTid) bulk_wait_read1();  // the previous item's N and Qe have left (A, T, Tb go there)
         ok = mma_wait();
         if (!ok) break;
         // ---- A = strict_lower(diag(beta) Kt Kh^T) -> fp32 scratch; P = lower(Qt Kh^T) -> fp16 tile;
@@ -1104,8 +1171,13 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
                 }
             }
         }
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        if (tid == kPBulkTid) {  // P is final
+            bulk_s2g(rec + kRP, sbase + kPP, 8192);
+            bulk_commit();
+        }
         // ---- T = (I + A)^-1, Tb = T diag(beta) -> the fp16 tile and its bf16 hi / lo split ----
         solve_tb16(sA, sT, s_beta, sm + kPTB, sm + kPTBH, sm + kPTBL, tid);
         // ---- W = Tb Kt (Kt: rows 0-63 of [Kt; Qt], read MN-major); U'^T = V^T (Tb_hi + Tb_lo)^T ----
@@ -1161,6 +1233,10 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        if (tid == kPBulkTid) {  // U'^T is final
+            bulk_s2g(rec + kRU, sbase + kPKH, 16384);
+            bulk_commit();
+        }
         if (warp == 0) {
             tc_fence_after();
             const uint64_t kg0 = smem_desc(sbase + kPKG, 8192, 1024, kLayoutSw128);  // MN chunks 8 KiB apart
@@ -1208,13 +1284,9 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == kPBulkTid) {
             bulk_s2g(rec + kRN, sbase + kPA, 32768);
             bulk_s2g(rec + kRQE, sbase + kPTB, 16384);
-            bulk_s2g(rec + kRKG, sbase + kPKG, 16384);
-            bulk_s2g(rec + kRP, sbase + kPP, 8192);
-            bulk_s2g(rec + kRU, sbase + kPKH, 16384);
-            bulk_s2g(rec + kRG, sbase + kPG, 512);
             bulk_commit();
         }
     }
@@ -1225,7 +1297,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         while (!mbar_try_wait(stage_bar, stage_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
         }
     }
-    if (tid == 0) bulk_wait_all();
+    if (tid == kPBulkTid) bulk_wait_all();
     if (warp == 0) {
         tc_commit(mma_bar);
         const uint64_t t0 = lad::dev::globaltimer_ns();
