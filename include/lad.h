@@ -216,20 +216,27 @@ int kda_conv_decode_step(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 
  *   S            fp32 [B][H][dk][dv]  initial state in, final state out
  *   o            [B][T][H][dv] bf16, or fp32 if flags & LAD_FLAG_OUT_FP32
  *   workspace    NULL, or device scratch of ws_bytes >= kda_prefill_workspace_size(...),
- *                16-byte aligned (else LAD_EWORKSPACE): with it the call runs two kernels per
- *                segment of up to 128 chunks (every chunk's state-independent operands in
- *                parallel, written to the workspace as one 145 KiB record per (sequence, head,
- *                chunk); then the state chain alone); without it, one kernel that does both per
- *                chunk. Same results within rounding.
+ *                256-byte aligned (else LAD_EWORKSPACE), owned by the caller and not read or
+ *                written by anything else until the call's work on `stream` is done. With it
+ *                the call runs two kernels per segment of up to 128 chunks: every chunk's
+ *                state-independent operands in parallel, written to the workspace as one
+ *                90,624-byte record per (sequence, head, chunk); then the state chain alone.
+ *                The chains run on a stream the library keeps per device (highest priority),
+ *                ordered by events: the chain of segment s overlaps the operands of segment
+ *                s + 1, and `stream` waits for the last chain before any later work on it (the
+ *                call stays capturable in a CUDA graph). Without a workspace, one kernel does
+ *                both per chunk on `stream`. Same results within rounding.
  * Supported: dk == dv == 128, chunk == 64; flags LAD_FLAG_L2NORM_QK, LAD_FLAG_OUT_FP32.
- * alpha must keep prod(alpha) over one chunk above ~1e-30 per channel (fp32 range of 1/g).
+ * alpha must keep prod(alpha) over one chunk above ~1e-30 per channel (fp32 range of 1/g); the
+ * workspace path also needs every K g_last / g and K / g of a chunk inside the fp16 range.
  */
 int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, const float *alpha,
                         const float *beta, float *S, void *o, int B, int T, int H, int dk, int dv, int chunk,
                         float scale, unsigned flags, void *workspace, size_t ws_bytes, void *stream);
-/* Workspace bytes of kda_prefill_chunked's two-kernel path: B * H * min(ceil(T / 64), 128) records
- * of 145 KiB (about 1.19 GB for one sequence of 64 heads and 8,192 tokens or more); 0 for
- * unsupported shapes. */
+/* Workspace bytes of kda_prefill_chunked's two-kernel path: a 256-byte header (item counters,
+ * one per segment, rounded up to 256 bytes) plus B * H * min(ceil(T / 64), 128) records of
+ * 90,624 bytes, twice over when T spans more than one segment of 128 chunks (about 1.48 GB for
+ * one sequence of 64 heads and more than 8,192 tokens); 0 for unsupported shapes. */
 size_t kda_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk);
 
 /*

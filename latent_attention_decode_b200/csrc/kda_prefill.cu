@@ -1,6 +1,6 @@
 // KDA chunked prefill on B200: the gated delta rule over T tokens in chunks of 64, in the WY / UT
-// form, with every contraction on the tensor cores (tcgen05, kind::tf32) and the fp32 state
-// carried in tensor memory from chunk to chunk.
+// form, with every contraction on the tensor cores (tcgen05) and the fp32 state carried in tensor
+// memory from chunk to chunk.
 //
 // Source: "Ling-3.1-flash: a 560B hybrid-attention MoE, counted from its safetensors headers",
 // section "How KDA and MLA split the work" (gated delta rule, per-channel decay alpha, per-head
@@ -13,13 +13,13 @@
 //   W  = Tb Kt,  U = Tb V - W S0
 //   O  = scale (Qt S0 + lower(Qt Kh^T) U)
 //   S  = Diag(g_last) (S0 + Kh^T U)        (= Diag(g_last) S0 + (K * g_last/g)^T U)
-// d_v columns of S are independent, so a CTA owns one (sequence, head, half of d_v) and walks
-// its chunks in order: 128 CTAs for one sequence of 64 heads.
 //
-// Two paths. With a workspace, two kernels per segment of up to 128 chunks: the prep kernel
-// computes every chunk's state-independent operands (W, Tb V, Qt, Kh^T, lower(Qt Kh^T), g_last)
-// in parallel into a record per chunk, and the scan kernel runs only the state chain, two MMA
-// batches per chunk (see "Split path" below). Without one, the single kernel does both, per chunk:
+// Two paths. With a workspace (the fast one), two kernels per segment of up to 128 chunks: the
+// prep kernel computes every chunk's state-independent operands in parallel (fp16 operands,
+// kind::f16) into a record per chunk, and the chain kernel runs only the state recurrence, one CTA
+// per (sequence, head) (see "Split path" below). Without one, a single kernel does both with tf32
+// operands; the d_v columns of S are independent, so there a CTA owns one (sequence, head, half
+// of d_v) and walks its chunks in order: 128 CTAs for one sequence of 64 heads.
 //
 // Single kernel, per chunk (two warpgroups; warp 0 issues the MMAs, converged, elect.sync):
 //   1. load q, k, alpha, v, beta; running products g; write the operand tiles
@@ -680,7 +680,8 @@ constexpr uint32_t kIdescO = make_idesc(128, 64, kFmtF16, 0, 0);     // O^T = U'
 struct PrepArgs {
     const uint16_t *v;  // [B][T][H][128] bf16 (the prep reads it through registers)
     const float *beta;
-    uint8_t *ws;  // this segment's records, [B*H][nseg]
+    uint8_t *ws;   // this segment's records, [B*H][nseg]
+    int *counter;  // the segment's item counter (zero at launch)
     int B, T, H;
     int c0, nseg;  // the segment: chunks c0 .. c0 + nseg - 1
     int l2norm;
@@ -716,7 +717,7 @@ constexpr int kPWarps = kPThreads / 32;
 constexpr int kPStageTid = 32;  // issues the input staging (warp 0 issues the MMAs)
 constexpr int kPBulkTid = 64;   // issues the record's bulk stores, in four groups an item, and waits on them
 constexpr uint32_t kPmBeta = 0, kPmRq = 256, kPmRk = 512, kPmOct = 768, kPmBar = 768 + kPWarps * 128 * 4,
-                   kPmTmem = kPmBar + 16, kPmAbort = kPmBar + 20, kPmRg = kPmBar + 32;
+                   kPmTmem = kPmBar + 16, kPmAbort = kPmBar + 20, kPmFetch = kPmBar + 24, kPmRg = kPmBar + 32;
 constexpr uint32_t kPSmemBytes = kPMisc + kPmRg + 512 + 1024;
 static_assert(kPSmemBytes <= 232448, "prep shared memory over the per-block limit");
 constexpr uint32_t kPStageTx = 16384 + 16384 + 32768;  // q, k, alpha (v comes through registers)
@@ -908,6 +909,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
     const uint32_t mma_bar = stage_bar + 8;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kPMisc + kPmTmem);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kPMisc + kPmAbort);
+    int *s_fetch = reinterpret_cast<int *>(sm + kPMisc + kPmFetch);  // items taken from the counter
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int sp = warp & 3, qd = warp >> 2;  // TMEM sub-partition; quarter of an accumulator's columns
@@ -918,6 +920,8 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         mbar_init(stage_bar, 1);
         mbar_init(mma_bar, 1);
         *abort_flag = 0;
+        s_fetch[0] = atomicAdd(p.counter, 1);  // the first item, and the one after it
+        s_fetch[1] = atomicAdd(p.counter, 1);
         mbar_fence_init();
     }
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kPTmemCols);
@@ -935,9 +939,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         b = bh / p.H;
         h = bh - b * p.H;
     };
-    auto stage_qka = [&](int item) {
-        int b, h, ch;
-        coords(item, b, h, ch);
+    auto stage_qka = [&](int b, int h, int ch) {
         fence_async_smem();
         mbar_arrive_tx_raw(stage_bar, kPStageTx);
         tma_load_3d(sbase + kPSQ, &maps.q, h * kDk, ch * kC, b, stage_bar);
@@ -946,11 +948,9 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
     };
     // v of an item: thread t holds 16-byte pieces 2t and 2t + 1 (piece p: token p / 16, values
     // 8 (p % 16) .. + 7); tokens past T read as zero
-    auto load_v = [&](int it, uint4 (&vr)[2]) {
+    auto load_v = [&](int it, int b, int h, int ch, uint4 (&vr)[2]) {
         vr[0] = vr[1] = make_uint4(0u, 0u, 0u, 0u);
         if (it >= nitems) return;
-        int b, h, ch;
-        coords(it, b, h, ch);
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int pc = 2 * tid + e, tok = pc >> 4, t = ch * kC + tok;
@@ -975,34 +975,36 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
     const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);  // K-major SW128 at offset 0
 
     int pending = 0;  // a staging phase is in flight
-    int item = blockIdx.x;
+    // items come from the segment's counter, one at a time (CTAs that start late, behind other
+    // work on their SM, take fewer); the next one is always known an item ahead, for the prefetch
+    int item = s_fetch[0], next = s_fetch[1];
     // beta of an item (threads 0-63, one token each, strided by H in memory): loaded one item ahead
-    auto load_beta = [&](int it) -> float {
+    auto load_beta = [&](int it, int b, int h, int ch) -> float {
         if (tid >= kC || it >= nitems) return 0.f;
-        int b, h, ch;
-        coords(it, b, h, ch);
         const int t = ch * kC + tid;
         return t < p.T ? p.beta[(static_cast<size_t>(b) * p.T + t) * p.H + h] : 0.f;
     };
-    float beta_next = load_beta(item);
+    // coordinates of the next item, computed once (the integer divisions are not cheap)
+    int nb, nh, nch;
+    coords(item, nb, nh, nch);
+    float beta_next = load_beta(item, nb, nh, nch);
     uint4 v_next[2];
-    load_v(item, v_next);
+    load_v(item, nb, nh, nch, v_next);
     if (item < nitems) {
-        if (tid == kPStageTid) stage_qka(item);
+        if (tid == kPStageTid) stage_qka(nb, nh, nch);
         pending = 1;
         put_v(v_next);  // the first item's v; the barrier after the staging wait publishes it
     }
-    for (; item < nitems && ok; item += gridDim.x) {
-        int b, h, ch;
-        coords(item, b, h, ch);
-        const int next = item + static_cast<int>(gridDim.x);
+    while (item < nitems && ok) {
+        const int ch = nch;
+        coords(next, nb, nh, nch);
         const int t0 = ch * kC;
         const int n = min(kC, p.T - t0);
         uint8_t *rec = p.ws + static_cast<size_t>(item) * kRecBytes;
 
         if (tid < kC) s_beta[tid] = beta_next;
-        beta_next = load_beta(next);
-        load_v(next, v_next);
+        beta_next = load_beta(next, nb, nh, nch);
+        load_v(next, nb, nh, nch, v_next);
         if (tid == kPBulkTid) bulk_wait_read1();  // the previous item's Kg, g, P, U'^T have left
         {
             const bool w = wait_bar(stage_bar, stage_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
@@ -1124,9 +1126,10 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         tc_fence_before();
         __syncthreads();  // q, k and alpha of this item are read: the next item's come in
         if (next < nitems) {
-            if (tid == kPStageTid) stage_qka(next);
+            if (tid == kPStageTid) stage_qka(nb, nh, nch);
             pending = 1;
         }
+        if (tid == 0) s_fetch[0] = atomicAdd(p.counter, 1);  // read after this item's last barrier
         if (tid == kPBulkTid) {  // the record's Kg and g_last are final
             bulk_s2g(rec + kRKG, sbase + kPKG, 16384);
             bulk_s2g(rec + kRG, sbase + kPG, 512);
@@ -1289,6 +1292,8 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
             bulk_s2g(rec + kRQE, sbase + kPTB, 16384);
             bulk_commit();
         }
+        item = next;
+        next = s_fetch[0];
     }
     // drain: a staging copy still in flight (after an abort) lands, the record stores complete and
     // every MMA this CTA issued completes, before shared memory and TMEM are released
@@ -1607,11 +1612,58 @@ int take_device_error_prefill(cudaStream_t s, int *code) {
 }
 }  // namespace lad
 
+namespace {
+// The split path's workspace: a header of per-segment item counters (256-byte granules), then one
+// segment buffer of records, or two when there are several segments (the prep of segment s + 1
+// writes one while the chain of segment s reads the other).
+struct WsLayout {
+    long long seg, nsegs, nbuf, header, buf_bytes;
+};
+WsLayout ws_layout(int B, int T, int H) {
+    WsLayout L;
+    const long long nch = (static_cast<long long>(T) + kC - 1) / kC;
+    L.seg = nch < kSegChunks ? nch : kSegChunks;
+    L.nsegs = (nch + L.seg - 1) / L.seg;
+    L.nbuf = L.nsegs > 1 ? 2 : 1;
+    L.header = (L.nsegs * 4 + 255) / 256 * 256;
+    L.buf_bytes = static_cast<long long>(B) * H * L.seg * kRecBytes;
+    return L;
+}
+
+// Per device: the stream the chain kernels run on, at the highest priority (when SMs free up, a
+// chain launch is placed ahead of the next segment's prep CTAs), and the events that order the two
+// streams. The mutex also serialises a call's whole enqueue sequence, as the events are shared.
+struct SideStream {
+    cudaStream_t st = nullptr;
+    cudaEvent_t prep_done = nullptr, chain_done[2] = {nullptr, nullptr};
+};
+std::mutex side_mu;
+SideStream side_streams[64];
+
+cudaError_t side_stream(int dev, SideStream **out) {
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    SideStream &s = side_streams[dev];
+    if (!s.st) {
+        int least = 0, greatest = 0;
+        cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+        if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&s.st, cudaStreamNonBlocking, greatest);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.prep_done, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.chain_done[0], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.chain_done[1], cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            s = SideStream{};  // handles created before the failure stay alive; nothing reuses them
+            return e;
+        }
+    }
+    *out = &s;
+    return cudaSuccess;
+}
+}  // namespace
+
 extern "C" size_t kda_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk) {
     if (B <= 0 || T <= 0 || H <= 0 || dk != kDk || dv != kDv || chunk != kC) return 0;
-    const long long nch = (static_cast<long long>(T) + kC - 1) / kC;
-    const long long seg = nch < kSegChunks ? nch : kSegChunks;
-    return static_cast<size_t>(B) * static_cast<size_t>(H) * static_cast<size_t>(seg) * kRecBytes;
+    const WsLayout L = ws_layout(B, T, H);
+    return static_cast<size_t>(L.header + L.nbuf * L.buf_bytes);
 }
 
 extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, const float *alpha,
@@ -1641,19 +1693,28 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
                          ws_need);
     if (split && static_cast<long long>(B) * H * kSegChunks > 0x7fffffffLL)
         return set_error(LAD_EUNSUPPORTED, "kda_prefill_chunked: B*H too large");
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(kda_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(kda_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            kPSmemBytes);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(kda_chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            kCSmemBytes);
-    });
-    if (attr_err != cudaSuccess)
-        return set_error(LAD_ECUDA, "kda_prefill_chunked: smem attribute: %s", cudaGetErrorString(attr_err));
+    {
+        // the dynamic shared memory limits, set once per device
+        static std::mutex attr_mu;
+        static bool attr_done[64] = {};
+        int adev = 0;
+        if (cudaGetDevice(&adev) != cudaSuccess || adev < 0 || adev >= 64)
+            return set_error(LAD_ECUDA, "kda_prefill_chunked: no current device");
+        std::lock_guard<std::mutex> lock(attr_mu);
+        if (!attr_done[adev]) {
+            cudaError_t attr_err =
+                cudaFuncSetAttribute(kda_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute(kda_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                kPSmemBytes);
+            if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute(kda_chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                kCSmemBytes);
+            if (attr_err != cudaSuccess)
+                return set_error(LAD_ECUDA, "kda_prefill_chunked: smem attribute: %s", cudaGetErrorString(attr_err));
+            attr_done[adev] = true;
+        }
+    }
     Args a{reinterpret_cast<const uint16_t *>(q), reinterpret_cast<const uint16_t *>(k),
            reinterpret_cast<const uint16_t *>(v), alpha, beta, S, o, B, T, H, scale,
            (flags & LAD_FLAG_L2NORM_QK) ? 1 : 0, f32 ? 1 : 0};
@@ -1693,22 +1754,44 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
         rc = make(&omap, o, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 ? 4 : 2, kDv,
                   false, f32 ? kC / 2 : kC);
     if (rc != LAD_OK) return rc;
+    const WsLayout L = ws_layout(B, T, H);
     const int nch = (T + kC - 1) / kC;
     const int sms = lad::device_sm_count();
     if (sms <= 0) return set_error(LAD_ECUDA, "kda_prefill_chunked: cannot query the SM count");
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return set_error(LAD_ECUDA, "kda_prefill_chunked: no current device");
+    std::lock_guard<std::mutex> lock(side_mu);
+    SideStream *side = nullptr;
+    cudaError_t e = side_stream(dev, &side);
+    if (e != cudaSuccess) return set_error(LAD_ECUDA, "kda_prefill_chunked: side stream: %s", cudaGetErrorString(e));
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    for (int c0 = 0; c0 < nch; c0 += kSegChunks) {
-        const int nseg = nch - c0 < kSegChunks ? nch - c0 : kSegChunks;
+    int *counters = reinterpret_cast<int *>(ws);
+    e = cudaMemsetAsync(counters, 0, static_cast<size_t>(L.header), st);
+    // segment s: prep on the caller's stream, then the chain on the side stream; the prep of s + 1
+    // runs beside the chain of s, and the prep of s + 2 waits for the chain of s to free its buffer
+    for (int sg = 0; sg < L.nsegs && e == cudaSuccess; ++sg) {
+        const int c0 = sg * static_cast<int>(L.seg);
+        const int nseg = nch - c0 < L.seg ? nch - c0 : static_cast<int>(L.seg);
+        uint8_t *buf = ws + L.header + (sg % L.nbuf) * L.buf_bytes;
+        if (sg >= 2) e = cudaStreamWaitEvent(st, side->chain_done[sg & 1], 0);
+        if (e != cudaSuccess) break;
         const long long items = static_cast<long long>(B) * H * nseg;
         const unsigned pg = static_cast<unsigned>(items < sms ? items : sms);
-        kda_chunk_prep_kernel<<<pg, kPThreads, kPSmemBytes, st>>>(PrepArgs{a.v, beta, ws, B, T, H, c0, nseg, a.l2norm},
-                                                                   pm);
-        rc = lad::check_launch("kda_prefill_chunked");
-        if (rc != LAD_OK) return rc;
-        kda_chunk_chain_kernel<<<static_cast<unsigned>(B * H), kChainThreads, kCSmemBytes, st>>>(
-            ChainArgs{S, o, ws, B, T, H, c0, nseg, scale, a.out_f32}, omap);
-        rc = lad::check_launch("kda_prefill_chunked");
-        if (rc != LAD_OK) return rc;
+        kda_chunk_prep_kernel<<<pg, kPThreads, kPSmemBytes, st>>>(
+            PrepArgs{a.v, beta, buf, counters + sg, B, T, H, c0, nseg, a.l2norm}, pm);
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaEventRecord(side->prep_done, st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side->st, side->prep_done, 0);
+        if (e != cudaSuccess) break;
+        kda_chunk_chain_kernel<<<static_cast<unsigned>(B * H), kChainThreads, kCSmemBytes, side->st>>>(
+            ChainArgs{S, o, buf, B, T, H, c0, nseg, scale, a.out_f32}, omap);
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaEventRecord(side->chain_done[sg & 1], side->st);
     }
+    // the caller's stream waits for the last chain (when the loop stopped early, for whatever was
+    // enqueued on the side stream)
+    const cudaError_t j = cudaStreamWaitEvent(st, side->chain_done[(L.nsegs - 1) & 1], 0);
+    if (e == cudaSuccess) e = j;
+    if (e != cudaSuccess) return set_error(LAD_ECUDA, "kda_prefill_chunked: %s", cudaGetErrorString(e));
     return LAD_OK;
 }

@@ -115,13 +115,17 @@ def test_host_side_validation_of_the_fp8_calls(lib):
 
 
 def test_prefill_workspace_size(lib):
-    """The two-kernel prefill path's workspace: one 90,624-byte record (fp16 operand tiles, g_last
-    and U') per (sequence, head, chunk) of a segment of at most 128 chunks; zero for shapes the call
-    does not support."""
-    rec = 90624
-    assert lib.kda_prefill_workspace_size(1, 32768, 64, 128, 128, 64) == 64 * 128 * rec
-    assert lib.kda_prefill_workspace_size(2, 100, 3, 128, 128, 64) == 2 * 3 * 2 * rec
-    assert lib.kda_prefill_workspace_size(1, 1, 1, 128, 128, 64) == rec
+    """The two-kernel prefill path's workspace: a 256-byte header of per-segment item counters,
+    then one 90,624-byte record (fp16 operand tiles, g_last and U') per (sequence, head, chunk) of
+    a segment of at most 128 chunks, twice over when there are several segments (one segment's
+    records are read while the next one's are written); zero for shapes the call does not
+    support."""
+    rec, hdr = 90624, 256
+    assert lib.kda_prefill_workspace_size(1, 32768, 64, 128, 128, 64) == hdr + 2 * 64 * 128 * rec
+    assert lib.kda_prefill_workspace_size(1, 128 * 64 + 1, 1, 128, 128, 64) == hdr + 2 * 128 * rec
+    assert lib.kda_prefill_workspace_size(1, 128 * 64, 1, 128, 128, 64) == hdr + 128 * rec
+    assert lib.kda_prefill_workspace_size(2, 100, 3, 128, 128, 64) == hdr + 2 * 3 * 2 * rec
+    assert lib.kda_prefill_workspace_size(1, 1, 1, 128, 128, 64) == hdr + rec
     assert lib.kda_prefill_workspace_size(1, 0, 64, 128, 128, 64) == 0
     assert lib.kda_prefill_workspace_size(1, 64, 64, 64, 128, 64) == 0
     assert lib.kda_prefill_workspace_size(1, 64, 64, 128, 128, 32) == 0
