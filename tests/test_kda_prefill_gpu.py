@@ -1,11 +1,12 @@
-"""Parity of kda_prefill_chunked (CUDA, tcgen05 tf32, through the C ABI) with the fp64 oracle's
-token-by-token recurrence.
+"""Parity of kda_prefill_chunked (CUDA, through the C ABI) with the fp64 oracle's token-by-token
+recurrence, on both paths: the two-kernel path (a workspace: every chunk's operands in parallel
+with fp16 operands, then the state chain with the fp32 master in tensor memory, segment by
+segment) and the single-kernel path (no workspace; tf32 operands).
 
-Outputs are held to the 2e-3 relative-L2 output budget (they come out near 3e-4: tf32 operands).
-The final state is held to 2e-3 as well: its chunk updates are tf32 contractions, so the 1e-4
-figure of the fp32 decode path does not apply (see the kernel header).
-Both paths are checked: the two-kernel path (a workspace: every chunk's operands in parallel, then
-the state chain, segment by segment) and the single-kernel path (no workspace).
+Outputs are held to the 2e-3 relative-L2 output budget; they come out near 4e-4. The final state
+is held to 1e-3: its chunk updates are fp16 / tf32 contractions (rounding unit 2^-11), so the
+1e-4 figure of the fp32 decode path does not apply. At full size (32,768 tokens, 64 heads) the
+measured state error is 2.9e-4 (3.1e-4 for the worst head) and the test asserts 5e-4 there.
 """
 import numpy as np
 import pytest
@@ -16,7 +17,8 @@ import workloads as wl
 from tests.parity import TOL_OUT, bf16_round, f64, max_rel_l2, rel_l2
 
 pytestmark = pytest.mark.gpu
-TOL_PREFILL_STATE = 2e-3
+TOL_PREFILL_STATE = 1e-3
+TOL_PREFILL_STATE_32K = 5e-4  # measured 2.9e-4 (3.1e-4 worst head)
 
 
 @pytest.fixture(scope="module")
@@ -52,6 +54,7 @@ def test_prefill_shapes(lad, cuda_device, B, H, T, split):
     inp = wl.kda_scan_inputs(cfg)
     o_ref, S_ref = _oracle(inp, scale=0.7)
     o, S = _run(lad, inp, cuda_device, scale=0.7, split=split)
+    print(f"prefill B={B} H={H} T={T} split={split}: o {rel_l2(o, o_ref):.2e} S {rel_l2(S, S_ref):.2e}")
     assert rel_l2(o, o_ref) < TOL_OUT
     assert rel_l2(S, S_ref) < TOL_PREFILL_STATE
 
@@ -130,5 +133,5 @@ def test_prefill_32k_full_size_sampled(lad, cuda_device):
             "S_max_head": max_rel_l2(Sg, S_ref, 2)}
     print("prefill 32k measured relative L2:", errs)
     assert errs["o"] < TOL_OUT and errs["o_max_head"] < TOL_OUT
-    assert errs["S"] < TOL_PREFILL_STATE and errs["S_max_head"] < TOL_PREFILL_STATE
+    assert errs["S"] < TOL_PREFILL_STATE_32K and errs["S_max_head"] < TOL_PREFILL_STATE_32K
     assert torch.isfinite(o).all()
