@@ -892,6 +892,7 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // into registers (32 bytes a thread) at the start of the current item and into the v tile (the
 // 128-byte swizzled MN-major operand layout) once the current item's last reader of that tile is
 // complete; beta is prefetched into a register the same way. The record leaves by bulk stores.
+template <bool kL2>  // kL2: q and k are L2-normalised per token (p.l2norm)
 __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p, const __grid_constant__ PrepMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1016,7 +1017,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         const uint16_t *sq = reinterpret_cast<const uint16_t *>(sm + kPSQ);
         const uint16_t *sk = reinterpret_cast<const uint16_t *>(sm + kPSK);
         const float *sa = reinterpret_cast<const float *>(sm + kPSA);
-        if (p.l2norm) {
+        if constexpr (kL2) {
 #pragma unroll 1
             for (int r = warp; r < kC; r += kPWarps) {
                 const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + 4 * lane);
@@ -1035,9 +1036,6 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
                     s_rk[r] = rsqrtf(sks + 1e-6f);
                 }
             }
-        } else if (tid < kC) {
-            s_rq[tid] = 1.f;
-            s_rk[tid] = 1.f;
         }
 
         // ---- running decays and the operand tiles. Per key channel, g_r = prod_{s <= r} alpha_s and
@@ -1099,9 +1097,16 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
                 const uint2 kw = *reinterpret_cast<const uint2 *>(sk + r * kDk + c4);
                 const float2 q0 = lad::dev::bf16x2_to_f32(qw.x), q1 = lad::dev::bf16x2_to_f32(qw.y);
                 const float2 k0 = lad::dev::bf16x2_to_f32(kw.x), k1 = lad::dev::bf16x2_to_f32(kw.y);
-                const float rq = s_rq[r], rk = s_rk[r];
-                const float qv[4] = {q0.x * rq, q0.y * rq, q1.x * rq, q1.y * rq};
-                const float kv[4] = {k0.x * rk, k0.y * rk, k1.x * rk, k1.y * rk};
+                float qv[4] = {q0.x, q0.y, q1.x, q1.y};
+                float kv[4] = {k0.x, k0.y, k1.x, k1.y};
+                if constexpr (kL2) {
+                    const float rq = s_rq[r], rk = s_rk[r];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        qv[e] *= rq;
+                        kv[e] *= rk;
+                    }
+                }
                 float kh[4], kg[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -1349,9 +1354,10 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
 // boxes of 128 channels x 64 tokens (32 for fp32, which stores a chunk in two halves).
 // Warps 0-7 own the master's rows (warp w: lanes 32 (w % 4) .., columns half w / 4); warp 8 issues
 // the MMAs and the record copies: per chunk the state part first (its own commit, which the master
-// pass waits for), then the output part. The master pass keeps the new state's fp16 copy in
-// registers and writes it over S0's only once the output MMAs (which read S0's) are complete; warp 8
-// waits for them too before reusing the record buffer.
+// pass waits for), then the output part that reads S0's fp16 copy (a second commit), then the rest
+// of the outputs (a third). The master pass keeps the new state's fp16 copy in registers and
+// writes it over S0's once the second commit has landed; warp 8 waits for the third before reusing
+// the record buffer.
 constexpr int kChainThreads = kThreads + 32;
 
 __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(ChainArgs p,
@@ -1359,7 +1365,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
-    const uint32_t rec_bar0 = sbase + kCMisc, mbar_s = sbase + kCMisc + 16, mbar_o = sbase + kCMisc + 24;
+    // mbar_s: the state MMAs; mbar_o: also the output MMAs that read S0's fp16 copy; mbar_p: every
+    // MMA of the chunk (the outputs complete)
+    const uint32_t rec_bar0 = sbase + kCMisc, mbar_s = sbase + kCMisc + 16, mbar_o = sbase + kCMisc + 24,
+                   mbar_p = sbase + kCMisc + 40;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kCMisc + 32);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kCMisc + 36);
 
@@ -1378,6 +1387,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
         mbar_init(rec_bar0 + 8, 1);
         mbar_init(mbar_s, 1);
         mbar_init(mbar_o, 1);
+        mbar_init(mbar_p, 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -1484,7 +1494,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
         bool w = true;
         if (issuer) {
             // ---- S^T += U'^T Kg + S0^T N^T (commit: the master pass may start);
-            //      O^T = U'^T P^T + S0^T Qe^T (commit: waited for here) ----
+            //      O^T = S0^T Qe^T (commit: S0's copy is free) + U'^T P^T (commit: waited for here) ----
             tc_fence_after();
             const uint64_t kg0 = smem_desc(sbase + rs + kRKG, 8192, 1024, kLayoutSw128);
             const uint64_t ua0 = d0 + ((rs + kRU) >> 4), sa0 = d0 + (kCS16 >> 4);
@@ -1496,15 +1506,18 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
                 tc_mma_f16(tmem + kCColS, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRN) >> 4), 16384, j),
                            kIdescSN, 1);
             tc_commit(mbar_s);
-#pragma unroll
-            for (int j = 0; j < kC / 16; ++j)
-                tc_mma_f16(od, kdesc16(ua0, 16384, j), kdesc16(d0 + ((rs + kRP) >> 4), 8192, j), kIdescO, j > 0);
+            // the part that reads S0's copy first, so that the copy is free as early as possible
 #pragma unroll
             for (int j = 0; j < kDk / 16; ++j)
-                tc_mma_f16(od, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRQE) >> 4), 8192, j), kIdescO, 1);
+                tc_mma_f16(od, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRQE) >> 4), 8192, j), kIdescO, j > 0);
             tc_commit(mbar_o);
-            // every MMA of the chunk is complete: its record buffer takes chunk i + 2's
-            w = wait_bar(mbar_o, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
+#pragma unroll
+            for (int j = 0; j < kC / 16; ++j)
+                tc_mma_f16(od, kdesc16(ua0, 16384, j), kdesc16(d0 + ((rs + kRP) >> 4), 8192, j), kIdescO, 1);
+            tc_commit(mbar_p);
+            // every MMA of the chunk is complete: its record buffer takes chunk i + 2's (and the
+            // barrier below publishes the outputs, stored at the next chunk's top)
+            w = wait_bar(mbar_p, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
             if (w && i + 2 < p.nseg) {
                 if (lane == 0) load_rec(i + 2);
                 pend |= 1u << (i & 1);
@@ -1705,8 +1718,11 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
             cudaError_t attr_err =
                 cudaFuncSetAttribute(kda_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
             if (attr_err == cudaSuccess)
-                attr_err = cudaFuncSetAttribute(kda_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                kPSmemBytes);
+                attr_err = cudaFuncSetAttribute(kda_chunk_prep_kernel<false>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
+            if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute(kda_chunk_prep_kernel<true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
             if (attr_err == cudaSuccess)
                 attr_err = cudaFuncSetAttribute(kda_chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 kCSmemBytes);
@@ -1777,8 +1793,11 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
         if (e != cudaSuccess) break;
         const long long items = static_cast<long long>(B) * H * nseg;
         const unsigned pg = static_cast<unsigned>(items < sms ? items : sms);
-        kda_chunk_prep_kernel<<<pg, kPThreads, kPSmemBytes, st>>>(
-            PrepArgs{a.v, beta, buf, counters + sg, B, T, H, c0, nseg, a.l2norm}, pm);
+        const PrepArgs pa{a.v, beta, buf, counters + sg, B, T, H, c0, nseg, a.l2norm};
+        if (a.l2norm)
+            kda_chunk_prep_kernel<true><<<pg, kPThreads, kPSmemBytes, st>>>(pa, pm);
+        else
+            kda_chunk_prep_kernel<false><<<pg, kPThreads, kPSmemBytes, st>>>(pa, pm);
         e = cudaGetLastError();
         if (e == cudaSuccess) e = cudaEventRecord(side->prep_done, st);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(side->st, side->prep_done, 0);
