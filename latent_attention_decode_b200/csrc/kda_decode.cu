@@ -368,6 +368,7 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
 // and the column sums S'^T k and S'^T q reduce over the 8 row groups with three shuffles: the
 // warps never wait for one another inside the token loop.
 constexpr int kMaxMultiTokens = 8;
+constexpr float kLazyMin = 1e-20f;  // smallest cumulative decay the lazy form takes (1 / L <= 1e20)
 constexpr int kMultiCtasPerSm = 2;
 constexpr int kPiecesPerToken = 80;  // 16-byte pieces of one token's inputs: q 16, k 16, v 16, alpha 32
 
@@ -476,14 +477,38 @@ kda_decode_multi_kernel(const uint16_t *__restrict__ q, const uint16_t *__restri
             }
         }
         __syncthreads();
-        // 3. per-row factors {alpha_i, k_i / |k|, q_i / |q|} of every token
-        for (int e = tid; e < n * kD; e += kThreads) {
-            const int t = e >> 7, i = e & (kD - 1);
-            const uint16_t *tq = reinterpret_cast<const uint16_t *>(raw + t * kRawTokenBytes);
-            const float a = reinterpret_cast<const float *>(raw + t * kRawTokenBytes + 768)[i];
-            const float kn = bf16_to_f32(tq[kD + i]) * s_rk[t];
-            rowf[e] = make_float4(a, kn, bf16_to_f32(tq[i]) * s_rq[t], 0.f);
-            rowk[e] = kn;
+        // 3. per-row factors of every token. The decays are applied lazily: with L_t = prod_{s<=t}
+        //    alpha_s per row, the registers hold S~ = S / L (row-wise), so that token t's column sums
+        //    take the coefficients L_t k and L_t q, its update adds (k / L_t) u^T to S~, and only
+        //    the final state is multiplied by L (no per-token decay pass over the state). Row
+        //    factors {L k, L q, L} and k / L. A head whose L falls below kLazyMin on some row (1 / L
+        //    would leave the safe fp32 range) takes the eager form instead: {alpha, k, q} and k.
+        bool lazy_ok = true;
+        if (tid < kD) {
+            const int i = tid;
+            float lam = 1.f, lo = 1.f;
+            for (int t = 0; t < n; ++t) {
+                const uint16_t *tq = reinterpret_cast<const uint16_t *>(raw + t * kRawTokenBytes);
+                const float a = reinterpret_cast<const float *>(raw + t * kRawTokenBytes + 768)[i];
+                const float kn = bf16_to_f32(tq[kD + i]) * s_rk[t];
+                const float qn = bf16_to_f32(tq[i]) * s_rq[t];
+                lam *= a;
+                lo = fminf(lo, lam);
+                rowf[t * kD + i] = make_float4(lam * kn, lam * qn, lam, 0.f);
+                rowk[t * kD + i] = kn / lam;
+            }
+            lazy_ok = lo >= kLazyMin;
+        }
+        const bool lazy = __syncthreads_and(lazy_ok) != 0;
+        if (!lazy) {
+            for (int e = tid; e < n * kD; e += kThreads) {
+                const int t = e >> 7, i = e & (kD - 1);
+                const uint16_t *tq = reinterpret_cast<const uint16_t *>(raw + t * kRawTokenBytes);
+                const float a = reinterpret_cast<const float *>(raw + t * kRawTokenBytes + 768)[i];
+                const float kn = bf16_to_f32(tq[kD + i]) * s_rk[t];
+                rowf[e] = make_float4(a, kn, bf16_to_f32(tq[i]) * s_rq[t], 0.f);
+                rowk[e] = kn;
+            }
         }
         // 4. this head's state: this thread's own slots
         float4 s[kRowsPerWarp];
@@ -501,71 +526,139 @@ kda_decode_multi_kernel(const uint16_t *__restrict__ q, const uint16_t *__restri
                             k, v, alpha, beta, nbh, H, T, nn);
             cp_async_commit();
         }
-        // 6. the tokens
-        for (int t = 0; t < n; ++t) {
-            const float4 *rf = rowf + t * kD + rsub;
-            float4 wk = make_float4(0.f, 0.f, 0.f, 0.f), wq = wk;
-            // two halves with a compiler fence between them, so that at most eight row-factor
-            // loads are hoisted at a time (all sixteen would not fit next to the state)
+        // 6. the tokens (lazy decays, or the eager form)
+        if (lazy) {
+            for (int t = 0; t < n; ++t) {
+                const float4 *rf = rowf + t * kD + rsub;
+                float4 wk = make_float4(0.f, 0.f, 0.f, 0.f), wq = wk;
+                // two halves with a compiler fence between them, so that at most eight row-factor
+                // loads are hoisted at a time (all sixteen would not fit next to the state)
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
+                for (int half = 0; half < 2; ++half) {
 #pragma unroll
-                for (int mm = 0; mm < kRowsPerWarp / 2; ++mm) {
-                    const int m = half * (kRowsPerWarp / 2) + mm;
-                    const float4 f = rf[8 * m];
-                    s[m].x *= f.x;
-                    s[m].y *= f.x;
-                    s[m].z *= f.x;
-                    s[m].w *= f.x;
-                    fma4(wk, f.y, s[m]);
-                    fma4(wq, f.z, s[m]);
+                    for (int mm = 0; mm < kRowsPerWarp / 2; ++mm) {
+                        const int m = half * (kRowsPerWarp / 2) + mm;
+                        const float4 f = rf[8 * m];
+                        fma4(wk, f.x, s[m]);
+                        fma4(wq, f.y, s[m]);
+                    }
+                    asm volatile("" ::: "memory");
                 }
-                asm volatile("" ::: "memory");
-            }
 #pragma unroll
-            for (int x = 4; x < 32; x <<= 1) {
-                wk.x += __shfl_xor_sync(0xffffffffu, wk.x, x);
-                wk.y += __shfl_xor_sync(0xffffffffu, wk.y, x);
-                wk.z += __shfl_xor_sync(0xffffffffu, wk.z, x);
-                wk.w += __shfl_xor_sync(0xffffffffu, wk.w, x);
-                wq.x += __shfl_xor_sync(0xffffffffu, wq.x, x);
-                wq.y += __shfl_xor_sync(0xffffffffu, wq.y, x);
-                wq.z += __shfl_xor_sync(0xffffffffu, wq.z, x);
-                wq.w += __shfl_xor_sync(0xffffffffu, wq.w, x);
-            }
-            const float bt = s_beta[t];
-            const uint2 xv = reinterpret_cast<const uint2 *>(raw + t * kRawTokenBytes + 512)[4 * warp + cq];
-            const float2 v0 = lad::dev::bf16x2_to_f32(xv.x), v1 = lad::dev::bf16x2_to_f32(xv.y);
-            float4 u;
-            u.x = bt * (v0.x - wk.x);
-            u.y = bt * (v0.y - wk.y);
-            u.z = bt * (v1.x - wk.z);
-            u.w = bt * (v1.y - wk.w);
+                for (int x = 4; x < 32; x <<= 1) {
+                    wk.x += __shfl_xor_sync(0xffffffffu, wk.x, x);
+                    wk.y += __shfl_xor_sync(0xffffffffu, wk.y, x);
+                    wk.z += __shfl_xor_sync(0xffffffffu, wk.z, x);
+                    wk.w += __shfl_xor_sync(0xffffffffu, wk.w, x);
+                    wq.x += __shfl_xor_sync(0xffffffffu, wq.x, x);
+                    wq.y += __shfl_xor_sync(0xffffffffu, wq.y, x);
+                    wq.z += __shfl_xor_sync(0xffffffffu, wq.z, x);
+                    wq.w += __shfl_xor_sync(0xffffffffu, wq.w, x);
+                }
+                const float bt = s_beta[t];
+                const uint2 xv = reinterpret_cast<const uint2 *>(raw + t * kRawTokenBytes + 512)[4 * warp + cq];
+                const float2 v0 = lad::dev::bf16x2_to_f32(xv.x), v1 = lad::dev::bf16x2_to_f32(xv.y);
+                float4 u;
+                u.x = bt * (v0.x - wk.x);
+                u.y = bt * (v0.y - wk.y);
+                u.z = bt * (v1.x - wk.z);
+                u.w = bt * (v1.y - wk.w);
 #pragma unroll
-            for (int m = 0; m < kRowsPerWarp; ++m) fma4(s[m], rowk[t * kD + 8 * m + rsub], u);
-            if (o && rsub == 0) {
-                const float qk = s_qk[t];
-                float4 ov;
-                ov.x = scale * fmaf(qk, u.x, wq.x);
-                ov.y = scale * fmaf(qk, u.y, wq.y);
-                ov.z = scale * fmaf(qk, u.z, wq.z);
-                ov.w = scale * fmaf(qk, u.w, wq.w);
-                const size_t orow = ((static_cast<size_t>(b) * T + t) * H + h) * kD;
-                if constexpr (kOutF32) {
-                    reinterpret_cast<float4 *>(static_cast<float *>(o) + orow)[4 * warp + cq] = ov;
-                } else {
-                    uint2 pk;
-                    pk.x = static_cast<uint32_t>(f32_to_bf16(ov.x)) | (static_cast<uint32_t>(f32_to_bf16(ov.y)) << 16);
-                    pk.y = static_cast<uint32_t>(f32_to_bf16(ov.z)) | (static_cast<uint32_t>(f32_to_bf16(ov.w)) << 16);
-                    reinterpret_cast<uint2 *>(static_cast<uint16_t *>(o) + orow)[4 * warp + cq] = pk;
+                for (int m = 0; m < kRowsPerWarp; ++m) fma4(s[m], rowk[t * kD + 8 * m + rsub], u);
+                if (o && rsub == 0) {
+                    const float qk = s_qk[t];
+                    float4 ov;
+                    ov.x = scale * fmaf(qk, u.x, wq.x);
+                    ov.y = scale * fmaf(qk, u.y, wq.y);
+                    ov.z = scale * fmaf(qk, u.z, wq.z);
+                    ov.w = scale * fmaf(qk, u.w, wq.w);
+                    const size_t orow = ((static_cast<size_t>(b) * T + t) * H + h) * kD;
+                    if constexpr (kOutF32) {
+                        reinterpret_cast<float4 *>(static_cast<float *>(o) + orow)[4 * warp + cq] = ov;
+                    } else {
+                        uint2 pk;
+                        pk.x = static_cast<uint32_t>(f32_to_bf16(ov.x)) | (static_cast<uint32_t>(f32_to_bf16(ov.y)) << 16);
+                        pk.y = static_cast<uint32_t>(f32_to_bf16(ov.z)) | (static_cast<uint32_t>(f32_to_bf16(ov.w)) << 16);
+                        reinterpret_cast<uint2 *>(static_cast<uint16_t *>(o) + orow)[4 * warp + cq] = pk;
+                    }
+                }
+            }
+        } else {
+            for (int t = 0; t < n; ++t) {
+                const float4 *rf = rowf + t * kD + rsub;
+                float4 wk = make_float4(0.f, 0.f, 0.f, 0.f), wq = wk;
+                // two halves with a compiler fence between them, so that at most eight row-factor
+                // loads are hoisted at a time (all sixteen would not fit next to the state)
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                    for (int mm = 0; mm < kRowsPerWarp / 2; ++mm) {
+                        const int m = half * (kRowsPerWarp / 2) + mm;
+                        const float4 f = rf[8 * m];
+                        s[m].x *= f.x;
+                        s[m].y *= f.x;
+                        s[m].z *= f.x;
+                        s[m].w *= f.x;
+                        fma4(wk, f.y, s[m]);
+                        fma4(wq, f.z, s[m]);
+                    }
+                    asm volatile("" ::: "memory");
+                }
+#pragma unroll
+                for (int x = 4; x < 32; x <<= 1) {
+                    wk.x += __shfl_xor_sync(0xffffffffu, wk.x, x);
+                    wk.y += __shfl_xor_sync(0xffffffffu, wk.y, x);
+                    wk.z += __shfl_xor_sync(0xffffffffu, wk.z, x);
+                    wk.w += __shfl_xor_sync(0xffffffffu, wk.w, x);
+                    wq.x += __shfl_xor_sync(0xffffffffu, wq.x, x);
+                    wq.y += __shfl_xor_sync(0xffffffffu, wq.y, x);
+                    wq.z += __shfl_xor_sync(0xffffffffu, wq.z, x);
+                    wq.w += __shfl_xor_sync(0xffffffffu, wq.w, x);
+                }
+                const float bt = s_beta[t];
+                const uint2 xv = reinterpret_cast<const uint2 *>(raw + t * kRawTokenBytes + 512)[4 * warp + cq];
+                const float2 v0 = lad::dev::bf16x2_to_f32(xv.x), v1 = lad::dev::bf16x2_to_f32(xv.y);
+                float4 u;
+                u.x = bt * (v0.x - wk.x);
+                u.y = bt * (v0.y - wk.y);
+                u.z = bt * (v1.x - wk.z);
+                u.w = bt * (v1.y - wk.w);
+#pragma unroll
+                for (int m = 0; m < kRowsPerWarp; ++m) fma4(s[m], rowk[t * kD + 8 * m + rsub], u);
+                if (o && rsub == 0) {
+                    const float qk = s_qk[t];
+                    float4 ov;
+                    ov.x = scale * fmaf(qk, u.x, wq.x);
+                    ov.y = scale * fmaf(qk, u.y, wq.y);
+                    ov.z = scale * fmaf(qk, u.z, wq.z);
+                    ov.w = scale * fmaf(qk, u.w, wq.w);
+                    const size_t orow = ((static_cast<size_t>(b) * T + t) * H + h) * kD;
+                    if constexpr (kOutF32) {
+                        reinterpret_cast<float4 *>(static_cast<float *>(o) + orow)[4 * warp + cq] = ov;
+                    } else {
+                        uint2 pk;
+                        pk.x = static_cast<uint32_t>(f32_to_bf16(ov.x)) | (static_cast<uint32_t>(f32_to_bf16(ov.y)) << 16);
+                        pk.y = static_cast<uint32_t>(f32_to_bf16(ov.z)) | (static_cast<uint32_t>(f32_to_bf16(ov.w)) << 16);
+                        reinterpret_cast<uint2 *>(static_cast<uint16_t *>(o) + orow)[4 * warp + cq] = pk;
+                    }
                 }
             }
         }
-        // 7. the new state
+        // 7. the new state (the lazy form's rows times their final L)
         if (write_state && n > 0) {
             float4 *dst = reinterpret_cast<float4 *>(S + static_cast<size_t>(bh) * kD * kD) + thread_f4;
+            const float4 *rl = rowf + (n - 1) * kD + rsub;
 #pragma unroll
-            for (int r = 0; r < kRowsPerWarp; ++r) __stcs(dst + r * 8 * kVec, s[r]);
+            for (int r = 0; r < kRowsPerWarp; ++r) {
+                if (lazy) {
+                    const float l = rl[8 * r].z;
+                    s[r].x *= l;
+                    s[r].y *= l;
+                    s[r].z *= l;
+                    s[r].w *= l;
+                }
+                __stcs(dst + r * 8 * kVec, s[r]);
+            }
         }
         // raw, rowf and the scalars are rewritten next iteration: every thread must be done
         __syncthreads();

@@ -52,6 +52,26 @@ def test_tokens_per_pass(lad, cuda_device, T, alpha_mode):
     assert torch.equal(S16, S)
 
 
+def test_strong_decays_lazy_and_eager(lad, cuda_device):
+    """The kernel applies a head's decays lazily (the registers hold the state divided by the
+    running decay product L of each row; the final state is multiplied back) unless L falls below
+    1e-20 on some row, where it decays the state token by token instead. Head 0 keeps the usual
+    decays, head 1 decays by 1e-4 a token on some rows (L reaches 1e-16: the lazy form with
+    1 / L = 1e16), head 2 by 1e-7 (L reaches 1e-28: the eager form); all three against the oracle."""
+    cfg = wl.KdaScan("sd", B=2, H=3, T=4, seed=46, state_std=0.02, alpha_mode="uniform")
+    inp = wl.kda_scan_inputs(cfg)
+    inp["alpha"][:, :, 1, :32] = 1e-4
+    inp["alpha"][:, :, 2, 64:96] = 1e-7
+    o_ref, S_ref = _oracle(inp)
+    d = _dev(inp, cuda_device)
+    S = d["S0"].clone()
+    o = _call(lad, d, S, out_fp32=True)
+    torch.cuda.synchronize()
+    for h in range(3):
+        assert rel_l2(o[:, :, h], o_ref[:, :, h]) < 1e-5, h
+        assert rel_l2(S[:, h], S_ref[:, h]) < TOL_STATE, h
+
+
 def test_one_token_equals_decode_step(lad, cuda_device):
     """T = 1 is kda_decode_step up to the fp32 summation order of the column sums."""
     cfg = wl.KdaScan("one", B=4, H=6, T=1, seed=50, state_std=0.02, alpha_mode="uniform")
