@@ -967,11 +967,15 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
             *reinterpret_cast<uint4 *>(sm + kPV + (c16 >> 3) * 8192 + tok * 128 + (((c16 & 7) ^ (tok & 7)) << 4)) = vr[e];
         }
     };
+    // one warp watches a barrier's phase; the others wait at the CTA barrier, which costs them no
+    // issue slots (sixteen warps polling the mbarrier would)
     auto mma_wait = [&]() {
-        const bool w = wait_bar(mma_bar, mma_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
+        bool w = true;
+        if (warp == 0) w = wait_bar(mma_bar, mma_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
         mma_phase ^= 1;
+        const bool r = __syncthreads_and(w) != 0;
         tc_fence_after();
-        return __syncthreads_and(w) != 0;
+        return r;
     };
     const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);  // K-major SW128 at offset 0
 
@@ -1008,7 +1012,8 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         load_v(next, nb, nh, nch, v_next);
         if (tid == kPBulkTid) bulk_wait_read1();  // the previous item's Kg, g, P, U'^T have left
         {
-            const bool w = wait_bar(stage_bar, stage_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            bool w = true;
+            if (warp == 0) w = wait_bar(stage_bar, stage_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
             stage_phase ^= 1;
             pending = 0;
             ok = __syncthreads_and(w) != 0;
@@ -1212,11 +1217,14 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         // ---- W -> rows 0-63 of [W; Qt] (over Kt); U'^T -> fp16 tile (over Kh) ----
         {
             // M = 64: row 16 sp + i sits in lane i (< 16) of sub-partition sp; the loads are
-            // collective, so the whole warp issues them and lanes 0-15 keep the rows
+            // collective, so the whole warp issues them and lanes 0-15 keep the rows. Both loads
+            // go out before the one wait.
+            float u[16];
             {
                 const int c0 = 32 * qd;
                 float w[32];
                 tmem_ld32(tmem + lane_base + kPColW + c0, w);
+                tmem_ld16(tmem + lane_base + kPColU + 16 * qd, u);
                 tmem_wait_ld();
                 if (lane < 16) {
                     const int r = 16 * sp + lane;
@@ -1227,9 +1235,6 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
                                        f32x2_to_f16x2(w[j + 4], w[j + 5]), f32x2_to_f16x2(w[j + 6], w[j + 7]));
                 }
             }
-            float u[16];
-            tmem_ld16(tmem + lane_base + kPColU + 16 * qd, u);
-            tmem_wait_ld();
             const int dv = 32 * sp + lane;
 #pragma unroll
             for (int j = 0; j < 16; j += 8)
@@ -1262,16 +1267,15 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         // ---- N = -Kg^T W -> fp16 tile (over the A / T scratch); Qe = Qt - P W -> fp16 tile (over Tb) ----
         {
             const int row = 32 * sp + lane, c0 = 32 * qd;  // d_k' of N; 32 columns
-            float x[32];
+            float x[32], y[32];  // both loads before the one wait
             tmem_ld32(tmem + lane_base + kPColN + c0, x);
+            tmem_ld32(tmem + lane_base + kPColPW + c0, y);  // M = 64: rows in lanes 0-15
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 32; j += 8)
                 *reinterpret_cast<uint4 *>(sm + kPA + sw128_off16(row, c0 + j, 16384)) =
                     make_uint4(f32x2_to_f16x2(-x[j], -x[j + 1]), f32x2_to_f16x2(-x[j + 2], -x[j + 3]),
                                f32x2_to_f16x2(-x[j + 4], -x[j + 5]), f32x2_to_f16x2(-x[j + 6], -x[j + 7]));
-            tmem_ld32(tmem + lane_base + kPColPW + c0, x);  // M = 64: rows in lanes 0-15
-            tmem_wait_ld();
             if (lane < 16) {
                 const int r = 16 * sp + lane;
 #pragma unroll
@@ -1282,7 +1286,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 qf = __half22float2(*reinterpret_cast<const __half2 *>(&qw[e]));
-                        ow[e] = f32x2_to_f16x2(qf.x - x[j + 2 * e], qf.y - x[j + 2 * e + 1]);
+                        ow[e] = f32x2_to_f16x2(qf.x - y[j + 2 * e], qf.y - y[j + 2 * e + 1]);
                     }
                     *reinterpret_cast<uint4 *>(sm + kPTB + sw128_off16(r, c0 + j, 8192)) =
                         make_uint4(ow[0], ow[1], ow[2], ow[3]);
