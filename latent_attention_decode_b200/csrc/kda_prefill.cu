@@ -1633,14 +1633,29 @@ namespace {
 // The split path's workspace: a header of per-segment item counters (256-byte granules), then one
 // segment buffer of records, or two when there are several segments (the prep of segment s + 1
 // writes one while the chain of segment s reads the other).
+// With several segments the last one is short (kTailChunks): its chain is the one piece of work
+// that nothing overlaps, so it should be brief; the segments before it hold up to kSegChunks.
+constexpr int kTailChunks = 32;
 struct WsLayout {
-    long long seg, nsegs, nbuf, header, buf_bytes;
+    long long nch, head, seg, nsegs, nbuf, header, buf_bytes;
+    bool tail(long long k) const { return nsegs > 1 && k == nsegs - 1; }
+    long long first(long long k) const { return tail(k) ? head : k * seg; }  // segment k's first chunk
+    long long count(long long k) const {
+        if (nsegs == 1) return nch;
+        return tail(k) ? nch - head : (seg < head - first(k) ? seg : head - first(k));
+    }
 };
 WsLayout ws_layout(int B, int T, int H) {
     WsLayout L;
-    const long long nch = (static_cast<long long>(T) + kC - 1) / kC;
-    L.seg = nch < kSegChunks ? nch : kSegChunks;
-    L.nsegs = (nch + L.seg - 1) / L.seg;
+    L.nch = (static_cast<long long>(T) + kC - 1) / kC;
+    if (L.nch <= kSegChunks) {
+        L.seg = L.head = L.nch;
+        L.nsegs = 1;
+    } else {
+        L.seg = kSegChunks;
+        L.head = L.nch - kTailChunks;                 // chunks before the tail segment
+        L.nsegs = (L.head + L.seg - 1) / L.seg + 1;  // the last of these starts at chunk `head`
+    }
     L.nbuf = L.nsegs > 1 ? 2 : 1;
     L.header = (L.nsegs * 4 + 255) / 256 * 256;
     L.buf_bytes = static_cast<long long>(B) * H * L.seg * kRecBytes;
@@ -1775,7 +1790,6 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
                   false, f32 ? kC / 2 : kC);
     if (rc != LAD_OK) return rc;
     const WsLayout L = ws_layout(B, T, H);
-    const int nch = (T + kC - 1) / kC;
     const int sms = lad::device_sm_count();
     if (sms <= 0) return set_error(LAD_ECUDA, "kda_prefill_chunked: cannot query the SM count");
     int dev = 0;
@@ -1787,22 +1801,33 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *counters = reinterpret_cast<int *>(ws);
     e = cudaMemsetAsync(counters, 0, static_cast<size_t>(L.header), st);
-    // segment s: prep on the caller's stream, then the chain on the side stream; the prep of s + 1
-    // runs beside the chain of s, and the prep of s + 2 waits for the chain of s to free its buffer
-    for (int sg = 0; sg < L.nsegs && e == cudaSuccess; ++sg) {
-        const int c0 = sg * static_cast<int>(L.seg);
-        const int nseg = nch - c0 < L.seg ? nch - c0 : static_cast<int>(L.seg);
-        uint8_t *buf = ws + L.header + (sg % L.nbuf) * L.buf_bytes;
-        if (sg >= 2) e = cudaStreamWaitEvent(st, side->chain_done[sg & 1], 0);
-        if (e != cudaSuccess) break;
-        const long long items = static_cast<long long>(B) * H * nseg;
-        const unsigned pg = static_cast<unsigned>(items < sms ? items : sms);
+    // Segment s: its prep, then its chain on the side stream. The prep of s + 1 runs beside the chain
+    // of s: `beside` CTAs on the caller's stream take the SMs the chain leaves (a launch that
+    // could take every SM would be placed first and hold them all, the chain waiting behind it),
+    // and the rest join on the side stream as soon as the chain is done, from the same item
+    // counter. The prep of s + 2 waits for the chain of s to free its buffer.
+    const int chain_ctas = B * H < sms ? B * H : sms;
+    const int beside = sms - chain_ctas > sms / 2 ? sms - chain_ctas : sms / 2;
+    auto prep = [&](cudaStream_t on, long long grid, int sg, uint8_t *buf, int c0, int nseg) {
         const PrepArgs pa{a.v, beta, buf, counters + sg, B, T, H, c0, nseg, a.l2norm};
         if (a.l2norm)
-            kda_chunk_prep_kernel<true><<<pg, kPThreads, kPSmemBytes, st>>>(pa, pm);
+            kda_chunk_prep_kernel<true><<<static_cast<unsigned>(grid), kPThreads, kPSmemBytes, on>>>(pa, pm);
         else
-            kda_chunk_prep_kernel<false><<<pg, kPThreads, kPSmemBytes, st>>>(pa, pm);
-        e = cudaGetLastError();
+            kda_chunk_prep_kernel<false><<<static_cast<unsigned>(grid), kPThreads, kPSmemBytes, on>>>(pa, pm);
+        return cudaGetLastError();
+    };
+    for (int sg = 0; sg < L.nsegs && e == cudaSuccess; ++sg) {
+        const int c0 = static_cast<int>(L.first(sg));
+        const int nseg = static_cast<int>(L.count(sg));
+        uint8_t *buf = ws + L.header + (sg % L.nbuf) * L.buf_bytes;
+        const long long items = static_cast<long long>(B) * H * nseg;
+        if (sg == 0) {
+            e = prep(st, items < sms ? items : sms, sg, buf, c0, nseg);
+        } else {
+            if (sg >= 2) e = cudaStreamWaitEvent(st, side->chain_done[sg & 1], 0);
+            if (e == cudaSuccess) e = prep(st, items < beside ? items : beside, sg, buf, c0, nseg);
+            if (e == cudaSuccess) e = prep(side->st, items < sms - beside ? items : sms - beside, sg, buf, c0, nseg);
+        }
         if (e == cudaSuccess) e = cudaEventRecord(side->prep_done, st);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(side->st, side->prep_done, 0);
         if (e != cudaSuccess) break;
