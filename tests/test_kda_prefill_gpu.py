@@ -109,6 +109,41 @@ def test_prefill_several_segments(lad, cuda_device):
     assert rel_l2(o, o1) < TOL_OUT and rel_l2(S, S1) < TOL_PREFILL_STATE
 
 
+def test_prefill_in_a_cuda_graph(lad, cuda_device):
+    """The two-kernel path forks onto the library's side stream and joins back by events, which a
+    stream capture follows: a graph of the call (three segments: 128, 8 and the 32-chunk tail, so
+    both prep launches of a segment and both record buffers take part), replayed twice on fresh
+    inputs, equals the eager call."""
+    cfg = wl.KdaScan("g", B=1, H=2, T=168 * 64, seed=14, state_std=0.02, alpha_mode="uniform")
+    inp = wl.kda_scan_inputs(cfg)
+    d = {n: inp[n].to(cuda_device) for n in ("q", "k", "v", "alpha", "beta")}
+    S = inp["S0"].to(cuda_device).clone()
+    o = torch.empty_like(d["v"])
+    ws = torch.empty(lad.kda_prefill_workspace_size(1, cfg.T, 2, 128, 128, 64), device=cuda_device,
+                     dtype=torch.uint8)
+    S_eager = inp["S0"].to(cuda_device).clone()
+    o_eager = lad.kda_prefill_chunked(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S_eager, workspace=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm the library's per-device state outside the capture
+        lad.kda_prefill_chunked(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S.clone(), o=o, workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        lad.kda_prefill_chunked(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S, o=o, workspace=ws)
+    for _ in range(2):
+        S.copy_(inp["S0"].to(cuda_device))
+        o.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert lad.lad_device_error() == 0
+        assert torch.equal(o, o_eager) and torch.equal(S, S_eager)
+    o_ref, S_ref = _oracle(inp)
+    assert rel_l2(o, o_ref) < TOL_OUT and rel_l2(S, S_ref) < TOL_PREFILL_STATE
+
+
 def test_prefill_empty_sequence_keeps_state(lad, cuda_device):
     cfg = wl.KdaScan("p", B=1, H=2, T=0, seed=12, state_std=0.02)
     inp = wl.kda_scan_inputs(cfg)
