@@ -748,8 +748,12 @@ class PrefillStep(Step):
         self.h_in = [t.cpu().pin_memory() for t in (self.q, self.k, self.v, self.alpha, self.beta)]
         self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
         self.tokens_per_step = cfg.B * cfg.T
-        # the two-kernel path (a workspace is given): prep + scan per segment of up to 128 chunks
-        self.launches_per_step = 2 * math.ceil(math.ceil(cfg.T / cfg.chunk) / 128)
+        # the two-kernel path (a workspace is given): segments of up to 128 chunks, the last one 32
+        # when there are several; the first segment's prep is one launch, every later one two (beside
+        # the previous chain, and behind it), and each segment has one chain launch
+        nch = math.ceil(cfg.T / cfg.chunk)
+        nsegs = 1 if nch <= 128 else math.ceil((nch - 32) / 128) + 1
+        self.launches_per_step = 2 + 3 * (nsegs - 1)
         self.dominant = "kda_prefill_chunked"
         self.config = {"workload": self.name, "batch_per_gpu": cfg.B, "seq_len": cfg.T, "heads": cfg.H,
                        "chunk": cfg.chunk, "l2": f"inputs larger than L2 ({self.algorithmic_bytes()['step'] / 1e9:.2f} GB per step)"}
