@@ -223,9 +223,12 @@ int kda_conv_decode_step(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 
  *                90,624-byte record per (sequence, head, chunk); then the state chain alone.
  *                The chains run on a stream the library keeps per device (highest priority),
  *                ordered by events: the chain of segment s overlaps the operands of segment
- *                s + 1, and `stream` waits for the last chain before any later work on it (the
- *                call stays capturable in a CUDA graph). Without a workspace, one kernel does
- *                both per chunk on `stream`. Same results within rounding.
+ *                s + 1, and `stream` waits for the last chain before any later work on it. The
+ *                call can be captured in a CUDA graph: make the first call on a device outside
+ *                a capture (it creates that stream and its events), and while a captured call's
+ *                capture is open, other threads' calls on the same device must wait for its end
+ *                (the side stream belongs to the capture until then). Without a workspace, one
+ *                kernel does both per chunk on `stream`. Same results within rounding.
  * Supported: dk == dv == 128, chunk == 64; flags LAD_FLAG_L2NORM_QK, LAD_FLAG_OUT_FP32.
  * alpha must keep prod(alpha) over one chunk above ~1e-30 per channel (fp32 range of 1/g); the
  * workspace path also needs every K g_last / g and K / g of a chunk inside the fp16 range.
