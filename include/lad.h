@@ -16,8 +16,10 @@
  *     input checks, read and cleared by lad_device_error()) and the scratch array of
  *     mla_latent_decode_noalloc (below).
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Every
- *     call only enqueues work on that stream and returns; results are ready when the stream
- *     reaches that point.
+ *     call only enqueues work and returns; results are ready when that stream reaches that
+ *     point. One call forks part of its work onto a stream of its own and joins it back by
+ *     events (kda_prefill_chunked with a workspace: one stream and three events per device,
+ *     created at the first such call and kept for the process).
  *   - Tensors are dense, row-major, in the index order written next to each argument.
  *     bf16 tensors hold IEEE bfloat16 bit patterns (lad_bf16); fp32 tensors hold float.
  *   - Return value: LAD_OK (0) or a negative status. On error nothing was launched, except
