@@ -1430,9 +1430,17 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
         tmem_wait_ld();
         const int t0 = (p.c0 + i) * kC;
         if (!p.out_f32) {
-            uint16_t *od = reinterpret_cast<uint16_t *>(sm + kCO) + dv;
+            // a lane pair (d_v, d_v + 1) trades values so that each lane writes a bf16 pair of one
+            // token: the even lane token j, the odd lane token j + 1 (one packed conversion and one
+            // 4-byte store per two values)
+            const int odd = lane & 1;
+            uint32_t *od = reinterpret_cast<uint32_t *>(sm + kCO) + ((32 * cg + odd) * kDv + dv - odd) / 2;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) od[(32 * cg + j) * kDv] = lad::dev::f32_to_bf16(p.scale * x[j]);
+            for (int j = 0; j < 32; j += 2) {
+                const float mine0 = p.scale * x[j], mine1 = p.scale * x[j + 1];
+                const float other = __shfl_xor_sync(0xffffffffu, odd ? mine0 : mine1, 1);
+                od[j * (kDv / 2)] = odd ? bf16x2_rn(other, mine1) : bf16x2_rn(mine0, other);
+            }
             fence_async_smem();
             bar256();
             if (tid == 0) {
