@@ -689,30 +689,57 @@ class HybridStep(Step):
             timer.end(kname)
         self.mla.run(timer)
 
+    def _io_names(self, part):
+        return ("q", "gate", "o") if part is self.mla else ("x", "alpha", "beta", "o")
+
     def run_e2e(self):
-        # Every layer's token inputs are known when the step starts: they go up on a copy stream,
-        # layer by layer, and each layer waits only for its own copy, so later copies overlap
-        # earlier layers. Outputs come back on the compute stream at the end.
+        # A serving loop: two sets of device input / output buffers, so that the next step's token
+        # inputs go up on one copy stream while this step computes, and this step's outputs come
+        # back on another while the next one computes. Every step still copies its own
+        # inputs in and its own outputs out; within a step each layer waits only for its own
+        # inputs. The state and conv tails stay on the device, updated in order by the compute
+        # stream.
         cur = torch.cuda.current_stream()
+        parts = (*self.kda, self.mla)
         if not hasattr(self, "_copy_stream"):
-            self._copy_stream = torch.cuda.Stream()
-        cs = self._copy_stream
-        cs.wait_stream(cur)   # the previous step's kernels are done with these buffers
-        events = []
+            self._copy_stream = torch.cuda.Stream()   # inputs up
+            self._back_stream = torch.cuda.Stream()   # outputs back
+            self._sets = [{id(pt): {n: getattr(pt, n) for n in self._io_names(pt)} for pt in parts}]
+            self._sets.append({id(pt): {n: torch.empty_like(getattr(pt, n)) for n in self._io_names(pt)}
+                               for pt in parts})
+            self._free = [None, None]  # copy-stream event: the set's last outputs are back on the host
+            self._parity = 0
+        cs, p = self._copy_stream, self._parity
+        self._parity ^= 1
+        for pt in parts:
+            for n, t in self._sets[p][id(pt)].items():
+                setattr(pt, n, t)
+        in_events = []
         with torch.cuda.stream(cs):
-            for part in (*self.kda, self.mla):
-                part.h2d()
+            if self._free[p] is not None:
+                cs.wait_event(self._free[p])
+            for pt in parts:
+                pt.h2d()
                 e = torch.cuda.Event()
                 e.record(cs)
-                events.append(e)
-        for layer, e in zip(self.kda, events):
+                in_events.append(e)
+        for pt, e in zip(parts, in_events):
             cur.wait_event(e)
-            layer.run()
-        cur.wait_event(events[-1])
-        self.mla.run()
-        for layer in self.kda:
-            layer.d2h()
-        self.mla.d2h()
+            pt.run()
+        done = torch.cuda.Event()
+        done.record(cur)
+        bs = self._back_stream
+        with torch.cuda.stream(bs):
+            bs.wait_event(done)
+            for pt in parts:
+                pt.d2h()
+            self._free[p] = torch.cuda.Event()
+            self._free[p].record(bs)
+
+    def e2e_drain(self):
+        """The compute stream waits for the outputs still on their way back."""
+        if hasattr(self, "_back_stream"):
+            torch.cuda.current_stream().wait_stream(self._back_stream)
 
     def e2e_bytes(self):
         hb = sum(layer.h2d_bytes() for layer in self.kda) + self.mla.e2e_bytes()[0]
@@ -1113,6 +1140,8 @@ def main(argv=None) -> int:
     e0.record()
     for _ in range(args.steps):
         step.run_e2e()
+    if hasattr(step, "e2e_drain"):
+        step.e2e_drain()
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
