@@ -136,8 +136,6 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
 
     __shared__ float sq[kUnits][kD], sk[kUnits][kD], sv[kUnits][kD], sa[kUnits][kD];
     __shared__ float4 red_k[kWarps][kVec], red_q[kWarps][kVec];
-    __shared__ uint2 s_gate[kVec];   // output gate logits, 4 bf16 per lane of warp 0
-    __shared__ float4 s_gw[kVec];    // norm weight, 4 per lane of warp 0
 
     // the heads' q, k, v (through the fused conv, or as given) and alpha into their slots. With the
     // fused conv, every input of every conv this thread does (q and k channels for threads 0-127, v
@@ -232,6 +230,14 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
     // stored and o written
     auto update = [&](int u, int bh) {
         const float bt = beta[bh];
+        // the output gate's logits and norm weight (4 of each per lane of warp 0, which computes the
+        // outputs): into registers now, used only in the epilogue, so nothing waits for them
+        uint2 gate4 = make_uint2(0u, 0u);
+        float4 w4 = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (gi.g && warp == 0) {
+            gate4 = reinterpret_cast<const uint2 *>(gi.g + static_cast<size_t>(bh) * kD)[lane];
+            if (gi.w) w4 = reinterpret_cast<const float4 *>(gi.w)[lane];
+        }
         // q.k, and the inverse norms when normalising; each warp reduces them itself.
         float qq = 0.f, kk = 0.f, qk = 0.f;
 #pragma unroll
@@ -250,16 +256,6 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
             rk = rsqrtf(kk + 1e-6f);
         }
         qk *= rq * rk;
-
-        // the gate's inputs are fetched here, to land during the decay and the column sums
-        if (gi.g) {
-            if (threadIdx.x < kVec)
-                s_gate[threadIdx.x] =
-                    reinterpret_cast<const uint2 *>(gi.g + static_cast<size_t>(bh) * kD)[threadIdx.x];
-            else if (threadIdx.x < 2 * kVec)
-                s_gw[threadIdx.x - kVec] = gi.w ? reinterpret_cast<const float4 *>(gi.w)[threadIdx.x - kVec]
-                                                : make_float4(1.f, 1.f, 1.f, 1.f);
-        }
 
         // S' = Diag(alpha) S and this warp's share of S'^T k and S'^T q.
         float4 wk = make_float4(0.f, 0.f, 0.f, 0.f), wq = wk;
@@ -310,9 +306,7 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
                 // gated RMSNorm over the head's 128 outputs (4 per lane)
                 const float ss = warp_sum(ov.x * ov.x + ov.y * ov.y + ov.z * ov.z + ov.w * ov.w);
                 const float inv = rsqrtf(ss * (1.f / kD) + gi.eps);
-                const uint2 gw = s_gate[lane];
-                const float2 g01 = lad::dev::bf16x2_to_f32(gw.x), g23 = lad::dev::bf16x2_to_f32(gw.y);
-                const float4 w4 = s_gw[lane];
+                const float2 g01 = lad::dev::bf16x2_to_f32(gate4.x), g23 = lad::dev::bf16x2_to_f32(gate4.y);
                 ov.x *= inv * w4.x / (1.f + __expf(-g01.x));
                 ov.y *= inv * w4.y / (1.f + __expf(-g01.y));
                 ov.z *= inv * w4.z / (1.f + __expf(-g23.x));
