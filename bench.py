@@ -236,6 +236,9 @@ class _KdaLayer:
     kda_decode_step on the conv output (two launches)."""
 
     fused = True
+    # launch the step as a programmatic dependent of the kernel before it (LAD_FLAG_OVERLAP_PREV):
+    # only where that kernel never writes this layer's state, i.e. between different layers
+    overlap = False
 
     def __init__(self, lad, B, seed, dev, tag=""):
         cfg = wl.KdaDecode(f"kda{tag}", B=B, seed=seed)
@@ -256,7 +259,8 @@ class _KdaLayer:
         if self.fused:
             if timer:
                 timer.begin("kda_conv_decode_step")
-            lad.kda_conv_decode_step(self.x, self.tail, self.w, self.alpha, self.beta, self.S, o=self.o)
+            lad.kda_conv_decode_step(self.x, self.tail, self.w, self.alpha, self.beta, self.S, o=self.o,
+                                     overlap_prev=self.overlap)
             if timer:
                 timer.end("kda_conv_decode_step")
             return
@@ -264,7 +268,7 @@ class _KdaLayer:
         if timer:
             timer.begin("kda_decode_step")
         lad.kda_decode_step(self.y[:, :hd], self.y[:, hd:2 * hd], self.y[:, 2 * hd:], self.alpha, self.beta,
-                            self.S, o=self.o, l2norm_qk=True)
+                            self.S, o=self.o, l2norm_qk=True, overlap_prev=self.overlap)
         if timer:
             timer.end("kda_decode_step")
 
@@ -668,13 +672,18 @@ class HybridStep(Step):
     def __init__(self, lad, dev, rank, B=8, ctx=1_000_000, kda_layers=7):
         seed = 1238 + 1000 * rank
         self.kda = [_KdaLayer(lad, B, seed, dev, tag=f"L{i}.") for i in range(kda_layers)]
+        # each layer's kernel follows another layer's (or the MLA combine), never its own state's
+        # previous step, so its state reads may start while that kernel drains
+        for layer in self.kda:
+            layer.overlap = True
         self.mla = MlaDecodeStep(lad, dev, rank, wl.MlaDecode("mla", B=B, seed=seed, fixed_len=ctx))
         self.tokens_per_step = B
         self.launches_per_step = (1 if _KdaLayer.fused else 2) * kda_layers + self.mla.launches_per_step
         self.dominant = "mla_latent_decode"
         self.dominant_units = lambda: self.mla.total_len
         self.config = {"workload": self.name, "batch_per_gpu": B, "layers": f"{kda_layers} KDA + 1 gated MLA",
-                       "kda_path": "fused conv+step" if _KdaLayer.fused else "conv, then step",
+                       "kda_path": ("fused conv+step" if _KdaLayer.fused else "conv, then step")
+                       + ", programmatic dependent launches (state reads overlap the previous layer's drain)",
                        "mla_context": ctx, "heads": H, "head_dim": D,
                        "l2": "inputs larger than L2 (9.2 GB latent cache + 235 MB KDA state per step)"}
 
@@ -696,9 +705,8 @@ class HybridStep(Step):
         # A serving loop: two sets of device input / output buffers, so that the next step's token
         # inputs go up on one copy stream while this step computes, and this step's outputs come
         # back on another while the next one computes. Every step still copies its own
-        # inputs in and its own outputs out; within a step each layer waits only for its own
-        # inputs. The state and conv tails stay on the device, updated in order by the compute
-        # stream.
+        # inputs in and its own outputs out. The state and conv tails stay on the device, updated
+        # in order by the compute stream.
         cur = torch.cuda.current_stream()
         parts = (*self.kda, self.mla)
         if not hasattr(self, "_copy_stream"):
@@ -714,17 +722,18 @@ class HybridStep(Step):
         for pt in parts:
             for n, t in self._sets[p][id(pt)].items():
                 setattr(pt, n, t)
-        in_events = []
         with torch.cuda.stream(cs):
             if self._free[p] is not None:
                 cs.wait_event(self._free[p])
             for pt in parts:
                 pt.h2d()
-                e = torch.cuda.Event()
-                e.record(cs)
-                in_events.append(e)
-        for pt, e in zip(parts, in_events):
-            cur.wait_event(e)
+            landed = torch.cuda.Event()
+            landed.record(cs)
+        # one wait for the whole step's inputs (they went up while the step before it ran), so
+        # that the layers' kernels follow one another on the stream with nothing in between and
+        # each KDA launch overlaps the one before it
+        cur.wait_event(landed)
+        for pt in parts:
             pt.run()
         done = torch.cuda.Event()
         done.record(cur)

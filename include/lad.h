@@ -54,6 +54,14 @@ typedef uint16_t lad_bf16; /* IEEE bfloat16 bit pattern */
 #define LAD_FLAG_OUT_FP32 (1u << 2)  /* KDA and MLA calls: write o as fp32 instead of bf16 */
 #define LAD_FLAG_KEEP_STATE (1u << 3) /* kda_decode_multi: read S but do not write it back */
 #define LAD_FLAG_ROPE_INTERLEAVED (1u << 4) /* RoPE calls: pair dims (2i, 2i+1) instead of (i, i+32) */
+/* kda_decode_step, kda_conv_decode_step(_gated): launch as a programmatic dependent of the kernel
+ * before this call on the stream. The call's CTAs may start, and read the state S, while that
+ * kernel still runs; they read everything else (q, k, v or x, the conv tails, alpha, beta, the
+ * gate) and write anything only once it has finished and its writes are visible. The caller
+ * guarantees that the kernel launched just before this call on the stream does not write S (it
+ * may be another layer's call; it must not be this state's previous step). Every kernel before
+ * that one has finished before this call starts. */
+#define LAD_FLAG_OVERLAP_PREV (1u << 5)
 
 /* Description of the calling thread's most recent error ("" if none). */
 const char *lad_last_error(void);
@@ -132,6 +140,7 @@ int kda_conv_update(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 *w, c
  *   beta      fp32 [B][H]         write strength
  *   S         fp32 [B][H][dk][dv] state, rows = key channels (read and updated in place)
  *   o         [B][H][dv], bf16, or fp32 if flags & LAD_FLAG_OUT_FP32
+ * flags: LAD_FLAG_L2NORM_QK, LAD_FLAG_OUT_FP32, LAD_FLAG_OVERLAP_PREV.
  * Supported: dk == dv == 128; S 16-byte aligned. B == 0 or H == 0 is a no-op.
  */
 int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, long long qkv_batch_stride,
@@ -195,7 +204,8 @@ int kda_decode_multi(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v, co
  *   conv_tail  bf16 [B][K-1][3*H*dk]  tails, oldest row first (read and updated in place)
  *   conv_w     bf16 [3*H*dk][K]       taps (8-byte aligned); conv_bias bf16 [3*H*dk] or NULL
  *   alpha, beta, S, o                 as in kda_decode_step
- * flags: LAD_FLAG_SILU (conv output through SiLU), LAD_FLAG_L2NORM_QK, LAD_FLAG_OUT_FP32.
+ * flags: LAD_FLAG_SILU (conv output through SiLU), LAD_FLAG_L2NORM_QK, LAD_FLAG_OUT_FP32,
+ * LAD_FLAG_OVERLAP_PREV.
  * Supported: dk == dv == 128, K == 4. B == 0 or H == 0 is a no-op.
  */
 int kda_conv_decode_step(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 *conv_w, const lad_bf16 *conv_bias,

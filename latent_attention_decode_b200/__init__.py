@@ -26,7 +26,7 @@ __all__ = [
     "mla_cache_append_fp8", "mla_latent_decode_noalloc",
     "lad_device_error", "lad_check_bounded_wait", "lad_version",
     "LadError", "LIB_PATH", "FLAG_SILU", "FLAG_L2NORM_QK", "FLAG_OUT_FP32", "FLAG_KEEP_STATE",
-    "FLAG_ROPE_INTERLEAVED", "MLA_SCALE", "ROPE_THETA",
+    "FLAG_ROPE_INTERLEAVED", "FLAG_OVERLAP_PREV", "MLA_SCALE", "ROPE_THETA",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblad.so")
@@ -36,6 +36,7 @@ FLAG_L2NORM_QK = 1 << 1
 FLAG_OUT_FP32 = 1 << 2
 FLAG_KEEP_STATE = 1 << 3
 FLAG_ROPE_INTERLEAVED = 1 << 4
+FLAG_OVERLAP_PREV = 1 << 5
 ROPE_THETA = 6.0e6
 MLA_SCALE = 1.0 / math.sqrt(192.0)
 
@@ -212,11 +213,12 @@ def _rows(t: torch.Tensor, name: str, B: int, H: int, d: int) -> int:
 
 def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor,
                     S: torch.Tensor, o: torch.Tensor | None = None, scale: float = 1.0, l2norm_qk: bool = False,
-                    out_fp32: bool = False, stream=None) -> torch.Tensor:
+                    out_fp32: bool = False, overlap_prev: bool = False, stream=None) -> torch.Tensor:
     """One KDA token: S [B,H,128,128] fp32 updated in place; returns o [B,H,128].
 
     q, k, v may be [B,H,128] or [B,H*128] views sharing one batch stride (for example the
-    q, k and v thirds of kda_conv_update's output).
+    q, k and v thirds of kda_conv_update's output). overlap_prev: launch as a programmatic
+    dependent of the kernel before it on the stream, which must not write S.
     """
     _contig(S, "S", torch.float32)
     B, H, dk, dv = S.shape
@@ -230,7 +232,8 @@ def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: to
     if o is None:
         o = torch.empty((B, H, dv), device=S.device, dtype=odt)
     _contig(o, "o", odt)
-    flags = (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
+    flags = ((FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
+             | (FLAG_OVERLAP_PREV if overlap_prev else 0))
     _check("kda_decode_step", _L().kda_decode_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), sq, alpha.data_ptr(),
                                                    beta.data_ptr(), S.data_ptr(), o.data_ptr(), B, H, dk, dv,
                                                    float(scale), flags, _stream(stream)))
@@ -241,9 +244,10 @@ def kda_conv_decode_step_gated(x: torch.Tensor, conv_tail: torch.Tensor, conv_w:
                                beta: torch.Tensor, S: torch.Tensor, gate: torch.Tensor,
                                norm_w: torch.Tensor | None = None, eps: float = 1e-5, o: torch.Tensor | None = None,
                                conv_bias: torch.Tensor | None = None, silu: bool = True, l2norm_qk: bool = True,
-                               scale: float = 1.0, out_fp32: bool = False, stream=None) -> torch.Tensor:
+                               scale: float = 1.0, out_fp32: bool = False, overlap_prev: bool = False,
+                               stream=None) -> torch.Tensor:
     """kda_conv_decode_step with the output gate (gated RMSNorm) fused: gate bf16 [B,H,128] logits,
-    norm_w fp32 [128] (or None). Returns o [B,H,128]."""
+    norm_w fp32 [128] (or None). Returns o [B,H,128]. overlap_prev as in kda_conv_decode_step."""
     bf = torch.bfloat16
     _contig(x, "x", bf), _contig(conv_tail, "conv_tail", bf), _contig(conv_w, "conv_w", bf)
     _contig(S, "S", torch.float32), _contig(alpha, "alpha", torch.float32), _contig(beta, "beta", torch.float32)
@@ -264,7 +268,8 @@ def kda_conv_decode_step_gated(x: torch.Tensor, conv_tail: torch.Tensor, conv_w:
     if o is None:
         o = torch.empty((B, H, dv), device=S.device, dtype=odt)
     _contig(o, "o", odt)
-    flags = ((FLAG_SILU if silu else 0) | (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0))
+    flags = ((FLAG_SILU if silu else 0) | (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
+             | (FLAG_OVERLAP_PREV if overlap_prev else 0))
     _check("kda_conv_decode_step_gated", _L().kda_conv_decode_step_gated(
         x.data_ptr(), conv_tail.data_ptr(), conv_w.data_ptr(), _ptr(conv_bias), alpha.data_ptr(), beta.data_ptr(),
         S.data_ptr(), gate.data_ptr(), _ptr(norm_w), float(eps), o.data_ptr(), B, H, dk, dv, K, float(scale), flags,
@@ -313,9 +318,14 @@ def kda_decode_multi(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: t
 def kda_conv_decode_step(x: torch.Tensor, conv_tail: torch.Tensor, conv_w: torch.Tensor, alpha: torch.Tensor,
                          beta: torch.Tensor, S: torch.Tensor, o: torch.Tensor | None = None,
                          conv_bias: torch.Tensor | None = None, silu: bool = True, l2norm_qk: bool = True,
-                         scale: float = 1.0, out_fp32: bool = False, stream=None) -> torch.Tensor:
+                         scale: float = 1.0, out_fp32: bool = False, overlap_prev: bool = False,
+                         stream=None) -> torch.Tensor:
     """Short conv + KDA step of one layer in one launch. x [B,3*H*128] raw token (q|k|v), conv_tail
-    [B,3,3*H*128] and S [B,H,128,128] updated in place; returns o [B,H,128]."""
+    [B,3,3*H*128] and S [B,H,128,128] updated in place; returns o [B,H,128].
+
+    overlap_prev: launch as a programmatic dependent of the kernel before it on the stream. The
+    call may start and read S while that kernel runs (all else waits for it), so that kernel must
+    not write S: another layer's call, for instance, but not this state's previous step."""
     bf = torch.bfloat16
     _contig(x, "x", bf), _contig(conv_tail, "conv_tail", bf), _contig(conv_w, "conv_w", bf)
     _contig(S, "S", torch.float32), _contig(alpha, "alpha", torch.float32), _contig(beta, "beta", torch.float32)
@@ -331,7 +341,8 @@ def kda_conv_decode_step(x: torch.Tensor, conv_tail: torch.Tensor, conv_w: torch
     if o is None:
         o = torch.empty((B, H, dv), device=S.device, dtype=odt)
     _contig(o, "o", odt)
-    flags = (FLAG_SILU if silu else 0) | (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
+    flags = ((FLAG_SILU if silu else 0) | (FLAG_L2NORM_QK if l2norm_qk else 0) | (FLAG_OUT_FP32 if out_fp32 else 0)
+             | (FLAG_OVERLAP_PREV if overlap_prev else 0))
     _check("kda_conv_decode_step", _L().kda_conv_decode_step(
         x.data_ptr(), conv_tail.data_ptr(), conv_w.data_ptr(), _ptr(conv_bias), alpha.data_ptr(), beta.data_ptr(),
         S.data_ptr(), o.data_ptr(), B, H, dk, dv, K, float(scale), flags, _stream(stream)))

@@ -133,6 +133,13 @@ kda_decode_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k
             "l"(reinterpret_cast<uint64_t>(S + static_cast<size_t>(bh1) * kD * kD)), "r"(kD * kD * 4), "r"(bar)
             : "memory");
     }
+    // Launched as a programmatic dependent (LAD_FLAG_OVERLAP_PREV), the CTAs start while the kernel
+    // before this one on the stream still runs: only the state reads above are issued before this
+    // wait, and everything else (the token inputs, the conv tails, every write) comes after it.
+    // Then the next such launch may start; its CTAs take SMs as these ones leave. Launched
+    // normally, the wait returns at once and the trigger does nothing.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     __shared__ float sq[kUnits][kD], sk[kUnits][kD], sv[kUnits][kD], sa[kUnits][kD];
     __shared__ float4 red_k[kWarps][kVec], red_q[kWarps][kVec];
@@ -684,10 +691,30 @@ int take_device_error_kda(cudaStream_t s, int *code) {
 namespace {
 // One head per CTA, or two (kPair) when B * H is between one and two times the resident CTAs:
 // then every CTA is resident at once and all state bytes are requested together.
+// With `overlap` the launch is a programmatic dependent of the kernel before it on the stream (see
+// the wait at the top of the kernel).
+template <bool kPair, bool kOutF32, bool kFusedConv>
+cudaError_t launch_one(unsigned grid, size_t smem, bool overlap, cudaStream_t s, const uint16_t *q, const uint16_t *k,
+                       const uint16_t *v, long long stride, const float *alpha, const float *beta, float *S, void *o,
+                       int H, float scale, int l2, const ConvIn &cv, const GateIn &gi, int units) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = overlap ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kda_decode_kernel<kOutF32, kFusedConv, kPair>, q, k, v, stride, alpha, beta, S, o,
+                              H, scale, l2, cv, gi, units);
+}
+
 template <bool kOutF32, bool kFusedConv>
 int launch_decode(const char *name, const uint16_t *q, const uint16_t *k, const uint16_t *v, long long stride,
                   const float *alpha, const float *beta, float *S, void *o, int units, int H, float scale, int l2,
-                  const ConvIn &cv, const GateIn &gi, cudaStream_t s) {
+                  const ConvIn &cv, const GateIn &gi, bool overlap, cudaStream_t s) {
     const int sms = lad::device_sm_count();
     const long long slots = 2LL * (sms > 0 ? sms : 0);
     if (sms > 0 && units > slots && units <= 2 * slots) {
@@ -707,11 +734,15 @@ int launch_decode(const char *name, const uint16_t *q, const uint16_t *k, const 
                 done[dev] = true;
             }
         }
-        kda_decode_kernel<kOutF32, kFusedConv, true><<<static_cast<unsigned>(slots), kThreads, kPairSmemBytes, s>>>(
-            q, k, v, stride, alpha, beta, S, o, H, scale, l2, cv, gi, units);
+        const cudaError_t e1 = launch_one<true, kOutF32, kFusedConv>(static_cast<unsigned>(slots), kPairSmemBytes,
+                                                                     overlap, s, q, k, v, stride, alpha, beta, S, o,
+                                                                     H, scale, l2, cv, gi, units);
+        if (e1 != cudaSuccess) return lad::set_error(LAD_ECUDA, "%s: launch: %s", name, cudaGetErrorString(e1));
     } else {
-        kda_decode_kernel<kOutF32, kFusedConv, false><<<static_cast<unsigned>(units), kThreads, 0, s>>>(
-            q, k, v, stride, alpha, beta, S, o, H, scale, l2, cv, gi, units);
+        const cudaError_t e1 = launch_one<false, kOutF32, kFusedConv>(static_cast<unsigned>(units), 0, overlap, s, q,
+                                                                      k, v, stride, alpha, beta, S, o, H, scale, l2,
+                                                                      cv, gi, units);
+        if (e1 != cudaSuccess) return lad::set_error(LAD_ECUDA, "%s: launch: %s", name, cudaGetErrorString(e1));
     }
     return lad::check_launch(name);
 }
@@ -733,7 +764,7 @@ extern "C" int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_b
     if (!lad::aligned(S, 16)) return set_error(LAD_EUNSUPPORTED, "kda_decode_step: S must be 16-byte aligned");
     const bool f32 = (flags & LAD_FLAG_OUT_FP32) != 0;
     if (!lad::aligned(o, f32 ? 16 : 8)) return set_error(LAD_EUNSUPPORTED, "kda_decode_step: o misaligned");
-    if (flags & ~(LAD_FLAG_OUT_FP32 | LAD_FLAG_L2NORM_QK))
+    if (flags & ~(LAD_FLAG_OUT_FP32 | LAD_FLAG_L2NORM_QK | LAD_FLAG_OVERLAP_PREV))
         return set_error(LAD_EINVAL, "kda_decode_step: unknown flags 0x%x", flags);
     const long long blocks = static_cast<long long>(B) * H;
     if (blocks > 0x7fffffffLL) return set_error(LAD_EUNSUPPORTED, "kda_decode_step: B*H too large");
@@ -743,10 +774,11 @@ extern "C" int kda_decode_step(const lad_bf16 *q, const lad_bf16 *k, const lad_b
     const uint16_t *qq = reinterpret_cast<const uint16_t *>(q), *kk = reinterpret_cast<const uint16_t *>(k),
                    *vv = reinterpret_cast<const uint16_t *>(v);
     const int units = static_cast<int>(blocks);
+    const bool ov = (flags & LAD_FLAG_OVERLAP_PREV) != 0;
     return f32 ? launch_decode<true, false>("kda_decode_step", qq, kk, vv, stride, alpha, beta, S, o, units, H, scale,
-                                            l2, none, GateIn{}, s)
+                                            l2, none, GateIn{}, ov, s)
                : launch_decode<false, false>("kda_decode_step", qq, kk, vv, stride, alpha, beta, S, o, units, H, scale,
-                                             l2, none, GateIn{}, s);
+                                             l2, none, GateIn{}, ov, s);
 }
 
 namespace {
@@ -757,7 +789,7 @@ int conv_decode(const char *name, const lad_bf16 *x, lad_bf16 *conv_tail, const 
     if (B < 0 || H < 0) return set_error(LAD_EINVAL, "%s: negative B or H", name);
     if (dk != kD || dv != kD) return set_error(LAD_EUNSUPPORTED, "%s: dk = dv = 128 only", name);
     if (K != 4) return set_error(LAD_EUNSUPPORTED, "%s: K = 4 only", name);
-    if (flags & ~(LAD_FLAG_OUT_FP32 | LAD_FLAG_L2NORM_QK | LAD_FLAG_SILU))
+    if (flags & ~(LAD_FLAG_OUT_FP32 | LAD_FLAG_L2NORM_QK | LAD_FLAG_SILU | LAD_FLAG_OVERLAP_PREV))
         return set_error(LAD_EINVAL, "%s: unknown flags 0x%x", name, flags);
     if (B == 0 || H == 0) return LAD_OK;
     if (!x || !conv_tail || !conv_w || !alpha || !beta || !S || !o) return set_error(LAD_EINVAL, "%s: null pointer", name);
@@ -773,10 +805,11 @@ int conv_decode(const char *name, const lad_bf16 *x, lad_bf16 *conv_tail, const 
     const ConvIn cv{x, conv_tail, conv_w, conv_bias, (flags & LAD_FLAG_SILU) ? 1 : 0};
     cudaStream_t s = lad::as_stream(stream);
     const int units = static_cast<int>(blocks);
+    const bool ov = (flags & LAD_FLAG_OVERLAP_PREV) != 0;
     return f32 ? launch_decode<true, true>(name, nullptr, nullptr, nullptr, 0, alpha, beta, S, o, units, H, scale, l2,
-                                           cv, gi, s)
+                                           cv, gi, ov, s)
                : launch_decode<false, true>(name, nullptr, nullptr, nullptr, 0, alpha, beta, S, o, units, H, scale, l2,
-                                            cv, gi, s);
+                                            cv, gi, ov, s);
 }
 }  // namespace
 

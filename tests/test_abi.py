@@ -49,6 +49,18 @@ def test_host_side_validation(lib):
     assert lad.lad_version() >= 100
 
 
+def test_flag_values_match_the_header(lib):
+    import latent_attention_decode_b200 as lad
+    src = open(os.path.join(ROOT, "include", "lad.h")).read()
+    flags = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define LAD_(FLAG_[A-Z0-9_]+) \(1u << (\d+)\)", src)}
+    assert {"FLAG_SILU", "FLAG_OVERLAP_PREV"} <= set(flags)
+    for name, bit in flags.items():
+        assert getattr(lad, name) == 1 << bit, name
+    # the overlap flag belongs to the single-token KDA calls; the multi-token call rejects it
+    assert lib.kda_decode_multi(16, 16, 16, 16, 16, 16, None, None, 1, 4, 1, 128, 128, 1.0, lad.FLAG_OVERLAP_PREV,
+                                None) == -1
+
+
 def test_host_side_validation_of_the_newer_calls(lib):
     """Each of these returns before any CUDA call (no GPU here)."""
     # kda_decode_multi: more than 8 tokens, unknown flag, head size, empty work

@@ -326,3 +326,43 @@ def test_fused_gated_output(lad, cuda_device, B, H, with_w):
     assert np.array_equal(f64(a["tail"]), tail_ref) and rel_l2(a["S"], S_ref) < TOL_STATE
     o16 = lad.kda_conv_decode_step_gated(b["x"], b["tail"], b["w"], b["alpha"], b["beta"], b["S"].clone(), gate, w)
     assert o16.dtype == torch.bfloat16
+
+
+@pytest.mark.parametrize("B", [8, 64])
+def test_overlap_prev_chain(lad, cuda_device, B):
+    """LAD_FLAG_OVERLAP_PREV: layers launched back to back as programmatic dependents give the
+    results of plain launches bit for bit (B = 8 runs the paired kernel, B = 64 one head a CTA).
+    Each layer's alpha is the fp32 output of the layer before it, so a read of the inputs before
+    the previous kernel has finished would see stale values; the unfused form's step follows the
+    conv that writes its q, k, v. The first layer is also checked against the oracle."""
+    n = 4
+    layers = [wl.kda_decode_inputs(wl.KdaDecode(f"ov{j}", B=B, seed=70 + j), cuda_device) for j in range(n)]
+    gate = wl.normal_bf16((B, 64, 128), 79, "gate", cuda_device, std=2.0)
+    hd = 64 * 128
+    o_ref, S_ref, tail_ref = _fused_oracle(layers[0], 64)
+
+    def run(overlap):
+        ls = [{k: t.clone() for k, t in L.items()} for L in layers]
+        outs = [torch.empty((B, 64, 128), device=cuda_device, dtype=torch.float32) for _ in range(n)]
+        for j, L in enumerate(ls):
+            alpha = L["alpha"] if j == 0 else outs[j - 1]
+            if j == 2:
+                lad.kda_conv_decode_step_gated(L["x"], L["tail"], L["w"], alpha, L["beta"], L["S"], gate, None,
+                                               eps=1e-5, o=outs[j], out_fp32=True, overlap_prev=overlap)
+            elif j == 3:
+                y = lad.kda_conv_update(L["x"], L["tail"], L["w"], silu=True)
+                lad.kda_decode_step(y[:, :hd], y[:, hd:2 * hd], y[:, 2 * hd:], alpha, L["beta"], L["S"], o=outs[j],
+                                    l2norm_qk=True, out_fp32=True, overlap_prev=overlap)
+            else:
+                lad.kda_conv_decode_step(L["x"], L["tail"], L["w"], alpha, L["beta"], L["S"], o=outs[j],
+                                         out_fp32=True, overlap_prev=overlap)
+        torch.cuda.synchronize()
+        return ls, outs
+
+    ls0, outs0 = run(False)
+    ls1, outs1 = run(True)
+    for j in range(n):
+        assert torch.equal(outs0[j], outs1[j]), j
+        assert torch.equal(ls0[j]["S"], ls1[j]["S"]) and torch.equal(ls0[j]["tail"], ls1[j]["tail"]), j
+    assert np.array_equal(f64(ls1[0]["tail"]), tail_ref)
+    assert max_rel_l2(outs1[0], o_ref, 2) < 1e-4 and max_rel_l2(ls1[0]["S"], S_ref, 2) < TOL_STATE
