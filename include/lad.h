@@ -232,7 +232,7 @@ int kda_conv_decode_step(const lad_bf16 *x, lad_bf16 *conv_tail, const lad_bf16 
  *                written by anything else until the call's work on `stream` is done. With it
  *                the call runs two kernels per segment of up to 128 chunks: every chunk's
  *                state-independent operands in parallel, written to the workspace as one
- *                90,624-byte record per (sequence, head, chunk); then the state chain alone.
+ *                74,240-byte record per (sequence, head, chunk); then the state chain alone.
  *                The chains run on a stream the library keeps per device (highest priority),
  *                ordered by events: the chain of segment s overlaps the operands of segment
  *                s + 1, and `stream` waits for the last chain before any later work on it. The
@@ -250,7 +250,7 @@ int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const lad_bf16 *v,
                         float scale, unsigned flags, void *workspace, size_t ws_bytes, void *stream);
 /* Workspace bytes of kda_prefill_chunked's two-kernel path: a 256-byte header (item counters,
  * one per segment, rounded up to 256 bytes) plus B * H * min(ceil(T / 64), 128) records of
- * 90,624 bytes, twice over when T spans more than one segment of 128 chunks (about 1.48 GB for
+ * 74,240 bytes, twice over when T spans more than one segment of 128 chunks (about 1.22 GB for
  * one sequence of 64 heads and more than 8,192 tokens); 0 for unsupported shapes. */
 size_t kda_prefill_workspace_size(int B, int T, int H, int dk, int dv, int chunk);
 

@@ -614,19 +614,19 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
 // ------------------------------------------------------------------------------------------
 // Split path (a workspace is given): the chunk-local, state-independent part of every chunk in
 // parallel (prep), then the state chain alone (chain), segment by segment. With S0 the state
-// entering a chunk, U' = Tb V, W = Tb Kt, P = lower(Qt Kh^T) and Kg = K * g_last / g (the chunk's
-// decay folded into the key), the chunk form
-//   X = W S0,  U = U' - X,  O = scale (Qt S0 + P U),  S = Diag(g_last) S0 + Kg^T U
-// regroups by what multiplies S0:
-//   S = Diag(g_last) S0 + Kg^T U' + N S0,        N = -Kg^T W
-//   O = scale (Qe S0 + P U'),                     Qe = Qt - P W
-// The prep computes N, Qe, Kg, P and U' (all chunk-local); the chain then holds S^T (rows d_v,
-// columns d_k) as an fp32 master in tensor memory and runs one tensor-core batch per chunk
-// (M = 128 value rows):
-//   S^T <- S^T Diag(g_last) (threads, fp32)  +  U'^T Kg  +  S0^T N^T
-//   O^T  = U'^T P^T + S0^T Qe^T
-// so the state makes one trip through the threads per chunk (fp32 master -> fp16 operand copy,
-// and the decay), the decay itself never rounded to fp16.
+// entering a chunk, Tb = (I + A)^-1 diag(beta), W = Tb Kt, P = lower(Qt Kh^T) and
+// Kg = K * g_last / g (the chunk's decay folded into the key), the chunk form is
+//   U' = Tb V,  X = W S0,  U = U' - X,  O = scale (Qt S0 + P U),  S = Diag(g_last) S0 + Kg^T U.
+// The prep computes what needs the CUDA cores (the decays, the operand tiles, the triangular
+// inverse) and one tensor-core product, W; it writes Qt, W, Kg, P, Tb (as a bf16 hi + lo pair)
+// and g_last as one record per chunk. The chain holds S^T (rows d_v, columns d_k) as an fp32
+// master in tensor memory and per chunk runs two tensor-core batches (M = 128 value rows), with
+// one pass through the threads between them and one after:
+//   X^T = S0^T W^T,  O^T = S0^T Qt^T,  U'^T = V^T (Tb_hi + Tb_lo)^T      (V by TMA from the input)
+//   U^T = U'^T - X^T  (threads: fp32 -> fp16 operand)
+//   S^T += U^T Kg,  O^T += U^T P^T
+//   S^T <- S^T Diag(g_last of the next chunk) (threads, fp32), and its fp16 copy (the next S0^T)
+// The decay itself is never rounded to fp16.
 // Every operand is fp16 (kind::f16, fp32 accumulation): its rounding unit is that of tf32 and it
 // runs at twice tf32's rate with half the bytes; each tile is stored once, rows as formed, and
 // the tensor cores read it K-major or MN-major as a contraction needs (no transposed copies).
@@ -635,15 +635,16 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
 // keys that needs a chunk's decay product below about 1.5e-5.
 // ------------------------------------------------------------------------------------------
 
-// Record of one (sequence, head, chunk) in the workspace: the chain's operand tiles (fp16, SW128)
-// and g_last, laid out exactly as in the chain's shared memory (one bulk copy).
-constexpr uint32_t kRN = 0;            // N [128 d_k'][128 d_k], K-major: 2 blocks x 16 KiB
-constexpr uint32_t kRQE = 32768;       // Qe [64 tok][128 d_k], K-major: 2 blocks x 8 KiB
-constexpr uint32_t kRKG = 49152;       // Kg [64 tok][128 d_k]: 2 blocks x 8 KiB (read MN-major)
-constexpr uint32_t kRP = 65536;        // P [64 r][64 s], K-major: 8 KiB
-constexpr uint32_t kRU = 73728;        // U'^T [128 d_v][64 tok], K-major: 16 KiB
-constexpr uint32_t kRG = 90112;        // g_last [128] fp32
-constexpr uint32_t kRecBytes = 90624;  // 708 lines of 128 bytes
+// Record of one (sequence, head, chunk) in the workspace: the chain's operand tiles (fp16 / bf16,
+// SW128) and g_last, laid out exactly as in the chain's shared memory (one bulk copy).
+constexpr uint32_t kRQ = 0;            // Qt [64 tok][128 d_k], K-major: 2 blocks x 8 KiB
+constexpr uint32_t kRW = 16384;        // W [64 tok][128 d_k], K-major: 2 blocks x 8 KiB
+constexpr uint32_t kRKG = 32768;       // Kg [64 tok][128 d_k]: 2 blocks x 8 KiB (read MN-major)
+constexpr uint32_t kRP = 49152;        // P [64 r][64 s], K-major: 8 KiB
+constexpr uint32_t kRTH = 57344;       // Tb, bf16 high part [64 r][64 s], K-major: 8 KiB
+constexpr uint32_t kRTL = 65536;       // Tb, bf16 low part (Tb - hi): 8 KiB
+constexpr uint32_t kRG = 73728;        // g_last [128] fp32
+constexpr uint32_t kRecBytes = 74240;  // 580 lines of 128 bytes
 #ifndef LAD_PREFILL_SEG_CHUNKS
 #define LAD_PREFILL_SEG_CHUNKS 128
 #endif
@@ -671,14 +672,10 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
 constexpr uint32_t kIdescA = make_idesc(128, 64, kFmtF16, 0, 0);     // [Kt; Qt] Kh^T
 constexpr uint32_t kIdescW = make_idesc(64, 128, kFmtF16, 0, 1);     // W = Tb Kt (Kt read MN-major)
 constexpr uint32_t kIdescU = make_idesc(128, 64, kFmtBf16, 1, 0);    // U'^T = V^T Tb^T (V read MN-major)
-constexpr uint32_t kIdescN = make_idesc(128, 128, kFmtF16, 1, 1);    // Kg^T W (both read MN-major)
-constexpr uint32_t kIdescPW = make_idesc(64, 128, kFmtF16, 0, 1);    // P W (W read MN-major)
-constexpr uint32_t kIdescSU = make_idesc(128, 128, kFmtF16, 0, 1);   // S^T += U'^T Kg (Kg read MN-major)
-constexpr uint32_t kIdescSN = make_idesc(128, 128, kFmtF16, 0, 0);   // S^T += S0^T N^T
-constexpr uint32_t kIdescO = make_idesc(128, 64, kFmtF16, 0, 0);     // O^T = U'^T P^T + S0^T Qe^T
+constexpr uint32_t kIdescSU = make_idesc(128, 128, kFmtF16, 0, 1);   // S^T += U^T Kg (Kg read MN-major)
+constexpr uint32_t kIdescO = make_idesc(128, 64, kFmtF16, 0, 0);     // X^T = S0^T W^T, O^T = S0^T Qt^T + U^T P^T
 
 struct PrepArgs {
-    const uint16_t *v;  // [B][T][H][128] bf16 (the prep reads it through registers)
     const float *beta;
     uint8_t *ws;   // this segment's records, [B*H][nseg]
     int *counter;  // the segment's item counter (zero at launch)
@@ -691,38 +688,37 @@ struct PrepMaps {
     CUtensorMap q, k, alpha;  // 3-D [B][T][H*128], boxes of 128 channels x 64 tokens, no swizzle
 };
 
-// prep shared memory (offsets from a 1024-aligned base). Regions are reused once their first
-// contents are dead: Kh (after the first MMA batch) holds U'^T, the Tb tiles (after the second)
-// hold Qe, the A / T scratch (after the solve) holds N. The record leaves by bulk stores from
-// where its tiles sit.
-constexpr uint32_t kPQW = 0;        // [Kt; Qt]: 128 rows x 128 d_k fp16, K-major, 2 blocks x 16 KiB;
-                                    //   rows 0-63 become W once Kt is read
-constexpr uint32_t kPKH = 32768;    // Kh [64 tok][128 d_k], 2 blocks x 8 KiB; then U'^T [128 d_v][64 tok]
+// prep shared memory (offsets from a 1024-aligned base). The A / T scratch holds W once the solve
+// is done with it. The record leaves by bulk stores from where its tiles sit.
+constexpr uint32_t kPQW = 0;        // [Kt; Qt]: 128 rows x 128 d_k fp16, K-major, 2 blocks x 16 KiB (Qt: record)
+constexpr uint32_t kPKH = 32768;    // Kh [64 tok][128 d_k], 2 blocks x 8 KiB
 constexpr uint32_t kPKG = 49152;    // Kg [64 tok][128 d_k], 2 blocks x 8 KiB (record)
 constexpr uint32_t kPP = 65536;     // P [64][64] (record)
 constexpr uint32_t kPG = 73728;     // g_last [128] fp32 (record)
-constexpr uint32_t kPTB = 74752;    // Tb [64 r][64 s] fp16 K-major; then (with TBH) Qe [64][128], 2 x 8 KiB
-constexpr uint32_t kPTBH = 82944;   // Tb, bf16 high part
+constexpr uint32_t kPTB = 74752;    // Tb [64 r][64 s] fp16 K-major
+constexpr uint32_t kPTBH = 82944;   // Tb, bf16 high part (record, with the low part right after it)
 constexpr uint32_t kPTBL = 91136;   // Tb, bf16 low part (Tb - hi)
-constexpr uint32_t kPV = 99328;     // v [64 tok][128 d_v] bf16, two SW128 blocks of 64 d_v (MN-major operand)
+constexpr uint32_t kPSuf = 99328;   // the decay scan's backward products [16 quartets][128] fp32
 constexpr uint32_t kPSQ = 115712;   // q [64 tok][128] bf16, plain (TMA)
 constexpr uint32_t kPSK = 132096;   // k, the same
 constexpr uint32_t kPSA = 148480;   // alpha [64 tok][128] fp32, plain (TMA)
 constexpr int kAS = 68;             // row stride (floats) of the A / T scratch (68: fewer bank conflicts)
-constexpr uint32_t kPA = 181248;    // A [64][kAS] fp32; then (with T) N [128][128] fp16, 2 x 16 KiB
+constexpr uint32_t kPA = 181248;    // A [64][kAS] fp32; then W [64 tok][128 d_k] fp16, 2 blocks x 8 KiB (record)
 constexpr uint32_t kPT = kPA + 64 * kAS * 4;   // T [64][kAS] fp32
 constexpr uint32_t kPMisc = kPT + 64 * kAS * 4;
 constexpr int kPThreads = 512;      // 16 warps: the CUDA-core phases are latency-bound
 constexpr int kPWarps = kPThreads / 32;
 constexpr int kPStageTid = 32;  // issues the input staging (warp 0 issues the MMAs)
 constexpr int kPBulkTid = 64;   // issues the record's bulk stores, in four groups an item, and waits on them
+// the record's four bulk groups of an item, in order: Qt, Kg and g_last (after the formation);
+// P (after the first extraction); Tb hi / lo (after the solve); W (last)
 constexpr uint32_t kPmBeta = 0, kPmRq = 256, kPmRk = 512, kPmOct = 768, kPmBar = 768 + kPWarps * 128 * 4,
                    kPmTmem = kPmBar + 16, kPmAbort = kPmBar + 20, kPmFetch = kPmBar + 24, kPmRg = kPmBar + 32;
 constexpr uint32_t kPSmemBytes = kPMisc + kPmRg + 512 + 1024;
 static_assert(kPSmemBytes <= 232448, "prep shared memory over the per-block limit");
-constexpr uint32_t kPStageTx = 16384 + 16384 + 32768;  // q, k, alpha (v comes through registers)
-// TMEM columns: [Kt; Qt] Kh^T, W, U'^T, Kg^T W, P W
-constexpr uint32_t kPColA = 0, kPColW = 64, kPColU = 192, kPColN = 256, kPColPW = 384, kPTmemCols = 512;
+constexpr uint32_t kPStageTx = 16384 + 16384 + 32768;  // q, k, alpha
+// TMEM columns: [Kt; Qt] Kh^T, W
+constexpr uint32_t kPColA = 0, kPColW = 64, kPTmemCols = 256;
 
 // element (r, s) of the three Tb tiles, four consecutive s at once (s % 4 == 0)
 __device__ __forceinline__ void put_tb4(uint8_t *tb16, uint8_t *tbh, uint8_t *tbl, int r, int s, float a, float b,
@@ -885,13 +881,12 @@ __device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read3() { asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // One CTA per SM walks the segment's (sequence, head, chunk) items with 16 warps. The next item's
-// q, k and alpha are staged (TMA) once the current item's operand tiles are formed; its v comes
-// into registers (32 bytes a thread) at the start of the current item and into the v tile (the
-// 128-byte swizzled MN-major operand layout) once the current item's last reader of that tile is
-// complete; beta is prefetched into a register the same way. The record leaves by bulk stores.
+// q, k and alpha are staged (TMA) once the current item's operand tiles are formed; its beta is
+// prefetched into a register at the start of the current item. The record leaves by bulk stores.
 template <bool kL2>  // kL2: q and k are L2-normalised per token (p.l2norm)
 __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p, const __grid_constant__ PrepMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -901,7 +896,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
     float *s_rq = reinterpret_cast<float *>(sm + kPMisc + kPmRq);
     float *s_rk = reinterpret_cast<float *>(sm + kPMisc + kPmRk);
     float *s_oct = reinterpret_cast<float *>(sm + kPMisc + kPmOct);  // per quartet: forward products
-    float *s_suf = reinterpret_cast<float *>(sm + kPTBL);           //   backward ones (Tb_lo is dead here)
+    float *s_suf = reinterpret_cast<float *>(sm + kPSuf);           //   backward ones
     float *s_rg = reinterpret_cast<float *>(sm + kPMisc + kPmRg);    // 1 / g_last
     float *s_g = reinterpret_cast<float *>(sm + kPG);
     float *sA = reinterpret_cast<float *>(sm + kPA);
@@ -947,26 +942,6 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         tma_load_3d(sbase + kPSK, &maps.k, h * kDk, ch * kC, b, stage_bar);
         tma_load_3d(sbase + kPSA, &maps.alpha, h * kDk, ch * kC, b, stage_bar);
     };
-    // v of an item: thread t holds 16-byte pieces 2t and 2t + 1 (piece p: token p / 16, values
-    // 8 (p % 16) .. + 7); tokens past T read as zero
-    auto load_v = [&](int it, int b, int h, int ch, uint4 (&vr)[2]) {
-        vr[0] = vr[1] = make_uint4(0u, 0u, 0u, 0u);
-        if (it >= nitems) return;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int pc = 2 * tid + e, tok = pc >> 4, t = ch * kC + tok;
-            if (t < p.T)
-                vr[e] = __ldcs(reinterpret_cast<const uint4 *>(p.v + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * kDv) +
-                               (pc & 15));
-        }
-    };
-    auto put_v = [&](const uint4 (&vr)[2]) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int pc = 2 * tid + e, tok = pc >> 4, c16 = pc & 15;
-            *reinterpret_cast<uint4 *>(sm + kPV + (c16 >> 3) * 8192 + tok * 128 + (((c16 & 7) ^ (tok & 7)) << 4)) = vr[e];
-        }
-    };
     // one warp watches a barrier's phase; the others wait at the CTA barrier, which costs them no
     // issue slots (sixteen warps polling the mbarrier would)
     auto mma_wait = [&]() {
@@ -993,12 +968,9 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
     int nb, nh, nch;
     coords(item, nb, nh, nch);
     float beta_next = load_beta(item, nb, nh, nch);
-    uint4 v_next[2];
-    load_v(item, nb, nh, nch, v_next);
     if (item < nitems) {
         if (tid == kPStageTid) stage_qka(nb, nh, nch);
         pending = 1;
-        put_v(v_next);  // the first item's v; the barrier after the staging wait publishes it
     }
     while (item < nitems && ok) {
         const int ch = nch;
@@ -1009,8 +981,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
 
         if (tid < kC) s_beta[tid] = beta_next;
         beta_next = load_beta(next, nb, nh, nch);
-        load_v(next, nb, nh, nch, v_next);
-        if (tid == kPBulkTid) bulk_wait_read1();  // the previous item's Kg, g, P, U'^T have left
+        if (tid == kPBulkTid) bulk_wait_read3();  // the previous item's Qt, Kg and g_last have left
         {
             bool w = true;
             if (warp == 0) w = wait_bar(stage_bar, stage_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
@@ -1140,7 +1111,9 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
             pending = 1;
         }
         if (tid == 0) s_fetch[0] = atomicAdd(p.counter, 1);  // read after this item's last barrier
-        if (tid == kPBulkTid) {  // the record's Kg and g_last are final
+        if (tid == kPBulkTid) {  // the record's Qt, Kg and g_last are final
+            bulk_s2g(rec + kRQ, sbase + kPQW + 8192, 8192);           // rows 64-127 of each block
+            bulk_s2g(rec + kRQ + 8192, sbase + kPQW + 16384 + 8192, 8192);
             bulk_s2g(rec + kRKG, sbase + kPKG, 16384);
             bulk_s2g(rec + kRG, sbase + kPG, 512);
             bulk_commit();
@@ -1153,7 +1126,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
                            kIdescA, j > 0);
             tc_commit(mma_bar);
         }
-        if (tid == kPBulkTid) bulk_wait_read1();  // the previous item's N and Qe have left (A, T, Tb go there)
+        if (tid == kPBulkTid) bulk_wait_read1();  // the previous item's P, Tb hi / lo and W have left
         ok = mma_wait();
         if (!ok) break;
         // ---- A = strict_lower(diag(beta) Kt Kh^T) -> fp32 scratch; P = lower(Qt Kh^T) -> fp16 tile;
@@ -1193,112 +1166,46 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         }
         // ---- T = (I + A)^-1, Tb = T diag(beta) -> the fp16 tile and its bf16 hi / lo split ----
         solve_tb16(sA, sT, s_beta, sm + kPTB, sm + kPTBH, sm + kPTBL, tid);
-        // ---- W = Tb Kt (Kt: rows 0-63 of [Kt; Qt], read MN-major); U'^T = V^T (Tb_hi + Tb_lo)^T ----
+        // ---- W = Tb Kt (Kt: rows 0-63 of [Kt; Qt], read MN-major) ----
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (warp == 0) {
-            tc_fence_after();
-            const uint64_t kt0 = smem_desc(sbase + kPQW, 16384, 1024, kLayoutSw128);  // MN chunks 16 KiB apart
-            const uint64_t v0 = smem_desc(sbase + kPV, 8192, 1024, kLayoutSw128);     // MN chunks 8 KiB apart
-#pragma unroll
-            for (int j = 0; j < kC / 16; ++j) {
-                tc_mma_f16(tmem + kPColW, kdesc16(d0 + (kPTB >> 4), 8192, j), kt0 + ((j * 2048) >> 4), kIdescW, j > 0);
-                tc_mma_f16(tmem + kPColU, v0 + ((j * 2048) >> 4), kdesc16(d0 + (kPTBH >> 4), 8192, j), kIdescU, j > 0);
-            }
-#pragma unroll
-            for (int j = 0; j < kC / 16; ++j)
-                tc_mma_f16(tmem + kPColU, v0 + ((j * 2048) >> 4), kdesc16(d0 + (kPTBL >> 4), 8192, j), kIdescU, 1);
-            tc_commit(mma_bar);
-        }
-        ok = mma_wait();
-        if (!ok) break;
-        put_v(v_next);  // the v tile is read: the next item's goes in (published by the barriers below)
-        // ---- W -> rows 0-63 of [W; Qt] (over Kt); U'^T -> fp16 tile (over Kh) ----
-        {
-            // M = 64: row 16 sp + i sits in lane i (< 16) of sub-partition sp; the loads are
-            // collective, so the whole warp issues them and lanes 0-15 keep the rows. Both loads
-            // go out before the one wait.
-            float u[16];
-            {
-                const int c0 = 32 * qd;
-                float w[32];
-                tmem_ld32(tmem + lane_base + kPColW + c0, w);
-                tmem_ld16(tmem + lane_base + kPColU + 16 * qd, u);
-                tmem_wait_ld();
-                if (lane < 16) {
-                    const int r = 16 * sp + lane;
-#pragma unroll
-                    for (int j = 0; j < 32; j += 8)
-                        *reinterpret_cast<uint4 *>(sm + kPQW + sw128_off16(r, c0 + j, 16384)) =
-                            make_uint4(f32x2_to_f16x2(w[j], w[j + 1]), f32x2_to_f16x2(w[j + 2], w[j + 3]),
-                                       f32x2_to_f16x2(w[j + 4], w[j + 5]), f32x2_to_f16x2(w[j + 6], w[j + 7]));
-                }
-            }
-            const int dv = 32 * sp + lane;
-#pragma unroll
-            for (int j = 0; j < 16; j += 8)
-                *reinterpret_cast<uint4 *>(sm + kPKH + sw128_off16(dv, 16 * qd + j, 16384)) =
-                    make_uint4(f32x2_to_f16x2(u[j], u[j + 1]), f32x2_to_f16x2(u[j + 2], u[j + 3]),
-                               f32x2_to_f16x2(u[j + 4], u[j + 5]), f32x2_to_f16x2(u[j + 6], u[j + 7]));
-        }
-        // ---- Kg^T W (both read MN-major) and P W ----
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == kPBulkTid) {  // U'^T is final
-            bulk_s2g(rec + kRU, sbase + kPKH, 16384);
+        if (tid == kPBulkTid) {  // Tb hi / lo are final
+            bulk_s2g(rec + kRTH, sbase + kPTBH, 16384);
             bulk_commit();
         }
         if (warp == 0) {
             tc_fence_after();
-            const uint64_t kg0 = smem_desc(sbase + kPKG, 8192, 1024, kLayoutSw128);  // MN chunks 8 KiB apart
-            const uint64_t w0 = smem_desc(sbase + kPQW, 16384, 1024, kLayoutSw128);  // MN chunks 16 KiB apart
+            const uint64_t kt0 = smem_desc(sbase + kPQW, 16384, 1024, kLayoutSw128);  // MN chunks 16 KiB apart
 #pragma unroll
-            for (int j = 0; j < kC / 16; ++j) {
-                const uint64_t wj = w0 + ((j * 2048) >> 4);
-                tc_mma_f16(tmem + kPColN, kg0 + ((j * 2048) >> 4), wj, kIdescN, j > 0);
-                tc_mma_f16(tmem + kPColPW, kdesc16(d0 + (kPP >> 4), 8192, j), wj, kIdescPW, j > 0);
-            }
+            for (int j = 0; j < kC / 16; ++j)
+                tc_mma_f16(tmem + kPColW, kdesc16(d0 + (kPTB >> 4), 8192, j), kt0 + ((j * 2048) >> 4), kIdescW, j > 0);
             tc_commit(mma_bar);
         }
         ok = mma_wait();
         if (!ok) break;
-        // ---- N = -Kg^T W -> fp16 tile (over the A / T scratch); Qe = Qt - P W -> fp16 tile (over Tb) ----
+        // ---- W -> fp16 tile over the A / T scratch. M = 64: row 16 sp + i sits in lane i (< 16) of
+        //      sub-partition sp; the load is collective, so the whole warp issues it and lanes 0-15
+        //      keep the rows ----
         {
-            const int row = 32 * sp + lane, c0 = 32 * qd;  // d_k' of N; 32 columns
-            float x[32], y[32];  // both loads before the one wait
-            tmem_ld32(tmem + lane_base + kPColN + c0, x);
-            tmem_ld32(tmem + lane_base + kPColPW + c0, y);  // M = 64: rows in lanes 0-15
+            const int c0 = 32 * qd;
+            float w[32];
+            tmem_ld32(tmem + lane_base + kPColW + c0, w);
             tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; j += 8)
-                *reinterpret_cast<uint4 *>(sm + kPA + sw128_off16(row, c0 + j, 16384)) =
-                    make_uint4(f32x2_to_f16x2(-x[j], -x[j + 1]), f32x2_to_f16x2(-x[j + 2], -x[j + 3]),
-                               f32x2_to_f16x2(-x[j + 4], -x[j + 5]), f32x2_to_f16x2(-x[j + 6], -x[j + 7]));
             if (lane < 16) {
                 const int r = 16 * sp + lane;
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    const uint4 qv = *reinterpret_cast<const uint4 *>(sm + kPQW + sw128_off16(kC + r, c0 + j, 16384));
-                    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-                    uint32_t ow[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 qf = __half22float2(*reinterpret_cast<const __half2 *>(&qw[e]));
-                        ow[e] = f32x2_to_f16x2(qf.x - y[j + 2 * e], qf.y - y[j + 2 * e + 1]);
-                    }
-                    *reinterpret_cast<uint4 *>(sm + kPTB + sw128_off16(r, c0 + j, 8192)) =
-                        make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                }
+                for (int j = 0; j < 32; j += 8)
+                    *reinterpret_cast<uint4 *>(sm + kPA + sw128_off16(r, c0 + j, 8192)) =
+                        make_uint4(f32x2_to_f16x2(w[j], w[j + 1]), f32x2_to_f16x2(w[j + 2], w[j + 3]),
+                                   f32x2_to_f16x2(w[j + 4], w[j + 5]), f32x2_to_f16x2(w[j + 6], w[j + 7]));
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         if (tid == kPBulkTid) {
-            bulk_s2g(rec + kRN, sbase + kPA, 32768);
-            bulk_s2g(rec + kRQE, sbase + kPTB, 16384);
+            bulk_s2g(rec + kRW, sbase + kPA, 16384);
             bulk_commit();
         }
         item = next;
@@ -1336,15 +1243,26 @@ struct ChainArgs {
 
 // chain shared memory (offsets from a 1024-aligned base)
 constexpr uint32_t kCS16 = 0;            // S0^T [128 d_v][128 d_k] fp16, K-major SW128, 2 blocks x 16 KiB
-constexpr uint32_t kCRec = 32768;        // two record buffers, each one record (kRecBytes)
-constexpr uint32_t kCRecStride = 91136;  // 89 KiB (1024-aligned); the barriers sit in buffer 0's slack
+constexpr uint32_t kCRec = 32768;        // two chunk buffers: the record, then the chunk's v tile
+constexpr uint32_t kCV = 74752;          // in a buffer: v [64 tok][128 d_v] bf16 (TMA, SW128, two blocks
+                                         //   of 64 d_v: the MN-major operand), then U^T [128 d_v][64 tok] fp16
+constexpr uint32_t kCRecStride = kCV + 16384;  // 89 KiB (1024-aligned); the barriers sit in buffer 0's slack
 constexpr uint32_t kCO = kCRec + 2 * kCRecStride;  // O [64 tok][128 d_v] bf16 (or 32 tokens x fp32), plain
-constexpr uint32_t kCMisc = kCRec + kRecBytes;     // inside buffer 0's last 512 bytes: 2 record
-                                                   // barriers, state and output MMA barriers, TMEM slot, abort
+constexpr uint32_t kCMisc = kCRec + kRecBytes;     // buffer 0's 512 bytes between record and v tile: 2 chunk
+                                                   // barriers, 3 MMA barriers, TMEM slot, abort
 constexpr uint32_t kCSmemBytes = kCO + 16384 + 1024;
-static_assert(kCMisc + 64 <= kCRec + kCRecStride, "chain barriers must fit in the record slack");
-// TMEM: the fp32 master S^T (128 lanes = d_v, 128 columns = d_k) and two O^T buffers of 64 columns
-constexpr uint32_t kCColS = 0, kCColO = 128, kCTmemCols = 256;
+static_assert(kCMisc + 64 <= kCRec + kCV, "chain barriers must fit in the record slack");
+static_assert(kCV % 1024 == 0 && kCRecStride % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(kCSmemBytes <= 232448, "chain shared memory over the per-block limit");
+constexpr uint32_t kCChunkTx = kRecBytes + 16384;  // a chunk buffer's bytes: the record and the v tile
+// TMEM: the fp32 master S^T (128 lanes = d_v, 128 columns = d_k), two O^T buffers of 64 columns,
+// X^T and U'^T (64 columns each)
+constexpr uint32_t kCColS = 0, kCColO = 128, kCColX = 256, kCColU = 320, kCTmemCols = 512;
+
+struct ChainMaps {
+    CUtensorMap o;  // o as [B][T][H * 128] (bf16, or fp32), boxes of 128 channels x 64 (32) tokens
+    CUtensorMap v;  // v as [B][T][H * 128] bf16, boxes of 64 channels x 64 tokens, 128-byte swizzle
+};
 
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int x, int y, int z) {
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
@@ -1354,24 +1272,23 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
 }
 
 // One CTA per (sequence, head) walks the segment's chunks with the state master in tensor memory.
-// omap: the outputs o as a 3-D tensor [B][T][H * 128] (bf16, or fp32 with LAD_FLAG_OUT_FP32),
-// boxes of 128 channels x 64 tokens (32 for fp32, which stores a chunk in two halves).
 // Warps 0-7 own the master's rows (warp w: lanes 32 (w % 4) .., columns half w / 4); warp 8 issues
-// the MMAs and the record copies: per chunk the state part first (its own commit, which the master
-// pass waits for), then the output part that reads S0's fp16 copy (a second commit), then the rest
-// of the outputs (a third). The master pass keeps the new state's fp16 copy in registers and
-// writes it over S0's once the second commit has landed; warp 8 waits for the third before reusing
-// the record buffer.
+// the MMAs and the chunk copies (the record by one bulk copy, the v tile by two TMA loads, two
+// chunks ahead). Per chunk: the first batch (X^T, the S0 part of O^T, U'^T; one commit); warps 0-7
+// form U^T = U'^T - X^T as the fp16 operand over the v tile and meet warp 8 at a named barrier; the
+// second batch (the state part, its own commit, then the rest of O^T, a third); warps 0-7 then read
+// the new master, write its fp16 copy over S0's (the first batch, its only reader, is complete) and
+// scale the master by the next chunk's decay. The outputs of a chunk leave at the top of the next
+// one, while its first batch runs.
 constexpr int kChainThreads = kThreads + 32;
 
 __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(ChainArgs p,
-                                                                          const __grid_constant__ CUtensorMap omap) {
+                                                                          const __grid_constant__ ChainMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
-    // mbar_s: the state MMAs; mbar_o: also the output MMAs that read S0's fp16 copy; mbar_p: every
-    // MMA of the chunk (the outputs complete)
-    const uint32_t rec_bar0 = sbase + kCMisc, mbar_s = sbase + kCMisc + 16, mbar_o = sbase + kCMisc + 24,
+    // mbar_a: the first batch; mbar_s: the state part of the second; mbar_p: every MMA of the chunk
+    const uint32_t rec_bar0 = sbase + kCMisc, mbar_s = sbase + kCMisc + 16, mbar_a = sbase + kCMisc + 24,
                    mbar_p = sbase + kCMisc + 40;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kCMisc + 32);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kCMisc + 36);
@@ -1390,7 +1307,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
         mbar_init(rec_bar0, 1);
         mbar_init(rec_bar0 + 8, 1);
         mbar_init(mbar_s, 1);
-        mbar_init(mbar_o, 1);
+        mbar_init(mbar_a, 1);
         mbar_init(mbar_p, 1);
         *abort_flag = 0;
         mbar_fence_init();
@@ -1401,18 +1318,22 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    auto load_rec = [&](int i) {  // chunk i's record into buffer i % 2 (one thread)
+    // chunk i's record and v tile into buffer i % 2 (one thread); the v rows past T read as zero
+    auto load_chunk = [&](int i) {
         const uint32_t bar = rec_bar0 + 8u * static_cast<uint32_t>(i & 1);
-        mbar_arrive_tx_raw(bar, kRecBytes);
-        bulk_g2s(sbase + kCRec + static_cast<uint32_t>(i & 1) * kCRecStride,
-                 recs + static_cast<size_t>(i) * kRecBytes, kRecBytes, bar);
+        const uint32_t buf = sbase + kCRec + static_cast<uint32_t>(i & 1) * kCRecStride;
+        mbar_arrive_tx_raw(bar, kCChunkTx);
+        bulk_g2s(buf, recs + static_cast<size_t>(i) * kRecBytes, kRecBytes, bar);
+        const int t0 = (p.c0 + i) * kC;
+        tma_load_3d(buf + kCV, &maps.v, h * kDv, t0, b, bar);
+        tma_load_3d(buf + kCV + 8192, &maps.v, h * kDv + 64, t0, b, bar);
     };
     uint32_t pend = p.nseg > 1 ? 3u : 1u;  // bit j: a copy into buffer j is in flight (issuer's view)
     if (issuer && lane == 0) {
-        load_rec(0);
-        if (p.nseg > 1) load_rec(1);
+        load_chunk(0);
+        if (p.nseg > 1) load_chunk(1);
     }
-    // waits by the calling warp (bounded; warp-uniform result); chunk i's record has landed
+    // waits by the calling warp (bounded; warp-uniform result); chunk i's buffer has landed
     auto rec_ready = [&](int i) {
         const int j = i & 1;
         return wait_bar(rec_bar0 + 8u * j, static_cast<uint32_t>(i >> 1) & 1u, abort_flag, &g_prefill_error,
@@ -1422,6 +1343,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
         return reinterpret_cast<const float *>(sm + kCRec + static_cast<uint32_t>(i & 1) * kCRecStride + kRG);
     };
     auto bar256 = []() { asm volatile("bar.sync 1, 256;" ::: "memory"); };  // warps 0-7 only
+    auto bar288 = []() { asm volatile("bar.sync 2, 288;" ::: "memory"); };  // warps 0-8
     // O of chunk i (O^T in buffer i % 2, complete), scaled, through the O tile and TMA stores;
     // warps 0-7, the previous store having read the tile
     auto store_o = [&](int i) {
@@ -1444,7 +1366,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
             fence_async_smem();
             bar256();
             if (tid == 0) {
-                tma_store_3d(&omap, sbase + kCO, h * kDv, t0, b);
+                tma_store_3d(&maps.o, sbase + kCO, h * kDv, t0, b);
                 bulk_commit();
             }
         } else {
@@ -1459,7 +1381,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
                 }
                 bar256();
                 if (tid == 0) {
-                    tma_store_3d(&omap, sbase + kCO, h * kDv, t0 + 32 * half, b);
+                    tma_store_3d(&maps.o, sbase + kCO, h * kDv, t0 + 32 * half, b);
                     bulk_commit();
                     bulk_wait_read0();
                 }
@@ -1499,50 +1421,81 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
     ok = __syncthreads_and(ok) != 0;
     tc_fence_after();
 
+
     for (int i = 0; i < p.nseg && ok; ++i) {
-        const uint32_t rs = kCRec + static_cast<uint32_t>(i & 1) * kCRecStride;  // this chunk's record
+        const uint32_t rs = kCRec + static_cast<uint32_t>(i & 1) * kCRecStride;  // this chunk's buffer
         const uint32_t od = tmem + kCColO + static_cast<uint32_t>(i & 1) * 64;
         const bool last = i == p.nseg - 1;
         bool w = true;
         if (issuer) {
-            // ---- S^T += U'^T Kg + S0^T N^T (commit: the master pass may start);
-            //      O^T = S0^T Qe^T (commit: S0's copy is free) + U'^T P^T (commit: waited for here) ----
+            // ---- first batch: X^T = S0^T W^T, O^T = S0^T Qt^T, U'^T = V^T (Tb_hi + Tb_lo)^T ----
             tc_fence_after();
+            const uint64_t sa0 = d0 + (kCS16 >> 4);
+            const uint64_t v0 = smem_desc(sbase + rs + kCV, 8192, 1024, kLayoutSw128);  // MN chunks 8 KiB apart
+#pragma unroll
+            for (int j = 0; j < kDk / 16; ++j) {
+                tc_mma_f16(tmem + kCColX, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRW) >> 4), 8192, j), kIdescO,
+                           j > 0);
+                tc_mma_f16(od, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRQ) >> 4), 8192, j), kIdescO, j > 0);
+            }
+#pragma unroll
+            for (int j = 0; j < kC / 16; ++j)
+                tc_mma_f16(tmem + kCColU, v0 + ((j * 2048) >> 4), kdesc16(d0 + ((rs + kRTH) >> 4), 8192, j), kIdescU,
+                           j > 0);
+#pragma unroll
+            for (int j = 0; j < kC / 16; ++j)
+                tc_mma_f16(tmem + kCColU, v0 + ((j * 2048) >> 4), kdesc16(d0 + ((rs + kRTL) >> 4), 8192, j), kIdescU,
+                           1);
+            tc_commit(mbar_a);
+            bar288();  // U^T is in place (over the v tile)
+            tc_fence_after();
+            // ---- second batch: S^T += U^T Kg (commit: the master pass may start); O^T += U^T P^T
+            //      (commit: waited for here) ----
+            const uint64_t ut0 = d0 + ((rs + kCV) >> 4);
             const uint64_t kg0 = smem_desc(sbase + rs + kRKG, 8192, 1024, kLayoutSw128);
-            const uint64_t ua0 = d0 + ((rs + kRU) >> 4), sa0 = d0 + (kCS16 >> 4);
 #pragma unroll
             for (int j = 0; j < kC / 16; ++j)
-                tc_mma_f16(tmem + kCColS, kdesc16(ua0, 16384, j), kg0 + ((j * 2048) >> 4), kIdescSU, 1);
-#pragma unroll
-            for (int j = 0; j < kDk / 16; ++j)
-                tc_mma_f16(tmem + kCColS, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRN) >> 4), 16384, j),
-                           kIdescSN, 1);
+                tc_mma_f16(tmem + kCColS, kdesc16(ut0, 16384, j), kg0 + ((j * 2048) >> 4), kIdescSU, 1);
             tc_commit(mbar_s);
-            // the part that reads S0's copy first, so that the copy is free as early as possible
-#pragma unroll
-            for (int j = 0; j < kDk / 16; ++j)
-                tc_mma_f16(od, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRQE) >> 4), 8192, j), kIdescO, j > 0);
-            tc_commit(mbar_o);
 #pragma unroll
             for (int j = 0; j < kC / 16; ++j)
-                tc_mma_f16(od, kdesc16(ua0, 16384, j), kdesc16(d0 + ((rs + kRP) >> 4), 8192, j), kIdescO, 1);
+                tc_mma_f16(od, kdesc16(ut0, 16384, j), kdesc16(d0 + ((rs + kRP) >> 4), 8192, j), kIdescO, 1);
             tc_commit(mbar_p);
-            // every MMA of the chunk is complete: its record buffer takes chunk i + 2's (and the
-            // barrier below publishes the outputs, stored at the next chunk's top)
+            // every MMA of the chunk is complete: its buffer takes chunk i + 2's (and the barrier
+            // below publishes the outputs, stored at the next chunk's top)
             w = wait_bar(mbar_p, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
             if (w && i + 2 < p.nseg) {
-                if (lane == 0) load_rec(i + 2);
+                if (lane == 0) load_chunk(i + 2);
                 pend |= 1u << (i & 1);
             }
         } else {
-            // ---- while they run: the previous chunk's outputs leave ----
+            // ---- while the first batch runs: the previous chunk's outputs leave ----
             if (i > 0) store_o(i - 1);
-            w = wait_bar(mbar_s, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            w = wait_bar(mbar_a, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            tc_fence_after();
+            // ---- U^T = U'^T - X^T -> the fp16 operand, over the v tile (its reader is complete) ----
+            if (w) {
+                float x[32], u[32];  // both loads before the one wait
+                tmem_ld32(tmem + lane_base + kCColX + 32 * cg, x);
+                tmem_ld32(tmem + lane_base + kCColU + 32 * cg, u);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; j += 8)
+                    *reinterpret_cast<uint4 *>(sm + rs + kCV + sw128_off16(dv, 32 * cg + j, 16384)) =
+                        make_uint4(f32x2_to_f16x2(u[j] - x[j], u[j + 1] - x[j + 1]),
+                                   f32x2_to_f16x2(u[j + 2] - x[j + 2], u[j + 3] - x[j + 3]),
+                                   f32x2_to_f16x2(u[j + 4] - x[j + 4], u[j + 5] - x[j + 5]),
+                                   f32x2_to_f16x2(u[j + 6] - x[j + 6], u[j + 7] - x[j + 7]));
+            }
+            fence_async_smem();
+            tc_fence_before();
+            bar288();
+            if (w) w = wait_bar(mbar_s, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
             if (w && !last) w = rec_ready(i + 1);  // the next chunk's decay
             tc_fence_after();
-            uint32_t hv[32];  // the new state's fp16 copy, held until the output MMAs have read S0
             if (w) {
-                // ---- the new state: its fp16 copy and the next chunk's decay (or the state out) ----
+                // ---- the new state: its fp16 copy over S0's (the first batch, S0's only reader, is
+                //      complete) and the next chunk's decay (or the state out) ----
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
                     const int c0 = 64 * cg + 32 * part;
@@ -1555,7 +1508,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
                         for (int j = 0; j < 32; ++j) Sout[static_cast<size_t>(c0 + j) * kDv] = v[j];
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) hv[16 * part + j] = f32x2_to_f16x2(v[2 * j], v[2 * j + 1]);
+                        for (int j = 0; j < 32; j += 8)
+                            *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, c0 + j, 16384)) =
+                                make_uint4(f32x2_to_f16x2(v[j], v[j + 1]), f32x2_to_f16x2(v[j + 2], v[j + 3]),
+                                           f32x2_to_f16x2(v[j + 4], v[j + 5]), f32x2_to_f16x2(v[j + 6], v[j + 7]));
                         const float4 *gn = reinterpret_cast<const float4 *>(gl_of(i + 1) + c0);
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
@@ -1570,14 +1526,6 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
                 }
                 tmem_wait_st();
             }
-            // the output MMAs read S0's fp16 copy: it is overwritten only once they are complete
-            if (w) w = wait_bar(mbar_o, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
-            if (w && !last) {
-#pragma unroll
-                for (int j = 0; j < 64; j += 8)
-                    *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, 64 * cg + j, 16384)) =
-                        make_uint4(hv[j / 2], hv[j / 2 + 1], hv[j / 2 + 2], hv[j / 2 + 3]);
-            }
             if (tid == 0) bulk_wait_read0();  // the previous outputs have left the O tile
         }
         fence_async_smem();
@@ -1586,7 +1534,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
         tc_fence_after();
         if (ok && last && !issuer) store_o(i);
     }
-    // drain: record copies still in flight (after an abort) land, the output stores complete and
+    // drain: chunk copies still in flight (after an abort) land, the output stores complete and
     // every MMA this CTA issued completes, before shared memory and TMEM are released
     if (issuer) {
         if (lane == 0) {
@@ -1602,10 +1550,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
             }
         }
         __syncwarp();
-        tc_commit(mbar_o);  // warp-wide (elect.sync): a fresh completion covering every MMA issued
+        tc_commit(mbar_a);  // warp-wide (elect.sync): a fresh completion covering every MMA issued
         if (lane == 0) {
             const uint64_t t1 = lad::dev::globaltimer_ns();
-            while (!mbar_try_wait(mbar_o, static_cast<uint32_t>(p.nseg) & 1u) &&
+            while (!mbar_try_wait(mbar_a, static_cast<uint32_t>(p.nseg) & 1u) &&
                    lad::dev::globaltimer_ns() - t1 < lad::dev::kWaitLimitNs) {
             }
         }
@@ -1792,10 +1740,11 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
     int rc = make(&pm.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk, false);
     if (rc == LAD_OK) rc = make(&pm.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDk, false);
     if (rc == LAD_OK) rc = make(&pm.alpha, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDk, false);
-    CUtensorMap omap;
+    ChainMaps cm;
     if (rc == LAD_OK)
-        rc = make(&omap, o, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 ? 4 : 2, kDv,
+        rc = make(&cm.o, o, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 ? 4 : 2, kDv,
                   false, f32 ? kC / 2 : kC);
+    if (rc == LAD_OK) rc = make(&cm.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, true);
     if (rc != LAD_OK) return rc;
     const WsLayout L = ws_layout(B, T, H);
     const int sms = lad::device_sm_count();
@@ -1817,7 +1766,7 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
     const int chain_ctas = B * H < sms ? B * H : sms;
     const int beside = sms - chain_ctas > sms / 2 ? sms - chain_ctas : sms / 2;
     auto prep = [&](cudaStream_t on, long long grid, int sg, uint8_t *buf, int c0, int nseg) {
-        const PrepArgs pa{a.v, beta, buf, counters + sg, B, T, H, c0, nseg, a.l2norm};
+        const PrepArgs pa{beta, buf, counters + sg, B, T, H, c0, nseg, a.l2norm};
         if (a.l2norm)
             kda_chunk_prep_kernel<true><<<static_cast<unsigned>(grid), kPThreads, kPSmemBytes, on>>>(pa, pm);
         else
@@ -1840,7 +1789,7 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
         if (e == cudaSuccess) e = cudaStreamWaitEvent(side->st, side->prep_done, 0);
         if (e != cudaSuccess) break;
         kda_chunk_chain_kernel<<<static_cast<unsigned>(B * H), kChainThreads, kCSmemBytes, side->st>>>(
-            ChainArgs{S, o, buf, B, T, H, c0, nseg, scale, a.out_f32}, omap);
+            ChainArgs{S, o, buf, B, T, H, c0, nseg, scale, a.out_f32}, cm);
         e = cudaGetLastError();
         if (e == cudaSuccess) e = cudaEventRecord(side->chain_done[sg & 1], side->st);
     }

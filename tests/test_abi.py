@@ -128,11 +128,11 @@ def test_host_side_validation_of_the_fp8_calls(lib):
 
 def test_prefill_workspace_size(lib):
     """The two-kernel prefill path's workspace: a 256-byte header of per-segment item counters,
-    then one 90,624-byte record (fp16 operand tiles, g_last and U') per (sequence, head, chunk) of
+    then one 74,240-byte record (fp16 / bf16 operand tiles and g_last) per (sequence, head, chunk) of
     a segment of at most 128 chunks, twice over when there are several segments (one segment's
     records are read while the next one's are written); zero for shapes the call does not
     support."""
-    rec, hdr = 90624, 256
+    rec, hdr = 74240, 256
     assert lib.kda_prefill_workspace_size(1, 32768, 64, 128, 128, 64) == hdr + 2 * 64 * 128 * rec
     assert lib.kda_prefill_workspace_size(1, 128 * 64 + 1, 1, 128, 128, 64) == hdr + 2 * 128 * rec
     assert lib.kda_prefill_workspace_size(1, 128 * 64, 1, 128, 128, 64) == hdr + 128 * rec
