@@ -637,8 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
 
 // Record of one (sequence, head, chunk) in the workspace: the chain's operand tiles (fp16 / bf16,
 // SW128) and g_last, laid out exactly as in the chain's shared memory (one bulk copy).
-constexpr uint32_t kRQ = 0;            // Qt [64 tok][128 d_k], K-major: 2 blocks x 8 KiB
-constexpr uint32_t kRW = 16384;        // W [64 tok][128 d_k], K-major: 2 blocks x 8 KiB
+constexpr uint32_t kRWQ = 0;           // [W; Qt] [128 rows: 64 W, 64 Qt tok][128 d_k], K-major: 2 blocks x 16 KiB
 constexpr uint32_t kRKG = 32768;       // Kg [64 tok][128 d_k]: 2 blocks x 8 KiB (read MN-major)
 constexpr uint32_t kRP = 49152;        // P [64 r][64 s], K-major: 8 KiB
 constexpr uint32_t kRTH = 57344;       // Tb, bf16 high part [64 r][64 s], K-major: 8 KiB
@@ -673,7 +672,8 @@ constexpr uint32_t kIdescA = make_idesc(128, 64, kFmtF16, 0, 0);     // [Kt; Qt]
 constexpr uint32_t kIdescW = make_idesc(64, 128, kFmtF16, 0, 1);     // W = Tb Kt (Kt read MN-major)
 constexpr uint32_t kIdescU = make_idesc(128, 64, kFmtBf16, 1, 0);    // U'^T = V^T Tb^T (V read MN-major)
 constexpr uint32_t kIdescSU = make_idesc(128, 128, kFmtF16, 0, 1);   // S^T += U^T Kg (Kg read MN-major)
-constexpr uint32_t kIdescO = make_idesc(128, 64, kFmtF16, 0, 0);     // X^T = S0^T W^T, O^T = S0^T Qt^T + U^T P^T
+constexpr uint32_t kIdescXO = make_idesc(128, 128, kFmtF16, 0, 0);  // [X^T | O^T] = S0^T [W; Qt]^T
+constexpr uint32_t kIdescO = make_idesc(128, 64, kFmtF16, 0, 0);     // O^T += U^T P^T
 
 struct PrepArgs {
     const float *beta;
@@ -1112,8 +1112,8 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         }
         if (tid == 0) s_fetch[0] = atomicAdd(p.counter, 1);  // read after this item's last barrier
         if (tid == kPBulkTid) {  // the record's Qt, Kg and g_last are final
-            bulk_s2g(rec + kRQ, sbase + kPQW + 8192, 8192);           // rows 64-127 of each block
-            bulk_s2g(rec + kRQ + 8192, sbase + kPQW + 16384 + 8192, 8192);
+            bulk_s2g(rec + kRWQ + 8192, sbase + kPQW + 8192, 8192);  // rows 64-127 of each block
+            bulk_s2g(rec + kRWQ + 16384 + 8192, sbase + kPQW + 16384 + 8192, 8192);
             bulk_s2g(rec + kRKG, sbase + kPKG, 16384);
             bulk_s2g(rec + kRG, sbase + kPG, 512);
             bulk_commit();
@@ -1205,7 +1205,8 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
         tc_fence_before();
         __syncthreads();
         if (tid == kPBulkTid) {
-            bulk_s2g(rec + kRW, sbase + kPA, 16384);
+            bulk_s2g(rec + kRWQ, sbase + kPA, 8192);  // rows 0-63 of each block
+            bulk_s2g(rec + kRWQ + 16384, sbase + kPA + 8192, 8192);
             bulk_commit();
         }
         item = next;
@@ -1255,9 +1256,9 @@ static_assert(kCMisc + 64 <= kCRec + kCV, "chain barriers must fit in the record
 static_assert(kCV % 1024 == 0 && kCRecStride % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(kCSmemBytes <= 232448, "chain shared memory over the per-block limit");
 constexpr uint32_t kCChunkTx = kRecBytes + 16384;  // a chunk buffer's bytes: the record and the v tile
-// TMEM: the fp32 master S^T (128 lanes = d_v, 128 columns = d_k), two O^T buffers of 64 columns,
-// X^T and U'^T (64 columns each)
-constexpr uint32_t kCColS = 0, kCColO = 128, kCColX = 256, kCColU = 320, kCTmemCols = 512;
+// TMEM: the fp32 master S^T (128 lanes = d_v, 128 columns = d_k), two [X^T | O^T] buffers of
+// 128 columns (chunk parity), U'^T (64 columns)
+constexpr uint32_t kCColS = 0, kCColXO = 128, kCColU = 384, kCTmemCols = 512;
 
 struct ChainMaps {
     CUtensorMap o;  // o as [B][T][H * 128] (bf16, or fp32), boxes of 128 channels x 64 (32) tokens
@@ -1274,12 +1275,13 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
 // One CTA per (sequence, head) walks the segment's chunks with the state master in tensor memory.
 // Warps 0-7 own the master's rows (warp w: lanes 32 (w % 4) .., columns half w / 4); warp 8 issues
 // the MMAs and the chunk copies (the record by one bulk copy, the v tile by two TMA loads, two
-// chunks ahead). Per chunk: the first batch (X^T, the S0 part of O^T, U'^T; one commit); warps 0-7
-// form U^T = U'^T - X^T as the fp16 operand over the v tile and meet warp 8 at a named barrier; the
-// second batch (the state part, its own commit, then the rest of O^T, a third); warps 0-7 then read
-// the new master, write its fp16 copy over S0's (the first batch, its only reader, is complete) and
-// scale the master by the next chunk's decay. The outputs of a chunk leave at the top of the next
-// one, while its first batch runs.
+// chunks ahead). Per chunk: the first batch ([X^T | O^T] from S0's fp16 copy, U'^T; one commit),
+// while warps 0-7 send the previous chunk's outputs out; warps 0-7 form U^T = U'^T - X^T as the
+// fp16 operand over the v tile and meet warp 8 at a named barrier; the second batch (the state
+// part, its own commit, then the rest of O^T, a third); warps 0-7 then read the new master, write
+// its fp16 copy over S0's (the first batch, its only reader, is complete) and scale the master by
+// the next chunk's decay. The threads touch tensor memory while the tensor cores are idle where
+// they can: a decay pass run beside the first batch took three times as long.
 constexpr int kChainThreads = kThreads + 32;
 
 __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(ChainArgs p,
@@ -1348,7 +1350,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
     // warps 0-7, the previous store having read the tile
     auto store_o = [&](int i) {
         float x[32];
-        tmem_ld32(tmem + lane_base + kCColO + static_cast<uint32_t>(i & 1) * 64 + 32 * cg, x);
+        tmem_ld32(tmem + lane_base + kCColXO + static_cast<uint32_t>(i & 1) * 128 + 64 + 32 * cg, x);
         tmem_wait_ld();
         const int t0 = (p.c0 + i) * kC;
         if (!p.out_f32) {
@@ -1424,20 +1426,17 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
 
     for (int i = 0; i < p.nseg && ok; ++i) {
         const uint32_t rs = kCRec + static_cast<uint32_t>(i & 1) * kCRecStride;  // this chunk's buffer
-        const uint32_t od = tmem + kCColO + static_cast<uint32_t>(i & 1) * 64;
+        const uint32_t xo = tmem + kCColXO + static_cast<uint32_t>(i & 1) * 128;  // [X^T | O^T]
         const bool last = i == p.nseg - 1;
         bool w = true;
         if (issuer) {
-            // ---- first batch: X^T = S0^T W^T, O^T = S0^T Qt^T, U'^T = V^T (Tb_hi + Tb_lo)^T ----
+            // ---- first batch: [X^T | O^T] = S0^T [W; Qt]^T, U'^T = V^T (Tb_hi + Tb_lo)^T ----
             tc_fence_after();
             const uint64_t sa0 = d0 + (kCS16 >> 4);
             const uint64_t v0 = smem_desc(sbase + rs + kCV, 8192, 1024, kLayoutSw128);  // MN chunks 8 KiB apart
 #pragma unroll
-            for (int j = 0; j < kDk / 16; ++j) {
-                tc_mma_f16(tmem + kCColX, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRW) >> 4), 8192, j), kIdescO,
-                           j > 0);
-                tc_mma_f16(od, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRQ) >> 4), 8192, j), kIdescO, j > 0);
-            }
+            for (int j = 0; j < kDk / 16; ++j)
+                tc_mma_f16(xo, kdesc16(sa0, 16384, j), kdesc16(d0 + ((rs + kRWQ) >> 4), 16384, j), kIdescXO, j > 0);
 #pragma unroll
             for (int j = 0; j < kC / 16; ++j)
                 tc_mma_f16(tmem + kCColU, v0 + ((j * 2048) >> 4), kdesc16(d0 + ((rs + kRTH) >> 4), 8192, j), kIdescU,
@@ -1459,10 +1458,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
             tc_commit(mbar_s);
 #pragma unroll
             for (int j = 0; j < kC / 16; ++j)
-                tc_mma_f16(od, kdesc16(ut0, 16384, j), kdesc16(d0 + ((rs + kRP) >> 4), 8192, j), kIdescO, 1);
+                tc_mma_f16(xo + 64, kdesc16(ut0, 16384, j), kdesc16(d0 + ((rs + kRP) >> 4), 8192, j), kIdescO, 1);
             tc_commit(mbar_p);
             // every MMA of the chunk is complete: its buffer takes chunk i + 2's (and the barrier
-            // below publishes the outputs, stored at the next chunk's top)
+            // below publishes the outputs, stored while the next chunk's first batch runs)
             w = wait_bar(mbar_p, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
             if (w && i + 2 < p.nseg) {
                 if (lane == 0) load_chunk(i + 2);
@@ -1476,7 +1475,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
             // ---- U^T = U'^T - X^T -> the fp16 operand, over the v tile (its reader is complete) ----
             if (w) {
                 float x[32], u[32];  // both loads before the one wait
-                tmem_ld32(tmem + lane_base + kCColX + 32 * cg, x);
+                tmem_ld32(xo + lane_base + 32 * cg, x);
                 tmem_ld32(tmem + lane_base + kCColU + 32 * cg, u);
                 tmem_wait_ld();
 #pragma unroll
@@ -1491,11 +1490,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
             tc_fence_before();
             bar288();
             if (w) w = wait_bar(mbar_s, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
-            if (w && !last) w = rec_ready(i + 1);  // the next chunk's decay
+            if (w && !last) w = rec_ready(i + 1);  // the next chunk's operands and decay
             tc_fence_after();
             if (w) {
                 // ---- the new state: its fp16 copy over S0's (the first batch, S0's only reader, is
-                //      complete) and the next chunk's decay (or the state out) ----
+                //      complete) and the next chunk's decay, or the state out ----
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
                     const int c0 = 64 * cg + 32 * part;
