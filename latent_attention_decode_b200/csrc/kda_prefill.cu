@@ -710,6 +710,7 @@ constexpr int kPThreads = 512;      // 16 warps: the CUDA-core phases are latenc
 constexpr int kPWarps = kPThreads / 32;
 constexpr int kPStageTid = 32;  // issues the input staging (warp 0 issues the MMAs)
 constexpr int kPBulkTid = 64;   // issues the record's bulk stores, in four groups an item, and waits on them
+constexpr int kPFetchTid = 128; // takes items from the segment's counter
 // the record's four bulk groups of an item, in order: Qt, Kg and g_last (after the formation);
 // P (after the first extraction); Tb hi / lo (after the solve); W (last)
 constexpr uint32_t kPmBeta = 0, kPmRq = 256, kPmRk = 512, kPmOct = 768, kPmBar = 768 + kPWarps * 128 * 4,
@@ -1110,7 +1111,9 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
             if (tid == kPStageTid) stage_qka(nb, nh, nch);
             pending = 1;
         }
-        if (tid == 0) s_fetch[0] = atomicAdd(p.counter, 1);  // read after this item's last barrier
+        // the item after next, read after this item's last barrier; taken by a thread outside warp 0,
+        // which issues the MMAs below and would otherwise wait for the atomic's round trip first
+        if (tid == kPFetchTid) s_fetch[0] = atomicAdd(p.counter, 1);
         if (tid == kPBulkTid) {  // the record's Qt, Kg and g_last are final
             bulk_s2g(rec + kRWQ + 8192, sbase + kPQW + 8192, 8192);  // rows 64-127 of each block
             bulk_s2g(rec + kRWQ + 16384 + 8192, sbase + kPQW + 16384 + 8192, 8192);
