@@ -15,9 +15,10 @@
 //   S  = Diag(g_last) (S0 + Kh^T U)        (= Diag(g_last) S0 + (K * g_last/g)^T U)
 //
 // Two paths. With a workspace (the fast one), two kernels per segment of up to 128 chunks: the
-// prep kernel computes every chunk's state-independent operands in parallel (fp16 operands,
-// kind::f16) into a record per chunk, and the chain kernel runs only the state recurrence, one CTA
-// per (sequence, head) (see "Split path" below). Without one, a single kernel does both with tf32
+// prep kernel computes, for every chunk in parallel, the state-independent operands that need the
+// CUDA cores (fp16 operands, kind::f16) into a record per chunk, and the chain kernel runs the
+// chunk's tensor-core work around the state, one CTA per (sequence, head) (see "Split path"
+// below). Without one, a single kernel does both with tf32
 // operands; the d_v columns of S are independent, so there a CTA owns one (sequence, head, half
 // of d_v) and walks its chunks in order: 128 CTAs for one sequence of 64 heads.
 //
