@@ -1498,13 +1498,16 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
             tc_fence_after();
             if (w) {
                 // ---- the new state: its fp16 copy over S0's (the first batch, S0's only reader, is
-                //      complete) and the next chunk's decay, or the state out ----
+                //      complete) and the next chunk's decay, or the state out; both halves of the
+                //      thread's row are loaded before the one wait ----
+                float vv[2][32];
+                tmem_ld32(tmem + lane_base + kCColS + 64 * cg, vv[0]);
+                tmem_ld32(tmem + lane_base + kCColS + 64 * cg + 32, vv[1]);
+                tmem_wait_ld();
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
                     const int c0 = 64 * cg + 32 * part;
-                    float v[32];
-                    tmem_ld32(tmem + lane_base + kCColS + c0, v);
-                    tmem_wait_ld();
+                    float (&v)[32] = vv[part];
                     if (last) {
                         float *Sout = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
 #pragma unroll
