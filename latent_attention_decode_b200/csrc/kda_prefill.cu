@@ -1031,17 +1031,20 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
                     const int r = 4 * o + u;
                     a4[u] = (r < n) ? *reinterpret_cast<const float4 *>(sa + r * kDk + c4) : make_float4(1.f, 1.f, 1.f, 1.f);
                 }
-                float4 run = make_float4(1.f, 1.f, 1.f, 1.f);
+                // (packed pairs: two products an instruction, each rounded as a scalar one)
+                float2 r01 = make_float2(1.f, 1.f), r23 = r01;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    run = make_float4(run.x * a4[u].x, run.y * a4[u].y, run.z * a4[u].z, run.w * a4[u].w);
-                    fw[u] = run;  // prod over the quartet's tokens up to u
+                    r01 = mul2(r01, make_float2(a4[u].x, a4[u].y));
+                    r23 = mul2(r23, make_float2(a4[u].z, a4[u].w));
+                    fw[u] = make_float4(r01.x, r01.y, r23.x, r23.y);  // prod over the quartet's tokens up to u
                 }
-                run = make_float4(1.f, 1.f, 1.f, 1.f);
+                r01 = r23 = make_float2(1.f, 1.f);
 #pragma unroll
                 for (int u = 3; u >= 0; --u) {
-                    bw[u] = run;  // prod over the quartet's tokens after u
-                    run = make_float4(run.x * a4[u].x, run.y * a4[u].y, run.z * a4[u].z, run.w * a4[u].w);
+                    bw[u] = make_float4(r01.x, r01.y, r23.x, r23.y);  // prod over the quartet's tokens after u
+                    r01 = mul2(r01, make_float2(a4[u].x, a4[u].y));
+                    r23 = mul2(r23, make_float2(a4[u].z, a4[u].w));
                 }
             }
             *reinterpret_cast<float4 *>(s_oct + o * kDk + c4) = fw[3];
@@ -1065,43 +1068,42 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
             const float4 ex = *reinterpret_cast<const float4 *>(s_oct + o * kDk + c4);
             const float4 sx = *reinterpret_cast<const float4 *>(s_suf + o * kDk + c4);
             const float4 rg = *reinterpret_cast<const float4 *>(s_rg + c4);
+            const float2 ex01 = make_float2(ex.x, ex.y), ex23 = make_float2(ex.z, ex.w);
+            const float2 sx01 = make_float2(sx.x, sx.y), sx23 = make_float2(sx.z, sx.w);
+            const float2 rg01 = make_float2(rg.x, rg.y), rg23 = make_float2(rg.z, rg.w);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int r = 4 * o + u;
-                const float g[4] = {ex.x * fw[u].x, ex.y * fw[u].y, ex.z * fw[u].z, ex.w * fw[u].w};
-                const float R[4] = {sx.x * bw[u].x, sx.y * bw[u].y, sx.z * bw[u].z, sx.w * bw[u].w};
-                const float rgl[4] = {rg.x, rg.y, rg.z, rg.w};
+                const float2 g01 = mul2(ex01, make_float2(fw[u].x, fw[u].y));
+                const float2 g23 = mul2(ex23, make_float2(fw[u].z, fw[u].w));
+                const float2 R01 = mul2(sx01, make_float2(bw[u].x, bw[u].y));
+                const float2 R23 = mul2(sx23, make_float2(bw[u].z, bw[u].w));
                 const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + c4);
                 const uint2 kw = *reinterpret_cast<const uint2 *>(sk + r * kDk + c4);
-                const float2 q0 = lad::dev::bf16x2_to_f32(qw.x), q1 = lad::dev::bf16x2_to_f32(qw.y);
-                const float2 k0 = lad::dev::bf16x2_to_f32(kw.x), k1 = lad::dev::bf16x2_to_f32(kw.y);
-                float qv[4] = {q0.x, q0.y, q1.x, q1.y};
-                float kv[4] = {k0.x, k0.y, k1.x, k1.y};
+                float2 q01 = lad::dev::bf16x2_to_f32(qw.x), q23 = lad::dev::bf16x2_to_f32(qw.y);
+                float2 k01 = lad::dev::bf16x2_to_f32(kw.x), k23 = lad::dev::bf16x2_to_f32(kw.y);
                 if constexpr (kL2) {
                     const float rq = s_rq[r], rk = s_rk[r];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        qv[e] *= rq;
-                        kv[e] *= rk;
-                    }
+                    q01 = mul2(q01, make_float2(rq, rq));
+                    q23 = mul2(q23, make_float2(rq, rq));
+                    k01 = mul2(k01, make_float2(rk, rk));
+                    k23 = mul2(k23, make_float2(rk, rk));
                 }
-                float kh[4], kg[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    kg[e] = kv[e] * R[e];
-                    kh[e] = kg[e] * rgl[e];
-                }
+                const float2 kg01 = mul2(k01, R01), kg23 = mul2(k23, R23);
+                const float2 kh01 = mul2(kg01, rg01), kh23 = mul2(kg23, rg23);
+                const float2 kt01 = mul2(k01, g01), kt23 = mul2(k23, g23);
+                const float2 qt01 = mul2(q01, g01), qt23 = mul2(q23, g23);
                 const uint32_t off = sw128_off16(r, c4, 8192);                 // 64-row tiles (Kh, Kg)
                 const uint32_t offq = sw128_off16(kC + r, c4, 16384);          // row 64 + r of [Kt; Qt]
                 const uint32_t offk = sw128_off16(r, c4, 16384);               // row r of [Kt; Qt]
                 *reinterpret_cast<uint2 *>(sm + kPQW + offk) =
-                    make_uint2(f32x2_to_f16x2(kv[0] * g[0], kv[1] * g[1]), f32x2_to_f16x2(kv[2] * g[2], kv[3] * g[3]));
+                    make_uint2(f32x2_to_f16x2(kt01.x, kt01.y), f32x2_to_f16x2(kt23.x, kt23.y));
                 *reinterpret_cast<uint2 *>(sm + kPQW + offq) =
-                    make_uint2(f32x2_to_f16x2(qv[0] * g[0], qv[1] * g[1]), f32x2_to_f16x2(qv[2] * g[2], qv[3] * g[3]));
+                    make_uint2(f32x2_to_f16x2(qt01.x, qt01.y), f32x2_to_f16x2(qt23.x, qt23.y));
                 *reinterpret_cast<uint2 *>(sm + kPKH + off) =
-                    make_uint2(f32x2_to_f16x2(kh[0], kh[1]), f32x2_to_f16x2(kh[2], kh[3]));
+                    make_uint2(f32x2_to_f16x2(kh01.x, kh01.y), f32x2_to_f16x2(kh23.x, kh23.y));
                 *reinterpret_cast<uint2 *>(sm + kPKG + off) =
-                    make_uint2(f32x2_to_f16x2(kg[0], kg[1]), f32x2_to_f16x2(kg[2], kg[3]));
+                    make_uint2(f32x2_to_f16x2(kg01.x, kg01.y), f32x2_to_f16x2(kg23.x, kg23.y));
             }
         }
         // ---- [Kt; Qt] Kh^T: rows 0-63 give Kt Kh^T, rows 64-127 Qt Kh^T ----
@@ -1484,11 +1486,17 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; j += 8)
+                {
+                    uint32_t h[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 d = sub2(make_float2(u[j + 2 * e], u[j + 2 * e + 1]),
+                                              make_float2(x[j + 2 * e], x[j + 2 * e + 1]));
+                        h[e] = f32x2_to_f16x2(d.x, d.y);
+                    }
                     *reinterpret_cast<uint4 *>(sm + rs + kCV + sw128_off16(dv, 32 * cg + j, 16384)) =
-                        make_uint4(f32x2_to_f16x2(u[j] - x[j], u[j + 1] - x[j + 1]),
-                                   f32x2_to_f16x2(u[j + 2] - x[j + 2], u[j + 3] - x[j + 3]),
-                                   f32x2_to_f16x2(u[j + 4] - x[j + 4], u[j + 5] - x[j + 5]),
-                                   f32x2_to_f16x2(u[j + 6] - x[j + 6], u[j + 7] - x[j + 7]));
+                        make_uint4(h[0], h[1], h[2], h[3]);
+                }
             }
             fence_async_smem();
             tc_fence_before();
@@ -1522,10 +1530,12 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             const float4 g4 = gn[j];
-                            v[4 * j] *= g4.x;
-                            v[4 * j + 1] *= g4.y;
-                            v[4 * j + 2] *= g4.z;
-                            v[4 * j + 3] *= g4.w;
+                            const float2 a = mul2(make_float2(v[4 * j], v[4 * j + 1]), make_float2(g4.x, g4.y));
+                            const float2 c = mul2(make_float2(v[4 * j + 2], v[4 * j + 3]), make_float2(g4.z, g4.w));
+                            v[4 * j] = a.x;
+                            v[4 * j + 1] = a.y;
+                            v[4 * j + 2] = c.x;
+                            v[4 * j + 3] = c.y;
                         }
                         tmem_st32(tmem + lane_base + kCColS + c0, v);
                     }
