@@ -756,18 +756,21 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             const float4 *arow = reinterpret_cast<const float4 *>(sA + (i0 + r) * kAS + i0);
-            float acc0 = 0.f, acc1 = 0.f;
+            float2 acc = make_float2(0.f, 0.f);  // the two partial sums, as one packed pair
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
-                if (4 * q4 < r) {
+                if (4 * q4 + 3 < r) {
                     const float4 a = arow[q4];
-                    acc0 = fmaf(a.x, t[4 * q4], acc0);
-                    if (4 * q4 + 1 < r) acc1 = fmaf(a.y, t[4 * q4 + 1], acc1);
-                    if (4 * q4 + 2 < r) acc0 = fmaf(a.z, t[4 * q4 + 2], acc0);
-                    if (4 * q4 + 3 < r) acc1 = fmaf(a.w, t[4 * q4 + 3], acc1);
+                    acc = fma2(make_float2(a.x, a.y), make_float2(t[4 * q4], t[4 * q4 + 1]), acc);
+                    acc = fma2(make_float2(a.z, a.w), make_float2(t[4 * q4 + 2], t[4 * q4 + 3]), acc);
+                } else if (4 * q4 < r) {
+                    const float4 a = arow[q4];
+                    acc.x = fmaf(a.x, t[4 * q4], acc.x);
+                    if (4 * q4 + 1 < r) acc.y = fmaf(a.y, t[4 * q4 + 1], acc.y);
+                    if (4 * q4 + 2 < r) acc.x = fmaf(a.z, t[4 * q4 + 2], acc.x);
                 }
             }
-            t[r] = r < c ? 0.f : (r == c ? 1.f : -(acc0 + acc1));
+            t[r] = r < c ? 0.f : (r == c ? 1.f : -(acc.x + acc.y));
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) sT[(i0 + r) * kAS + i0 + c] = t[r];  // zeros above the diagonal too
@@ -776,32 +779,29 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
     // (1a) Y_p = A_{2p+1,2p} T_{2p,2p} into A at rows 32p .. 32p+15, columns 32p+16 .. 32p+31
     const int q0 = 32 * (warp >> 1), rr = 8 * (warp & 1) + (lane >> 2), cc = 4 * (lane & 3);
     if (warp < 4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float2 acc01 = make_float2(0.f, 0.f), acc23 = acc01;
 #pragma unroll
         for (int s2 = 0; s2 < 16; ++s2) {
             const float a = sA[(q0 + 16 + rr) * kAS + q0 + s2];
             const float4 t = *reinterpret_cast<const float4 *>(sT + (q0 + s2) * kAS + q0 + cc);
-            acc.x = fmaf(a, t.x, acc.x);
-            acc.y = fmaf(a, t.y, acc.y);
-            acc.z = fmaf(a, t.z, acc.z);
-            acc.w = fmaf(a, t.w, acc.w);
+            acc01 = fma2(make_float2(a, a), make_float2(t.x, t.y), acc01);
+            acc23 = fma2(make_float2(a, a), make_float2(t.z, t.w), acc23);
         }
-        *reinterpret_cast<float4 *>(sA + (q0 + rr) * kAS + q0 + 16 + cc) = acc;
+        *reinterpret_cast<float4 *>(sA + (q0 + rr) * kAS + q0 + 16 + cc) = make_float4(acc01.x, acc01.y, acc23.x, acc23.y);
     }
     __syncthreads();
     // (1b) T_{2p+1,2p} = -T_{2p+1,2p+1} Y_p; T_{2p,2p+1} = 0
     if (warp < 4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float2 acc01 = make_float2(0.f, 0.f), acc23 = acc01;
 #pragma unroll
         for (int s2 = 0; s2 < 16; ++s2) {
             const float t = sT[(q0 + 16 + rr) * kAS + q0 + 16 + s2];
             const float4 y = *reinterpret_cast<const float4 *>(sA + (q0 + s2) * kAS + q0 + 16 + cc);
-            acc.x = fmaf(t, y.x, acc.x);
-            acc.y = fmaf(t, y.y, acc.y);
-            acc.z = fmaf(t, y.z, acc.z);
-            acc.w = fmaf(t, y.w, acc.w);
+            acc01 = fma2(make_float2(t, t), make_float2(y.x, y.y), acc01);
+            acc23 = fma2(make_float2(t, t), make_float2(y.z, y.w), acc23);
         }
-        *reinterpret_cast<float4 *>(sT + (q0 + 16 + rr) * kAS + q0 + cc) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        *reinterpret_cast<float4 *>(sT + (q0 + 16 + rr) * kAS + q0 + cc) =
+            make_float4(-acc01.x, -acc01.y, -acc23.x, -acc23.y);
         *reinterpret_cast<float4 *>(sT + (q0 + rr) * kAS + q0 + 16 + cc) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
@@ -810,22 +810,19 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
     // (2a) R = A_{hi,lo} T_lo into A at rows 0 .. 31, columns 32 .. 63. Warps 4-15: Tb rows 0-31
     //      (T_lo times beta; zero right of column 31)
     if (warp < 4) {
-        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+        float2 a00 = make_float2(0.f, 0.f), a01 = a00, a10 = a00, a11 = a00;  // row, column pair
 #pragma unroll 8
         for (int s = 0; s < 32; ++s) {
-            const float a0 = sA[(32 + r2) * kAS + s], a1 = sA[(33 + r2) * kAS + s];
+            const float x0 = sA[(32 + r2) * kAS + s], x1 = sA[(33 + r2) * kAS + s];
             const float4 t = *reinterpret_cast<const float4 *>(sT + s * kAS + c2);
-            acc0.x = fmaf(a0, t.x, acc0.x);
-            acc0.y = fmaf(a0, t.y, acc0.y);
-            acc0.z = fmaf(a0, t.z, acc0.z);
-            acc0.w = fmaf(a0, t.w, acc0.w);
-            acc1.x = fmaf(a1, t.x, acc1.x);
-            acc1.y = fmaf(a1, t.y, acc1.y);
-            acc1.z = fmaf(a1, t.z, acc1.z);
-            acc1.w = fmaf(a1, t.w, acc1.w);
+            const float2 tlo = make_float2(t.x, t.y), thi = make_float2(t.z, t.w);
+            a00 = fma2(make_float2(x0, x0), tlo, a00);
+            a01 = fma2(make_float2(x0, x0), thi, a01);
+            a10 = fma2(make_float2(x1, x1), tlo, a10);
+            a11 = fma2(make_float2(x1, x1), thi, a11);
         }
-        *reinterpret_cast<float4 *>(sA + r2 * kAS + 32 + c2) = acc0;
-        *reinterpret_cast<float4 *>(sA + (r2 + 1) * kAS + 32 + c2) = acc1;
+        *reinterpret_cast<float4 *>(sA + r2 * kAS + 32 + c2) = make_float4(a00.x, a00.y, a01.x, a01.y);
+        *reinterpret_cast<float4 *>(sA + (r2 + 1) * kAS + 32 + c2) = make_float4(a10.x, a10.y, a11.x, a11.y);
     } else {
         for (int e = tid - 128; e < 32 * 16; e += kPThreads - 128) {
             const int r = e >> 4, c = (e & 15) * 4;
@@ -839,20 +836,18 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
     // (2b) T[32 + r][0 .. 31] = -T_hi R, times beta, straight into Tb (T_hi is lower triangular: a
     //      warp's rows end at 8 warp + 7). Warps 4-15: Tb rows 32-63, columns 32-63 (T_hi times beta)
     if (warp < 4) {
-        float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+        float2 a00 = make_float2(0.f, 0.f), a01 = a00, a10 = a00, a11 = a00;  // row, column pair
 #pragma unroll 8
         for (int s = 0; s < 8 * warp + 8; ++s) {
             const float t0 = sT[(32 + r2) * kAS + 32 + s], t1 = sT[(33 + r2) * kAS + 32 + s];
             const float4 y = *reinterpret_cast<const float4 *>(sA + s * kAS + 32 + c2);
-            acc0.x = fmaf(t0, y.x, acc0.x);
-            acc0.y = fmaf(t0, y.y, acc0.y);
-            acc0.z = fmaf(t0, y.z, acc0.z);
-            acc0.w = fmaf(t0, y.w, acc0.w);
-            acc1.x = fmaf(t1, y.x, acc1.x);
-            acc1.y = fmaf(t1, y.y, acc1.y);
-            acc1.z = fmaf(t1, y.z, acc1.z);
-            acc1.w = fmaf(t1, y.w, acc1.w);
+            const float2 ylo = make_float2(y.x, y.y), yhi = make_float2(y.z, y.w);
+            a00 = fma2(make_float2(t0, t0), ylo, a00);
+            a01 = fma2(make_float2(t0, t0), yhi, a01);
+            a10 = fma2(make_float2(t1, t1), ylo, a10);
+            a11 = fma2(make_float2(t1, t1), yhi, a11);
         }
+        const float4 acc0 = make_float4(a00.x, a00.y, a01.x, a01.y), acc1 = make_float4(a10.x, a10.y, a11.x, a11.y);
         const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + c2);
         put_tb4(tb16, tbh, tbl, 32 + r2, c2, -acc0.x * b4.x, -acc0.y * b4.y, -acc0.z * b4.z, -acc0.w * b4.w);
         put_tb4(tb16, tbh, tbl, 33 + r2, c2, -acc1.x * b4.x, -acc1.y * b4.y, -acc1.z * b4.z, -acc1.w * b4.w);
