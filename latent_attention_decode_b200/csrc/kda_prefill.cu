@@ -723,14 +723,19 @@ constexpr uint32_t kPStageTx = 16384 + 16384 + 32768;  // q, k, alpha
 constexpr uint32_t kPColA = 0, kPColW = 64, kPTmemCols = 256;
 
 // element (r, s) of the three Tb tiles, four consecutive s at once (s % 4 == 0)
-__device__ __forceinline__ void put_tb4(uint8_t *tb16, uint8_t *tbh, uint8_t *tbl, int r, int s, float a, float b,
-                                        float c, float d) {
+__device__ __forceinline__ void put_tb4(uint8_t *tb16, uint8_t *tbh, uint8_t *tbl, int r, int s, float2 ab, float2 cd) {
     const uint32_t off = sw128_off16(r, s, 8192);
-    *reinterpret_cast<uint2 *>(tb16 + off) = make_uint2(f32x2_to_f16x2(a, b), f32x2_to_f16x2(c, d));
-    const uint32_t h0 = bf16x2_rn(a, b), h1 = bf16x2_rn(c, d);
+    *reinterpret_cast<uint2 *>(tb16 + off) = make_uint2(f32x2_to_f16x2(ab.x, ab.y), f32x2_to_f16x2(cd.x, cd.y));
+    const uint32_t h0 = bf16x2_rn(ab.x, ab.y), h1 = bf16x2_rn(cd.x, cd.y);
     *reinterpret_cast<uint2 *>(tbh + off) = make_uint2(h0, h1);
-    const float2 fa = lad::dev::bf16x2_to_f32(h0), fc = lad::dev::bf16x2_to_f32(h1);
-    *reinterpret_cast<uint2 *>(tbl + off) = make_uint2(bf16x2_rn(a - fa.x, b - fa.y), bf16x2_rn(c - fc.x, d - fc.y));
+    const float2 la = sub2(ab, lad::dev::bf16x2_to_f32(h0)), lc = sub2(cd, lad::dev::bf16x2_to_f32(h1));
+    *reinterpret_cast<uint2 *>(tbl + off) = make_uint2(bf16x2_rn(la.x, la.y), bf16x2_rn(lc.x, lc.y));
+}
+// T times beta, four columns: the element products of put_tb4's arguments
+__device__ __forceinline__ void put_tb4_scaled(uint8_t *tb16, uint8_t *tbh, uint8_t *tbl, int r, int s, float4 t,
+                                               float4 b) {
+    put_tb4(tb16, tbh, tbl, r, s, mul2(make_float2(t.x, t.y), make_float2(b.x, b.y)),
+            mul2(make_float2(t.z, t.w), make_float2(b.z, b.w)));
 }
 
 
@@ -829,7 +834,7 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
             float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
             if (c < 32) t4 = *reinterpret_cast<const float4 *>(sT + r * kAS + c);
             const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + c);
-            put_tb4(tb16, tbh, tbl, r, c, t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
+            put_tb4_scaled(tb16, tbh, tbl, r, c, t4, b4);
         }
     }
     __syncthreads();
@@ -849,14 +854,14 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
         }
         const float4 acc0 = make_float4(a00.x, a00.y, a01.x, a01.y), acc1 = make_float4(a10.x, a10.y, a11.x, a11.y);
         const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + c2);
-        put_tb4(tb16, tbh, tbl, 32 + r2, c2, -acc0.x * b4.x, -acc0.y * b4.y, -acc0.z * b4.z, -acc0.w * b4.w);
-        put_tb4(tb16, tbh, tbl, 33 + r2, c2, -acc1.x * b4.x, -acc1.y * b4.y, -acc1.z * b4.z, -acc1.w * b4.w);
+        put_tb4_scaled(tb16, tbh, tbl, 32 + r2, c2, make_float4(-acc0.x, -acc0.y, -acc0.z, -acc0.w), b4);
+        put_tb4_scaled(tb16, tbh, tbl, 33 + r2, c2, make_float4(-acc1.x, -acc1.y, -acc1.z, -acc1.w), b4);
     } else {
         for (int e = tid - 128; e < 32 * 8; e += kPThreads - 128) {
             const int r = 32 + (e >> 3), c = 32 + (e & 7) * 4;
             const float4 t4 = *reinterpret_cast<const float4 *>(sT + r * kAS + c);
             const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + c);
-            put_tb4(tb16, tbh, tbl, r, c, t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
+            put_tb4_scaled(tb16, tbh, tbl, r, c, t4, b4);
         }
     }
 }
@@ -1142,9 +1147,12 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
                 const float br = s_beta[r];
                 float4 *dst = reinterpret_cast<float4 *>(sA + r * kAS + c0);
 #pragma unroll
-                for (int j = 0; j < 16; j += 4)
-                    dst[j / 4] = make_float4(c0 + j < r ? br * x[j] : 0.f, c0 + j + 1 < r ? br * x[j + 1] : 0.f,
-                                             c0 + j + 2 < r ? br * x[j + 2] : 0.f, c0 + j + 3 < r ? br * x[j + 3] : 0.f);
+                for (int j = 0; j < 16; j += 4) {
+                    const float2 p01 = mul2(make_float2(br, br), make_float2(x[j], x[j + 1]));
+                    const float2 p23 = mul2(make_float2(br, br), make_float2(x[j + 2], x[j + 3]));
+                    dst[j / 4] = make_float4(c0 + j < r ? p01.x : 0.f, c0 + j + 1 < r ? p01.y : 0.f,
+                                             c0 + j + 2 < r ? p23.x : 0.f, c0 + j + 3 < r ? p23.y : 0.f);
+                }
             } else {
                 const int r = row - kC;
 #pragma unroll
@@ -1362,9 +1370,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
             uint32_t *od = reinterpret_cast<uint32_t *>(sm + kCO) + ((32 * cg + odd) * kDv + dv - odd) / 2;
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-                const float mine0 = p.scale * x[j], mine1 = p.scale * x[j + 1];
-                const float other = __shfl_xor_sync(0xffffffffu, odd ? mine0 : mine1, 1);
-                od[j * (kDv / 2)] = odd ? bf16x2_rn(other, mine1) : bf16x2_rn(mine0, other);
+                const float2 mine = mul2(make_float2(p.scale, p.scale), make_float2(x[j], x[j + 1]));
+                const float other = __shfl_xor_sync(0xffffffffu, odd ? mine.x : mine.y, 1);
+                od[j * (kDv / 2)] = odd ? bf16x2_rn(other, mine.y) : bf16x2_rn(mine.x, other);
             }
             fence_async_smem();
             bar256();
