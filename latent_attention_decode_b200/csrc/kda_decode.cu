@@ -44,6 +44,13 @@ __device__ __forceinline__ void fma4(float4 &acc, float a, const float4 &x) {
     acc.w = fmaf(a, x.w, acc.w);
 }
 
+// fma4 as two packed fp32 pair instructions (each lane rounded as the scalar FMA): the same bits
+__device__ __forceinline__ void fma4p(float4 &acc, float a, const float4 &x) {
+    const float2 lo = lad::ptx::fma2(make_float2(a, a), make_float2(x.x, x.y), make_float2(acc.x, acc.y));
+    const float2 hi = lad::ptx::fma2(make_float2(a, a), make_float2(x.z, x.w), make_float2(acc.z, acc.w));
+    acc = make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
 __device__ __forceinline__ void add4(float4 &acc, const float4 &x) {
     acc.x += x.x;
     acc.y += x.y;
@@ -540,8 +547,8 @@ kda_decode_multi_kernel(const uint16_t *__restrict__ q, const uint16_t *__restri
                     for (int mm = 0; mm < kRowsPerWarp / 2; ++mm) {
                         const int m = half * (kRowsPerWarp / 2) + mm;
                         const float4 f = rf[8 * m];
-                        fma4(wk, f.x, s[m]);
-                        fma4(wq, f.y, s[m]);
+                        fma4p(wk, f.x, s[m]);
+                        fma4p(wq, f.y, s[m]);
                     }
                     asm volatile("" ::: "memory");
                 }
@@ -565,7 +572,7 @@ kda_decode_multi_kernel(const uint16_t *__restrict__ q, const uint16_t *__restri
                 u.z = bt * (v1.x - wk.z);
                 u.w = bt * (v1.y - wk.w);
 #pragma unroll
-                for (int m = 0; m < kRowsPerWarp; ++m) fma4(s[m], rowk[t * kD + 8 * m + rsub], u);
+                for (int m = 0; m < kRowsPerWarp; ++m) fma4p(s[m], rowk[t * kD + 8 * m + rsub], u);
                 if (o && rsub == 0) {
                     const float qk = s_qk[t];
                     float4 ov;
