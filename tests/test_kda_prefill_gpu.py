@@ -109,6 +109,25 @@ def test_prefill_several_segments(lad, cuda_device):
     assert rel_l2(o, o1) < TOL_OUT and rel_l2(S, S1) < TOL_PREFILL_STATE
 
 
+def test_prefill_several_segments_batched(lad, cuda_device):
+    """Three sequences through two segments (140 chunks: 108, then the 32-chunk tail, the last
+    chunk ragged): each sequence's v tiles, records and states are its own. Every (sequence,
+    head) against the oracle, and the bf16 outputs against the fp32 ones rounded."""
+    cfg = wl.KdaScan("p", B=3, H=2, T=128 * 64 + 12 * 64 - 28, seed=17, state_std=0.02, alpha_mode="uniform")
+    inp = wl.kda_scan_inputs(cfg)
+    o_ref, S_ref = _oracle(inp)
+    o, S = _run(lad, inp, cuda_device)
+    # o is [B, T, H, d]: one norm per (sequence, head) over its tokens
+    o_h, o_ref_h = o.permute(0, 2, 1, 3), np.transpose(o_ref, (0, 2, 1, 3))
+    print(f"prefill batched segments: o {rel_l2(o, o_ref):.2e} (worst head {max_rel_l2(o_h, o_ref_h, 2):.2e}) "
+          f"S {rel_l2(S, S_ref):.2e} (worst head {max_rel_l2(S, S_ref, 2):.2e})")
+    assert rel_l2(o, o_ref) < TOL_OUT and max_rel_l2(o_h, o_ref_h, 2) < TOL_OUT
+    assert rel_l2(S, S_ref) < TOL_PREFILL_STATE and max_rel_l2(S, S_ref, 2) < TOL_PREFILL_STATE
+    o16, S16 = _run(lad, inp, cuda_device, out_fp32=False)
+    assert torch.equal(S16, S)
+    assert torch.equal(o16.float(), o.to(torch.bfloat16).float())
+
+
 def test_prefill_in_a_cuda_graph(lad, cuda_device):
     """The two-kernel path forks onto the library's side stream and joins back by events, which a
     stream capture follows: a graph of the call (three segments: 128, 8 and the 32-chunk tail, so
