@@ -645,6 +645,9 @@ constexpr uint32_t kRTH = 57344;       // Tb, bf16 high part [64 r][64 s], K-maj
 constexpr uint32_t kRTL = 65536;       // Tb, bf16 low part (Tb - hi): 8 KiB
 constexpr uint32_t kRG = 73728;        // g_last [128] fp32
 constexpr uint32_t kRecBytes = 74240;  // 580 lines of 128 bytes
+#ifndef LAD_PREFILL_PREP_WS
+#define LAD_PREFILL_PREP_WS 1  // the warp-specialised prep (kda_chunk_prep_ws_kernel)
+#endif
 #ifndef LAD_PREFILL_SEG_CHUNKS
 #define LAD_PREFILL_SEG_CHUNKS 128
 #endif
@@ -747,11 +750,14 @@ __device__ __forceinline__ void put_tb4_scaled(uint8_t *tb16, uint8_t *tbh, uint
 //   (2) the lower-left 32x32 block, -T_hi A_{hi,lo} T_lo.
 // The products A T of (1) and (2) are parked in A's upper triangle, which holds no data; the blocks
 // of T above its diagonal blocks are zeroed in (1), so that (2) runs over whole 32x32 blocks. Steps
-// (1) and (2) run on warps 0-3 (a row, or a row pair, and four columns a thread); in (2) warps 4-15
-// write the rows of Tb that are final already. Called by all kPThreads threads; contains block-wide
-// barriers.
-__device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_beta, uint8_t *tb16, uint8_t *tbh,
-                                          uint8_t *tbl, int tid) {
+// (1) and (2) run on the group's warps 0-3 (a row, or a row pair, and four columns a thread); in (2)
+// its other warps write the rows of Tb that are final already. Called by all kTh threads of a group
+// (tid: the thread's index in it), with `sync` that group's barrier. tbh / tbl may point to global
+// memory (the record) rather than shared memory: the stores are generic.
+template <int kTh, typename Sync>
+__device__ __forceinline__ void solve_tb(float *sA, float *sT, const float *s_beta, uint8_t *tb16, uint8_t *tbh,
+                                         uint8_t *tbl, int tid, Sync sync) {
+    static_assert(kTh > 128 && kTh % 32 == 0, "the solve needs warps beyond the first four");
     const int warp = tid >> 5, lane = tid & 31;
     if (tid < kC) {
         // column c of (I + A_ii)^-1: t_r = [r == c] - sum_{s < r} A_rs t_s (t_s = 0 for s < c); a
@@ -780,7 +786,7 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
 #pragma unroll
         for (int r = 0; r < 16; ++r) sT[(i0 + r) * kAS + i0 + c] = t[r];  // zeros above the diagonal too
     }
-    __syncthreads();
+    sync();
     // (1a) Y_p = A_{2p+1,2p} T_{2p,2p} into A at rows 32p .. 32p+15, columns 32p+16 .. 32p+31
     const int q0 = 32 * (warp >> 1), rr = 8 * (warp & 1) + (lane >> 2), cc = 4 * (lane & 3);
     if (warp < 4) {
@@ -794,7 +800,7 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
         }
         *reinterpret_cast<float4 *>(sA + (q0 + rr) * kAS + q0 + 16 + cc) = make_float4(acc01.x, acc01.y, acc23.x, acc23.y);
     }
-    __syncthreads();
+    sync();
     // (1b) T_{2p+1,2p} = -T_{2p+1,2p+1} Y_p; T_{2p,2p+1} = 0
     if (warp < 4) {
         float2 acc01 = make_float2(0.f, 0.f), acc23 = acc01;
@@ -809,7 +815,7 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
             make_float4(-acc01.x, -acc01.y, -acc23.x, -acc23.y);
         *reinterpret_cast<float4 *>(sT + (q0 + rr) * kAS + q0 + 16 + cc) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    __syncthreads();
+    sync();
     // thread (warps 0-3) of steps (2a) / (2b): rows r2, r2 + 1 of a 32-row block, columns c2 .. c2 + 3
     const int r2 = 2 * (tid >> 3), c2 = 4 * (tid & 7);
     // (2a) R = A_{hi,lo} T_lo into A at rows 0 .. 31, columns 32 .. 63. Warps 4-15: Tb rows 0-31
@@ -829,7 +835,7 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
         *reinterpret_cast<float4 *>(sA + r2 * kAS + 32 + c2) = make_float4(a00.x, a00.y, a01.x, a01.y);
         *reinterpret_cast<float4 *>(sA + (r2 + 1) * kAS + 32 + c2) = make_float4(a10.x, a10.y, a11.x, a11.y);
     } else {
-        for (int e = tid - 128; e < 32 * 16; e += kPThreads - 128) {
+        for (int e = tid - 128; e < 32 * 16; e += kTh - 128) {
             const int r = e >> 4, c = (e & 15) * 4;
             float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
             if (c < 32) t4 = *reinterpret_cast<const float4 *>(sT + r * kAS + c);
@@ -837,7 +843,7 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
             put_tb4_scaled(tb16, tbh, tbl, r, c, t4, b4);
         }
     }
-    __syncthreads();
+    sync();
     // (2b) T[32 + r][0 .. 31] = -T_hi R, times beta, straight into Tb (T_hi is lower triangular: a
     //      warp's rows end at 8 warp + 7). Warps 4-15: Tb rows 32-63, columns 32-63 (T_hi times beta)
     if (warp < 4) {
@@ -857,7 +863,7 @@ __device__ __forceinline__ void solve_tb16(float *sA, float *sT, const float *s_
         put_tb4_scaled(tb16, tbh, tbl, 32 + r2, c2, make_float4(-acc0.x, -acc0.y, -acc0.z, -acc0.w), b4);
         put_tb4_scaled(tb16, tbh, tbl, 33 + r2, c2, make_float4(-acc1.x, -acc1.y, -acc1.z, -acc1.w), b4);
     } else {
-        for (int e = tid - 128; e < 32 * 8; e += kPThreads - 128) {
+        for (int e = tid - 128; e < 32 * 8; e += kTh - 128) {
             const int r = 32 + (e >> 3), c = 32 + (e & 7) * 4;
             const float4 t4 = *reinterpret_cast<const float4 *>(sT + r * kAS + c);
             const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + c);
@@ -1174,7 +1180,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
             bulk_commit();
         }
         // ---- T = (I + A)^-1, Tb = T diag(beta) -> the fp16 tile and its bf16 hi / lo split ----
-        solve_tb16(sA, sT, s_beta, sm + kPTB, sm + kPTBH, sm + kPTBL, tid);
+        solve_tb<kPThreads>(sA, sT, s_beta, sm + kPTB, sm + kPTBH, sm + kPTBL, tid, []() { __syncthreads(); });
         // ---- W = Tb Kt (Kt: rows 0-63 of [Kt; Qt], read MN-major) ----
         fence_async_smem();
         tc_fence_before();
@@ -1239,6 +1245,469 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p
     __syncthreads();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, kPTmemCols);
+}
+
+// ------------------------------------------------------------------------------------------
+// The prep, warp-specialised (what the split path runs). Half the CTA forms an item's operands
+// while the other half finishes the item before it, so the solve's long serial chain (run by four
+// warps, the others waiting at its barriers) overlaps the next item's formation:
+//   warps 0-7, the former: staging wait, decays and operand tiles ([Kt; Qt] into one of two
+//     buffers, Kh, Kg), [Kt; Qt] Kh^T on the tensor cores, A (into one of two scratch buffers) and P;
+//   warps 8-15, the solver: (I + A)^-1 and the Tb tiles, W = Tb Kt on the tensor cores, W out.
+// An item passes from the former to the solver through buffer j % 2 (the [Kt; Qt] tile and the A
+// scratch) with two mbarriers per buffer: full (the former's item is in it) and empty (the solver is
+// done with it: its W MMA has read Kt, and the solve has read A). Each half synchronises on its own
+// named barrier. The record leaves as the former writes it (Kg, g_last, P: stores from registers;
+// Qt: one bulk store from the tile) and as the solver finishes it (Tb hi / lo, W: stores from
+// registers), so neither half waits on the other's stores. Every wait is bounded; the former ends
+// the solver's loop with an item of -1.
+// ------------------------------------------------------------------------------------------
+constexpr uint32_t kWQW = 0;                          // [Kt; Qt] x 2, 32 KiB each (the record's Qt)
+constexpr uint32_t kWKH = 65536;                      // Kh [64 tok][128 d_k], 2 blocks x 8 KiB
+constexpr uint32_t kWSuf = 81920;                     // the decay scan's backward products [16][128] fp32
+constexpr uint32_t kWSQ = 90112, kWSK = 106496, kWSA = 122880;  // q, k, alpha staging (TMA, plain)
+constexpr uint32_t kWAStride = 64 * kAS * 4;          // one A / T scratch [64][kAS] fp32
+constexpr uint32_t kWA = 155648;                      // A scratch x 2
+constexpr uint32_t kWT = kWA + 2 * kWAStride;         // T scratch (the solver's)
+constexpr uint32_t kWTB = kWT + kWAStride;            // Tb [64 r][64 s] fp16 K-major (the W MMA's A)
+constexpr uint32_t kWMisc = kWTB + 8192;
+constexpr uint32_t kWmBeta = 0, kWmBetaS = 256, kWmRq = 768, kWmRk = 1024, kWmRg = 1280, kWmOct = 1792,
+                   kWmBar = kWmOct + 16 * 128 * 4, kWmTmem = kWmBar + 64, kWmAbort = kWmTmem + 4,
+                   kWmFetch = kWmTmem + 8, kWmItem = kWmTmem + 16, kWmEnd = kWmTmem + 32;
+constexpr uint32_t kWSmemBytes = kWMisc + kWmEnd + 1024;
+static_assert(kWSmemBytes <= 232448, "prep shared memory over the per-block limit");
+static_assert(kWTB % 1024 == 0 && kWQW % 1024 == 0 && kWKH % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+constexpr int kWHalf = 256;                           // threads of each half
+constexpr int kWFetchTid = 128, kWStageTid = 32, kWBulkTid = 64;  // former threads with a side job
+// TMEM columns: [Kt; Qt] Kh^T (the former's), W (the solver's)
+constexpr uint32_t kWColA = 0, kWColW = 64, kWTmemCols = 256;
+
+__device__ __forceinline__ void half_bar(int id) { asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory"); }
+// the AND of `v` over a half's 256 threads, at its named barrier
+__device__ __forceinline__ bool half_and(int id, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v)), "r"(id)
+        : "memory");
+    return r != 0;
+}
+
+template <bool kL2>  // kL2: q and k are L2-normalised per token (p.l2norm)
+__global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArgs p,
+                                                                         const __grid_constant__ PrepMaps maps) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint8_t *misc = sm + kWMisc;
+    const uint32_t stage_bar = sbase + kWMisc + kWmBar, mmaf_bar = stage_bar + 8, mmas_bar = stage_bar + 16;
+    const uint32_t full_bar = stage_bar + 24, empty_bar = stage_bar + 40;  // two each, 8 bytes apart
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + kWmTmem);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + kWmAbort);
+    int *s_fetch = reinterpret_cast<int *>(misc + kWmFetch);
+    volatile int *s_item = reinterpret_cast<volatile int *>(misc + kWmItem);  // per buffer: the item, or -1
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int sp = warp & 3;  // TMEM sub-partition
+    const uint32_t lane_base = static_cast<uint32_t>(32 * sp) << 16;
+    const int nitems = p.B * p.H * p.nseg;
+    const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);
+
+    if (tid == 0) {
+        mbar_init(stage_bar, 1);
+        mbar_init(mmaf_bar, 1);
+        mbar_init(mmas_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(full_bar + 8 * b, 1);
+            mbar_init(empty_bar + 8 * b, 1);
+        }
+        *abort_flag = 0;
+        s_fetch[0] = atomicAdd(p.counter, 1);  // the first item, and the one after it
+        s_fetch[1] = atomicAdd(p.counter, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kWTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < 8) {
+        // ============================== the former ==============================
+        const int ft = tid;  // 0-255
+        float *s_beta = reinterpret_cast<float *>(misc + kWmBeta);
+        float *s_rq = reinterpret_cast<float *>(misc + kWmRq);
+        float *s_rk = reinterpret_cast<float *>(misc + kWmRk);
+        float *s_rg = reinterpret_cast<float *>(misc + kWmRg);
+        float *s_oct = reinterpret_cast<float *>(misc + kWmOct);
+        float *s_suf = reinterpret_cast<float *>(sm + kWSuf);
+        uint32_t stage_phase = 0, mma_phase = 0;
+        bool ok = true;
+        auto coords = [&](int item, int &b, int &h, int &ch) {
+            const int bh = item / p.nseg;
+            ch = p.c0 + (item - bh * p.nseg);
+            b = bh / p.H;
+            h = bh - b * p.H;
+        };
+        auto stage_qka = [&](int b, int h, int ch) {
+            fence_async_smem();
+            mbar_arrive_tx_raw(stage_bar, kPStageTx);
+            tma_load_3d(sbase + kWSQ, &maps.q, h * kDk, ch * kC, b, stage_bar);
+            tma_load_3d(sbase + kWSK, &maps.k, h * kDk, ch * kC, b, stage_bar);
+            tma_load_3d(sbase + kWSA, &maps.alpha, h * kDk, ch * kC, b, stage_bar);
+        };
+        auto load_beta = [&](int it, int b, int h, int ch) -> float {
+            if (ft >= kC || it >= nitems) return 0.f;
+            const int t = ch * kC + ft;
+            return t < p.T ? p.beta[(static_cast<size_t>(b) * p.T + t) * p.H + h] : 0.f;
+        };
+        int item = s_fetch[0], next = s_fetch[1];
+        int nb, nh, nch;
+        coords(item, nb, nh, nch);
+        float beta_next = load_beta(item, nb, nh, nch);
+        int pending = 0;
+        if (item < nitems) {
+            if (ft == kWStageTid) stage_qka(nb, nh, nch);
+            pending = 1;
+        }
+        for (int j = 0;; ++j) {
+            const int bf = j & 1;
+            // the buffer's previous item (j - 2) must be done with: the solver's W has read its Kt and
+            // its solve its A; the bulk store of that item's Qt has read the tile
+            if (j >= 2) {
+                bool w = true;
+                if (warp == 0)
+                    w = wait_bar(empty_bar + 8 * bf, static_cast<uint32_t>((j - 2) >> 1) & 1u, abort_flag,
+                                 &g_prefill_error, lad::kErrPrefill);
+                if (ft == kWBulkTid) bulk_wait_read1();
+                ok = half_and(1, w && ok);
+            }
+            if (item >= nitems || !ok) {
+                if (ft == 0) {
+                    s_item[bf] = -1;
+                    mbar_arrive(full_bar + 8 * bf);
+                }
+                break;
+            }
+            const int ch = nch;
+            coords(next, nb, nh, nch);
+            const int t0 = ch * kC;
+            const int n = min(kC, p.T - t0);
+            uint8_t *rec = p.ws + static_cast<size_t>(item) * kRecBytes;
+            float *sA = reinterpret_cast<float *>(sm + kWA + bf * kWAStride);
+            float *s_betaS = reinterpret_cast<float *>(misc + kWmBetaS) + bf * kC;
+            const uint32_t qw = kWQW + bf * 32768u;
+
+            if (ft < kC) {
+                s_beta[ft] = beta_next;
+                s_betaS[ft] = beta_next;
+            }
+            beta_next = load_beta(next, nb, nh, nch);
+            {
+                bool w = true;
+                if (warp == 0) w = wait_bar(stage_bar, stage_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
+                stage_phase ^= 1;
+                pending = 0;
+                ok = half_and(1, w);
+                if (!ok) {
+                    if (ft == 0) {
+                        s_item[bf] = -1;
+                        mbar_arrive(full_bar + 8 * bf);
+                    }
+                    break;
+                }
+            }
+            const uint16_t *sq = reinterpret_cast<const uint16_t *>(sm + kWSQ);
+            const uint16_t *sk = reinterpret_cast<const uint16_t *>(sm + kWSK);
+            const float *sa = reinterpret_cast<const float *>(sm + kWSA);
+            if constexpr (kL2) {
+#pragma unroll 1
+                for (int r = warp; r < kC; r += 8) {
+                    const uint2 qv = *reinterpret_cast<const uint2 *>(sq + r * kDk + 4 * lane);
+                    const uint2 kv = *reinterpret_cast<const uint2 *>(sk + r * kDk + 4 * lane);
+                    const float2 q0 = lad::dev::bf16x2_to_f32(qv.x), q1 = lad::dev::bf16x2_to_f32(qv.y);
+                    const float2 k0 = lad::dev::bf16x2_to_f32(kv.x), k1 = lad::dev::bf16x2_to_f32(kv.y);
+                    float sqs = q0.x * q0.x + q0.y * q0.y + q1.x * q1.x + q1.y * q1.y;
+                    float sks = k0.x * k0.x + k0.y * k0.y + k1.x * k1.x + k1.y * k1.y;
+#pragma unroll
+                    for (int o = 16; o; o >>= 1) {
+                        sqs += __shfl_xor_sync(0xffffffffu, sqs, o);
+                        sks += __shfl_xor_sync(0xffffffffu, sks, o);
+                    }
+                    if (lane == 0) {
+                        s_rq[r] = rsqrtf(sqs + 1e-6f);
+                        s_rk[r] = rsqrtf(sks + 1e-6f);
+                    }
+                }
+            }
+            // ---- the decays and the operand tiles, as in kda_chunk_prep_kernel, with warp w taking
+            //      the two quartets 2w, 2w + 1 (tokens 8w .. 8w+7): their products first, then after the
+            //      scan each quartet's running products again (from alpha) and its four tokens ----
+            const int c4 = 4 * lane;
+            auto quartet_products = [&](int o, float4 (&fw)[4], float4 (&bw)[4]) {
+                float4 a4[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int r = 4 * o + u;
+                    a4[u] = (r < n) ? *reinterpret_cast<const float4 *>(sa + r * kDk + c4) : make_float4(1.f, 1.f, 1.f, 1.f);
+                }
+                float2 r01 = make_float2(1.f, 1.f), r23 = r01;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    r01 = mul2(r01, make_float2(a4[u].x, a4[u].y));
+                    r23 = mul2(r23, make_float2(a4[u].z, a4[u].w));
+                    fw[u] = make_float4(r01.x, r01.y, r23.x, r23.y);
+                }
+                r01 = r23 = make_float2(1.f, 1.f);
+#pragma unroll
+                for (int u = 3; u >= 0; --u) {
+                    bw[u] = make_float4(r01.x, r01.y, r23.x, r23.y);
+                    r01 = mul2(r01, make_float2(a4[u].x, a4[u].y));
+                    r23 = mul2(r23, make_float2(a4[u].z, a4[u].w));
+                }
+            };
+#pragma unroll 1
+            for (int qq = 0; qq < 2; ++qq) {
+                float4 fw[4], bw[4];
+                quartet_products(2 * warp + qq, fw, bw);
+                *reinterpret_cast<float4 *>(s_oct + (2 * warp + qq) * kDk + c4) = fw[3];
+            }
+            half_bar(1);
+            if (ft < kDk) {
+                float y[16];
+#pragma unroll
+                for (int oo = 0; oo < 16; ++oo) y[oo] = s_oct[oo * kDk + ft];
+                float pre = 1.f, suf = 1.f;
+#pragma unroll
+                for (int oo = 0; oo < 16; ++oo) {
+                    s_oct[oo * kDk + ft] = pre;  // before quartet oo
+                    pre *= y[oo];
+                    s_suf[(15 - oo) * kDk + ft] = suf;  // after quartet 15 - oo
+                    suf *= y[15 - oo];
+                }
+                reinterpret_cast<float *>(rec + kRG)[ft] = pre;  // g_last, for the record
+                s_rg[ft] = __frcp_rn(pre);
+            }
+            half_bar(1);
+            const float4 rg = *reinterpret_cast<const float4 *>(s_rg + c4);
+            const float2 rg01 = make_float2(rg.x, rg.y), rg23 = make_float2(rg.z, rg.w);
+#pragma unroll 1
+            for (int qq = 0; qq < 2; ++qq) {
+                const int o = 2 * warp + qq;
+                float4 fw[4], bw[4];
+                quartet_products(o, fw, bw);
+                const float4 ex = *reinterpret_cast<const float4 *>(s_oct + o * kDk + c4);
+                const float4 sx = *reinterpret_cast<const float4 *>(s_suf + o * kDk + c4);
+                const float2 ex01 = make_float2(ex.x, ex.y), ex23 = make_float2(ex.z, ex.w);
+                const float2 sx01 = make_float2(sx.x, sx.y), sx23 = make_float2(sx.z, sx.w);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int r = 4 * o + u;
+                    const float2 g01 = mul2(ex01, make_float2(fw[u].x, fw[u].y));
+                    const float2 g23 = mul2(ex23, make_float2(fw[u].z, fw[u].w));
+                    const float2 R01 = mul2(sx01, make_float2(bw[u].x, bw[u].y));
+                    const float2 R23 = mul2(sx23, make_float2(bw[u].z, bw[u].w));
+                    const uint2 qv = *reinterpret_cast<const uint2 *>(sq + r * kDk + c4);
+                    const uint2 kv = *reinterpret_cast<const uint2 *>(sk + r * kDk + c4);
+                    float2 q01 = lad::dev::bf16x2_to_f32(qv.x), q23 = lad::dev::bf16x2_to_f32(qv.y);
+                    float2 k01 = lad::dev::bf16x2_to_f32(kv.x), k23 = lad::dev::bf16x2_to_f32(kv.y);
+                    if constexpr (kL2) {
+                        const float rq = s_rq[r], rk = s_rk[r];
+                        q01 = mul2(q01, make_float2(rq, rq));
+                        q23 = mul2(q23, make_float2(rq, rq));
+                        k01 = mul2(k01, make_float2(rk, rk));
+                        k23 = mul2(k23, make_float2(rk, rk));
+                    }
+                    const float2 kg01 = mul2(k01, R01), kg23 = mul2(k23, R23);
+                    const float2 kh01 = mul2(kg01, rg01), kh23 = mul2(kg23, rg23);
+                    const float2 kt01 = mul2(k01, g01), kt23 = mul2(k23, g23);
+                    const float2 qt01 = mul2(q01, g01), qt23 = mul2(q23, g23);
+                    const uint32_t off = sw128_off16(r, c4, 8192);         // 64-row tiles (Kh; the record's Kg)
+                    const uint32_t offq = sw128_off16(kC + r, c4, 16384);  // row 64 + r of [Kt; Qt]
+                    const uint32_t offk = sw128_off16(r, c4, 16384);       // row r of [Kt; Qt]
+                    *reinterpret_cast<uint2 *>(sm + qw + offk) =
+                        make_uint2(f32x2_to_f16x2(kt01.x, kt01.y), f32x2_to_f16x2(kt23.x, kt23.y));
+                    *reinterpret_cast<uint2 *>(sm + qw + offq) =
+                        make_uint2(f32x2_to_f16x2(qt01.x, qt01.y), f32x2_to_f16x2(qt23.x, qt23.y));
+                    *reinterpret_cast<uint2 *>(sm + kWKH + off) =
+                        make_uint2(f32x2_to_f16x2(kh01.x, kh01.y), f32x2_to_f16x2(kh23.x, kh23.y));
+                    *reinterpret_cast<uint2 *>(rec + kRKG + off) =
+                        make_uint2(f32x2_to_f16x2(kg01.x, kg01.y), f32x2_to_f16x2(kg23.x, kg23.y));
+                }
+            }
+            // ---- [Kt; Qt] Kh^T: rows 0-63 give Kt Kh^T, rows 64-127 Qt Kh^T ----
+            fence_async_smem();
+            tc_fence_before();
+            half_bar(1);  // q, k and alpha of this item are read: the next item's come in
+            if (next < nitems) {
+                if (ft == kWStageTid) stage_qka(nb, nh, nch);
+                pending = 1;
+            }
+            if (ft == kWFetchTid) s_fetch[0] = atomicAdd(p.counter, 1);  // read after this item's last barrier
+            if (ft == kWBulkTid) {  // the record's Qt (rows 64-127 of each block of the tile)
+                bulk_s2g(rec + kRWQ + 8192, sbase + qw + 8192, 8192);
+                bulk_s2g(rec + kRWQ + 16384 + 8192, sbase + qw + 16384 + 8192, 8192);
+                bulk_commit();
+            }
+            if (warp == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int jj = 0; jj < kDk / 16; ++jj)
+                    tc_mma_f16(tmem + kWColA, kdesc16(d0 + (qw >> 4), 16384, jj), kdesc16(d0 + (kWKH >> 4), 8192, jj),
+                               kIdescA, jj > 0);
+                tc_commit(mmaf_bar);
+            }
+            {
+                bool w = true;
+                if (warp == 0) w = wait_bar(mmaf_bar, mma_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
+                mma_phase ^= 1;
+                ok = half_and(1, w);
+                tc_fence_after();
+                if (!ok) {
+                    if (ft == 0) {
+                        s_item[bf] = -1;
+                        mbar_arrive(full_bar + 8 * bf);
+                    }
+                    break;
+                }
+            }
+            // ---- A = strict_lower(diag(beta) Kt Kh^T) -> fp32 scratch; P = lower(Qt Kh^T) -> the
+            //      record (fp16); a warp takes 32 of a row's 64 columns, in two 16-column loads ----
+#pragma unroll 1
+            for (int qq = 0; qq < 2; ++qq) {
+                const int qd = 2 * (warp >> 2) + qq;
+                float x[16];
+                tmem_ld16(tmem + lane_base + kWColA + 16 * qd, x);
+                tmem_wait_ld();
+                const int row = 32 * sp + lane, c0 = 16 * qd;
+                if (row < kC) {
+                    const int r = row;
+                    const float br = s_beta[r];
+                    float4 *dst = reinterpret_cast<float4 *>(sA + r * kAS + c0);
+#pragma unroll
+                    for (int jj = 0; jj < 16; jj += 4) {
+                        const float2 p01 = mul2(make_float2(br, br), make_float2(x[jj], x[jj + 1]));
+                        const float2 p23 = mul2(make_float2(br, br), make_float2(x[jj + 2], x[jj + 3]));
+                        dst[jj / 4] = make_float4(c0 + jj < r ? p01.x : 0.f, c0 + jj + 1 < r ? p01.y : 0.f,
+                                                  c0 + jj + 2 < r ? p23.x : 0.f, c0 + jj + 3 < r ? p23.y : 0.f);
+                    }
+                } else {
+                    const int r = row - kC;
+#pragma unroll
+                    for (int jj = 0; jj < 16; jj += 8) {
+                        float y[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y[e] = (c0 + jj + e <= r) ? x[jj + e] : 0.f;
+                        *reinterpret_cast<uint4 *>(rec + kRP + sw128_off16(r, c0 + jj, 8192)) =
+                            make_uint4(f32x2_to_f16x2(y[0], y[1]), f32x2_to_f16x2(y[2], y[3]),
+                                       f32x2_to_f16x2(y[4], y[5]), f32x2_to_f16x2(y[6], y[7]));
+                    }
+                }
+            }
+            tc_fence_before();
+            half_bar(1);  // A and beta of the item are in place (and TMEM's column block is read)
+            if (ft == 0) {
+                s_item[bf] = item;
+                mbar_arrive(full_bar + 8 * bf);
+            }
+            item = next;
+            next = s_fetch[0];
+        }
+        // drain: a staging copy still in flight (after an abort) lands and the Qt stores have read
+        // their tiles
+        if (ft == 0 && pending) {
+            const uint64_t t0 = lad::dev::globaltimer_ns();
+            while (!mbar_try_wait(stage_bar, stage_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+            }
+        }
+        if (ft == kWBulkTid) bulk_wait_all();
+        // every [Kt; Qt] Kh^T MMA has completed (after an abort, a fresh commit is waited for, bounded)
+        if (warp == 0) {
+            tc_commit(mmaf_bar);
+            if (lane == 0) {
+                const uint64_t t0 = lad::dev::globaltimer_ns();
+                while (!mbar_try_wait(mmaf_bar, mma_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+                }
+            }
+            __syncwarp();
+        }
+    } else {
+        // ============================== the solver ==============================
+        const int st = tid - kWHalf;  // 0-255
+        const int sw = st >> 5;       // the solver's warp, 0-7
+        float *sT = reinterpret_cast<float *>(sm + kWT);
+        uint32_t mma_phase = 0;
+        for (int j = 0;; ++j) {
+            const int bf = j & 1;
+            bool w = true;
+            if (sw == 0)
+                w = wait_bar(full_bar + 8 * bf, static_cast<uint32_t>(j >> 1) & 1u, abort_flag, &g_prefill_error,
+                             lad::kErrPrefill);
+            if (!half_and(2, w)) break;
+            const int item = s_item[bf];
+            if (item < 0) break;
+            uint8_t *rec = p.ws + static_cast<size_t>(item) * kRecBytes;
+            float *sA = reinterpret_cast<float *>(sm + kWA + bf * kWAStride);
+            const float *s_betaS = reinterpret_cast<const float *>(misc + kWmBetaS) + bf * kC;
+            // ---- T = (I + A)^-1, Tb = T diag(beta): the fp16 tile here, the bf16 hi / lo pair straight
+            //      into the record ----
+            solve_tb<kWHalf>(sA, sT, s_betaS, sm + kWTB, rec + kRTH, rec + kRTL, st, []() { half_bar(2); });
+            // ---- W = Tb Kt (Kt: rows 0-63 of the buffer's [Kt; Qt], read MN-major) ----
+            fence_async_smem();
+            tc_fence_before();
+            half_bar(2);
+            if (sw == 0) {
+                tc_fence_after();
+                const uint64_t kt0 = smem_desc(sbase + kWQW + bf * 32768u, 16384, 1024, kLayoutSw128);
+#pragma unroll
+                for (int jj = 0; jj < kC / 16; ++jj)
+                    tc_mma_f16(tmem + kWColW, kdesc16(d0 + (kWTB >> 4), 8192, jj), kt0 + ((jj * 2048) >> 4), kIdescW,
+                               jj > 0);
+                tc_commit(mmas_bar);
+            }
+            bool w2 = true;
+            if (sw == 0) w2 = wait_bar(mmas_bar, mma_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
+            mma_phase ^= 1;
+            const bool ok = half_and(2, w2);
+            tc_fence_after();
+            if (!ok) break;
+            if (st == 0) mbar_arrive(empty_bar + 8 * bf);  // the buffer's Kt and A are free
+            // ---- W -> the record's [W; Qt] tile (rows 0-63). M = 64: row 16 sp + i sits in lane i
+            //      (< 16) of sub-partition sp; the loads are collective, so the whole warp issues them
+            //      and lanes 0-15 keep the rows. A warp takes 64 of the 128 columns ----
+#pragma unroll 1
+            for (int qq = 0; qq < 2; ++qq) {
+                const int c0 = 64 * (sw >> 2) + 32 * qq;
+                float wv[32];
+                tmem_ld32(tmem + lane_base + kWColW + c0, wv);
+                tmem_wait_ld();
+                if (lane < 16) {
+                    const int r = 16 * sp + lane;
+#pragma unroll
+                    for (int jj = 0; jj < 32; jj += 8)
+                        *reinterpret_cast<uint4 *>(rec + kRWQ + sw128_off16(r, c0 + jj, 16384)) =
+                            make_uint4(f32x2_to_f16x2(wv[jj], wv[jj + 1]), f32x2_to_f16x2(wv[jj + 2], wv[jj + 3]),
+                                       f32x2_to_f16x2(wv[jj + 4], wv[jj + 5]), f32x2_to_f16x2(wv[jj + 6], wv[jj + 7]));
+                }
+            }
+            tc_fence_before();  // the W loads are done before the next item's W MMA
+        }
+        // every W MMA has completed (after an abort, a fresh commit is waited for, bounded)
+        if (sw == 0) {
+            tc_commit(mmas_bar);
+            if (lane == 0) {
+                const uint64_t t0 = lad::dev::globaltimer_ns();
+                while (!mbar_try_wait(mmas_bar, mma_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
+                }
+            }
+            __syncwarp();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kWTmemCols);
 }
 
 struct ChainArgs {
@@ -1718,6 +2187,12 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
                 attr_err = cudaFuncSetAttribute(kda_chunk_prep_kernel<true>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
             if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute(kda_chunk_prep_ws_kernel<false>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kWSmemBytes);
+            if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute(kda_chunk_prep_ws_kernel<true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kWSmemBytes);
+            if (attr_err == cudaSuccess)
                 attr_err = cudaFuncSetAttribute(kda_chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 kCSmemBytes);
             if (attr_err != cudaSuccess)
@@ -1786,10 +2261,17 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
     const int beside = sms - chain_ctas > sms / 2 ? sms - chain_ctas : sms / 2;
     auto prep = [&](cudaStream_t on, long long grid, int sg, uint8_t *buf, int c0, int nseg) {
         const PrepArgs pa{beta, buf, counters + sg, B, T, H, c0, nseg, a.l2norm};
+#if LAD_PREFILL_PREP_WS
+        if (a.l2norm)
+            kda_chunk_prep_ws_kernel<true><<<static_cast<unsigned>(grid), kPThreads, kWSmemBytes, on>>>(pa, pm);
+        else
+            kda_chunk_prep_ws_kernel<false><<<static_cast<unsigned>(grid), kPThreads, kWSmemBytes, on>>>(pa, pm);
+#else
         if (a.l2norm)
             kda_chunk_prep_kernel<true><<<static_cast<unsigned>(grid), kPThreads, kPSmemBytes, on>>>(pa, pm);
         else
             kda_chunk_prep_kernel<false><<<static_cast<unsigned>(grid), kPThreads, kPSmemBytes, on>>>(pa, pm);
+#endif
         return cudaGetLastError();
     };
     for (int sg = 0; sg < L.nsegs && e == cudaSuccess; ++sg) {
