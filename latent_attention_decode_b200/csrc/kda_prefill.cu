@@ -615,18 +615,18 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
 // ------------------------------------------------------------------------------------------
 // Split path (a workspace is given): the chunk-local, state-independent part of every chunk in
 // parallel (prep), then the state chain alone (chain), segment by segment. With S0 the state
-// entering a chunk, Tb = (I + A)^-1 diag(beta), W = Tb Kt, P = lower(Qt Kh^T) and
-// Kg = K * g_last / g (the chunk's decay folded into the key), the chunk form is
-//   U' = Tb V,  X = W S0,  U = U' - X,  O = scale (Qt S0 + P U),  S = Diag(g_last) S0 + Kg^T U.
+// entering a chunk, Tb = (I + A)^-1 diag(beta), W = Tb Kt and P = lower(Qt Kh^T), the chunk form is
+//   U' = Tb V,  X = W S0,  U = U' - X,  O = scale (Qt S0 + P U),  S = Diag(g_last) (S0 + Kh^T U)
+// (the last is Diag(g_last) S0 + (K * g_last / g)^T U with the chunk's decay taken out of the key).
 // The prep computes what needs the CUDA cores (the decays, the operand tiles, the triangular
-// inverse) and one tensor-core product, W; it writes Qt, W, Kg, P, Tb (as a bf16 hi + lo pair)
+// inverse) and one tensor-core product, W; it writes Qt, W, Kh, P, Tb (as a bf16 hi + lo pair)
 // and g_last as one record per chunk. The chain holds S^T (rows d_v, columns d_k) as an fp32
 // master in tensor memory and per chunk runs two tensor-core batches (M = 128 value rows), with
 // one pass through the threads between them and one after:
 //   X^T = S0^T W^T,  O^T = S0^T Qt^T,  U'^T = V^T (Tb_hi + Tb_lo)^T      (V by TMA from the input)
 //   U^T = U'^T - X^T  (threads: fp32 -> fp16 operand)
-//   S^T += U^T Kg,  O^T += U^T P^T
-//   S^T <- S^T Diag(g_last of the next chunk) (threads, fp32), and its fp16 copy (the next S0^T)
+//   S^T += U^T Kh,  O^T += U^T P^T
+//   S^T <- S^T Diag(g_last) (threads, fp32), and its fp16 copy (the next chunk's S0^T)
 // The decay itself is never rounded to fp16.
 // Every operand is fp16 (kind::f16, fp32 accumulation): its rounding unit is that of tf32 and it
 // runs at twice tf32's rate with half the bytes; each tile is stored once, rows as formed, and
@@ -639,15 +639,12 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_kernel(Args p, const 
 // Record of one (sequence, head, chunk) in the workspace: the chain's operand tiles (fp16 / bf16,
 // SW128) and g_last, laid out exactly as in the chain's shared memory (one bulk copy).
 constexpr uint32_t kRWQ = 0;           // [W; Qt] [128 rows: 64 W, 64 Qt tok][128 d_k], K-major: 2 blocks x 16 KiB
-constexpr uint32_t kRKG = 32768;       // Kg [64 tok][128 d_k]: 2 blocks x 8 KiB (read MN-major)
+constexpr uint32_t kRKH = 32768;       // Kh [64 tok][128 d_k]: 2 blocks x 8 KiB (read MN-major)
 constexpr uint32_t kRP = 49152;        // P [64 r][64 s], K-major: 8 KiB
 constexpr uint32_t kRTH = 57344;       // Tb, bf16 high part [64 r][64 s], K-major: 8 KiB
 constexpr uint32_t kRTL = 65536;       // Tb, bf16 low part (Tb - hi): 8 KiB
 constexpr uint32_t kRG = 73728;        // g_last [128] fp32
 constexpr uint32_t kRecBytes = 74240;  // 580 lines of 128 bytes
-#ifndef LAD_PREFILL_PREP_WS
-#define LAD_PREFILL_PREP_WS 1  // the warp-specialised prep (kda_chunk_prep_ws_kernel)
-#endif
 #ifndef LAD_PREFILL_SEG_CHUNKS
 #define LAD_PREFILL_SEG_CHUNKS 128
 #endif
@@ -675,7 +672,7 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
 constexpr uint32_t kIdescA = make_idesc(128, 64, kFmtF16, 0, 0);     // [Kt; Qt] Kh^T
 constexpr uint32_t kIdescW = make_idesc(64, 128, kFmtF16, 0, 1);     // W = Tb Kt (Kt read MN-major)
 constexpr uint32_t kIdescU = make_idesc(128, 64, kFmtBf16, 1, 0);    // U'^T = V^T Tb^T (V read MN-major)
-constexpr uint32_t kIdescSU = make_idesc(128, 128, kFmtF16, 0, 1);   // S^T += U^T Kg (Kg read MN-major)
+constexpr uint32_t kIdescSU = make_idesc(128, 128, kFmtF16, 0, 1);   // S^T += U^T Kh (Kh read MN-major)
 constexpr uint32_t kIdescXO = make_idesc(128, 128, kFmtF16, 0, 0);  // [X^T | O^T] = S0^T [W; Qt]^T
 constexpr uint32_t kIdescO = make_idesc(128, 64, kFmtF16, 0, 0);     // O^T += U^T P^T
 
@@ -692,38 +689,9 @@ struct PrepMaps {
     CUtensorMap q, k, alpha;  // 3-D [B][T][H*128], boxes of 128 channels x 64 tokens, no swizzle
 };
 
-// prep shared memory (offsets from a 1024-aligned base). The A / T scratch holds W once the solve
-// is done with it. The record leaves by bulk stores from where its tiles sit.
-constexpr uint32_t kPQW = 0;        // [Kt; Qt]: 128 rows x 128 d_k fp16, K-major, 2 blocks x 16 KiB (Qt: record)
-constexpr uint32_t kPKH = 32768;    // Kh [64 tok][128 d_k], 2 blocks x 8 KiB
-constexpr uint32_t kPKG = 49152;    // Kg [64 tok][128 d_k], 2 blocks x 8 KiB (record)
-constexpr uint32_t kPP = 65536;     // P [64][64] (record)
-constexpr uint32_t kPG = 73728;     // g_last [128] fp32 (record)
-constexpr uint32_t kPTB = 74752;    // Tb [64 r][64 s] fp16 K-major
-constexpr uint32_t kPTBH = 82944;   // Tb, bf16 high part (record, with the low part right after it)
-constexpr uint32_t kPTBL = 91136;   // Tb, bf16 low part (Tb - hi)
-constexpr uint32_t kPSuf = 99328;   // the decay scan's backward products [16 quartets][128] fp32
-constexpr uint32_t kPSQ = 115712;   // q [64 tok][128] bf16, plain (TMA)
-constexpr uint32_t kPSK = 132096;   // k, the same
-constexpr uint32_t kPSA = 148480;   // alpha [64 tok][128] fp32, plain (TMA)
 constexpr int kAS = 68;             // row stride (floats) of the A / T scratch (68: fewer bank conflicts)
-constexpr uint32_t kPA = 181248;    // A [64][kAS] fp32; then W [64 tok][128 d_k] fp16, 2 blocks x 8 KiB (record)
-constexpr uint32_t kPT = kPA + 64 * kAS * 4;   // T [64][kAS] fp32
-constexpr uint32_t kPMisc = kPT + 64 * kAS * 4;
-constexpr int kPThreads = 512;      // 16 warps: the CUDA-core phases are latency-bound
-constexpr int kPWarps = kPThreads / 32;
-constexpr int kPStageTid = 32;  // issues the input staging (warp 0 issues the MMAs)
-constexpr int kPBulkTid = 64;   // issues the record's bulk stores, in four groups an item, and waits on them
-constexpr int kPFetchTid = 128; // takes items from the segment's counter
-// the record's four bulk groups of an item, in order: Qt, Kg and g_last (after the formation);
-// P (after the first extraction); Tb hi / lo (after the solve); W (last)
-constexpr uint32_t kPmBeta = 0, kPmRq = 256, kPmRk = 512, kPmOct = 768, kPmBar = 768 + kPWarps * 128 * 4,
-                   kPmTmem = kPmBar + 16, kPmAbort = kPmBar + 20, kPmFetch = kPmBar + 24, kPmRg = kPmBar + 32;
-constexpr uint32_t kPSmemBytes = kPMisc + kPmRg + 512 + 1024;
-static_assert(kPSmemBytes <= 232448, "prep shared memory over the per-block limit");
-constexpr uint32_t kPStageTx = 16384 + 16384 + 32768;  // q, k, alpha
-// TMEM columns: [Kt; Qt] Kh^T, W
-constexpr uint32_t kPColA = 0, kPColW = 64, kPTmemCols = 256;
+constexpr int kPThreads = 512;      // the prep's 16 warps
+constexpr uint32_t kPStageTx = 16384 + 16384 + 32768;  // q, k, alpha of an item
 
 // element (r, s) of the three Tb tiles, four consecutive s at once (s % 4 == 0)
 __device__ __forceinline__ void put_tb4(uint8_t *tb16, uint8_t *tbh, uint8_t *tbl, int r, int s, float2 ab, float2 cd) {
@@ -888,379 +856,25 @@ __device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read3() { asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// One CTA per SM walks the segment's (sequence, head, chunk) items with 16 warps. The next item's
-// q, k and alpha are staged (TMA) once the current item's operand tiles are formed; its beta is
-// prefetched into a register at the start of the current item. The record leaves by bulk stores.
-template <bool kL2>  // kL2: q and k are L2-normalised per token (p.l2norm)
-__global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_kernel(PrepArgs p, const __grid_constant__ PrepMaps maps) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t sbase = smem_u32(sm);
-    float *s_beta = reinterpret_cast<float *>(sm + kPMisc + kPmBeta);
-    float *s_rq = reinterpret_cast<float *>(sm + kPMisc + kPmRq);
-    float *s_rk = reinterpret_cast<float *>(sm + kPMisc + kPmRk);
-    float *s_oct = reinterpret_cast<float *>(sm + kPMisc + kPmOct);  // per quartet: forward products
-    float *s_suf = reinterpret_cast<float *>(sm + kPSuf);           //   backward ones
-    float *s_rg = reinterpret_cast<float *>(sm + kPMisc + kPmRg);    // 1 / g_last
-    float *s_g = reinterpret_cast<float *>(sm + kPG);
-    float *sA = reinterpret_cast<float *>(sm + kPA);
-    float *sT = reinterpret_cast<float *>(sm + kPT);
-    const uint32_t stage_bar = sbase + kPMisc + kPmBar;
-    const uint32_t mma_bar = stage_bar + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kPMisc + kPmTmem);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kPMisc + kPmAbort);
-    int *s_fetch = reinterpret_cast<int *>(sm + kPMisc + kPmFetch);  // items taken from the counter
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int sp = warp & 3, qd = warp >> 2;  // TMEM sub-partition; quarter of an accumulator's columns
-    const uint32_t lane_base = static_cast<uint32_t>(32 * sp) << 16;
-    const int nitems = p.B * p.H * p.nseg;
-
-    if (tid == 0) {
-        mbar_init(stage_bar, 1);
-        mbar_init(mma_bar, 1);
-        *abort_flag = 0;
-        s_fetch[0] = atomicAdd(p.counter, 1);  // the first item, and the one after it
-        s_fetch[1] = atomicAdd(p.counter, 1);
-        mbar_fence_init();
-    }
-    if (warp == 0) tmem_alloc(smem_u32(tmem_slot), kPTmemCols);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    uint32_t stage_phase = 0, mma_phase = 0;
-    bool ok = true;
-
-    // item -> (b, h, chunk); the items of one (b, h) are consecutive
-    auto coords = [&](int item, int &b, int &h, int &ch) {
-        const int bh = item / p.nseg;
-        ch = p.c0 + (item - bh * p.nseg);
-        b = bh / p.H;
-        h = bh - b * p.H;
-    };
-    auto stage_qka = [&](int b, int h, int ch) {
-        fence_async_smem();
-        mbar_arrive_tx_raw(stage_bar, kPStageTx);
-        tma_load_3d(sbase + kPSQ, &maps.q, h * kDk, ch * kC, b, stage_bar);
-        tma_load_3d(sbase + kPSK, &maps.k, h * kDk, ch * kC, b, stage_bar);
-        tma_load_3d(sbase + kPSA, &maps.alpha, h * kDk, ch * kC, b, stage_bar);
-    };
-    // one warp watches a barrier's phase; the others wait at the CTA barrier, which costs them no
-    // issue slots (sixteen warps polling the mbarrier would)
-    auto mma_wait = [&]() {
-        bool w = true;
-        if (warp == 0) w = wait_bar(mma_bar, mma_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
-        mma_phase ^= 1;
-        const bool r = __syncthreads_and(w) != 0;
-        tc_fence_after();
-        return r;
-    };
-    const uint64_t d0 = smem_desc(sbase, 16, 1024, kLayoutSw128);  // K-major SW128 at offset 0
-
-    int pending = 0;  // a staging phase is in flight
-    // items come from the segment's counter, one at a time (CTAs that start late, behind other
-    // work on their SM, take fewer); the next one is always known an item ahead, for the prefetch
-    int item = s_fetch[0], next = s_fetch[1];
-    // beta of an item (threads 0-63, one token each, strided by H in memory): loaded one item ahead
-    auto load_beta = [&](int it, int b, int h, int ch) -> float {
-        if (tid >= kC || it >= nitems) return 0.f;
-        const int t = ch * kC + tid;
-        return t < p.T ? p.beta[(static_cast<size_t>(b) * p.T + t) * p.H + h] : 0.f;
-    };
-    // coordinates of the next item, computed once (the integer divisions are not cheap)
-    int nb, nh, nch;
-    coords(item, nb, nh, nch);
-    float beta_next = load_beta(item, nb, nh, nch);
-    if (item < nitems) {
-        if (tid == kPStageTid) stage_qka(nb, nh, nch);
-        pending = 1;
-    }
-    while (item < nitems && ok) {
-        const int ch = nch;
-        coords(next, nb, nh, nch);
-        const int t0 = ch * kC;
-        const int n = min(kC, p.T - t0);
-        uint8_t *rec = p.ws + static_cast<size_t>(item) * kRecBytes;
-
-        if (tid < kC) s_beta[tid] = beta_next;
-        beta_next = load_beta(next, nb, nh, nch);
-        if (tid == kPBulkTid) bulk_wait_read3();  // the previous item's Qt, Kg and g_last have left
-        {
-            bool w = true;
-            if (warp == 0) w = wait_bar(stage_bar, stage_phase, abort_flag, &g_prefill_error, lad::kErrPrefill);
-            stage_phase ^= 1;
-            pending = 0;
-            ok = __syncthreads_and(w) != 0;
-            if (!ok) break;
-        }
-        const uint16_t *sq = reinterpret_cast<const uint16_t *>(sm + kPSQ);
-        const uint16_t *sk = reinterpret_cast<const uint16_t *>(sm + kPSK);
-        const float *sa = reinterpret_cast<const float *>(sm + kPSA);
-        if constexpr (kL2) {
-#pragma unroll 1
-            for (int r = warp; r < kC; r += kPWarps) {
-                const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + 4 * lane);
-                const uint2 kw = *reinterpret_cast<const uint2 *>(sk + r * kDk + 4 * lane);
-                const float2 q0 = lad::dev::bf16x2_to_f32(qw.x), q1 = lad::dev::bf16x2_to_f32(qw.y);
-                const float2 k0 = lad::dev::bf16x2_to_f32(kw.x), k1 = lad::dev::bf16x2_to_f32(kw.y);
-                float sqs = q0.x * q0.x + q0.y * q0.y + q1.x * q1.x + q1.y * q1.y;
-                float sks = k0.x * k0.x + k0.y * k0.y + k1.x * k1.x + k1.y * k1.y;
-#pragma unroll
-                for (int o = 16; o; o >>= 1) {
-                    sqs += __shfl_xor_sync(0xffffffffu, sqs, o);
-                    sks += __shfl_xor_sync(0xffffffffu, sks, o);
-                }
-                if (lane == 0) {
-                    s_rq[r] = rsqrtf(sqs + 1e-6f);
-                    s_rk[r] = rsqrtf(sks + 1e-6f);
-                }
-            }
-        }
-
-        // ---- running decays and the operand tiles. Per key channel, g_r = prod_{s <= r} alpha_s and
-        //      R_r = prod_{s > r} alpha_s (so Kg = K R = K g_last / g and Kh = Kg / g_last: one
-        //      reciprocal per channel, none per element). Warp w takes tokens 4w .. 4w+3, lane l the
-        //      channels 4l .. 4l+3; the 16 quartet products of a channel are scanned both ways by
-        //      threads 0-127, one channel each ----
-        {
-            const int o = warp, c4 = 4 * lane;
-            float4 fw[4], bw[4];
-            {
-                float4 a4[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int r = 4 * o + u;
-                    a4[u] = (r < n) ? *reinterpret_cast<const float4 *>(sa + r * kDk + c4) : make_float4(1.f, 1.f, 1.f, 1.f);
-                }
-                // (packed pairs: two products an instruction, each rounded as a scalar one)
-                float2 r01 = make_float2(1.f, 1.f), r23 = r01;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    r01 = mul2(r01, make_float2(a4[u].x, a4[u].y));
-                    r23 = mul2(r23, make_float2(a4[u].z, a4[u].w));
-                    fw[u] = make_float4(r01.x, r01.y, r23.x, r23.y);  // prod over the quartet's tokens up to u
-                }
-                r01 = r23 = make_float2(1.f, 1.f);
-#pragma unroll
-                for (int u = 3; u >= 0; --u) {
-                    bw[u] = make_float4(r01.x, r01.y, r23.x, r23.y);  // prod over the quartet's tokens after u
-                    r01 = mul2(r01, make_float2(a4[u].x, a4[u].y));
-                    r23 = mul2(r23, make_float2(a4[u].z, a4[u].w));
-                }
-            }
-            *reinterpret_cast<float4 *>(s_oct + o * kDk + c4) = fw[3];
-            __syncthreads();
-            if (tid < kDk) {
-                float y[kPWarps];
-#pragma unroll
-                for (int oo = 0; oo < kPWarps; ++oo) y[oo] = s_oct[oo * kDk + tid];
-                float pre = 1.f, suf = 1.f;
-#pragma unroll
-                for (int oo = 0; oo < kPWarps; ++oo) {
-                    s_oct[oo * kDk + tid] = pre;  // before quartet oo
-                    pre *= y[oo];
-                    s_suf[(kPWarps - 1 - oo) * kDk + tid] = suf;  // after quartet 15 - oo
-                    suf *= y[kPWarps - 1 - oo];
-                }
-                s_g[tid] = pre;  // g_last, for the record
-                s_rg[tid] = __frcp_rn(pre);
-            }
-            __syncthreads();
-            const float4 ex = *reinterpret_cast<const float4 *>(s_oct + o * kDk + c4);
-            const float4 sx = *reinterpret_cast<const float4 *>(s_suf + o * kDk + c4);
-            const float4 rg = *reinterpret_cast<const float4 *>(s_rg + c4);
-            const float2 ex01 = make_float2(ex.x, ex.y), ex23 = make_float2(ex.z, ex.w);
-            const float2 sx01 = make_float2(sx.x, sx.y), sx23 = make_float2(sx.z, sx.w);
-            const float2 rg01 = make_float2(rg.x, rg.y), rg23 = make_float2(rg.z, rg.w);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int r = 4 * o + u;
-                const float2 g01 = mul2(ex01, make_float2(fw[u].x, fw[u].y));
-                const float2 g23 = mul2(ex23, make_float2(fw[u].z, fw[u].w));
-                const float2 R01 = mul2(sx01, make_float2(bw[u].x, bw[u].y));
-                const float2 R23 = mul2(sx23, make_float2(bw[u].z, bw[u].w));
-                const uint2 qw = *reinterpret_cast<const uint2 *>(sq + r * kDk + c4);
-                const uint2 kw = *reinterpret_cast<const uint2 *>(sk + r * kDk + c4);
-                float2 q01 = lad::dev::bf16x2_to_f32(qw.x), q23 = lad::dev::bf16x2_to_f32(qw.y);
-                float2 k01 = lad::dev::bf16x2_to_f32(kw.x), k23 = lad::dev::bf16x2_to_f32(kw.y);
-                if constexpr (kL2) {
-                    const float rq = s_rq[r], rk = s_rk[r];
-                    q01 = mul2(q01, make_float2(rq, rq));
-                    q23 = mul2(q23, make_float2(rq, rq));
-                    k01 = mul2(k01, make_float2(rk, rk));
-                    k23 = mul2(k23, make_float2(rk, rk));
-                }
-                const float2 kg01 = mul2(k01, R01), kg23 = mul2(k23, R23);
-                const float2 kh01 = mul2(kg01, rg01), kh23 = mul2(kg23, rg23);
-                const float2 kt01 = mul2(k01, g01), kt23 = mul2(k23, g23);
-                const float2 qt01 = mul2(q01, g01), qt23 = mul2(q23, g23);
-                const uint32_t off = sw128_off16(r, c4, 8192);                 // 64-row tiles (Kh, Kg)
-                const uint32_t offq = sw128_off16(kC + r, c4, 16384);          // row 64 + r of [Kt; Qt]
-                const uint32_t offk = sw128_off16(r, c4, 16384);               // row r of [Kt; Qt]
-                *reinterpret_cast<uint2 *>(sm + kPQW + offk) =
-                    make_uint2(f32x2_to_f16x2(kt01.x, kt01.y), f32x2_to_f16x2(kt23.x, kt23.y));
-                *reinterpret_cast<uint2 *>(sm + kPQW + offq) =
-                    make_uint2(f32x2_to_f16x2(qt01.x, qt01.y), f32x2_to_f16x2(qt23.x, qt23.y));
-                *reinterpret_cast<uint2 *>(sm + kPKH + off) =
-                    make_uint2(f32x2_to_f16x2(kh01.x, kh01.y), f32x2_to_f16x2(kh23.x, kh23.y));
-                *reinterpret_cast<uint2 *>(sm + kPKG + off) =
-                    make_uint2(f32x2_to_f16x2(kg01.x, kg01.y), f32x2_to_f16x2(kg23.x, kg23.y));
-            }
-        }
-        // ---- [Kt; Qt] Kh^T: rows 0-63 give Kt Kh^T, rows 64-127 Qt Kh^T ----
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();  // q, k and alpha of this item are read: the next item's come in
-        if (next < nitems) {
-            if (tid == kPStageTid) stage_qka(nb, nh, nch);
-            pending = 1;
-        }
-        // the item after next, read after this item's last barrier; taken by a thread outside warp 0,
-        // which issues the MMAs below and would otherwise wait for the atomic's round trip first
-        if (tid == kPFetchTid) s_fetch[0] = atomicAdd(p.counter, 1);
-        if (tid == kPBulkTid) {  // the record's Qt, Kg and g_last are final
-            bulk_s2g(rec + kRWQ + 8192, sbase + kPQW + 8192, 8192);  // rows 64-127 of each block
-            bulk_s2g(rec + kRWQ + 16384 + 8192, sbase + kPQW + 16384 + 8192, 8192);
-            bulk_s2g(rec + kRKG, sbase + kPKG, 16384);
-            bulk_s2g(rec + kRG, sbase + kPG, 512);
-            bulk_commit();
-        }
-        if (warp == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < kDk / 16; ++j)
-                tc_mma_f16(tmem + kPColA, kdesc16(d0 + (kPQW >> 4), 16384, j), kdesc16(d0 + (kPKH >> 4), 8192, j),
-                           kIdescA, j > 0);
-            tc_commit(mma_bar);
-        }
-        if (tid == kPBulkTid) bulk_wait_read1();  // the previous item's P, Tb hi / lo and W have left
-        ok = mma_wait();
-        if (!ok) break;
-        // ---- A = strict_lower(diag(beta) Kt Kh^T) -> fp32 scratch; P = lower(Qt Kh^T) -> fp16 tile;
-        //      a thread takes 16 of a row's 64 columns ----
-        {
-            float x[16];
-            tmem_ld16(tmem + lane_base + kPColA + 16 * qd, x);
-            tmem_wait_ld();
-            const int row = 32 * sp + lane, c0 = 16 * qd;
-            if (row < kC) {
-                const int r = row;
-                const float br = s_beta[r];
-                float4 *dst = reinterpret_cast<float4 *>(sA + r * kAS + c0);
-#pragma unroll
-                for (int j = 0; j < 16; j += 4) {
-                    const float2 p01 = mul2(make_float2(br, br), make_float2(x[j], x[j + 1]));
-                    const float2 p23 = mul2(make_float2(br, br), make_float2(x[j + 2], x[j + 3]));
-                    dst[j / 4] = make_float4(c0 + j < r ? p01.x : 0.f, c0 + j + 1 < r ? p01.y : 0.f,
-                                             c0 + j + 2 < r ? p23.x : 0.f, c0 + j + 3 < r ? p23.y : 0.f);
-                }
-            } else {
-                const int r = row - kC;
-#pragma unroll
-                for (int j = 0; j < 16; j += 8) {
-                    float y[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) y[e] = (c0 + j + e <= r) ? x[j + e] : 0.f;
-                    *reinterpret_cast<uint4 *>(sm + kPP + sw128_off16(r, c0 + j, 8192)) =
-                        make_uint4(f32x2_to_f16x2(y[0], y[1]), f32x2_to_f16x2(y[2], y[3]), f32x2_to_f16x2(y[4], y[5]),
-                                   f32x2_to_f16x2(y[6], y[7]));
-                }
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == kPBulkTid) {  // P is final
-            bulk_s2g(rec + kRP, sbase + kPP, 8192);
-            bulk_commit();
-        }
-        // ---- T = (I + A)^-1, Tb = T diag(beta) -> the fp16 tile and its bf16 hi / lo split ----
-        solve_tb<kPThreads>(sA, sT, s_beta, sm + kPTB, sm + kPTBH, sm + kPTBL, tid, []() { __syncthreads(); });
-        // ---- W = Tb Kt (Kt: rows 0-63 of [Kt; Qt], read MN-major) ----
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == kPBulkTid) {  // Tb hi / lo are final
-            bulk_s2g(rec + kRTH, sbase + kPTBH, 16384);
-            bulk_commit();
-        }
-        if (warp == 0) {
-            tc_fence_after();
-            const uint64_t kt0 = smem_desc(sbase + kPQW, 16384, 1024, kLayoutSw128);  // MN chunks 16 KiB apart
-#pragma unroll
-            for (int j = 0; j < kC / 16; ++j)
-                tc_mma_f16(tmem + kPColW, kdesc16(d0 + (kPTB >> 4), 8192, j), kt0 + ((j * 2048) >> 4), kIdescW, j > 0);
-            tc_commit(mma_bar);
-        }
-        ok = mma_wait();
-        if (!ok) break;
-        // ---- W -> fp16 tile over the A / T scratch. M = 64: row 16 sp + i sits in lane i (< 16) of
-        //      sub-partition sp; the load is collective, so the whole warp issues it and lanes 0-15
-        //      keep the rows ----
-        {
-            const int c0 = 32 * qd;
-            float w[32];
-            tmem_ld32(tmem + lane_base + kPColW + c0, w);
-            tmem_wait_ld();
-            if (lane < 16) {
-                const int r = 16 * sp + lane;
-#pragma unroll
-                for (int j = 0; j < 32; j += 8)
-                    *reinterpret_cast<uint4 *>(sm + kPA + sw128_off16(r, c0 + j, 8192)) =
-                        make_uint4(f32x2_to_f16x2(w[j], w[j + 1]), f32x2_to_f16x2(w[j + 2], w[j + 3]),
-                                   f32x2_to_f16x2(w[j + 4], w[j + 5]), f32x2_to_f16x2(w[j + 6], w[j + 7]));
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == kPBulkTid) {
-            bulk_s2g(rec + kRWQ, sbase + kPA, 8192);  // rows 0-63 of each block
-            bulk_s2g(rec + kRWQ + 16384, sbase + kPA + 8192, 8192);
-            bulk_commit();
-        }
-        item = next;
-        next = s_fetch[0];
-    }
-    // drain: a staging copy still in flight (after an abort) lands, the record stores complete and
-    // every MMA this CTA issued completes, before shared memory and TMEM are released
-    if (tid == 0 && pending) {
-        const uint64_t t0 = lad::dev::globaltimer_ns();
-        while (!mbar_try_wait(stage_bar, stage_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
-        }
-    }
-    if (tid == kPBulkTid) bulk_wait_all();
-    if (warp == 0) {
-        tc_commit(mma_bar);
-        const uint64_t t0 = lad::dev::globaltimer_ns();
-        while (!mbar_try_wait(mma_bar, mma_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, kPTmemCols);
-}
-
 // ------------------------------------------------------------------------------------------
-// The prep, warp-specialised (what the split path runs). Half the CTA forms an item's operands
-// while the other half finishes the item before it, so the solve's long serial chain (run by four
-// warps, the others waiting at its barriers) overlaps the next item's formation:
+// The prep: one CTA of 16 warps per SM walks the segment's (sequence, head, chunk) items, taken
+// from a counter (CTAs that start late, behind other work on their SM, take fewer). Half the CTA
+// forms an item's operands while the other half finishes the item before it, so the solve's long
+// serial chain (run by four warps, the others waiting at its barriers) overlaps the next item's
+// formation:
 //   warps 0-7, the former: staging wait, decays and operand tiles ([Kt; Qt] into one of two
-//     buffers, Kh, Kg), [Kt; Qt] Kh^T on the tensor cores, A (into one of two scratch buffers) and P;
+//     buffers, Kh), [Kt; Qt] Kh^T on the tensor cores, A (into one of two scratch buffers) and P;
 //   warps 8-15, the solver: (I + A)^-1 and the Tb tiles, W = Tb Kt on the tensor cores, W out.
 // An item passes from the former to the solver through buffer j % 2 (the [Kt; Qt] tile and the A
 // scratch) with two mbarriers per buffer: full (the former's item is in it) and empty (the solver is
 // done with it: its W MMA has read Kt, and the solve has read A). Each half synchronises on its own
-// named barrier. The record leaves as the former writes it (Kg, g_last, P: stores from registers;
-// Qt: one bulk store from the tile) and as the solver finishes it (Tb hi / lo, W: stores from
-// registers), so neither half waits on the other's stores. Every wait is bounded; the former ends
-// the solver's loop with an item of -1.
+// named barrier. The record leaves as each half finishes its part: the former's Qt and Kh (bulk,
+// from their tiles), P (bulk, from a tile over the scan's buffer) and g_last; the solver's Tb hi /
+// lo (stores from registers) and W (bulk, from a tile over the T scratch). Each half's bulk
+// stores are its own, so neither waits on the other's. Every wait is bounded; the former ends the
+// solver's loop with an item of -1.
 // ------------------------------------------------------------------------------------------
 constexpr uint32_t kWQW = 0;                          // [Kt; Qt] x 2, 32 KiB each (the record's Qt)
 constexpr uint32_t kWKH = 65536;                      // Kh [64 tok][128 d_k], 2 blocks x 8 KiB
@@ -1279,6 +893,7 @@ static_assert(kWSmemBytes <= 232448, "prep shared memory over the per-block limi
 static_assert(kWTB % 1024 == 0 && kWQW % 1024 == 0 && kWKH % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 constexpr int kWHalf = 256;                           // threads of each half
 constexpr int kWFetchTid = 128, kWStageTid = 32, kWBulkTid = 64;  // former threads with a side job
+constexpr int kWSBulkTid = 32;  // the solver's thread (in its own numbering) that stores W in bulk
 // TMEM columns: [Kt; Qt] Kh^T (the former's), W (the solver's)
 constexpr uint32_t kWColA = 0, kWColW = 64, kWTmemCols = 256;
 
@@ -1374,13 +989,12 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
         for (int j = 0;; ++j) {
             const int bf = j & 1;
             // the buffer's previous item (j - 2) must be done with: the solver's W has read its Kt and
-            // its solve its A; the bulk store of that item's Qt has read the tile
+            // its solve its A
             if (j >= 2) {
                 bool w = true;
                 if (warp == 0)
                     w = wait_bar(empty_bar + 8 * bf, static_cast<uint32_t>((j - 2) >> 1) & 1u, abort_flag,
                                  &g_prefill_error, lad::kErrPrefill);
-                if (ft == kWBulkTid) bulk_wait_read1();
                 ok = half_and(1, w && ok);
             }
             if (item >= nitems || !ok) {
@@ -1441,9 +1055,12 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
                     }
                 }
             }
-            // ---- the decays and the operand tiles, as in kda_chunk_prep_kernel, with warp w taking
-            //      the two quartets 2w, 2w + 1 (tokens 8w .. 8w+7): their products first, then after the
-            //      scan each quartet's running products again (from alpha) and its four tokens ----
+            // ---- the decays and the operand tiles. Per key channel, g_r = prod_{s <= r} alpha_s and
+            //      R_r = prod_{s > r} alpha_s, so that Kh = K R / g_last takes one reciprocal per channel
+            //      and none per element. Warp w takes the two quartets 2w, 2w + 1 (tokens 8w .. 8w+7),
+            //      lane l the channels 4l .. 4l+3: the quartets' products first; threads 0-127 scan a
+            //      channel's 16 quartet products both ways; then each quartet's running products again
+            //      (from alpha) and its four tokens ----
             const int c4 = 4 * lane;
             auto quartet_products = [&](int o, float4 (&fw)[4], float4 (&bw)[4]) {
                 float4 a4[4];
@@ -1473,6 +1090,8 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
                 quartet_products(2 * warp + qq, fw, bw);
                 *reinterpret_cast<float4 *>(s_oct + (2 * warp + qq) * kDk + c4) = fw[3];
             }
+            // the previous item's bulk stores have read Qt, Kh and P (their regions are written next)
+            if (ft == kWBulkTid) bulk_wait_read0();
             half_bar(1);
             if (ft < kDk) {
                 float y[16];
@@ -1519,11 +1138,10 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
                         k01 = mul2(k01, make_float2(rk, rk));
                         k23 = mul2(k23, make_float2(rk, rk));
                     }
-                    const float2 kg01 = mul2(k01, R01), kg23 = mul2(k23, R23);
-                    const float2 kh01 = mul2(kg01, rg01), kh23 = mul2(kg23, rg23);
+                    const float2 kh01 = mul2(mul2(k01, R01), rg01), kh23 = mul2(mul2(k23, R23), rg23);
                     const float2 kt01 = mul2(k01, g01), kt23 = mul2(k23, g23);
                     const float2 qt01 = mul2(q01, g01), qt23 = mul2(q23, g23);
-                    const uint32_t off = sw128_off16(r, c4, 8192);         // 64-row tiles (Kh; the record's Kg)
+                    const uint32_t off = sw128_off16(r, c4, 8192);         // Kh, a 64-row tile
                     const uint32_t offq = sw128_off16(kC + r, c4, 16384);  // row 64 + r of [Kt; Qt]
                     const uint32_t offk = sw128_off16(r, c4, 16384);       // row r of [Kt; Qt]
                     *reinterpret_cast<uint2 *>(sm + qw + offk) =
@@ -1532,8 +1150,6 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
                         make_uint2(f32x2_to_f16x2(qt01.x, qt01.y), f32x2_to_f16x2(qt23.x, qt23.y));
                     *reinterpret_cast<uint2 *>(sm + kWKH + off) =
                         make_uint2(f32x2_to_f16x2(kh01.x, kh01.y), f32x2_to_f16x2(kh23.x, kh23.y));
-                    *reinterpret_cast<uint2 *>(rec + kRKG + off) =
-                        make_uint2(f32x2_to_f16x2(kg01.x, kg01.y), f32x2_to_f16x2(kg23.x, kg23.y));
                 }
             }
             // ---- [Kt; Qt] Kh^T: rows 0-63 give Kt Kh^T, rows 64-127 Qt Kh^T ----
@@ -1545,9 +1161,10 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
                 pending = 1;
             }
             if (ft == kWFetchTid) s_fetch[0] = atomicAdd(p.counter, 1);  // read after this item's last barrier
-            if (ft == kWBulkTid) {  // the record's Qt (rows 64-127 of each block of the tile)
+            if (ft == kWBulkTid) {  // the record's Qt (rows 64-127 of each block of the tile) and Kh
                 bulk_s2g(rec + kRWQ + 8192, sbase + qw + 8192, 8192);
                 bulk_s2g(rec + kRWQ + 16384 + 8192, sbase + qw + 16384 + 8192, 8192);
+                bulk_s2g(rec + kRKH, sbase + kWKH, 16384);
                 bulk_commit();
             }
             if (warp == 0) {
@@ -1572,8 +1189,9 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
                     break;
                 }
             }
-            // ---- A = strict_lower(diag(beta) Kt Kh^T) -> fp32 scratch; P = lower(Qt Kh^T) -> the
-            //      record (fp16); a warp takes 32 of a row's 64 columns, in two 16-column loads ----
+            // ---- A = strict_lower(diag(beta) Kt Kh^T) -> fp32 scratch; P = lower(Qt Kh^T) -> fp16 tile
+            //      over the scan's buffer (read by now), stored to the record in bulk; a warp takes 32 of
+            //      a row's 64 columns, in two 16-column loads ----
 #pragma unroll 1
             for (int qq = 0; qq < 2; ++qq) {
                 const int qd = 2 * (warp >> 2) + qq;
@@ -1599,23 +1217,27 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
                         float y[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) y[e] = (c0 + jj + e <= r) ? x[jj + e] : 0.f;
-                        *reinterpret_cast<uint4 *>(rec + kRP + sw128_off16(r, c0 + jj, 8192)) =
+                        *reinterpret_cast<uint4 *>(sm + kWSuf + sw128_off16(r, c0 + jj, 8192)) =
                             make_uint4(f32x2_to_f16x2(y[0], y[1]), f32x2_to_f16x2(y[2], y[3]),
                                        f32x2_to_f16x2(y[4], y[5]), f32x2_to_f16x2(y[6], y[7]));
                     }
                 }
             }
+            fence_async_smem();
             tc_fence_before();
             half_bar(1);  // A and beta of the item are in place (and TMEM's column block is read)
             if (ft == 0) {
                 s_item[bf] = item;
                 mbar_arrive(full_bar + 8 * bf);
             }
+            if (ft == kWBulkTid) {
+                bulk_s2g(rec + kRP, sbase + kWSuf, 8192);
+                bulk_commit();
+            }
             item = next;
             next = s_fetch[0];
         }
-        // drain: a staging copy still in flight (after an abort) lands and the Qt stores have read
-        // their tiles
+        // drain: a staging copy still in flight (after an abort) lands and the bulk stores complete
         if (ft == 0 && pending) {
             const uint64_t t0 = lad::dev::globaltimer_ns();
             while (!mbar_try_wait(stage_bar, stage_phase) && lad::dev::globaltimer_ns() - t0 < lad::dev::kWaitLimitNs) {
@@ -1644,6 +1266,7 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
             if (sw == 0)
                 w = wait_bar(full_bar + 8 * bf, static_cast<uint32_t>(j >> 1) & 1u, abort_flag, &g_prefill_error,
                              lad::kErrPrefill);
+            if (st == kWSBulkTid) bulk_wait_read0();  // the previous W has left the T scratch
             if (!half_and(2, w)) break;
             const int item = s_item[bf];
             if (item < 0) break;
@@ -1673,7 +1296,8 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
             tc_fence_after();
             if (!ok) break;
             if (st == 0) mbar_arrive(empty_bar + 8 * bf);  // the buffer's Kt and A are free
-            // ---- W -> the record's [W; Qt] tile (rows 0-63). M = 64: row 16 sp + i sits in lane i
+            // ---- W -> fp16 tile over the T scratch (the solve is done with it), then the record's
+            //      [W; Qt] tile (rows 0-63 of each block) in bulk. M = 64: row 16 sp + i sits in lane i
             //      (< 16) of sub-partition sp; the loads are collective, so the whole warp issues them
             //      and lanes 0-15 keep the rows. A warp takes 64 of the 128 columns ----
 #pragma unroll 1
@@ -1686,13 +1310,21 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
                     const int r = 16 * sp + lane;
 #pragma unroll
                     for (int jj = 0; jj < 32; jj += 8)
-                        *reinterpret_cast<uint4 *>(rec + kRWQ + sw128_off16(r, c0 + jj, 16384)) =
+                        *reinterpret_cast<uint4 *>(sm + kWT + sw128_off16(r, c0 + jj, 8192)) =
                             make_uint4(f32x2_to_f16x2(wv[jj], wv[jj + 1]), f32x2_to_f16x2(wv[jj + 2], wv[jj + 3]),
                                        f32x2_to_f16x2(wv[jj + 4], wv[jj + 5]), f32x2_to_f16x2(wv[jj + 6], wv[jj + 7]));
                 }
             }
+            fence_async_smem();
             tc_fence_before();  // the W loads are done before the next item's W MMA
+            half_bar(2);
+            if (st == kWSBulkTid) {
+                bulk_s2g(rec + kRWQ, sbase + kWT, 8192);
+                bulk_s2g(rec + kRWQ + 16384, sbase + kWT + 8192, 8192);
+                bulk_commit();
+            }
         }
+        if (st == kWSBulkTid) bulk_wait_all();
         // every W MMA has completed (after an abort, a fresh commit is waited for, bounded)
         if (sw == 0) {
             tc_commit(mmas_bar);
@@ -1731,9 +1363,12 @@ constexpr uint32_t kCMisc = kCRec + kRecBytes;     // buffer 0's 512 bytes betwe
                                                    // barriers, 3 MMA barriers, TMEM slot, abort
 constexpr uint32_t kCSmemBytes = kCO + 16384 + 1024;
 static_assert(kCMisc + 64 <= kCRec + kCV, "chain barriers must fit in the record slack");
+static_assert(kRecBytes + 512 <= kCV, "the g_last copy must fit in buffer 1's slack");
 static_assert(kCV % 1024 == 0 && kCRecStride % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(kCSmemBytes <= 232448, "chain shared memory over the per-block limit");
 constexpr uint32_t kCChunkTx = kRecBytes + 16384;  // a chunk buffer's bytes: the record and the v tile
+constexpr uint32_t kCGl = kCRec + kCRecStride + kRecBytes;  // buffer 1's slack: the current chunk's g_last,
+                                                            // copied out before its buffer is refilled
 // TMEM: the fp32 master S^T (128 lanes = d_v, 128 columns = d_k), two [X^T | O^T] buffers of
 // 128 columns (chunk parity), U'^T (64 columns)
 constexpr uint32_t kCColS = 0, kCColXO = 128, kCColU = 384, kCTmemCols = 512;
@@ -1870,14 +1505,12 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
         }
     };
 
-    // ---- the state entering the segment: the fp16 copy (S0^T), and the master scaled by chunk
-    //      0's decay, ready for chunk 0's contraction ----
+    // ---- the state entering the segment: the fp16 copy (S0^T) and the fp32 master ----
     bool ok = true;
     if (!issuer) {
         ok = rec_ready(0);
         if (ok) {
             const float *S0 = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
-            const float *gl = gl_of(0);
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
                 const int c0 = 64 * cg + 32 * part;
@@ -1889,8 +1522,6 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
                     *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, c0 + j, 16384)) =
                         make_uint4(f32x2_to_f16x2(v[j], v[j + 1]), f32x2_to_f16x2(v[j + 2], v[j + 3]),
                                    f32x2_to_f16x2(v[j + 4], v[j + 5]), f32x2_to_f16x2(v[j + 6], v[j + 7]));
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] *= gl[c0 + j];
                 tmem_st32(tmem + lane_base + kCColS + c0, v);
             }
             tmem_wait_st();
@@ -1926,10 +1557,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
             tc_commit(mbar_a);
             bar288();  // U^T is in place (over the v tile)
             tc_fence_after();
-            // ---- second batch: S^T += U^T Kg (commit: the master pass may start); O^T += U^T P^T
+            // ---- second batch: S^T += U^T Kh (commit: the master pass may start); O^T += U^T P^T
             //      (commit: waited for here) ----
             const uint64_t ut0 = d0 + ((rs + kCV) >> 4);
-            const uint64_t kg0 = smem_desc(sbase + rs + kRKG, 8192, 1024, kLayoutSw128);
+            const uint64_t kg0 = smem_desc(sbase + rs + kRKH, 8192, 1024, kLayoutSw128);
 #pragma unroll
             for (int j = 0; j < kC / 16; ++j)
                 tc_mma_f16(tmem + kCColS, kdesc16(ut0, 16384, j), kg0 + ((j * 2048) >> 4), kIdescSU, 1);
@@ -1950,7 +1581,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
             if (i > 0) store_o(i - 1);
             w = wait_bar(mbar_a, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
             tc_fence_after();
-            // ---- U^T = U'^T - X^T -> the fp16 operand, over the v tile (its reader is complete) ----
+            // ---- U^T = U'^T - X^T -> the fp16 operand, over the v tile (its reader is complete). The
+            //      chunk's g_last is copied out of its buffer too: the buffer takes chunk i + 2's
+            //      record once this chunk's MMAs are complete, before the master pass reads it ----
+            if (tid < kDk) reinterpret_cast<float *>(sm + kCGl)[tid] = gl_of(i)[tid];
             if (w) {
                 float x[32], u[32];  // both loads before the one wait
                 tmem_ld32(xo + lane_base + 32 * cg, x);
@@ -1974,20 +1608,32 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
             tc_fence_before();
             bar288();
             if (w) w = wait_bar(mbar_s, static_cast<uint32_t>(i) & 1u, abort_flag, &g_prefill_error, lad::kErrPrefill);
-            if (w && !last) w = rec_ready(i + 1);  // the next chunk's operands and decay
+            if (w && !last) w = rec_ready(i + 1);  // the next chunk's operands
             tc_fence_after();
             if (w) {
-                // ---- the new state: its fp16 copy over S0's (the first batch, S0's only reader, is
-                //      complete) and the next chunk's decay, or the state out; both halves of the
-                //      thread's row are loaded before the one wait ----
+                // ---- the new state S = (S0 + Kh^T U) Diag(g_last): the chunk's decay on the master
+                //      in fp32, then its fp16 copy over S0's (the first batch, S0's only reader, is
+                //      complete), or the state out; both halves of the thread's row are loaded before
+                //      the one wait ----
                 float vv[2][32];
                 tmem_ld32(tmem + lane_base + kCColS + 64 * cg, vv[0]);
                 tmem_ld32(tmem + lane_base + kCColS + 64 * cg + 32, vv[1]);
                 tmem_wait_ld();
+                const float4 *gn = reinterpret_cast<const float4 *>(sm + kCGl) + 16 * cg;
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
                     const int c0 = 64 * cg + 32 * part;
                     float (&v)[32] = vv[part];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 g4 = gn[8 * part + j];
+                        const float2 a = mul2(make_float2(v[4 * j], v[4 * j + 1]), make_float2(g4.x, g4.y));
+                        const float2 c = mul2(make_float2(v[4 * j + 2], v[4 * j + 3]), make_float2(g4.z, g4.w));
+                        v[4 * j] = a.x;
+                        v[4 * j + 1] = a.y;
+                        v[4 * j + 2] = c.x;
+                        v[4 * j + 3] = c.y;
+                    }
                     if (last) {
                         float *Sout = p.S + static_cast<size_t>(bh) * kDk * kDv + dv;
 #pragma unroll
@@ -1998,17 +1644,6 @@ __global__ void __launch_bounds__(kChainThreads, 1) kda_chunk_chain_kernel(Chain
                             *reinterpret_cast<uint4 *>(sm + kCS16 + sw128_off16(dv, c0 + j, 16384)) =
                                 make_uint4(f32x2_to_f16x2(v[j], v[j + 1]), f32x2_to_f16x2(v[j + 2], v[j + 3]),
                                            f32x2_to_f16x2(v[j + 4], v[j + 5]), f32x2_to_f16x2(v[j + 6], v[j + 7]));
-                        const float4 *gn = reinterpret_cast<const float4 *>(gl_of(i + 1) + c0);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float4 g4 = gn[j];
-                            const float2 a = mul2(make_float2(v[4 * j], v[4 * j + 1]), make_float2(g4.x, g4.y));
-                            const float2 c = mul2(make_float2(v[4 * j + 2], v[4 * j + 3]), make_float2(g4.z, g4.w));
-                            v[4 * j] = a.x;
-                            v[4 * j + 1] = a.y;
-                            v[4 * j + 2] = c.x;
-                            v[4 * j + 3] = c.y;
-                        }
                         tmem_st32(tmem + lane_base + kCColS + c0, v);
                     }
                 }
@@ -2181,12 +1816,6 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
             cudaError_t attr_err =
                 cudaFuncSetAttribute(kda_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
             if (attr_err == cudaSuccess)
-                attr_err = cudaFuncSetAttribute(kda_chunk_prep_kernel<false>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
-            if (attr_err == cudaSuccess)
-                attr_err = cudaFuncSetAttribute(kda_chunk_prep_kernel<true>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmemBytes);
-            if (attr_err == cudaSuccess)
                 attr_err = cudaFuncSetAttribute(kda_chunk_prep_ws_kernel<false>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kWSmemBytes);
             if (attr_err == cudaSuccess)
@@ -2261,17 +1890,10 @@ extern "C" int kda_prefill_chunked(const lad_bf16 *q, const lad_bf16 *k, const l
     const int beside = sms - chain_ctas > sms / 2 ? sms - chain_ctas : sms / 2;
     auto prep = [&](cudaStream_t on, long long grid, int sg, uint8_t *buf, int c0, int nseg) {
         const PrepArgs pa{beta, buf, counters + sg, B, T, H, c0, nseg, a.l2norm};
-#if LAD_PREFILL_PREP_WS
         if (a.l2norm)
             kda_chunk_prep_ws_kernel<true><<<static_cast<unsigned>(grid), kPThreads, kWSmemBytes, on>>>(pa, pm);
         else
             kda_chunk_prep_ws_kernel<false><<<static_cast<unsigned>(grid), kPThreads, kWSmemBytes, on>>>(pa, pm);
-#else
-        if (a.l2norm)
-            kda_chunk_prep_kernel<true><<<static_cast<unsigned>(grid), kPThreads, kPSmemBytes, on>>>(pa, pm);
-        else
-            kda_chunk_prep_kernel<false><<<static_cast<unsigned>(grid), kPThreads, kPSmemBytes, on>>>(pa, pm);
-#endif
         return cudaGetLastError();
     };
     for (int sg = 0; sg < L.nsegs && e == cudaSuccess; ++sg) {
