@@ -128,6 +128,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// a tile into L2 only (no shared memory, no barrier; a hint): a later load of it is served from L2
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -1006,6 +1014,13 @@ __global__ void __launch_bounds__(kPThreads, 1) kda_chunk_prep_ws_kernel(PrepArg
             }
             const int ch = nch;
             coords(next, nb, nh, nch);
+            // the next item's q, k and alpha start for L2 now; they are staged (TMA) only once this
+            // item's formation has read the staging buffers
+            if (ft == kWStageTid && next < nitems) {
+                tma_prefetch_3d(&maps.q, nh * kDk, nch * kC, nb);
+                tma_prefetch_3d(&maps.k, nh * kDk, nch * kC, nb);
+                tma_prefetch_3d(&maps.alpha, nh * kDk, nch * kC, nb);
+            }
             const int t0 = ch * kC;
             const int n = min(kC, p.T - t0);
             uint8_t *rec = p.ws + static_cast<size_t>(item) * kRecBytes;
