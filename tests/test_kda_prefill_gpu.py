@@ -6,7 +6,7 @@ segment) and the single-kernel path (no workspace; tf32 operands).
 Outputs are held to the 2e-3 relative-L2 output budget; they come out near 4e-4. The final state
 is held to 1e-3: its chunk updates are fp16 / tf32 contractions (rounding unit 2^-11), so the
 1e-4 figure of the fp32 decode path does not apply. At full size (32,768 tokens, 64 heads) the
-measured state error is 2.9e-4 (3.1e-4 for the worst head) and the test asserts 5e-4 there.
+measured state error is 3.0e-4 (3.05e-4 for the worst head) and the test asserts 5e-4 there.
 """
 import numpy as np
 import pytest
@@ -18,7 +18,7 @@ from tests.parity import TOL_OUT, bf16_round, f64, max_rel_l2, rel_l2
 
 pytestmark = pytest.mark.gpu
 TOL_PREFILL_STATE = 1e-3
-TOL_PREFILL_STATE_32K = 5e-4  # measured 2.9e-4 (3.1e-4 worst head)
+TOL_PREFILL_STATE_32K = 5e-4  # measured 3.0e-4 (3.05e-4 worst head)
 
 
 @pytest.fixture(scope="module")
